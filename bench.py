@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the Fast LapSum soft top-k (forward + backward) on B200.
+
+One step = one forward (exact threshold b and p) plus one backward (VJP g)
+over one batch of synthetic scores, through the library's C ABI.  The default
+workload is the 10^8-score row (k = 1e5, t = 0.005, 50/50 N(0,1)/U(-4,4)
+scores) that the headline metric is quoted on.
+
+Usage:
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-table] [--no-cpu-baseline]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU)
+
+With N ranks every rank solves its own independent workload instance (seed =
+rank): the path shards by problem, no collective touches the data path, and
+the reported value is the elements of all ranks per max-over-ranks time
+(weak scaling).  Rank 0 prints one JSON line.
+
+`--impl reference` times the fp64 CPU oracle (the reference for this method)
+on a bounded prefix of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import ORDER, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "soft top-k elements/s fwd+bwd"
+UNIT = "elements/s"
+
+# Algorithmic bytes per element of each kernel (what the kernel must move:
+# reads of its inputs and writes of its outputs, once).
+KERNEL_BYTES_PER_ELEMENT = {
+    "onchip_fwd": 8,      # read r, write p
+    "onchip_bwd": 12,     # read r, v, write g
+    "emit": 8,            # read r, write p
+    "bwd_reduce": 8,      # read r, v
+    "bwd_apply": 12,      # read r, v, write g
+    "bracket_fold": 4,    # read r
+    "radix_prep": 8,      # read r, write keys
+    "radix_upsweep": 4,   # read keys (per pass)
+    "radix_downsweep": 8,  # read keys, write keys (per pass)
+    "rowsolve": 4,        # read sorted keys
+}
+# Algorithmic bytes per element of one fwd+bwd step, per solver: on-chip rows
+# move r, p, r, v, g once (20 B); the long-row paths read r twice in the
+# forward and r, v twice in the backward (32 B).
+STEP_BYTES_PER_ELEMENT = {"bitonic": 20, "radix": 20, "bracket": 32}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# nvidia-smi clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        exe = shutil.which("nvidia-smi")
+        if exe is None:
+            return
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = subprocess.Popen(
+            [exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+             "-i", str(self.gpu_index)], stdout=self.out, stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [ln.strip().split(",") for ln in self.out.read().splitlines() if ln.strip()]
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for row in rows:
+            try:
+                sm.append(float(row[1]))
+                mx = max(mx, float(row[2]))
+                for nm, val in zip(names, row[5:9]):
+                    if val.strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle leg (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample_run(w, r_row, v_row, n_sample):
+    """Oracle fwd+bwd on the first n_sample scores of one row (k scaled to keep k/n)."""
+    import oracle
+    n_s = min(n_sample, r_row.size)
+    k_s = w.k * n_s / w.n if n_s < w.n else w.k
+    k_s = min(max(k_s, 1e-3), n_s - 1e-3)
+    t0 = time.perf_counter()
+    b = oracle.solve_b(r_row[:n_s], k_s, w.t)
+    oracle.emit_p(r_row[:n_s], b, w.t)
+    oracle.vjp(r_row[:n_s], v_row[:n_s], b, w.t)
+    return n_s, k_s, time.perf_counter() - t0
+
+
+def cpu_sample_size(w):
+    # about 10 s of single-thread oracle work on this machine's cores
+    return min(w.elements, 1 << 23)
+
+
+def cpu_baseline(w, r, v):
+    n_s, k_s, sec = oracle_sample_run(w, r[0], v[0], cpu_sample_size(w))
+    return {"value": n_s / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {n_s} scores of row 0 of {w.name}, k={k_s:g} (same k/n), "
+                      f"t={w.t}; fp64 full sort + bisection, p, VJP; {sec:.1f} s single thread",
+            "host_cpu_count": os.cpu_count()}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    r, v = make_inputs(w, seed=0)
+    n_s = min(cpu_sample_size(w), w.n)
+    # warm-up steps on a tiny prefix, then K timed steps on the bounded sample
+    for _ in range(args.warmup):
+        oracle_sample_run(w, r[0], v[0], min(4096, w.n))
+    n_step = max(1 << 16, n_s // max(1, args.steps))
+    times = []
+    for _ in range(args.steps):
+        n_done, k_s, sec = oracle_sample_run(w, r[0], v[0], n_step)
+        times.append(sec)
+    ms = 1e3 * statistics.mean(times)
+    value = n_done / (ms / 1e3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "n": w.n, "k": w.k, "t": w.t,
+                   "step_sample": f"first {n_done} scores of row 0 (k scaled to {k_s:g})"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} steps, each the first {n_done} scores of row 0"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="extreme_1e8", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-table", action="store_true", help="skip the per-workload table")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_selection_primitive_b200 as L
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        tt = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        return float(tt.item())
+
+    L._build.build()
+    w = WORKLOADS[args.workload]
+    r_h, v_h = make_inputs(w, seed=rank)
+    stream = torch.cuda.current_stream(dev)
+
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_buf = torch.empty(2 * l2_bytes // 4 + 1024, dtype=torch.float32, device=dev)
+
+    def run_workload(w, r_h, v_h, steps, warmup, table=False):
+        rd = torch.from_numpy(r_h).to(dev)
+        vd = torch.from_numpy(v_h).to(dev)
+        pd = torch.empty_like(rd)
+        gd = torch.empty_like(rd)
+        bd = torch.empty(w.B, dtype=torch.float64, device=dev)
+        ws = L.Workspace(w.B, w.n, w.k, "auto", dev)
+        working = 4 * rd.numel() * 4
+        flush = working < 2 * l2_bytes
+
+        def fwd():
+            L.forward(rd, w.k, w.t, ws=ws, p=pd, b=bd)
+
+        def bwd():
+            L.backward(rd, bd, vd, w.t, ws=ws, g=gd)
+
+        def timed(fn, k_steps, profile=False):
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(k_steps)]
+            torch.cuda.synchronize(dev)
+            if profile:
+                L.profile_enable(True)
+            for s, e in evs:
+                if flush:
+                    flush_buf.zero_()
+                s.record(stream)
+                fn()
+                e.record(stream)
+            torch.cuda.synchronize(dev)
+            prof = L.profile_read() if profile else None
+            if profile:
+                L.profile_enable(False)
+            return [s.elapsed_time(e) for s, e in evs], prof
+
+        for _ in range(warmup):
+            fwd()
+            bwd()
+        torch.cuda.synchronize(dev)
+        res = {"flush": flush, "ws": ws, "rd": rd, "vd": vd, "pd": pd, "gd": gd, "bd": bd,
+               "fwd": fwd, "bwd": bwd, "timed": timed}
+        if table:
+            tf, _ = timed(fwd, steps)
+            tb, _ = timed(bwd, steps)
+            tfb, _ = timed(lambda: (fwd(), bwd()), steps)
+            res["table"] = {"fwd_ms": statistics.median(tf), "bwd_ms": statistics.median(tb),
+                            "fwdbwd_ms": statistics.median(tfb)}
+        return res
+
+    peak_gbs, peak_kind = load_peaks()
+    R = run_workload(w, r_h, v_h, args.steps, args.warmup)
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    step_ms, prof = R["timed"](lambda: (R["fwd"](), R["bwd"]()), args.steps, profile=True)
+    barrier()
+    clocks = sampler.stop()
+    ms_local = statistics.mean(step_ms)
+    ms = max_over_ranks(ms_local)
+    elements = w.elements * world
+    value = elements / (ms / 1e3)
+
+    # dominant kernel of the timed region
+    dom_name, (dom_launch, dom_ms) = max(prof.items(), key=lambda kv: kv[1][1])
+    per_launch_ms = dom_ms / dom_launch
+    bpe = KERNEL_BYTES_PER_ELEMENT.get(dom_name)
+    per_launch_elems = w.elements if dom_name not in ("radix_upsweep", "radix_downsweep") else w.elements
+    achieved = (bpe * per_launch_elems / (per_launch_ms / 1e3)) / 1e9 if bpe else None
+    traffic = read_traffic(dom_name, w.name)
+    roofline = {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak_gbs,
+                "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": (achieved / peak_gbs) if achieved else None,
+                "traffic": traffic, "algorithmic_bytes_per_launch": (bpe or 0) * per_launch_elems,
+                "launch_ms": per_launch_ms}
+    step_bytes = STEP_BYTES_PER_ELEMENT[w.path] * w.elements
+    step_gbs = step_bytes / (ms_local / 1e3) / 1e9
+    kernels = {k: {"launches": v[0], "total_ms": round(v[1], 4),
+                   "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
+               for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    gpu_launches = int(sum(v[0] for v in prof.values()))
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        import torch as _t
+        r_pin = _t.from_numpy(r_h).pin_memory()
+        v_pin = _t.from_numpy(v_h).pin_memory()
+        p_pin = _t.empty_like(r_pin).pin_memory()
+        g_pin = _t.empty_like(r_pin).pin_memory()
+
+        def e2e_step():
+            R["rd"].copy_(r_pin, non_blocking=True)
+            R["vd"].copy_(v_pin, non_blocking=True)
+            R["fwd"]()
+            R["bwd"]()
+            p_pin.copy_(R["pd"], non_blocking=True)
+            g_pin.copy_(R["gd"], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        k_e2e = max(3, min(args.steps, 10))
+        e_s.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        e_e.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / k_e2e)
+        nb = r_pin.numel() * 4
+        e2e = {"value": elements / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 2 * nb, "d2h_bytes_per_step": 2 * nb}
+
+    # per-workload table (fwd, bwd, fwd+bwd) on this GPU
+    table = None
+    if not args.no_table and rank == 0:
+        table = {}
+        for name in ORDER:
+            wk = WORKLOADS[name]
+            if name == w.name:
+                rr, vv = r_h, v_h
+            else:
+                rr, vv = make_inputs(wk, seed=0)
+            T = run_workload(wk, rr, vv, 10, 3, table=True)["table"]
+            table[name] = {
+                "fwd_ms": round(T["fwd_ms"], 5), "bwd_ms": round(T["bwd_ms"], 5),
+                "fwdbwd_ms": round(T["fwdbwd_ms"], 5),
+                "fwd_elements_per_s": wk.elements / (T["fwd_ms"] / 1e3),
+                "bwd_elements_per_s": wk.elements / (T["bwd_ms"] / 1e3),
+                "fwdbwd_elements_per_s": wk.elements / (T["fwdbwd_ms"] / 1e3),
+                "fwdbwd_algorithmic_gbs": STEP_BYTES_PER_ELEMENT[wk.path] * wk.elements
+                / (T["fwdbwd_ms"] / 1e3) / 1e9,
+            }
+            table[name]["fwdbwd_frac_of_peak"] = table[name]["fwdbwd_algorithmic_gbs"] / peak_gbs
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, r_h, v_h)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "n": w.n, "k": w.k, "t": w.t,
+                       "distribution": w.dist, "solver": w.path,
+                       "l2": "flushed before each step" if R["flush"] else
+                             "inputs larger than L2 (no flush)",
+                       "parallelism": f"{world} independent instances (one per GPU)"},
+            "step_algorithmic_gbs": step_gbs,
+            "step_frac_of_peak": step_gbs / peak_gbs,
+            "roofline": roofline,
+            "kernels": kernels,
+            "gpu_launches": gpu_launches,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "workloads": table,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def read_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for ln in f:
+            parts = ln.split()
+            if len(parts) >= 3 and not ln.startswith("#") and parts[0] == kernel and \
+                    parts[1] == workload:
+                try:
+                    return float(parts[2])
+                except ValueError:
+                    return None
+    return None
+
+
+if __name__ == "__main__":
+    main()

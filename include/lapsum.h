@@ -1,0 +1,172 @@
+/*
+ * lapsum.h -- C ABI of the B200 (sm_100a) Fast LapSum soft top-k library.
+ *
+ * The operator, from "Fast LapSum: Exact Differentiable Top-k at Million Scale"
+ * (gist.science explainer pages), section 2.1 "The LapSum operator": for each
+ * row of scores r[0..n), a budget k (0 < k < n) and a temperature t > 0,
+ *
+ *     p_i = sigma((r_i - b) / t),   sigma = CDF of Laplace(0,1),
+ *     sum_i p_i = k                 (b is the unique scalar threshold),
+ *
+ * and the backward pass is the analytic vector-Jacobian product
+ *
+ *     g_i = (f_i / t) (v_i - sum_j v_j f_j / sum_j f_j),   f_i = 0.5 exp(-|r_i - b| / t).
+ *
+ * Section 2.2 "Fast LapSum: the GPU solver" gives the two solvers built here:
+ * a full-sort solver (sort, one numerically stable prefix/suffix scan, an
+ * index lookup of the balancing segment, a closed-form root) and, for rows
+ * with n > 10^6, probabilistic bracketing (sample, binomial order-statistic
+ * bracket, one streaming fold, exact solve on the middle band, certification
+ * with widening).
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains device memory.
+ *   - Rows are row-major with leading dimension ld >= n (elements): element i
+ *     of row j of r, p, v and g is at [j * ld + i].  Vectorised loads are used
+ *     when the base pointers are 16-byte aligned and ld is a multiple of 4.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is ordered on it; no call synchronises the host except
+ *     lapsum_read_status and lapsum_row_info.
+ *   - Argument errors are detected on the host, returned at once, and launch
+ *     nothing.  Conditions found on the device (non-finite scores, exhausted
+ *     bracket retries) are OR-ed into a sticky status word inside the
+ *     workspace and reported by lapsum_read_status, which also clears it.
+ *   - Calls that share a workspace must be ordered on one stream (or be
+ *     otherwise serialised); concurrent calls on one workspace race.
+ */
+#ifndef LAPSUM_H
+#define LAPSUM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes and device status bits. */
+enum lapsum_status {
+    LAPSUM_OK = 0,
+    LAPSUM_EINVAL = 1,     /* B < 1, n < 1, ld < n, !(0 < k < n), !(t > 0), NULL pointer, bad path */
+    LAPSUM_EWORKSPACE = 2, /* ws NULL, not 256-byte aligned, or smaller than lapsum_workspace_bytes */
+    LAPSUM_ENONFINITE = 3, /* device: a score was NaN or infinite; b of that row is NaN */
+    LAPSUM_EBRACKET = 4,   /* device: every allowed bracket failed certification; b is NaN */
+    LAPSUM_ECUDA = 5       /* a CUDA runtime call failed (launch error, bad stream, ...) */
+};
+
+/* Solver selection (low byte of `path`). */
+enum lapsum_path {
+    LAPSUM_PATH_AUTO = 0,     /* n <= 4096: bitonic; n <= 2^20: radix full sort; else bracketing */
+    LAPSUM_PATH_FULLSORT = 1, /* full sort: bitonic for n <= 4096, radix above */
+    LAPSUM_PATH_BRACKET = 2,  /* probabilistic bracketing (any n >= 2) */
+    LAPSUM_PATH_RADIX = 3     /* full sort with the radix sorter at any n */
+};
+
+/* Test and diagnostic flags, OR-ed into `path`. */
+enum lapsum_flags {
+    LAPSUM_FLAG_FORCE_MISS = 0x100, /* bracketing: start from a bracket that excludes b */
+    LAPSUM_FLAG_NO_RETRY = 0x200    /* bracketing: allow no widening (a miss => LAPSUM_EBRACKET) */
+};
+
+/* Version of this ABI (incremented on any incompatible change). */
+int lapsum_abi_version(void);
+
+/* Static, human-readable name of a return code or status bit set. */
+const char* lapsum_status_string(int status);
+
+/*
+ * Bytes of device workspace that lapsum_forward and lapsum_backward need for
+ * this problem size and path (the same buffer serves both).  Returns 0 for
+ * invalid sizes.  The workspace must be 256-byte aligned and must be cleared
+ * once with lapsum_workspace_init before first use.
+ */
+size_t lapsum_workspace_bytes(int64_t B, int64_t n, double k, int path);
+
+/*
+ * Bytes of workspace lapsum_backward needs on its own (a prefix of any forward
+ * workspace for the same B and n, so the forward's buffer can be reused).
+ * Returns 0 for invalid sizes.
+ */
+size_t lapsum_backward_workspace_bytes(int64_t B, int64_t n);
+
+/* Zero the workspace's status word and bookkeeping (stream-ordered). */
+int lapsum_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Forward: for every row, the exact threshold b[row] (fp64) and
+ * p[row*ld + i] = sigma((r_i - b)/t) (fp32).  sum_f (may be NULL) receives
+ * sum_i f_i per row in fp64.  `seed` drives the bracketing sample (a
+ * counter-based SplitMix64 stream); results do not depend on it except for
+ * rounding in the last bits.  r and p must not overlap.
+ */
+int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
+                   int64_t n, double k, double t, int path, uint64_t seed, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/*
+ * Backward: g[row*ld + i] = (f_i/t)(v_i - R_row), R_row = sum_j v_j f_j / sum_j f_j,
+ * with f_i = 0.5 exp(-|r_i - b_row|/t) and b from lapsum_forward.  R is formed
+ * with weights shifted by the row's smallest |r_i - b|/t, so it stays finite
+ * when every f_i underflows.  g must not overlap r or v.
+ */
+int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v, float* g,
+                    int64_t B, int64_t n, double t, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, copies the sticky device status word to
+ * *device_status (LAPSUM_OK, or a LAPSUM_E* code for the first condition
+ * seen) and clears it.  Returns LAPSUM_OK or LAPSUM_ECUDA.
+ */
+int lapsum_read_status(void* ws, void* stream, int* device_status);
+
+/* Per-row record of the last forward call (diagnostics; host copy, syncs `stream`). */
+typedef struct lapsum_row_info {
+    double b;          /* threshold */
+    double sum_f;      /* sum_i f_i at b */
+    double S_L, S_R;   /* bracketing tail sums of the certified bracket */
+    float a_L, a_R;    /* certified bracket (+-inf for an open side) */
+    int64_t cnt_R;     /* scores >= a_R */
+    int64_t n_band;    /* scores in [a_L, a_R) after the fold */
+    int32_t path;      /* solver that ran (LAPSUM_PATH_*) */
+    int32_t attempts;  /* brackets tried (1 = first bracket held) */
+    int32_t sample_m;  /* bracketing sample size */
+    int32_t rank_l;    /* first-attempt order-statistic ranks (descending, 1-based) */
+    int32_t rank_h;
+    int32_t refine_levels; /* histogram narrowing levels used on the band */
+    int32_t status;    /* device status bits of this row */
+    int32_t reserved;
+} lapsum_row_info;
+
+int lapsum_row_info_get(void* ws, int64_t row, lapsum_row_info* out, void* stream);
+
+/*
+ * Copies the bracketing sample of the last forward call on row `row`
+ * (m values y_s = r[I_s] + eps_s, in draw order) to host memory `out`.
+ * Syncs `stream`.  Returns LAPSUM_EINVAL if the last call did not bracket.
+ */
+int lapsum_sample_get(void* ws, int64_t row, float* out, int64_t m, void* stream);
+
+/*
+ * Optional per-kernel timing: while enabled, every kernel the library launches
+ * is bracketed by a pair of CUDA events recorded on the launch stream.
+ * lapsum_profile_enable(1) starts a fresh record, lapsum_profile_enable(0)
+ * stops and clears it.  lapsum_profile_read waits for the recorded events and
+ * returns, per kernel name, the number of launches and their summed device
+ * time (first max_entries names; *n_entries gets the total count).  The
+ * switch is process-wide and host-thread-safe; it is meant for benchmarks.
+ */
+typedef struct lapsum_kernel_time {
+    char name[48];
+    int64_t launches;
+    double total_ms;
+} lapsum_kernel_time;
+
+int lapsum_profile_enable(int on);
+int lapsum_profile_read(lapsum_kernel_time* out, int max_entries, int* n_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAPSUM_H */

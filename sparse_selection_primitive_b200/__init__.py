@@ -1,0 +1,269 @@
+"""Fast LapSum soft top-k on B200 (sm_100a): Python binding of ``liblapsum.so``.
+
+The operator ("Fast LapSum: Exact Differentiable Top-k at Million Scale",
+gist.science explainer pages, section 2.1): per row of scores ``r``,
+
+    p_i = sigma((r_i - b)/t),  sigma = Laplace(0,1) CDF,  sum_i p_i = k,
+
+with the exact threshold ``b`` and the analytic VJP
+``g_i = (f_i/t)(v_i - sum_j v_j f_j / sum_j f_j)``, ``f_i = 0.5 exp(-|r_i - b|/t)``.
+
+This module only marshals arguments: it takes torch CUDA tensors, passes their
+device pointers and the current stream to the C ABI declared in
+``include/lapsum.h``, and raises on a non-zero return code.  Every step of the
+computation runs in the library's CUDA kernels; there is no CPU or PyTorch
+fallback, and importing the package fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import _build
+
+__all__ = [
+    "LapSumError", "Workspace", "forward", "backward", "read_status", "row_info", "sample_values",
+    "workspace_bytes", "soft_topk", "LapSumTopK", "PATHS", "FLAG_FORCE_MISS", "FLAG_NO_RETRY",
+    "library_path", "profile_enable", "profile_read",
+]
+
+PATHS = {"auto": 0, "fullsort": 1, "bracket": 2, "radix": 3}
+FLAG_FORCE_MISS = 0x100
+FLAG_NO_RETRY = 0x200
+
+_c_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+
+
+class LapSumError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_lib().lapsum_status_string(code).decode()} (code {code})")
+
+
+class RowInfo(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_double), ("sum_f", ctypes.c_double), ("S_L", ctypes.c_double),
+                ("S_R", ctypes.c_double), ("a_L", ctypes.c_float), ("a_R", ctypes.c_float),
+                ("cnt_R", ctypes.c_int64), ("n_band", ctypes.c_int64), ("path", ctypes.c_int32),
+                ("attempts", ctypes.c_int32), ("sample_m", ctypes.c_int32),
+                ("rank_l", ctypes.c_int32), ("rank_h", ctypes.c_int32),
+                ("refine_levels", ctypes.c_int32), ("status", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double)]
+
+
+_LIB = None
+
+
+def library_path() -> str:
+    return _build.SO
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(_build.SO):
+            raise ImportError(
+                f"liblapsum.so is not built ({_build.SO}); run __graft_entry__.build() or "
+                "python -m sparse_selection_primitive_b200._build")
+        lib = ctypes.CDLL(_build.SO)
+        lib.lapsum_abi_version.restype = ctypes.c_int
+        lib.lapsum_status_string.restype = ctypes.c_char_p
+        lib.lapsum_status_string.argtypes = [ctypes.c_int]
+        lib.lapsum_workspace_bytes.restype = ctypes.c_size_t
+        lib.lapsum_workspace_bytes.argtypes = [_c_i64, _c_i64, ctypes.c_double, ctypes.c_int]
+        lib.lapsum_backward_workspace_bytes.restype = ctypes.c_size_t
+        lib.lapsum_backward_workspace_bytes.argtypes = [_c_i64, _c_i64]
+        lib.lapsum_workspace_init.restype = ctypes.c_int
+        lib.lapsum_workspace_init.argtypes = [_vp, ctypes.c_size_t, _vp]
+        lib.lapsum_forward.restype = ctypes.c_int
+        lib.lapsum_forward.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64, ctypes.c_double,
+                                       ctypes.c_double, ctypes.c_int, ctypes.c_uint64, _vp,
+                                       ctypes.c_size_t, _vp]
+        lib.lapsum_backward.restype = ctypes.c_int
+        lib.lapsum_backward.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64,
+                                        ctypes.c_double, _vp, ctypes.c_size_t, _vp]
+        lib.lapsum_read_status.restype = ctypes.c_int
+        lib.lapsum_read_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
+        lib.lapsum_row_info_get.restype = ctypes.c_int
+        lib.lapsum_row_info_get.argtypes = [_vp, _c_i64, ctypes.POINTER(RowInfo), _vp]
+        lib.lapsum_profile_enable.restype = ctypes.c_int
+        lib.lapsum_profile_enable.argtypes = [ctypes.c_int]
+        lib.lapsum_profile_read.restype = ctypes.c_int
+        lib.lapsum_profile_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int,
+                                            ctypes.POINTER(ctypes.c_int)]
+        lib.lapsum_sample_get.restype = ctypes.c_int
+        lib.lapsum_sample_get.argtypes = [_vp, _c_i64, _vp, _c_i64, _vp]
+        _LIB = lib
+    return _LIB
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise LapSumError(code, where)
+
+
+def _path_code(path) -> int:
+    if isinstance(path, str):
+        return PATHS[path]
+    return int(path)
+
+
+def workspace_bytes(B: int, n: int, k: float, path="auto") -> int:
+    return int(_lib().lapsum_workspace_bytes(B, n, float(k), _path_code(path)))
+
+
+class Workspace:
+    """Device workspace for forward/backward, allocated once with torch and reused.
+
+    The library itself never allocates; this object owns the bytes (a torch
+    uint8 tensor, 256-byte aligned) and clears them once with
+    ``lapsum_workspace_init``.
+    """
+
+    def __init__(self, B: int, n: int, k: float, path="auto", device=None):
+        device = torch.device(device or "cuda")
+        self.nbytes = workspace_bytes(B, n, k, path)
+        if self.nbytes == 0:
+            raise LapSumError(1, "workspace_bytes")
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+        base = self.buf.data_ptr()
+        self.ptr = (base + 255) // 256 * 256
+        self.device = device
+        _check(_lib().lapsum_workspace_init(self.ptr, self.nbytes, _stream_ptr(device)),
+               "lapsum_workspace_init")
+
+    def fits(self, B, n, k, path) -> bool:
+        return workspace_bytes(B, n, k, path) <= self.nbytes
+
+    def fits_backward(self, B, n) -> bool:
+        return int(_lib().lapsum_backward_workspace_bytes(B, n)) <= self.nbytes
+
+
+def _as_rows(x: torch.Tensor) -> torch.Tensor:
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if x.dim() != 2:
+        raise ValueError("scores must be 1-D or 2-D (rows x n)")
+    if x.dtype != torch.float32 or not x.is_cuda:
+        raise TypeError("scores must be a float32 CUDA tensor")
+    if x.stride(1) != 1:
+        x = x.contiguous()
+    return x
+
+
+def forward(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0, ws: Workspace = None,
+            want_sum_f: bool = False, p: torch.Tensor = None, b: torch.Tensor = None):
+    """Returns (p, b[, sum_f]) for each row of r (float32 CUDA, rows x n or n)."""
+    squeeze = r.dim() == 1
+    r2 = _as_rows(r)
+    B, n = r2.shape
+    ld = r2.stride(0)
+    code = _path_code(path)
+    if ws is None or not ws.fits(B, n, k, code):
+        ws = Workspace(B, n, k, code, r2.device)
+    if p is None:
+        p = torch.empty_like(r2)
+    if b is None:
+        b = torch.empty(B, dtype=torch.float64, device=r2.device)
+    sf = torch.empty(B, dtype=torch.float64, device=r2.device) if want_sum_f else None
+    _check(_lib().lapsum_forward(r2.data_ptr(), ld, p.data_ptr(), b.data_ptr(),
+                                 sf.data_ptr() if sf is not None else None, B, n, float(k),
+                                 float(t), code, seed & (2**64 - 1), ws.ptr, ws.nbytes,
+                                 _stream_ptr(r2.device)), "lapsum_forward")
+    if squeeze:
+        p = p[0]
+    return (p, b, sf) if want_sum_f else (p, b)
+
+
+def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Workspace = None,
+             g: torch.Tensor = None):
+    """g = J^T v for each row (J the Jacobian of p with respect to r)."""
+    squeeze = r.dim() == 1
+    r2 = _as_rows(r)
+    v2 = _as_rows(v)
+    B, n = r2.shape
+    if v2.shape != r2.shape:
+        raise ValueError("v must have the shape of r")
+    if v2.stride(0) != r2.stride(0):
+        v2 = v2.contiguous()
+        r2 = r2.contiguous()
+    ld = r2.stride(0)
+    if ws is None or not ws.fits_backward(B, n):
+        ws = Workspace(B, n, 0.5, "fullsort", r2.device)
+    if g is None:
+        g = torch.empty_like(r2)
+    if b.dtype != torch.float64 or not b.is_cuda:
+        raise TypeError("b must be a float64 CUDA tensor")
+    _check(_lib().lapsum_backward(r2.data_ptr(), ld, b.data_ptr(), v2.data_ptr(), g.data_ptr(), B,
+                                  n, float(t), ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
+           "lapsum_backward")
+    return g[0] if squeeze else g
+
+
+def read_status(ws: Workspace) -> int:
+    st = ctypes.c_int(0)
+    _check(_lib().lapsum_read_status(ws.ptr, _stream_ptr(ws.device), ctypes.byref(st)),
+           "lapsum_read_status")
+    return st.value
+
+
+def row_info(ws: Workspace, row: int = 0) -> dict:
+    info = RowInfo()
+    _check(_lib().lapsum_row_info_get(ws.ptr, row, ctypes.byref(info), _stream_ptr(ws.device)),
+           "lapsum_row_info_get")
+    return {name: getattr(info, name) for name, _ in RowInfo._fields_ if name != "reserved"}
+
+
+def sample_values(ws: Workspace, row: int, m: int):
+    import numpy as np
+    out = np.empty(m, dtype=np.float32)
+    _check(_lib().lapsum_sample_get(ws.ptr, row, out.ctypes.data, m, _stream_ptr(ws.device)),
+           "lapsum_sample_get")
+    return out
+
+
+def profile_enable(on: bool = True):
+    """Start (or stop) per-kernel CUDA-event timing inside the library."""
+    _check(_lib().lapsum_profile_enable(1 if on else 0), "lapsum_profile_enable")
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total device ms)} since profile_enable(True)."""
+    buf = (KernelTime * 64)()
+    cnt = ctypes.c_int(0)
+    _check(_lib().lapsum_profile_read(buf, 64, ctypes.byref(cnt)), "lapsum_profile_read")
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms))
+            for i in range(min(cnt.value, 64))}
+
+
+class LapSumTopK(torch.autograd.Function):
+    """Autograd wrapper: forward through lapsum_forward, backward through lapsum_backward."""
+
+    @staticmethod
+    def forward(ctx, r, k, t, path="auto", seed=0):
+        p, b = forward(r.detach(), k, t, path=path, seed=seed)
+        ctx.save_for_backward(r, b)
+        ctx.t = t
+        return p
+
+    @staticmethod
+    def backward(ctx, gp):
+        r, b = ctx.saved_tensors
+        g = backward(r.detach(), b, gp.contiguous(), ctx.t)
+        return g, None, None, None, None
+
+
+def soft_topk(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0) -> torch.Tensor:
+    """Differentiable soft top-k probabilities p with sum p = k per row."""
+    return LapSumTopK.apply(r, k, t, path, seed)

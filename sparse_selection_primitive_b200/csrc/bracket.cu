@@ -1,0 +1,790 @@
+// Probabilistic bracketing for very long rows.
+//
+// "Fast LapSum: Exact Differentiable Top-k at Million Scale" (gist.science
+// explainer pages), section 2.2, probabilistic bracketing:
+//   1. localization: draw a small sample of Laplace-noised scores and take two
+//      binomial order statistics as a bracket [a_L, a_R) holding b with high
+//      probability;
+//   2. streaming and filtering: one pass over the row folds the scores outside
+//      the bracket into stable tail sums and keeps the in-bracket middle band;
+//   3. exact solution: the exact solver runs on the band only;
+//   4. verification: a certification step checks the bracket and widens it
+//      when it fails, so the budget always holds exactly.
+//
+// Kernels (per row, stream-ordered, no host round trip):
+//   sample_kernel   1 CTA: counter-based sample y_s = r[I_s] + eps_s, radix
+//                   select of the descending ranks l and h -> (a_L, a_R);
+//   fold_kernel     grid: one pass over r (float4 loads); tail counts/sums per
+//                   thread in fp64, band compaction by warp ballot; per-CTA
+//                   partials combined in CTA order by the last CTA;
+//   solve_kernel    1 CTA: certify F(a_L) >= k >= F(a_R) from the tails and the
+//                   band; narrow a large band with exact histogram levels; sort
+//                   the final band (<= 4096) with the register bitonic network;
+//                   solve with the tails as virtual end anchors.  A failed
+//                   bracket moves the failing end to the next rung of its
+//                   ladder (4x the rank, then open) and the same CTA re-folds r.
+#include "bitonic.cuh"
+#include "lapsum_common.cuh"
+#include "lapsum_kernels.h"
+#include "solve_sorted.cuh"
+
+namespace lapsum {
+namespace {
+
+constexpr int kBlk = 1024;
+constexpr int kFoldThreads = 256;
+
+struct Ladder {
+    int64_t l[kLadder];  // descending ranks for a_R (0 = open)
+    int64_t h[kLadder];  // descending ranks for a_L (> m = open)
+};
+
+// ----------------------------------------------------------------------------
+// Block radix select: key of the rho-th largest (1-based) of m keys read via
+// `get`.  Levels of 11, 11 and 10 bits; the histogram lives in `hist` (2048
+// words of shared memory).  Every thread gets the result.
+// ----------------------------------------------------------------------------
+template <class Get>
+__device__ uint32_t block_select_desc(Get get, int m, int64_t rho, uint32_t* hist,
+                                      uint32_t* wsum, uint32_t* bcast) {
+    uint32_t prefix = 0, mask = 0;
+    int64_t remaining = rho;
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+    for (int lev = 0; lev < 3; ++lev) {
+        const int sh = shifts[lev];
+        const uint32_t nb = 1u << widths[lev];
+        for (uint32_t i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < m; i += blockDim.x) {
+            const uint32_t key = get(i);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+        }
+        __syncthreads();
+        // Suffix counts over bins: thread i owns bins 2i, 2i+1 (1024 threads).
+        const int i0 = 2 * threadIdx.x;
+        const uint32_t c0 = hist[i0], c1 = hist[i0 + 1];
+        uint32_t mine = c0 + c1;
+        // exclusive suffix over threads (higher threads first)
+        uint32_t incl = mine;
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t o = __shfl_down_sync(0xffffffffu, incl, d);
+            if (lane + d < 32) incl += o;
+        }
+        if (lane == 0) wsum[w] = incl;
+        __syncthreads();
+        uint32_t above = incl - mine;
+        for (int u = w + 1; u < (int)(blockDim.x >> 5); ++u) above += wsum[u];
+        // bins in descending order: bin i0+1 then i0
+        const int64_t s1 = above, s0 = above + c1;  // counts strictly above bin i0+1 / i0
+        if (s1 < remaining && remaining <= s1 + c1) {
+            bcast[0] = i0 + 1;
+            bcast[1] = (uint32_t)s1;
+        }
+        if (s0 < remaining && remaining <= s0 + c0) {
+            bcast[0] = i0;
+            bcast[1] = (uint32_t)s0;
+        }
+        __syncthreads();
+        const uint32_t bin = bcast[0];
+        remaining -= bcast[1];
+        prefix |= bin << sh;
+        mask |= (nb - 1) << sh;
+        __syncthreads();
+    }
+    return prefix;
+}
+
+struct SmemKeyGet {
+    const uint32_t* k;
+    __device__ __forceinline__ uint32_t operator()(int i) const { return k[i]; }
+};
+struct GlobalSampleKeyGet {
+    const float* y;
+    __device__ __forceinline__ uint32_t operator()(int i) const { return to_key(y[i]); }
+};
+
+// ----------------------------------------------------------------------------
+// 1. Localization sample.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ r, int64_t n,
+                                                      double t, uint64_t seed, uint64_t c0, int m,
+                                                      Ladder lad, int force_miss, int max_attempts,
+                                                      float* __restrict__ sample_out,
+                                                      RowState* st) {
+    extern __shared__ uint32_t dyn[];
+    uint32_t* keys = dyn;              // m keys
+    __shared__ uint32_t hist[2048];
+    __shared__ uint32_t wsum[32];
+    __shared__ uint32_t bcast[4];
+    const float tf = (float)t;
+    for (int s = threadIdx.x; s < m; s += kBlk) {
+        const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
+        const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
+        const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
+        const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
+        const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
+        const float eps = (u < 0.0 ? 1.f : -1.f) * tf * logf(a);
+        const float y = __ldg(r + I) + eps;
+        sample_out[s] = y;
+        keys[s] = to_key(y);
+    }
+    __syncthreads();
+    float aR = INFINITY, aL = -INFINITY;
+    if (lad.l[0] >= 1) {
+        const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.l[0], hist, wsum, bcast);
+        aR = from_key(kk);
+    }
+    if (lad.h[0] <= m) {
+        const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.h[0], hist, wsum, bcast);
+        aL = from_key(kk);
+    }
+    if (threadIdx.x == 0) {
+        st->ladder_R[0] = aR;
+        st->ladder_L[0] = aL;
+        st->rung_L = 0;
+        st->rung_R = 0;
+        if (force_miss) {
+            // A bracket above every sample value: F(a_L) < k, so it must fail.
+            uint32_t kmax = 0;
+            for (int s = 0; s < m; ++s) kmax = max(kmax, keys[s]);
+            const float top = from_key(kmax);
+            st->a_L = top + fabsf(top) + 1.f;
+            st->a_R = INFINITY;
+            st->rung_L = -1;
+        } else {
+            st->a_L = aL;
+            st->a_R = aR;
+        }
+        st->sample_m = m;
+        st->rank_l = (int32_t)lad.l[0];
+        st->rank_h = (int32_t)lad.h[0];
+        st->n_band = 0;
+        st->attempts = 1;
+        st->max_attempts = max_attempts;
+        st->force_miss = force_miss;
+        st->path = LAPSUM_PATH_BRACKET;
+        st->refine_levels = 0;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// 2. Streaming fold.
+// ----------------------------------------------------------------------------
+struct FoldAcc {
+    unsigned long long cntR;
+    double SL, SR;
+    bool bad;
+};
+
+__device__ __forceinline__ void fold_one(float x, float aL, float aR, float inv_t, FoldAcc& acc,
+                                         bool& in_band) {
+    acc.bad |= !finite_f(x);
+    in_band = false;
+    if (x >= aR) {
+        acc.cntR += 1;
+        acc.SR += (double)__expf((aR - x) * inv_t);
+    } else if (x < aL) {
+        acc.SL += (double)__expf((x - aL) * inv_t);
+    } else {
+        in_band = true;
+    }
+}
+
+// Warp-aggregated append of the lanes with `take` into band[] (capacity cap).
+__device__ __forceinline__ void band_append(bool take, float x, float* band,
+                                            unsigned long long* counter, unsigned long long cap) {
+    const unsigned ball = __ballot_sync(0xffffffffu, take);
+    if (ball == 0) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(ball) - 1;
+    unsigned long long base = 0;
+    if (lane == leader) base = atomicAdd(counter, (unsigned long long)__popc(ball));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (take) {
+        const unsigned long long pos = base + __popc(ball & ((1u << lane) - 1u));
+        if (pos < cap) band[pos] = x;
+    }
+}
+
+__global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restrict__ r, int64_t n,
+                                                            double t, RowState* st,
+                                                            float* __restrict__ band,
+                                                            double* __restrict__ part,
+                                                            uint32_t* __restrict__ ticket,
+                                                            WsHeader* hdr, int vec) {
+    __shared__ double red[kFoldThreads / 32];
+    __shared__ long long lred[kFoldThreads / 32];
+    __shared__ int flag;
+    const float aL = st->a_L, aR = st->a_R;
+    const float inv_t = (float)(1.0 / t);
+    FoldAcc acc{0ull, 0.0, 0.0, false};
+    unsigned long long* counter = &st->n_band;
+    const unsigned long long cap = (unsigned long long)n;
+    const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+    const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (vec) {
+        const int64_t n4 = n >> 2;
+        const float4* r4 = reinterpret_cast<const float4*>(r);
+        // uniform trip count per warp so the ballots below see full warps
+        const int64_t iters = (n4 + nthreads - 1) / nthreads;
+        for (int64_t it = 0; it < iters; ++it) {
+            const int64_t i = it * nthreads + gtid;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            const bool ok = i < n4;
+            if (ok) v = __ldcs(r4 + i);
+            bool b0 = false, b1 = false, b2 = false, b3 = false;
+            if (ok) {
+                fold_one(v.x, aL, aR, inv_t, acc, b0);
+                fold_one(v.y, aL, aR, inv_t, acc, b1);
+                fold_one(v.z, aL, aR, inv_t, acc, b2);
+                fold_one(v.w, aL, aR, inv_t, acc, b3);
+            }
+            band_append(b0, v.x, band, counter, cap);
+            band_append(b1, v.y, band, counter, cap);
+            band_append(b2, v.z, band, counter, cap);
+            band_append(b3, v.w, band, counter, cap);
+        }
+        // tail elements (n not a multiple of 4)
+        const int64_t rem0 = n4 << 2;
+        if (blockIdx.x == 0 && threadIdx.x < 32) {
+            const int64_t i = rem0 + threadIdx.x;
+            bool bb = false;
+            float x = 0.f;
+            if (i < n) {
+                x = r[i];
+                fold_one(x, aL, aR, inv_t, acc, bb);
+            }
+            band_append(bb, x, band, counter, cap);
+        }
+    } else {
+        const int64_t iters = (n + nthreads - 1) / nthreads;
+        for (int64_t it = 0; it < iters; ++it) {
+            const int64_t i = it * nthreads + gtid;
+            bool bb = false;
+            float x = 0.f;
+            if (i < n) {
+                x = r[i];
+                fold_one(x, aL, aR, inv_t, acc, bb);
+            }
+            band_append(bb, x, band, counter, cap);
+        }
+    }
+    const long long cR = block_sum_ll((long long)acc.cntR, lred);
+    const double sL = block_sum_d(acc.SL, red);
+    const double sR = block_sum_d(acc.SR, red);
+    const int any_bad = __syncthreads_or(acc.bad);
+    if (threadIdx.x == 0) {
+        part[blockIdx.x * 4 + 0] = (double)cR;
+        part[blockIdx.x * 4 + 1] = sL;
+        part[blockIdx.x * 4 + 2] = sR;
+        part[blockIdx.x * 4 + 3] = any_bad ? 1.0 : 0.0;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t prev = atomicAdd(ticket, 1u);
+        flag = (prev == gridDim.x - 1);
+        if (flag) *ticket = 0u;
+    }
+    __syncthreads();
+    if (!flag) return;
+    __threadfence();
+    double c = 0.0, a = 0.0, bsum = 0.0, badsum = 0.0;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x) {
+        c += part[i * 4 + 0];
+        a += part[i * 4 + 1];
+        bsum += part[i * 4 + 2];
+        badsum += part[i * 4 + 3];
+    }
+    c = block_sum_d(c, red);
+    a = block_sum_d(a, red);
+    bsum = block_sum_d(bsum, red);
+    badsum = block_sum_d(badsum, red);
+    if (threadIdx.x == 0) {
+        st->cnt_R = (unsigned long long)c;
+        st->S_L = a;
+        st->S_R = bsum;
+        if (badsum > 0.0) {
+            st->status |= kDevNonFinite;
+            set_status(hdr, kDevNonFinite);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// 3-4. Exact band solve, certification, narrowing and widening (one CTA).
+// ----------------------------------------------------------------------------
+struct FloatGet {
+    const float* s;
+    __device__ __forceinline__ float operator()(long long j) const { return s[j]; }
+};
+struct ConstGet {
+    float v;
+    __device__ __forceinline__ float operator()(long long) const { return v; }
+};
+
+struct SolveSmemAll {
+    SolveScratch ss;
+    SolveResult res;
+    double red[32];
+    float fred[32];
+    long long lred[32];
+    uint32_t wsum[32];
+    uint32_t bcast[8];
+    unsigned long long cnt;
+    int flag;
+    union {
+        struct {
+            uint32_t xch[4 * kBlk];
+            float sorted[kBandSortMax];
+        } sort;
+        struct {
+            uint32_t cnt[kRefineBins];
+            float U[kRefineBins];
+            float L[kRefineBins];
+            double F[kRefineBins + 1];
+        } hist;
+        uint32_t sel_hist[2048];
+    } u;
+};
+
+// Band of size <= 4096: sort on chip and solve with the tails.
+__device__ void solve_small_band(const float* band, long long nb, const Tails& tl, double k,
+                                 double t, SolveSmemAll* sm) {
+    uint32_t key[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const long long j = (long long)threadIdx.x * 4 + e;
+        key[e] = j < nb ? to_key(band[j]) : 0xffffffffu;
+    }
+    bitonic_sort_row<4, kBlk, kBlk>(key, threadIdx.x, sm->u.sort.xch);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const long long j = (long long)threadIdx.x * 4 + e;
+        if (j < nb) sm->u.sort.sorted[j] = from_key(key[e]);
+    }
+    __syncthreads();
+    solve_sorted_block(FloatGet{sm->u.sort.sorted}, nb, tl, k, t, &sm->ss, &sm->res);
+}
+
+// Exact F at the ends of [tl.aL, tl.aR) from a band in global memory (any size),
+// plus the band's key range.
+__device__ void certify_big_band(const float* band, long long nb, const Tails& tl, double t,
+                                 SolveSmemAll* sm, double* F_aL, double* F_aR, uint32_t* kmin,
+                                 uint32_t* kmax) {
+    double wl = 0.0, vr = 0.0;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    const double inv_t = 1.0 / t;
+    for (long long j = threadIdx.x; j < nb; j += blockDim.x) {
+        const float s = band[j];
+        if (tl.hasL) wl += (double)__expf((float)((tl.aL - s) * inv_t));
+        if (tl.hasR) vr += (double)__expf((float)((s - tl.aR) * inv_t));
+        const uint32_t kk = to_key(s);
+        lo = min(lo, kk);
+        hi = max(hi, kk);
+    }
+    wl = block_sum_d(wl, sm->red);
+    vr = block_sum_d(vr, sm->red);
+    // key min/max through the float reductions' shared slots
+    {
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, d));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, d));
+        }
+        __syncthreads();
+        if (lane == 0) {
+            sm->wsum[w] = lo;
+            sm->u.sel_hist[w] = hi;
+        }
+        __syncthreads();
+        lo = 0xffffffffu;
+        hi = 0u;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+            lo = min(lo, sm->wsum[i]);
+            hi = max(hi, sm->u.sel_hist[i]);
+        }
+        __syncthreads();
+    }
+    const double lnw = (tl.hasL && tl.hasR) ? ((double)tl.aL - (double)tl.aR) / t : -INFINITY;
+    *F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * (wl + tl.SR * exp(lnw)) + 0.5 * tl.SL : INFINITY;
+    *F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * (vr + tl.SL * exp(lnw)) : -INFINITY;
+    *kmin = lo;
+    *kmax = hi;
+}
+
+// One narrowing level of a certified band in `in` (nb > 4096, kmin < kmax):
+// histogram the band over <= 2048 key bins with per-bin exponential sums,
+// evaluate F at every bin edge by two affine scans, pick the edge pair that
+// straddles k, verify it with exact fp64 sums (moving one bin if rounding in
+// the histogram picked the wrong one), and compact that bin into `out`.
+// Returns the new band size; updates the tails in place.
+__device__ long long refine_level(const float* in, long long nb, float* out, Tails& tl,
+                                  uint32_t kmin, uint32_t kmax, double k, double t,
+                                  SolveSmemAll* sm, uint32_t* nkmin, uint32_t* nkmax) {
+    const float inv_t = (float)(1.0 / t);
+    const uint32_t range = kmax - kmin;
+    int sh = 0;
+    while ((range >> sh) >= (uint32_t)kRefineBins) ++sh;
+    const int nbin = (int)(range >> sh) + 1;
+    auto edge_key = [&](int j) -> uint32_t {
+        const unsigned long long e = (unsigned long long)kmin + ((unsigned long long)j << sh);
+        const unsigned long long top = (unsigned long long)kmax + 1ull;
+        return (uint32_t)(e < top ? e : top);
+    };
+    auto edge = [&](int j) -> float { return from_key(edge_key(j)); };
+
+    for (int j = threadIdx.x; j < kRefineBins; j += blockDim.x) {
+        sm->u.hist.cnt[j] = 0;
+        sm->u.hist.U[j] = 0.f;
+        sm->u.hist.L[j] = 0.f;
+    }
+    __syncthreads();
+    for (long long i = threadIdx.x; i < nb; i += blockDim.x) {
+        const float s = in[i];
+        const int j = (int)((to_key(s) - kmin) >> sh);
+        atomicAdd(&sm->u.hist.cnt[j], 1u);
+        atomicAdd(&sm->u.hist.U[j], __expf((edge(j) - s) * inv_t));
+        atomicAdd(&sm->u.hist.L[j], __expf((s - edge(j + 1)) * inv_t));
+    }
+    __syncthreads();
+    // F at every edge (one thread; nbin <= 2048, fp64).  Runs once per level.
+    if (threadIdx.x == 0) {
+        double Q = tl.hasR ? tl.SR * exp(((double)edge(nbin) - (double)tl.aR) / t) : 0.0;
+        double above = tl.cntR;
+        sm->u.hist.F[nbin] = 0.0;  // filled below with the forward part
+        // backward: store cnt_above - Q/2 at each edge
+        double* F = sm->u.hist.F;
+        F[nbin] = above - 0.5 * Q;
+        for (int j = nbin - 1; j >= 0; --j) {
+            const double gam = exp(((double)edge(j) - (double)edge(j + 1)) / t);
+            Q = (double)sm->u.hist.U[j] + Q * gam;
+            above += (double)sm->u.hist.cnt[j];
+            F[j] = above - 0.5 * Q;
+        }
+        double P = tl.hasL ? tl.SL * exp(((double)tl.aL - (double)edge(0)) / t) : 0.0;
+        F[0] += 0.5 * P;
+        for (int j = 1; j <= nbin; ++j) {
+            const double gam = exp(((double)edge(j - 1) - (double)edge(j)) / t);
+            P = (double)sm->u.hist.L[j - 1] + P * gam;
+            F[j] += 0.5 * P;
+        }
+        int c = 0;
+        for (int j = 0; j <= nbin; ++j) c += (F[j] >= k) ? 1 : 0;
+        sm->bcast[0] = (uint32_t)(c - 1);  // edge index of the new lower end (-1: use aL)
+    }
+    __syncthreads();
+    int jc = (int)sm->bcast[0];
+    long long cnt = 0;
+    for (int guard = 0; guard < nbin + 2; ++guard) {
+        const bool useL = jc < 0, useR = jc + 1 > nbin;
+        const float Elo = useL ? tl.aL : edge(jc);
+        const float Ehi = useR ? tl.aR : edge(jc + 1);
+        const bool hasLo = useL ? tl.hasL : true;
+        const bool hasHi = useR ? tl.hasR : true;
+        if (threadIdx.x == 0) sm->cnt = 0ull;
+        __syncthreads();
+        double sl = 0.0, sr = 0.0, w = 0.0, v = 0.0;
+        long long cr = 0;
+        uint32_t lo = 0xffffffffu, hi = 0u;
+        for (long long i = threadIdx.x; i < nb; i += blockDim.x) {
+            const float s = in[i];
+            bool take = false;
+            if (hasHi && s >= Ehi) {
+                cr += 1;
+                sr += (double)__expf((Ehi - s) * inv_t);
+            } else if (hasLo && s < Elo) {
+                sl += (double)__expf((s - Elo) * inv_t);
+            } else {
+                take = true;
+                if (hasLo) w += (double)__expf((Elo - s) * inv_t);
+                if (hasHi) v += (double)__expf((s - Ehi) * inv_t);
+                const uint32_t kk = to_key(s);
+                lo = min(lo, kk);
+                hi = max(hi, kk);
+            }
+            if (take) {
+                const unsigned long long pos = atomicAdd(&sm->cnt, 1ull);
+                out[pos] = s;
+            }
+        }
+        sl = block_sum_d(sl, sm->red);
+        sr = block_sum_d(sr, sm->red);
+        w = block_sum_d(w, sm->red);
+        v = block_sum_d(v, sm->red);
+        cr = block_sum_ll(cr, sm->lred);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, d));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, d));
+        }
+        if ((threadIdx.x & 31) == 0) {
+            atomicMin(&sm->bcast[2], lo);
+            atomicMax(&sm->bcast[3], hi);
+        }
+        __syncthreads();
+        cnt = (long long)sm->cnt;
+        // new tails
+        Tails nt;
+        nt.hasL = hasLo;
+        nt.aL = Elo;
+        nt.SL = (useL ? tl.SL : (tl.hasL ? tl.SL * exp(((double)tl.aL - (double)Elo) / t) : 0.0)) + sl;
+        nt.hasR = hasHi;
+        nt.aR = Ehi;
+        nt.SR = (useR ? tl.SR : (tl.hasR ? tl.SR * exp(((double)Ehi - (double)tl.aR) / t) : 0.0)) + sr;
+        nt.cntR = tl.cntR + (double)cr;
+        const double lnw = (hasLo && hasHi) ? ((double)Elo - (double)Ehi) / t : -INFINITY;
+        const double FL = hasLo ? nt.cntR + (double)cnt - 0.5 * (w + nt.SR * exp(lnw)) + 0.5 * nt.SL
+                                : INFINITY;
+        const double FR = hasHi ? nt.cntR - 0.5 * nt.SR + 0.5 * (v + nt.SL * exp(lnw)) : -INFINITY;
+        const uint32_t klo = sm->bcast[2], khi = sm->bcast[3];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            sm->bcast[2] = 0xffffffffu;
+            sm->bcast[3] = 0u;
+        }
+        if (FL < k && jc >= 0) {
+            --jc;
+        } else if (FR > k && jc + 1 <= nbin) {
+            ++jc;
+        } else {
+            tl = nt;
+            *nkmin = klo;
+            *nkmax = khi;
+            __syncthreads();
+            return cnt;
+        }
+        __syncthreads();
+    }
+    return -1;  // unreachable for a certified input band
+}
+
+// Single-CTA fold of the whole row (used only after a failed bracket).
+__device__ void refold_row(const float* __restrict__ r, int64_t n, float aL, float aR, double t,
+                           float* band, SolveSmemAll* sm, Tails& tl, long long* nb) {
+    const float inv_t = (float)(1.0 / t);
+    if (threadIdx.x == 0) sm->cnt = 0ull;
+    __syncthreads();
+    FoldAcc acc{0ull, 0.0, 0.0, false};
+    const int64_t iters = (n + blockDim.x - 1) / blockDim.x;
+    for (int64_t it = 0; it < iters; ++it) {
+        const int64_t i = it * blockDim.x + threadIdx.x;
+        bool bb = false;
+        float x = 0.f;
+        if (i < n) {
+            x = r[i];
+            fold_one(x, aL, aR, inv_t, acc, bb);
+        }
+        band_append(bb, x, band, &sm->cnt, (unsigned long long)n);
+    }
+    const double sL = block_sum_d(acc.SL, sm->red);
+    const double sR = block_sum_d(acc.SR, sm->red);
+    const long long cR = block_sum_ll((long long)acc.cntR, sm->lred);
+    __syncthreads();
+    tl.hasL = isfinite(aL);
+    tl.aL = aL;
+    tl.SL = sL;
+    tl.hasR = isfinite(aR);
+    tl.aR = aR;
+    tl.SR = sR;
+    tl.cntR = (double)cR;
+    *nb = (long long)sm->cnt;
+}
+
+__global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r, int64_t n,
+                                                     double k, double t, RowState* st,
+                                                     float* __restrict__ band0,
+                                                     float* __restrict__ band1,
+                                                     const float* __restrict__ sample, int m,
+                                                     Ladder lad, double* __restrict__ b_out,
+                                                     WsHeader* hdr) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    if (threadIdx.x == 0) {
+        sm->bcast[2] = 0xffffffffu;
+        sm->bcast[3] = 0u;
+    }
+    __syncthreads();
+    if (st->status & kDevNonFinite) {
+        if (threadIdx.x == 0) {
+            st->b = nan("");
+            *b_out = nan("");
+        }
+        return;
+    }
+    Tails tl;
+    tl.hasL = isfinite(st->a_L);
+    tl.aL = st->a_L;
+    tl.SL = st->S_L;
+    tl.hasR = isfinite(st->a_R);
+    tl.aR = st->a_R;
+    tl.SR = st->S_R;
+    tl.cntR = (double)st->cnt_R;
+    long long nb = (long long)st->n_band;
+    int rungL = st->rung_L, rungR = st->rung_R;
+    const int max_attempts = st->max_attempts;
+    int attempt = 1;
+    int levels = 0;
+    bool done = false;
+    double b = nan("");
+    Tails cert = tl;
+    long long nb_cert = nb;
+    while (true) {
+        float* cur = band0;
+        float* nxt = band1;
+        bool certified;
+        cert = tl;
+        nb_cert = nb;
+        if (nb <= kBandSortMax) {
+            solve_small_band(cur, nb, tl, k, t, sm);
+            certified = sm->res.F_aL >= k && sm->res.F_aR <= k;
+            if (certified) {
+                b = sm->res.b;
+                done = true;
+            }
+        } else {
+            double FL, FR;
+            uint32_t kmin, kmax;
+            certify_big_band(cur, nb, tl, t, sm, &FL, &FR, &kmin, &kmax);
+            certified = FL >= k && FR <= k;
+            if (certified) {
+                // narrow until the band fits on chip or holds a single value
+                while (nb > kBandSortMax && kmin < kmax) {
+                    uint32_t nkmin = 0, nkmax = 0;
+                    nb = refine_level(cur, nb, nxt, tl, kmin, kmax, k, t, sm, &nkmin, &nkmax);
+                    if (nb < 0) break;  // no certified bin (not expected): reported as a failure
+                    ++levels;
+                    float* tmp = cur;
+                    cur = nxt;
+                    nxt = tmp;
+                    kmin = nkmin;
+                    kmax = nkmax;
+                }
+                if (nb < 0) {
+                    certified = false;
+                    break;
+                } else if (nb <= kBandSortMax) {
+                    solve_small_band(cur, nb, tl, k, t, sm);
+                } else {
+                    solve_sorted_block(ConstGet{from_key(kmin)}, nb, tl, k, t, &sm->ss, &sm->res);
+                }
+                b = sm->res.b;
+                done = true;
+            } else {
+                // F at the ends is enough to know which end failed
+                if (threadIdx.x == 0) {
+                    sm->res.F_aL = FL;
+                    sm->res.F_aR = FR;
+                }
+                __syncthreads();
+            }
+        }
+        if (done || attempt >= max_attempts) break;
+        // widen the failing end to its next rung and fold again
+        const bool fail_left = sm->res.F_aL < k;
+        float aL = tl.aL, aR = tl.aR;
+        if (!tl.hasL) aL = -INFINITY;
+        if (!tl.hasR) aR = INFINITY;
+        if (fail_left) {
+            ++rungL;
+            if (rungL >= kLadder - 1 || lad.h[rungL] > m) {
+                aL = -INFINITY;
+            } else {
+                aL = from_key(block_select_desc(GlobalSampleKeyGet{sample}, m, lad.h[rungL],
+                                                sm->u.sel_hist, sm->wsum, sm->bcast + 4));
+            }
+        } else {
+            ++rungR;
+            if (rungR >= kLadder - 1 || lad.l[rungR] < 1) {
+                aR = INFINITY;
+            } else {
+                aR = from_key(block_select_desc(GlobalSampleKeyGet{sample}, m, lad.l[rungR],
+                                                sm->u.sel_hist, sm->wsum, sm->bcast + 4));
+            }
+        }
+        ++attempt;
+        refold_row(r, n, aL, aR, t, band0, sm, tl, &nb);
+    }
+    if (threadIdx.x == 0) {
+        st->attempts = attempt;
+        st->refine_levels = levels;
+        st->rung_L = rungL;
+        st->rung_R = rungR;
+        st->a_L = cert.hasL ? cert.aL : -INFINITY;
+        st->a_R = cert.hasR ? cert.aR : INFINITY;
+        st->S_L = cert.SL;
+        st->S_R = cert.SR;
+        st->cnt_R = (unsigned long long)cert.cntR;
+        st->n_band = (unsigned long long)nb_cert;
+        st->certified = done ? 1 : 0;
+        if (!done) {
+            b = nan("");
+            st->status |= kDevBracketExhausted;
+            set_status(hdr, kDevBracketExhausted);
+        }
+        st->b = b;
+        *b_out = b;
+    }
+}
+
+}  // namespace
+
+int bracket_fold_grid() {
+    static int grid = 0;
+    if (grid == 0) {
+        int dev = 0, sms = 148, per = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fold_kernel, kFoldThreads, 0);
+        grid = sms * (per > 0 ? per : 1);
+    }
+    return grid;
+}
+
+cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t, uint64_t seed,
+                               int64_t row, int m, int64_t rank_l[kLadder],
+                               int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,
+                               RowState* st_row, double* b_out, WsHeader* hdr, cudaStream_t st) {
+    static bool attr_done = false;
+    const size_t solve_smem = sizeof(SolveSmemAll);
+    const size_t sample_smem = (size_t)m * sizeof(uint32_t);
+    if (!attr_done) {
+        cudaFuncSetAttribute(solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)solve_smem);
+        cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kSampleMax * sizeof(uint32_t)));
+        attr_done = true;
+    }
+    Ladder lad;
+    for (int i = 0; i < kLadder; ++i) {
+        lad.l[i] = rank_l[i];
+        lad.h[i] = rank_h[i];
+    }
+    const int force_miss = (flags & LAPSUM_FLAG_FORCE_MISS) ? 1 : 0;
+    const int max_attempts = (flags & LAPSUM_FLAG_NO_RETRY) ? 1 : kMaxAttempts;
+    float* sample = buf.sample + row * (int64_t)kSampleMax;
+    const uint64_t c0 = (uint64_t)row << 32;
+    {
+        ProfScope ps_("bracket_sample", st);
+        sample_kernel<<<1, kBlk, sample_smem, st>>>(r_row, n, t, seed, c0, m, lad, force_miss,
+                                                max_attempts, sample, st_row);
+    }
+    const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
+    {
+        ProfScope ps_("bracket_fold", st);
+        fold_kernel<<<buf.fold_grid, kFoldThreads, 0, st>>>(r_row, n, t, st_row, buf.band[0],
+                                                        buf.fold_part, buf.ticket, hdr, vec);
+    }
+    {
+        ProfScope ps_("bracket_solve", st);
+        solve_kernel<<<1, kBlk, solve_smem, st>>>(r_row, n, k, t, st_row, buf.band[0], buf.band[1],
+                                              sample, m, lad, b_out, hdr);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace lapsum

@@ -1,0 +1,425 @@
+// C ABI of the Fast LapSum library: argument checks, workspace layout, solver
+// dispatch.  Every entry point is declared and documented in include/lapsum.h.
+//
+// Solver choice follows "Fast LapSum: Exact Differentiable Top-k at Million
+// Scale" (gist.science explainer pages), section 2.2: the full-sort solver
+// where sorting is affordable, probabilistic bracketing for n > 10^6.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "lapsum_common.cuh"
+#include "lapsum_kernels.h"
+
+namespace lapsum {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int64_t kOnchipMax = 4096;
+constexpr int64_t kRadixMax = int64_t(1) << 20;
+constexpr int kFoldGridMax = 4096;
+constexpr int64_t kGridYMax = 65535;
+constexpr double kBracketAlpha = 1e-6;  // miss probability allowed per bracket end
+
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int resolve_path(int64_t n, int path) {
+    switch (path & 0xff) {
+        case LAPSUM_PATH_AUTO:
+            return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT
+                                   : (n <= kRadixMax ? LAPSUM_PATH_RADIX : LAPSUM_PATH_BRACKET);
+        case LAPSUM_PATH_FULLSORT:
+            return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT : LAPSUM_PATH_RADIX;
+        case LAPSUM_PATH_BRACKET: return LAPSUM_PATH_BRACKET;
+        case LAPSUM_PATH_RADIX: return LAPSUM_PATH_RADIX;
+        default: return -1;
+    }
+}
+
+struct Layout {
+    size_t header, rows, partials, row_R, tickets;
+    size_t keys0, keys1, seg_hist, tile_hist, plan;
+    size_t sample, band0, band1, fold_part, fold_ticket;
+    size_t total;
+};
+
+Layout make_layout(int64_t B, int64_t n, int rpath) {
+    Layout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += up(bytes);
+        return o;
+    };
+    const int64_t tiles = stream_tiles(n);
+    L.header = take(sizeof(WsHeader));
+    L.tickets = take((size_t)B * 2 * sizeof(uint32_t) + sizeof(uint32_t));
+    L.fold_ticket = L.tickets + (size_t)B * 2 * sizeof(uint32_t);
+    L.rows = take((size_t)B * 512);
+    L.partials = take((size_t)B * (size_t)tiles * 3 * sizeof(double));
+    L.row_R = take((size_t)B * sizeof(double));
+    if (rpath == LAPSUM_PATH_RADIX) {
+        const int64_t rt = radix_tiles(n);
+        L.keys0 = take((size_t)B * (size_t)n * sizeof(uint32_t));
+        L.keys1 = take((size_t)B * (size_t)n * sizeof(uint32_t));
+        L.seg_hist = take((size_t)B * 1024 * sizeof(uint32_t));
+        L.tile_hist = take((size_t)B * 256 * (size_t)rt * sizeof(uint32_t));
+        L.plan = take((size_t)B * 8 * sizeof(int32_t));
+    }
+    if (rpath == LAPSUM_PATH_BRACKET) {
+        L.sample = take((size_t)B * kSampleMax * sizeof(float));
+        L.band0 = take((size_t)n * sizeof(float));
+        L.band1 = take((size_t)n * sizeof(float));
+        L.fold_part = take((size_t)kFoldGridMax * 4 * sizeof(double));
+    }
+    L.total = off;
+    return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA; }
+
+// Binomial(m, q) order-statistic ranks (descending, 1-based) for one bracket:
+// l = largest with P(C < l) <= alpha, h = smallest with P(C >= h) <= alpha.
+void binomial_ranks(int64_t m, double q, double alpha, int64_t* l, int64_t* h) {
+    auto logpmf = [&](int64_t c) {
+        return std::lgamma((double)m + 1.0) - std::lgamma((double)c + 1.0) -
+               std::lgamma((double)(m - c) + 1.0) + (double)c * std::log(q) +
+               (double)(m - c) * std::log1p(-q);
+    };
+    double cdf = 0.0;
+    int64_t lo = 0;
+    for (int64_t c = 0; c <= m; ++c) {
+        cdf += std::exp(logpmf(c));
+        if (cdf <= alpha) lo = c + 1;
+        else break;
+    }
+    double sf = 0.0;
+    int64_t hi = m + 1;
+    for (int64_t c = m; c >= 0; --c) {
+        sf += std::exp(logpmf(c));
+        if (sf <= alpha) hi = c;
+        else break;
+    }
+    *l = lo;
+    *h = hi;
+}
+
+int sample_size(int64_t n, double k) {
+    const double q = k / (double)n;
+    double want = 64.0 / q;
+    int m = 4096;
+    while (m < kSampleMax && m < want) m <<= 1;
+    return m;
+}
+
+// --- optional per-kernel event timing ---------------------------------------
+struct ProfRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    std::vector<ProfRec> recs;
+    std::vector<cudaEvent_t> pool;
+    int open = -1;
+    cudaEvent_t get() {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        cudaEventCreate(&e);
+        return e;
+    }
+    void recycle() {
+        for (auto& r : recs) {
+            pool.push_back(r.a);
+            pool.push_back(r.b);
+        }
+        recs.clear();
+        open = -1;
+    }
+};
+Profiler& profiler() {
+    static Profiler p;
+    return p;
+}
+
+}  // namespace
+
+void prof_begin(const char* name, cudaStream_t st) {
+    Profiler& p = profiler();
+    if (!p.on) return;
+    std::lock_guard<std::mutex> g(p.mu);
+    ProfRec r{name, p.get(), p.get()};
+    cudaEventRecord(r.a, st);
+    p.recs.push_back(r);
+    p.open = (int)p.recs.size() - 1;
+}
+
+void prof_end(cudaStream_t st) {
+    Profiler& p = profiler();
+    if (!p.on) return;
+    std::lock_guard<std::mutex> g(p.mu);
+    if (p.open >= 0) cudaEventRecord(p.recs[p.open].b, st);
+    p.open = -1;
+}
+
+}  // namespace lapsum
+
+using namespace lapsum;
+
+extern "C" {
+
+int lapsum_abi_version(void) { return 1; }
+
+const char* lapsum_status_string(int status) {
+    switch (status) {
+        case LAPSUM_OK: return "ok";
+        case LAPSUM_EINVAL: return "invalid argument";
+        case LAPSUM_EWORKSPACE: return "workspace missing, misaligned or too small";
+        case LAPSUM_ENONFINITE: return "non-finite score";
+        case LAPSUM_EBRACKET: return "bracketing retries exhausted";
+        case LAPSUM_ECUDA: return "CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+size_t lapsum_workspace_bytes(int64_t B, int64_t n, double k, int path) {
+    (void)k;
+    if (B < 1 || n < 1) return 0;
+    const int rp = resolve_path(n, path);
+    if (rp < 0) return 0;
+    return make_layout(B, n, rp).total;
+}
+
+size_t lapsum_backward_workspace_bytes(int64_t B, int64_t n) {
+    if (B < 1 || n < 1) return 0;
+    return make_layout(B, n, LAPSUM_PATH_FULLSORT).total;
+}
+
+int lapsum_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (ws == nullptr || ws_bytes < sizeof(WsHeader) ||
+        (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0)
+        return LAPSUM_EWORKSPACE;
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
+                   int64_t n, double k, double t, int path, uint64_t seed, void* ws,
+                   size_t ws_bytes, void* stream) {
+    if (r == nullptr || p == nullptr || b == nullptr) return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
+    if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    const int rp = resolve_path(n, path);
+    if (rp < 0 || (path & ~0x3ff) != 0) return LAPSUM_EINVAL;
+    if (n > INT32_MAX && rp != LAPSUM_PATH_BRACKET) return LAPSUM_EINVAL;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const Layout L = make_layout(B, n, rp);
+    if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* w = static_cast<char*>(ws);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(w + L.header);
+    RowState* rows = reinterpret_cast<RowState*>(w + L.rows);
+    uint32_t* tickets = reinterpret_cast<uint32_t*>(w + L.tickets);
+    double* partials = reinterpret_cast<double*>(w + L.partials);
+    const int vec = (aligned16(r) && aligned16(p) && (ld % 4) == 0) ? 1 : 0;
+    cudaError_t e = cudaSuccess;
+
+    if (rp == LAPSUM_PATH_FULLSORT) {
+        e = launch_onchip_forward(r, ld, p, b, sum_f, B, (int)n, k, t, hdr, vec, st);
+        return cuda_status(e);
+    }
+    e = cudaMemsetAsync(rows, 0, (size_t)B * 512, st);
+    if (e != cudaSuccess) return LAPSUM_ECUDA;
+    if (rp == LAPSUM_PATH_RADIX) {
+        RadixBuffers rb;
+        rb.keys[0] = reinterpret_cast<uint32_t*>(w + L.keys0);
+        rb.keys[1] = reinterpret_cast<uint32_t*>(w + L.keys1);
+        rb.seg_hist = reinterpret_cast<uint32_t*>(w + L.seg_hist);
+        rb.tile_hist = reinterpret_cast<uint32_t*>(w + L.tile_hist);
+        rb.plan = reinterpret_cast<int32_t*>(w + L.plan);
+        for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
+            const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+            RadixBuffers sub = rb;
+            sub.keys[0] += r0 * n;
+            sub.keys[1] += r0 * n;
+            sub.seg_hist += r0 * 1024;
+            sub.tile_hist += r0 * 256 * radix_tiles(n);
+            sub.plan += r0 * 8;
+            e = launch_radix_sort_rows(r + r0 * ld, ld, nb, n, sub, rows + r0, hdr, st);
+            if (e == cudaSuccess)
+                e = launch_rowsolve_sorted_keys(sub, nb, n, k, t, b + r0, rows + r0, hdr, st);
+        }
+    } else {
+        BracketBuffers bb;
+        bb.sample = reinterpret_cast<float*>(w + L.sample);
+        bb.band[0] = reinterpret_cast<float*>(w + L.band0);
+        bb.band[1] = reinterpret_cast<float*>(w + L.band1);
+        bb.fold_part = reinterpret_cast<double*>(w + L.fold_part);
+        bb.ticket = reinterpret_cast<uint32_t*>(w + L.fold_ticket);
+        bb.fold_grid = bracket_fold_grid();
+        if (bb.fold_grid > kFoldGridMax) bb.fold_grid = kFoldGridMax;
+        const int m = sample_size(n, k);
+        int64_t l0, h0;
+        binomial_ranks(m, k / (double)n, kBracketAlpha, &l0, &h0);
+        int64_t rl[kLadder], rh[kLadder];
+        for (int i = 0; i < kLadder - 1; ++i) {
+            rl[i] = l0 >> (2 * i);
+            rh[i] = h0 << (2 * i);
+            if (rh[i] > m) rh[i] = m + 1;
+        }
+        rl[kLadder - 1] = 0;
+        rh[kLadder - 1] = m + 1;
+        for (int64_t row = 0; row < B && e == cudaSuccess; ++row) {
+            e = launch_bracket_row(r + row * ld, n, k, t, seed, row, m, rl, rh, path, bb,
+                                   rows + row, b + row, hdr, st);
+        }
+    }
+    if (e != cudaSuccess) return LAPSUM_ECUDA;
+    for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
+        const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+        e = launch_emit(r + r0 * ld, ld, p + r0 * ld, b + r0, sum_f ? sum_f + r0 : nullptr, nb, n,
+                        t, partials + r0 * stream_tiles(n), tickets + r0, vec,
+                        r0 == 0 ? hdr : nullptr, B, rp, st);
+    }
+    return cuda_status(e);
+}
+
+int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v, float* g,
+                    int64_t B, int64_t n, double t, void* ws, size_t ws_bytes, void* stream) {
+    if (r == nullptr || b == nullptr || v == nullptr || g == nullptr) return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int vec = (aligned16(r) && aligned16(v) && aligned16(g) && (ld % 4) == 0) ? 1 : 0;
+    if (n <= kOnchipMax) {
+        return cuda_status(launch_onchip_backward(r, ld, b, v, g, B, (int)n, t, vec, st));
+    }
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const Layout L = make_layout(B, n, LAPSUM_PATH_FULLSORT);  // the streaming buffers only
+    if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+    char* w = static_cast<char*>(ws);
+    uint32_t* tickets = reinterpret_cast<uint32_t*>(w + L.tickets);
+    double* partials = reinterpret_cast<double*>(w + L.partials);
+    double* row_R = reinterpret_cast<double*>(w + L.row_R);
+    cudaError_t e = cudaSuccess;
+    for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
+        const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+        e = launch_backward_stream(r + r0 * ld, ld, b + r0, v + r0 * ld, g + r0 * ld, nb, n, t,
+                                   partials + r0 * stream_tiles(n) * 3, row_R + r0,
+                                   tickets + B + r0, vec, st);
+    }
+    return cuda_status(e);
+}
+
+int lapsum_read_status(void* ws, void* stream, int* device_status) {
+    if (ws == nullptr || device_status == nullptr) return LAPSUM_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    WsHeader* hdr = static_cast<WsHeader*>(ws);
+    uint32_t bits = 0;
+    cudaError_t e = cudaMemcpyAsync(&bits, &hdr->status, sizeof(bits), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(&hdr->status, 0, sizeof(uint32_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return LAPSUM_ECUDA;
+    *device_status = (bits & kDevNonFinite) ? LAPSUM_ENONFINITE
+                     : (bits & kDevBracketExhausted) ? LAPSUM_EBRACKET
+                                                     : LAPSUM_OK;
+    return LAPSUM_OK;
+}
+
+int lapsum_row_info_get(void* ws, int64_t row, lapsum_row_info* out, void* stream) {
+    if (ws == nullptr || out == nullptr || row < 0) return LAPSUM_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    // The record's offset depends on (B, n, path) of the last forward call,
+    // which that call left in the workspace header.
+    RowState rs;
+    WsHeader h;
+    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return LAPSUM_ECUDA;
+    if (h.last_B <= 0 || row >= h.last_B || h.last_path == LAPSUM_PATH_FULLSORT)
+        return LAPSUM_EINVAL;
+    const Layout L = make_layout(h.last_B, h.last_n, (int)h.last_path);
+    const char* base = static_cast<const char*>(ws) + L.rows + (size_t)row * 512;
+    e = cudaMemcpyAsync(&rs, base, sizeof(rs), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return LAPSUM_ECUDA;
+    std::memset(out, 0, sizeof(*out));
+    out->b = rs.b;
+    out->sum_f = rs.sum_f;
+    out->S_L = rs.S_L;
+    out->S_R = rs.S_R;
+    out->a_L = rs.a_L;
+    out->a_R = rs.a_R;
+    out->cnt_R = (int64_t)rs.cnt_R;
+    out->n_band = (int64_t)rs.n_band;
+    out->path = rs.path;
+    out->attempts = rs.attempts;
+    out->sample_m = rs.sample_m;
+    out->rank_l = rs.rank_l;
+    out->rank_h = rs.rank_h;
+    out->refine_levels = rs.refine_levels;
+    out->status = (int32_t)rs.status;
+    return LAPSUM_OK;
+}
+
+int lapsum_profile_enable(int on) {
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    p.recycle();
+    p.on = on != 0;
+    return LAPSUM_OK;
+}
+
+int lapsum_profile_read(lapsum_kernel_time* out, int max_entries, int* n_entries) {
+    if (n_entries == nullptr || (out == nullptr && max_entries > 0)) return LAPSUM_EINVAL;
+    Profiler& p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    std::vector<lapsum_kernel_time> acc;
+    for (auto& r : p.recs) {
+        if (cudaEventSynchronize(r.b) != cudaSuccess) return LAPSUM_ECUDA;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return LAPSUM_ECUDA;
+        size_t i = 0;
+        for (; i < acc.size(); ++i)
+            if (std::strncmp(acc[i].name, r.name, sizeof(acc[i].name)) == 0) break;
+        if (i == acc.size()) {
+            lapsum_kernel_time kt;
+            std::memset(&kt, 0, sizeof(kt));
+            std::strncpy(kt.name, r.name, sizeof(kt.name) - 1);
+            acc.push_back(kt);
+        }
+        acc[i].launches += 1;
+        acc[i].total_ms += (double)ms;
+    }
+    *n_entries = (int)acc.size();
+    for (int i = 0; i < (int)acc.size() && i < max_entries; ++i) out[i] = acc[i];
+    return LAPSUM_OK;
+}
+
+int lapsum_sample_get(void* ws, int64_t row, float* out, int64_t m, void* stream) {
+    if (ws == nullptr || out == nullptr || row < 0 || m < 1 || m > kSampleMax) return LAPSUM_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    WsHeader h;
+    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return LAPSUM_ECUDA;
+    if (h.last_path != LAPSUM_PATH_BRACKET || row >= h.last_B) return LAPSUM_EINVAL;
+    const Layout L = make_layout(h.last_B, h.last_n, LAPSUM_PATH_BRACKET);
+    const char* base = static_cast<const char*>(ws) + L.sample + (size_t)row * kSampleMax * 4;
+    e = cudaMemcpyAsync(out, base, (size_t)m * sizeof(float), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(e);
+}
+
+}  // extern "C"

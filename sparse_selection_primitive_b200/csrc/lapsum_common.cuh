@@ -1,0 +1,286 @@
+// Shared device-side building blocks of the Fast LapSum kernels (sm_100a).
+//
+// Method: "Fast LapSum: Exact Differentiable Top-k at Million Scale"
+// (gist.science explainer pages).  Section 2.1 defines p_i = sigma((r_i-b)/t)
+// with sigma the Laplace(0,1) CDF and sum_i p_i = k; section 2.2 solves for b
+// after a sort with one stable prefix/suffix scan, an index lookup and a
+// closed-form root in the balancing segment.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/lapsum.h"
+
+namespace lapsum {
+
+// ---------------------------------------------------------------------------
+// Device status bits (sticky, OR-ed into the workspace header).
+// ---------------------------------------------------------------------------
+enum : uint32_t {
+    kDevNonFinite = 1u << 0,
+    kDevBracketExhausted = 1u << 1,
+};
+
+constexpr int kMaxAttempts = 7;     // 1 + 3 widenings per side; the last rungs are open
+constexpr int kLadder = 4;          // rungs per side: ranks r, 4r, 16r, open
+constexpr int kBandSortMax = 4096;  // band solved on chip once it is this small
+constexpr int kRefineBins = 2048;   // histogram bins per narrowing level
+
+// Workspace header (first 256 bytes of the workspace).
+struct WsHeader {
+    uint32_t status;       // sticky device status bits
+    uint32_t last_path;    // path of the last forward call
+    int64_t last_B, last_n;
+    uint32_t fold_ticket;  // last-block counters (reset by the block that wins them)
+    uint32_t emit_ticket;
+    uint32_t bwd_ticket;
+    uint32_t pad0;
+    uint64_t reserved[27];
+};
+static_assert(sizeof(WsHeader) == 256, "header is one 256-byte slot");
+
+// Per-row record (radix and bracketing paths), 512 bytes.
+struct RowState {
+    double b;
+    double sum_f;
+    double S_L, S_R;      // tail sums of the current bracket
+    double R;             // backward ratio sum v f / sum f
+    double mu;            // backward shift: min |x|
+    float a_L, a_R;       // current bracket
+    unsigned long long cnt_R;   // scores >= a_R
+    unsigned long long n_band;  // scores in [a_L, a_R) (fold counter)
+    int32_t path;
+    int32_t attempts;
+    int32_t sample_m;
+    int32_t rank_l, rank_h;
+    int32_t refine_levels;
+    uint32_t status;
+    int32_t certified;
+    int32_t rung_L, rung_R;
+    int32_t force_miss;
+    int32_t max_attempts;
+    float ladder_L[kLadder];  // a_L rungs (descending ranks h, 4h, 16h, open)
+    float ladder_R[kLadder];  // a_R rungs (ranks l, l/4, l/16, open)
+    double scratch[40];       // kernel-to-kernel scalars
+};
+static_assert(sizeof(RowState) <= 512, "row record fits its slot");
+
+// ---------------------------------------------------------------------------
+// Order-preserving fp32 <-> u32 keys: flip every bit of a negative float,
+// only the sign bit of a non-negative one.  Unsigned key order is value order.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t to_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_key(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+__device__ __forceinline__ bool finite_f(float x) { return fabsf(x) <= 3.402823466e38f; }
+
+// ---------------------------------------------------------------------------
+// Threshold carried as two floats b = hi + lo, so that per element the scaled
+// margin x = (r - b)/t is formed in fp32 with the accuracy of an fp64 b: the
+// subtraction r - hi is exact near the threshold (Sterbenz), lo is tiny.
+// ---------------------------------------------------------------------------
+struct Thr {
+    float hi, lo, inv_t;
+};
+__device__ __forceinline__ Thr make_thr(double b, double t) {
+    Thr h;
+    h.hi = (float)b;
+    h.lo = (float)(b - (double)h.hi);
+    h.inv_t = (float)(1.0 / t);
+    return h;
+}
+__device__ __forceinline__ float scaled_margin(float r, const Thr& h) {
+    return __fmul_rn(__fsub_rn(__fsub_rn(r, h.hi), h.lo), h.inv_t);
+}
+
+// e = exp(-|x|); p = sigma(x) = x < 0 ? e/2 : 1 - e/2; f = e/2.  One exp.
+__device__ __forceinline__ float neg_abs_exp(float x) { return __expf(-fabsf(x)); }
+__device__ __forceinline__ float cdf_from(float x, float e) { return x < 0.f ? 0.5f * e : 1.f - 0.5f * e; }
+
+// ---------------------------------------------------------------------------
+// Affine maps x -> a x + c, the element of the stable prefix/suffix scans.
+// The prefix sum P_j = sum_{i<=j} e^{(s_i - s_j)/t} obeys P_j = 1 + g_j P_{j-1}
+// with the gap factor g_j = e^{(s_{j-1} - s_j)/t} in (0, 1]; the suffix sum Q_j
+// obeys Q_j = 1 + g_{j+1} Q_{j+1}.  Every factor is at most 1, so nothing
+// overflows, and composing maps is associative.
+// ---------------------------------------------------------------------------
+struct Aff {
+    double a, c;
+};
+__device__ __forceinline__ Aff aff_id() { return {1.0, 0.0}; }
+// Apply `first`, then `second`.
+__device__ __forceinline__ Aff aff_then(const Aff& first, const Aff& second) {
+    return {second.a * first.a, fma(second.a, first.c, second.c)};
+}
+
+__device__ __forceinline__ Aff shfl_up_aff(const Aff& v, int d) {
+    return {__shfl_up_sync(0xffffffffu, v.a, d), __shfl_up_sync(0xffffffffu, v.c, d)};
+}
+__device__ __forceinline__ Aff shfl_down_aff(const Aff& v, int d) {
+    return {__shfl_down_sync(0xffffffffu, v.a, d), __shfl_down_sync(0xffffffffu, v.c, d)};
+}
+
+// Inclusive warp scan in lane order (lane 0 applied first).
+__device__ __forceinline__ Aff warp_scan_fwd(Aff v, int lane) {
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        Aff o = shfl_up_aff(v, d);
+        if (lane >= d) v = aff_then(o, v);
+    }
+    return v;
+}
+// Inclusive warp scan in reverse lane order (lane 31 applied first).
+__device__ __forceinline__ Aff warp_scan_bwd(Aff v, int lane) {
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        Aff o = shfl_down_aff(v, d);
+        if (lane + d < 32) v = aff_then(o, v);
+    }
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// Closed-form root of the budget equation inside one segment of the sorted
+// order (section 2.2, "closed-form root").  Let the segment lie between a left
+// anchor sL (prefix weight Bh = sum over scores <= sL of e^{(s - sL)/t}) and a
+// right anchor sR (suffix weight Ah = sum over scores >= sR of e^{-(s - sR)/t}),
+// with m scores at or above sR and c = m - k.  With y = e^{(b - sR)/t} and
+// delta = e^{(sL - sR)/t} the equation F(b) = k reads
+//     Ah y^2 - 2 c y - Bh delta = 0,
+// whose positive root is taken in the log domain (delta underflows when t is
+// far below the gap):
+//     c = 0:  ln y = (ln Bh + ln delta - ln Ah)/2
+//     c > 0:  ln y = ln(c + S) - ln Ah
+//     c < 0:  ln y = ln Bh + ln delta - ln(S - c),      S = sqrt(c^2 + Ah Bh delta).
+// A missing anchor (no scores on that side, weight 0) leaves a single
+// exponential:  Bh = 0: b = sR + t ln(2c/Ah);  Ah = 0: b = sL + t ln(Bh/(-2c)).
+// The result is clamped into [sL, sR].
+// ---------------------------------------------------------------------------
+__device__ inline double segment_root(bool hasL, double sL, double Bh, bool hasR, double sR,
+                                      double Ah, double c, double t) {
+    hasL = hasL && Bh > 0.0;
+    hasR = hasR && Ah > 0.0;
+    double b;
+    if (!hasL && !hasR) return nan("");
+    if (!hasL) {
+        b = sR + t * log(2.0 * c / Ah);
+    } else if (!hasR) {
+        b = sL + t * log(Bh / (-2.0 * c));
+    } else {
+        double lnd = (sL - sR) / t;
+        double lnA = log(Ah), lnB = log(Bh);
+        double ln_y;
+        if (c == 0.0) {
+            ln_y = 0.5 * (lnB + lnd - lnA);
+        } else {
+            double lnc = log(fabs(c));
+            double lnrho = lnA + lnB + lnd - 2.0 * lnc;  // rho = Ah Bh delta / c^2
+            double lnS = lnrho > 0.0 ? 0.5 * (lnA + lnB + lnd) + 0.5 * log1p(exp(-lnrho))
+                                     : lnc + 0.5 * log1p(exp(lnrho));
+            double rc = exp(lnc - lnS);                   // |c| / S <= 1
+            if (c > 0.0) ln_y = lnS + log1p(rc) - lnA;     // ln(c + S) - ln Ah
+            else ln_y = lnB + lnd - (lnS + log1p(rc));    // ln Bh + ln delta - ln(S - c)
+        }
+        b = sR + t * ln_y;
+        if (b < sL) b = sL;
+        if (b > sR) b = sR;
+    }
+    return b;
+}
+
+// ---------------------------------------------------------------------------
+// Small block utilities.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    return v;
+}
+__device__ __forceinline__ float warp_min_f(float v) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, d));
+    return v;
+}
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, d));
+    return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    return v;
+}
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    return v;
+}
+
+// Block-wide sum of a double; every thread gets the result.  `red` needs
+// blockDim.x/32 doubles.  Fixed tree order, so the result is deterministic.
+__device__ inline double block_sum_d(double v, double* red) {
+    int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_sum_d(v);
+    __syncthreads();
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    double s = 0.0;
+    for (int i = 0; i < nw; ++i) s += red[i];
+    return s;
+}
+__device__ inline float block_min_f(float v, float* red) {
+    int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_min_f(v);
+    __syncthreads();
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    float s = red[0];
+    for (int i = 1; i < nw; ++i) s = fminf(s, red[i]);
+    return s;
+}
+__device__ inline float block_max_f(float v, float* red) {
+    int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_max_f(v);
+    __syncthreads();
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    float s = red[0];
+    for (int i = 1; i < nw; ++i) s = fmaxf(s, red[i]);
+    return s;
+}
+__device__ inline long long block_sum_ll(long long v, long long* red) {
+    int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    __syncthreads();
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    long long s = 0;
+    for (int i = 0; i < nw; ++i) s += red[i];
+    return s;
+}
+
+// ---------------------------------------------------------------------------
+// SplitMix64 (Steele, Lea and Flood 2014) as a counter-based generator:
+// output c of the stream seeded with `seed` is mix(seed + (c+1) * golden gamma).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t c) {
+    uint64_t z = seed + (c + 1ull) * 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ void set_status(WsHeader* hdr, uint32_t bits) {
+    atomicOr(&hdr->status, bits);
+}
+
+}  // namespace lapsum

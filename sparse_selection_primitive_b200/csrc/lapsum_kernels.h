@@ -1,0 +1,73 @@
+// Host-side launchers of the Fast LapSum kernels (internal to the library).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lapsum_common.cuh"
+
+namespace lapsum {
+
+// Optional per-kernel CUDA-event timing (lapsum_profile_enable).  A ProfScope
+// records an event pair around the launches in its lifetime when enabled.
+void prof_begin(const char* name, cudaStream_t st);
+void prof_end(cudaStream_t st);
+struct ProfScope {
+    cudaStream_t st;
+    ProfScope(const char* name, cudaStream_t s) : st(s) { prof_begin(name, s); }
+    ~ProfScope() { prof_end(st); }
+};
+
+// --- on-chip full sort (n <= 4096) -------------------------------------------
+int onchip_npad(int64_t n);
+cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,
+                                  int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
+                                  cudaStream_t st);
+cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
+                                   float* g, int64_t B, int n, double t, int vec, cudaStream_t st);
+
+// --- radix full sort (segmented LSD, keys only) ------------------------------
+constexpr int kRadixTile = 4096;
+struct RadixBuffers {
+    uint32_t* keys[2];     // ping-pong key buffers, B*n each (rows dense, stride n)
+    uint32_t* seg_hist;    // [B][4][256] digit counts of every segment
+    uint32_t* tile_hist;   // [B][256][tiles] per-tile digit counts, scanned into offsets
+    int32_t* plan;         // [B][8]: parity before pass d (d=0..4), trivial-pass mask
+};
+int64_t radix_tiles(int64_t n);
+cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_t n,
+                                   const RadixBuffers& buf, RowState* rows, WsHeader* hdr,
+                                   cudaStream_t st);
+// Solve every row from its sorted keys (one CTA per row); writes b and RowState.
+cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
+                                        double t, double* b, RowState* rows, WsHeader* hdr,
+                                        cudaStream_t st);
+
+// --- streaming kernels over long rows ----------------------------------------
+constexpr int kStreamTile = 4096;  // elements per CTA tile of the streaming kernels
+int64_t stream_tiles(int64_t n);
+// p = sigma((r - b)/t) and sum f per row; partials: [B][tiles] doubles.
+cudaError_t launch_emit(const float* r, int64_t ld, float* p, const double* b, double* sumf,
+                        int64_t B, int64_t n, double t, double* partials, uint32_t* tickets,
+                        int vec, WsHeader* hdr, int64_t B_total, int path_code, cudaStream_t st);
+// Backward for long rows: reduce (mu, sum w, sum w v) per row, then g.
+cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, const float* v,
+                                   float* g, int64_t B, int64_t n, double t, double* partials,
+                                   double* row_R, uint32_t* tickets, int vec, cudaStream_t st);
+
+// --- probabilistic bracketing --------------------------------------------------
+constexpr int kSampleMax = 32768;
+struct BracketBuffers {
+    float* sample;       // [B][m]
+    float* band[2];      // capacity n each
+    double* fold_part;   // fold partials, one record per CTA
+    uint32_t* ticket;    // last-block counter
+    int fold_grid;
+};
+int bracket_fold_grid();
+cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t, uint64_t seed,
+                               int64_t row, int m, int64_t rank_l[kLadder],
+                               int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,
+                               RowState* st_row, double* b_out, WsHeader* hdr, cudaStream_t st);
+
+}  // namespace lapsum

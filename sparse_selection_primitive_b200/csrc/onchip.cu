@@ -1,0 +1,415 @@
+// On-chip full-sort solver for rows of n <= 4096 scores, fused with p emission,
+// and the fused one-pass VJP for the same rows.
+//
+// "Fast LapSum: Exact Differentiable Top-k at Million Scale" (gist.science
+// explainer pages), section 2.2, full-sort solver: sort the row, run one
+// numerically stable prefix/suffix scan over the sorted scores to obtain the
+// threshold curve F(s_j), look up the segment where F crosses k, and take the
+// closed-form root there.  Section 2.1 gives p and the analytic VJP.
+//
+// Layout: a row of NPAD = E * RT keys (n padded with +inf keys) is held by RT
+// threads, E consecutive elements each, entirely in registers.  Bitonic stages
+// with a partner in the same thread swap registers, partners in the same warp
+// exchange through shuffles, and only partners in another warp go through
+// shared memory.  The scan carries fp64 affine maps (gap factor, 1) whose
+// composition is a warp shuffle scan plus one shared-memory step across warps.
+#include "lapsum_common.cuh"
+#include "lapsum_kernels.h"
+#include "bitonic.cuh"
+
+namespace lapsum {
+namespace {
+
+constexpr uint32_t kPadKey = 0xffffffffu;
+
+template <int E, int RT, int CTA>
+struct Shape {
+    static constexpr int NPAD = E * RT;
+    static constexpr int ROWS = CTA / RT;
+    static constexpr int WPR = RT / 32;  // warps per row
+    static constexpr int NW = CTA / 32;
+    static_assert(RT % 32 == 0 && CTA % RT == 0, "rows are whole warps");
+};
+
+// Load E consecutive elements of a row (idx = tid*E + e), padding past n.
+template <int E>
+__device__ __forceinline__ void load_row(const float* __restrict__ row, int n, int tid, bool vec,
+                                         bool row_ok, float (&x)[E], bool (&valid)[E]) {
+    const int base = tid * E;
+    if constexpr (E % 4 == 0) {
+        if (vec && row_ok && base + E <= n) {
+#pragma unroll
+            for (int q = 0; q < E / 4; ++q) {
+                float4 v4 = __ldg(reinterpret_cast<const float4*>(row + base) + q);
+                x[4 * q + 0] = v4.x;
+                x[4 * q + 1] = v4.y;
+                x[4 * q + 2] = v4.z;
+                x[4 * q + 3] = v4.w;
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) valid[e] = true;
+            return;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        valid[e] = row_ok && (base + e < n);
+        x[e] = valid[e] ? __ldg(row + base + e) : 0.f;
+    }
+}
+
+template <int E>
+__device__ __forceinline__ void store_row(float* __restrict__ row, int n, int tid, bool vec,
+                                          bool row_ok, const float (&y)[E]) {
+    if (!row_ok) return;
+    const int base = tid * E;
+    if constexpr (E % 4 == 0) {
+        if (vec && base + E <= n) {
+#pragma unroll
+            for (int q = 0; q < E / 4; ++q)
+                reinterpret_cast<float4*>(row + base)[q] =
+                    make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+            return;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (base + e < n) row[base + e] = y[e];
+}
+
+// Sum of an int over the threads of one row.
+template <int E, int RT, int CTA>
+__device__ __forceinline__ int row_sum_i(int v, int* red) {
+    using S = Shape<E, RT, CTA>;
+    v = warp_sum_i(v);
+    if constexpr (S::WPR == 1) {
+        return v;
+    } else {
+        const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        if (lane == 0) red[w] = v;
+        __syncthreads();
+        const int w0 = (w / S::WPR) * S::WPR;
+        int s = 0;
+#pragma unroll
+        for (int i = 0; i < S::WPR; ++i) s += red[w0 + i];
+        __syncthreads();
+        return s;
+    }
+}
+template <int E, int RT, int CTA>
+__device__ __forceinline__ double row_sum_d(double v, double* red) {
+    using S = Shape<E, RT, CTA>;
+    v = warp_sum_d(v);
+    if constexpr (S::WPR == 1) {
+        return v;
+    } else {
+        const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        if (lane == 0) red[w] = v;
+        __syncthreads();
+        const int w0 = (w / S::WPR) * S::WPR;
+        double s = 0.0;
+#pragma unroll
+        for (int i = 0; i < S::WPR; ++i) s += red[w0 + i];
+        __syncthreads();
+        return s;
+    }
+}
+template <int E, int RT, int CTA>
+__device__ __forceinline__ float row_min_f(float v, float* red) {
+    using S = Shape<E, RT, CTA>;
+    v = warp_min_f(v);
+    if constexpr (S::WPR == 1) {
+        return v;
+    } else {
+        const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        if (lane == 0) red[w] = v;
+        __syncthreads();
+        const int w0 = (w / S::WPR) * S::WPR;
+        float s = red[w0];
+#pragma unroll
+        for (int i = 1; i < S::WPR; ++i) s = fminf(s, red[w0 + i]);
+        __syncthreads();
+        return s;
+    }
+}
+
+template <int E, int RT, int CTA>
+__global__ void __launch_bounds__(CTA) onchip_forward_kernel(
+    const float* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
+    double* __restrict__ sumf_out, int64_t B, int n, double k, double t, WsHeader* hdr, int vec) {
+    using S = Shape<E, RT, CTA>;
+    __shared__ uint32_t xch[(RT > 32) ? CTA * E : 1];
+    __shared__ uint32_t last_key[CTA];
+    __shared__ float first_gap[CTA];
+    __shared__ Aff wf[S::NW], wb[S::NW];
+    __shared__ int ired[S::NW];
+    __shared__ double dred[S::NW];
+    __shared__ double anchor[S::ROWS][4];
+    __shared__ int row_flag[S::ROWS];
+    __shared__ double row_b[S::ROWS];
+
+    const int rloc = threadIdx.x / RT;
+    const int tid = threadIdx.x % RT;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * S::ROWS + rloc;
+    const bool row_ok = row < B;
+    const float* rrow = r + (row_ok ? row : 0) * ld;
+    const float inv_t = (float)(1.0 / t);
+
+    if (threadIdx.x < S::ROWS) row_flag[threadIdx.x] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        hdr->last_B = B;
+        hdr->last_n = n;
+        hdr->last_path = LAPSUM_PATH_FULLSORT;
+    }
+
+    float orig[E];
+    bool valid[E];
+    load_row<E>(rrow, n, tid, vec != 0, row_ok, orig, valid);
+    uint32_t key[E];
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        key[e] = valid[e] ? to_key(orig[e]) : kPadKey;
+        bad |= valid[e] && !finite_f(orig[e]);
+    }
+    __syncthreads();
+    if (bad) atomicOr(&row_flag[rloc], 1);
+
+    bitonic_sort_row<E, RT, CTA>(key, tid, xch);
+
+    // Sorted values and gap factors g_j = exp((s_{j-1} - s_j)/t), 0 at j = 0 and past n.
+    float s[E], g[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[e] = from_key(key[e]);
+    last_key[threadIdx.x] = key[E - 1];
+    __syncthreads();
+    const float s_prev = (tid > 0) ? from_key(last_key[threadIdx.x - 1]) : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = tid * E + e;
+        const float sp = (e == 0) ? s_prev : s[e - 1];
+        g[e] = (j >= 1 && j < n) ? __expf((sp - s[e]) * inv_t) : 0.f;
+    }
+    first_gap[threadIdx.x] = g[0];
+    __syncthreads();
+    const float g_next = (tid + 1 < RT) ? first_gap[threadIdx.x + 1] : 0.f;
+
+    // Thread aggregates of the forward (prefix) and backward (suffix) maps.
+    Aff af = aff_id(), ab = aff_id();
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = tid * E + e;
+        const Aff m = (j < n) ? Aff{(double)g[e], 1.0} : aff_id();
+        af = aff_then(af, m);
+    }
+#pragma unroll
+    for (int e = E - 1; e >= 0; --e) {
+        const int j = tid * E + e;
+        const float gn = (e + 1 < E) ? g[e + 1] : g_next;
+        const Aff m = (j < n) ? Aff{(double)gn, 1.0} : Aff{0.0, 0.0};
+        ab = aff_then(ab, m);
+    }
+    // Exclusive prefix (maps of earlier threads) and suffix (later threads).
+    Aff inc_f = warp_scan_fwd(af, lane);
+    Aff inc_b = warp_scan_bwd(ab, lane);
+    Aff ex_f = shfl_up_aff(inc_f, 1);
+    Aff ex_b = shfl_down_aff(inc_b, 1);
+    if (lane == 0) ex_f = aff_id();
+    if (lane == 31) ex_b = aff_id();
+    if constexpr (S::WPR > 1) {
+        if (lane == 31) wf[warp] = inc_f;
+        if (lane == 0) wb[warp] = inc_b;
+        __syncthreads();
+        const int w0 = (warp / S::WPR) * S::WPR;
+        Aff pre = aff_id();
+        for (int w = w0; w < warp; ++w) pre = aff_then(pre, wf[w]);
+        ex_f = aff_then(pre, ex_f);
+        Aff suf = aff_id();
+        for (int w = w0 + S::WPR - 1; w > warp; --w) suf = aff_then(suf, wb[w]);
+        ex_b = aff_then(suf, ex_b);
+    }
+
+    // Threshold curve G_j = F(s_j) = (n - j) - Q_j/2 + (P_j - 1)/2 and its count.
+    double P[E], Q[E];
+    double x = ex_f.c;  // P just before this thread's first element
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        x = fma((double)g[e], x, 1.0);
+        P[e] = x;
+    }
+    double y = ex_b.c;  // Q just after this thread's last element
+    int cnt = 0;
+#pragma unroll
+    for (int e = E - 1; e >= 0; --e) {
+        const int j = tid * E + e;
+        const float gn = (e + 1 < E) ? g[e + 1] : g_next;
+        y = (j < n) ? fma((double)gn, y, 1.0) : 0.0;
+        Q[e] = y;
+        const double G = (double)(n - j) - 0.5 * Q[e] + 0.5 * (P[e] - 1.0);
+        cnt += (j < n && G >= k) ? 1 : 0;
+    }
+    const int jstar = row_sum_i<E, RT, CTA>(cnt, ired);
+
+    // Anchors of the balancing segment: left = sorted position j*-1, right = j*.
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = tid * E + e;
+        if (j == jstar - 1) {
+            anchor[rloc][0] = s[e];
+            anchor[rloc][1] = P[e];
+        }
+        if (j == jstar && j < n) {
+            anchor[rloc][2] = s[e];
+            anchor[rloc][3] = Q[e];
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double bb;
+        if (row_flag[rloc] || !row_ok) {
+            bb = nan("");
+            if (row_ok) set_status(hdr, kDevNonFinite);
+        } else {
+            const bool hasL = jstar >= 1, hasR = jstar < n;
+            bb = segment_root(hasL, anchor[rloc][0], hasL ? anchor[rloc][1] : 0.0, hasR,
+                              anchor[rloc][2], hasR ? anchor[rloc][3] : 0.0,
+                              (double)(n - jstar) - k, t);
+        }
+        row_b[rloc] = bb;
+        if (row_ok) b_out[row] = bb;
+    }
+    __syncthreads();
+
+    // Emit p_i = sigma((r_i - b)/t) in the original order, and sum f.
+    const Thr th = make_thr(row_b[rloc], t);
+    float pv[E];
+    double sf = 0.0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const float xs = scaled_margin(orig[e], th);
+        const float ex = neg_abs_exp(xs);
+        pv[e] = cdf_from(xs, ex);
+        if (valid[e]) sf += 0.5 * (double)ex;
+    }
+    store_row<E>(p + (row_ok ? row : 0) * ld, n, tid, vec != 0, row_ok, pv);
+    if (sumf_out != nullptr) {
+        const double tot = row_sum_d<E, RT, CTA>(sf, dred);
+        if (tid == 0 && row_ok) sumf_out[row] = tot;
+    }
+}
+
+template <int E, int RT, int CTA>
+__global__ void __launch_bounds__(CTA) onchip_backward_kernel(
+    const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
+    const float* __restrict__ v, float* __restrict__ g, int64_t B, int n, double t, int vec) {
+    using S = Shape<E, RT, CTA>;
+    __shared__ float fred[S::NW];
+    __shared__ double dred[S::NW];
+    const int rloc = threadIdx.x / RT;
+    const int tid = threadIdx.x % RT;
+    const int64_t row = (int64_t)blockIdx.x * S::ROWS + rloc;
+    const bool row_ok = row < B;
+    const int64_t off = (row_ok ? row : 0) * ld;
+
+    float rv[E], vv[E];
+    bool valid[E];
+    load_row<E>(r + off, n, tid, vec != 0, row_ok, rv, valid);
+    load_row<E>(v + off, n, tid, vec != 0, row_ok, vv, valid);
+    const Thr th = make_thr(row_ok ? b[row] : 0.0, t);
+    float ax[E];
+    float mloc = INFINITY;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        ax[e] = valid[e] ? fabsf(scaled_margin(rv[e], th)) : INFINITY;
+        mloc = fminf(mloc, ax[e]);
+    }
+    const float mu = row_min_f<E, RT, CTA>(mloc, fred);
+    // R = sum v f / sum f with weights w = exp(-(|x| - mu)) <= 1.
+    double sw = 0.0, swv = 0.0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        if (valid[e]) {
+            const double w = (double)__expf(mu - ax[e]);
+            sw += w;
+            swv += w * (double)vv[e];
+        }
+    }
+    sw = row_sum_d<E, RT, CTA>(sw, dred);
+    swv = row_sum_d<E, RT, CTA>(swv, dred);
+    const double R = swv / sw;
+    float gv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const float f = 0.5f * __expf(-ax[e]);
+        gv[e] = f * th.inv_t * (float)((double)vv[e] - R);
+    }
+    store_row<E>(g + off, n, tid, vec != 0, row_ok, gv);
+}
+
+template <int E, int RT, int CTA>
+cudaError_t launch_fwd(const float* r, int64_t ld, float* p, double* b, double* sumf, int64_t B,
+                       int n, double k, double t, WsHeader* hdr, int vec, cudaStream_t st) {
+    using S = Shape<E, RT, CTA>;
+    const int64_t grid = (B + S::ROWS - 1) / S::ROWS;
+    {
+        ProfScope ps_("onchip_fwd", st);
+        onchip_forward_kernel<E, RT, CTA>
+        <<<(unsigned)grid, CTA, 0, st>>>(r, ld, p, b, sumf, B, n, k, t, hdr, vec);
+    }
+    return cudaGetLastError();
+}
+
+template <int E, int RT, int CTA>
+cudaError_t launch_bwd(const float* r, int64_t ld, const double* b, const float* v, float* g,
+                       int64_t B, int n, double t, int vec, cudaStream_t st) {
+    using S = Shape<E, RT, CTA>;
+    const int64_t grid = (B + S::ROWS - 1) / S::ROWS;
+    {
+        ProfScope ps_("onchip_bwd", st);
+        onchip_backward_kernel<E, RT, CTA><<<(unsigned)grid, CTA, 0, st>>>(r, ld, b, v, g, B, n, t, vec);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int onchip_npad(int64_t n) {
+    int np = 32;
+    while (np < n) np <<= 1;
+    return np;
+}
+
+cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,
+                                  int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
+                                  cudaStream_t st) {
+    switch (onchip_npad(n)) {
+        case 32: return launch_fwd<1, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 64: return launch_fwd<2, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 128: return launch_fwd<4, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 256: return launch_fwd<8, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 512: return launch_fwd<8, 64, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 1024: return launch_fwd<8, 128, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 2048: return launch_fwd<8, 256, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 4096: return launch_fwd<8, 512, 512>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
+                                   float* g, int64_t B, int n, double t, int vec, cudaStream_t st) {
+    switch (onchip_npad(n)) {
+        case 32: return launch_bwd<1, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
+        case 64: return launch_bwd<2, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
+        case 128: return launch_bwd<4, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
+        case 256: return launch_bwd<8, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
+        case 512: return launch_bwd<8, 64, 256>(r, ld, b, v, g, B, n, t, vec, st);
+        case 1024: return launch_bwd<8, 128, 256>(r, ld, b, v, g, B, n, t, vec, st);
+        case 2048: return launch_bwd<8, 256, 256>(r, ld, b, v, g, B, n, t, vec, st);
+        case 4096: return launch_bwd<8, 512, 512>(r, ld, b, v, g, B, n, t, vec, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace lapsum

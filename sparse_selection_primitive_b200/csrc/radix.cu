@@ -1,0 +1,345 @@
+// Segmented LSD radix sort of fp32 scores (as order-preserving u32 keys, no
+// payload) and the per-row solve over the sorted keys.
+//
+// "Fast LapSum: Exact Differentiable Top-k at Million Scale" (gist.science
+// explainer pages), section 2.2: the full-sort solver sorts the scores, after
+// which all remaining work is linear.  p and g are elementwise in (r_i, b), so
+// only the keys are sorted; no index permutation is carried.
+//
+// Sort structure, per 8-bit digit pass (4 passes for 32-bit keys):
+//   upsweep   one CTA per 4096-key tile: digit histogram of the tile;
+//   scan      exclusive scan of (digit, tile) counts per row -> scatter bases;
+//   downsweep one CTA per tile: stable rank of every key inside the tile
+//             (warp match + per-warp digit counters), a local reorder in
+//             shared memory, then coalesced runs written to the bases.
+// A prep pass converts r into keys and histograms all four digits of every
+// row at once (those histograms do not depend on the key order), so a digit
+// that is the same for every key of a row is known up front and its pass is
+// skipped for that row.  Each row tracks which ping-pong buffer holds it.
+#include "lapsum_common.cuh"
+#include "lapsum_kernels.h"
+#include "solve_sorted.cuh"
+
+namespace lapsum {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kPerThread = kRadixTile / kThreads;  // 16
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// r (row stride ld) -> keys (row stride n); all-digit histograms per row.
+__global__ void __launch_bounds__(kThreads) radix_prep_kernel(const float* __restrict__ r,
+                                                              int64_t ld, int64_t n,
+                                                              uint32_t* __restrict__ keys,
+                                                              uint32_t* __restrict__ seg_hist,
+                                                              RowState* rows, WsHeader* hdr) {
+    __shared__ uint32_t h[4][256];
+    const int64_t row = blockIdx.y;
+    const int64_t base = (int64_t)blockIdx.x * kRadixTile;
+    for (int i = threadIdx.x; i < 4 * 256; i += kThreads) (&h[0][0])[i] = 0;
+    __syncthreads();
+    bool bad = false;
+    const float* rr = r + row * ld;
+    uint32_t* kk = keys + row * n;
+    for (int i = threadIdx.x; i < kRadixTile; i += kThreads) {
+        const int64_t idx = base + i;
+        if (idx < n) {
+            const float x = __ldg(rr + idx);
+            bad |= !finite_f(x);
+            const uint32_t key = to_key(x);
+            kk[idx] = key;
+#pragma unroll
+            for (int d = 0; d < 4; ++d) atomicAdd(&h[d][(key >> (8 * d)) & 255u], 1u);
+        }
+    }
+    if (bad) {
+        atomicOr(&rows[row].status, kDevNonFinite);
+        set_status(hdr, kDevNonFinite);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 4 * 256; i += kThreads) {
+        const uint32_t c = (&h[0][0])[i];
+        if (c) atomicAdd(&seg_hist[row * 1024 + i], c);
+    }
+}
+
+// Per row: which digits are trivial, and which buffer holds the data before
+// each pass (plan[row][d], d = 0..4), plus the trivial mask in plan[row][5].
+__global__ void radix_plan_kernel(const uint32_t* __restrict__ seg_hist, int64_t B, int64_t n,
+                                  int32_t* __restrict__ plan) {
+    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= B) return;
+    int par = 0, mask = 0;
+    for (int d = 0; d < 4; ++d) {
+        plan[row * 8 + d] = par;
+        uint32_t mx = 0;
+        for (int v = 0; v < 256; ++v) mx = max(mx, seg_hist[row * 1024 + d * 256 + v]);
+        const bool trivial = (int64_t)mx == n;
+        if (trivial) mask |= 1 << d;
+        else par ^= 1;
+    }
+    plan[row * 8 + 4] = par;
+    plan[row * 8 + 5] = mask;
+}
+
+__global__ void __launch_bounds__(kThreads) radix_upsweep_kernel(
+    const uint32_t* __restrict__ k0, const uint32_t* __restrict__ k1, int64_t n, int64_t tiles,
+    int d, const int32_t* __restrict__ plan, uint32_t* __restrict__ tile_hist) {
+    __shared__ uint32_t h[256];
+    const int64_t row = blockIdx.y;
+    if (plan[row * 8 + 5] & (1 << d)) return;
+    const uint32_t* src = (plan[row * 8 + d] ? k1 : k0) + row * n;
+    const int64_t base = (int64_t)blockIdx.x * kRadixTile;
+    h[threadIdx.x] = 0;
+    __syncthreads();
+    const int shift = 8 * d;
+    for (int i = threadIdx.x; i < kRadixTile; i += kThreads) {
+        const int64_t idx = base + i;
+        if (idx < n) atomicAdd(&h[(src[idx] >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    tile_hist[(row * 256 + threadIdx.x) * tiles + blockIdx.x] = h[threadIdx.x];
+}
+
+// Exclusive scan over (digit, tile) of one row; one thread per digit walks the
+// tiles.  Rows with many tiles use radix_scan_wide_kernel instead.
+__global__ void __launch_bounds__(256) radix_scan_kernel(const uint32_t* __restrict__ seg_hist,
+                                                         int64_t tiles, int d,
+                                                         const int32_t* __restrict__ plan,
+                                                         uint32_t* __restrict__ tile_hist) {
+    __shared__ uint32_t base[256];
+    const int64_t row = blockIdx.x;
+    if (plan[row * 8 + 5] & (1 << d)) return;
+    const int v = threadIdx.x;
+    // digit bases from the row histogram (exclusive scan over 256 digits)
+    uint32_t c = seg_hist[row * 1024 + d * 256 + v];
+    base[v] = c;
+    __syncthreads();
+    for (int off = 1; off < 256; off <<= 1) {
+        uint32_t add = v >= off ? base[v - off] : 0u;
+        __syncthreads();
+        base[v] += add;
+        __syncthreads();
+    }
+    uint32_t run = base[v] - c;
+    uint32_t* th = tile_hist + (row * 256 + v) * tiles;
+    for (int64_t tI = 0; tI < tiles; ++tI) {
+        const uint32_t x = th[tI];
+        th[tI] = run;
+        run += x;
+    }
+}
+
+// Same scan for rows with many tiles: one CTA per (row, digit).
+__global__ void __launch_bounds__(256) radix_scan_wide_kernel(const uint32_t* __restrict__ seg_hist,
+                                                              int64_t tiles, int d,
+                                                              const int32_t* __restrict__ plan,
+                                                              uint32_t* __restrict__ tile_hist) {
+    __shared__ uint32_t part[256];
+    const int64_t row = blockIdx.y;
+    const int v = blockIdx.x;
+    if (plan[row * 8 + 5] & (1 << d)) return;
+    uint32_t dbase = 0;
+    for (int u = threadIdx.x; u < v; u += 256) dbase += seg_hist[row * 1024 + d * 256 + u];
+    part[threadIdx.x] = dbase;
+    __syncthreads();
+    for (int off = 128; off > 0; off >>= 1) {
+        if (threadIdx.x < off) part[threadIdx.x] += part[threadIdx.x + off];
+        __syncthreads();
+    }
+    uint32_t carry = part[0];
+    __syncthreads();
+    uint32_t* th = tile_hist + (row * 256 + v) * tiles;
+    for (int64_t c0 = 0; c0 < tiles; c0 += 256) {
+        const int64_t i = c0 + threadIdx.x;
+        const uint32_t x = i < tiles ? th[i] : 0u;
+        part[threadIdx.x] = x;
+        __syncthreads();
+        for (int off = 1; off < 256; off <<= 1) {
+            uint32_t add = threadIdx.x >= off ? part[threadIdx.x - off] : 0u;
+            __syncthreads();
+            part[threadIdx.x] += add;
+            __syncthreads();
+        }
+        if (i < tiles) th[i] = carry + part[threadIdx.x] - x;
+        carry += part[255];
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) radix_downsweep_kernel(
+    uint32_t* __restrict__ k0, uint32_t* __restrict__ k1, int64_t n, int64_t tiles, int d,
+    const int32_t* __restrict__ plan, const uint32_t* __restrict__ tile_hist) {
+    __shared__ uint32_t wcnt[kWarps][256];
+    __shared__ uint32_t tstart[256];
+    __shared__ uint32_t gbase[256];
+    __shared__ uint32_t sorted[kRadixTile];
+    const int64_t row = blockIdx.y;
+    if (plan[row * 8 + 5] & (1 << d)) return;
+    const int par = plan[row * 8 + d];
+    const uint32_t* src = (par ? k1 : k0) + row * n;
+    uint32_t* dst = (par ? k0 : k1) + row * n;
+    const int64_t base = (int64_t)blockIdx.x * kRadixTile;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int shift = 8 * d;
+
+    for (int i = threadIdx.x; i < kWarps * 256; i += kThreads) (&wcnt[0][0])[i] = 0;
+    gbase[threadIdx.x] = tile_hist[(row * 256 + threadIdx.x) * tiles + blockIdx.x];
+    __syncthreads();
+
+    // Striped ownership keeps the rank stable: warp w owns keys
+    // [w*512, (w+1)*512) of the tile, visited 32 at a time in index order.
+    uint32_t key[kPerThread], lrank[kPerThread];
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
+        const bool ok = idx < n;
+        key[e] = ok ? src[idx] : 0u;
+        const uint32_t dig = (key[e] >> shift) & 255u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, ok ? dig : 256u + lane);
+        const int leader = __ffs(peers) - 1;
+        uint32_t bse = 0;
+        if (ok && lane == leader) {
+            bse = wcnt[warp][dig];
+            wcnt[warp][dig] = bse + __popc(peers);
+        }
+        bse = __shfl_sync(0xffffffffu, bse, leader);
+        lrank[e] = bse + __popc(peers & lt);
+        __syncwarp();
+    }
+    __syncthreads();
+    // per digit: exclusive over warps, and the tile count of the digit
+    {
+        const int v = threadIdx.x;
+        uint32_t run = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const uint32_t c = wcnt[w][v];
+            wcnt[w][v] = run;
+            run += c;
+        }
+        tstart[v] = run;
+    }
+    __syncthreads();
+    // exclusive scan of tile digit counts -> local start of each digit
+    {
+        const int v = threadIdx.x;
+        const uint32_t c = tstart[v];
+        for (int off = 1; off < 256; off <<= 1) {
+            uint32_t add = v >= off ? tstart[v - off] : 0u;
+            __syncthreads();
+            tstart[v] += add;
+            __syncthreads();
+        }
+        tstart[v] -= c;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
+        if (idx < n) {
+            const uint32_t dig = (key[e] >> shift) & 255u;
+            sorted[tstart[dig] + wcnt[warp][dig] + lrank[e]] = key[e];
+        }
+    }
+    __syncthreads();
+    const int valid = (int)min((int64_t)kRadixTile, n - base);
+    for (int i = threadIdx.x; i < valid; i += kThreads) {
+        const uint32_t kv = sorted[i];
+        const uint32_t dig = (kv >> shift) & 255u;
+        dst[gbase[dig] + (uint32_t)i - tstart[dig]] = kv;
+    }
+}
+
+struct KeyGet {
+    const uint32_t* k;
+    __device__ __forceinline__ float operator()(long long j) const { return from_key(k[j]); }
+};
+
+__global__ void __launch_bounds__(1024) rowsolve_keys_kernel(const uint32_t* __restrict__ k0,
+                                                              const uint32_t* __restrict__ k1,
+                                                              int64_t n, double k, double t,
+                                                              const int32_t* __restrict__ plan,
+                                                              double* __restrict__ b_out,
+                                                              RowState* rows) {
+    __shared__ SolveScratch sm;
+    __shared__ SolveResult res;
+    const int64_t row = blockIdx.x;
+    const uint32_t* keys = (plan[row * 8 + 4] ? k1 : k0) + row * n;
+    Tails tl{false, 0.f, 0.0, false, 0.f, 0.0, 0.0};
+    solve_sorted_block(KeyGet{keys}, (long long)n, tl, k, t, &sm, &res);
+    if (threadIdx.x == 0) {
+        const double b = (rows[row].status & kDevNonFinite) ? nan("") : res.b;
+        rows[row].b = b;
+        rows[row].path = LAPSUM_PATH_RADIX;
+        rows[row].attempts = 1;
+        b_out[row] = b;
+    }
+}
+
+}  // namespace
+
+int64_t radix_tiles(int64_t n) { return (n + kRadixTile - 1) / kRadixTile; }
+
+cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_t n,
+                                   const RadixBuffers& buf, RowState* rows, WsHeader* hdr,
+                                   cudaStream_t st) {
+    const int64_t tiles = radix_tiles(n);
+    cudaError_t e = cudaMemsetAsync(buf.seg_hist, 0, (size_t)B * 1024 * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)tiles, (unsigned)B);
+    {
+        ProfScope ps_("radix_prep", st);
+        radix_prep_kernel<<<grid, kThreads, 0, st>>>(r, ld, n, buf.keys[0], buf.seg_hist, rows, hdr);
+    }
+    {
+        ProfScope ps_("radix_plan", st);
+        radix_plan_kernel<<<(unsigned)((B + 127) / 128), 128, 0, st>>>(buf.seg_hist, B, n, buf.plan);
+    }
+    for (int d = 0; d < 4; ++d) {
+        {
+            ProfScope ps_("radix_upsweep", st);
+            radix_upsweep_kernel<<<grid, kThreads, 0, st>>>(buf.keys[0], buf.keys[1], n, tiles, d,
+                                                        buf.plan, buf.tile_hist);
+        }
+        if (tiles <= 64)
+            {
+                ProfScope ps_("radix_scan", st);
+                radix_scan_kernel<<<(unsigned)B, 256, 0, st>>>(buf.seg_hist, tiles, d, buf.plan,
+                                                           buf.tile_hist);
+            }
+        else
+            {
+                ProfScope ps_("radix_scan", st);
+                radix_scan_wide_kernel<<<dim3(256, (unsigned)B), 256, 0, st>>>(
+                buf.seg_hist, tiles, d, buf.plan, buf.tile_hist);
+            }
+        {
+            ProfScope ps_("radix_downsweep", st);
+            radix_downsweep_kernel<<<grid, kThreads, 0, st>>>(buf.keys[0], buf.keys[1], n, tiles, d,
+                                                          buf.plan, buf.tile_hist);
+        }
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
+                                        double t, double* b, RowState* rows, WsHeader* hdr,
+                                        cudaStream_t st) {
+    (void)hdr;
+    {
+        ProfScope ps_("rowsolve", st);
+        rowsolve_keys_kernel<<<(unsigned)B, 1024, 0, st>>>(buf.keys[0], buf.keys[1], n, k, t,
+                                                       buf.plan, b, rows);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace lapsum

@@ -1,0 +1,229 @@
+// Block-level solve of the budget equation over a sorted array with optional
+// folded tails: the stable prefix/suffix scan, the index lookup of the
+// balancing segment and the closed-form root ("Fast LapSum: Exact
+// Differentiable Top-k at Million Scale", gist.science explainer pages,
+// section 2.2, full-sort solver; the tails implement step 3 of the bracketing
+// pipeline, the exact solve on the middle band).
+//
+// Sorted scores s_0 <= ... <= s_{nb-1} may sit between two virtual anchors:
+// a left anchor aL carrying SL = sum_{r < aL} e^{(r - aL)/t} (the folded left
+// tail) and a right anchor aR carrying SR = sum_{r >= aR} e^{-(r - aR)/t} and
+// cntR scores (the folded right tail).  With gap factors gap(j) between
+// neighbours (the anchors count as positions -1 and nb), the prefix and
+// suffix weights obey P_j = 1 + gap(j) P_{j-1} (P_{-1} = SL) and
+// Q_j = 1 + gap(j+1) Q_{j+1} (Q_nb = SR), and the threshold curve is
+//     F(s_j) = cntR + (nb - j) - Q_j / 2 + (P_j - 1) / 2.
+// The balancing segment is found with counts of F(s_j) >= k taken over thread
+// chunks, then recursively over 32 warp lanes, so no per-element storage is
+// needed at any n.
+#pragma once
+
+#include "lapsum_common.cuh"
+
+namespace lapsum {
+
+struct Tails {
+    bool hasL;
+    float aL;
+    double SL;
+    bool hasR;
+    float aR;
+    double SR;
+    double cntR;
+};
+
+struct SolveResult {
+    double b;
+    double F_aL, F_aR;  // budget sum at the bracket ends (+inf / -inf for open ends)
+    long long jstar;    // number of sorted band scores with F(s_j) >= k
+};
+
+struct SolveScratch {
+    Aff wf[32], wb[32];
+    double d[8];
+    long long ll[4];
+};
+
+template <class Get>
+struct GapFn {
+    Get get;
+    long long nb;
+    Tails tl;
+    float inv_t;
+    // factor between positions j-1 and j (anchors at -1 and nb)
+    __device__ __forceinline__ float operator()(long long j) const {
+        if (j <= 0) return (j == 0 && tl.hasL && nb > 0) ? __expf((tl.aL - get(0)) * inv_t) : 0.f;
+        if (j >= nb) return (j == nb && tl.hasR) ? __expf((get(nb - 1) - tl.aR) * inv_t) : 0.f;
+        return __expf((get(j - 1) - get(j)) * inv_t);
+    }
+};
+
+// One warp narrows [lo, hi) -- whose first element satisfies F >= k -- to the
+// last element with F >= k.  P_before = P_{lo-1}, Q_after = Q_hi.  Lane 0
+// returns j* and the anchor weights through the out-parameters.
+template <class Get>
+__device__ void warp_find_crossing(const GapFn<Get>& gap, long long lo, long long hi,
+                                   double P_before, double Q_after, double k, long long* jstar,
+                                   double* P_left, double* Q_right) {
+    const int lane = threadIdx.x & 31;
+    const long long nb = gap.nb;
+    const double cntR = gap.tl.cntR;
+    while (hi - lo > 32) {
+        const long long sc = (hi - lo + 31) / 32;
+        const long long l0 = min(hi, lo + lane * sc), l1 = min(hi, l0 + sc);
+        Aff af = aff_id(), ab = aff_id();
+        float g_first = 0.f;
+        for (long long j = l0; j < l1; ++j) {
+            const float gj = gap(j);
+            if (j == l0) g_first = gj;
+            af = aff_then(af, Aff{(double)gj, 1.0});
+            if (j > l0) ab = aff_then(Aff{(double)gj, 1.0}, ab);
+        }
+        if (l1 > l0) ab = aff_then(Aff{(double)gap(l1), 1.0}, ab);
+        Aff ef = shfl_up_aff(warp_scan_fwd(af, lane), 1);
+        Aff eb = shfl_down_aff(warp_scan_bwd(ab, lane), 1);
+        if (lane == 0) ef = aff_id();
+        if (lane == 31) eb = aff_id();
+        const double pb = fma(ef.a, P_before, ef.c);   // P_{l0-1}
+        const double qa = fma(eb.a, Q_after, eb.c);    // Q_{l1}
+        const double P0 = fma((double)g_first, pb, 1.0);
+        const double Q0 = fma(ab.a, qa, ab.c);
+        const double G0 = cntR + (double)(nb - l0) - 0.5 * Q0 + 0.5 * (P0 - 1.0);
+        const unsigned ball = __ballot_sync(0xffffffffu, l0 < l1 && G0 >= k);
+        const int L = max(0, __popc(ball) - 1);
+        lo = __shfl_sync(0xffffffffu, l0, L);
+        hi = __shfl_sync(0xffffffffu, l1, L);
+        P_before = __shfl_sync(0xffffffffu, pb, L);
+        Q_after = __shfl_sync(0xffffffffu, qa, L);
+    }
+    // At most 32 elements: one per lane.
+    const long long j = lo + lane;
+    const bool valid = j < hi;
+    const float gj = valid ? gap(j) : 1.f;
+    const float gn = valid ? gap(j + 1) : 1.f;
+    const Aff mf = valid ? Aff{(double)gj, 1.0} : aff_id();
+    const Aff mb = valid ? Aff{(double)gn, 1.0} : aff_id();
+    const Aff inf_ = warp_scan_fwd(mf, lane);
+    const Aff inb = warp_scan_bwd(mb, lane);
+    const double Pj = fma(inf_.a, P_before, inf_.c);
+    const double Qj = fma(inb.a, Q_after, inb.c);
+    const double Gj = cntR + (double)(nb - j) - 0.5 * Qj + 0.5 * (Pj - 1.0);
+    const unsigned ball = __ballot_sync(0xffffffffu, valid && Gj >= k);
+    const int c = __popc(ball);  // >= 1 by the invariant on lo
+    const long long js = lo + c;
+    const double Pl = __shfl_sync(0xffffffffu, Pj, max(0, c - 1));
+    const double Qr_in = __shfl_sync(0xffffffffu, Qj, min(31, c));
+    if (lane == 0) {
+        *jstar = js;
+        *P_left = Pl;
+        *Q_right = (js < hi) ? Qr_in : Q_after;  // Q_hi when the right anchor opens the next range
+    }
+}
+
+// Whole-block solve.  Every thread of the block must call it; the result is
+// valid in `out` for every thread after return.
+template <class Get>
+__device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, double k, double t,
+                                   SolveScratch* sm, SolveResult* out) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    GapFn<Get> gap{get, nb, tl, (float)(1.0 / t)};
+    const double P_start = tl.hasL ? tl.SL : 0.0;
+    const double Q_end = tl.hasR ? tl.SR : 0.0;
+
+    if (nb == 0) {
+        if (tid == 0) {
+            out->jstar = 0;
+            out->b = segment_root(tl.hasL, tl.aL, tl.SL, tl.hasR, tl.aR, tl.SR, tl.cntR - k, t);
+            const double lnw = (tl.hasL && tl.hasR) ? ((double)tl.aL - (double)tl.aR) / t : -INFINITY;
+            out->F_aL = tl.hasL ? tl.cntR - 0.5 * tl.SR * exp(lnw) + 0.5 * tl.SL : INFINITY;
+            out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * tl.SL * exp(lnw) : -INFINITY;
+        }
+        __syncthreads();
+        return;
+    }
+
+    const long long chunk = (nb + blockDim.x - 1) / blockDim.x;
+    const long long lo = min(nb, (long long)tid * chunk), hi = min(nb, lo + chunk);
+    const bool valid = lo < hi;
+    Aff af = aff_id(), ab = aff_id();
+    float g_first = 0.f;
+    for (long long j = lo; j < hi; ++j) {
+        const float gj = gap(j);
+        if (j == lo) g_first = gj;
+        af = aff_then(af, Aff{(double)gj, 1.0});
+        if (j > lo) ab = aff_then(Aff{(double)gj, 1.0}, ab);
+    }
+    if (valid) ab = aff_then(Aff{(double)gap(hi), 1.0}, ab);
+
+    Aff ef = shfl_up_aff(warp_scan_fwd(af, lane), 1);
+    Aff inc_b = warp_scan_bwd(ab, lane);
+    Aff inc_f_last = warp_scan_fwd(af, lane);
+    Aff eb = shfl_down_aff(inc_b, 1);
+    if (lane == 0) ef = aff_id();
+    if (lane == 31) eb = aff_id();
+    if (lane == 31) sm->wf[warp] = inc_f_last;
+    if (lane == 0) sm->wb[warp] = inc_b;
+    __syncthreads();
+    {
+        Aff pre = aff_id();
+        for (int w = 0; w < warp; ++w) pre = aff_then(pre, sm->wf[w]);
+        ef = aff_then(pre, ef);
+        Aff suf = aff_id();
+        for (int w = nwarps - 1; w > warp; --w) suf = aff_then(suf, sm->wb[w]);
+        eb = aff_then(suf, eb);
+    }
+    const double P_before = fma(ef.a, P_start, ef.c);  // P_{lo-1}
+    const double Q_after = fma(eb.a, Q_end, eb.c);     // Q_hi
+    const double P_lo = fma((double)g_first, P_before, 1.0);
+    const double Q_lo = fma(ab.a, Q_after, ab.c);
+    const double G_lo = tl.cntR + (double)(nb - lo) - 0.5 * Q_lo + 0.5 * (P_lo - 1.0);
+    const double P_end = fma(af.a, P_before, af.c);    // P_{hi-1}
+    const int count = __syncthreads_count(valid && G_lo >= k);
+    const int T = count - 1;
+    if (tid == 0) sm->d[0] = Q_lo;                      // Q_0
+    if (valid && hi == nb) sm->d[1] = P_end;            // P_{nb-1}
+    if (tid == T) {
+        sm->ll[0] = lo;
+        sm->ll[1] = hi;
+        sm->d[2] = P_before;
+        sm->d[3] = Q_after;
+    }
+    __syncthreads();
+
+    if (count > 0 && warp == 0) {
+        long long js;
+        double Pl, Qr;
+        warp_find_crossing(gap, sm->ll[0], sm->ll[1], sm->d[2], sm->d[3], k, &js, &Pl, &Qr);
+        if (lane == 0) {
+            sm->ll[2] = js;
+            sm->d[4] = Pl;
+            sm->d[5] = Qr;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double b;
+        long long js;
+        if (count == 0) {
+            js = 0;
+            b = segment_root(tl.hasL, tl.aL, tl.hasL ? tl.SL : 0.0, true, get(0), sm->d[0],
+                             tl.cntR + (double)nb - k, t);
+        } else {
+            js = sm->ll[2];
+            const bool hasR = js < nb || tl.hasR;
+            const double sR = js < nb ? (double)get(js) : (double)tl.aR;
+            const double Ah = js < nb ? sm->d[5] : (tl.hasR ? tl.SR : 0.0);
+            b = segment_root(true, get(js - 1), sm->d[4], hasR, sR, Ah,
+                             tl.cntR + (double)(nb - js) - k, t);
+        }
+        out->b = b;
+        out->jstar = js;
+        const double Q0 = sm->d[0], Pl = sm->d[1];
+        out->F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * (double)gap(0) * Q0 + 0.5 * tl.SL
+                            : INFINITY;
+        out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * (double)gap(nb) * Pl : -INFINITY;
+    }
+    __syncthreads();
+}
+
+}  // namespace lapsum

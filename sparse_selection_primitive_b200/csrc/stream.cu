@@ -1,0 +1,267 @@
+// Streaming elementwise kernels over long rows: emission of p and the VJP.
+//
+// "Fast LapSum: Exact Differentiable Top-k at Million Scale" (gist.science
+// explainer pages), section 2.1: p_i = sigma((r_i - b)/t) and an analytic
+// VJP.  The VJP used is g_i = (f_i/t)(v_i - R), R = sum_j v_j f_j / sum_j f_j,
+// f_i = 0.5 exp(-|r_i - b|/t) (implicit differentiation of sum_i p_i = k).
+//
+// Each CTA owns a 4096-element tile of one row (256 threads, 16 elements per
+// thread as 4 striped float4 accesses, so every warp access is 512 contiguous
+// bytes).  Per-row reductions go through per-tile partials in the workspace;
+// the last CTA of a row (atomic ticket) combines them in tile order, so the
+// row results are deterministic.  No CTA ever waits for another.
+#include "lapsum_common.cuh"
+#include "lapsum_kernels.h"
+
+namespace lapsum {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kPer = kStreamTile / kThreads;  // 16
+
+template <bool VEC>
+__device__ __forceinline__ void load_tile(const float* __restrict__ row, int64_t n, int64_t base,
+                                          float (&x)[kPer], bool (&ok)[kPer]) {
+    if constexpr (VEC) {
+#pragma unroll
+        for (int q = 0; q < kPer / 4; ++q) {
+            const int64_t i0 = base + ((int64_t)q * kThreads + threadIdx.x) * 4;
+            if (i0 + 4 <= n) {
+                const float4 v = __ldcs(reinterpret_cast<const float4*>(row + i0));
+                x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ok[4 * q + c] = true;
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    ok[4 * q + c] = i0 + c < n;
+                    x[4 * q + c] = ok[4 * q + c] ? row[i0 + c] : 0.f;
+                }
+            }
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int64_t i = base + (int64_t)q * kThreads + threadIdx.x;
+            ok[q] = i < n;
+            x[q] = ok[q] ? row[i] : 0.f;
+        }
+    }
+}
+
+template <bool VEC>
+__device__ __forceinline__ void store_tile(float* __restrict__ row, int64_t n, int64_t base,
+                                           const float (&y)[kPer]) {
+    if constexpr (VEC) {
+#pragma unroll
+        for (int q = 0; q < kPer / 4; ++q) {
+            const int64_t i0 = base + ((int64_t)q * kThreads + threadIdx.x) * 4;
+            if (i0 + 4 <= n) {
+                __stcs(reinterpret_cast<float4*>(row + i0),
+                       make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]));
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    if (i0 + c < n) row[i0 + c] = y[4 * q + c];
+            }
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int64_t i = base + (int64_t)q * kThreads + threadIdx.x;
+            if (i < n) row[i] = y[q];
+        }
+    }
+}
+
+// True for exactly one CTA per row: the last to finish.  Release/acquire
+// through a fence around the ticket; the winner resets the ticket.
+__device__ __forceinline__ bool last_block_of_row(uint32_t* ticket, uint32_t nblocks, int* flag) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t prev = atomicAdd(ticket, 1u);
+        *flag = (prev == nblocks - 1);
+        if (*flag) *ticket = 0u;
+    }
+    __syncthreads();
+    if (*flag) __threadfence();
+    return *flag != 0;
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict__ r, int64_t ld,
+                                                        float* __restrict__ p,
+                                                        const double* __restrict__ b,
+                                                        double* __restrict__ sumf, int64_t n,
+                                                        double t, double* __restrict__ partials,
+                                                        uint32_t* __restrict__ tickets,
+                                                        WsHeader* hdr, int64_t B_total,
+                                                        int path_code) {
+    __shared__ double red[kThreads / 32];
+    __shared__ int flag;
+    const int64_t row = blockIdx.y;
+    if (hdr != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        hdr->last_B = B_total;
+        hdr->last_n = n;
+        hdr->last_path = (uint32_t)path_code;
+    }
+    const int64_t tiles = gridDim.x;
+    const int64_t base = (int64_t)blockIdx.x * kStreamTile;
+    const Thr th = make_thr(b[row], t);
+    float x[kPer], y[kPer];
+    bool ok[kPer];
+    load_tile<VEC>(r + row * ld, n, base, x, ok);
+    double sf = 0.0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const float xs = scaled_margin(x[q], th);
+        const float e = neg_abs_exp(xs);
+        y[q] = cdf_from(xs, e);
+        if (ok[q]) sf += 0.5 * (double)e;
+    }
+    store_tile<VEC>(p + row * ld, n, base, y);
+    if (sumf == nullptr) return;
+    sf = block_sum_d(sf, red);
+    if (threadIdx.x == 0) partials[row * tiles + blockIdx.x] = sf;
+    if (last_block_of_row(&tickets[row], (uint32_t)tiles, &flag)) {
+        double s = 0.0;
+        for (int64_t i = threadIdx.x; i < tiles; i += kThreads) s += partials[row * tiles + i];
+        s = block_sum_d(s, red);
+        if (threadIdx.x == 0) sumf[row] = s;
+    }
+}
+
+// Pass 1 of the VJP: per tile (mu, sum w, sum w v) with w = exp(-(|x| - mu));
+// the last CTA of the row rescales the tiles to the row minimum and forms R.
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
+    const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
+    const float* __restrict__ v, int64_t n, double t, double* __restrict__ partials,
+    double* __restrict__ row_R, uint32_t* __restrict__ tickets) {
+    __shared__ double red[kThreads / 32];
+    __shared__ float fred[kThreads / 32];
+    __shared__ int flag;
+    const int64_t row = blockIdx.y;
+    const int64_t tiles = gridDim.x;
+    const int64_t base = (int64_t)blockIdx.x * kStreamTile;
+    const Thr th = make_thr(b[row], t);
+    float x[kPer], vv[kPer];
+    bool ok[kPer];
+    load_tile<VEC>(r + row * ld, n, base, x, ok);
+    load_tile<VEC>(v + row * ld, n, base, vv, ok);
+    float m = INFINITY;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        x[q] = ok[q] ? fabsf(scaled_margin(x[q], th)) : INFINITY;
+        m = fminf(m, x[q]);
+    }
+    const float mu = block_min_f(m, fred);
+    double sw = 0.0, swv = 0.0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        if (ok[q]) {
+            const double w = (double)__expf(mu - x[q]);
+            sw += w;
+            swv += w * (double)vv[q];
+        }
+    }
+    sw = block_sum_d(sw, red);
+    swv = block_sum_d(swv, red);
+    if (threadIdx.x == 0) {
+        double* pr = partials + (row * tiles + blockIdx.x) * 3;
+        pr[0] = (double)mu;
+        pr[1] = sw;
+        pr[2] = swv;
+    }
+    if (last_block_of_row(&tickets[row], (uint32_t)tiles, &flag)) {
+        float mloc = INFINITY;
+        for (int64_t i = threadIdx.x; i < tiles; i += kThreads)
+            mloc = fminf(mloc, (float)partials[(row * tiles + i) * 3]);
+        const double mrow = (double)block_min_f(mloc, fred);
+        double s = 0.0, sv = 0.0;
+        for (int64_t i = threadIdx.x; i < tiles; i += kThreads) {
+            const double* pr = partials + (row * tiles + i) * 3;
+            const double sc = exp(mrow - pr[0]);
+            s += pr[1] * sc;
+            sv += pr[2] * sc;
+        }
+        s = block_sum_d(s, red);
+        sv = block_sum_d(sv, red);
+        if (threadIdx.x == 0) row_R[row] = sv / s;
+    }
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads) bwd_apply_kernel(
+    const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
+    const float* __restrict__ v, float* __restrict__ g, int64_t n, double t,
+    const double* __restrict__ row_R) {
+    const int64_t row = blockIdx.y;
+    const int64_t base = (int64_t)blockIdx.x * kStreamTile;
+    const Thr th = make_thr(b[row], t);
+    const double R = row_R[row];
+    float x[kPer], vv[kPer], y[kPer];
+    bool ok[kPer];
+    load_tile<VEC>(r + row * ld, n, base, x, ok);
+    load_tile<VEC>(v + row * ld, n, base, vv, ok);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const float f = 0.5f * neg_abs_exp(scaled_margin(x[q], th));
+        y[q] = f * th.inv_t * (float)((double)vv[q] - R);
+    }
+    store_tile<VEC>(g + row * ld, n, base, y);
+}
+
+}  // namespace
+
+int64_t stream_tiles(int64_t n) { return (n + kStreamTile - 1) / kStreamTile; }
+
+cudaError_t launch_emit(const float* r, int64_t ld, float* p, const double* b, double* sumf,
+                        int64_t B, int64_t n, double t, double* partials, uint32_t* tickets,
+                        int vec, WsHeader* hdr, int64_t B_total, int path_code, cudaStream_t st) {
+    const dim3 grid((unsigned)stream_tiles(n), (unsigned)B);
+    if (vec)
+        {
+            ProfScope ps_("emit", st);
+            emit_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets,
+                                                     hdr, B_total, path_code);
+        }
+    else
+        {
+            ProfScope ps_("emit", st);
+            emit_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets,
+                                                      hdr, B_total, path_code);
+        }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, const float* v,
+                                   float* g, int64_t B, int64_t n, double t, double* partials,
+                                   double* row_R, uint32_t* tickets, int vec, cudaStream_t st) {
+    const dim3 grid((unsigned)stream_tiles(n), (unsigned)B);
+    if (vec) {
+        {
+            ProfScope ps_("bwd_reduce", st);
+            bwd_reduce_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
+                                                           tickets);
+        }
+        {
+            ProfScope ps_("bwd_apply", st);
+            bwd_apply_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R);
+        }
+    } else {
+        {
+            ProfScope ps_("bwd_reduce", st);
+            bwd_reduce_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
+                                                            tickets);
+        }
+        {
+            ProfScope ps_("bwd_apply", st);
+            bwd_apply_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R);
+        }
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace lapsum

@@ -1,0 +1,64 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
+binding and compare with the fp64 oracle at the tolerances the benchmark spec fixes:
+
+    |b_gpu - b_ref| <= 1e-5 max(t, |b_ref|)
+    max |p_gpu - p_ref| <= 1e-5
+    |sum p_gpu - k| <= 1e-3          (summed in fp64)
+    max |g_gpu - g_ref| <= 1e-4 max |g_ref|
+
+Expected values come only from the oracle, evaluated on the same seeded
+inputs; nothing computed on the GPU is fed back to the oracle.
+"""
+import numpy as np
+import torch
+
+import oracle
+import sparse_selection_primitive_b200 as L
+
+TOL_B = 1e-5
+TOL_P = 1e-5
+TOL_SUM = 1e-3
+TOL_G = 1e-4
+# fp32 cannot represent |g| below its smallest subnormal; when every reference
+# value of a row lies below this floor the relative test is meaningless.
+G_FLOOR = 1e-37
+
+
+def run_gpu(r: np.ndarray, k: float, t: float, path="auto", v: np.ndarray = None, seed=0,
+            device="cuda:0", want_sum_f=False, ws=None):
+    rt = torch.from_numpy(np.ascontiguousarray(r, dtype=np.float32)).to(device)
+    if rt.dim() == 1:
+        rt = rt.unsqueeze(0)
+    out = L.forward(rt, k, t, path=path, seed=seed, ws=ws, want_sum_f=want_sum_f)
+    p, b = out[0], out[1]
+    res = {"p": p.cpu().numpy().astype(np.float64), "b": b.cpu().numpy()}
+    if want_sum_f:
+        res["sum_f"] = out[2].cpu().numpy()
+    if v is not None:
+        vt = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).to(device)
+        if vt.dim() == 1:
+            vt = vt.unsqueeze(0)
+        g = L.backward(rt, b, vt, t, ws=ws)
+        res["g"] = g.cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    return res
+
+
+def check_row(r_row, v_row, k, t, b_gpu, p_gpu, g_gpu=None, b_ref=None, label=""):
+    """Compare one row of GPU output with the oracle; returns the reference b."""
+    if b_ref is None:
+        b_ref = oracle.solve_b(r_row, k, t)
+    assert abs(b_gpu - b_ref) <= TOL_B * max(t, abs(b_ref)), \
+        f"{label}: b {b_gpu!r} vs oracle {b_ref!r} (t={t})"
+    p_ref = oracle.emit_p(r_row, b_ref, t)
+    dp = np.max(np.abs(p_gpu - p_ref))
+    assert dp <= TOL_P, f"{label}: max|dp| = {dp:.3e}"
+    s = float(np.sum(p_gpu, dtype=np.float64))
+    assert abs(s - k) <= TOL_SUM, f"{label}: sum p = {s!r}, k = {k}"
+    if g_gpu is not None:
+        g_ref, _, _ = oracle.vjp(r_row, v_row, b_ref, t)
+        scale = np.max(np.abs(g_ref))
+        dg = np.max(np.abs(g_gpu - g_ref))
+        assert dg <= max(TOL_G * scale, G_FLOOR), \
+            f"{label}: max|dg| = {dg:.3e} vs {TOL_G} * {scale:.3e}"
+    return b_ref

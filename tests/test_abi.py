@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load, export every function declared in include/lapsum.h,
+reject invalid arguments on the host before any CUDA call, and size its
+workspace consistently.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_selection_primitive_b200 as L
+from sparse_selection_primitive_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return L._lib()
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(lapsum_[a-z_0-9]+)\s*\(", text,
+                            flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10, names
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.lapsum_abi_version() == 1
+    for code in range(6):
+        assert lib.lapsum_status_string(code)
+    assert lib.lapsum_status_string(99) == b"unknown status"
+
+
+def test_invalid_arguments_rejected_on_host(lib):
+    f = lib.lapsum_forward
+    ws = ctypes.c_void_p(256)  # never dereferenced: every call below fails validation first
+    d = ctypes.c_void_p(4096)
+    # null pointers
+    assert f(None, 8, d, d, None, 1, 8, 2.0, 0.1, 0, 0, ws, 1 << 20, None) == 1
+    # B < 1, n < 1, ld < n
+    assert f(d, 8, d, d, None, 0, 8, 2.0, 0.1, 0, 0, ws, 1 << 20, None) == 1
+    assert f(d, 8, d, d, None, 1, 0, 0.5, 0.1, 0, 0, ws, 1 << 20, None) == 1
+    assert f(d, 4, d, d, None, 1, 8, 2.0, 0.1, 0, 0, ws, 1 << 20, None) == 1
+    # k outside (0, n), t <= 0, non-finite
+    for k, t in [(0.0, 0.1), (8.0, 0.1), (-1.0, 0.1), (2.0, 0.0), (2.0, -1.0),
+                 (float("nan"), 0.1), (2.0, float("inf"))]:
+        assert f(d, 8, d, d, None, 1, 8, k, t, 0, 0, ws, 1 << 20, None) == 1
+    # bad path code / unknown flag bits
+    assert f(d, 8, d, d, None, 1, 8, 2.0, 0.1, 7, 0, ws, 1 << 20, None) == 1
+    assert f(d, 8, d, d, None, 1, 8, 2.0, 0.1, 0x1000, 0, ws, 1 << 20, None) == 1
+    # workspace: null, misaligned, too small
+    assert f(d, 8, d, d, None, 1, 8, 2.0, 0.1, 0, 0, None, 1 << 20, None) == 2
+    assert f(d, 8, d, d, None, 1, 8, 2.0, 0.1, 0, 0, ctypes.c_void_p(257), 1 << 20, None) == 2
+    assert f(d, 8, d, d, None, 1, 8, 2.0, 0.1, 0, 0, ws, 16, None) == 2
+    b = lib.lapsum_backward
+    assert b(None, 8, d, d, d, 1, 8, 0.1, ws, 1 << 20, None) == 1
+    assert b(d, 8, d, d, d, 1, 8, 0.0, ws, 1 << 20, None) == 1
+    assert b(d, 8, d, d, d, 1, 8000, 0.1, ws, 1 << 20, None) == 1  # ld < n
+    assert b(d, 8000, d, d, d, 1, 8000, 0.1, None, 1 << 20, None) == 2
+
+
+def test_workspace_sizes(lib):
+    wb = L.workspace_bytes
+    assert wb(0, 10, 1.0) == 0 and wb(1, 0, 1.0) == 0
+    assert wb(1, 10, 1.0, path=9) == 0
+    # sizes grow with the problem and are multiples of 256
+    for B, n in [(1, 1024), (16384, 256), (256, 65536), (1, 3342336), (1, 10**8)]:
+        s = wb(B, n, 1.0)
+        assert s > 0 and s % 256 == 0
+        assert int(lib.lapsum_backward_workspace_bytes(B, n)) <= s
+    # the radix path holds two key buffers; the bracket path holds two band buffers
+    assert wb(256, 65536, 1024.0) >= 2 * 256 * 65536 * 4
+    assert wb(1, 10**8, 1e5) >= 2 * 10**8 * 4

@@ -1,0 +1,108 @@
+"""GPU parity of the bracketing steps themselves ("Fast LapSum: Exact
+Differentiable Top-k at Million Scale", gist.science explainer pages,
+section 2.2, probabilistic bracketing, steps 1-4).
+
+* step 1: the GPU's sample equals the oracle's draw of the same counter-based
+  SplitMix64 stream (indices exactly, values to fp32 rounding of the noise),
+  and the bracket ends equal the oracle's order statistics of its own sample;
+* step 2: the fold's tail counts and sums equal the oracle's fold over the
+  oracle's bracket;
+* steps 3-4: a bracket forced to miss is widened and still gives the exact b;
+  with widening disabled the miss is reported, and b is NaN.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_selection_primitive_b200 as L
+from tests.gpu_helpers import check_row
+from workloads import random_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def _forward(r, k, t, flags=0, seed=0):
+    n = r.shape[-1]
+    ws = L.Workspace(1, n, k, "bracket")
+    rt = torch.from_numpy(r.reshape(1, -1)).cuda()
+    p, b = L.forward(rt, k, t, path=2 | flags, seed=seed, ws=ws)
+    torch.cuda.synchronize()
+    return ws, p.cpu().numpy()[0].astype(np.float64), b.item()
+
+
+@pytest.mark.parametrize("n,k,t,seed", [(200000, 150.0, 0.01, 0), (1 << 20, 1000.0, 0.005, 7),
+                                        (50000, 25000.0, 0.3, 3)])
+def test_sample_and_bracket_match_oracle(cuda_device, n, k, t, seed):
+    r, _ = random_rows(seed, 1, n, "mix_nu")
+    ws, _, _ = _forward(r[0], k, t, seed=seed)
+    info = L.row_info(ws, 0)
+    m = info["sample_m"]
+    y_gpu = L.sample_values(ws, 0, m).astype(np.float64)
+    y_ref, _ = oracle.sample(r[0], t, seed=seed, c0=0, m=m)
+    assert np.max(np.abs(y_gpu - y_ref)) <= 1e-6 * max(1.0, np.max(np.abs(y_ref)))
+    l, h = oracle.binom_ranks(m, k / n, 1e-6)
+    assert (info["rank_l"], info["rank_h"]) == (l, h)
+    aL, aR = oracle.bracket_from_sample(y_ref, l, h)
+    if info["attempts"] == 1:
+        assert abs(info["a_L"] - aL) <= 1e-6 * max(1.0, abs(aL)) or (aL == -math.inf and
+                                                                     info["a_L"] == -math.inf)
+        assert abs(info["a_R"] - aR) <= 1e-6 * max(1.0, abs(aR)) or (aR == math.inf and
+                                                                    info["a_R"] == math.inf)
+
+
+@pytest.mark.parametrize("n,k,t", [(300000, 200.0, 0.01), (1 << 21, 2000.0, 0.003)])
+def test_fold_matches_oracle(cuda_device, n, k, t):
+    r, _ = random_rows(11, 1, n, "normal")
+    ws, _, _ = _forward(r[0], k, t)
+    info = L.row_info(ws, 0)
+    m = info["sample_m"]
+    y_ref, _ = oracle.sample(r[0], t, seed=0, c0=0, m=m)
+    l, h = oracle.binom_ranks(m, k / n, 1e-6)
+    aL, aR = oracle.bracket_from_sample(y_ref, l, h)
+    fo = oracle.fold(r[0], aL, aR, t)
+    assert info["attempts"] == 1
+    # the two brackets agree to fp32 rounding; scores falling between them may
+    # change sides, so the counts may differ by exactly those scores
+    lo_gap = np.sum((r[0] >= min(aL, info["a_L"])) & (r[0] < max(aL, info["a_L"])))
+    hi_gap = np.sum((r[0] >= min(aR, info["a_R"])) & (r[0] < max(aR, info["a_R"])))
+    assert abs(info["cnt_R"] - fo["cnt_R"]) <= hi_gap
+    assert abs(info["n_band"] - fo["n_band"]) <= lo_gap + hi_gap
+    if lo_gap == 0 and hi_gap == 0:
+        assert info["cnt_R"] == fo["cnt_R"] and info["n_band"] == fo["n_band"]
+        assert abs(info["S_R"] - fo["S_R"]) <= 1e-5 * max(1.0, fo["S_R"])
+        assert abs(info["S_L"] - fo["S_L"]) <= 1e-5 * max(1.0, fo["S_L"])
+
+
+@pytest.mark.parametrize("n", [20000, 400000])
+def test_forced_miss_is_widened_and_exact(cuda_device, n):
+    r, v = random_rows(5, 1, n)
+    k, t = 60.0, 0.01
+    ws, p, b = _forward(r[0], k, t, flags=L.FLAG_FORCE_MISS)
+    info = L.row_info(ws, 0)
+    assert info["attempts"] >= 2
+    assert L.read_status(ws) == 0
+    check_row(r[0], v[0], k, t, b, p, label=f"forced miss n={n}")
+
+
+def test_forced_miss_without_retry_reports(cuda_device):
+    r, _ = random_rows(6, 1, 30000)
+    ws, _, b = _forward(r[0], 40.0, 0.01, flags=L.FLAG_FORCE_MISS | L.FLAG_NO_RETRY)
+    assert L.read_status(ws) == 4
+    assert math.isnan(b)
+    assert L.row_info(ws, 0)["attempts"] == 1
+
+
+def test_large_band_narrowing(cuda_device):
+    # q = 1/2 makes the binomial bracket hold ~n/10 scores: the band is far
+    # larger than the on-chip sort and must be narrowed by histogram levels
+    n = 1 << 20
+    r, v = random_rows(8, 1, n, "normal_q64")
+    k, t = n / 2.0, 0.05
+    ws, p, b = _forward(r[0], k, t)
+    info = L.row_info(ws, 0)
+    assert info["n_band"] > 4096
+    assert info["refine_levels"] >= 1
+    check_row(r[0], v[0], k, t, b, p, label="large band")

@@ -1,0 +1,169 @@
+"""GPU parity of every solver against the fp64 oracle on seeded inputs.
+
+Sizes are chosen so the oracle finishes in seconds while the CUDA path still
+crosses its tile boundaries (warp, CTA, 4096-key bitonic capacity, 4096-key
+radix tiles) and ragged tails.  Solvers: the on-chip bitonic full sort, the
+radix full sort, and probabilistic bracketing, each also forced onto sizes it
+would not pick by itself.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_selection_primitive_b200 as L
+from tests.gpu_helpers import check_row, run_gpu
+from workloads import random_rows
+
+pytestmark = pytest.mark.gpu
+
+SIZES_ONCHIP = [1, 2, 3, 7, 31, 32, 33, 64, 100, 255, 256, 257, 511, 1000, 1024, 2047, 2049, 4095,
+                4096]
+SIZES_LONG = [4097, 5000, 8192, 12345, 65536, 70001]
+
+
+def k_values(n):
+    ks = {min(n - 0.5, 0.5), max(0.25, n / 3.0)}
+    if n > 2:
+        ks |= {1.0, float(n - 1), float(max(1, n // 8))}
+    return sorted(k for k in ks if 0 < k < n)
+
+
+@pytest.mark.parametrize("n", SIZES_ONCHIP)
+def test_onchip_bitonic_sizes(cuda_device, n):
+    B = 3
+    r, v = random_rows(10 + n, B, n)
+    for k in k_values(n):
+        for t in (0.05, 1.0):
+            out = run_gpu(r, k, t, path="fullsort", v=v)
+            for i in range(B):
+                check_row(r[i], v[i], k, t, out["b"][i], out["p"][i], out["g"][i],
+                          label=f"bitonic n={n} k={k} t={t} row={i}")
+
+
+@pytest.mark.parametrize("n", [300, 4096, 5000, 12345, 70001])
+def test_radix_sizes(cuda_device, n):
+    B = 2
+    r, v = random_rows(20 + n, B, n)
+    for k in k_values(n):
+        out = run_gpu(r, k, 0.05, path="radix", v=v)
+        for i in range(B):
+            check_row(r[i], v[i], k, 0.05, out["b"][i], out["p"][i], out["g"][i],
+                      label=f"radix n={n} k={k} row={i}")
+
+
+@pytest.mark.parametrize("n", [64, 5000, 65536, 300000])
+def test_bracket_sizes(cuda_device, n):
+    r, v = random_rows(30 + n, 1, n)
+    for k in k_values(n):
+        out = run_gpu(r, k, 0.02, path="bracket", v=v)
+        check_row(r[0], v[0], k, 0.02, out["b"][0], out["p"][0], out["g"][0],
+                  label=f"bracket n={n} k={k}")
+
+
+@pytest.mark.parametrize("dist", ["normal", "normal_q64", "abs_t3", "mix_nu"])
+@pytest.mark.parametrize("path", ["fullsort", "radix", "bracket"])
+def test_distributions_and_ties(cuda_device, dist, path):
+    n = 3000 if path == "fullsort" else 20000
+    r, v = random_rows(7, 2, n, dist)
+    for k, t in [(10.0, 0.1), (123.5, 0.01), (n / 2, 0.3)]:
+        out = run_gpu(r, k, t, path=path, v=v)
+        for i in range(2):
+            check_row(r[i], v[i], k, t, out["b"][i], out["p"][i], out["g"][i],
+                      label=f"{path} {dist} k={k} t={t}")
+
+
+@pytest.mark.parametrize("path", ["fullsort", "radix", "bracket"])
+def test_degenerate_rows(cuda_device, path):
+    n = 1000 if path == "fullsort" else 9000
+    # all equal: p = k/n everywhere
+    r = np.full((1, n), 1.25, dtype=np.float32)
+    v = np.random.default_rng(0).standard_normal((1, n)).astype(np.float32)
+    out = run_gpu(r, 7.0, 0.1, path=path, v=v)
+    check_row(r[0], v[0], 7.0, 0.1, out["b"][0], out["p"][0], out["g"][0], label="all equal")
+    # two distinct values, huge gap relative to t (flat plateau of F)
+    r2 = np.zeros((1, n), dtype=np.float32)
+    r2[0, : n // 10] = 5.0
+    out = run_gpu(r2, float(n // 10), 1e-3, path=path, v=v)
+    check_row(r2[0], v[0], float(n // 10), 1e-3, out["b"][0], out["p"][0], out["g"][0],
+              label="plateau")
+    # wide score range
+    r3, _ = random_rows(5, 1, n)
+    r3 = (r3 * 1e4).astype(np.float32)
+    out = run_gpu(r3, 50.0, 30.0, path=path, v=v)
+    check_row(r3[0], v[0], 50.0, 30.0, out["b"][0], out["p"][0], out["g"][0], label="wide")
+    # tiny temperature, well separated scores: close to the hard top-k mask
+    r4 = np.random.default_rng(3).permutation(n).astype(np.float32)[None, :]
+    out = run_gpu(r4, 17.0, 1e-3, path=path, v=v)
+    check_row(r4[0], v[0], 17.0, 1e-3, out["b"][0], out["p"][0], out["g"][0], label="t->0")
+
+
+def test_k_extremes(cuda_device):
+    n = 777
+    r, v = random_rows(9, 1, n)
+    for k in (1e-6, 1e-3, n - 1e-3, n - 1e-6):
+        for path in ("fullsort", "radix", "bracket"):
+            out = run_gpu(r, k, 0.2, path=path, v=v)
+            check_row(r[0], v[0], k, 0.2, out["b"][0], out["p"][0], out["g"][0],
+                      label=f"{path} k={k}")
+
+
+def test_strided_rows_and_unaligned(cuda_device):
+    # ld > n and a base pointer that is not 16-byte aligned take the scalar paths
+    B, n, ld = 5, 300, 333
+    r, v = random_rows(11, B, ld)
+    full = torch.from_numpy(r).cuda()
+    vv = torch.from_numpy(v).cuda()
+    for path in ("fullsort", "radix"):
+        sub = full[:, 1:1 + n]
+        p, b = L.forward(sub, 12.0, 0.1, path=path)
+        g = L.backward(sub, b, vv[:, 1:1 + n], 0.1)
+        for i in range(B):
+            check_row(r[i, 1:1 + n], v[i, 1:1 + n], 12.0, 0.1, b[i].item(),
+                      p[i].cpu().numpy().astype(np.float64), g[i].cpu().numpy().astype(np.float64),
+                      label=f"strided {path} row={i}")
+
+
+def test_nonfinite_scores_reported(cuda_device):
+    for path, n in (("fullsort", 100), ("radix", 5000), ("bracket", 5000)):
+        r, _ = random_rows(1, 2, n)
+        r[1, n // 2] = np.nan
+        ws = L.Workspace(2, n, 3.0, path)
+        _, b = L.forward(torch.from_numpy(r).cuda(), 3.0, 0.1, path=path, ws=ws)
+        assert L.read_status(ws) == 3, path
+        bb = b.cpu().numpy()
+        assert math.isnan(bb[1]), path
+        if path != "bracket":
+            assert not math.isnan(bb[0])
+        assert L.read_status(ws) == 0  # cleared by the read
+
+
+def test_sum_f_output(cuda_device):
+    for path, n in (("fullsort", 1000), ("radix", 6000), ("bracket", 6000)):
+        r, _ = random_rows(2, 2, n)
+        out = run_gpu(r, 20.0, 0.05, path=path, want_sum_f=True)
+        for i in range(2):
+            f = oracle.density(r[i], oracle.solve_b(r[i], 20.0, 0.05), 0.05)
+            assert abs(out["sum_f"][i] - f.sum()) <= 1e-4 * f.sum()
+
+
+def test_autograd_matches_library_backward(cuda_device):
+    r, v = random_rows(4, 3, 600)
+    rt = torch.from_numpy(r).cuda().requires_grad_(True)
+    p = L.soft_topk(rt, 9.0, 0.1)
+    p.backward(torch.from_numpy(v).cuda())
+    _, b = L.forward(rt.detach(), 9.0, 0.1)
+    g = L.backward(rt.detach(), b, torch.from_numpy(v).cuda(), 0.1)
+    assert torch.equal(rt.grad, g)
+
+
+def test_repeat_calls_are_deterministic(cuda_device):
+    for path, n in (("fullsort", 2000), ("radix", 20000), ("bracket", 20000)):
+        r, v = random_rows(6, 2, n)
+        a = run_gpu(r, 50.0, 0.05, path=path, v=v)
+        c = run_gpu(r, 50.0, 0.05, path=path, v=v)
+        assert np.array_equal(a["b"], c["b"]), path
+        assert np.array_equal(a["p"], c["p"]), path
+        assert np.array_equal(a["g"], c["g"]), path
