@@ -195,6 +195,8 @@ def main():
     ap.add_argument("--no-table", action="store_true", help="skip the per-workload table")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--n-override", type=int, default=0,
+                    help="profiling runs: shrink the workload's row length (k scaled to keep k/n)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -232,6 +234,10 @@ def main():
 
     L._build.build()
     w = WORKLOADS[args.workload]
+    if args.n_override:
+        from dataclasses import replace
+        w = replace(w, n=args.n_override, k=max(1.0, round(w.k * args.n_override / w.n)),
+                    name=f"{w.name}@n={args.n_override}")
     r_h, v_h = make_inputs(w, seed=rank)
     stream = torch.cuda.current_stream(dev)
 
@@ -278,6 +284,10 @@ def main():
         torch.cuda.synchronize(dev)
         res = {"flush": flush, "ws": ws, "rd": rd, "vd": vd, "pd": pd, "gd": gd, "bd": bd,
                "fwd": fwd, "bwd": bwd, "timed": timed}
+        if w.path == "bracket":
+            info = L.row_info(ws, 0)
+            res["bracket"] = {key: info[key] for key in ("attempts", "n_band", "refine_levels",
+                                                       "sample_m", "rank_l", "rank_h")}
         if table:
             tf, _ = timed(fwd, steps)
             tb, _ = timed(bwd, steps)
@@ -364,7 +374,8 @@ def main():
                 rr, vv = r_h, v_h
             else:
                 rr, vv = make_inputs(wk, seed=0)
-            T = run_workload(wk, rr, vv, 10, 3, table=True)["table"]
+            RW = run_workload(wk, rr, vv, 10, 3, table=True)
+            T = RW["table"]
             table[name] = {
                 "fwd_ms": round(T["fwd_ms"], 5), "bwd_ms": round(T["bwd_ms"], 5),
                 "fwdbwd_ms": round(T["fwdbwd_ms"], 5),
@@ -375,6 +386,9 @@ def main():
                 / (T["fwdbwd_ms"] / 1e3) / 1e9,
             }
             table[name]["fwdbwd_frac_of_peak"] = table[name]["fwdbwd_algorithmic_gbs"] / peak_gbs
+            if "bracket" in RW:
+                table[name]["bracket"] = RW["bracket"]
+            del RW
             torch.cuda.empty_cache()
 
     cpu = None
@@ -391,6 +405,7 @@ def main():
                        "l2": "flushed before each step" if R["flush"] else
                              "inputs larger than L2 (no flush)",
                        "parallelism": f"{world} independent instances (one per GPU)"},
+            "bracket": R.get("bracket"),
             "step_algorithmic_gbs": step_gbs,
             "step_frac_of_peak": step_gbs / peak_gbs,
             "roofline": roofline,

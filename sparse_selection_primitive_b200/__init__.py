@@ -157,9 +157,29 @@ def _as_rows(x: torch.Tensor) -> torch.Tensor:
         raise ValueError("scores must be 1-D or 2-D (rows x n)")
     if x.dtype != torch.float32 or not x.is_cuda:
         raise TypeError("scores must be a float32 CUDA tensor")
-    if x.stride(1) != 1:
+    B, n = x.shape
+    if x.stride(1) != 1 or (B > 1 and x.stride(0) < n):
         x = x.contiguous()
     return x
+
+
+def _ld(x: torch.Tensor) -> int:
+    """Leading dimension of a row-major (B, n) view; a single row has ld = n."""
+    return x.stride(0) if x.shape[0] > 1 else x.shape[1]
+
+
+def _like_rows(x: torch.Tensor, ld: int) -> torch.Tensor:
+    """Uninitialised (B, n) float32 buffer with the same leading dimension as x."""
+    B, n = x.shape
+    if ld == n:
+        return torch.empty((B, n), dtype=torch.float32, device=x.device)
+    return torch.empty((B, ld), dtype=torch.float32, device=x.device)[:, :n]
+
+
+def _check_out(out: torch.Tensor, ref: torch.Tensor, ld: int, what: str):
+    if out.shape != ref.shape or out.dtype != torch.float32 or not out.is_cuda or \
+            out.stride(1) != 1 or _ld(out) != ld:
+        raise ValueError(f"{what} must be float32 CUDA with the shape and row stride of r")
 
 
 def forward(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0, ws: Workspace = None,
@@ -168,14 +188,19 @@ def forward(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0, ws:
     squeeze = r.dim() == 1
     r2 = _as_rows(r)
     B, n = r2.shape
-    ld = r2.stride(0)
+    ld = _ld(r2)
     code = _path_code(path)
     if ws is None or not ws.fits(B, n, k, code):
         ws = Workspace(B, n, k, code, r2.device)
     if p is None:
-        p = torch.empty_like(r2)
+        p = _like_rows(r2, ld)
+    else:
+        p = p.view(B, n) if p.dim() == 1 else p
+        _check_out(p, r2, ld, "p")
     if b is None:
         b = torch.empty(B, dtype=torch.float64, device=r2.device)
+    elif b.dtype != torch.float64 or b.numel() != B or not b.is_contiguous():
+        raise ValueError("b must be a contiguous float64 CUDA tensor with one entry per row")
     sf = torch.empty(B, dtype=torch.float64, device=r2.device) if want_sum_f else None
     _check(_lib().lapsum_forward(r2.data_ptr(), ld, p.data_ptr(), b.data_ptr(),
                                  sf.data_ptr() if sf is not None else None, B, n, float(k),
@@ -195,16 +220,19 @@ def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Wo
     B, n = r2.shape
     if v2.shape != r2.shape:
         raise ValueError("v must have the shape of r")
-    if v2.stride(0) != r2.stride(0):
+    if _ld(v2) != _ld(r2):
         v2 = v2.contiguous()
         r2 = r2.contiguous()
-    ld = r2.stride(0)
+    ld = _ld(r2)
     if ws is None or not ws.fits_backward(B, n):
         ws = Workspace(B, n, 0.5, "fullsort", r2.device)
     if g is None:
-        g = torch.empty_like(r2)
-    if b.dtype != torch.float64 or not b.is_cuda:
-        raise TypeError("b must be a float64 CUDA tensor")
+        g = _like_rows(r2, ld)
+    else:
+        g = g.view(B, n) if g.dim() == 1 else g
+        _check_out(g, r2, ld, "g")
+    if b.dtype != torch.float64 or not b.is_cuda or b.numel() != B:
+        raise TypeError("b must be a float64 CUDA tensor with one entry per row")
     _check(_lib().lapsum_backward(r2.data_ptr(), ld, b.data_ptr(), v2.data_ptr(), g.data_ptr(), B,
                                   n, float(t), ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
            "lapsum_backward")

@@ -106,6 +106,79 @@ struct GlobalSampleKeyGet {
     __device__ __forceinline__ uint32_t operator()(int i) const { return to_key(y[i]); }
 };
 
+// The rho_a-th and rho_b-th largest of m keys in shared memory (1-based;
+// 0 = not wanted), rho_max = the larger.  One histogram pass on the top 11 key
+// bits finds the bin holding rank rho_max; every key in that bin or above is a
+// candidate.  If there are at most 4096 candidates they are compacted and
+// sorted with the register bitonic network and both ranks are read off;
+// otherwise returns false and the caller selects by full radix select.
+__device__ bool top_ranks(const uint32_t* keys, int m, int64_t rho_max, int64_t rho_a,
+                          int64_t rho_b, uint32_t* hist, uint32_t* wsum, uint32_t* bcast,
+                          uint32_t* cand, uint32_t* xch, float* out_a, float* out_b) {
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < m; i += blockDim.x) atomicAdd(&hist[keys[i] >> 21], 1u);
+    __syncthreads();
+    // suffix counts: thread i owns bins 2i, 2i+1
+    const int i0 = 2 * threadIdx.x;
+    const uint32_t c0 = hist[i0], c1 = hist[i0 + 1];
+    const uint32_t mine = c0 + c1;
+    uint32_t incl = mine;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t o = __shfl_down_sync(0xffffffffu, incl, d);
+        if (lane + d < 32) incl += o;
+    }
+    if (lane == 0) wsum[w] = incl;
+    __syncthreads();
+    uint32_t above = incl - mine;
+    for (int u = w + 1; u < (int)(blockDim.x >> 5); ++u) above += wsum[u];
+    if (above < rho_max && rho_max <= (int64_t)above + c1) {
+        bcast[0] = i0 + 1;
+        bcast[1] = above + c1;  // candidates: keys in this bin or above
+    }
+    if ((int64_t)above + c1 < rho_max && rho_max <= (int64_t)above + c1 + c0) {
+        bcast[0] = i0;
+        bcast[1] = above + c1 + c0;
+    }
+    __syncthreads();
+    const uint32_t bin = bcast[0], ncand = bcast[1];
+    __syncthreads();
+    if (ncand > (uint32_t)kBandSortMax) return false;
+    if (threadIdx.x == 0) bcast[2] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+        const uint32_t kk = keys[i];
+        if ((kk >> 21) >= bin) cand[atomicAdd(&bcast[2], 1u)] = kk;
+    }
+    __syncthreads();
+    // ascending sort of the candidates (padding 0 sorts first); rank r from the
+    // top is at position npad - r
+    uint32_t key[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int j = threadIdx.x * 4 + e;
+        key[e] = j < (int)ncand ? cand[j] : 0u;
+    }
+    bitonic_sort_row<4, kBlk, kBlk>(key, threadIdx.x, xch);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cand[threadIdx.x * 4 + e] = key[e];
+    __syncthreads();
+    constexpr int npad = 4 * kBlk;
+    if (threadIdx.x == 0) {
+        if (rho_a >= 1) *out_a = from_key(cand[npad - rho_a]);
+        if (rho_b >= 1) *out_b = from_key(cand[npad - rho_b]);
+        wsum[0] = __float_as_uint(*out_a);
+        wsum[1] = __float_as_uint(*out_b);
+    }
+    __syncthreads();
+    *out_a = __uint_as_float(wsum[0]);
+    *out_b = __uint_as_float(wsum[1]);
+    __syncthreads();
+    return true;
+}
+
 // ----------------------------------------------------------------------------
 // 1. Localization sample.
 // ----------------------------------------------------------------------------
@@ -113,33 +186,61 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
                                                       double t, uint64_t seed, uint64_t c0, int m,
                                                       Ladder lad, int force_miss, int max_attempts,
                                                       float* __restrict__ sample_out,
+                                                      unsigned long long* __restrict__ bins,
                                                       RowState* st) {
+    for (int i = threadIdx.x; i < 3 * kBins; i += kBlk) bins[i] = 0ull;
     extern __shared__ uint32_t dyn[];
     uint32_t* keys = dyn;              // m keys
+    uint32_t* cand = dyn + m;          // up to 4096 candidate keys
+    uint32_t* xch = cand + kBandSortMax;  // bitonic exchange area (4096 words)
     __shared__ uint32_t hist[2048];
     __shared__ uint32_t wsum[32];
     __shared__ uint32_t bcast[4];
     const float tf = (float)t;
-    for (int s = threadIdx.x; s < m; s += kBlk) {
-        const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
-        const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
-        const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
-        const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
-        const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
-        const float eps = (u < 0.0 ? 1.f : -1.f) * tf * logf(a);
-        const float y = __ldg(r + I) + eps;
-        sample_out[s] = y;
-        keys[s] = to_key(y);
+    // m is a multiple of 8 * kBlk / 4: each thread issues its gathers in groups
+    // of 8 independent loads so their latencies overlap.
+    constexpr int G = 8;
+    for (int s0 = threadIdx.x; s0 < m; s0 += G * kBlk) {
+        float rv[G];
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+            const int s = s0 + q * kBlk;
+            rv[q] = 0.f;
+            if (s < m) {
+                const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
+                const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
+                rv[q] = __ldg(r + I);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+            const int s = s0 + q * kBlk;
+            if (s < m) {
+                const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
+                const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
+                const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
+                const float eps = (u < 0.0 ? 1.f : -1.f) * tf * logf(a);
+                const float y = rv[q] + eps;
+                sample_out[s] = y;
+                keys[s] = to_key(y);
+            }
+        }
     }
     __syncthreads();
     float aR = INFINITY, aL = -INFINITY;
-    if (lad.l[0] >= 1) {
-        const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.l[0], hist, wsum, bcast);
-        aR = from_key(kk);
-    }
-    if (lad.h[0] <= m) {
-        const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.h[0], hist, wsum, bcast);
-        aL = from_key(kk);
+    const int64_t rmax = lad.h[0] <= m ? lad.h[0] : lad.l[0];
+    if (rmax >= 1 && top_ranks(keys, m, rmax, lad.l[0], lad.h[0] <= m ? lad.h[0] : 0, hist, wsum,
+                               bcast, cand, xch, &aR, &aL)) {
+        // both order statistics read off the sorted top candidates
+    } else {
+        if (lad.l[0] >= 1) {
+            const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.l[0], hist, wsum, bcast);
+            aR = from_key(kk);
+        }
+        if (lad.h[0] <= m) {
+            const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.h[0], hist, wsum, bcast);
+            aL = from_key(kk);
+        }
     }
     if (threadIdx.x == 0) {
         st->ladder_R[0] = aR;
@@ -158,6 +259,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
             st->a_L = aL;
             st->a_R = aR;
         }
+        bracket_key_range(st->a_L, st->a_R, &st->bin_kmin, &st->bin_kmax);
         st->sample_m = m;
         st->rank_l = (int32_t)lad.l[0];
         st->rank_h = (int32_t)lad.h[0];
@@ -193,59 +295,117 @@ __device__ __forceinline__ void fold_one(float x, float aL, float aR, float inv_
     }
 }
 
-// Warp-aggregated append of the lanes with `take` into band[] (capacity cap).
-__device__ __forceinline__ void band_append(bool take, float x, float* band,
-                                            unsigned long long* counter, unsigned long long cap) {
+// Adds one band score to the fixed-point band histogram (global atomics).
+__device__ __forceinline__ void bin_add(float x, const BinLayout& BL, float inv_t,
+                                        unsigned long long* bins) {
+    const int j = bin_of(BL, to_key(x));
+    const float lo = bin_edge(BL, j), hi = bin_edge(BL, j + 1);
+    atomicAdd(&bins[j], 1ull);
+    atomicAdd(&bins[kBins + j], __float2ull_rn(__expf((lo - x) * inv_t) * (float)kFixScale));
+    atomicAdd(&bins[2 * kBins + j], __float2ull_rn(__expf((x - hi) * inv_t) * (float)kFixScale));
+}
+
+constexpr int kStage = 2048;  // band scores staged per CTA before one global append
+
+// Warp-aggregated append of the lanes with `take` to the CTA's staging buffer;
+// lanes past its capacity go straight to the global band (rare).
+__device__ __forceinline__ void band_stage(bool take, float x, float* sband, int* scount,
+                                           float* band, unsigned long long* counter,
+                                           unsigned long long cap, const BinLayout& BL,
+                                           float inv_t, unsigned long long* bins) {
     const unsigned ball = __ballot_sync(0xffffffffu, take);
     if (ball == 0) return;
     const int lane = threadIdx.x & 31;
     const int leader = __ffs(ball) - 1;
-    unsigned long long base = 0;
-    if (lane == leader) base = atomicAdd(counter, (unsigned long long)__popc(ball));
+    int base = 0;
+    if (lane == leader) base = atomicAdd(scount, __popc(ball));
     base = __shfl_sync(0xffffffffu, base, leader);
     if (take) {
-        const unsigned long long pos = base + __popc(ball & ((1u << lane) - 1u));
-        if (pos < cap) band[pos] = x;
+        const int pos = base + __popc(ball & ((1u << lane) - 1u));
+        if (pos < kStage) {
+            sband[pos] = x;
+        } else {
+            const unsigned long long g = atomicAdd(counter, 1ull);
+            if (g < cap) band[g] = x;
+            bin_add(x, BL, inv_t, bins);
+        }
+    }
+}
+
+// Moves the staged band scores to the global band and histogram.
+__device__ __forceinline__ void band_flush(const float* sband, int scount, float* band,
+                                           unsigned long long* counter, unsigned long long cap,
+                                           const BinLayout& BL, float inv_t,
+                                           unsigned long long* bins,
+                                           unsigned long long* gbase_sh) {
+    const int ns = scount < kStage ? scount : kStage;
+    if (threadIdx.x == 0) *gbase_sh = ns > 0 ? atomicAdd(counter, (unsigned long long)ns) : 0ull;
+    __syncthreads();
+    const unsigned long long gb = *gbase_sh;
+    for (int i = threadIdx.x; i < ns; i += blockDim.x) {
+        const float x = sband[i];
+        if (gb + i < cap) band[gb + i] = x;
+        bin_add(x, BL, inv_t, bins);
     }
 }
 
 __global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restrict__ r, int64_t n,
                                                             double t, RowState* st,
                                                             float* __restrict__ band,
+                                                            unsigned long long* __restrict__ bins,
                                                             double* __restrict__ part,
                                                             uint32_t* __restrict__ ticket,
                                                             WsHeader* hdr, int vec) {
     __shared__ double red[kFoldThreads / 32];
     __shared__ long long lred[kFoldThreads / 32];
+    __shared__ float sband[kStage];
+    __shared__ int scount;
+    __shared__ unsigned long long gbase;
     __shared__ int flag;
     const float aL = st->a_L, aR = st->a_R;
+    const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
     const float inv_t = (float)(1.0 / t);
+    if (threadIdx.x == 0) scount = 0;
+    __syncthreads();
     FoldAcc acc{0ull, 0.0, 0.0, false};
     unsigned long long* counter = &st->n_band;
     const unsigned long long cap = (unsigned long long)n;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
     const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+#define LAPSUM_STAGE(take, x) \
+    band_stage(take, x, sband, &scount, band, counter, cap, BL, inv_t, bins)
     if (vec) {
         const int64_t n4 = n >> 2;
         const float4* r4 = reinterpret_cast<const float4*>(r);
-        // uniform trip count per warp so the ballots below see full warps
-        const int64_t iters = (n4 + nthreads - 1) / nthreads;
+        // Four independent 16-byte loads per thread per trip keep enough bytes
+        // in flight; the trip count is uniform so the ballots see full warps.
+        constexpr int U = 4;
+        const int64_t iters = (n4 + (int64_t)U * nthreads - 1) / ((int64_t)U * nthreads);
         for (int64_t it = 0; it < iters; ++it) {
-            const int64_t i = it * nthreads + gtid;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            const bool ok = i < n4;
-            if (ok) v = __ldcs(r4 + i);
-            bool b0 = false, b1 = false, b2 = false, b3 = false;
-            if (ok) {
-                fold_one(v.x, aL, aR, inv_t, acc, b0);
-                fold_one(v.y, aL, aR, inv_t, acc, b1);
-                fold_one(v.z, aL, aR, inv_t, acc, b2);
-                fold_one(v.w, aL, aR, inv_t, acc, b3);
+            float4 v[U];
+            bool ok[U];
+#pragma unroll
+            for (int q = 0; q < U; ++q) {
+                const int64_t i = (it * U + q) * nthreads + gtid;
+                ok[q] = i < n4;
+                v[q] = ok[q] ? __ldcs(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            band_append(b0, v.x, band, counter, cap);
-            band_append(b1, v.y, band, counter, cap);
-            band_append(b2, v.z, band, counter, cap);
-            band_append(b3, v.w, band, counter, cap);
+#pragma unroll
+            for (int q = 0; q < U; ++q) {
+                bool b0 = false, b1 = false, b2 = false, b3 = false;
+                if (ok[q]) {
+                    fold_one(v[q].x, aL, aR, inv_t, acc, b0);
+                    fold_one(v[q].y, aL, aR, inv_t, acc, b1);
+                    fold_one(v[q].z, aL, aR, inv_t, acc, b2);
+                    fold_one(v[q].w, aL, aR, inv_t, acc, b3);
+                }
+                if (__any_sync(0xffffffffu, b0 | b1 | b2 | b3)) {
+                    LAPSUM_STAGE(b0, v[q].x);
+                    LAPSUM_STAGE(b1, v[q].y);
+                    LAPSUM_STAGE(b2, v[q].z);
+                    LAPSUM_STAGE(b3, v[q].w);
+                }
+            }
         }
         // tail elements (n not a multiple of 4)
         const int64_t rem0 = n4 << 2;
@@ -257,7 +417,7 @@ __global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restr
                 x = r[i];
                 fold_one(x, aL, aR, inv_t, acc, bb);
             }
-            band_append(bb, x, band, counter, cap);
+            LAPSUM_STAGE(bb, x);
         }
     } else {
         const int64_t iters = (n + nthreads - 1) / nthreads;
@@ -269,9 +429,12 @@ __global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restr
                 x = r[i];
                 fold_one(x, aL, aR, inv_t, acc, bb);
             }
-            band_append(bb, x, band, counter, cap);
+            LAPSUM_STAGE(bb, x);
         }
     }
+#undef LAPSUM_STAGE
+    __syncthreads();
+    band_flush(sband, scount, band, counter, cap, BL, inv_t, bins, &gbase);
     const long long cR = block_sum_ll((long long)acc.cntR, lred);
     const double sL = block_sum_d(acc.SL, red);
     const double sR = block_sum_d(acc.SR, red);
@@ -314,6 +477,22 @@ __global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restr
     }
 }
 
+// Warp-aggregated append of the lanes with `take` into band[] (capacity cap).
+__device__ __forceinline__ void band_append(bool take, float x, float* band,
+                                            unsigned long long* counter, unsigned long long cap) {
+    const unsigned ball = __ballot_sync(0xffffffffu, take);
+    if (ball == 0) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(ball) - 1;
+    unsigned long long base = 0;
+    if (lane == leader) base = atomicAdd(counter, (unsigned long long)__popc(ball));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (take) {
+        const unsigned long long pos = base + __popc(ball & ((1u << lane) - 1u));
+        if (pos < cap) band[pos] = x;
+    }
+}
+
 // ----------------------------------------------------------------------------
 // 3-4. Exact band solve, certification, narrowing and widening (one CTA).
 // ----------------------------------------------------------------------------
@@ -329,6 +508,8 @@ struct ConstGet {
 struct SolveSmemAll {
     SolveScratch ss;
     SolveResult res;
+    Tails sub;          // tails of a histogram sub-bracket
+    double binF[2];     // F at the first and last histogram edge
     double red[32];
     float fred[32];
     long long lred[32];
@@ -345,7 +526,6 @@ struct SolveSmemAll {
             uint32_t cnt[kRefineBins];
             float U[kRefineBins];
             float L[kRefineBins];
-            double F[kRefineBins + 1];
         } hist;
         uint32_t sel_hist[2048];
     } u;
@@ -452,30 +632,41 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
         atomicAdd(&sm->u.hist.L[j], __expf((s - edge(j + 1)) * inv_t));
     }
     __syncthreads();
-    // F at every edge (one thread; nbin <= 2048, fp64).  Runs once per level.
-    if (threadIdx.x == 0) {
-        double Q = tl.hasR ? tl.SR * exp(((double)edge(nbin) - (double)tl.aR) / t) : 0.0;
-        double above = tl.cntR;
-        sm->u.hist.F[nbin] = 0.0;  // filled below with the forward part
-        // backward: store cnt_above - Q/2 at each edge
-        double* F = sm->u.hist.F;
-        F[nbin] = above - 0.5 * Q;
-        for (int j = nbin - 1; j >= 0; --j) {
-            const double gam = exp(((double)edge(j) - (double)edge(j + 1)) / t);
-            Q = (double)sm->u.hist.U[j] + Q * gam;
-            above += (double)sm->u.hist.cnt[j];
-            F[j] = above - 0.5 * Q;
-        }
-        double P = tl.hasL ? tl.SL * exp(((double)tl.aL - (double)edge(0)) / t) : 0.0;
-        F[0] += 0.5 * P;
-        for (int j = 1; j <= nbin; ++j) {
-            const double gam = exp(((double)edge(j - 1) - (double)edge(j)) / t);
-            P = (double)sm->u.hist.L[j - 1] + P * gam;
-            F[j] += 0.5 * P;
-        }
+    // F at every bin edge e_0..e_nbin from the bin aggregates, by two affine
+    // scans over the bins (thread i owns bins 2i and 2i+1; bins past nbin are
+    // empty and their edges coincide, so their maps are the identity).
+    //   Q_j = U_j + g_j Q_{j+1}, Q_nbin = SR e^{(e_nbin - aR)/t}    (weights above e_j)
+    //   P_j = L_{j-1} + g_{j-1} P_{j-1}, P_0 = SL e^{(aL - e_0)/t}  (weights below e_j)
+    //   F(e_j) = cntR + #{scores in bins >= j} - Q_j/2 + P_j/2,   g_j = e^{(e_j - e_{j+1})/t}
+    {
+        const int b0 = 2 * threadIdx.x, b1 = b0 + 1;
+        const double e0 = (double)edge(b0), e1 = (double)edge(b1), e2 = (double)edge(b1 + 1);
+        const double g0 = exp((e0 - e1) / t), g1 = exp((e1 - e2) / t);
+        const double U0 = sm->u.hist.U[b0], U1 = sm->u.hist.U[b1];
+        const double L0 = sm->u.hist.L[b0], L1 = sm->u.hist.L[b1];
+        const long long c01 = (long long)sm->u.hist.cnt[b0] + (long long)sm->u.hist.cnt[b1];
+        const Aff mb = aff_then(Aff{g1, U1}, Aff{g0, U0});      // apply bin b1, then b0
+        const Aff mf = aff_then(Aff{g0, L0}, Aff{g1, L1});      // edge b0+1, then b0+2
+        const Aff eb = block_excl_scan_bwd(mb, sm->ss.wb);
+        const Aff ef = block_excl_scan_fwd(mf, sm->ss.wf);
+        const long long above = block_excl_suffix_ll(c01, sm->lred);
+        const double Qend = tl.hasR ? tl.SR * exp(((double)edge(kRefineBins) - (double)tl.aR) / t) : 0.0;
+        const double Pstart = tl.hasL ? tl.SL * exp(((double)tl.aL - (double)edge(0)) / t) : 0.0;
+        const double Q2 = fma(eb.a, Qend, eb.c);                // Q at edge b0+2
+        const double Q1 = fma(g1, Q2, U1);
+        const double Q0 = fma(g0, Q1, U0);
+        const double P0 = fma(ef.a, Pstart, ef.c);              // P at edge b0
+        const double P1 = fma(g0, P0, L0);
+        const double F0 = tl.cntR + (double)(above + c01) - 0.5 * Q0 + 0.5 * P0;
+        const double F1 = tl.cntR + (double)(above + (long long)sm->u.hist.cnt[b1]) - 0.5 * Q1 +
+                          0.5 * P1;
         int c = 0;
-        for (int j = 0; j <= nbin; ++j) c += (F[j] >= k) ? 1 : 0;
-        sm->bcast[0] = (uint32_t)(c - 1);  // edge index of the new lower end (-1: use aL)
+        if (b0 <= nbin && F0 >= k) ++c;
+        if (b1 <= nbin && F1 >= k) ++c;
+        // Edge e_2048 itself is not evaluated; when b lies above every edge
+        // evaluated here, the exact check below moves the bracket up to it.
+        const int tot = __syncthreads_count(c >= 1) + __syncthreads_count(c >= 2);
+        if (threadIdx.x == 0) sm->bcast[0] = (uint32_t)(tot - 1);
     }
     __syncthreads();
     int jc = (int)sm->bcast[0];
@@ -563,6 +754,141 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
     return -1;  // unreachable for a certified input band
 }
 
+// F at every edge of the fold's band histogram, by two affine scans over the
+// bins (thread i owns bins 2i and 2i+1; bins past nbin are empty with equal
+// edges, so their maps are the identity):
+//   Q_j = U_j + g_j Q_{j+1}   (weights of scores >= e_j),  Q at the top edge = S_R
+//   P_j = L_{j-1} + g_{j-1} P_{j-1}  (weights of scores < e_j),  P_0 = S_L
+//   F(e_j) = #{scores >= e_j} - Q_j/2 + P_j/2,   g_j = e^{(e_j - e_{j+1})/t}.
+// Returns #{edges 0..nbin with F >= k}; F at edge 0 and edge nbin go to
+// sm->binF.  With want >= 0 the tails of the sub-bracket [e_want, e_want+1)
+// go to sm->sub.  Every thread of the (1024-thread) block must call it.
+__device__ int bin_scan(const BinLayout& BL, const unsigned long long* __restrict__ bins,
+                        const Tails& tl, double k, double t, SolveSmemAll* sm, int want) {
+    const int b0 = 2 * threadIdx.x, b1 = b0 + 1;
+    const double e0 = (double)bin_edge(BL, b0), e1 = (double)bin_edge(BL, b1);
+    const double e2 = (double)bin_edge(BL, b1 + 1);
+    const double g0 = (e1 > e0) ? exp((e0 - e1) / t) : 1.0;
+    const double g1 = (e2 > e1) ? exp((e1 - e2) / t) : 1.0;
+    const long long c0 = (long long)bins[b0], c1 = (long long)bins[b1];
+    const double U0 = (double)bins[kBins + b0] / kFixScale, U1 = (double)bins[kBins + b1] / kFixScale;
+    const double L0 = (double)bins[2 * kBins + b0] / kFixScale;
+    const double L1 = (double)bins[2 * kBins + b1] / kFixScale;
+    const Aff mb = aff_then(Aff{g1, U1}, Aff{g0, U0});  // bin b1 first, then b0
+    const Aff mf = aff_then(Aff{g0, L0}, Aff{g1, L1});  // edge b0+1, then b0+2
+    const Aff eb = block_excl_scan_bwd(mb, sm->ss.wb);
+    const Aff ef = block_excl_scan_fwd(mf, sm->ss.wf);
+    const long long above = block_excl_suffix_ll(c0 + c1, sm->lred);
+    const double etop = (double)bin_edge(BL, kBins), efirst = (double)bin_edge(BL, 0);
+    const double Qend = (tl.hasR && tl.SR > 0.0) ? tl.SR * exp((etop - (double)tl.aR) / t) : 0.0;
+    const double Pst = (tl.hasL && tl.SL > 0.0) ? tl.SL * exp(((double)tl.aL - efirst) / t) : 0.0;
+    const double Q2 = fma(eb.a, Qend, eb.c), Q1 = fma(g1, Q2, U1), Q0 = fma(g0, Q1, U0);
+    const double P0 = fma(ef.a, Pst, ef.c), P1 = fma(g0, P0, L0), P2 = fma(g1, P1, L1);
+    const double A2 = tl.cntR + (double)above, A1 = A2 + (double)c1, A0 = A1 + (double)c0;
+    const double F0 = A0 - 0.5 * Q0 + 0.5 * P0, F1 = A1 - 0.5 * Q1 + 0.5 * P1;
+    const double F2 = A2 - 0.5 * Q2 + 0.5 * P2;
+    const int nb = BL.nbin;
+    int c = 0;
+    if (b0 <= nb && F0 >= k) ++c;
+    if (b1 <= nb && F1 >= k) ++c;
+    if (b1 + 1 == kBins && kBins <= nb && F2 >= k) ++c;
+    if (b0 == 0) sm->binF[0] = F0;
+    if (b0 == nb) sm->binF[1] = F0;
+    if (b1 == nb) sm->binF[1] = F1;
+    if (b1 + 1 == nb) sm->binF[1] = F2;
+    if (want >= 0) {
+        // lower end e_want: weights below it; upper end e_want+1: weights and count above it
+        if (b0 == want) sm->sub.SL = P0;
+        if (b1 == want) sm->sub.SL = P1;
+        if (b0 == want + 1) { sm->sub.SR = Q0; sm->sub.cntR = A0; }
+        if (b1 == want + 1) { sm->sub.SR = Q1; sm->sub.cntR = A1; }
+        if (b1 + 1 == want + 1) { sm->sub.SR = Q2; sm->sub.cntR = A2; }
+        if (threadIdx.x == 0) {
+            sm->sub.hasL = true;
+            sm->sub.aL = bin_edge(BL, want);
+            const float hi = bin_edge(BL, want + 1);
+            sm->sub.hasR = isfinite(hi);
+            sm->sub.aR = hi;
+        }
+    }
+    const int tot = __syncthreads_count(c >= 1) + __syncthreads_count(c >= 2) +
+                    __syncthreads_count(c >= 3);
+    return tot;
+}
+
+// Copies the band scores that fall in histogram bin `j` into sm->u.sort.sorted
+// (at most kBandSortMax of them); returns how many there were.
+__device__ long long extract_bin(const float* __restrict__ band, long long nb, const BinLayout& BL,
+                                 int j, SolveSmemAll* sm) {
+    if (threadIdx.x == 0) sm->cnt = 0ull;
+    __syncthreads();
+    const long long n4 = nb >> 2;
+    const float4* b4 = reinterpret_cast<const float4*>(band);
+    for (long long i = threadIdx.x; i < n4; i += blockDim.x) {
+        const float4 v = b4[i];
+        const float xs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (bin_of(BL, to_key(xs[q])) == j) {
+                const unsigned long long pos = atomicAdd(&sm->cnt, 1ull);
+                if (pos < (unsigned long long)kBandSortMax) sm->u.sort.sorted[pos] = xs[q];
+            }
+        }
+    }
+    for (long long i = (n4 << 2) + threadIdx.x; i < nb; i += blockDim.x) {
+        const float x = band[i];
+        if (bin_of(BL, to_key(x)) == j) {
+            const unsigned long long pos = atomicAdd(&sm->cnt, 1ull);
+            if (pos < (unsigned long long)kBandSortMax) sm->u.sort.sorted[pos] = x;
+        }
+    }
+    __syncthreads();
+    return (long long)sm->cnt;
+}
+
+// Solve through the fold's histogram: certify the bracket from the bin sums,
+// pick the bin whose edges straddle k, and solve exactly on that bin's scores
+// with the other bins folded into its tails.  A bin picked wrongly by the
+// fixed-point rounding fails its own end check and the neighbour is tried.
+// Returns 1 (solved, b in sm->res), 0 (bracket failed: F at the ends in
+// sm->res), or -1 (the bin is too full for the on-chip sort: use the exact
+// narrowing path).
+__device__ int solve_with_bins(const float* __restrict__ band, long long nb,
+                               const unsigned long long* __restrict__ bins, const BinLayout& BL,
+                               const Tails& tl, double k, double t, SolveSmemAll* sm) {
+    const int cntF = bin_scan(BL, bins, tl, k, t, sm, -1);
+    const double FL = tl.hasL ? sm->binF[0] : INFINITY;
+    const double FR = tl.hasR ? sm->binF[1] : -INFINITY;
+    if (!(FL >= k && FR <= k)) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            sm->res.F_aL = FL;
+            sm->res.F_aR = FR;
+        }
+        __syncthreads();
+        return 0;
+    }
+    int jc = cntF - 1;
+    if (jc < 0) jc = 0;
+    if (jc > BL.nbin - 1) jc = BL.nbin - 1;
+    for (int guard = 0; guard < 8; ++guard) {
+        __syncthreads();
+        bin_scan(BL, bins, tl, k, t, sm, jc);
+        if ((long long)bins[jc] > kBandSortMax) return -1;
+        const long long c = extract_bin(band, nb, BL, jc, sm);
+        Tails sub = sm->sub;
+        solve_small_band(sm->u.sort.sorted, c, sub, k, t, sm);
+        if (sm->res.F_aL < k && jc > 0) {
+            --jc;
+        } else if (sm->res.F_aR > k && jc < BL.nbin - 1) {
+            ++jc;
+        } else {
+            return 1;
+        }
+    }
+    return -1;
+}
+
 // Single-CTA fold of the whole row (used only after a failed bracket).
 __device__ void refold_row(const float* __restrict__ r, int64_t n, float aL, float aR, double t,
                            float* band, SolveSmemAll* sm, Tails& tl, long long* nb) {
@@ -599,6 +925,7 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
                                                      double k, double t, RowState* st,
                                                      float* __restrict__ band0,
                                                      float* __restrict__ band1,
+                                                     const unsigned long long* __restrict__ bins,
                                                      const float* __restrict__ sample, int m,
                                                      Ladder lad, double* __restrict__ b_out,
                                                      WsHeader* hdr) {
@@ -639,7 +966,22 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
         bool certified;
         cert = tl;
         nb_cert = nb;
-        if (nb <= kBandSortMax) {
+        int via_bins = -1;
+        if (nb > kBandSortMax && attempt == 1) {
+            // the fold built the band histogram for this first bracket
+            const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
+            via_bins = solve_with_bins(cur, nb, bins, BL, tl, k, t, sm);
+            if (via_bins == 1) {
+                b = sm->res.b;
+                done = true;
+                certified = true;
+            } else if (via_bins == 0) {
+                certified = false;
+            }
+        }
+        if (via_bins >= 0) {
+            // handled through the histogram
+        } else if (nb <= kBandSortMax) {
             solve_small_band(cur, nb, tl, k, t, sm);
             certified = sm->res.F_aL >= k && sm->res.F_aR <= k;
             if (certified) {
@@ -751,12 +1093,12 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                                RowState* st_row, double* b_out, WsHeader* hdr, cudaStream_t st) {
     static bool attr_done = false;
     const size_t solve_smem = sizeof(SolveSmemAll);
-    const size_t sample_smem = (size_t)m * sizeof(uint32_t);
+    const size_t sample_smem = ((size_t)m + 2 * kBandSortMax) * sizeof(uint32_t);
     if (!attr_done) {
         cudaFuncSetAttribute(solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)solve_smem);
         cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(kSampleMax * sizeof(uint32_t)));
+                             (int)((kSampleMax + 2 * kBandSortMax) * sizeof(uint32_t)));
         attr_done = true;
     }
     Ladder lad;
@@ -771,18 +1113,19 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     {
         ProfScope ps_("bracket_sample", st);
         sample_kernel<<<1, kBlk, sample_smem, st>>>(r_row, n, t, seed, c0, m, lad, force_miss,
-                                                max_attempts, sample, st_row);
+                                                max_attempts, sample, buf.bins, st_row);
     }
     const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
     {
         ProfScope ps_("bracket_fold", st);
         fold_kernel<<<buf.fold_grid, kFoldThreads, 0, st>>>(r_row, n, t, st_row, buf.band[0],
-                                                        buf.fold_part, buf.ticket, hdr, vec);
+                                                        buf.bins, buf.fold_part, buf.ticket, hdr,
+                                                        vec);
     }
     {
         ProfScope ps_("bracket_solve", st);
         solve_kernel<<<1, kBlk, solve_smem, st>>>(r_row, n, k, t, st_row, buf.band[0], buf.band[1],
-                                              sample, m, lad, b_out, hdr);
+                                              buf.bins, sample, m, lad, b_out, hdr);
     }
     return cudaGetLastError();
 }

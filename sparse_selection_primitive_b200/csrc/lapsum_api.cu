@@ -42,7 +42,7 @@ int resolve_path(int64_t n, int path) {
 struct Layout {
     size_t header, rows, partials, row_R, tickets;
     size_t keys0, keys1, seg_hist, tile_hist, plan;
-    size_t sample, band0, band1, fold_part, fold_ticket;
+    size_t sample, band0, band1, bins, fold_part, fold_ticket;
     size_t total;
 };
 
@@ -73,6 +73,7 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
         L.sample = take((size_t)B * kSampleMax * sizeof(float));
         L.band0 = take((size_t)n * sizeof(float));
         L.band1 = take((size_t)n * sizeof(float));
+        L.bins = take((size_t)3 * kBins * sizeof(unsigned long long));
         L.fold_part = take((size_t)kFoldGridMax * 4 * sizeof(double));
     }
     L.total = off;
@@ -85,11 +86,29 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? LAPSUM_OK : LAPSUM_EC
 
 // Binomial(m, q) order-statistic ranks (descending, 1-based) for one bracket:
 // l = largest with P(C < l) <= alpha, h = smallest with P(C >= h) <= alpha.
+// The upper tail is accumulated downward from mq + 40 sd + 64, past which every
+// probability is below 1e-300; results are cached per (m, q, alpha).
 void binomial_ranks(int64_t m, double q, double alpha, int64_t* l, int64_t* h) {
+    struct Entry {
+        int64_t m;
+        double q, alpha;
+        int64_t l, h;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        for (const Entry& e : cache)
+            if (e.m == m && e.q == q && e.alpha == alpha) {
+                *l = e.l;
+                *h = e.h;
+                return;
+            }
+    }
+    const double lgm = std::lgamma((double)m + 1.0), lq = std::log(q), l1q = std::log1p(-q);
     auto logpmf = [&](int64_t c) {
-        return std::lgamma((double)m + 1.0) - std::lgamma((double)c + 1.0) -
-               std::lgamma((double)(m - c) + 1.0) + (double)c * std::log(q) +
-               (double)(m - c) * std::log1p(-q);
+        return lgm - std::lgamma((double)c + 1.0) - std::lgamma((double)(m - c) + 1.0) +
+               (double)c * lq + (double)(m - c) * l1q;
     };
     double cdf = 0.0;
     int64_t lo = 0;
@@ -98,15 +117,20 @@ void binomial_ranks(int64_t m, double q, double alpha, int64_t* l, int64_t* h) {
         if (cdf <= alpha) lo = c + 1;
         else break;
     }
+    const double mean = (double)m * q, sd = std::sqrt((double)m * q * (1.0 - q));
+    int64_t top = (int64_t)std::ceil(mean + 40.0 * sd + 64.0);
+    if (top > m) top = m;
     double sf = 0.0;
-    int64_t hi = m + 1;
-    for (int64_t c = m; c >= 0; --c) {
+    int64_t hi = top + 1 <= m ? top + 1 : m + 1;
+    for (int64_t c = top; c >= 0; --c) {
         sf += std::exp(logpmf(c));
         if (sf <= alpha) hi = c;
         else break;
     }
     *l = lo;
     *h = hi;
+    std::lock_guard<std::mutex> g(mu);
+    if (cache.size() < 64) cache.push_back(Entry{m, q, alpha, lo, hi});
 }
 
 int sample_size(int64_t n, double k) {
@@ -264,6 +288,7 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
         bb.sample = reinterpret_cast<float*>(w + L.sample);
         bb.band[0] = reinterpret_cast<float*>(w + L.band0);
         bb.band[1] = reinterpret_cast<float*>(w + L.band1);
+        bb.bins = reinterpret_cast<unsigned long long*>(w + L.bins);
         bb.fold_part = reinterpret_cast<double*>(w + L.fold_part);
         bb.ticket = reinterpret_cast<uint32_t*>(w + L.fold_ticket);
         bb.fold_grid = bracket_fold_grid();

@@ -62,7 +62,8 @@ struct RowState {
     int32_t max_attempts;
     float ladder_L[kLadder];  // a_L rungs (descending ranks h, 4h, 16h, open)
     float ladder_R[kLadder];  // a_R rungs (ranks l, l/4, l/16, open)
-    double scratch[40];       // kernel-to-kernel scalars
+    uint32_t bin_kmin, bin_kmax;  // key range of the band histogram of the current bracket
+    double scratch[39];       // kernel-to-kernel scalars
 };
 static_assert(sizeof(RowState) <= 512, "row record fits its slot");
 
@@ -104,6 +105,15 @@ __device__ __forceinline__ float scaled_margin(float r, const Thr& h) {
 __device__ __forceinline__ float neg_abs_exp(float x) { return __expf(-fabsf(x)); }
 __device__ __forceinline__ float cdf_from(float x, float e) { return x < 0.f ? 0.5f * e : 1.f - 0.5f * e; }
 
+// Gap factor e^{(lo - hi)/t} between two neighbouring sorted scores lo <= hi.
+// The difference of two fp32 values is exact in fp64 and the exponential is
+// taken in fp64: the scans chain these factors over up to n positions, and an
+// fp32 factor's rounding would build up along the chain whenever t is large
+// compared with the gaps (weights that barely decay).
+__device__ __forceinline__ double gap_factor(float lo, float hi, double inv_t) {
+    return exp(((double)lo - (double)hi) * inv_t);
+}
+
 // ---------------------------------------------------------------------------
 // Affine maps x -> a x + c, the element of the stable prefix/suffix scans.
 // The prefix sum P_j = sum_{i<=j} e^{(s_i - s_j)/t} obeys P_j = 1 + g_j P_{j-1}
@@ -144,6 +154,51 @@ __device__ __forceinline__ Aff warp_scan_bwd(Aff v, int lane) {
         if (lane + d < 32) v = aff_then(o, v);
     }
     return v;
+}
+
+// Block-wide exclusive scans of affine maps (every thread calls; `wt` holds
+// blockDim.x/32 maps of shared memory).  Forward: composition of the maps of
+// all lower threads (thread 0 applied first).  Backward: of all higher
+// threads (the last thread applied first).
+__device__ inline Aff block_excl_scan_fwd(const Aff& v, Aff* wt) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const Aff inc = warp_scan_fwd(v, lane);
+    Aff ex = shfl_up_aff(inc, 1);
+    if (lane == 0) ex = aff_id();
+    __syncthreads();
+    if (lane == 31) wt[w] = inc;
+    __syncthreads();
+    Aff pre = aff_id();
+    for (int u = 0; u < w; ++u) pre = aff_then(pre, wt[u]);
+    return aff_then(pre, ex);
+}
+__device__ inline Aff block_excl_scan_bwd(const Aff& v, Aff* wt) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const Aff inc = warp_scan_bwd(v, lane);
+    Aff ex = shfl_down_aff(inc, 1);
+    if (lane == 31) ex = aff_id();
+    __syncthreads();
+    if (lane == 0) wt[w] = inc;
+    __syncthreads();
+    Aff suf = aff_id();
+    for (int u = nw - 1; u > w; --u) suf = aff_then(suf, wt[u]);
+    return aff_then(suf, ex);
+}
+// Block-wide exclusive suffix sum of a count (sum over higher threads).
+__device__ inline long long block_excl_suffix_ll(long long v, long long* wt) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    long long inc = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const long long o = __shfl_down_sync(0xffffffffu, inc, d);
+        if (lane + d < 32) inc += o;
+    }
+    __syncthreads();
+    if (lane == 0) wt[w] = inc;
+    __syncthreads();
+    long long s = inc - v;
+    for (int u = w + 1; u < nw; ++u) s += wt[u];
+    return s;
 }
 
 // ---------------------------------------------------------------------------
@@ -193,6 +248,51 @@ __device__ inline double segment_root(bool hasL, double sL, double Bh, bool hasR
         if (b > sR) b = sR;
     }
     return b;
+}
+
+// ---------------------------------------------------------------------------
+// Band histogram layout: the key range [kmin, kmax] of a bracket [a_L, a_R)
+// split into nbin <= 2048 bins of 2^sh consecutive keys.  Edge j is the float
+// with key kmin + j 2^sh (the last edge is kmax + 1, the key of a_R), so bin j
+// holds the scores e_j <= s < e_{j+1}.  Per-bin sums are kept in fixed point
+// (2^-32 units, every term is at most 1) so that atomic accumulation in any
+// order gives the same bits.
+// ---------------------------------------------------------------------------
+constexpr int kBins = 2048;
+constexpr double kFixScale = 4294967296.0;  // 2^32
+
+struct BinLayout {
+    uint32_t kmin, kmax;
+    int sh, nbin;
+};
+__device__ __forceinline__ BinLayout make_bins(uint32_t kmin, uint32_t kmax) {
+    BinLayout B;
+    B.kmin = kmin;
+    B.kmax = kmax < kmin ? kmin : kmax;
+    B.sh = 0;
+    while (((B.kmax - B.kmin) >> B.sh) >= (uint32_t)kBins) ++B.sh;
+    B.nbin = (int)((B.kmax - B.kmin) >> B.sh) + 1;
+    return B;
+}
+__device__ __forceinline__ uint32_t bin_edge_key(const BinLayout& B, int j) {
+    const unsigned long long e = (unsigned long long)B.kmin + ((unsigned long long)j << B.sh);
+    const unsigned long long top = (unsigned long long)B.kmax + 1ull;
+    const unsigned long long v = e < top ? e : top;
+    return v > 0xffffffffull ? 0xffffffffu : (uint32_t)v;
+}
+__device__ __forceinline__ float bin_edge(const BinLayout& B, int j) {
+    return from_key(bin_edge_key(B, j));
+}
+__device__ __forceinline__ int bin_of(const BinLayout& B, uint32_t key) {
+    if (key <= B.kmin) return 0;
+    const uint32_t j = (key - B.kmin) >> B.sh;
+    return j >= (uint32_t)B.nbin ? B.nbin - 1 : (int)j;
+}
+// Key range of the histogram of bracket [aL, aR) (open ends: the finite range).
+__device__ __forceinline__ void bracket_key_range(float aL, float aR, uint32_t* kmin,
+                                                  uint32_t* kmax) {
+    *kmin = (aL >= -3.402823466e38f) ? to_key(aL) : 0x00800000u;  // key of -FLT_MAX
+    *kmax = (aR <= 3.402823466e38f) ? to_key(aR) - 1u : 0xff7fffffu;  // key of +FLT_MAX
 }
 
 // ---------------------------------------------------------------------------

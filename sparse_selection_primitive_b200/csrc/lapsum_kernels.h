@@ -60,6 +60,7 @@ constexpr int kSampleMax = 32768;
 struct BracketBuffers {
     float* sample;       // [B][m]
     float* band[2];      // capacity n each
+    unsigned long long* bins;  // band histogram of the first bracket: [3][2048]
     double* fold_part;   // fold partials, one record per CTA
     uint32_t* ticket;    // last-block counter
     int fold_grid;

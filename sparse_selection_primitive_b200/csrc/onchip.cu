@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(CTA) onchip_forward_kernel(
     using S = Shape<E, RT, CTA>;
     __shared__ uint32_t xch[(RT > 32) ? CTA * E : 1];
     __shared__ uint32_t last_key[CTA];
-    __shared__ float first_gap[CTA];
+    __shared__ double first_gap[CTA];
     __shared__ Aff wf[S::NW], wb[S::NW];
     __shared__ int ired[S::NW];
     __shared__ double dred[S::NW];
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(CTA) onchip_forward_kernel(
     const int64_t row = (int64_t)blockIdx.x * S::ROWS + rloc;
     const bool row_ok = row < B;
     const float* rrow = r + (row_ok ? row : 0) * ld;
-    const float inv_t = (float)(1.0 / t);
+    const double inv_t = 1.0 / t;
 
     if (threadIdx.x < S::ROWS) row_flag[threadIdx.x] = 0;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -180,7 +180,8 @@ __global__ void __launch_bounds__(CTA) onchip_forward_kernel(
     bitonic_sort_row<E, RT, CTA>(key, tid, xch);
 
     // Sorted values and gap factors g_j = exp((s_{j-1} - s_j)/t), 0 at j = 0 and past n.
-    float s[E], g[E];
+    float s[E];
+    double g[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) s[e] = from_key(key[e]);
     last_key[threadIdx.x] = key[E - 1];
@@ -190,25 +191,25 @@ __global__ void __launch_bounds__(CTA) onchip_forward_kernel(
     for (int e = 0; e < E; ++e) {
         const int j = tid * E + e;
         const float sp = (e == 0) ? s_prev : s[e - 1];
-        g[e] = (j >= 1 && j < n) ? __expf((sp - s[e]) * inv_t) : 0.f;
+        g[e] = (j >= 1 && j < n) ? gap_factor(sp, s[e], inv_t) : 0.0;
     }
     first_gap[threadIdx.x] = g[0];
     __syncthreads();
-    const float g_next = (tid + 1 < RT) ? first_gap[threadIdx.x + 1] : 0.f;
+    const double g_next = (tid + 1 < RT) ? first_gap[threadIdx.x + 1] : 0.0;
 
     // Thread aggregates of the forward (prefix) and backward (suffix) maps.
     Aff af = aff_id(), ab = aff_id();
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int j = tid * E + e;
-        const Aff m = (j < n) ? Aff{(double)g[e], 1.0} : aff_id();
+        const Aff m = (j < n) ? Aff{g[e], 1.0} : aff_id();
         af = aff_then(af, m);
     }
 #pragma unroll
     for (int e = E - 1; e >= 0; --e) {
         const int j = tid * E + e;
-        const float gn = (e + 1 < E) ? g[e + 1] : g_next;
-        const Aff m = (j < n) ? Aff{(double)gn, 1.0} : Aff{0.0, 0.0};
+        const double gn = (e + 1 < E) ? g[e + 1] : g_next;
+        const Aff m = (j < n) ? Aff{gn, 1.0} : Aff{0.0, 0.0};
         ab = aff_then(ab, m);
     }
     // Exclusive prefix (maps of earlier threads) and suffix (later threads).
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(CTA) onchip_forward_kernel(
     double x = ex_f.c;  // P just before this thread's first element
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-        x = fma((double)g[e], x, 1.0);
+        x = fma(g[e], x, 1.0);
         P[e] = x;
     }
     double y = ex_b.c;  // Q just after this thread's last element
@@ -244,8 +245,8 @@ __global__ void __launch_bounds__(CTA) onchip_forward_kernel(
 #pragma unroll
     for (int e = E - 1; e >= 0; --e) {
         const int j = tid * E + e;
-        const float gn = (e + 1 < E) ? g[e + 1] : g_next;
-        y = (j < n) ? fma((double)gn, y, 1.0) : 0.0;
+        const double gn = (e + 1 < E) ? g[e + 1] : g_next;
+        y = (j < n) ? fma(gn, y, 1.0) : 0.0;
         Q[e] = y;
         const double G = (double)(n - j) - 0.5 * Q[e] + 0.5 * (P[e] - 1.0);
         cnt += (j < n && G >= k) ? 1 : 0;

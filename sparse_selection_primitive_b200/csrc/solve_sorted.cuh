@@ -49,12 +49,12 @@ struct GapFn {
     Get get;
     long long nb;
     Tails tl;
-    float inv_t;
+    double inv_t;
     // factor between positions j-1 and j (anchors at -1 and nb)
-    __device__ __forceinline__ float operator()(long long j) const {
-        if (j <= 0) return (j == 0 && tl.hasL && nb > 0) ? __expf((tl.aL - get(0)) * inv_t) : 0.f;
-        if (j >= nb) return (j == nb && tl.hasR) ? __expf((get(nb - 1) - tl.aR) * inv_t) : 0.f;
-        return __expf((get(j - 1) - get(j)) * inv_t);
+    __device__ __forceinline__ double operator()(long long j) const {
+        if (j <= 0) return (j == 0 && tl.hasL && nb > 0) ? gap_factor(tl.aL, get(0), inv_t) : 0.0;
+        if (j >= nb) return (j == nb && tl.hasR) ? gap_factor(get(nb - 1), tl.aR, inv_t) : 0.0;
+        return gap_factor(get(j - 1), get(j), inv_t);
     }
 };
 
@@ -72,21 +72,21 @@ __device__ void warp_find_crossing(const GapFn<Get>& gap, long long lo, long lon
         const long long sc = (hi - lo + 31) / 32;
         const long long l0 = min(hi, lo + lane * sc), l1 = min(hi, l0 + sc);
         Aff af = aff_id(), ab = aff_id();
-        float g_first = 0.f;
+        double g_first = 0.0;
         for (long long j = l0; j < l1; ++j) {
-            const float gj = gap(j);
+            const double gj = gap(j);
             if (j == l0) g_first = gj;
-            af = aff_then(af, Aff{(double)gj, 1.0});
-            if (j > l0) ab = aff_then(Aff{(double)gj, 1.0}, ab);
+            af = aff_then(af, Aff{gj, 1.0});
+            if (j > l0) ab = aff_then(Aff{gj, 1.0}, ab);
         }
-        if (l1 > l0) ab = aff_then(Aff{(double)gap(l1), 1.0}, ab);
+        if (l1 > l0) ab = aff_then(Aff{gap(l1), 1.0}, ab);
         Aff ef = shfl_up_aff(warp_scan_fwd(af, lane), 1);
         Aff eb = shfl_down_aff(warp_scan_bwd(ab, lane), 1);
         if (lane == 0) ef = aff_id();
         if (lane == 31) eb = aff_id();
         const double pb = fma(ef.a, P_before, ef.c);   // P_{l0-1}
         const double qa = fma(eb.a, Q_after, eb.c);    // Q_{l1}
-        const double P0 = fma((double)g_first, pb, 1.0);
+        const double P0 = fma(g_first, pb, 1.0);
         const double Q0 = fma(ab.a, qa, ab.c);
         const double G0 = cntR + (double)(nb - l0) - 0.5 * Q0 + 0.5 * (P0 - 1.0);
         const unsigned ball = __ballot_sync(0xffffffffu, l0 < l1 && G0 >= k);
@@ -99,10 +99,10 @@ __device__ void warp_find_crossing(const GapFn<Get>& gap, long long lo, long lon
     // At most 32 elements: one per lane.
     const long long j = lo + lane;
     const bool valid = j < hi;
-    const float gj = valid ? gap(j) : 1.f;
-    const float gn = valid ? gap(j + 1) : 1.f;
-    const Aff mf = valid ? Aff{(double)gj, 1.0} : aff_id();
-    const Aff mb = valid ? Aff{(double)gn, 1.0} : aff_id();
+    const double gj = valid ? gap(j) : 1.0;
+    const double gn = valid ? gap(j + 1) : 1.0;
+    const Aff mf = valid ? Aff{gj, 1.0} : aff_id();
+    const Aff mb = valid ? Aff{gn, 1.0} : aff_id();
     const Aff inf_ = warp_scan_fwd(mf, lane);
     const Aff inb = warp_scan_bwd(mb, lane);
     const double Pj = fma(inf_.a, P_before, inf_.c);
@@ -126,7 +126,7 @@ template <class Get>
 __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, double k, double t,
                                    SolveScratch* sm, SolveResult* out) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    GapFn<Get> gap{get, nb, tl, (float)(1.0 / t)};
+    GapFn<Get> gap{get, nb, tl, 1.0 / t};
     const double P_start = tl.hasL ? tl.SL : 0.0;
     const double Q_end = tl.hasR ? tl.SR : 0.0;
 
@@ -146,22 +146,22 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
     const long long lo = min(nb, (long long)tid * chunk), hi = min(nb, lo + chunk);
     const bool valid = lo < hi;
     Aff af = aff_id(), ab = aff_id();
-    float g_first = 0.f;
+    double g_first = 0.0;
     for (long long j = lo; j < hi; ++j) {
-        const float gj = gap(j);
+        const double gj = gap(j);
         if (j == lo) g_first = gj;
-        af = aff_then(af, Aff{(double)gj, 1.0});
-        if (j > lo) ab = aff_then(Aff{(double)gj, 1.0}, ab);
+        af = aff_then(af, Aff{gj, 1.0});
+        if (j > lo) ab = aff_then(Aff{gj, 1.0}, ab);
     }
-    if (valid) ab = aff_then(Aff{(double)gap(hi), 1.0}, ab);
+    if (valid) ab = aff_then(Aff{gap(hi), 1.0}, ab);
 
-    Aff ef = shfl_up_aff(warp_scan_fwd(af, lane), 1);
-    Aff inc_b = warp_scan_bwd(ab, lane);
-    Aff inc_f_last = warp_scan_fwd(af, lane);
+    const Aff inc_f = warp_scan_fwd(af, lane);
+    const Aff inc_b = warp_scan_bwd(ab, lane);
+    Aff ef = shfl_up_aff(inc_f, 1);
     Aff eb = shfl_down_aff(inc_b, 1);
     if (lane == 0) ef = aff_id();
     if (lane == 31) eb = aff_id();
-    if (lane == 31) sm->wf[warp] = inc_f_last;
+    if (lane == 31) sm->wf[warp] = inc_f;
     if (lane == 0) sm->wb[warp] = inc_b;
     __syncthreads();
     {
@@ -174,7 +174,7 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
     }
     const double P_before = fma(ef.a, P_start, ef.c);  // P_{lo-1}
     const double Q_after = fma(eb.a, Q_end, eb.c);     // Q_hi
-    const double P_lo = fma((double)g_first, P_before, 1.0);
+    const double P_lo = fma(g_first, P_before, 1.0);
     const double Q_lo = fma(ab.a, Q_after, ab.c);
     const double G_lo = tl.cntR + (double)(nb - lo) - 0.5 * Q_lo + 0.5 * (P_lo - 1.0);
     const double P_end = fma(af.a, P_before, af.c);    // P_{hi-1}
@@ -219,9 +219,9 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
         out->b = b;
         out->jstar = js;
         const double Q0 = sm->d[0], Pl = sm->d[1];
-        out->F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * (double)gap(0) * Q0 + 0.5 * tl.SL
+        out->F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * gap(0) * Q0 + 0.5 * tl.SL
                             : INFINITY;
-        out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * (double)gap(nb) * Pl : -INFINITY;
+        out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * gap(nb) * Pl : -INFINITY;
     }
     __syncthreads();
 }

@@ -132,8 +132,23 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
     }
 }
 
-// Pass 1 of the VJP: per tile (mu, sum w, sum w v) with w = exp(-(|x| - mu));
-// the last CTA of the row rescales the tiles to the row minimum and forms R.
+// Pass 1 of the VJP.  Each CTA walks a strided share of the row's float4
+// groups and keeps, per thread, (mu, S, Sv) with mu the smallest |x| seen and
+// S = sum exp(-(|x| - mu)), Sv = sum v exp(-(|x| - mu)); a smaller |x| rescales
+// the sums once.  The CTA then reduces to one record, and the last CTA of the
+// row combines the records in CTA order into R = Sv / S.
+__device__ __forceinline__ void online_add(float ax, float vv, float& mu, double& s, double& sv) {
+    if (ax < mu) {
+        const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(ax - mu);
+        s *= sc;
+        sv *= sc;
+        mu = ax;
+    }
+    const double w = (double)__expf(mu - ax);
+    s += w;
+    sv += w * (double)vv;
+}
+
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
@@ -143,52 +158,71 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     __shared__ float fred[kThreads / 32];
     __shared__ int flag;
     const int64_t row = blockIdx.y;
-    const int64_t tiles = gridDim.x;
-    const int64_t base = (int64_t)blockIdx.x * kStreamTile;
+    const int64_t nblk = gridDim.x;
     const Thr th = make_thr(b[row], t);
-    float x[kPer], vv[kPer];
-    bool ok[kPer];
-    load_tile<VEC>(r + row * ld, n, base, x, ok);
-    load_tile<VEC>(v + row * ld, n, base, vv, ok);
-    float m = INFINITY;
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        x[q] = ok[q] ? fabsf(scaled_margin(x[q], th)) : INFINITY;
-        m = fminf(m, x[q]);
-    }
-    const float mu = block_min_f(m, fred);
-    double sw = 0.0, swv = 0.0;
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        if (ok[q]) {
-            const double w = (double)__expf(mu - x[q]);
-            sw += w;
-            swv += w * (double)vv[q];
+    const float* rr = r + row * ld;
+    const float* vr = v + row * ld;
+    float mu = INFINITY;
+    double s = 0.0, sv = 0.0;
+    const int64_t stride = nblk * kThreads;
+    const int64_t gt = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if constexpr (VEC) {
+        const int64_t n4 = n >> 2;
+        const float4* r4 = reinterpret_cast<const float4*>(rr);
+        const float4* v4 = reinterpret_cast<const float4*>(vr);
+        int64_t i = gt;
+        for (; i + stride < n4; i += 2 * stride) {
+            const float4 x0 = __ldcs(r4 + i), y0 = __ldcs(v4 + i);
+            const float4 x1 = __ldcs(r4 + i + stride), y1 = __ldcs(v4 + i + stride);
+            online_add(fabsf(scaled_margin(x0.x, th)), y0.x, mu, s, sv);
+            online_add(fabsf(scaled_margin(x0.y, th)), y0.y, mu, s, sv);
+            online_add(fabsf(scaled_margin(x0.z, th)), y0.z, mu, s, sv);
+            online_add(fabsf(scaled_margin(x0.w, th)), y0.w, mu, s, sv);
+            online_add(fabsf(scaled_margin(x1.x, th)), y1.x, mu, s, sv);
+            online_add(fabsf(scaled_margin(x1.y, th)), y1.y, mu, s, sv);
+            online_add(fabsf(scaled_margin(x1.z, th)), y1.z, mu, s, sv);
+            online_add(fabsf(scaled_margin(x1.w, th)), y1.w, mu, s, sv);
         }
+        for (; i < n4; i += stride) {
+            const float4 x0 = __ldcs(r4 + i), y0 = __ldcs(v4 + i);
+            online_add(fabsf(scaled_margin(x0.x, th)), y0.x, mu, s, sv);
+            online_add(fabsf(scaled_margin(x0.y, th)), y0.y, mu, s, sv);
+            online_add(fabsf(scaled_margin(x0.z, th)), y0.z, mu, s, sv);
+            online_add(fabsf(scaled_margin(x0.w, th)), y0.w, mu, s, sv);
+        }
+        for (int64_t j = (n4 << 2) + gt; j < n; j += stride)
+            online_add(fabsf(scaled_margin(rr[j], th)), vr[j], mu, s, sv);
+    } else {
+        for (int64_t j = gt; j < n; j += stride)
+            online_add(fabsf(scaled_margin(rr[j], th)), vr[j], mu, s, sv);
     }
-    sw = block_sum_d(sw, red);
-    swv = block_sum_d(swv, red);
+    // CTA record: rescale every thread to the CTA minimum, then sum.
+    const float mb = block_min_f(mu, fred);
+    const double sc = (mu == INFINITY) ? 0.0 : exp((double)mb - (double)mu);
+    s = block_sum_d(s * sc, red);
+    sv = block_sum_d(sv * sc, red);
     if (threadIdx.x == 0) {
-        double* pr = partials + (row * tiles + blockIdx.x) * 3;
-        pr[0] = (double)mu;
-        pr[1] = sw;
-        pr[2] = swv;
+        double* pr = partials + (row * nblk + blockIdx.x) * 3;
+        pr[0] = (double)mb;
+        pr[1] = s;
+        pr[2] = sv;
     }
-    if (last_block_of_row(&tickets[row], (uint32_t)tiles, &flag)) {
+    if (last_block_of_row(&tickets[row], (uint32_t)nblk, &flag)) {
         float mloc = INFINITY;
-        for (int64_t i = threadIdx.x; i < tiles; i += kThreads)
-            mloc = fminf(mloc, (float)partials[(row * tiles + i) * 3]);
+        for (int64_t i = threadIdx.x; i < nblk; i += kThreads)
+            mloc = fminf(mloc, (float)partials[(row * nblk + i) * 3]);
         const double mrow = (double)block_min_f(mloc, fred);
-        double s = 0.0, sv = 0.0;
-        for (int64_t i = threadIdx.x; i < tiles; i += kThreads) {
-            const double* pr = partials + (row * tiles + i) * 3;
-            const double sc = exp(mrow - pr[0]);
-            s += pr[1] * sc;
-            sv += pr[2] * sc;
+        double a = 0.0, av = 0.0;
+        for (int64_t i = threadIdx.x; i < nblk; i += kThreads) {
+            const double* pr = partials + (row * nblk + i) * 3;
+            if (pr[0] == INFINITY) continue;
+            const double f = exp(mrow - pr[0]);
+            a += pr[1] * f;
+            av += pr[2] * f;
         }
-        s = block_sum_d(s, red);
-        sv = block_sum_d(sv, red);
-        if (threadIdx.x == 0) row_R[row] = sv / s;
+        a = block_sum_d(a, red);
+        av = block_sum_d(av, red);
+        if (threadIdx.x == 0) row_R[row] = av / a;
     }
 }
 
@@ -240,10 +274,21 @@ cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, 
                                    float* g, int64_t B, int64_t n, double t, double* partials,
                                    double* row_R, uint32_t* tickets, int vec, cudaStream_t st) {
     const dim3 grid((unsigned)stream_tiles(n), (unsigned)B);
+    // pass 1 runs persistent CTAs: about 8 per SM over all rows, at most one per tile
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    int64_t per_row = ((int64_t)sms * 8 + B - 1) / B;
+    if (per_row > stream_tiles(n)) per_row = stream_tiles(n);
+    if (per_row < 1) per_row = 1;
+    const dim3 rgrid((unsigned)per_row, (unsigned)B);
     if (vec) {
         {
             ProfScope ps_("bwd_reduce", st);
-            bwd_reduce_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
+            bwd_reduce_kernel<true><<<rgrid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
                                                            tickets);
         }
         {
@@ -253,7 +298,7 @@ cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, 
     } else {
         {
             ProfScope ps_("bwd_reduce", st);
-            bwd_reduce_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
+            bwd_reduce_kernel<false><<<rgrid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
                                                             tickets);
         }
         {

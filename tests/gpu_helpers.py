@@ -44,8 +44,13 @@ def run_gpu(r: np.ndarray, k: float, t: float, path="auto", v: np.ndarray = None
     return res
 
 
-def check_row(r_row, v_row, k, t, b_gpu, p_gpu, g_gpu=None, b_ref=None, label=""):
-    """Compare one row of GPU output with the oracle; returns the reference b."""
+def check_row(r_row, v_row, k, t, b_gpu, p_gpu, g_gpu=None, b_ref=None, label="",
+              sum_ref="k"):
+    """Compare one row of GPU output with the oracle; returns the reference b.
+
+    sum_ref="k" checks |sum p - k| <= 1e-3 (the workloads' bar).  sum_ref="fp32"
+    compares with the sum of the oracle's p rounded to fp32, for stress cases
+    with k so large that fp32 output rounding alone exceeds 1e-3."""
     if b_ref is None:
         b_ref = oracle.solve_b(r_row, k, t)
     assert abs(b_gpu - b_ref) <= TOL_B * max(t, abs(b_ref)), \
@@ -54,7 +59,8 @@ def check_row(r_row, v_row, k, t, b_gpu, p_gpu, g_gpu=None, b_ref=None, label=""
     dp = np.max(np.abs(p_gpu - p_ref))
     assert dp <= TOL_P, f"{label}: max|dp| = {dp:.3e}"
     s = float(np.sum(p_gpu, dtype=np.float64))
-    assert abs(s - k) <= TOL_SUM, f"{label}: sum p = {s!r}, k = {k}"
+    target = k if sum_ref == "k" else float(np.sum(p_ref.astype(np.float32), dtype=np.float64))
+    assert abs(s - target) <= TOL_SUM, f"{label}: sum p = {s!r}, target {target!r}, k = {k}"
     if g_gpu is not None:
         g_ref, _, _ = oracle.vjp(r_row, v_row, b_ref, t)
         scale = np.max(np.abs(g_ref))
