@@ -282,8 +282,22 @@ def main():
             fwd()
             bwd()
         torch.cuda.synchronize(dev)
+        # the same step captured once into a CUDA graph (the library's calls are
+        # stream-ordered and allocate nothing, so they capture as they are)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fwd()
+            bwd()
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(graph):
+            fwd()
+            bwd()
+        torch.cuda.synchronize(dev)
         res = {"flush": flush, "ws": ws, "rd": rd, "vd": vd, "pd": pd, "gd": gd, "bd": bd,
-               "fwd": fwd, "bwd": bwd, "timed": timed}
+               "fwd": fwd, "bwd": bwd, "timed": timed, "graph": graph}
         if w.path == "bracket":
             info = L.row_info(ws, 0)
             res["bracket"] = {key: info[key] for key in ("attempts", "n_band", "refine_levels",
@@ -292,8 +306,10 @@ def main():
             tf, _ = timed(fwd, steps)
             tb, _ = timed(bwd, steps)
             tfb, _ = timed(lambda: (fwd(), bwd()), steps)
+            tg, _ = timed(graph.replay, steps)
             res["table"] = {"fwd_ms": statistics.median(tf), "bwd_ms": statistics.median(tb),
-                            "fwdbwd_ms": statistics.median(tfb)}
+                            "fwdbwd_ms": statistics.median(tfb),
+                            "fwdbwd_graph_ms": statistics.median(tg)}
         return res
 
     peak_gbs, peak_kind = load_peaks()
@@ -302,10 +318,16 @@ def main():
     sampler.start()
     barrier()
     torch.cuda.synchronize(dev)
-    step_ms, prof = R["timed"](lambda: (R["fwd"](), R["bwd"]()), args.steps, profile=True)
+    # per-kernel device times from an eager (profiled) pass over the same steps
+    eager_ms, prof = R["timed"](lambda: (R["fwd"](), R["bwd"]()), args.steps, profile=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    # the timed region proper: K replays of the captured step
+    step_ms, _ = R["timed"](R["graph"].replay, args.steps)
     barrier()
     clocks = sampler.stop()
     ms_local = statistics.mean(step_ms)
+    eager_ms_max = max_over_ranks(statistics.mean(eager_ms))
     ms = max_over_ranks(ms_local)
     elements = w.elements * world
     value = elements / (ms / 1e3)
@@ -379,6 +401,8 @@ def main():
             table[name] = {
                 "fwd_ms": round(T["fwd_ms"], 5), "bwd_ms": round(T["bwd_ms"], 5),
                 "fwdbwd_ms": round(T["fwdbwd_ms"], 5),
+                "fwdbwd_graph_ms": round(T["fwdbwd_graph_ms"], 5),
+                "fwdbwd_graph_elements_per_s": wk.elements / (T["fwdbwd_graph_ms"] / 1e3),
                 "fwd_elements_per_s": wk.elements / (T["fwd_ms"] / 1e3),
                 "bwd_elements_per_s": wk.elements / (T["bwd_ms"] / 1e3),
                 "fwdbwd_elements_per_s": wk.elements / (T["fwdbwd_ms"] / 1e3),
@@ -406,6 +430,9 @@ def main():
                              "inputs larger than L2 (no flush)",
                        "parallelism": f"{world} independent instances (one per GPU)"},
             "bracket": R.get("bracket"),
+            "timing": "CUDA-graph replay of one fwd+bwd step; eager calls in eager_ms_per_step",
+            "eager_ms_per_step": eager_ms_max,
+            "eager_value": elements / (eager_ms_max / 1e3),
             "step_algorithmic_gbs": step_gbs,
             "step_frac_of_peak": step_gbs / peak_gbs,
             "roofline": roofline,

@@ -56,9 +56,14 @@ __device__ uint32_t block_select_desc(Get get, int m, int64_t rho, uint32_t* his
         const uint32_t nb = 1u << widths[lev];
         for (uint32_t i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
         __syncthreads();
-        for (int i = threadIdx.x; i < m; i += blockDim.x) {
-            const uint32_t key = get(i);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+        for (int i0 = 0; i0 < m; i0 += blockDim.x) {
+            const int i = i0 + threadIdx.x;
+            const uint32_t key = i < m ? get(i) : 0u;
+            const bool in = i < m && (key & mask) == prefix;
+            const uint32_t bn = in ? ((key >> sh) & (nb - 1)) : 0xffffffffu;
+            const unsigned peers = __match_any_sync(0xffffffffu, bn);
+            if (in && (threadIdx.x & 31) == __ffs(peers) - 1)
+                atomicAdd(&hist[bn], (uint32_t)__popc(peers));
         }
         __syncthreads();
         // Suffix counts over bins: thread i owns bins 2i, 2i+1 (1024 threads).
@@ -97,28 +102,21 @@ __device__ uint32_t block_select_desc(Get get, int m, int64_t rho, uint32_t* his
     return prefix;
 }
 
-struct SmemKeyGet {
-    const uint32_t* k;
-    __device__ __forceinline__ uint32_t operator()(int i) const { return k[i]; }
-};
 struct GlobalSampleKeyGet {
     const float* y;
     __device__ __forceinline__ uint32_t operator()(int i) const { return to_key(y[i]); }
 };
 
-// The rho_a-th and rho_b-th largest of m keys in shared memory (1-based;
-// 0 = not wanted), rho_max = the larger.  One histogram pass on the top 11 key
-// bits finds the bin holding rank rho_max; every key in that bin or above is a
-// candidate.  If there are at most 4096 candidates they are compacted and
-// sorted with the register bitonic network and both ranks are read off;
-// otherwise returns false and the caller selects by full radix select.
-__device__ bool top_ranks(const uint32_t* keys, int m, int64_t rho_max, int64_t rho_a,
-                          int64_t rho_b, uint32_t* hist, uint32_t* wsum, uint32_t* bcast,
+// The rho_a-th and rho_b-th largest of the m sample values y[] (1-based;
+// 0 = not wanted), rho_max = the larger, given `hist`: the counts of the
+// samples' keys by their top 11 bits (2048 words of shared memory).  The bin
+// holding rank rho_max is found by a suffix scan; every sample in that bin or
+// above is a candidate.  If there are at most 4096 candidates they are
+// compacted and sorted with the register bitonic network and both ranks are
+// read off; otherwise returns false.  Needs blockDim.x == 1024.
+__device__ bool top_ranks(const float* __restrict__ y, int m, int64_t rho_max, int64_t rho_a,
+                          int64_t rho_b, const uint32_t* hist, uint32_t* wsum, uint32_t* bcast,
                           uint32_t* cand, uint32_t* xch, float* out_a, float* out_b) {
-    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < m; i += blockDim.x) atomicAdd(&hist[keys[i] >> 21], 1u);
-    __syncthreads();
     // suffix counts: thread i owns bins 2i, 2i+1
     const int i0 = 2 * threadIdx.x;
     const uint32_t c0 = hist[i0], c1 = hist[i0 + 1];
@@ -142,30 +140,55 @@ __device__ bool top_ranks(const uint32_t* keys, int m, int64_t rho_max, int64_t 
         bcast[0] = i0;
         bcast[1] = above + c1 + c0;
     }
-    __syncthreads();
-    const uint32_t bin = bcast[0], ncand = bcast[1];
-    __syncthreads();
-    if (ncand > (uint32_t)kBandSortMax) return false;
     if (threadIdx.x == 0) bcast[2] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < m; i += blockDim.x) {
-        const uint32_t kk = keys[i];
-        if ((kk >> 21) >= bin) cand[atomicAdd(&bcast[2], 1u)] = kk;
+    const uint32_t bin = bcast[0], ncand = bcast[1];
+    if (ncand > (uint32_t)kBandSortMax) return false;
+    // candidate pass: 8 samples per thread per trip, loads issued together
+    for (int s0 = 0; s0 < m; s0 += 8 * kBlk) {
+        float yv[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int s = s0 + q * kBlk + threadIdx.x;
+            yv[q] = s < m ? __ldcg(y + s) : -INFINITY;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const uint32_t kk = to_key(yv[q]);
+            const bool take = (s0 + q * kBlk + (int)threadIdx.x < m) && (kk >> 21) >= bin;
+            const unsigned ball = __ballot_sync(0xffffffffu, take);
+            if (ball != 0u) {
+                const int leader = __ffs(ball) - 1;
+                uint32_t base = 0;
+                if (lane == leader) base = atomicAdd(&bcast[2], (uint32_t)__popc(ball));
+                base = __shfl_sync(0xffffffffu, base, leader);
+                if (take) cand[base + __popc(ball & ((1u << lane) - 1u))] = kk;
+            }
+        }
     }
     __syncthreads();
     // ascending sort of the candidates (padding 0 sorts first); rank r from the
     // top is at position npad - r
-    uint32_t key[4];
+    int npad;
+    if (ncand <= (uint32_t)kBlk) {
+        uint32_t key[1];
+        key[0] = (int)threadIdx.x < (int)ncand ? cand[threadIdx.x] : 0u;
+        bitonic_sort_row<1, kBlk, kBlk>(key, threadIdx.x, xch);
+        cand[threadIdx.x] = key[0];
+        npad = kBlk;
+    } else {
+        uint32_t key[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int j = threadIdx.x * 4 + e;
-        key[e] = j < (int)ncand ? cand[j] : 0u;
+        for (int e = 0; e < 4; ++e) {
+            const int j = threadIdx.x * 4 + e;
+            key[e] = j < (int)ncand ? cand[j] : 0u;
+        }
+        bitonic_sort_row<4, kBlk, kBlk>(key, threadIdx.x, xch);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cand[threadIdx.x * 4 + e] = key[e];
+        npad = 4 * kBlk;
     }
-    bitonic_sort_row<4, kBlk, kBlk>(key, threadIdx.x, xch);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) cand[threadIdx.x * 4 + e] = key[e];
     __syncthreads();
-    constexpr int npad = 4 * kBlk;
     if (threadIdx.x == 0) {
         if (rho_a >= 1) *out_a = from_key(cand[npad - rho_a]);
         if (rho_b >= 1) *out_b = from_key(cand[npad - rho_b]);
@@ -182,65 +205,97 @@ __device__ bool top_ranks(const uint32_t* keys, int m, int64_t rho_max, int64_t 
 // ----------------------------------------------------------------------------
 // 1. Localization sample.
 // ----------------------------------------------------------------------------
+// Grid of m / 1024 CTAs: every thread draws one sample and every CTA adds its
+// samples to a global histogram of the keys' top 11 bits; the last CTA to
+// finish (atomic ticket) selects the two order statistics from it and clears
+// the histogram for the next call.
 __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ r, int64_t n,
                                                       double t, uint64_t seed, uint64_t c0, int m,
                                                       Ladder lad, int force_miss, int max_attempts,
                                                       float* __restrict__ sample_out,
                                                       unsigned long long* __restrict__ bins,
+                                                      uint32_t* __restrict__ ghist,
+                                                      uint32_t* __restrict__ ticket,
                                                       RowState* st) {
-    for (int i = threadIdx.x; i < 3 * kBins; i += kBlk) bins[i] = 0ull;
+    if (blockIdx.x == 0) {
+        // this kernel starts the row's forward: clear its record and histogram
+        for (int i = threadIdx.x; i < (int)(sizeof(RowState) / 4); i += kBlk)
+            reinterpret_cast<uint32_t*>(st)[i] = 0u;
+        for (int i = threadIdx.x; i < 3 * kBins; i += kBlk) bins[i] = 0ull;
+    }
     extern __shared__ uint32_t dyn[];
-    uint32_t* keys = dyn;              // m keys
-    uint32_t* cand = dyn + m;          // up to 4096 candidate keys
+    uint32_t* cand = dyn;                 // up to 4096 candidate keys
     uint32_t* xch = cand + kBandSortMax;  // bitonic exchange area (4096 words)
     __shared__ uint32_t hist[2048];
     __shared__ uint32_t wsum[32];
     __shared__ uint32_t bcast[4];
-    const float tf = (float)t;
-    // m is a multiple of 8 * kBlk / 4: each thread issues its gathers in groups
-    // of 8 independent loads so their latencies overlap.
-    constexpr int G = 8;
-    for (int s0 = threadIdx.x; s0 < m; s0 += G * kBlk) {
-        float rv[G];
-#pragma unroll
-        for (int q = 0; q < G; ++q) {
-            const int s = s0 + q * kBlk;
-            rv[q] = 0.f;
-            if (s < m) {
-                const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
-                const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
-                rv[q] = __ldg(r + I);
-            }
+    __shared__ int flag;
+    for (int i = threadIdx.x; i < 2048; i += kBlk) hist[i] = 0u;
+    __syncthreads();
+    {
+        const int s = blockIdx.x * kBlk + threadIdx.x;
+        uint32_t bn = 0xffffffffu;
+        if (s < m) {
+            const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
+            const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
+            const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
+            const float rv = __ldg(r + I);
+            const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
+            const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
+            const float eps = (u < 0.0 ? 1.f : -1.f) * (float)t * logf(a);
+            const float y = rv + eps;
+            sample_out[s] = y;
+            bn = to_key(y) >> 21;
         }
-#pragma unroll
-        for (int q = 0; q < G; ++q) {
-            const int s = s0 + q * kBlk;
-            if (s < m) {
-                const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
-                const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
-                const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
-                const float eps = (u < 0.0 ? 1.f : -1.f) * tf * logf(a);
-                const float y = rv[q] + eps;
-                sample_out[s] = y;
-                keys[s] = to_key(y);
-            }
-        }
+        // lanes with the same bin add once (samples crowd into few top bins)
+        const unsigned peers = __match_any_sync(0xffffffffu, bn);
+        if (bn != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
+            atomicAdd(&hist[bn], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 2048; i += kBlk)
+        if (hist[i] != 0u) atomicAdd(&ghist[i], hist[i]);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t prev = atomicAdd(ticket, 1u);
+        flag = (prev == gridDim.x - 1);
+        if (flag) *ticket = 0u;
+    }
+    __syncthreads();
+    if (!flag) return;
+    __threadfence();
+    for (int i = threadIdx.x; i < 2048; i += kBlk) {
+        hist[i] = __ldcg(ghist + i);
+        ghist[i] = 0u;  // ready for the next call
     }
     __syncthreads();
     float aR = INFINITY, aL = -INFINITY;
     const int64_t rmax = lad.h[0] <= m ? lad.h[0] : lad.l[0];
-    if (rmax >= 1 && top_ranks(keys, m, rmax, lad.l[0], lad.h[0] <= m ? lad.h[0] : 0, hist, wsum,
-                               bcast, cand, xch, &aR, &aL)) {
+    if (rmax >= 1 && top_ranks(sample_out, m, rmax, lad.l[0], lad.h[0] <= m ? lad.h[0] : 0, hist,
+                               wsum, bcast, cand, xch, &aR, &aL)) {
         // both order statistics read off the sorted top candidates
     } else {
         if (lad.l[0] >= 1) {
-            const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.l[0], hist, wsum, bcast);
+            const uint32_t kk = block_select_desc(GlobalSampleKeyGet{sample_out}, m, lad.l[0],
+                                                  hist, wsum, bcast);
             aR = from_key(kk);
         }
         if (lad.h[0] <= m) {
-            const uint32_t kk = block_select_desc(SmemKeyGet{keys}, m, lad.h[0], hist, wsum, bcast);
+            const uint32_t kk = block_select_desc(GlobalSampleKeyGet{sample_out}, m, lad.h[0],
+                                                  hist, wsum, bcast);
             aL = from_key(kk);
         }
+    }
+    if (force_miss) {
+        uint32_t kmax = 0;
+        for (int s = threadIdx.x; s < m; s += kBlk) kmax = max(kmax, to_key(__ldcg(sample_out + s)));
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, d));
+        if (threadIdx.x == 0) bcast[3] = 0u;
+        __syncthreads();
+        if ((threadIdx.x & 31) == 0) atomicMax(&bcast[3], kmax);
+        __syncthreads();
     }
     if (threadIdx.x == 0) {
         st->ladder_R[0] = aR;
@@ -249,9 +304,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
         st->rung_R = 0;
         if (force_miss) {
             // A bracket above every sample value: F(a_L) < k, so it must fail.
-            uint32_t kmax = 0;
-            for (int s = 0; s < m; ++s) kmax = max(kmax, keys[s]);
-            const float top = from_key(kmax);
+            const float top = from_key(bcast[3]);
             st->a_L = top + fabsf(top) + 1.f;
             st->a_R = INFINITY;
             st->rung_L = -1;
@@ -276,23 +329,32 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
 // 2. Streaming fold.
 // ----------------------------------------------------------------------------
 struct FoldAcc {
-    unsigned long long cntR;
+    uint32_t cntR;  // per thread: at most n / (grid threads)
     double SL, SR;
     bool bad;
 };
 
+// One score: right tail (count and e^{-(x - aR)/t}), left tail (e^{(x - aL)/t})
+// or band.  The tail terms go to fp32 partials that the caller flushes into
+// the fp64 accumulators every few scores.
+__device__ __forceinline__ void fold_one(float x, float aL, float aR, float inv_t, FoldAcc& acc,
+                                         float& sl, float& sr, bool& in_band) {
+    acc.bad |= !finite_f(x);
+    const bool right = x >= aR, left = x < aL;
+    // one exponential serves whichever tail the score is in (band scores are
+    // masked out; their argument is a finite dummy)
+    const float e = __expf((right ? (aR - x) : (left ? (x - aL) : 0.f)) * inv_t);
+    acc.cntR += right ? 1u : 0u;
+    sr += right ? e : 0.f;
+    sl += left ? e : 0.f;
+    in_band = !(right | left);
+}
 __device__ __forceinline__ void fold_one(float x, float aL, float aR, float inv_t, FoldAcc& acc,
                                          bool& in_band) {
-    acc.bad |= !finite_f(x);
-    in_band = false;
-    if (x >= aR) {
-        acc.cntR += 1;
-        acc.SR += (double)__expf((aR - x) * inv_t);
-    } else if (x < aL) {
-        acc.SL += (double)__expf((x - aL) * inv_t);
-    } else {
-        in_band = true;
-    }
+    float sl = 0.f, sr = 0.f;
+    fold_one(x, aL, aR, inv_t, acc, sl, sr, in_band);
+    acc.SL += (double)sl;
+    acc.SR += (double)sr;
 }
 
 // Adds one band score to the fixed-point band histogram (global atomics).
@@ -306,6 +368,22 @@ __device__ __forceinline__ void bin_add(float x, const BinLayout& BL, float inv_
 }
 
 constexpr int kStage = 2048;  // band scores staged per CTA before one global append
+
+// One lane appends one band score to the CTA staging buffer (or, when it is
+// full, straight to the global band).
+__device__ __forceinline__ void band_stage_lane(float x, float* sband, int* scount, float* band,
+                                                unsigned long long* counter,
+                                                unsigned long long cap, const BinLayout& BL,
+                                                float inv_t, unsigned long long* bins) {
+    const int pos = atomicAdd(scount, 1);
+    if (pos < kStage) {
+        sband[pos] = x;
+    } else {
+        const unsigned long long g = atomicAdd(counter, 1ull);
+        if (g < cap) band[g] = x;
+        bin_add(x, BL, inv_t, bins);
+    }
+}
 
 // Warp-aggregated append of the lanes with `take` to the CTA's staging buffer;
 // lanes past its capacity go straight to the global band (rare).
@@ -349,7 +427,7 @@ __device__ __forceinline__ void band_flush(const float* sband, int scount, float
     }
 }
 
-__global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restrict__ r, int64_t n,
+__global__ void __launch_bounds__(kFoldThreads, 6) fold_kernel(const float* __restrict__ r, int64_t n,
                                                             double t, RowState* st,
                                                             float* __restrict__ band,
                                                             unsigned long long* __restrict__ bins,
@@ -367,7 +445,7 @@ __global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restr
     const float inv_t = (float)(1.0 / t);
     if (threadIdx.x == 0) scount = 0;
     __syncthreads();
-    FoldAcc acc{0ull, 0.0, 0.0, false};
+    FoldAcc acc{0u, 0.0, 0.0, false};
     unsigned long long* counter = &st->n_band;
     const unsigned long long cap = (unsigned long long)n;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
@@ -377,35 +455,62 @@ __global__ void __launch_bounds__(kFoldThreads) fold_kernel(const float* __restr
     if (vec) {
         const int64_t n4 = n >> 2;
         const float4* r4 = reinterpret_cast<const float4*>(r);
-        // Four independent 16-byte loads per thread per trip keep enough bytes
-        // in flight; the trip count is uniform so the ballots see full warps.
+        // Main part: full trips only (every load in range for every thread), so
+        // the loop body is branch-free arithmetic over 16 scores per thread:
+        // four independent 16-byte loads, then one warp vote over a 16-bit
+        // band mask.  In-band scores (rare) go to the CTA staging buffer one
+        // by one through a shared-memory slot counter.
         constexpr int U = 4;
-        const int64_t iters = (n4 + (int64_t)U * nthreads - 1) / ((int64_t)U * nthreads);
-        for (int64_t it = 0; it < iters; ++it) {
+        const int64_t step = (int64_t)U * nthreads;
+        const int64_t full = n4 / step;
+        const float4* p = r4 + gtid;
+        for (int64_t it = 0; it < full; ++it, p += step) {
             float4 v[U];
-            bool ok[U];
+#pragma unroll
+            for (int q = 0; q < U; ++q) v[q] = __ldcs(p + (int64_t)q * nthreads);
+            float sl = 0.f, sr = 0.f;  // at most 16 terms <= 1 each
+            uint32_t mask = 0u;
 #pragma unroll
             for (int q = 0; q < U; ++q) {
-                const int64_t i = (it * U + q) * nthreads + gtid;
-                ok[q] = i < n4;
-                v[q] = ok[q] ? __ldcs(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                bool b0, b1, b2, b3;
+                fold_one(v[q].x, aL, aR, inv_t, acc, sl, sr, b0);
+                fold_one(v[q].y, aL, aR, inv_t, acc, sl, sr, b1);
+                fold_one(v[q].z, aL, aR, inv_t, acc, sl, sr, b2);
+                fold_one(v[q].w, aL, aR, inv_t, acc, sl, sr, b3);
+                mask |= ((uint32_t)b0 | ((uint32_t)b1 << 1) | ((uint32_t)b2 << 2) |
+                         ((uint32_t)b3 << 3)) << (4 * q);
             }
+            acc.SL += (double)sl;
+            acc.SR += (double)sr;
+            if (__any_sync(0xffffffffu, mask != 0u)) {
 #pragma unroll
-            for (int q = 0; q < U; ++q) {
-                bool b0 = false, b1 = false, b2 = false, b3 = false;
-                if (ok[q]) {
-                    fold_one(v[q].x, aL, aR, inv_t, acc, b0);
-                    fold_one(v[q].y, aL, aR, inv_t, acc, b1);
-                    fold_one(v[q].z, aL, aR, inv_t, acc, b2);
-                    fold_one(v[q].w, aL, aR, inv_t, acc, b3);
-                }
-                if (__any_sync(0xffffffffu, b0 | b1 | b2 | b3)) {
-                    LAPSUM_STAGE(b0, v[q].x);
-                    LAPSUM_STAGE(b1, v[q].y);
-                    LAPSUM_STAGE(b2, v[q].z);
-                    LAPSUM_STAGE(b3, v[q].w);
+                for (int q = 0; q < U; ++q) {
+                    const float xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (mask & (1u << (4 * q + c)))
+                            band_stage_lane(xs[c], sband, &scount, band, counter, cap, BL, inv_t,
+                                            bins);
                 }
             }
+        }
+        // Remainder: the last partial trip, with bounds checks and warp ballots.
+        const int64_t rem_iters = (n4 - full * step + nthreads - 1) / nthreads;
+        for (int64_t it = 0; it < rem_iters; ++it) {
+            const int64_t i = full * step + it * nthreads + gtid;
+            const bool ok = i < n4;
+            const float4 v = ok ? __ldcs(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            bool b0 = false, b1 = false, b2 = false, b3 = false;
+            if (ok) {
+                fold_one(v.x, aL, aR, inv_t, acc, b0);
+                fold_one(v.y, aL, aR, inv_t, acc, b1);
+                fold_one(v.z, aL, aR, inv_t, acc, b2);
+                fold_one(v.w, aL, aR, inv_t, acc, b3);
+            }
+            LAPSUM_STAGE(b0, v.x);
+            LAPSUM_STAGE(b1, v.y);
+            LAPSUM_STAGE(b2, v.z);
+            LAPSUM_STAGE(b3, v.w);
         }
         // tail elements (n not a multiple of 4)
         const int64_t rem0 = n4 << 2;
@@ -531,22 +636,29 @@ struct SolveSmemAll {
     } u;
 };
 
-// Band of size <= 4096: sort on chip and solve with the tails.
-__device__ void solve_small_band(const float* band, long long nb, const Tails& tl, double k,
-                                 double t, SolveSmemAll* sm) {
-    uint32_t key[4];
+// Band of size <= 4096: sort on chip and solve with the tails.  The network
+// size follows the band: 1, 2 or 4 keys per thread.
+template <int E>
+__device__ void sort_band_into(const float* band, long long nb, SolveSmemAll* sm) {
+    uint32_t key[E];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const long long j = (long long)threadIdx.x * 4 + e;
+    for (int e = 0; e < E; ++e) {
+        const long long j = (long long)threadIdx.x * E + e;
         key[e] = j < nb ? to_key(band[j]) : 0xffffffffu;
     }
-    bitonic_sort_row<4, kBlk, kBlk>(key, threadIdx.x, sm->u.sort.xch);
+    bitonic_sort_row<E, kBlk, kBlk>(key, threadIdx.x, sm->u.sort.xch);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const long long j = (long long)threadIdx.x * 4 + e;
+    for (int e = 0; e < E; ++e) {
+        const long long j = (long long)threadIdx.x * E + e;
         if (j < nb) sm->u.sort.sorted[j] = from_key(key[e]);
     }
     __syncthreads();
+}
+__device__ void solve_small_band(const float* band, long long nb, const Tails& tl, double k,
+                                 double t, SolveSmemAll* sm) {
+    if (nb <= kBlk) sort_band_into<1>(band, nb, sm);
+    else if (nb <= 2 * kBlk) sort_band_into<2>(band, nb, sm);
+    else sort_band_into<4>(band, nb, sm);
     solve_sorted_block(FloatGet{sm->u.sort.sorted}, nb, tl, k, t, &sm->ss, &sm->res);
 }
 
@@ -895,7 +1007,7 @@ __device__ void refold_row(const float* __restrict__ r, int64_t n, float aL, flo
     const float inv_t = (float)(1.0 / t);
     if (threadIdx.x == 0) sm->cnt = 0ull;
     __syncthreads();
-    FoldAcc acc{0ull, 0.0, 0.0, false};
+    FoldAcc acc{0u, 0.0, 0.0, false};
     const int64_t iters = (n + blockDim.x - 1) / blockDim.x;
     for (int64_t it = 0; it < iters; ++it) {
         const int64_t i = it * blockDim.x + threadIdx.x;
@@ -1093,12 +1205,12 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                                RowState* st_row, double* b_out, WsHeader* hdr, cudaStream_t st) {
     static bool attr_done = false;
     const size_t solve_smem = sizeof(SolveSmemAll);
-    const size_t sample_smem = ((size_t)m + 2 * kBandSortMax) * sizeof(uint32_t);
+    const size_t sample_smem = (size_t)2 * kBandSortMax * sizeof(uint32_t);
     if (!attr_done) {
         cudaFuncSetAttribute(solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)solve_smem);
         cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)((kSampleMax + 2 * kBandSortMax) * sizeof(uint32_t)));
+                             (int)(2 * kBandSortMax * sizeof(uint32_t)));
         attr_done = true;
     }
     Ladder lad;
@@ -1112,8 +1224,9 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     const uint64_t c0 = (uint64_t)row << 32;
     {
         ProfScope ps_("bracket_sample", st);
-        sample_kernel<<<1, kBlk, sample_smem, st>>>(r_row, n, t, seed, c0, m, lad, force_miss,
-                                                max_attempts, sample, buf.bins, st_row);
+        sample_kernel<<<(m + kBlk - 1) / kBlk, kBlk, sample_smem, st>>>(
+            r_row, n, t, seed, c0, m, lad, force_miss, max_attempts, sample, buf.bins,
+            buf.ticket + 2, buf.ticket + 1, st_row);
     }
     const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
     {

@@ -56,7 +56,9 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
     };
     const int64_t tiles = stream_tiles(n);
     L.header = take(sizeof(WsHeader));
-    L.tickets = take((size_t)B * 2 * sizeof(uint32_t) + sizeof(uint32_t));
+    // per-row emit/backward tickets, then the fold and sample tickets and the
+    // sample kernel's 2048-bin key histogram (all self-clearing)
+    L.tickets = take((size_t)B * 2 * sizeof(uint32_t) + (2 + 2048) * sizeof(uint32_t));
     L.fold_ticket = L.tickets + (size_t)B * 2 * sizeof(uint32_t);
     L.rows = take((size_t)B * 512);
     L.partials = take((size_t)B * (size_t)tiles * 3 * sizeof(double));
@@ -262,9 +264,9 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
         e = launch_onchip_forward(r, ld, p, b, sum_f, B, (int)n, k, t, hdr, vec, st);
         return cuda_status(e);
     }
-    e = cudaMemsetAsync(rows, 0, (size_t)B * 512, st);
-    if (e != cudaSuccess) return LAPSUM_ECUDA;
     if (rp == LAPSUM_PATH_RADIX) {
+        e = cudaMemsetAsync(rows, 0, (size_t)B * 512, st);
+        if (e != cudaSuccess) return LAPSUM_ECUDA;
         RadixBuffers rb;
         rb.keys[0] = reinterpret_cast<uint32_t*>(w + L.keys0);
         rb.keys[1] = reinterpret_cast<uint32_t*>(w + L.keys1);

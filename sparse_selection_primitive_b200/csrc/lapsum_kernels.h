@@ -62,7 +62,7 @@ struct BracketBuffers {
     float* band[2];      // capacity n each
     unsigned long long* bins;  // band histogram of the first bracket: [3][2048]
     double* fold_part;   // fold partials, one record per CTA
-    uint32_t* ticket;    // last-block counter
+    uint32_t* ticket;    // last-block counters: [0] fold, [1] sample; [2..2050) sample histogram
     int fold_grid;
 };
 int bracket_fold_grid();

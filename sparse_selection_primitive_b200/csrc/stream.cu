@@ -137,16 +137,25 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
 // S = sum exp(-(|x| - mu)), Sv = sum v exp(-(|x| - mu)); a smaller |x| rescales
 // the sums once.  The CTA then reduces to one record, and the last CTA of the
 // row combines the records in CTA order into R = Sv / S.
-__device__ __forceinline__ void online_add(float ax, float vv, float& mu, double& s, double& sv) {
-    if (ax < mu) {
-        const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(ax - mu);
+// Four scores at a time: a new minimum rescales the fp64 sums once, then the
+// four weights are summed in fp32 (each at most 1) and added in fp64.
+__device__ __forceinline__ void online_add4(float a0, float a1, float a2, float a3, float v0,
+                                            float v1, float v2, float v3, float& mu, double& s,
+                                            double& sv) {
+    const float m4 = fminf(fminf(a0, a1), fminf(a2, a3));
+    if (m4 < mu) {
+        const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(m4 - mu);
         s *= sc;
         sv *= sc;
-        mu = ax;
+        mu = m4;
     }
-    const double w = (double)__expf(mu - ax);
-    s += w;
-    sv += w * (double)vv;
+    const float w0 = __expf(mu - a0), w1 = __expf(mu - a1), w2 = __expf(mu - a2),
+                w3 = __expf(mu - a3);
+    s += (double)((w0 + w1) + (w2 + w3));
+    sv += (double)(fmaf(w0, v0, w1 * v1) + fmaf(w2, v2, w3 * v3));
+}
+__device__ __forceinline__ void online_add(float ax, float vv, float& mu, double& s, double& sv) {
+    online_add4(ax, INFINITY, INFINITY, INFINITY, vv, 0.f, 0.f, 0.f, mu, s, sv);
 }
 
 template <bool VEC>
@@ -171,24 +180,25 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
         const float4* r4 = reinterpret_cast<const float4*>(rr);
         const float4* v4 = reinterpret_cast<const float4*>(vr);
         int64_t i = gt;
-        for (; i + stride < n4; i += 2 * stride) {
-            const float4 x0 = __ldcs(r4 + i), y0 = __ldcs(v4 + i);
-            const float4 x1 = __ldcs(r4 + i + stride), y1 = __ldcs(v4 + i + stride);
-            online_add(fabsf(scaled_margin(x0.x, th)), y0.x, mu, s, sv);
-            online_add(fabsf(scaled_margin(x0.y, th)), y0.y, mu, s, sv);
-            online_add(fabsf(scaled_margin(x0.z, th)), y0.z, mu, s, sv);
-            online_add(fabsf(scaled_margin(x0.w, th)), y0.w, mu, s, sv);
-            online_add(fabsf(scaled_margin(x1.x, th)), y1.x, mu, s, sv);
-            online_add(fabsf(scaled_margin(x1.y, th)), y1.y, mu, s, sv);
-            online_add(fabsf(scaled_margin(x1.z, th)), y1.z, mu, s, sv);
-            online_add(fabsf(scaled_margin(x1.w, th)), y1.w, mu, s, sv);
+        // four (r, v) float4 pairs in flight per thread
+        for (; i + 3 * stride < n4; i += 4 * stride) {
+            float4 x[4], y[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                x[q] = __ldcs(r4 + i + q * stride);
+                y[q] = __ldcs(v4 + i + q * stride);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                online_add4(fabsf(scaled_margin(x[q].x, th)), fabsf(scaled_margin(x[q].y, th)),
+                            fabsf(scaled_margin(x[q].z, th)), fabsf(scaled_margin(x[q].w, th)),
+                            y[q].x, y[q].y, y[q].z, y[q].w, mu, s, sv);
         }
         for (; i < n4; i += stride) {
             const float4 x0 = __ldcs(r4 + i), y0 = __ldcs(v4 + i);
-            online_add(fabsf(scaled_margin(x0.x, th)), y0.x, mu, s, sv);
-            online_add(fabsf(scaled_margin(x0.y, th)), y0.y, mu, s, sv);
-            online_add(fabsf(scaled_margin(x0.z, th)), y0.z, mu, s, sv);
-            online_add(fabsf(scaled_margin(x0.w, th)), y0.w, mu, s, sv);
+            online_add4(fabsf(scaled_margin(x0.x, th)), fabsf(scaled_margin(x0.y, th)),
+                        fabsf(scaled_margin(x0.z, th)), fabsf(scaled_margin(x0.w, th)), y0.x,
+                        y0.y, y0.z, y0.w, mu, s, sv);
         }
         for (int64_t j = (n4 << 2) + gt; j < n; j += stride)
             online_add(fabsf(scaled_margin(rr[j], th)), vr[j], mu, s, sv);
