@@ -165,6 +165,30 @@ typedef struct lapsum_kernel_time {
 int lapsum_profile_enable(int on);
 int lapsum_profile_read(lapsum_kernel_time* out, int max_entries, int* n_entries);
 
+/*
+ * lapsum_backward_noalloc: the same result as lapsum_backward, for callers
+ * that cannot allocate device memory (no workspace argument).  The pages have
+ * no counterpart of this call; it exists for code that must not allocate at
+ * the point it needs the gradient: work recorded during a CUDA graph capture
+ * under a no-allocation rule, hosts that reserve all device memory up front,
+ * and plugin hosts that own every allocation.
+ *
+ * Scratch: a fixed 108 KiB array inside the library (one per GPU that loads
+ * it, held until the process exits).  Limits: B <= 1024 rows, and for rows
+ * longer than 4096 scores also 8 * (SM count) + B <= 4096 (true for every
+ * B <= 1024 on a 148-SM B200); other calls return LAPSUM_EINVAL and launch
+ * nothing.
+ * The first call on each device looks up the array's device address (one
+ * cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call on a device shares the one array and clears the part that must
+ * start at zero itself, so calls that overlap on the GPU (different streams
+ * without ordering between them) race and give wrong results; order them.
+ * Never allocates or frees memory.  Returns LAPSUM_OK, LAPSUM_EINVAL or
+ * LAPSUM_ECUDA.
+ */
+int lapsum_backward_noalloc(const float* r, int64_t ld, const double* b, const float* v, float* g,
+                            int64_t B, int64_t n, double t, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,7 @@ from . import _build
 __all__ = [
     "LapSumError", "Workspace", "forward", "backward", "read_status", "row_info", "sample_values",
     "workspace_bytes", "soft_topk", "LapSumTopK", "PATHS", "FLAG_FORCE_MISS", "FLAG_NO_RETRY",
-    "library_path", "profile_enable", "profile_read",
+    "library_path", "profile_enable", "profile_read", "backward_noalloc",
 ]
 
 PATHS = {"auto": 0, "fullsort": 1, "bracket": 2, "radix": 3}
@@ -236,6 +236,40 @@ def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Wo
     _check(_lib().lapsum_backward(r2.data_ptr(), ld, b.data_ptr(), v2.data_ptr(), g.data_ptr(), B,
                                   n, float(t), ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
            "lapsum_backward")
+    return g[0] if squeeze else g
+
+
+def backward_noalloc(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float,
+                     g: torch.Tensor = None):
+    """Backward without a workspace, for callers that cannot allocate device memory.
+
+    Same result as backward(); the library keeps its scratch in a fixed array
+    (limits: at most 1024 rows).  Calls on one device must not overlap on the
+    GPU, and the first call on a device must come before any stream capture.
+    """
+    lib = _lib()
+    fn = lib.lapsum_backward_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64, ctypes.c_double, _vp]
+    squeeze = r.dim() == 1
+    r2 = _as_rows(r)
+    v2 = _as_rows(v)
+    B, n = r2.shape
+    if v2.shape != r2.shape:
+        raise ValueError("v must have the shape of r")
+    if _ld(v2) != _ld(r2):
+        v2 = v2.contiguous()
+        r2 = r2.contiguous()
+    ld = _ld(r2)
+    if g is None:
+        g = _like_rows(r2, ld)
+    else:
+        g = g.view(B, n) if g.dim() == 1 else g
+        _check_out(g, r2, ld, "g")
+    if b.dtype != torch.float64 or not b.is_cuda or b.numel() != B:
+        raise TypeError("b must be a float64 CUDA tensor with one entry per row")
+    _check(fn(r2.data_ptr(), ld, b.data_ptr(), v2.data_ptr(), g.data_ptr(), B, n, float(t),
+              _stream_ptr(r2.device)), "lapsum_backward_noalloc")
     return g[0] if squeeze else g
 
 
