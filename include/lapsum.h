@@ -173,7 +173,7 @@ int lapsum_profile_read(lapsum_kernel_time* out, int max_entries, int* n_entries
  * under a no-allocation rule, hosts that reserve all device memory up front,
  * and plugin hosts that own every allocation.
  *
- * Scratch: a fixed 108 KiB array inside the library (one per GPU that loads
+ * Scratch: a fixed 140 KiB array inside the library (one per GPU that loads
  * it, held until the process exits).  Limits: B <= 1024 rows, and for rows
  * longer than 4096 scores also 8 * (SM count) + B <= 4096 (true for every
  * B <= 1024 on a 148-SM B200); other calls return LAPSUM_EINVAL and launch

@@ -427,7 +427,9 @@ __device__ __forceinline__ void band_flush(const float* sband, int scount, float
     }
 }
 
-__global__ void __launch_bounds__(kFoldThreads, 6) fold_kernel(const float* __restrict__ r, int64_t n,
+constexpr int kQ = 1024;  // per-warp circular queue of near scores (power of two)
+
+__global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __restrict__ r, int64_t n,
                                                             double t, RowState* st,
                                                             float* __restrict__ band,
                                                             unsigned long long* __restrict__ bins,
@@ -437,107 +439,130 @@ __global__ void __launch_bounds__(kFoldThreads, 6) fold_kernel(const float* __re
     __shared__ double red[kFoldThreads / 32];
     __shared__ long long lred[kFoldThreads / 32];
     __shared__ float sband[kStage];
+    __shared__ float wq[kFoldThreads / 32][kQ];
     __shared__ int scount;
     __shared__ unsigned long long gbase;
     __shared__ int flag;
     const float aL = st->a_L, aR = st->a_R;
+    // Scores more than 90 t below the bracket add exactly 0 to the left tail
+    // sum in fp32, and scores more than 90 t above it add 1 to the right count
+    // and 0 to its sum; only the scores between these limits ("near") need
+    // the full fold.  Each trip builds a 16-bit near mask per thread; a warp
+    // that has near scores appends them to its circular queue (one warp scan)
+    // and folds them 32 at a time, so the lanes stay busy on them however
+    // sparse they are.
+    const float aLf = aL - (float)(90.0 * t), aRf = aR + (float)(90.0 * t);
     const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
     const float inv_t = (float)(1.0 / t);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* q = wq[warp];
+    uint32_t head = 0, tail = 0;  // warp-uniform; tail - head = queued scores
     if (threadIdx.x == 0) scount = 0;
     __syncthreads();
     FoldAcc acc{0u, 0.0, 0.0, false};
+    uint32_t far_right = 0u;
+    bool bad = false;
     unsigned long long* counter = &st->n_band;
     const unsigned long long cap = (unsigned long long)n;
     const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
     const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-#define LAPSUM_STAGE(take, x) \
-    band_stage(take, x, sband, &scount, band, counter, cap, BL, inv_t, bins)
+    auto drain = [&](int cnt) {  // fold `cnt` (<= 32) queued scores, one per lane
+        const bool ok = lane < cnt;
+        const float x = ok ? q[(head + lane) & (kQ - 1)] : 0.f;
+        bool inb = false;
+        if (ok) fold_one(x, aL, aR, inv_t, acc, inb);
+        band_stage(inb, x, sband, &scount, band, counter, cap, BL, inv_t, bins);
+        head += cnt;
+    };
+    auto push = [&](const float* xs, uint32_t m, int cnt_max) {
+        __syncwarp();
+        const int c = __popc(m);
+        int incl = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        uint32_t off = tail + (uint32_t)(incl - c);
+        for (int j = 0; j < cnt_max; ++j)
+            if (m & (1u << j)) q[(off++) & (kQ - 1)] = xs[j];
+        tail += (uint32_t)total;
+        __syncwarp();
+        while (tail - head >= 32u) drain(32);
+    };
+    auto classify = [&](float x, bool valid, uint32_t& m, int j) {
+        const bool nr = valid && (x >= aLf) && (x < aRf);
+        m |= (uint32_t)nr << j;
+        far_right += (valid && x >= aRf) ? 1u : 0u;
+        bad |= valid && !(fabsf(x) <= 3.402823466e38f);
+    };
     if (vec) {
         const int64_t n4 = n >> 2;
         const float4* r4 = reinterpret_cast<const float4*>(r);
-        // Main part: full trips only (every load in range for every thread), so
-        // the loop body is branch-free arithmetic over 16 scores per thread:
-        // four independent 16-byte loads, then one warp vote over a 16-bit
-        // band mask.  In-band scores (rare) go to the CTA staging buffer one
-        // by one through a shared-memory slot counter.
+        // Main part: full trips only (every load in range for every thread);
+        // the loads run one trip ahead of the processing.
         constexpr int U = 4;
         const int64_t step = (int64_t)U * nthreads;
         const int64_t full = n4 / step;
         const float4* p = r4 + gtid;
-        for (int64_t it = 0; it < full; ++it, p += step) {
-            float4 v[U];
+        float4 nv[U];
+        if (full > 0) {
 #pragma unroll
-            for (int q = 0; q < U; ++q) v[q] = __ldcs(p + (int64_t)q * nthreads);
-            float sl = 0.f, sr = 0.f;  // at most 16 terms <= 1 each
-            uint32_t mask = 0u;
-#pragma unroll
-            for (int q = 0; q < U; ++q) {
-                bool b0, b1, b2, b3;
-                fold_one(v[q].x, aL, aR, inv_t, acc, sl, sr, b0);
-                fold_one(v[q].y, aL, aR, inv_t, acc, sl, sr, b1);
-                fold_one(v[q].z, aL, aR, inv_t, acc, sl, sr, b2);
-                fold_one(v[q].w, aL, aR, inv_t, acc, sl, sr, b3);
-                mask |= ((uint32_t)b0 | ((uint32_t)b1 << 1) | ((uint32_t)b2 << 2) |
-                         ((uint32_t)b3 << 3)) << (4 * q);
-            }
-            acc.SL += (double)sl;
-            acc.SR += (double)sr;
-            if (__any_sync(0xffffffffu, mask != 0u)) {
-#pragma unroll
-                for (int q = 0; q < U; ++q) {
-                    const float xs[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        if (mask & (1u << (4 * q + c)))
-                            band_stage_lane(xs[c], sband, &scount, band, counter, cap, BL, inv_t,
-                                            bins);
-                }
-            }
+            for (int qq = 0; qq < U; ++qq) nv[qq] = __ldcs(p + (int64_t)qq * nthreads);
         }
-        // Remainder: the last partial trip, with bounds checks and warp ballots.
+        for (int64_t it = 0; it < full; ++it, p += step) {
+            float xs[4 * U];
+#pragma unroll
+            for (int qq = 0; qq < U; ++qq) {
+                xs[4 * qq] = nv[qq].x;
+                xs[4 * qq + 1] = nv[qq].y;
+                xs[4 * qq + 2] = nv[qq].z;
+                xs[4 * qq + 3] = nv[qq].w;
+            }
+            if (it + 1 < full) {
+#pragma unroll
+                for (int qq = 0; qq < U; ++qq) nv[qq] = __ldcs(p + step + (int64_t)qq * nthreads);
+            }
+            uint32_t m = 0u;
+#pragma unroll
+            for (int j = 0; j < 4 * U; ++j) classify(xs[j], true, m, j);
+            if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 4 * U);
+        }
+        // Remainder: the last partial trip, with bounds checks.
         const int64_t rem_iters = (n4 - full * step + nthreads - 1) / nthreads;
         for (int64_t it = 0; it < rem_iters; ++it) {
             const int64_t i = full * step + it * nthreads + gtid;
             const bool ok = i < n4;
             const float4 v = ok ? __ldcs(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            bool b0 = false, b1 = false, b2 = false, b3 = false;
-            if (ok) {
-                fold_one(v.x, aL, aR, inv_t, acc, b0);
-                fold_one(v.y, aL, aR, inv_t, acc, b1);
-                fold_one(v.z, aL, aR, inv_t, acc, b2);
-                fold_one(v.w, aL, aR, inv_t, acc, b3);
-            }
-            LAPSUM_STAGE(b0, v.x);
-            LAPSUM_STAGE(b1, v.y);
-            LAPSUM_STAGE(b2, v.z);
-            LAPSUM_STAGE(b3, v.w);
+            const float xs[4] = {v.x, v.y, v.z, v.w};
+            uint32_t m = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) classify(xs[j], ok, m, j);
+            if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 4);
         }
         // tail elements (n not a multiple of 4)
         const int64_t rem0 = n4 << 2;
         if (blockIdx.x == 0 && threadIdx.x < 32) {
             const int64_t i = rem0 + threadIdx.x;
-            bool bb = false;
-            float x = 0.f;
-            if (i < n) {
-                x = r[i];
-                fold_one(x, aL, aR, inv_t, acc, bb);
-            }
-            LAPSUM_STAGE(bb, x);
+            const float xs[1] = {i < n ? r[i] : 0.f};
+            uint32_t m = 0u;
+            classify(xs[0], i < n, m, 0);
+            if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 1);
         }
     } else {
         const int64_t iters = (n + nthreads - 1) / nthreads;
         for (int64_t it = 0; it < iters; ++it) {
             const int64_t i = it * nthreads + gtid;
-            bool bb = false;
-            float x = 0.f;
-            if (i < n) {
-                x = r[i];
-                fold_one(x, aL, aR, inv_t, acc, bb);
-            }
-            LAPSUM_STAGE(bb, x);
+            const float xs[1] = {i < n ? r[i] : 0.f};
+            uint32_t m = 0u;
+            classify(xs[0], i < n, m, 0);
+            if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 1);
         }
     }
-#undef LAPSUM_STAGE
+    while (tail != head) drain((int)min(32u, tail - head));
+    acc.cntR += far_right;
+    acc.bad |= bad;
     __syncthreads();
     band_flush(sband, scount, band, counter, cap, BL, inv_t, bins, &gbase);
     const long long cR = block_sum_ll((long long)acc.cntR, lred);

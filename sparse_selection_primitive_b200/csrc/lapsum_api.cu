@@ -40,7 +40,7 @@ int resolve_path(int64_t n, int path) {
 }
 
 struct Layout {
-    size_t header, rows, partials, row_R, tickets;
+    size_t header, rows, partials, row_R, tickets, wlist, wtab, wflag;
     size_t keys0, keys1, seg_hist, tile_hist, plan;
     size_t sample, band0, band1, bins, fold_part, fold_ticket;
     size_t total;
@@ -61,8 +61,14 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
     L.tickets = take((size_t)B * 2 * sizeof(uint32_t) + (2 + 2048) * sizeof(uint32_t));
     L.fold_ticket = L.tickets + (size_t)B * 2 * sizeof(uint32_t);
     L.rows = take((size_t)B * 512);
-    L.partials = take((size_t)B * (size_t)tiles * 3 * sizeof(double));
+    L.partials = take((size_t)B * (size_t)tiles * 4 * sizeof(double));
     L.row_R = take((size_t)B * sizeof(double));
+    if (n > kOnchipMax) {  // windowed backward of long rows
+        // the pass CTAs of a row split the capacity evenly (rounded up per CTA)
+        L.wlist = take((size_t)B * ((size_t)window_capacity(n) + 8192) * sizeof(WinEntry));
+        L.wtab = take((size_t)B * (size_t)window_tiles(n) * sizeof(uint2));
+        L.wflag = take((size_t)B * sizeof(uint32_t));
+    }
     if (rpath == LAPSUM_PATH_RADIX) {
         const int64_t rt = radix_tiles(n);
         L.keys0 = take((size_t)B * (size_t)n * sizeof(uint32_t));
@@ -315,8 +321,8 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
     for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
         const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
         e = launch_emit(r + r0 * ld, ld, p + r0 * ld, b + r0, sum_f ? sum_f + r0 : nullptr, nb, n,
-                        t, partials + r0 * stream_tiles(n), tickets + r0, vec,
-                        r0 == 0 ? hdr : nullptr, B, rp, st);
+                        t, partials + r0 * stream_tiles(n), tickets + r0, vec, hdr, r0 == 0 ? 1 : 0,
+                        B, rp, st);
     }
     return cuda_status(e);
 }
@@ -339,11 +345,22 @@ int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v,
     double* partials = reinterpret_cast<double*>(w + L.partials);
     double* row_R = reinterpret_cast<double*>(w + L.row_R);
     cudaError_t e = cudaSuccess;
+    const bool windowed = n <= (int64_t)0xffffffffll;  // window entries index rows with 32 bits
     for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
         const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
-        e = launch_backward_stream(r + r0 * ld, ld, b + r0, v + r0 * ld, g + r0 * ld, nb, n, t,
-                                   partials + r0 * stream_tiles(n) * 3, row_R + r0,
-                                   tickets + B + r0, vec, st);
+        if (windowed) {
+            WindowBuffers wb;
+            wb.list = reinterpret_cast<WinEntry*>(w + L.wlist);
+            wb.tab = reinterpret_cast<uint2*>(w + L.wtab) + r0 * window_tiles(n);
+            wb.flag = reinterpret_cast<uint32_t*>(w + L.wflag) + r0;
+            e = launch_backward_window(r + r0 * ld, ld, b + r0, v + r0 * ld, g + r0 * ld, nb, n,
+                                       t, wb, partials + r0 * stream_tiles(n) * 4, row_R + r0,
+                                       tickets + B + r0, vec, st);
+        } else {
+            e = launch_backward_stream(r + r0 * ld, ld, b + r0, v + r0 * ld, g + r0 * ld, nb, n,
+                                       t, partials + r0 * stream_tiles(n) * 4, row_R + r0,
+                                       tickets + B + r0, vec, st);
+        }
     }
     return cuda_status(e);
 }

@@ -101,8 +101,19 @@ __device__ __forceinline__ float scaled_margin(float r, const Thr& h) {
     return __fmul_rn(__fsub_rn(__fsub_rn(r, h.hi), h.lo), h.inv_t);
 }
 
+// 2^y with flush-to-zero for results below the smallest normal float (the
+// hardware ex2 approximation; about 2 ulp).  Flushing is harmless here: every
+// exponential feeds a probability, a weight or a sum in which a term below
+// 1.2e-38 is negligible.
+__device__ __forceinline__ float ex2_ftz(float y) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+    return r;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 // e = exp(-|x|); p = sigma(x) = x < 0 ? e/2 : 1 - e/2; f = e/2.  One exp.
-__device__ __forceinline__ float neg_abs_exp(float x) { return __expf(-fabsf(x)); }
+__device__ __forceinline__ float neg_abs_exp(float x) { return ex2_ftz(-fabsf(x) * kLog2e); }
 __device__ __forceinline__ float cdf_from(float x, float e) { return x < 0.f ? 0.5f * e : 1.f - 0.5f * e; }
 
 // Gap factor e^{(lo - hi)/t} between two neighbouring sorted scores lo <= hi.

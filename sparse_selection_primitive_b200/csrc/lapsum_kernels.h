@@ -47,13 +47,38 @@ cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int6
 constexpr int kStreamTile = 4096;  // elements per CTA tile of the streaming kernels
 int64_t stream_tiles(int64_t n);
 // p = sigma((r - b)/t) and sum f per row; partials: [B][tiles] doubles.
-cudaError_t launch_emit(const float* r, int64_t ld, float* p, const double* b, double* sumf,
+cudaError_t launch_emit(const float* r, int64_t ld, float* p, double* b, double* sumf,
                         int64_t B, int64_t n, double t, double* partials, uint32_t* tickets,
-                        int vec, WsHeader* hdr, int64_t B_total, int path_code, cudaStream_t st);
+                        int vec, WsHeader* hdr, int record_call, int64_t B_total, int path_code,
+                        cudaStream_t st);
 // Backward for long rows: reduce (mu, sum w, sum w v) per row, then g.
+// partials: 4 doubles per CTA record.
 cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, const float* v,
                                    float* g, int64_t B, int64_t n, double t, double* partials,
                                    double* row_R, uint32_t* tickets, int vec, cudaStream_t st);
+// Same, but rows with need[row] == 0 are skipped by every CTA (need on the device).
+cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* b,
+                                      const float* v, float* g, int64_t B, int64_t n, double t,
+                                      double* partials, double* row_R, uint32_t* tickets, int vec,
+                                      const uint32_t* need, cudaStream_t st);
+
+// --- windowed backward (scores with |x| <= 90 only) ----------------------------
+struct WinEntry {
+    uint32_t idx;  // position in the row
+    float x;       // (r - b)/t
+    float v;       // upstream gradient
+};
+struct WindowBuffers {
+    WinEntry* list;   // [B][window_capacity(n)], split evenly between the pass CTAs
+    uint2* tab;       // [B][window_tiles(n)]: (start, count) of each tile's entries
+    uint32_t* flag;   // [B] 1 = the dense kernels recompute this row
+};
+uint32_t window_capacity(int64_t n);
+int64_t window_tiles(int64_t n);
+cudaError_t launch_backward_window(const float* r, int64_t ld, const double* b, const float* v,
+                                   float* g, int64_t B, int64_t n, double t,
+                                   const WindowBuffers& wb, double* partials, double* row_R,
+                                   uint32_t* tickets, int vec, cudaStream_t st);
 
 // --- probabilistic bracketing --------------------------------------------------
 constexpr int kSampleMax = 32768;

@@ -24,10 +24,10 @@ namespace {
 constexpr int kNoAllocRows = 1024;        // most rows per call
 constexpr int kNoAllocRecords = 4096;     // most per-CTA partial records per call
 constexpr int kNoAllocMaxDevices = 64;
-constexpr size_t kPartialBytes = (size_t)kNoAllocRecords * 3 * sizeof(double);
+constexpr size_t kPartialBytes = (size_t)kNoAllocRecords * 4 * sizeof(double);
 constexpr size_t kRowBytes = (size_t)kNoAllocRows * sizeof(double);
 constexpr size_t kTicketBytes = (size_t)kNoAllocRows * sizeof(uint32_t);
-constexpr size_t kScratchBytes = kPartialBytes + kRowBytes + kTicketBytes;  // 108 KiB
+constexpr size_t kScratchBytes = kPartialBytes + kRowBytes + kTicketBytes;  // 140 KiB
 
 // Shared by every call on a device; it keeps the contents of the last call.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];

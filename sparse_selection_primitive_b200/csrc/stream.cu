@@ -89,19 +89,22 @@ __device__ __forceinline__ bool last_block_of_row(uint32_t* ticket, uint32_t nbl
     return *flag != 0;
 }
 
-template <bool VEC>
+// p = sigma((r - b)/t) for one 4096-score tile per CTA; sum f per row when
+// asked for (per-tile partials, combined in tile order by the row's last CTA).
+// Full tiles take unchecked 16-byte accesses.
+template <bool VEC, bool SUMF>
 __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict__ r, int64_t ld,
                                                         float* __restrict__ p,
                                                         const double* __restrict__ b,
                                                         double* __restrict__ sumf, int64_t n,
                                                         double t, double* __restrict__ partials,
                                                         uint32_t* __restrict__ tickets,
-                                                        WsHeader* hdr, int64_t B_total,
-                                                        int path_code) {
+                                                        WsHeader* hdr, int record_call,
+                                                        int64_t B_total, int path_code) {
     __shared__ double red[kThreads / 32];
     __shared__ int flag;
     const int64_t row = blockIdx.y;
-    if (hdr != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    if (record_call && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         hdr->last_B = B_total;
         hdr->last_n = n;
         hdr->last_path = (uint32_t)path_code;
@@ -109,19 +112,40 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
     const int64_t tiles = gridDim.x;
     const int64_t base = (int64_t)blockIdx.x * kStreamTile;
     const Thr th = make_thr(b[row], t);
-    float x[kPer], y[kPer];
-    bool ok[kPer];
-    load_tile<VEC>(r + row * ld, n, base, x, ok);
+    const float* rr = r + row * ld;
+    float* pr = p + row * ld;
     double sf = 0.0;
+    if (VEC && base + kStreamTile <= n) {
+        const float4* r4 = reinterpret_cast<const float4*>(rr + base);
+        float4* p4 = reinterpret_cast<float4*>(pr + base);
+        float4 x[kPer / 4];
 #pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        const float xs = scaled_margin(x[q], th);
-        const float e = neg_abs_exp(xs);
-        y[q] = cdf_from(xs, e);
-        if (ok[q]) sf += 0.5 * (double)e;
+        for (int q = 0; q < kPer / 4; ++q) x[q] = __ldcs(r4 + q * kThreads + threadIdx.x);
+#pragma unroll
+        for (int q = 0; q < kPer / 4; ++q) {
+            const float m0 = scaled_margin(x[q].x, th), m1 = scaled_margin(x[q].y, th);
+            const float m2 = scaled_margin(x[q].z, th), m3 = scaled_margin(x[q].w, th);
+            const float e0 = neg_abs_exp(m0), e1 = neg_abs_exp(m1), e2 = neg_abs_exp(m2),
+                        e3 = neg_abs_exp(m3);
+            __stcs(p4 + q * kThreads + threadIdx.x,
+                   make_float4(cdf_from(m0, e0), cdf_from(m1, e1), cdf_from(m2, e2),
+                               cdf_from(m3, e3)));
+            if (SUMF) sf += 0.5 * (double)((e0 + e1) + (e2 + e3));
+        }
+    } else {
+        float x[kPer], y[kPer];
+        bool ok[kPer];
+        load_tile<VEC>(rr, n, base, x, ok);
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const float xs = scaled_margin(x[q], th);
+            const float e = neg_abs_exp(xs);
+            y[q] = cdf_from(xs, e);
+            if (SUMF && ok[q]) sf += 0.5 * (double)e;
+        }
+        store_tile<VEC>(pr, n, base, y);
     }
-    store_tile<VEC>(p + row * ld, n, base, y);
-    if (sumf == nullptr) return;
+    if (!SUMF) return;
     sf = block_sum_d(sf, red);
     if (threadIdx.x == 0) partials[row * tiles + blockIdx.x] = sf;
     if (last_block_of_row(&tickets[row], (uint32_t)tiles, &flag)) {
@@ -162,11 +186,13 @@ template <bool VEC>
 __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
     const float* __restrict__ v, int64_t n, double t, double* __restrict__ partials,
-    double* __restrict__ row_R, uint32_t* __restrict__ tickets) {
+    double* __restrict__ row_R, uint32_t* __restrict__ tickets,
+    const uint32_t* __restrict__ need) {
     __shared__ double red[kThreads / 32];
     __shared__ float fred[kThreads / 32];
     __shared__ int flag;
     const int64_t row = blockIdx.y;
+    if (need != nullptr && need[row] == 0u) return;  // the whole row skips
     const int64_t nblk = gridDim.x;
     const Thr th = make_thr(b[row], t);
     const float* rr = r + row * ld;
@@ -212,7 +238,7 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     s = block_sum_d(s * sc, red);
     sv = block_sum_d(sv * sc, red);
     if (threadIdx.x == 0) {
-        double* pr = partials + (row * nblk + blockIdx.x) * 3;
+        double* pr = partials + (row * nblk + blockIdx.x) * 4;
         pr[0] = (double)mb;
         pr[1] = s;
         pr[2] = sv;
@@ -220,11 +246,11 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     if (last_block_of_row(&tickets[row], (uint32_t)nblk, &flag)) {
         float mloc = INFINITY;
         for (int64_t i = threadIdx.x; i < nblk; i += kThreads)
-            mloc = fminf(mloc, (float)partials[(row * nblk + i) * 3]);
+            mloc = fminf(mloc, (float)partials[(row * nblk + i) * 4]);
         const double mrow = (double)block_min_f(mloc, fred);
         double a = 0.0, av = 0.0;
         for (int64_t i = threadIdx.x; i < nblk; i += kThreads) {
-            const double* pr = partials + (row * nblk + i) * 3;
+            const double* pr = partials + (row * nblk + i) * 4;
             if (pr[0] == INFINITY) continue;
             const double f = exp(mrow - pr[0]);
             a += pr[1] * f;
@@ -236,54 +262,60 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     }
 }
 
+// Pass 2 of the VJP: g = (f/t)(v - R), persistent CTAs striding over tiles.
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) bwd_apply_kernel(
     const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
     const float* __restrict__ v, float* __restrict__ g, int64_t n, double t,
-    const double* __restrict__ row_R) {
+    const double* __restrict__ row_R, const uint32_t* __restrict__ need) {
     const int64_t row = blockIdx.y;
-    const int64_t base = (int64_t)blockIdx.x * kStreamTile;
+    if (need != nullptr && need[row] == 0u) return;
     const Thr th = make_thr(b[row], t);
     const double R = row_R[row];
-    float x[kPer], vv[kPer], y[kPer];
-    bool ok[kPer];
-    load_tile<VEC>(r + row * ld, n, base, x, ok);
-    load_tile<VEC>(v + row * ld, n, base, vv, ok);
+    const int64_t tiles = (n + kStreamTile - 1) / kStreamTile;
+    for (int64_t T = blockIdx.x; T < tiles; T += gridDim.x) {
+        const int64_t base = T * kStreamTile;
+        float x[kPer], vv[kPer], y[kPer];
+        bool ok[kPer];
+        load_tile<VEC>(r + row * ld, n, base, x, ok);
+        load_tile<VEC>(v + row * ld, n, base, vv, ok);
 #pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-        const float f = 0.5f * neg_abs_exp(scaled_margin(x[q], th));
-        y[q] = f * th.inv_t * (float)((double)vv[q] - R);
+        for (int q = 0; q < kPer; ++q) {
+            const float f = 0.5f * neg_abs_exp(scaled_margin(x[q], th));
+            y[q] = f * th.inv_t * (float)((double)vv[q] - R);
+        }
+        store_tile<VEC>(g + row * ld, n, base, y);
     }
-    store_tile<VEC>(g + row * ld, n, base, y);
 }
 
 }  // namespace
 
 int64_t stream_tiles(int64_t n) { return (n + kStreamTile - 1) / kStreamTile; }
 
-cudaError_t launch_emit(const float* r, int64_t ld, float* p, const double* b, double* sumf,
+cudaError_t launch_emit(const float* r, int64_t ld, float* p, double* b, double* sumf,
                         int64_t B, int64_t n, double t, double* partials, uint32_t* tickets,
-                        int vec, WsHeader* hdr, int64_t B_total, int path_code, cudaStream_t st) {
+                        int vec, WsHeader* hdr, int record_call, int64_t B_total, int path_code,
+                        cudaStream_t st) {
     const dim3 grid((unsigned)stream_tiles(n), (unsigned)B);
-    if (vec)
-        {
-            ProfScope ps_("emit", st);
-            emit_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets,
-                                                     hdr, B_total, path_code);
-        }
-    else
-        {
-            ProfScope ps_("emit", st);
-            emit_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets,
-                                                      hdr, B_total, path_code);
-        }
+    ProfScope ps_("emit", st);
+#define LAPSUM_EMIT(V, S)                                                                     \
+    emit_kernel<V, S><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets, hdr, \
+                                                 record_call, B_total, path_code)
+    if (vec) {
+        if (sumf) LAPSUM_EMIT(true, true);
+        else LAPSUM_EMIT(true, false);
+    } else {
+        if (sumf) LAPSUM_EMIT(false, true);
+        else LAPSUM_EMIT(false, false);
+    }
+#undef LAPSUM_EMIT
     return cudaGetLastError();
 }
 
-cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, const float* v,
-                                   float* g, int64_t B, int64_t n, double t, double* partials,
-                                   double* row_R, uint32_t* tickets, int vec, cudaStream_t st) {
-    const dim3 grid((unsigned)stream_tiles(n), (unsigned)B);
+cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* b,
+                                      const float* v, float* g, int64_t B, int64_t n, double t,
+                                      double* partials, double* row_R, uint32_t* tickets, int vec,
+                                      const uint32_t* need, cudaStream_t st) {
     // pass 1 runs persistent CTAs: about 8 per SM over all rows, at most one per tile
     static int sms = 0;
     if (sms == 0) {
@@ -295,28 +327,41 @@ cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, 
     if (per_row > stream_tiles(n)) per_row = stream_tiles(n);
     if (per_row < 1) per_row = 1;
     const dim3 rgrid((unsigned)per_row, (unsigned)B);
+    int64_t apply_row = ((int64_t)sms * 16 + B - 1) / B;
+    if (apply_row > stream_tiles(n)) apply_row = stream_tiles(n);
+    if (apply_row < 1) apply_row = 1;
+    const dim3 grid_apply((unsigned)apply_row, (unsigned)B);
     if (vec) {
         {
             ProfScope ps_("bwd_reduce", st);
             bwd_reduce_kernel<true><<<rgrid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
-                                                           tickets);
+                                                                tickets, need);
         }
         {
             ProfScope ps_("bwd_apply", st);
-            bwd_apply_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R);
+            bwd_apply_kernel<true><<<grid_apply, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R,
+                                                                    need);
         }
     } else {
         {
             ProfScope ps_("bwd_reduce", st);
-            bwd_reduce_kernel<false><<<rgrid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
-                                                            tickets);
+            bwd_reduce_kernel<false><<<rgrid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials,
+                                                                 row_R, tickets, need);
         }
         {
             ProfScope ps_("bwd_apply", st);
-            bwd_apply_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R);
+            bwd_apply_kernel<false><<<grid_apply, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R,
+                                                                     need);
         }
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, const float* v,
+                                   float* g, int64_t B, int64_t n, double t, double* partials,
+                                   double* row_R, uint32_t* tickets, int vec, cudaStream_t st) {
+    return launch_backward_stream_if(r, ld, b, v, g, B, n, t, partials, row_R, tickets, vec,
+                                     nullptr, st);
 }
 
 }  // namespace lapsum

@@ -167,3 +167,27 @@ def test_repeat_calls_are_deterministic(cuda_device):
         assert np.array_equal(a["b"], c["b"]), path
         assert np.array_equal(a["p"], c["p"]), path
         assert np.array_equal(a["g"], c["g"]), path
+
+
+# ---------------------------------------------------------------------------
+# Windowed backward of long rows: only |x| <= 90 carries gradient in fp32.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n,k,t,dist", [
+    (1 << 20, 1000.0, 0.001, "normal"),     # window ~4% of the row: served by the window pass
+    (1 << 18, 2000.0, 0.05, "normal"),      # window holds the whole row: list overflow, dense
+    (300001, 77.0, 0.0004, "mix_nu"),       # odd length, scalar tail of the window pass
+])
+def test_windowed_backward(cuda_device, n, k, t, dist):
+    r, v = random_rows(51, 1, n, dist)
+    out = run_gpu(r, k, t, path="radix" if n <= (1 << 20) else "bracket", v=v)
+    check_row(r[0], v[0], k, t, out["b"][0], out["p"][0], out["g"][0], label=f"window n={n}")
+
+
+def test_windowed_backward_far_threshold_falls_back(cuda_device):
+    # gap 1 and t = 0.008: the nearest scores sit at |x| = 62.5, inside the
+    # window but above 50, so the row is recomputed by the dense kernels
+    n = 6000
+    r = np.random.default_rng(4).permutation(n).astype(np.float32)[None, :]
+    v = np.random.default_rng(5).standard_normal((1, n)).astype(np.float32)
+    out = run_gpu(r, 17.0, 0.008, path="radix", v=v)
+    check_row(r[0], v[0], 17.0, 0.008, out["b"][0], out["p"][0], out["g"][0], label="far")
