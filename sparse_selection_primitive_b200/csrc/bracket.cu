@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
     __syncthreads();
     if (!flag) return;
     __threadfence();
+    phase_mark(st, 0);
     for (int i = threadIdx.x; i < 2048; i += kBlk) {
         hist[i] = __ldcg(ghist + i);
         ghist[i] = 0u;  // ready for the next call
@@ -287,6 +288,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
             aL = from_key(kk);
         }
     }
+    phase_mark(st, 1);
     if (force_miss) {
         uint32_t kmax = 0;
         for (int s = threadIdx.x; s < m; s += kBlk) kmax = max(kmax, to_key(__ldcg(sample_out + s)));
@@ -961,14 +963,24 @@ __device__ long long extract_bin(const float* __restrict__ band, long long nb, c
     __syncthreads();
     const long long n4 = nb >> 2;
     const float4* b4 = reinterpret_cast<const float4*>(band);
-    for (long long i = threadIdx.x; i < n4; i += blockDim.x) {
-        const float4 v = b4[i];
-        const float xs[4] = {v.x, v.y, v.z, v.w};
+    // eight 16-byte loads per thread in flight per trip (the band sits in L2)
+    constexpr int G = 8;
+    for (long long i0 = 0; i0 < n4; i0 += (long long)G * blockDim.x) {
+        float4 v[G];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            if (bin_of(BL, to_key(xs[q])) == j) {
-                const unsigned long long pos = atomicAdd(&sm->cnt, 1ull);
-                if (pos < (unsigned long long)kBandSortMax) sm->u.sort.sorted[pos] = xs[q];
+        for (int g = 0; g < G; ++g) {
+            const long long i = i0 + (long long)g * blockDim.x + threadIdx.x;
+            v[g] = i < n4 ? __ldcg(b4 + i) : make_float4(NAN, NAN, NAN, NAN);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float xs[4] = {v[g].x, v[g].y, v[g].z, v[g].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (xs[q] == xs[q] && bin_of(BL, to_key(xs[q])) == j) {
+                    const unsigned long long pos = atomicAdd(&sm->cnt, 1ull);
+                    if (pos < (unsigned long long)kBandSortMax) sm->u.sort.sorted[pos] = xs[q];
+                }
             }
         }
     }
@@ -992,7 +1004,8 @@ __device__ long long extract_bin(const float* __restrict__ band, long long nb, c
 // narrowing path).
 __device__ int solve_with_bins(const float* __restrict__ band, long long nb,
                                const unsigned long long* __restrict__ bins, const BinLayout& BL,
-                               const Tails& tl, double k, double t, SolveSmemAll* sm) {
+                               const Tails& tl, double k, double t, SolveSmemAll* sm,
+                               RowState* probe) {
     const int cntF = bin_scan(BL, bins, tl, k, t, sm, -1);
     const double FL = tl.hasL ? sm->binF[0] : INFINITY;
     const double FR = tl.hasR ? sm->binF[1] : -INFINITY;
@@ -1012,9 +1025,12 @@ __device__ int solve_with_bins(const float* __restrict__ band, long long nb,
         __syncthreads();
         bin_scan(BL, bins, tl, k, t, sm, jc);
         if ((long long)bins[jc] > kBandSortMax) return -1;
+        if (probe) phase_mark(probe, 6 + 3 * min(guard, 1));
         const long long c = extract_bin(band, nb, BL, jc, sm);
+        if (probe) phase_mark(probe, 7 + 3 * min(guard, 1));
         Tails sub = sm->sub;
         solve_small_band(sm->u.sort.sorted, c, sub, k, t, sm);
+        if (probe) phase_mark(probe, 8 + 3 * min(guard, 1));
         if (sm->res.F_aL < k && jc > 0) {
             --jc;
         } else if (sm->res.F_aR > k && jc < BL.nbin - 1) {
@@ -1024,6 +1040,82 @@ __device__ int solve_with_bins(const float* __restrict__ band, long long nb,
         }
     }
     return -1;
+}
+
+// Exact solve of a band too large for the on-chip sort: certify the bracket,
+// then narrow by key histograms (ping-ponging between cur and nxt) until the
+// band fits on chip or holds a single value.  Returns 1 (solved, b in
+// sm->res), 0 (the bracket failed: F at the ends in sm->res) or -1 (no bin
+// certified while narrowing; not expected, reported as a failure).
+__device__ int solve_exact(float* cur, float* nxt, long long nb, Tails tl, double k,
+                           double t, SolveSmemAll* sm, int* levels) {
+    double FL, FR;
+    uint32_t kmin, kmax;
+    certify_big_band(cur, nb, tl, t, sm, &FL, &FR, &kmin, &kmax);
+    if (!(FL >= k && FR <= k)) {
+        // F at the ends is enough to know which end failed
+        if (threadIdx.x == 0) {
+            sm->res.F_aL = FL;
+            sm->res.F_aR = FR;
+        }
+        __syncthreads();
+        return 0;
+    }
+    while (nb > kBandSortMax && kmin < kmax) {
+        uint32_t nkmin = 0, nkmax = 0;
+        nb = refine_level(cur, nb, nxt, tl, kmin, kmax, k, t, sm, &nkmin, &nkmax);
+        if (nb < 0) return -1;
+        ++*levels;
+        float* tmp = cur;
+        cur = nxt;
+        nxt = tmp;
+        kmin = nkmin;
+        kmax = nkmax;
+    }
+    if (nb <= kBandSortMax)
+        solve_small_band(cur, nb, tl, k, t, sm);
+    else
+        solve_sorted_block(ConstGet{from_key(kmin)}, nb, tl, k, t, &sm->ss, &sm->res);
+    return 1;
+}
+
+// First half of the histogram solve: certify the bracket from the bin sums and
+// choose the bin whose edges straddle k, leaving its tails in the row record
+// for the extract and final solve kernels.  Returns 1 (bin chosen), 0 (the
+// bracket failed: F at the ends in sm->res) or -1 (that bin is too full for
+// the on-chip sort: use the exact narrowing path).
+__device__ int plan_with_bins(const unsigned long long* __restrict__ bins, const BinLayout& BL,
+                              const Tails& tl, double k, double t, SolveSmemAll* sm,
+                              RowState* st) {
+    const int cntF = bin_scan(BL, bins, tl, k, t, sm, -1);
+    const double FL = tl.hasL ? sm->binF[0] : INFINITY;
+    const double FR = tl.hasR ? sm->binF[1] : -INFINITY;
+    if (!(FL >= k && FR <= k)) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            sm->res.F_aL = FL;
+            sm->res.F_aR = FR;
+        }
+        __syncthreads();
+        return 0;
+    }
+    int jc = cntF - 1;
+    if (jc < 0) jc = 0;
+    if (jc > BL.nbin - 1) jc = BL.nbin - 1;
+    __syncthreads();
+    bin_scan(BL, bins, tl, k, t, sm, jc);
+    if ((long long)bins[jc] > kBandSortMax) return -1;
+    if (threadIdx.x == 0) {
+        st->sub_bin = jc;
+        st->sub_aL = sm->sub.aL;
+        st->sub_aR = sm->sub.aR;
+        st->sub_hasR = sm->sub.hasR ? 1 : 0;
+        st->sub_SL = sm->sub.SL;
+        st->sub_SR = sm->sub.SR;
+        st->sub_cntR = sm->sub.cntR;
+        st->n_sub = 0ull;
+    }
+    return 1;
 }
 
 // Single-CTA fold of the whole row (used only after a failed bracket).
@@ -1068,6 +1160,7 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
                                                      WsHeader* hdr) {
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    phase_mark(st, 2);
     if (threadIdx.x == 0) {
         sm->bcast[2] = 0xffffffffu;
         sm->bcast[3] = 0u;
@@ -1105,13 +1198,19 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
         nb_cert = nb;
         int via_bins = -1;
         if (nb > kBandSortMax && attempt == 1) {
-            // the fold built the band histogram for this first bracket
+            // the fold built the band histogram for this first bracket; the
+            // chosen bin is extracted and solved by the next two kernels
             const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
-            via_bins = solve_with_bins(cur, nb, bins, BL, tl, k, t, sm);
+            via_bins = plan_with_bins(bins, BL, tl, k, t, sm, st);
             if (via_bins == 1) {
-                b = sm->res.b;
-                done = true;
-                certified = true;
+                phase_mark(st, 3);
+                if (threadIdx.x == 0) {
+                    st->stage = 1;
+                    st->attempts = attempt;
+                    st->refine_levels = 0;
+                    st->certified = 1;
+                }
+                return;
             } else if (via_bins == 0) {
                 certified = false;
             }
@@ -1126,40 +1225,12 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
                 done = true;
             }
         } else {
-            double FL, FR;
-            uint32_t kmin, kmax;
-            certify_big_band(cur, nb, tl, t, sm, &FL, &FR, &kmin, &kmax);
-            certified = FL >= k && FR <= k;
-            if (certified) {
-                // narrow until the band fits on chip or holds a single value
-                while (nb > kBandSortMax && kmin < kmax) {
-                    uint32_t nkmin = 0, nkmax = 0;
-                    nb = refine_level(cur, nb, nxt, tl, kmin, kmax, k, t, sm, &nkmin, &nkmax);
-                    if (nb < 0) break;  // no certified bin (not expected): reported as a failure
-                    ++levels;
-                    float* tmp = cur;
-                    cur = nxt;
-                    nxt = tmp;
-                    kmin = nkmin;
-                    kmax = nkmax;
-                }
-                if (nb < 0) {
-                    certified = false;
-                    break;
-                } else if (nb <= kBandSortMax) {
-                    solve_small_band(cur, nb, tl, k, t, sm);
-                } else {
-                    solve_sorted_block(ConstGet{from_key(kmin)}, nb, tl, k, t, &sm->ss, &sm->res);
-                }
+            const int e = solve_exact(cur, nxt, nb, tl, k, t, sm, &levels);
+            certified = e != 0;
+            if (e < 0) break;
+            if (e > 0) {
                 b = sm->res.b;
                 done = true;
-            } else {
-                // F at the ends is enough to know which end failed
-                if (threadIdx.x == 0) {
-                    sm->res.F_aL = FL;
-                    sm->res.F_aR = FR;
-                }
-                __syncthreads();
             }
         }
         if (done || attempt >= max_attempts) break;
@@ -1188,6 +1259,7 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
         ++attempt;
         refold_row(r, n, aL, aR, t, band0, sm, tl, &nb);
     }
+    phase_mark(st, 12);
     if (threadIdx.x == 0) {
         st->attempts = attempt;
         st->refine_levels = levels;
@@ -1203,6 +1275,109 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
         if (!done) {
             b = nan("");
             st->status |= kDevBracketExhausted;
+            set_status(hdr, kDevBracketExhausted);
+        }
+        st->b = b;
+        *b_out = b;
+    }
+}
+
+// Scores of the chosen histogram bin, gathered from the band by the whole
+// grid (the band is large; the bin holds at most 4096 scores).
+__global__ void __launch_bounds__(256) extract_kernel(const float* __restrict__ band,
+                                                      RowState* st, float* __restrict__ sub) {
+    if (st->stage != 1) return;
+    const long long nb = (long long)st->n_band;
+    const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
+    const int j = st->sub_bin;
+    const long long n4 = nb >> 2;
+    const float4* b4 = reinterpret_cast<const float4*>(band);
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const int lane = threadIdx.x & 31;
+    auto take = [&](bool hit, float x) {
+        const unsigned ball = __ballot_sync(0xffffffffu, hit);
+        if (ball == 0u) return;
+        const int leader = __ffs(ball) - 1;
+        unsigned long long base = 0;
+        if (lane == leader) base = atomicAdd(&st->n_sub, (unsigned long long)__popc(ball));
+        base = __shfl_sync(0xffffffffu, base, leader);
+        const unsigned long long pos = base + __popc(ball & ((1u << lane) - 1u));
+        if (hit && pos < (unsigned long long)kBandSortMax) sub[pos] = x;
+    };
+    const long long trips = (n4 + stride - 1) / stride;  // same in every lane
+    for (long long tr = 0; tr < trips; ++tr) {
+        const long long i = tr * stride + (long long)blockIdx.x * blockDim.x + threadIdx.x;
+        const bool ok = i < n4;
+        const float4 v = ok ? __ldcg(b4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        take(ok && bin_of(BL, to_key(v.x)) == j, v.x);
+        take(ok && bin_of(BL, to_key(v.y)) == j, v.y);
+        take(ok && bin_of(BL, to_key(v.z)) == j, v.z);
+        take(ok && bin_of(BL, to_key(v.w)) == j, v.w);
+    }
+    if (blockIdx.x == 0 && threadIdx.x < 32) {
+        const long long i = (n4 << 2) + threadIdx.x;
+        const bool ok = i < nb;
+        const float x = ok ? band[i] : 0.f;
+        take(ok && bin_of(BL, to_key(x)) == j, x);
+    }
+}
+
+// Exact solve on the extracted bin with the rest of the row folded into its
+// tails.  If rounding in the fixed-point histogram chose the wrong bin (its own
+// end check fails), the single-CTA histogram solve walks to the right one.
+__global__ void __launch_bounds__(kBlk) solve2_kernel(double k, double t, RowState* st,
+                                                      float* __restrict__ band0,
+                                                      float* __restrict__ sub,
+                                                      const unsigned long long* __restrict__ bins,
+                                                      double* __restrict__ b_out, WsHeader* hdr) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    if (st->stage != 1) return;
+    phase_mark(st, 4);
+    const long long ns = (long long)st->n_sub;
+    Tails s;
+    s.hasL = true;
+    s.aL = st->sub_aL;
+    s.SL = st->sub_SL;
+    s.hasR = st->sub_hasR != 0;
+    s.aR = st->sub_aR;
+    s.SR = st->sub_SR;
+    s.cntR = st->sub_cntR;
+    double b = nan("");
+    bool ok = false;
+    if (ns <= kBandSortMax) {
+        solve_small_band(sub, ns, s, k, t, sm);
+        ok = sm->res.F_aL >= k && sm->res.F_aR <= k;
+        b = sm->res.b;
+    }
+    phase_mark(st, 5);
+    if (!ok) {
+        Tails tl;
+        tl.hasL = isfinite(st->a_L);
+        tl.aL = st->a_L;
+        tl.SL = st->S_L;
+        tl.hasR = isfinite(st->a_R);
+        tl.aR = st->a_R;
+        tl.SR = st->S_R;
+        tl.cntR = (double)st->cnt_R;
+        const long long nb = (long long)st->n_band;
+        const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
+        int v = solve_with_bins(band0, nb, bins, BL, tl, k, t, sm, nullptr);
+        if (v < 0) {
+            // a neighbouring bin too full for the on-chip sort: exact narrowing,
+            // with the extracted bin's buffer as the second band
+            int levels = 0;
+            v = solve_exact(band0, sub, nb, tl, k, t, sm, &levels);
+            if (threadIdx.x == 0) st->refine_levels = levels;
+        }
+        b = v == 1 ? sm->res.b : nan("");
+        ok = v == 1;
+    }
+    if (threadIdx.x == 0) {
+        st->stage = 0;
+        if (!ok) {
+            st->status |= kDevBracketExhausted;
+            st->certified = 0;
             set_status(hdr, kDevBracketExhausted);
         }
         st->b = b;
@@ -1234,6 +1409,8 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     if (!attr_done) {
         cudaFuncSetAttribute(solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)solve_smem);
+        cudaFuncSetAttribute(solve2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)solve_smem);
         cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(2 * kBandSortMax * sizeof(uint32_t)));
         attr_done = true;
@@ -1264,6 +1441,16 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
         ProfScope ps_("bracket_solve", st);
         solve_kernel<<<1, kBlk, solve_smem, st>>>(r_row, n, k, t, st_row, buf.band[0], buf.band[1],
                                               buf.bins, sample, m, lad, b_out, hdr);
+    }
+    {
+        ProfScope ps_("bracket_extract", st);
+        extract_kernel<<<bracket_fold_grid() / 2 > 0 ? bracket_fold_grid() / 2 : 1, 256, 0, st>>>(
+            buf.band[0], st_row, buf.band[1]);
+    }
+    {
+        ProfScope ps_("bracket_solve2", st);
+        solve2_kernel<<<1, kBlk, solve_smem, st>>>(k, t, st_row, buf.band[0], buf.band[1],
+                                                   buf.bins, b_out, hdr);
     }
     return cudaGetLastError();
 }

@@ -63,7 +63,13 @@ struct RowState {
     float ladder_L[kLadder];  // a_L rungs (descending ranks h, 4h, 16h, open)
     float ladder_R[kLadder];  // a_R rungs (ranks l, l/4, l/16, open)
     uint32_t bin_kmin, bin_kmax;  // key range of the band histogram of the current bracket
-    double scratch[39];       // kernel-to-kernel scalars
+    int32_t stage;            // 1: the histogram bin `sub_bin` is left for extract + solve2
+    int32_t sub_bin;
+    unsigned long long n_sub;  // scores extracted from that bin
+    float sub_aL, sub_aR;      // sub-bracket [sub_aL, sub_aR) = that bin's edges
+    int32_t sub_hasR, pad1;
+    double sub_SL, sub_SR, sub_cntR;  // tails of the sub-bracket
+    double scratch[32];       // kernel-to-kernel scalars (phase timestamps)
 };
 static_assert(sizeof(RowState) <= 512, "row record fits its slot");
 
@@ -388,6 +394,16 @@ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t c) {
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
     z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
     return z ^ (z >> 31);
+}
+
+// Phase timestamps (ns, global timer) of the single-CTA bracketing steps, kept
+// in the row record's scratch words for diagnostics.
+__device__ __forceinline__ void phase_mark(RowState* st, int slot) {
+    if (threadIdx.x == 0) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        reinterpret_cast<unsigned long long*>(st->scratch)[slot] = t;
+    }
 }
 
 __device__ __forceinline__ void set_status(WsHeader* hdr, uint32_t bits) {
