@@ -51,6 +51,9 @@ KERNEL_BYTES_PER_ELEMENT = {
     "bwd_reduce": 8,      # read r, v
     "bwd_apply": 12,      # read r, v, write g
     "bracket_fold": 4,    # read r
+    "sup_write": 4,       # write g (plus the support list, counted per entry elsewhere)
+    "window_pass": 4,     # read r (v only inside the window)
+    "window_write": 4,    # write g
     "radix_prep": 8,      # read r, write keys
     "radix_upsweep": 4,   # read keys (per pass)
     "radix_downsweep": 8,  # read keys, write keys (per pass)
@@ -251,13 +254,19 @@ def main():
         gd = torch.empty_like(rd)
         bd = torch.empty(w.B, dtype=torch.float64, device=dev)
         ws = L.Workspace(w.B, w.n, w.k, "auto", dev)
+        # rows longer than 4096 hand the gradient support from forward to
+        # backward, as the autograd wrapper does
+        sup = L.Support(w.B, w.n, dev) if L.support_bytes(w.B, w.n) > 0 else None
         working = 4 * rd.numel() * 4
         flush = working < 2 * l2_bytes
 
         def fwd():
-            L.forward(rd, w.k, w.t, ws=ws, p=pd, b=bd)
+            L.forward(rd, w.k, w.t, ws=ws, p=pd, b=bd, support=sup)
 
         def bwd():
+            L.backward(rd, bd, vd, w.t, ws=ws, g=gd, support=sup)
+
+        def bwd_plain():
             L.backward(rd, bd, vd, w.t, ws=ws, g=gd)
 
         def timed(fn, k_steps, profile=False):
@@ -297,7 +306,8 @@ def main():
             bwd()
         torch.cuda.synchronize(dev)
         res = {"flush": flush, "ws": ws, "rd": rd, "vd": vd, "pd": pd, "gd": gd, "bd": bd,
-               "fwd": fwd, "bwd": bwd, "timed": timed, "graph": graph}
+               "fwd": fwd, "bwd": bwd, "timed": timed, "graph": graph, "sup": sup}
+        res["near"] = support_count(r_h, bd.cpu().numpy(), w.t) if sup is not None else 0
         if w.path == "bracket":
             info = L.row_info(ws, 0)
             res["bracket"] = {key: info[key] for key in ("attempts", "n_band", "refine_levels",
@@ -310,6 +320,9 @@ def main():
             res["table"] = {"fwd_ms": statistics.median(tf), "bwd_ms": statistics.median(tb),
                             "fwdbwd_ms": statistics.median(tfb),
                             "fwdbwd_graph_ms": statistics.median(tg)}
+            if sup is not None:
+                tp, _ = timed(bwd_plain, steps)
+                res["table"]["bwd_without_support_ms"] = statistics.median(tp)
         return res
 
     peak_gbs, peak_kind = load_peaks()
@@ -346,6 +359,8 @@ def main():
                 "launch_ms": per_launch_ms}
     step_bytes = STEP_BYTES_PER_ELEMENT[w.path] * w.elements
     step_gbs = step_bytes / (ms_local / 1e3) / 1e9
+    path_bytes = path_step_bytes(w, R["near"])
+    path_gbs = path_bytes / (ms_local / 1e3) / 1e9
     kernels = {k: {"launches": v[0], "total_ms": round(v[1], 4),
                    "share": round(v[1] / sum(x[1] for x in prof.values()), 4)}
                for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
@@ -410,6 +425,10 @@ def main():
                 / (T["fwdbwd_ms"] / 1e3) / 1e9,
             }
             table[name]["fwdbwd_frac_of_peak"] = table[name]["fwdbwd_algorithmic_gbs"] / peak_gbs
+            if "bwd_without_support_ms" in T:
+                table[name]["bwd_without_support_ms"] = round(T["bwd_without_support_ms"], 5)
+            table[name]["path_frac_of_peak"] = (path_step_bytes(wk, RW["near"])
+                                                / (T["fwdbwd_graph_ms"] / 1e3) / 1e9 / peak_gbs)
             if "bracket" in RW:
                 table[name]["bracket"] = RW["bracket"]
             del RW
@@ -435,6 +454,13 @@ def main():
             "eager_value": elements / (eager_ms_max / 1e3),
             "step_algorithmic_gbs": step_gbs,
             "step_frac_of_peak": step_gbs / peak_gbs,
+            "step_bytes_note": "step_* count the fixed per-element bytes of the method's two "
+                               "passes (fwd 12, bwd 20 B/score on long rows); path_* count what "
+                               "this path must move: r read by the fold, r read + p written by "
+                               "the emit, g written, plus 36 B per gradient-support entry",
+            "path_step_bytes": path_bytes,
+            "path_support_entries": R["near"],
+            "path_frac_of_peak": path_gbs / peak_gbs,
             "roofline": roofline,
             "kernels": kernels,
             "gpu_launches": gpu_launches,
@@ -447,6 +473,31 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def support_count(r_h, b_h, t):
+    """Scores with |r - b|/t <= 90 (the gradient support), summed over rows."""
+    import numpy as np
+    tot = 0
+    for i in range(r_h.shape[0]):
+        row = r_h[i]
+        for s0 in range(0, row.size, 1 << 24):
+            x = (row[s0:s0 + (1 << 24)].astype(np.float64) - float(b_h[i])) / t
+            tot += int(np.count_nonzero(np.abs(x) <= 90.0))
+    return tot
+
+
+def path_step_bytes(w, near):
+    """Bytes one fwd+bwd step of this library's path must move on workload w.
+
+    On-chip rows: r, p, r, v, g once (20 B/score).  Longer rows: r read by the
+    solve (radix prep or the bracketing fold; the radix passes are counted as
+    measured, not here), r read and p written by the emit, g written by the
+    backward, and per gradient-support entry 8 B listed + 8 B read back + 4 B
+    v + 4 B kept + 8 + 4 B read by the write pass = 36 B."""
+    if w.path == "bitonic":
+        return 20 * w.elements
+    return 16 * w.elements + 36 * near
 
 
 def read_traffic(kernel, workload):

@@ -114,6 +114,44 @@ int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v,
                     int64_t B, int64_t n, double t, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Gradient support: a forward-to-backward hand-over for rows with n > 4096.
+ * The pages define only the VJP itself (section 2.1); this pair is a layout
+ * choice of this library.  f_i = 0.5 exp(-|x_i|) is exactly 0 in fp32 once
+ * |x_i| = |r_i - b|/t exceeds 87.4, so only the scores with |x| <= 90 carry
+ * gradient.  lapsum_forward_support computes everything lapsum_forward does
+ * and, in the same pass that writes p, lists those scores (position and x)
+ * in the caller's `support` buffer.  lapsum_backward_support then produces
+ * the same g as lapsum_backward while reading v only at the listed scores and
+ * not reading r at all: its traffic is the g write plus the list.
+ *
+ * lapsum_support_bytes: size of `support` for B rows of n scores (0 when
+ * n <= 4096: those rows need no support and `support` may be NULL).  The
+ * buffer is owned by the caller, must be 256-byte aligned, needs no
+ * initialisation, and is written only by lapsum_forward_support (the backward
+ * also keeps the gathered v beside each entry).  It stays valid until the
+ * next forward into it; r and b must not change in between.
+ *
+ * The backward checks (on the device) that the list was written for the same
+ * n and B and for this b of each row, and that no list share overflowed (at
+ * most half of every 512 consecutive scores inside the window); rows that
+ * fail any check, or whose smallest |x| is above 50 (then scores outside the
+ * window could weigh in R), are recomputed from r and v by the dense
+ * kernels, so the result never depends on the list being usable.
+ * Errors: as lapsum_forward / lapsum_backward, plus LAPSUM_EWORKSPACE when
+ * n > 4096 and `support` is NULL, misaligned or smaller than
+ * lapsum_support_bytes(B, n).  The backward's `ws` is a lapsum_backward
+ * workspace (lapsum_backward_workspace_bytes).
+ */
+size_t lapsum_support_bytes(int64_t B, int64_t n);
+int lapsum_forward_support(const float* r, int64_t ld, float* p, double* b, double* sum_f,
+                           int64_t B, int64_t n, double k, double t, int path, uint64_t seed,
+                           void* ws, size_t ws_bytes, void* support, size_t support_bytes,
+                           void* stream);
+int lapsum_backward_support(const float* r, int64_t ld, const double* b, const float* v, float* g,
+                            int64_t B, int64_t n, double t, const void* support,
+                            size_t support_bytes, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Synchronises `stream`, copies the sticky device status word to
  * *device_status (LAPSUM_OK, or a LAPSUM_E* code for the first condition
  * seen) and clears it.  Returns LAPSUM_OK or LAPSUM_ECUDA.

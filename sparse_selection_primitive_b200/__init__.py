@@ -26,7 +26,8 @@ from . import _build
 __all__ = [
     "LapSumError", "Workspace", "forward", "backward", "read_status", "row_info", "sample_values",
     "workspace_bytes", "soft_topk", "LapSumTopK", "PATHS", "FLAG_FORCE_MISS", "FLAG_NO_RETRY",
-    "library_path", "profile_enable", "profile_read", "backward_noalloc",
+    "library_path", "profile_enable", "profile_read", "backward_noalloc", "Support",
+    "support_bytes",
 ]
 
 PATHS = {"auto": 0, "fullsort": 1, "bracket": 2, "radix": 3}
@@ -98,6 +99,17 @@ def _lib():
         lib.lapsum_profile_read.restype = ctypes.c_int
         lib.lapsum_profile_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int,
                                             ctypes.POINTER(ctypes.c_int)]
+        lib.lapsum_support_bytes.restype = ctypes.c_size_t
+        lib.lapsum_support_bytes.argtypes = [_c_i64, _c_i64]
+        lib.lapsum_forward_support.restype = ctypes.c_int
+        lib.lapsum_forward_support.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64,
+                                               ctypes.c_double, ctypes.c_double, ctypes.c_int,
+                                               ctypes.c_uint64, _vp, ctypes.c_size_t, _vp,
+                                               ctypes.c_size_t, _vp]
+        lib.lapsum_backward_support.restype = ctypes.c_int
+        lib.lapsum_backward_support.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64,
+                                                ctypes.c_double, _vp, ctypes.c_size_t, _vp,
+                                                ctypes.c_size_t, _vp]
         lib.lapsum_sample_get.restype = ctypes.c_int
         lib.lapsum_sample_get.argtypes = [_vp, _c_i64, _vp, _c_i64, _vp]
         _LIB = lib
@@ -150,6 +162,33 @@ class Workspace:
         return int(_lib().lapsum_backward_workspace_bytes(B, n)) <= self.nbytes
 
 
+def support_bytes(B: int, n: int) -> int:
+    return int(_lib().lapsum_support_bytes(B, n))
+
+
+class Support:
+    """Gradient-support buffer handed from forward to backward (rows with n > 4096).
+
+    The forward lists the scores with |r - b|/t <= 90 (the only ones with a
+    non-zero gradient in fp32); the backward then reads v only there and never
+    reads r.  Owned by torch (uint8, 256-byte aligned); no initialisation.
+    For n <= 4096 it holds no memory and the plain entry points run.
+    """
+
+    def __init__(self, B: int, n: int, device=None):
+        device = torch.device(device or "cuda")
+        self.B, self.n = B, n
+        self.nbytes = support_bytes(B, n)
+        self.buf = torch.empty(self.nbytes + 256 if self.nbytes else 0, dtype=torch.uint8,
+                               device=device)
+        base = self.buf.data_ptr()
+        self.ptr = (base + 255) // 256 * 256 if self.nbytes else None
+        self.device = device
+
+    def fits(self, B, n) -> bool:
+        return support_bytes(B, n) <= self.nbytes
+
+
 def _as_rows(x: torch.Tensor) -> torch.Tensor:
     if x.dim() == 1:
         x = x.unsqueeze(0)
@@ -183,8 +222,12 @@ def _check_out(out: torch.Tensor, ref: torch.Tensor, ld: int, what: str):
 
 
 def forward(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0, ws: Workspace = None,
-            want_sum_f: bool = False, p: torch.Tensor = None, b: torch.Tensor = None):
-    """Returns (p, b[, sum_f]) for each row of r (float32 CUDA, rows x n or n)."""
+            want_sum_f: bool = False, p: torch.Tensor = None, b: torch.Tensor = None,
+            support: Support = None):
+    """Returns (p, b[, sum_f]) for each row of r (float32 CUDA, rows x n or n).
+
+    With ``support`` (a Support for the same B, n) the forward also lists the
+    gradient support for backward(..., support=...)."""
     squeeze = r.dim() == 1
     r2 = _as_rows(r)
     B, n = r2.shape
@@ -202,18 +245,30 @@ def forward(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0, ws:
     elif b.dtype != torch.float64 or b.numel() != B or not b.is_contiguous():
         raise ValueError("b must be a contiguous float64 CUDA tensor with one entry per row")
     sf = torch.empty(B, dtype=torch.float64, device=r2.device) if want_sum_f else None
-    _check(_lib().lapsum_forward(r2.data_ptr(), ld, p.data_ptr(), b.data_ptr(),
-                                 sf.data_ptr() if sf is not None else None, B, n, float(k),
-                                 float(t), code, seed & (2**64 - 1), ws.ptr, ws.nbytes,
-                                 _stream_ptr(r2.device)), "lapsum_forward")
+    if support is not None:
+        if not support.fits(B, n):
+            raise ValueError("support buffer too small for (B, n)")
+        _check(_lib().lapsum_forward_support(
+            r2.data_ptr(), ld, p.data_ptr(), b.data_ptr(),
+            sf.data_ptr() if sf is not None else None, B, n, float(k), float(t), code,
+            seed & (2**64 - 1), ws.ptr, ws.nbytes, support.ptr, support.nbytes,
+            _stream_ptr(r2.device)), "lapsum_forward_support")
+    else:
+        _check(_lib().lapsum_forward(r2.data_ptr(), ld, p.data_ptr(), b.data_ptr(),
+                                     sf.data_ptr() if sf is not None else None, B, n, float(k),
+                                     float(t), code, seed & (2**64 - 1), ws.ptr, ws.nbytes,
+                                     _stream_ptr(r2.device)), "lapsum_forward")
     if squeeze:
         p = p[0]
     return (p, b, sf) if want_sum_f else (p, b)
 
 
 def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Workspace = None,
-             g: torch.Tensor = None):
-    """g = J^T v for each row (J the Jacobian of p with respect to r)."""
+             g: torch.Tensor = None, support: Support = None):
+    """g = J^T v for each row (J the Jacobian of p with respect to r).
+
+    With ``support`` (filled by forward(..., support=...) for this r and b)
+    v is read only at the listed scores and r is not read."""
     squeeze = r.dim() == 1
     r2 = _as_rows(r)
     v2 = _as_rows(v)
@@ -233,9 +288,17 @@ def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Wo
         _check_out(g, r2, ld, "g")
     if b.dtype != torch.float64 or not b.is_cuda or b.numel() != B:
         raise TypeError("b must be a float64 CUDA tensor with one entry per row")
-    _check(_lib().lapsum_backward(r2.data_ptr(), ld, b.data_ptr(), v2.data_ptr(), g.data_ptr(), B,
-                                  n, float(t), ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
-           "lapsum_backward")
+    if support is not None:
+        if not support.fits(B, n):
+            raise ValueError("support buffer too small for (B, n)")
+        _check(_lib().lapsum_backward_support(
+            r2.data_ptr(), ld, b.data_ptr(), v2.data_ptr(), g.data_ptr(), B, n, float(t),
+            support.ptr, support.nbytes, ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
+            "lapsum_backward_support")
+    else:
+        _check(_lib().lapsum_backward(r2.data_ptr(), ld, b.data_ptr(), v2.data_ptr(),
+                                      g.data_ptr(), B, n, float(t), ws.ptr, ws.nbytes,
+                                      _stream_ptr(r2.device)), "lapsum_backward")
     return g[0] if squeeze else g
 
 
@@ -310,19 +373,27 @@ def profile_read() -> dict:
 
 
 class LapSumTopK(torch.autograd.Function):
-    """Autograd wrapper: forward through lapsum_forward, backward through lapsum_backward."""
+    """Autograd wrapper.  Rows longer than 4096 go through lapsum_forward_support
+    and lapsum_backward_support (the gradient support is kept for backward);
+    shorter rows through lapsum_forward and lapsum_backward."""
 
     @staticmethod
     def forward(ctx, r, k, t, path="auto", seed=0):
-        p, b = forward(r.detach(), k, t, path=path, seed=seed)
+        rd = r.detach()
+        B = 1 if rd.dim() == 1 else rd.shape[0]
+        n = rd.shape[-1]
+        sup = Support(B, n, rd.device) if support_bytes(B, n) > 0 else None
+        p, b = forward(rd, k, t, path=path, seed=seed, support=sup)
         ctx.save_for_backward(r, b)
         ctx.t = t
+        ctx.sup = sup
         return p
 
     @staticmethod
     def backward(ctx, gp):
         r, b = ctx.saved_tensors
-        g = backward(r.detach(), b, gp.contiguous(), ctx.t)
+        g = backward(r.detach(), b, gp.contiguous(), ctx.t, support=ctx.sup)
+        ctx.sup = None
         return g, None, None, None, None
 
 

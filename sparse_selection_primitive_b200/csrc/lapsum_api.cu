@@ -244,9 +244,20 @@ int lapsum_workspace_init(void* ws, size_t ws_bytes, void* stream) {
     return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
 }
 
-int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
-                   int64_t n, double k, double t, int path, uint64_t seed, void* ws,
-                   size_t ws_bytes, void* stream) {
+size_t lapsum_support_bytes(int64_t B, int64_t n) {
+    if (B < 1 || n <= kOnchipMax) return 0;
+    return support_bytes(B, n);
+}
+
+}  // extern "C"
+
+namespace {
+
+// The forward of lapsum_forward and lapsum_forward_support; `support` is null
+// for the former.
+int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
+                 int64_t n, double k, double t, int path, uint64_t seed, void* ws, size_t ws_bytes,
+                 void* support, size_t support_size, void* stream) {
     if (r == nullptr || p == nullptr || b == nullptr) return LAPSUM_EINVAL;
     if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
     if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
@@ -257,6 +268,10 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
     const Layout L = make_layout(B, n, rp);
     if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+    const bool want_sup = support != nullptr && n > kOnchipMax;
+    if (want_sup && ((reinterpret_cast<uintptr_t>(support) % kAlign) != 0 ||
+                     support_size < support_bytes(B, n)))
+        return LAPSUM_EWORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     char* w = static_cast<char*>(ws);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(w + L.header);
@@ -318,11 +333,66 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
         }
     }
     if (e != cudaSuccess) return LAPSUM_ECUDA;
+    const SupportView sv_all = want_sup ? support_view(support, B, n) : SupportView{};
     for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
         const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+        const SupportView sv = want_sup ? support_rows(sv_all, r0, n) : SupportView{};
         e = launch_emit(r + r0 * ld, ld, p + r0 * ld, b + r0, sum_f ? sum_f + r0 : nullptr, nb, n,
                         t, partials + r0 * stream_tiles(n), tickets + r0, vec, hdr, r0 == 0 ? 1 : 0,
-                        B, rp, st);
+                        B, rp, want_sup ? &sv : nullptr, st);
+    }
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
+                   int64_t n, double k, double t, int path, uint64_t seed, void* ws,
+                   size_t ws_bytes, void* stream) {
+    return forward_impl(r, ld, p, b, sum_f, B, n, k, t, path, seed, ws, ws_bytes, nullptr, 0,
+                        stream);
+}
+
+int lapsum_forward_support(const float* r, int64_t ld, float* p, double* b, double* sum_f,
+                           int64_t B, int64_t n, double k, double t, int path, uint64_t seed,
+                           void* ws, size_t ws_bytes, void* support, size_t support_size,
+                           void* stream) {
+    if (support == nullptr && n > kOnchipMax) return LAPSUM_EWORKSPACE;
+    return forward_impl(r, ld, p, b, sum_f, B, n, k, t, path, seed, ws, ws_bytes, support,
+                        support_size, stream);
+}
+
+int lapsum_backward_support(const float* r, int64_t ld, const double* b, const float* v, float* g,
+                            int64_t B, int64_t n, double t, const void* support,
+                            size_t support_size, void* ws, size_t ws_bytes, void* stream) {
+    if (r == nullptr || b == nullptr || v == nullptr || g == nullptr) return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int vec = (aligned16(r) && aligned16(v) && aligned16(g) && (ld % 4) == 0) ? 1 : 0;
+    if (n <= kOnchipMax) {
+        return cuda_status(launch_onchip_backward(r, ld, b, v, g, B, (int)n, t, vec, st));
+    }
+    if (support == nullptr || (reinterpret_cast<uintptr_t>(support) % kAlign) != 0 ||
+        support_size < support_bytes(B, n))
+        return LAPSUM_EWORKSPACE;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const Layout L = make_layout(B, n, LAPSUM_PATH_FULLSORT);  // the streaming buffers only
+    if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+    char* w = static_cast<char*>(ws);
+    uint32_t* tickets = reinterpret_cast<uint32_t*>(w + L.tickets);
+    double* partials = reinterpret_cast<double*>(w + L.partials);
+    double* row_R = reinterpret_cast<double*>(w + L.row_R);
+    uint32_t* dflag = reinterpret_cast<uint32_t*>(w + L.wflag);
+    const SupportView sv_all = support_view(const_cast<void*>(support), B, n);
+    cudaError_t e = cudaSuccess;
+    for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
+        const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+        e = launch_backward_support(r + r0 * ld, ld, b + r0, v + r0 * ld, g + r0 * ld, nb, n, t,
+                                    support_rows(sv_all, r0, n), B, partials + r0 * stream_tiles(n) * 4,
+                                    row_R + r0, tickets + B + r0, dflag + r0, vec, st);
     }
     return cuda_status(e);
 }

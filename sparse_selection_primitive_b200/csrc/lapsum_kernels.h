@@ -46,11 +46,39 @@ cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int6
 // --- streaming kernels over long rows ----------------------------------------
 constexpr int kStreamTile = 4096;  // elements per CTA tile of the streaming kernels
 int64_t stream_tiles(int64_t n);
+
+// Gradient support of long rows, written by the forward and read by the
+// backward: every score with |x| <= kSupWindow, listed per warp share of each
+// 4096-score tile (8 shares of 512 scores, kSupCap entries each).
+constexpr int kSupWarps = 8;
+constexpr int kSupCap = 256;
+constexpr float kSupWindow = 90.f;  // f == 0 in fp32 beyond this |x|
+struct SupportView {
+    int64_t* hdr;    // [0] n and [1] B of the forward that wrote the list
+    double* b;       // [B] threshold of each row at that forward
+    uint32_t* cnt;   // [B][tiles][8] entries found per share (> kSupCap: overflow)
+    uint2* ent;      // [B][tiles][8][kSupCap] (position in the tile, x bits)
+    float* val;      // [B][tiles][8][kSupCap] v at each entry (written by the backward)
+};
+size_t support_bytes(int64_t B, int64_t n);
+SupportView support_view(void* base, int64_t B, int64_t n);
+SupportView support_rows(const SupportView& s, int64_t r0, int64_t n);  // rows from r0 on
+
 // p = sigma((r - b)/t) and sum f per row; partials: [B][tiles] doubles.
+// With sup != nullptr the gradient support is written as well.
 cudaError_t launch_emit(const float* r, int64_t ld, float* p, double* b, double* sumf,
                         int64_t B, int64_t n, double t, double* partials, uint32_t* tickets,
                         int vec, WsHeader* hdr, int record_call, int64_t B_total, int path_code,
-                        cudaStream_t st);
+                        const SupportView* sup, cudaStream_t st);
+// Backward from the gradient support: v is read only at the listed scores.
+// Rows whose list overflowed, does not match (n, b), or whose smallest |x| is
+// above 50 are recomputed by the dense kernels.
+// B_total: the rows of the whole call (checked against the forward's).
+cudaError_t launch_backward_support(const float* r, int64_t ld, const double* b, const float* v,
+                                    float* g, int64_t B, int64_t n, double t,
+                                    const SupportView& sup, int64_t B_total, double* partials,
+                                    double* row_R, uint32_t* tickets, uint32_t* dense_flag,
+                                    int vec, cudaStream_t st);
 // Backward for long rows: reduce (mu, sum w, sum w v) per row, then g.
 // partials: 4 doubles per CTA record.
 cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, const float* v,

@@ -92,7 +92,13 @@ __device__ __forceinline__ bool last_block_of_row(uint32_t* ticket, uint32_t nbl
 // p = sigma((r - b)/t) for one 4096-score tile per CTA; sum f per row when
 // asked for (per-tile partials, combined in tile order by the row's last CTA).
 // Full tiles take unchecked 16-byte accesses.
-template <bool VEC, bool SUMF>
+//
+// With SUP, every score with |x| <= 90 (the only ones whose f is not 0 in
+// fp32) is also listed in the gradient support: each warp appends
+// (position in the tile, x) to its own share of the tile's list, in a fixed
+// order, and records how many it found (a count above the share's capacity
+// marks an overflow; the backward then recomputes the row densely).
+template <bool VEC, bool SUMF, bool SUP>
 __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict__ r, int64_t ld,
                                                         float* __restrict__ p,
                                                         const double* __restrict__ b,
@@ -100,7 +106,8 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
                                                         double t, double* __restrict__ partials,
                                                         uint32_t* __restrict__ tickets,
                                                         WsHeader* hdr, int record_call,
-                                                        int64_t B_total, int path_code) {
+                                                        int64_t B_total, int path_code,
+                                                        SupportView sup) {
     __shared__ double red[kThreads / 32];
     __shared__ int flag;
     const int64_t row = blockIdx.y;
@@ -108,13 +115,30 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
         hdr->last_B = B_total;
         hdr->last_n = n;
         hdr->last_path = (uint32_t)path_code;
+        if (SUP) {
+            sup.hdr[0] = n;
+            sup.hdr[1] = B_total;
+        }
     }
     const int64_t tiles = gridDim.x;
     const int64_t base = (int64_t)blockIdx.x * kStreamTile;
-    const Thr th = make_thr(b[row], t);
+    const double brow = b[row];
+    const Thr th = make_thr(brow, t);
     const float* rr = r + row * ld;
     float* pr = p + row * ld;
     double sf = 0.0;
+    // gradient support of this warp's share of the tile
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int64_t share = (row * tiles + blockIdx.x) * kSupWarps + warp;
+    uint2* ent = SUP ? sup.ent + share * kSupCap : nullptr;
+    uint32_t cnt = 0;  // warp-uniform
+    auto put = [&](bool near, unsigned ball, uint32_t pos_in_tile, float x) {
+        const uint32_t at = cnt + __popc(ball & lt);
+        if (near && at < (uint32_t)kSupCap) ent[at] = make_uint2(pos_in_tile, __float_as_uint(x));
+        cnt += __popc(ball);
+    };
+    if (SUP && blockIdx.x == 0 && threadIdx.x == 0) sup.b[row] = brow;
     if (VEC && base + kStreamTile <= n) {
         const float4* r4 = reinterpret_cast<const float4*>(rr + base);
         float4* p4 = reinterpret_cast<float4*>(pr + base);
@@ -131,6 +155,21 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
                    make_float4(cdf_from(m0, e0), cdf_from(m1, e1), cdf_from(m2, e2),
                                cdf_from(m3, e3)));
             if (SUMF) sf += 0.5 * (double)((e0 + e1) + (e2 + e3));
+            if (SUP) {
+                const bool k0 = fabsf(m0) <= kSupWindow, k1 = fabsf(m1) <= kSupWindow;
+                const bool k2 = fabsf(m2) <= kSupWindow, k3 = fabsf(m3) <= kSupWindow;
+                const unsigned b0 = __ballot_sync(0xffffffffu, k0);
+                const unsigned b1 = __ballot_sync(0xffffffffu, k1);
+                const unsigned b2 = __ballot_sync(0xffffffffu, k2);
+                const unsigned b3 = __ballot_sync(0xffffffffu, k3);
+                if ((b0 | b1 | b2 | b3) != 0u) {
+                    const uint32_t i0 = 4u * (uint32_t)(q * kThreads + threadIdx.x);
+                    put(k0, b0, i0, m0);
+                    put(k1, b1, i0 + 1, m1);
+                    put(k2, b2, i0 + 2, m2);
+                    put(k3, b3, i0 + 3, m3);
+                }
+            }
         }
     } else {
         float x[kPer], y[kPer];
@@ -142,9 +181,17 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
             const float e = neg_abs_exp(xs);
             y[q] = cdf_from(xs, e);
             if (SUMF && ok[q]) sf += 0.5 * (double)e;
+            if (SUP) {
+                // load_tile's element order: float4 groups, or plain striding
+                const uint32_t pos = VEC ? (uint32_t)(4 * ((q / 4) * kThreads + threadIdx.x) + q % 4)
+                                         : (uint32_t)(q * kThreads + threadIdx.x);
+                const bool k0 = ok[q] && fabsf(xs) <= kSupWindow;
+                put(k0, __ballot_sync(0xffffffffu, k0), pos, xs);
+            }
         }
         store_tile<VEC>(pr, n, base, y);
     }
+    if (SUP && lane == 0) sup.cnt[share] = cnt;
     if (!SUMF) return;
     sf = block_sum_d(sf, red);
     if (threadIdx.x == 0) partials[row * tiles + blockIdx.x] = sf;
@@ -295,18 +342,27 @@ int64_t stream_tiles(int64_t n) { return (n + kStreamTile - 1) / kStreamTile; }
 cudaError_t launch_emit(const float* r, int64_t ld, float* p, double* b, double* sumf,
                         int64_t B, int64_t n, double t, double* partials, uint32_t* tickets,
                         int vec, WsHeader* hdr, int record_call, int64_t B_total, int path_code,
-                        cudaStream_t st) {
+                        const SupportView* sup, cudaStream_t st) {
     const dim3 grid((unsigned)stream_tiles(n), (unsigned)B);
     ProfScope ps_("emit", st);
-#define LAPSUM_EMIT(V, S)                                                                     \
-    emit_kernel<V, S><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets, hdr, \
-                                                 record_call, B_total, path_code)
-    if (vec) {
-        if (sumf) LAPSUM_EMIT(true, true);
-        else LAPSUM_EMIT(true, false);
+    const SupportView sv = sup ? *sup : SupportView{};
+#define LAPSUM_EMIT(V, S, U)                                                                  \
+    emit_kernel<V, S, U><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets, \
+                                                    hdr, record_call, B_total, path_code, sv)
+    if (sup) {
+        if (vec) {
+            if (sumf) LAPSUM_EMIT(true, true, true);
+            else LAPSUM_EMIT(true, false, true);
+        } else {
+            if (sumf) LAPSUM_EMIT(false, true, true);
+            else LAPSUM_EMIT(false, false, true);
+        }
+    } else if (vec) {
+        if (sumf) LAPSUM_EMIT(true, true, false);
+        else LAPSUM_EMIT(true, false, false);
     } else {
-        if (sumf) LAPSUM_EMIT(false, true);
-        else LAPSUM_EMIT(false, false);
+        if (sumf) LAPSUM_EMIT(false, true, false);
+        else LAPSUM_EMIT(false, false, false);
     }
 #undef LAPSUM_EMIT
     return cudaGetLastError();

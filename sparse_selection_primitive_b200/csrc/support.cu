@@ -1,0 +1,336 @@
+// Backward of long rows from the gradient support left by the forward.
+//
+// The VJP of "Fast LapSum: Exact Differentiable Top-k at Million Scale"
+// (gist.science explainer pages), section 2.1, is g_i = (f_i/t)(v_i - R) with
+// f_i = 0.5 exp(-|x_i|), x_i = (r_i - b)/t and R = sum v f / sum f.  f_i is 0
+// in fp32 once |x_i| > 87.4, so only the scores with |x| <= 90 carry gradient.
+// The forward's emit pass already computes every x_i; with the support output
+// it also lists those scores (position in the tile and x) per warp share of
+// each 4096-score tile.  The backward then never reads r:
+//
+// Pass A (sup_reduce_kernel): each CTA takes a group of tiles, scans the
+//   shares' counts, and walks the listed entries with all its threads: v is
+//   gathered at each entry (and kept next to it for pass B), the terms go into
+//   an online (mu, sum w, sum w v), w = exp(-(|x| - mu)).  The last CTA of the
+//   row combines the CTA records in a fixed order into R and decides whether
+//   the list serves the row.
+// Pass B (sup_write_kernel): g tile by tile; the tile is zeroed in shared
+//   memory, its entries are placed, and it is written out with coalesced
+//   16-byte stores, so every g value is written exactly once.
+//
+// A row is handed to the dense two-pass kernels when its list overflowed, was
+// written for another (n, B) or another b, holds an index out of range, or
+// its smallest |x| is above 50 (then scores outside the list could weigh in R).
+#include "lapsum_common.cuh"
+#include "lapsum_kernels.h"
+
+namespace lapsum {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTile = kStreamTile;
+constexpr int kShares = kSupWarps;
+constexpr int kGroupMax = kThreads / kShares;  // tiles per pass-A CTA (one share per thread)
+constexpr float kDenseAbove = 50.f;
+constexpr size_t kAlignSup = 256;
+
+size_t up256(size_t x) { return (x + kAlignSup - 1) / kAlignSup * kAlignSup; }
+
+__device__ __forceinline__ void sup_add(float ax, float vv, float& mu, double& s, double& sv) {
+    if (ax < mu) {
+        const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(ax - mu);
+        s *= sc;
+        sv *= sc;
+        mu = ax;
+    }
+    const float w = __expf(mu - ax);
+    s += (double)w;
+    sv += (double)(w * vv);
+}
+
+__global__ void __launch_bounds__(kThreads) sup_reduce_kernel(
+    const double* __restrict__ b, const float* __restrict__ v, int64_t ld, int64_t n,
+    int64_t B_total, int group, SupportView sup, double* __restrict__ partials,
+    double* __restrict__ row_R, uint32_t* __restrict__ tickets, uint32_t* __restrict__ dense_flag) {
+    __shared__ uint32_t pre[kThreads + 1];  // exclusive prefix of the group's share counts
+    __shared__ uint32_t wtot[kThreads / 32];
+    __shared__ double red[kThreads / 32];
+    __shared__ float fred[kThreads / 32];
+    __shared__ int flag;
+    const int64_t row = blockIdx.y;
+    const int64_t nblk = gridDim.x;
+    const int64_t tiles = (n + kTile - 1) / kTile;
+    const int64_t t0 = (int64_t)blockIdx.x * group;
+    const int64_t t1 = t0 + group < tiles ? t0 + group : tiles;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float* vr = v + row * ld;
+    // the list must come from a forward over the same (n, B) with this b
+    const bool match = sup.hdr[0] == n && sup.hdr[1] == B_total &&
+                       __double_as_longlong(sup.b[row]) == __double_as_longlong(b[row]);
+    // one share per thread: (tile t0 + i / 8, share i % 8)
+    uint32_t c = 0;
+    int bad = match ? 0 : 1;
+    if (match && t0 + (int64_t)threadIdx.x / kShares < t1) {
+        c = sup.cnt[(row * tiles + t0) * kShares + threadIdx.x];
+        if (c > (uint32_t)kSupCap) {
+            bad = 1;
+            c = 0;
+        }
+    }
+    // block exclusive scan of the counts
+    uint32_t inc = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc += o;
+    }
+    if (lane == 31) wtot[warp] = inc;
+    __syncthreads();
+    uint32_t wpre = 0;
+    for (int u = 0; u < warp; ++u) wpre += wtot[u];
+    pre[threadIdx.x] = wpre + inc - c;
+    if (threadIdx.x == kThreads - 1) pre[kThreads] = wpre + inc;
+    __syncthreads();
+    const uint32_t total = pre[kThreads];
+    const uint2* ent = sup.ent + (row * tiles + t0) * kShares * kSupCap;
+    float* val = sup.val + (row * tiles + t0) * kShares * kSupCap;
+    float mu = INFINITY, amin = INFINITY;
+    double s = 0.0, sv = 0.0;
+    constexpr int U = 4;  // entries per thread in flight
+    for (uint32_t j0 = 0; j0 < total; j0 += U * kThreads) {
+        uint2 e[U];
+        int64_t slot[U], gpos[U];
+        bool ok[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t j = j0 + u * kThreads + threadIdx.x;
+            ok[u] = j < total;
+            slot[u] = 0;
+            if (ok[u]) {
+                // share holding entry j: the last with pre[share] <= j
+                int lo = 0, hi = kThreads - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (pre[mid] <= j) lo = mid;
+                    else hi = mid - 1;
+                }
+                slot[u] = (int64_t)lo * kSupCap + (j - pre[lo]);
+                e[u] = __ldcs(ent + slot[u]);
+                const int64_t tile = t0 + lo / kShares;
+                gpos[u] = tile * kTile + e[u].x;
+                if (e[u].x >= (uint32_t)kTile || gpos[u] >= n) {
+                    ok[u] = false;
+                    bad = 1;
+                }
+            }
+        }
+        float vv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) vv[u] = ok[u] ? __ldcs(vr + gpos[u]) : 0.f;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (!ok[u]) continue;
+            const float ax = fabsf(__uint_as_float(e[u].y));
+            amin = fminf(amin, ax);
+            sup_add(ax, vv[u], mu, s, sv);
+            val[slot[u]] = vv[u];
+        }
+    }
+    // CTA record (mu, S, Sv, min |x| or -1 when the list cannot serve the row)
+    const int anybad_cta = __syncthreads_or(bad);
+    const float mb = block_min_f(mu, fred);
+    const double sc = (mu == INFINITY) ? 0.0 : exp((double)mb - (double)mu);
+    s = block_sum_d(s * sc, red);
+    sv = block_sum_d(sv * sc, red);
+    const float am = block_min_f(amin, fred);
+    if (threadIdx.x == 0) {
+        double* pr = partials + (row * nblk + blockIdx.x) * 4;
+        pr[0] = (double)mb;
+        pr[1] = s;
+        pr[2] = sv;
+        pr[3] = anybad_cta ? -1.0 : (double)am;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t prev = atomicAdd(&tickets[row], 1u);
+        flag = (prev == (uint32_t)nblk - 1u);
+        if (flag) tickets[row] = 0u;
+    }
+    __syncthreads();
+    if (!flag) return;
+    __threadfence();
+    float mloc = INFINITY, aloc = INFINITY;
+    int rbad = 0;
+    for (int64_t k = threadIdx.x; k < nblk; k += kThreads) {
+        const double* pr = partials + (row * nblk + k) * 4;
+        mloc = fminf(mloc, (float)pr[0]);
+        if (pr[3] < 0.0) rbad = 1;
+        else aloc = fminf(aloc, (float)pr[3]);
+    }
+    const double mrow = (double)block_min_f(mloc, fred);
+    const float arow = block_min_f(aloc, fred);
+    const int anybad = __syncthreads_or(rbad);
+    double a = 0.0, av = 0.0;
+    for (int64_t k = threadIdx.x; k < nblk; k += kThreads) {
+        const double* pr = partials + (row * nblk + k) * 4;
+        if (pr[0] == INFINITY) continue;
+        const double f = exp(mrow - pr[0]);
+        a += pr[1] * f;
+        av += pr[2] * f;
+    }
+    a = block_sum_d(a, red);
+    av = block_sum_d(av, red);
+    if (threadIdx.x == 0) {
+        row_R[row] = a > 0.0 ? av / a : 0.0;
+        dense_flag[row] = (anybad || arow > kDenseAbove) ? 1u : 0u;
+    }
+}
+
+// g for one tile per CTA: zeroed in shared memory, the listed entries placed,
+// then written with 16-byte streaming stores.
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads) sup_write_kernel(
+    SupportView sup, const uint32_t* __restrict__ dense_flag, const double* __restrict__ row_R,
+    float* __restrict__ g, int64_t ld, int64_t n, double t) {
+    __shared__ __align__(16) float tile[kTile];
+    __shared__ uint32_t pre[kShares + 1];
+    const int64_t row = blockIdx.y;
+    if (dense_flag[row]) return;  // the dense kernels own this row
+    const int64_t tiles = (n + kTile - 1) / kTile;
+    const int64_t T = blockIdx.x;
+    const int64_t base = T * kTile;
+    const double R = row_R[row];
+    const float hinv = (float)(0.5 / t);
+    float4* t4 = reinterpret_cast<float4*>(tile);
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < kTile / 4 / kThreads; ++q) t4[q * kThreads + threadIdx.x] = z4;
+    if (threadIdx.x < 32) {
+        // counts were checked (<= kSupCap) by pass A before it cleared the row
+        const uint32_t c = threadIdx.x < kShares ? sup.cnt[(row * tiles + T) * kShares + threadIdx.x]
+                                                 : 0u;
+        uint32_t inc = c;
+#pragma unroll
+        for (int d = 1; d < kShares; d <<= 1) {
+            const uint32_t o = __shfl_up_sync(0xffffffffu, inc, d);
+            if (threadIdx.x >= d) inc += o;
+        }
+        if (threadIdx.x < kShares) pre[threadIdx.x] = inc - c;
+        if (threadIdx.x == kShares - 1) pre[kShares] = inc;
+    }
+    __syncthreads();
+    const uint32_t total = pre[kShares];
+    const uint2* ent = sup.ent + (row * tiles + T) * kShares * kSupCap;
+    const float* val = sup.val + (row * tiles + T) * kShares * kSupCap;
+    for (uint32_t j = threadIdx.x; j < total; j += kThreads) {
+        int sh = 0;
+#pragma unroll
+        for (int u = 1; u < kShares; ++u) sh += (pre[u] <= j) ? 1 : 0;
+        const int64_t slot = (int64_t)sh * kSupCap + (j - pre[sh]);
+        const uint2 e = __ldcs(ent + slot);
+        const float vv = __ldcs(val + slot);
+        const float ax = fabsf(__uint_as_float(e.y));
+        tile[e.x & (kTile - 1)] = hinv * __expf(-ax) * (float)((double)vv - R);
+    }
+    __syncthreads();
+    float* gr = g + row * ld + base;
+    if (VEC && base + kTile <= n) {
+        float4* g4 = reinterpret_cast<float4*>(gr);
+#pragma unroll
+        for (int q = 0; q < kTile / 4 / kThreads; ++q)
+            __stcs(g4 + q * kThreads + threadIdx.x, t4[q * kThreads + threadIdx.x]);
+    } else {
+        for (int e = threadIdx.x; e < kTile && base + e < n; e += kThreads) gr[e] = tile[e];
+    }
+}
+
+int sm_count() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    return sms;
+}
+
+struct SupOffsets {
+    size_t hdr, b, cnt, ent, val, total;
+};
+
+SupOffsets sup_offsets(int64_t B, int64_t n) {
+    const size_t tiles = (size_t)stream_tiles(n);
+    SupOffsets o{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += up256(bytes);
+        return at;
+    };
+    o.hdr = take(2 * sizeof(int64_t));
+    o.b = take((size_t)B * sizeof(double));
+    o.cnt = take((size_t)B * tiles * kShares * sizeof(uint32_t));
+    o.ent = take((size_t)B * tiles * kShares * kSupCap * sizeof(uint2));
+    o.val = take((size_t)B * tiles * kShares * kSupCap * sizeof(float));
+    o.total = off;
+    return o;
+}
+
+}  // namespace
+
+size_t support_bytes(int64_t B, int64_t n) { return sup_offsets(B, n).total; }
+
+SupportView support_view(void* base, int64_t B, int64_t n) {
+    const SupOffsets o = sup_offsets(B, n);
+    char* p = static_cast<char*>(base);
+    SupportView s;
+    s.hdr = reinterpret_cast<int64_t*>(p + o.hdr);
+    s.b = reinterpret_cast<double*>(p + o.b);
+    s.cnt = reinterpret_cast<uint32_t*>(p + o.cnt);
+    s.ent = reinterpret_cast<uint2*>(p + o.ent);
+    s.val = reinterpret_cast<float*>(p + o.val);
+    return s;
+}
+
+SupportView support_rows(const SupportView& s, int64_t r0, int64_t n) {
+    const int64_t per_row = stream_tiles(n) * kShares;
+    SupportView o = s;
+    o.b += r0;
+    o.cnt += r0 * per_row;
+    o.ent += r0 * per_row * kSupCap;
+    o.val += r0 * per_row * kSupCap;
+    return o;
+}
+
+cudaError_t launch_backward_support(const float* r, int64_t ld, const double* b, const float* v,
+                                    float* g, int64_t B, int64_t n, double t,
+                                    const SupportView& sup, int64_t B_total, double* partials,
+                                    double* row_R, uint32_t* tickets, uint32_t* dense_flag,
+                                    int vec, cudaStream_t st) {
+    const int64_t tiles = stream_tiles(n);
+    // pass A: groups of tiles sized so all rows together give about 8 CTAs per SM
+    int64_t group = (B * tiles + (int64_t)sm_count() * 8 - 1) / ((int64_t)sm_count() * 8);
+    if (group < 1) group = 1;
+    if (group > kGroupMax) group = kGroupMax;
+    const int64_t per_row = (tiles + group - 1) / group;
+    {
+        ProfScope ps_("sup_reduce", st);
+        sup_reduce_kernel<<<dim3((unsigned)per_row, (unsigned)B), kThreads, 0, st>>>(
+            b, v, ld, n, B_total, (int)group, sup, partials, row_R, tickets, dense_flag);
+    }
+    {
+        ProfScope ps_("sup_write", st);
+        const dim3 grid((unsigned)tiles, (unsigned)B);
+        if (vec)
+            sup_write_kernel<true><<<grid, kThreads, 0, st>>>(sup, dense_flag, row_R, g, ld, n, t);
+        else
+            sup_write_kernel<false><<<grid, kThreads, 0, st>>>(sup, dense_flag, row_R, g, ld, n,
+                                                                t);
+    }
+    // rows the list could not serve: dense recompute (exits at once otherwise)
+    return launch_backward_stream_if(r, ld, b, v, g, B, n, t, partials, row_R, tickets, vec,
+                                     dense_flag, st);
+}
+
+}  // namespace lapsum

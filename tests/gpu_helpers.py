@@ -25,11 +25,14 @@ G_FLOOR = 1e-37
 
 
 def run_gpu(r: np.ndarray, k: float, t: float, path="auto", v: np.ndarray = None, seed=0,
-            device="cuda:0", want_sum_f=False, ws=None):
+            device="cuda:0", want_sum_f=False, ws=None, support=False):
+    """Forward (and backward when v is given) through the binding.  With
+    support=True the gradient-support pair of entry points is used."""
     rt = torch.from_numpy(np.ascontiguousarray(r, dtype=np.float32)).to(device)
     if rt.dim() == 1:
         rt = rt.unsqueeze(0)
-    out = L.forward(rt, k, t, path=path, seed=seed, ws=ws, want_sum_f=want_sum_f)
+    sup = L.Support(rt.shape[0], rt.shape[1], rt.device) if support else None
+    out = L.forward(rt, k, t, path=path, seed=seed, ws=ws, want_sum_f=want_sum_f, support=sup)
     p, b = out[0], out[1]
     res = {"p": p.cpu().numpy().astype(np.float64), "b": b.cpu().numpy()}
     if want_sum_f:
@@ -38,7 +41,7 @@ def run_gpu(r: np.ndarray, k: float, t: float, path="auto", v: np.ndarray = None
         vt = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).to(device)
         if vt.dim() == 1:
             vt = vt.unsqueeze(0)
-        g = L.backward(rt, b, vt, t, ws=ws)
+        g = L.backward(rt, b, vt, t, ws=ws, support=sup)
         res["g"] = g.cpu().numpy().astype(np.float64)
     torch.cuda.synchronize()
     return res

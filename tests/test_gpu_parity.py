@@ -191,3 +191,93 @@ def test_windowed_backward_far_threshold_falls_back(cuda_device):
     v = np.random.default_rng(5).standard_normal((1, n)).astype(np.float32)
     out = run_gpu(r, 17.0, 0.008, path="radix", v=v)
     check_row(r[0], v[0], 17.0, 0.008, out["b"][0], out["p"][0], out["g"][0], label="far")
+
+
+# ---------------------------------------------------------------------------
+# Gradient support handed from the forward to the backward (rows > 4096).
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,n,k,t,dist,path", [
+    (1, 1 << 20, 1000.0, 0.001, "normal", "radix"),     # sparse support, full tiles
+    (1, 1 << 18, 2000.0, 0.05, "normal", "radix"),      # support above half of every share: dense
+    (1, 300001, 77.0, 0.0004, "mix_nu", "bracket"),     # ragged last tile
+    (3, 70001, 500.0, 0.01, "normal_q64", "radix"),     # several rows, ties
+    (2, 20000, 123.5, 0.01, "abs_t3", "bracket"),
+])
+def test_support_backward(cuda_device, B, n, k, t, dist, path):
+    r, v = random_rows(61 + n, B, n, dist)
+    out = run_gpu(r, k, t, path=path, v=v, support=True)
+    for i in range(B):
+        check_row(r[i], v[i], k, t, out["b"][i], out["p"][i], out["g"][i],
+                  label=f"support n={n} row={i}")
+
+
+def test_support_far_threshold_falls_back(cuda_device):
+    # every |x| is at least 62.5 (> 50): the row is recomputed by the dense kernels
+    n = 6000
+    r = np.random.default_rng(4).permutation(n).astype(np.float32)[None, :]
+    v = np.random.default_rng(5).standard_normal((1, n)).astype(np.float32)
+    out = run_gpu(r, 17.0, 0.008, path="radix", v=v, support=True)
+    check_row(r[0], v[0], 17.0, 0.008, out["b"][0], out["p"][0], out["g"][0], label="far")
+
+
+def test_support_matches_plain_backward_and_is_deterministic(cuda_device):
+    B, n = 2, 1 << 17
+    r, v = random_rows(77, B, n)
+    rt = torch.from_numpy(r).cuda()
+    vt = torch.from_numpy(v).cuda()
+    sup = L.Support(B, n)
+    p1, b1 = L.forward(rt, 300.0, 0.002, support=sup)
+    p0, b0 = L.forward(rt, 300.0, 0.002)
+    assert torch.equal(p0, p1) and torch.equal(b0, b1)
+    g_plain = L.backward(rt, b0, vt, 0.002)
+    g1 = L.backward(rt, b1, vt, 0.002, support=sup)
+    g2 = L.backward(rt, b1, vt, 0.002, support=sup)
+    assert torch.equal(g1, g2)
+    scale = g_plain.abs().max().item()
+    assert (g1 - g_plain).abs().max().item() <= 1e-5 * scale
+    for i in range(B):
+        check_row(r[i], v[i], 300.0, 0.002, b1[i].item(), p1[i].cpu().numpy().astype(np.float64),
+                  g1[i].cpu().numpy().astype(np.float64), label=f"row {i}")
+
+
+def test_support_from_another_forward_is_not_trusted(cuda_device):
+    # the list was written for other scores (another b): the backward notices
+    # the mismatch and recomputes the rows densely, so g is still right
+    B, n = 2, 50000
+    r, v = random_rows(81, B, n)
+    r_other, _ = random_rows(82, B, n)
+    sup = L.Support(B, n)
+    L.forward(torch.from_numpy(r_other).cuda(), 40.0, 0.01, support=sup)
+    rt = torch.from_numpy(r).cuda()
+    p, b = L.forward(rt, 40.0, 0.01)
+    g = L.backward(rt, b, torch.from_numpy(v).cuda(), 0.01, support=sup)
+    for i in range(B):
+        check_row(r[i], v[i], 40.0, 0.01, b[i].item(), p[i].cpu().numpy().astype(np.float64),
+                  g[i].cpu().numpy().astype(np.float64), label=f"stale list row {i}")
+
+
+def test_support_strided_rows(cuda_device):
+    # ld > n and an unaligned base: the scalar paths of the emit and write kernels
+    B, n, ld = 3, 9000, 9011
+    r, v = random_rows(12, B, ld)
+    full = torch.from_numpy(r).cuda()
+    vv = torch.from_numpy(v).cuda()
+    sub = full[:, 1:1 + n]
+    sup = L.Support(B, n)
+    p, b = L.forward(sub, 30.0, 0.02, path="radix", support=sup)
+    g = L.backward(sub, b, vv[:, 1:1 + n], 0.02, support=sup)
+    for i in range(B):
+        check_row(r[i, 1:1 + n], v[i, 1:1 + n], 30.0, 0.02, b[i].item(),
+                  p[i].cpu().numpy().astype(np.float64), g[i].cpu().numpy().astype(np.float64),
+                  label=f"strided support row={i}")
+
+
+def test_autograd_long_rows_use_support(cuda_device):
+    r, v = random_rows(14, 2, 30000)
+    rt = torch.from_numpy(r).cuda().requires_grad_(True)
+    p = L.soft_topk(rt, 25.0, 0.01)
+    p.backward(torch.from_numpy(v).cuda())
+    _, b = L.forward(rt.detach(), 25.0, 0.01)
+    g = L.backward(rt.detach(), b, torch.from_numpy(v).cuda(), 0.01)
+    scale = g.abs().max().item()
+    assert (rt.grad - g).abs().max().item() <= 1e-5 * scale
