@@ -173,7 +173,7 @@ __device__ bool top_ranks(const float* __restrict__ y, int m, int64_t rho_max, i
     if (ncand <= (uint32_t)kBlk) {
         uint32_t key[1];
         key[0] = (int)threadIdx.x < (int)ncand ? cand[threadIdx.x] : 0u;
-        bitonic_sort_row<1, kBlk, kBlk>(key, threadIdx.x, xch);
+        bitonic_sort_block_rolled<1, kBlk>(key, threadIdx.x, xch);
         cand[threadIdx.x] = key[0];
         npad = kBlk;
     } else {
@@ -183,7 +183,7 @@ __device__ bool top_ranks(const float* __restrict__ y, int m, int64_t rho_max, i
             const int j = threadIdx.x * 4 + e;
             key[e] = j < (int)ncand ? cand[j] : 0u;
         }
-        bitonic_sort_row<4, kBlk, kBlk>(key, threadIdx.x, xch);
+        bitonic_sort_block_rolled<4, kBlk>(key, threadIdx.x, xch);
 #pragma unroll
         for (int e = 0; e < 4; ++e) cand[threadIdx.x * 4 + e] = key[e];
         npad = 4 * kBlk;
@@ -222,6 +222,8 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
         for (int i = threadIdx.x; i < (int)(sizeof(RowState) / 4); i += kBlk)
             reinterpret_cast<uint32_t*>(st)[i] = 0u;
         for (int i = threadIdx.x; i < 3 * kBins; i += kBlk) bins[i] = 0ull;
+        __syncthreads();
+        phase_mark(st, 14);
     }
     extern __shared__ uint32_t dyn[];
     uint32_t* cand = dyn;                 // up to 4096 candidate keys
@@ -253,6 +255,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
             atomicAdd(&hist[bn], (uint32_t)__popc(peers));
     }
     __syncthreads();
+    if (blockIdx.x == 0) phase_mark(st, 15);
     for (int i = threadIdx.x; i < 2048; i += kBlk)
         if (hist[i] != 0u) atomicAdd(&ghist[i], hist[i]);
     __threadfence();
@@ -460,6 +463,7 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     float* q = wq[warp];
     uint32_t head = 0, tail = 0;  // warp-uniform; tail - head = queued scores
     if (threadIdx.x == 0) scount = 0;
+    if (blockIdx.x == 0) phase_mark(st, 16);
     __syncthreads();
     FoldAcc acc{0u, 0.0, 0.0, false};
     uint32_t far_right = 0u;
@@ -598,6 +602,7 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     a = block_sum_d(a, red);
     bsum = block_sum_d(bsum, red);
     badsum = block_sum_d(badsum, red);
+    phase_mark(st, 17);
     if (threadIdx.x == 0) {
         st->cnt_R = (unsigned long long)c;
         st->S_L = a;
@@ -673,7 +678,7 @@ __device__ void sort_band_into(const float* band, long long nb, SolveSmemAll* sm
         const long long j = (long long)threadIdx.x * E + e;
         key[e] = j < nb ? to_key(band[j]) : 0xffffffffu;
     }
-    bitonic_sort_row<E, kBlk, kBlk>(key, threadIdx.x, sm->u.sort.xch);
+    bitonic_sort_block_rolled<E, kBlk>(key, threadIdx.x, sm->u.sort.xch);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const long long j = (long long)threadIdx.x * E + e;
@@ -730,8 +735,8 @@ __device__ void certify_big_band(const float* band, long long nb, const Tails& t
         __syncthreads();
     }
     const double lnw = (tl.hasL && tl.hasR) ? ((double)tl.aL - (double)tl.aR) / t : -INFINITY;
-    *F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * (wl + tl.SR * exp(lnw)) + 0.5 * tl.SL : INFINITY;
-    *F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * (vr + tl.SL * exp(lnw)) : -INFINITY;
+    *F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * (wl + tl.SR * cold_exp(lnw)) + 0.5 * tl.SL : INFINITY;
+    *F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * (vr + tl.SL * cold_exp(lnw)) : -INFINITY;
     *kmin = lo;
     *kmax = hi;
 }
@@ -780,7 +785,7 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
     {
         const int b0 = 2 * threadIdx.x, b1 = b0 + 1;
         const double e0 = (double)edge(b0), e1 = (double)edge(b1), e2 = (double)edge(b1 + 1);
-        const double g0 = exp((e0 - e1) / t), g1 = exp((e1 - e2) / t);
+        const double g0 = cold_exp((e0 - e1) / t), g1 = cold_exp((e1 - e2) / t);
         const double U0 = sm->u.hist.U[b0], U1 = sm->u.hist.U[b1];
         const double L0 = sm->u.hist.L[b0], L1 = sm->u.hist.L[b1];
         const long long c01 = (long long)sm->u.hist.cnt[b0] + (long long)sm->u.hist.cnt[b1];
@@ -789,8 +794,8 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
         const Aff eb = block_excl_scan_bwd(mb, sm->ss.wb);
         const Aff ef = block_excl_scan_fwd(mf, sm->ss.wf);
         const long long above = block_excl_suffix_ll(c01, sm->lred);
-        const double Qend = tl.hasR ? tl.SR * exp(((double)edge(kRefineBins) - (double)tl.aR) / t) : 0.0;
-        const double Pstart = tl.hasL ? tl.SL * exp(((double)tl.aL - (double)edge(0)) / t) : 0.0;
+        const double Qend = tl.hasR ? tl.SR * cold_exp(((double)edge(kRefineBins) - (double)tl.aR) / t) : 0.0;
+        const double Pstart = tl.hasL ? tl.SL * cold_exp(((double)tl.aL - (double)edge(0)) / t) : 0.0;
         const double Q2 = fma(eb.a, Qend, eb.c);                // Q at edge b0+2
         const double Q1 = fma(g1, Q2, U1);
         const double Q0 = fma(g0, Q1, U0);
@@ -862,15 +867,15 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
         Tails nt;
         nt.hasL = hasLo;
         nt.aL = Elo;
-        nt.SL = (useL ? tl.SL : (tl.hasL ? tl.SL * exp(((double)tl.aL - (double)Elo) / t) : 0.0)) + sl;
+        nt.SL = (useL ? tl.SL : (tl.hasL ? tl.SL * cold_exp(((double)tl.aL - (double)Elo) / t) : 0.0)) + sl;
         nt.hasR = hasHi;
         nt.aR = Ehi;
-        nt.SR = (useR ? tl.SR : (tl.hasR ? tl.SR * exp(((double)Ehi - (double)tl.aR) / t) : 0.0)) + sr;
+        nt.SR = (useR ? tl.SR : (tl.hasR ? tl.SR * cold_exp(((double)Ehi - (double)tl.aR) / t) : 0.0)) + sr;
         nt.cntR = tl.cntR + (double)cr;
         const double lnw = (hasLo && hasHi) ? ((double)Elo - (double)Ehi) / t : -INFINITY;
-        const double FL = hasLo ? nt.cntR + (double)cnt - 0.5 * (w + nt.SR * exp(lnw)) + 0.5 * nt.SL
+        const double FL = hasLo ? nt.cntR + (double)cnt - 0.5 * (w + nt.SR * cold_exp(lnw)) + 0.5 * nt.SL
                                 : INFINITY;
-        const double FR = hasHi ? nt.cntR - 0.5 * nt.SR + 0.5 * (v + nt.SL * exp(lnw)) : -INFINITY;
+        const double FR = hasHi ? nt.cntR - 0.5 * nt.SR + 0.5 * (v + nt.SL * cold_exp(lnw)) : -INFINITY;
         const uint32_t klo = sm->bcast[2], khi = sm->bcast[3];
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -907,8 +912,8 @@ __device__ int bin_scan(const BinLayout& BL, const unsigned long long* __restric
     const int b0 = 2 * threadIdx.x, b1 = b0 + 1;
     const double e0 = (double)bin_edge(BL, b0), e1 = (double)bin_edge(BL, b1);
     const double e2 = (double)bin_edge(BL, b1 + 1);
-    const double g0 = (e1 > e0) ? exp((e0 - e1) / t) : 1.0;
-    const double g1 = (e2 > e1) ? exp((e1 - e2) / t) : 1.0;
+    const double g0 = (e1 > e0) ? cold_exp((e0 - e1) / t) : 1.0;
+    const double g1 = (e2 > e1) ? cold_exp((e1 - e2) / t) : 1.0;
     const long long c0 = (long long)bins[b0], c1 = (long long)bins[b1];
     const double U0 = (double)bins[kBins + b0] / kFixScale, U1 = (double)bins[kBins + b1] / kFixScale;
     const double L0 = (double)bins[2 * kBins + b0] / kFixScale;
@@ -919,8 +924,8 @@ __device__ int bin_scan(const BinLayout& BL, const unsigned long long* __restric
     const Aff ef = block_excl_scan_fwd(mf, sm->ss.wf);
     const long long above = block_excl_suffix_ll(c0 + c1, sm->lred);
     const double etop = (double)bin_edge(BL, kBins), efirst = (double)bin_edge(BL, 0);
-    const double Qend = (tl.hasR && tl.SR > 0.0) ? tl.SR * exp((etop - (double)tl.aR) / t) : 0.0;
-    const double Pst = (tl.hasL && tl.SL > 0.0) ? tl.SL * exp(((double)tl.aL - efirst) / t) : 0.0;
+    const double Qend = (tl.hasR && tl.SR > 0.0) ? tl.SR * cold_exp((etop - (double)tl.aR) / t) : 0.0;
+    const double Pst = (tl.hasL && tl.SL > 0.0) ? tl.SL * cold_exp(((double)tl.aL - efirst) / t) : 0.0;
     const double Q2 = fma(eb.a, Qend, eb.c), Q1 = fma(g1, Q2, U1), Q0 = fma(g0, Q1, U0);
     const double P0 = fma(ef.a, Pst, ef.c), P1 = fma(g0, P0, L0), P2 = fma(g1, P1, L1);
     const double A2 = tl.cntR + (double)above, A1 = A2 + (double)c1, A0 = A1 + (double)c0;
@@ -1287,6 +1292,7 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
 __global__ void __launch_bounds__(256) extract_kernel(const float* __restrict__ band,
                                                       RowState* st, float* __restrict__ sub) {
     if (st->stage != 1) return;
+    if (blockIdx.x == 0) phase_mark(st, 18);
     const long long nb = (long long)st->n_band;
     const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
     const int j = st->sub_bin;
@@ -1346,7 +1352,11 @@ __global__ void __launch_bounds__(kBlk) solve2_kernel(double k, double t, RowSta
     double b = nan("");
     bool ok = false;
     if (ns <= kBandSortMax) {
-        solve_small_band(sub, ns, s, k, t, sm);
+        if (ns <= kBlk) sort_band_into<1>(sub, ns, sm);
+        else if (ns <= 2 * kBlk) sort_band_into<2>(sub, ns, sm);
+        else sort_band_into<4>(sub, ns, sm);
+        phase_mark(st, 13);
+        solve_sorted_block(FloatGet{sm->u.sort.sorted}, ns, s, k, t, &sm->ss, &sm->res);
         ok = sm->res.F_aL >= k && sm->res.F_aR <= k;
         b = sm->res.b;
     }

@@ -131,6 +131,17 @@ __device__ __forceinline__ double gap_factor(float lo, float hi, double inv_t) {
     return exp(((double)lo - (double)hi) * inv_t);
 }
 
+// Out-of-line fp64 exponential and logarithms for the single-CTA solve steps.
+// Those steps run most of their code once, so every inlined copy of a libm
+// routine is fetched cold into the instruction cache; one shared copy per
+// routine is fetched once and then stays hot.
+static __device__ __noinline__ double cold_exp(double x) { return exp(x); }
+static __device__ __noinline__ double cold_log(double x) { return log(x); }
+static __device__ __noinline__ double cold_log1p(double x) { return log1p(x); }
+__device__ __forceinline__ double gap_factor_cold(float lo, float hi, double inv_t) {
+    return cold_exp(((double)lo - (double)hi) * inv_t);
+}
+
 // ---------------------------------------------------------------------------
 // Affine maps x -> a x + c, the element of the stable prefix/suffix scans.
 // The prefix sum P_j = sum_{i<=j} e^{(s_i - s_j)/t} obeys P_j = 1 + g_j P_{j-1}
@@ -242,23 +253,23 @@ __device__ inline double segment_root(bool hasL, double sL, double Bh, bool hasR
     double b;
     if (!hasL && !hasR) return nan("");
     if (!hasL) {
-        b = sR + t * log(2.0 * c / Ah);
+        b = sR + t * cold_log(2.0 * c / Ah);
     } else if (!hasR) {
-        b = sL + t * log(Bh / (-2.0 * c));
+        b = sL + t * cold_log(Bh / (-2.0 * c));
     } else {
         double lnd = (sL - sR) / t;
-        double lnA = log(Ah), lnB = log(Bh);
+        double lnA = cold_log(Ah), lnB = cold_log(Bh);
         double ln_y;
         if (c == 0.0) {
             ln_y = 0.5 * (lnB + lnd - lnA);
         } else {
-            double lnc = log(fabs(c));
+            double lnc = cold_log(fabs(c));
             double lnrho = lnA + lnB + lnd - 2.0 * lnc;  // rho = Ah Bh delta / c^2
-            double lnS = lnrho > 0.0 ? 0.5 * (lnA + lnB + lnd) + 0.5 * log1p(exp(-lnrho))
-                                     : lnc + 0.5 * log1p(exp(lnrho));
-            double rc = exp(lnc - lnS);                   // |c| / S <= 1
-            if (c > 0.0) ln_y = lnS + log1p(rc) - lnA;     // ln(c + S) - ln Ah
-            else ln_y = lnB + lnd - (lnS + log1p(rc));    // ln Bh + ln delta - ln(S - c)
+            double lnS = lnrho > 0.0 ? 0.5 * (lnA + lnB + lnd) + 0.5 * cold_log1p(cold_exp(-lnrho))
+                                     : lnc + 0.5 * cold_log1p(cold_exp(lnrho));
+            double rc = cold_exp(lnc - lnS);                   // |c| / S <= 1
+            if (c > 0.0) ln_y = lnS + cold_log1p(rc) - lnA;     // ln(c + S) - ln Ah
+            else ln_y = lnB + lnd - (lnS + cold_log1p(rc));    // ln Bh + ln delta - ln(S - c)
         }
         b = sR + t * ln_y;
         if (b < sL) b = sL;

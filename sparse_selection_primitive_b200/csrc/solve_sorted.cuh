@@ -52,9 +52,9 @@ struct GapFn {
     double inv_t;
     // factor between positions j-1 and j (anchors at -1 and nb)
     __device__ __forceinline__ double operator()(long long j) const {
-        if (j <= 0) return (j == 0 && tl.hasL && nb > 0) ? gap_factor(tl.aL, get(0), inv_t) : 0.0;
-        if (j >= nb) return (j == nb && tl.hasR) ? gap_factor(get(nb - 1), tl.aR, inv_t) : 0.0;
-        return gap_factor(get(j - 1), get(j), inv_t);
+        if (j <= 0) return (j == 0 && tl.hasL && nb > 0) ? gap_factor_cold(tl.aL, get(0), inv_t) : 0.0;
+        if (j >= nb) return (j == nb && tl.hasR) ? gap_factor_cold(get(nb - 1), tl.aR, inv_t) : 0.0;
+        return gap_factor_cold(get(j - 1), get(j), inv_t);
     }
 };
 
@@ -135,8 +135,8 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
             out->jstar = 0;
             out->b = segment_root(tl.hasL, tl.aL, tl.SL, tl.hasR, tl.aR, tl.SR, tl.cntR - k, t);
             const double lnw = (tl.hasL && tl.hasR) ? ((double)tl.aL - (double)tl.aR) / t : -INFINITY;
-            out->F_aL = tl.hasL ? tl.cntR - 0.5 * tl.SR * exp(lnw) + 0.5 * tl.SL : INFINITY;
-            out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * tl.SL * exp(lnw) : -INFINITY;
+            out->F_aL = tl.hasL ? tl.cntR - 0.5 * tl.SR * cold_exp(lnw) + 0.5 * tl.SL : INFINITY;
+            out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * tl.SL * cold_exp(lnw) : -INFINITY;
         }
         __syncthreads();
         return;

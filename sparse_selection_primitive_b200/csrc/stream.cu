@@ -40,9 +40,10 @@ __device__ __forceinline__ void load_tile(const float* __restrict__ row, int64_t
             }
         }
     } else {
+        // scalar accesses in the same element order as the float4 path
 #pragma unroll
         for (int q = 0; q < kPer; ++q) {
-            const int64_t i = base + (int64_t)q * kThreads + threadIdx.x;
+            const int64_t i = base + ((int64_t)(q / 4) * kThreads + threadIdx.x) * 4 + q % 4;
             ok[q] = i < n;
             x[q] = ok[q] ? row[i] : 0.f;
         }
@@ -68,7 +69,7 @@ __device__ __forceinline__ void store_tile(float* __restrict__ row, int64_t n, i
     } else {
 #pragma unroll
         for (int q = 0; q < kPer; ++q) {
-            const int64_t i = base + (int64_t)q * kThreads + threadIdx.x;
+            const int64_t i = base + ((int64_t)(q / 4) * kThreads + threadIdx.x) * 4 + q % 4;
             if (i < n) row[i] = y[q];
         }
     }
@@ -182,9 +183,8 @@ __global__ void __launch_bounds__(kThreads) emit_kernel(const float* __restrict_
             y[q] = cdf_from(xs, e);
             if (SUMF && ok[q]) sf += 0.5 * (double)e;
             if (SUP) {
-                // load_tile's element order: float4 groups, or plain striding
-                const uint32_t pos = VEC ? (uint32_t)(4 * ((q / 4) * kThreads + threadIdx.x) + q % 4)
-                                         : (uint32_t)(q * kThreads + threadIdx.x);
+                // load_tile's element order (the same with and without float4)
+                const uint32_t pos = (uint32_t)(4 * ((q / 4) * kThreads + threadIdx.x) + q % 4);
                 const bool k0 = ok[q] && fabsf(xs) <= kSupWindow;
                 put(k0, __ballot_sync(0xffffffffu, k0), pos, xs);
             }

@@ -8,15 +8,15 @@
 // it also lists those scores (position in the tile and x) per warp share of
 // each 4096-score tile.  The backward then never reads r:
 //
-// Pass A (sup_reduce_kernel): each CTA takes a group of tiles, scans the
-//   shares' counts, and walks the listed entries with all its threads: v is
-//   gathered at each entry (and kept next to it for pass B), the terms go into
-//   an online (mu, sum w, sum w v), w = exp(-(|x| - mu)).  The last CTA of the
-//   row combines the CTA records in a fixed order into R and decides whether
-//   the list serves the row.
-// Pass B (sup_write_kernel): g tile by tile; the tile is zeroed in shared
-//   memory, its entries are placed, and it is written out with coalesced
-//   16-byte stores, so every g value is written exactly once.
+// Pass A (sup_reduce_kernel): one wave of resident CTAs; each walks groups of
+//   up to 32 tiles, scans the shares' counts, and works through the listed
+//   entries with all its threads: v is gathered at each entry (and kept next
+//   to it for pass B), the terms go into an online (mu, sum w, sum w v),
+//   w = exp(-(|x| - mu)).  The last CTA of the row combines the CTA records in
+//   a fixed order into R and decides whether the list serves the row.
+// Pass B (sup_write_kernel): one CTA per tile, one warp per share; the share is
+//   zeroed in shared memory, its entries are placed, and it is written out
+//   with coalesced 16-byte stores, so every g value is written exactly once.
 //
 // A row is handed to the dense two-pass kernels when its list overflowed, was
 // written for another (n, B) or another b, holds an index out of range, or
@@ -48,7 +48,7 @@ __device__ __forceinline__ void sup_add(float ax, float vv, float& mu, double& s
     sv += (double)(w * vv);
 }
 
-__global__ void __launch_bounds__(kThreads) sup_reduce_kernel(
+__global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     const double* __restrict__ b, const float* __restrict__ v, int64_t ld, int64_t n,
     int64_t B_total, int group, SupportView sup, double* __restrict__ partials,
     double* __restrict__ row_R, uint32_t* __restrict__ tickets, uint32_t* __restrict__ dense_flag) {
@@ -60,80 +60,98 @@ __global__ void __launch_bounds__(kThreads) sup_reduce_kernel(
     const int64_t row = blockIdx.y;
     const int64_t nblk = gridDim.x;
     const int64_t tiles = (n + kTile - 1) / kTile;
-    const int64_t t0 = (int64_t)blockIdx.x * group;
-    const int64_t t1 = t0 + group < tiles ? t0 + group : tiles;
+    const int64_t ngroups = (tiles + group - 1) / group;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* vr = v + row * ld;
     // the list must come from a forward over the same (n, B) with this b
     const bool match = sup.hdr[0] == n && sup.hdr[1] == B_total &&
                        __double_as_longlong(sup.b[row]) == __double_as_longlong(b[row]);
-    // one share per thread: (tile t0 + i / 8, share i % 8)
-    uint32_t c = 0;
     int bad = match ? 0 : 1;
-    if (match && t0 + (int64_t)threadIdx.x / kShares < t1) {
-        c = sup.cnt[(row * tiles + t0) * kShares + threadIdx.x];
+    float mu = INFINITY, amin = INFINITY;
+    double s = 0.0, sv = 0.0;
+    // count of share i of group gi: (tile gi * group + i / 8, share i % 8), or 0
+    auto share_count = [&](int64_t gi) -> uint32_t {
+        const int64_t t0 = gi * group;
+        const int64_t t1 = t0 + group < tiles ? t0 + group : tiles;
+        if (!match || gi >= ngroups || t0 + (int64_t)threadIdx.x / kShares >= t1) return 0u;
+        return __ldcs(sup.cnt + (row * tiles + t0) * kShares + threadIdx.x);
+    };
+    // persistent over groups of tiles; the next group's counts load while
+    // the current group's entries are gathered
+    uint32_t c_next = share_count(blockIdx.x);
+    for (int64_t gi = blockIdx.x; gi < ngroups; gi += nblk) {
+        const int64_t t0 = gi * group;
+        uint32_t c = c_next;
         if (c > (uint32_t)kSupCap) {
             bad = 1;
             c = 0;
         }
-    }
-    // block exclusive scan of the counts
-    uint32_t inc = c;
+        // block exclusive scan of the counts
+        uint32_t inc = c;
 #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, inc, d);
-        if (lane >= d) inc += o;
-    }
-    if (lane == 31) wtot[warp] = inc;
-    __syncthreads();
-    uint32_t wpre = 0;
-    for (int u = 0; u < warp; ++u) wpre += wtot[u];
-    pre[threadIdx.x] = wpre + inc - c;
-    if (threadIdx.x == kThreads - 1) pre[kThreads] = wpre + inc;
-    __syncthreads();
-    const uint32_t total = pre[kThreads];
-    const uint2* ent = sup.ent + (row * tiles + t0) * kShares * kSupCap;
-    float* val = sup.val + (row * tiles + t0) * kShares * kSupCap;
-    float mu = INFINITY, amin = INFINITY;
-    double s = 0.0, sv = 0.0;
-    constexpr int U = 4;  // entries per thread in flight
-    for (uint32_t j0 = 0; j0 < total; j0 += U * kThreads) {
-        uint2 e[U];
-        int64_t slot[U], gpos[U];
-        bool ok[U];
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t o = __shfl_up_sync(0xffffffffu, inc, d);
+            if (lane >= d) inc += o;
+        }
+        __syncthreads();  // the previous group is done with pre[] and wtot[]
+        if (lane == 31) wtot[warp] = inc;
+        __syncthreads();
+        uint32_t wpre = 0;
+        for (int u = 0; u < warp; ++u) wpre += wtot[u];
+        pre[threadIdx.x] = wpre + inc - c;
+        if (threadIdx.x == kThreads - 1) pre[kThreads] = wpre + inc;
+        __syncthreads();
+        c_next = share_count(gi + nblk);
+        const uint32_t total = pre[kThreads];
+        const uint2* ent = sup.ent + (row * tiles + t0) * kShares * kSupCap;
+        float* val = sup.val + (row * tiles + t0) * kShares * kSupCap;
+        const float* vg = vr + t0 * kTile;                  // v of the group's first tile
+        const int64_t lim = n - t0 * kTile;                 // scores of the row from there on
+        constexpr int U = 4;  // entries per thread in flight
+        for (uint32_t j0 = 0; j0 < total; j0 += U * kThreads) {
+            uint2 e[U];
+            int32_t slot[U];
+            int32_t gpos[U];  // position from the group's first score
+            bool ok[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint32_t j = j0 + u * kThreads + threadIdx.x;
-            ok[u] = j < total;
-            slot[u] = 0;
-            if (ok[u]) {
-                // share holding entry j: the last with pre[share] <= j
-                int lo = 0, hi = kThreads - 1;
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (pre[mid] <= j) lo = mid;
-                    else hi = mid - 1;
+            for (int u = 0; u < U; ++u) {
+                const uint32_t j = j0 + u * kThreads + threadIdx.x;
+                ok[u] = j < total;
+                slot[u] = 0;
+                gpos[u] = 0;
+                if (ok[u]) {
+                    // share holding entry j: the last with pre[share] <= j
+                    int lo = 0, hi = kThreads - 1;
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (pre[mid] <= j) lo = mid;
+                        else hi = mid - 1;
+                    }
+                    slot[u] = lo * kSupCap + (int32_t)(j - pre[lo]);
+                    e[u] = __ldcs(ent + slot[u]);
+                    gpos[u] = (lo / kShares) * kTile;
                 }
-                slot[u] = (int64_t)lo * kSupCap + (j - pre[lo]);
-                e[u] = __ldcs(ent + slot[u]);
-                const int64_t tile = t0 + lo / kShares;
-                gpos[u] = tile * kTile + e[u].x;
-                if (e[u].x >= (uint32_t)kTile || gpos[u] >= n) {
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                gpos[u] += (int32_t)(e[u].x & (kTile - 1));
+                if (e[u].x >= (uint32_t)kTile || gpos[u] >= lim) {
                     ok[u] = false;
                     bad = 1;
                 }
             }
-        }
-        float vv[U];
+            float vv[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) vv[u] = ok[u] ? __ldcs(vr + gpos[u]) : 0.f;
+            for (int u = 0; u < U; ++u) vv[u] = ok[u] ? __ldcs(vg + gpos[u]) : 0.f;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            if (!ok[u]) continue;
-            const float ax = fabsf(__uint_as_float(e[u].y));
-            amin = fminf(amin, ax);
-            sup_add(ax, vv[u], mu, s, sv);
-            val[slot[u]] = vv[u];
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                const float ax = fabsf(__uint_as_float(e[u].y));
+                amin = fminf(amin, ax);
+                sup_add(ax, vv[u], mu, s, sv);
+                val[slot[u]] = vv[u];
+            }
         }
     }
     // CTA record (mu, S, Sv, min |x| or -1 when the list cannot serve the row)
@@ -189,59 +207,58 @@ __global__ void __launch_bounds__(kThreads) sup_reduce_kernel(
 
 // g for one tile per CTA: zeroed in shared memory, the listed entries placed,
 // then written with 16-byte streaming stores.
+// g from the list, one CTA per tile.  Each warp owns one share of the tile,
+// the same 512 scores the emit kernel's warp listed (four runs of 128 at
+// q * 1024 + warp * 128), so no warp needs another's entries and there is no
+// block barrier.  The share's count and its first 32 entries are loaded
+// together (the entries speculatively), so a tile costs one memory round
+// trip; the share is zeroed in the warp's 2 KB of shared memory, its entries
+// are placed, and it is written with 16-byte streaming stores.
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) sup_write_kernel(
     SupportView sup, const uint32_t* __restrict__ dense_flag, const double* __restrict__ row_R,
     float* __restrict__ g, int64_t ld, int64_t n, double t) {
-    __shared__ __align__(16) float tile[kTile];
-    __shared__ uint32_t pre[kShares + 1];
+    __shared__ __align__(16) float stage[kShares][kTile / kShares];
     const int64_t row = blockIdx.y;
-    if (dense_flag[row]) return;  // the dense kernels own this row
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t tiles = (n + kTile - 1) / kTile;
     const int64_t T = blockIdx.x;
     const int64_t base = T * kTile;
+    const int64_t share = (row * tiles + T) * kShares + warp;
+    const uint2* ent = sup.ent + share * kSupCap;
+    const float* val = sup.val + share * kSupCap;
+    // independent loads, issued together
+    const uint32_t dflag = dense_flag[row];
     const double R = row_R[row];
+    const uint32_t c = __ldcs(sup.cnt + share);  // <= kSupCap: checked by pass A
+    const uint2 e0 = __ldcs(ent + lane);
+    const float v0 = __ldcs(val + lane);
+    if (dflag) return;  // the dense kernels own this row
     const float hinv = (float)(0.5 / t);
-    float4* t4 = reinterpret_cast<float4*>(tile);
+    float* st = stage[warp];
+    float4* s4 = reinterpret_cast<float4*>(st);
+    constexpr int kRun = kTile / kShares / 4;  // 128 scores per run, four runs per share
     const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int q = 0; q < kTile / 4 / kThreads; ++q) t4[q * kThreads + threadIdx.x] = z4;
-    if (threadIdx.x < 32) {
-        // counts were checked (<= kSupCap) by pass A before it cleared the row
-        const uint32_t c = threadIdx.x < kShares ? sup.cnt[(row * tiles + T) * kShares + threadIdx.x]
-                                                 : 0u;
-        uint32_t inc = c;
-#pragma unroll
-        for (int d = 1; d < kShares; d <<= 1) {
-            const uint32_t o = __shfl_up_sync(0xffffffffu, inc, d);
-            if (threadIdx.x >= d) inc += o;
-        }
-        if (threadIdx.x < kShares) pre[threadIdx.x] = inc - c;
-        if (threadIdx.x == kShares - 1) pre[kShares] = inc;
-    }
-    __syncthreads();
-    const uint32_t total = pre[kShares];
-    const uint2* ent = sup.ent + (row * tiles + T) * kShares * kSupCap;
-    const float* val = sup.val + (row * tiles + T) * kShares * kSupCap;
-    for (uint32_t j = threadIdx.x; j < total; j += kThreads) {
-        int sh = 0;
-#pragma unroll
-        for (int u = 1; u < kShares; ++u) sh += (pre[u] <= j) ? 1 : 0;
-        const int64_t slot = (int64_t)sh * kSupCap + (j - pre[sh]);
-        const uint2 e = __ldcs(ent + slot);
-        const float vv = __ldcs(val + slot);
-        const float ax = fabsf(__uint_as_float(e.y));
-        tile[e.x & (kTile - 1)] = hinv * __expf(-ax) * (float)((double)vv - R);
-    }
-    __syncthreads();
-    float* gr = g + row * ld + base;
+    for (int q = 0; q < 4; ++q) s4[q * 32 + lane] = z4;
+    __syncwarp();
+    auto place = [&](uint2 en, float vv) {
+        const uint32_t p = en.x & (kTile - 1);
+        const uint32_t li = (p >> 10) * kRun + (p & (kRun - 1));  // run q = p / 1024
+        st[li] = hinv * __expf(-fabsf(__uint_as_float(en.y))) * (float)((double)vv - R);
+    };
+    if ((uint32_t)lane < c) place(e0, v0);
+    for (uint32_t e = 32 + lane; e < c; e += 32) place(__ldcs(ent + e), __ldcs(val + e));
+    __syncwarp();
+    float* gs = g + row * ld + base + warp * kRun;
     if (VEC && base + kTile <= n) {
-        float4* g4 = reinterpret_cast<float4*>(gr);
 #pragma unroll
-        for (int q = 0; q < kTile / 4 / kThreads; ++q)
-            __stcs(g4 + q * kThreads + threadIdx.x, t4[q * kThreads + threadIdx.x]);
+        for (int q = 0; q < 4; ++q)
+            __stcs(reinterpret_cast<float4*>(gs + q * 1024) + lane, s4[q * 32 + lane]);
     } else {
-        for (int e = threadIdx.x; e < kTile && base + e < n; e += kThreads) gr[e] = tile[e];
+        for (int q = 0; q < 4; ++q)
+            for (int e = lane; e < kRun; e += 32)
+                if (base + warp * kRun + q * 1024 + e < n) gs[q * 1024 + e] = st[q * kRun + e];
     }
 }
 
@@ -309,11 +326,23 @@ cudaError_t launch_backward_support(const float* r, int64_t ld, const double* b,
                                     double* row_R, uint32_t* tickets, uint32_t* dense_flag,
                                     int vec, cudaStream_t st) {
     const int64_t tiles = stream_tiles(n);
-    // pass A: groups of tiles sized so all rows together give about 8 CTAs per SM
-    int64_t group = (B * tiles + (int64_t)sm_count() * 8 - 1) / ((int64_t)sm_count() * 8);
+    // pass A: one wave of resident CTAs walking groups of up to 32 tiles;
+    // pass B: one CTA per tile
+    static int cap_a = 0;
+    if (cap_a == 0) {
+        int pa = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pa, sup_reduce_kernel, kThreads, 0);
+        cap_a = (pa > 0 ? pa : 1) * sm_count();
+    }
+    int64_t want = cap_a / B;
+    if (want < 1) want = 1;
+    // groups of at most 32 tiles, as many per CTA as it takes, all CTAs alike
+    const int64_t rounds = (tiles + kGroupMax * want - 1) / (kGroupMax * want);
+    int64_t group = (tiles + rounds * want - 1) / (rounds * want);
     if (group < 1) group = 1;
     if (group > kGroupMax) group = kGroupMax;
-    const int64_t per_row = (tiles + group - 1) / group;
+    const int64_t ngroups = (tiles + group - 1) / group;
+    const int64_t per_row = ngroups < want ? ngroups : want;
     {
         ProfScope ps_("sup_reduce", st);
         sup_reduce_kernel<<<dim3((unsigned)per_row, (unsigned)B), kThreads, 0, st>>>(

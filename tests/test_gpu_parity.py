@@ -281,3 +281,4 @@ def test_autograd_long_rows_use_support(cuda_device):
     g = L.backward(rt.detach(), b, torch.from_numpy(v).cuda(), 0.01)
     scale = g.abs().max().item()
     assert (rt.grad - g).abs().max().item() <= 1e-5 * scale
+
