@@ -76,6 +76,31 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
+# Ranks: one process per GPU, each solving its own workload instance
+# ---------------------------------------------------------------------------
+def rank_env():
+    """(world, rank, local_rank) from the launcher's environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (every rank gets it); x itself when alone."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_value(elements_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the elements of every rank over the slowest rank's time."""
+    return elements_per_rank * world / (ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # nvidia-smi clock sampling during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -204,9 +229,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
 
     if args.impl == "reference":
         run_reference(args, rank, world)
@@ -227,13 +250,6 @@ def main():
     def barrier():
         if world > 1:
             dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        tt = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        return float(tt.item())
 
     L._build.build()
     w = WORKLOADS[args.workload]
@@ -340,10 +356,10 @@ def main():
     barrier()
     clocks = sampler.stop()
     ms_local = statistics.mean(step_ms)
-    eager_ms_max = max_over_ranks(statistics.mean(eager_ms))
-    ms = max_over_ranks(ms_local)
+    eager_ms_max = max_over_ranks(statistics.mean(eager_ms), world, dev)
+    ms = max_over_ranks(ms_local, world, dev)
     elements = w.elements * world
-    value = elements / (ms / 1e3)
+    value = job_value(w.elements, world, ms)
 
     # dominant kernel of the timed region
     dom_name, (dom_launch, dom_ms) = max(prof.items(), key=lambda kv: kv[1][1])
@@ -396,7 +412,7 @@ def main():
         e_e.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / k_e2e)
+        e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / k_e2e, world, dev)
         nb = r_pin.numel() * 4
         e2e = {"value": elements / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 2 * nb, "d2h_bytes_per_step": 2 * nb}
