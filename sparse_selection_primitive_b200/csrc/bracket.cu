@@ -372,7 +372,7 @@ __device__ __forceinline__ void bin_add(float x, const BinLayout& BL, float inv_
     atomicAdd(&bins[2 * kBins + j], __float2ull_rn(__expf((x - hi) * inv_t) * (float)kFixScale));
 }
 
-constexpr int kStage = 2048;  // band scores staged per CTA before one global append
+constexpr int kStage = 1024;  // band scores staged per CTA before one global append
 
 // One lane appends one band score to the CTA staging buffer (or, when it is
 // full, straight to the global band).
@@ -433,6 +433,13 @@ __device__ __forceinline__ void band_flush(const float* sband, int scount, float
 }
 
 constexpr int kQ = 1024;  // per-warp circular queue of near scores (power of two)
+constexpr size_t kFoldDynSmem = (size_t)(kFoldThreads / 32) * (kQ + 32 * 16) * sizeof(float);
+
+// Swizzled slot of value j (0..15) in a lane's 16-float staging row, so that a
+// warp's 16-byte stores of the four float4 groups hit distinct banks.
+__device__ __forceinline__ int stage_slot(int lane, int j) {
+    return lane * 16 + ((((j >> 2) ^ (lane >> 1)) & 3) << 2) + (j & 3);
+}
 
 __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __restrict__ r, int64_t n,
                                                             double t, RowState* st,
@@ -444,7 +451,8 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     __shared__ double red[kFoldThreads / 32];
     __shared__ long long lred[kFoldThreads / 32];
     __shared__ float sband[kStage];
-    __shared__ float wq[kFoldThreads / 32][kQ];
+    // dynamic: per-warp queues (kQ floats each), then per-warp staging rows
+    extern __shared__ __align__(16) float fold_dyn[];
     __shared__ int scount;
     __shared__ unsigned long long gbase;
     __shared__ int flag;
@@ -452,21 +460,26 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     // Scores more than 90 t below the bracket add exactly 0 to the left tail
     // sum in fp32, and scores more than 90 t above it add 1 to the right count
     // and 0 to its sum; only the scores between these limits ("near") need
-    // the full fold.  Each trip builds a 16-bit near mask per thread; a warp
-    // that has near scores appends them to its circular queue (one warp scan)
-    // and folds them 32 at a time, so the lanes stay busy on them however
-    // sparse they are.
+    // the full fold.  Each trip classifies 16 scores per thread with two
+    // compares each (a 16-bit near mask and the far-right count); a warp with
+    // near scores stages the trip's values in shared memory, and each lane
+    // copies its near ones into the warp's circular queue at its scan offset.
+    // The queue is folded 32 scores at a time, so the lanes stay busy on the
+    // near scores however sparse they are.  Non-finite scores are caught by a
+    // running sum (checked exactly if it overflows).
     const float aLf = aL - (float)(90.0 * t), aRf = aR + (float)(90.0 * t);
     const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
     const float inv_t = (float)(1.0 / t);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float* q = wq[warp];
+    float* q = fold_dyn + warp * kQ;
+    float* stg = fold_dyn + (kFoldThreads / 32) * kQ + warp * (32 * 16);
     uint32_t head = 0, tail = 0;  // warp-uniform; tail - head = queued scores
     if (threadIdx.x == 0) scount = 0;
     if (blockIdx.x == 0) phase_mark(st, 16);
     __syncthreads();
     FoldAcc acc{0u, 0.0, 0.0, false};
     uint32_t far_right = 0u;
+    float xsum = 0.f;
     bool bad = false;
     unsigned long long* counter = &st->n_band;
     const unsigned long long cap = (unsigned long long)n;
@@ -480,6 +493,28 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
         band_stage(inb, x, sband, &scount, band, counter, cap, BL, inv_t, bins);
         head += cnt;
     };
+    // appends the near values of a staged trip (16 per lane, mask m) to the queue
+    auto push_staged = [&](uint32_t m) {
+        const int c = __popc(m);
+        int incl = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        __syncwarp();
+        uint32_t off = tail + (uint32_t)(incl - c);
+        while (m != 0u) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1u;
+            q[(off++) & (kQ - 1)] = stg[stage_slot(lane, j)];
+        }
+        tail += (uint32_t)total;
+        __syncwarp();
+        while (tail - head >= 32u) drain(32);
+    };
+    // the generic path for short or ragged parts: values in registers
     auto push = [&](const float* xs, uint32_t m, int cnt_max) {
         __syncwarp();
         const int c = __popc(m);
@@ -498,10 +533,10 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
         while (tail - head >= 32u) drain(32);
     };
     auto classify = [&](float x, bool valid, uint32_t& m, int j) {
-        const bool nr = valid && (x >= aLf) && (x < aRf);
-        m |= (uint32_t)nr << j;
-        far_right += (valid && x >= aRf) ? 1u : 0u;
-        bad |= valid && !(fabsf(x) <= 3.402823466e38f);
+        const bool ge_l = valid && x >= aLf, ge_r = valid && x >= aRf;
+        m |= (uint32_t)(ge_l && !ge_r) << j;
+        far_right += ge_r ? 1u : 0u;
+        if (valid) xsum += x;
     };
     if (vec) {
         const int64_t n4 = n >> 2;
@@ -518,22 +553,27 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
             for (int qq = 0; qq < U; ++qq) nv[qq] = __ldcs(p + (int64_t)qq * nthreads);
         }
         for (int64_t it = 0; it < full; ++it, p += step) {
-            float xs[4 * U];
+            float4 cur[U];
 #pragma unroll
-            for (int qq = 0; qq < U; ++qq) {
-                xs[4 * qq] = nv[qq].x;
-                xs[4 * qq + 1] = nv[qq].y;
-                xs[4 * qq + 2] = nv[qq].z;
-                xs[4 * qq + 3] = nv[qq].w;
-            }
+            for (int qq = 0; qq < U; ++qq) cur[qq] = nv[qq];
             if (it + 1 < full) {
 #pragma unroll
                 for (int qq = 0; qq < U; ++qq) nv[qq] = __ldcs(p + step + (int64_t)qq * nthreads);
             }
             uint32_t m = 0u;
 #pragma unroll
-            for (int j = 0; j < 4 * U; ++j) classify(xs[j], true, m, j);
-            if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 4 * U);
+            for (int qq = 0; qq < U; ++qq) {
+                classify(cur[qq].x, true, m, 4 * qq);
+                classify(cur[qq].y, true, m, 4 * qq + 1);
+                classify(cur[qq].z, true, m, 4 * qq + 2);
+                classify(cur[qq].w, true, m, 4 * qq + 3);
+            }
+            if (__any_sync(0xffffffffu, m != 0u)) {
+#pragma unroll
+                for (int qq = 0; qq < U; ++qq)
+                    *reinterpret_cast<float4*>(stg + stage_slot(lane, 4 * qq)) = cur[qq];
+                push_staged(m);
+            }
         }
         // Remainder: the last partial trip, with bounds checks.
         const int64_t rem_iters = (n4 - full * step + nthreads - 1) / nthreads;
@@ -564,6 +604,21 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
             uint32_t m = 0u;
             classify(xs[0], i < n, m, 0);
             if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 1);
+        }
+    }
+    if (!(fabsf(xsum) <= 3.402823466e38f)) {
+        // a NaN or an infinity, or only an overflowing sum: check this
+        // thread's scores one by one (rare)
+        if (vec) {
+            const int64_t n4 = n >> 2;
+            for (int64_t i = gtid; i < n4; i += nthreads) {
+                const float4 v = reinterpret_cast<const float4*>(r)[i];
+                bad |= !finite_f(v.x) || !finite_f(v.y) || !finite_f(v.z) || !finite_f(v.w);
+            }
+            if (blockIdx.x == 0 && threadIdx.x < 32 && (n4 << 2) + threadIdx.x < n)
+                bad |= !finite_f(r[(n4 << 2) + threadIdx.x]);
+        } else {
+            for (int64_t i = gtid; i < n; i += nthreads) bad |= !finite_f(r[i]);
         }
     }
     while (tail != head) drain((int)min(32u, tail - head));
@@ -1403,7 +1458,10 @@ int bracket_fold_grid() {
         int dev = 0, sms = 148, per = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fold_kernel, kFoldThreads, 0);
+        cudaFuncSetAttribute(fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kFoldDynSmem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fold_kernel, kFoldThreads,
+                                                      kFoldDynSmem);
         grid = sms * (per > 0 ? per : 1);
     }
     return grid;
@@ -1413,17 +1471,24 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                                int64_t row, int m, int64_t rank_l[kLadder],
                                int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,
                                RowState* st_row, double* b_out, WsHeader* hdr, cudaStream_t st) {
-    static bool attr_done = false;
+    // dynamic shared memory limits, set once per device (they belong to the
+    // device's copy of the module)
+    static unsigned long long attr_devices = 0ull;
     const size_t solve_smem = sizeof(SolveSmemAll);
     const size_t sample_smem = (size_t)2 * kBandSortMax * sizeof(uint32_t);
-    if (!attr_done) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if ((attr_devices & bit) == 0ull || bit == 0ull) {
         cudaFuncSetAttribute(solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)solve_smem);
         cudaFuncSetAttribute(solve2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)solve_smem);
         cudaFuncSetAttribute(sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(2 * kBandSortMax * sizeof(uint32_t)));
-        attr_done = true;
+                             (int)sample_smem);
+        cudaFuncSetAttribute(fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kFoldDynSmem);
+        attr_devices |= bit;
     }
     Ladder lad;
     for (int i = 0; i < kLadder; ++i) {
@@ -1443,7 +1508,8 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
     {
         ProfScope ps_("bracket_fold", st);
-        fold_kernel<<<buf.fold_grid, kFoldThreads, 0, st>>>(r_row, n, t, st_row, buf.band[0],
+        fold_kernel<<<buf.fold_grid, kFoldThreads, kFoldDynSmem, st>>>(r_row, n, t, st_row,
+                                                                    buf.band[0],
                                                         buf.bins, buf.fold_part, buf.ticket, hdr,
                                                         vec);
     }

@@ -19,6 +19,12 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kPer = kStreamTile / kThreads;  // 16
 
+// Swizzled slot of value j (0..15) in a lane's 16-float staging row, so that a
+// warp's 16-byte stores of the four float4 groups hit distinct banks.
+__device__ __forceinline__ int stage_slot16(int lane, int j) {
+    return lane * 16 + ((((j >> 2) ^ (lane >> 1)) & 3) << 2) + (j & 3);
+}
+
 template <bool VEC>
 __device__ __forceinline__ void load_tile(const float* __restrict__ row, int64_t n, int64_t base,
                                           float (&x)[kPer], bool (&ok)[kPer]) {
@@ -128,17 +134,14 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
     const float* rr = r + row * ld;
     float* pr = p + row * ld;
     double sf = 0.0;
-    // gradient support of this warp's share of the tile
+    // gradient support of this warp's share of the tile: the margins are
+    // staged in shared memory with a near mask per thread; a warp with near
+    // scores then writes them (lane by lane, at scan offsets) to its share
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = (1u << lane) - 1u;
+    __shared__ __align__(16) float mstage[SUP ? kThreads * kPer : 1];
+    float* stg = mstage + (SUP ? warp * 32 * kPer : 0);
     const int64_t share = (row * tiles + blockIdx.x) * kSupWarps + warp;
-    uint2* ent = SUP ? sup.ent + share * kSupCap : nullptr;
-    uint32_t cnt = 0;  // warp-uniform
-    auto put = [&](bool near, unsigned ball, uint32_t pos_in_tile, float x) {
-        const uint32_t at = cnt + __popc(ball & lt);
-        if (near && at < (uint32_t)kSupCap) ent[at] = make_uint2(pos_in_tile, __float_as_uint(x));
-        cnt += __popc(ball);
-    };
+    uint32_t nm = 0u;  // near mask of this thread's 16 scores
     if (SUP && blockIdx.x == 0 && threadIdx.x == 0) sup.b[row] = brow;
     if (VEC && base + kStreamTile <= n) {
         const float4* r4 = reinterpret_cast<const float4*>(rr + base);
@@ -157,19 +160,12 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
                                cdf_from(m3, e3)));
             if (SUMF) sf += 0.5 * (double)((e0 + e1) + (e2 + e3));
             if (SUP) {
-                const bool k0 = fabsf(m0) <= kSupWindow, k1 = fabsf(m1) <= kSupWindow;
-                const bool k2 = fabsf(m2) <= kSupWindow, k3 = fabsf(m3) <= kSupWindow;
-                const unsigned b0 = __ballot_sync(0xffffffffu, k0);
-                const unsigned b1 = __ballot_sync(0xffffffffu, k1);
-                const unsigned b2 = __ballot_sync(0xffffffffu, k2);
-                const unsigned b3 = __ballot_sync(0xffffffffu, k3);
-                if ((b0 | b1 | b2 | b3) != 0u) {
-                    const uint32_t i0 = 4u * (uint32_t)(q * kThreads + threadIdx.x);
-                    put(k0, b0, i0, m0);
-                    put(k1, b1, i0 + 1, m1);
-                    put(k2, b2, i0 + 2, m2);
-                    put(k3, b3, i0 + 3, m3);
-                }
+                nm |= (fabsf(m0) <= kSupWindow ? 1u : 0u) << (4 * q);
+                nm |= (fabsf(m1) <= kSupWindow ? 1u : 0u) << (4 * q + 1);
+                nm |= (fabsf(m2) <= kSupWindow ? 1u : 0u) << (4 * q + 2);
+                nm |= (fabsf(m3) <= kSupWindow ? 1u : 0u) << (4 * q + 3);
+                *reinterpret_cast<float4*>(stg + stage_slot16(lane, 4 * q)) =
+                    make_float4(m0, m1, m2, m3);
             }
         }
     } else {
@@ -183,13 +179,35 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
             y[q] = cdf_from(xs, e);
             if (SUMF && ok[q]) sf += 0.5 * (double)e;
             if (SUP) {
-                // load_tile's element order (the same with and without float4)
-                const uint32_t pos = (uint32_t)(4 * ((q / 4) * kThreads + threadIdx.x) + q % 4);
-                const bool k0 = ok[q] && fabsf(xs) <= kSupWindow;
-                put(k0, __ballot_sync(0xffffffffu, k0), pos, xs);
+                nm |= ((ok[q] && fabsf(xs) <= kSupWindow) ? 1u : 0u) << q;
+                stg[stage_slot16(lane, q)] = xs;
             }
         }
         store_tile<VEC>(pr, n, base, y);
+    }
+    uint32_t cnt = 0;  // warp-uniform: entries found in this warp's share
+    if (SUP && __any_sync(0xffffffffu, nm != 0u)) {
+        const int c = __popc(nm);
+        int incl = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        cnt = (uint32_t)__shfl_sync(0xffffffffu, incl, 31);
+        __syncwarp();
+        uint2* ent = sup.ent + share * kSupCap;
+        uint32_t at = (uint32_t)(incl - c);
+        uint32_t mm = nm;
+        while (mm != 0u) {  // this lane's near scores, in element order
+            const int j = __ffs(mm) - 1;
+            mm &= mm - 1u;
+            // load_tile's element order (the same with and without float4)
+            const uint32_t pos = (uint32_t)(4 * ((j >> 2) * kThreads + threadIdx.x) + (j & 3));
+            if (at < (uint32_t)kSupCap)
+                ent[at] = make_uint2(pos, __float_as_uint(stg[stage_slot16(lane, j)]));
+            ++at;
+        }
     }
     if (SUP && lane == 0) sup.cnt[share] = cnt;
     if (!SUMF) return;
