@@ -66,7 +66,10 @@ enum lapsum_path {
 /* Test and diagnostic flags, OR-ed into `path`. */
 enum lapsum_flags {
     LAPSUM_FLAG_FORCE_MISS = 0x100, /* bracketing: start from a bracket that excludes b */
-    LAPSUM_FLAG_NO_RETRY = 0x200    /* bracketing: allow no widening (a miss => LAPSUM_EBRACKET) */
+    LAPSUM_FLAG_NO_RETRY = 0x200,   /* bracketing: allow no widening (a miss => LAPSUM_EBRACKET) */
+    LAPSUM_FLAG_ONE_CTA_SOLVE = 0x400 /* bracketing: solve every band inside the single-CTA
+                                         solve kernel, without the grid-wide extraction that
+                                         large first bands otherwise use */
 };
 
 /* Version of this ABI (incremented on any incompatible change). */

@@ -26,13 +26,14 @@ from . import _build
 __all__ = [
     "LapSumError", "Workspace", "forward", "backward", "read_status", "row_info", "sample_values",
     "workspace_bytes", "soft_topk", "LapSumTopK", "PATHS", "FLAG_FORCE_MISS", "FLAG_NO_RETRY",
-    "library_path", "profile_enable", "profile_read", "backward_noalloc", "Support",
+    "FLAG_ONE_CTA_SOLVE", "library_path", "profile_enable", "profile_read", "backward_noalloc", "Support",
     "support_bytes",
 ]
 
 PATHS = {"auto": 0, "fullsort": 1, "bracket": 2, "radix": 3}
 FLAG_FORCE_MISS = 0x100
 FLAG_NO_RETRY = 0x200
+FLAG_ONE_CTA_SOLVE = 0x400
 
 _c_i64 = ctypes.c_int64
 _vp = ctypes.c_void_p

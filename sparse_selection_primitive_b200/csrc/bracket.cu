@@ -32,6 +32,7 @@ namespace lapsum {
 namespace {
 
 constexpr int kBlk = 1024;
+constexpr int kWarpSortMax = 256;  // bands up to this size are sorted and solved by one warp
 constexpr int kFoldThreads = 256;
 
 struct Ladder {
@@ -107,99 +108,155 @@ struct GlobalSampleKeyGet {
     __device__ __forceinline__ uint32_t operator()(int i) const { return to_key(y[i]); }
 };
 
-// The rho_a-th and rho_b-th largest of the m sample values y[] (1-based;
-// 0 = not wanted), rho_max = the larger, given `hist`: the counts of the
-// samples' keys by their top 11 bits (2048 words of shared memory).  The bin
-// holding rank rho_max is found by a suffix scan; every sample in that bin or
-// above is a candidate.  If there are at most 4096 candidates they are
-// compacted and sorted with the register bitonic network and both ranks are
-// read off; otherwise returns false.  Needs blockDim.x == 1024.
-__device__ bool top_ranks(const float* __restrict__ y, int m, int64_t rho_max, int64_t rho_a,
-                          int64_t rho_b, const uint32_t* hist, uint32_t* wsum, uint32_t* bcast,
-                          uint32_t* cand, uint32_t* xch, float* out_a, float* out_b) {
-    // suffix counts: thread i owns bins 2i, 2i+1
+// For two ranks at once (1-based, descending; 0 = not wanted): the bin of
+// hist_a holding the ra-th largest and the bin of hist_b holding the rb-th
+// largest (hist_b may be hist_a), with the counts in higher bins.  Bins
+// 0..2047 in descending order; 1024 threads, two bins each; every thread gets
+// the results.  bcast: 4 words.
+__device__ void rank_bins2(const uint32_t* hist_a, const uint32_t* hist_b, int64_t ra, int64_t rb,
+                           uint32_t* wsum /*64*/, uint32_t* bcast, uint32_t* bin_a,
+                           uint32_t* above_a, uint32_t* bin_b, uint32_t* above_b) {
     const int i0 = 2 * threadIdx.x;
-    const uint32_t c0 = hist[i0], c1 = hist[i0 + 1];
-    const uint32_t mine = c0 + c1;
-    uint32_t incl = mine;
+    const uint32_t a0 = hist_a[i0], a1 = hist_a[i0 + 1];
+    const uint32_t b0 = hist_b[i0], b1 = hist_b[i0 + 1];
+    uint32_t ia = a0 + a1, ib = b0 + b1;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t o = __shfl_down_sync(0xffffffffu, incl, d);
-        if (lane + d < 32) incl += o;
-    }
-    if (lane == 0) wsum[w] = incl;
-    __syncthreads();
-    uint32_t above = incl - mine;
-    for (int u = w + 1; u < (int)(blockDim.x >> 5); ++u) above += wsum[u];
-    if (above < rho_max && rho_max <= (int64_t)above + c1) {
-        bcast[0] = i0 + 1;
-        bcast[1] = above + c1;  // candidates: keys in this bin or above
-    }
-    if ((int64_t)above + c1 < rho_max && rho_max <= (int64_t)above + c1 + c0) {
-        bcast[0] = i0;
-        bcast[1] = above + c1 + c0;
-    }
-    if (threadIdx.x == 0) bcast[2] = 0;
-    __syncthreads();
-    const uint32_t bin = bcast[0], ncand = bcast[1];
-    if (ncand > (uint32_t)kBandSortMax) return false;
-    // candidate pass: 8 samples per thread per trip, loads issued together
-    for (int s0 = 0; s0 < m; s0 += 8 * kBlk) {
-        float yv[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int s = s0 + q * kBlk + threadIdx.x;
-            yv[q] = s < m ? __ldcg(y + s) : -INFINITY;
+        const uint32_t oa = __shfl_down_sync(0xffffffffu, ia, d);
+        const uint32_t ob = __shfl_down_sync(0xffffffffu, ib, d);
+        if (lane + d < 32) {
+            ia += oa;
+            ib += ob;
         }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const uint32_t kk = to_key(yv[q]);
-            const bool take = (s0 + q * kBlk + (int)threadIdx.x < m) && (kk >> 21) >= bin;
+    }
+    if (lane == 0) {
+        wsum[w] = ia;
+        wsum[32 + w] = ib;
+    }
+    __syncthreads();
+    uint32_t xa = ia - (a0 + a1), xb = ib - (b0 + b1);  // counts above this thread's bins
+    for (int u = w + 1; u < (int)(blockDim.x >> 5); ++u) {
+        xa += wsum[u];
+        xb += wsum[32 + u];
+    }
+    auto find = [&](int64_t rho, uint32_t above, uint32_t c0, uint32_t c1, int slot) {
+        const int64_t s1 = above, s0 = (int64_t)above + c1;  // above bin i0+1 / bin i0
+        if (s1 < rho && rho <= s1 + c1) {
+            bcast[slot] = i0 + 1;
+            bcast[slot + 1] = (uint32_t)s1;
+        }
+        if (s0 < rho && rho <= s0 + c0) {
+            bcast[slot] = i0;
+            bcast[slot + 1] = (uint32_t)s0;
+        }
+    };
+    if (ra >= 1) find(ra, xa, a0, a1, 0);
+    if (rb >= 1) find(rb, xb, b0, b1, 2);
+    __syncthreads();
+    *bin_a = bcast[0];
+    *above_a = bcast[1];
+    *bin_b = bcast[2];
+    *above_b = bcast[3];
+    __syncthreads();
+}
+
+// Keys of the ra-th and rb-th largest (1-based; 0 = not wanted) of m sample
+// keys staged in shared memory, by a radix select whose first level (the
+// keys' top 11 bits) is the histogram hist1 the sample kernel already built;
+// levels two and three (11 and 10 bits) count, for each rank, only the keys
+// sharing its prefix (a few percent of the sample, so most warps skip the
+// counting).  h2: 2 x 2048 words.  Needs blockDim.x == 1024.
+__device__ void select_two_ranks(const uint32_t* keys, int m, const uint32_t* hist1, int64_t ra,
+                                 int64_t rb, uint32_t* h2, uint32_t* wsum, uint32_t* bcast,
+                                 uint32_t* key_a, uint32_t* key_b) {
+    const int lane = threadIdx.x & 31;
+    const bool wa = ra >= 1, wb = rb >= 1;
+    if (!wa && !wb) {  // both ends open
+        *key_a = 0u;
+        *key_b = 0u;
+        return;
+    }
+    uint32_t pa, pb, xa, xb;
+    rank_bins2(hist1, hist1, ra, rb, wsum, bcast, &pa, &xa, &pb, &xb);
+    // Keys in the lowest wanted bin or above: when there are few (the usual
+    // case for a small budget) one warp sorts them all and reads both ranks off.
+    const uint32_t low = wb ? pb : pa;
+    const uint32_t ncand = wb ? xb + hist1[pb] : xa + hist1[pa];
+    if (ncand <= (uint32_t)kWarpSortMax) {
+        uint32_t* cand = h2;
+        if (threadIdx.x == 0) bcast[0] = 0u;
+        __syncthreads();
+        for (int s0 = 0; s0 < m; s0 += blockDim.x) {  // same trip count in every lane
+            const int s = s0 + threadIdx.x;
+            const uint32_t k = s < m ? keys[s] : 0u;
+            const bool take = s < m && (k >> 21) >= low;
             const unsigned ball = __ballot_sync(0xffffffffu, take);
-            if (ball != 0u) {
-                const int leader = __ffs(ball) - 1;
-                uint32_t base = 0;
-                if (lane == leader) base = atomicAdd(&bcast[2], (uint32_t)__popc(ball));
-                base = __shfl_sync(0xffffffffu, base, leader);
-                if (take) cand[base + __popc(ball & ((1u << lane) - 1u))] = kk;
+            if (ball == 0u) continue;
+            const int leader = __ffs(ball) - 1;
+            uint32_t base = 0;
+            if (lane == leader) base = atomicAdd(&bcast[0], (uint32_t)__popc(ball));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            if (take) cand[base + __popc(ball & ((1u << lane) - 1u))] = k;
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            constexpr int E = kWarpSortMax / 32;
+            uint32_t key[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const uint32_t j = threadIdx.x * E + e;
+                key[e] = j < ncand ? cand[j] : 0u;  // padding sorts first
+            }
+            bitonic_sort_row<E, 32, 32>(key, threadIdx.x, nullptr);
+            // ascending: the r-th largest sits at position kWarpSortMax - r
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int j = threadIdx.x * E + e;
+                if (wa && j == kWarpSortMax - ra) bcast[2] = key[e];
+                if (wb && j == kWarpSortMax - rb) bcast[3] = key[e];
             }
         }
+        __syncthreads();
+        *key_a = bcast[2];
+        *key_b = bcast[3];
+        __syncthreads();
+        return;
     }
-    __syncthreads();
-    // ascending sort of the candidates (padding 0 sorts first); rank r from the
-    // top is at position npad - r
-    int npad;
-    if (ncand <= (uint32_t)kBlk) {
-        uint32_t key[1];
-        key[0] = (int)threadIdx.x < (int)ncand ? cand[threadIdx.x] : 0u;
-        bitonic_sort_block_rolled<1, kBlk>(key, threadIdx.x, xch);
-        cand[threadIdx.x] = key[0];
-        npad = kBlk;
-    } else {
-        uint32_t key[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int j = threadIdx.x * 4 + e;
-            key[e] = j < (int)ncand ? cand[j] : 0u;
+    int64_t rema = ra - xa, remb = rb - xb;
+#pragma unroll 1
+    for (int lev = 0; lev < 2; ++lev) {
+        const int sh = lev == 0 ? 10 : 0;          // position of this level's digit
+        const int psh = lev == 0 ? 21 : 10;        // the prefix is key >> psh
+        const uint32_t dmask = lev == 0 ? 2047u : 1023u;
+        for (int i = threadIdx.x; i < 2 * 2048; i += blockDim.x) h2[i] = 0u;
+        __syncthreads();
+        for (int s0 = 0; s0 < m; s0 += blockDim.x) {  // same trip count in every lane
+            const int s = s0 + threadIdx.x;
+            const uint32_t k = s < m ? keys[s] : 0u;
+            const bool ina = s < m && wa && (k >> psh) == pa;
+            const bool inb = s < m && wb && (k >> psh) == pb;
+            if (!__any_sync(0xffffffffu, ina || inb)) continue;
+            // lanes with the same digit add once (ties crowd into one bin)
+            const uint32_t da = ina ? ((k >> sh) & dmask) : 0xffffffffu;
+            const unsigned peers_a = __match_any_sync(0xffffffffu, da);
+            if (ina && lane == __ffs(peers_a) - 1) atomicAdd(&h2[da], (uint32_t)__popc(peers_a));
+            const uint32_t db = inb ? ((k >> sh) & dmask) : 0xffffffffu;
+            const unsigned peers_b = __match_any_sync(0xffffffffu, db);
+            if (inb && lane == __ffs(peers_b) - 1)
+                atomicAdd(&h2[2048 + db], (uint32_t)__popc(peers_b));
         }
-        bitonic_sort_block_rolled<4, kBlk>(key, threadIdx.x, xch);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) cand[threadIdx.x * 4 + e] = key[e];
-        npad = 4 * kBlk;
+        __syncthreads();
+        uint32_t ba, bb;
+        rank_bins2(h2, h2 + 2048, wa ? rema : 0, wb ? remb : 0, wsum, bcast, &ba, &xa, &bb, &xb);
+        const int width = lev == 0 ? 11 : 10;
+        pa = (pa << width) | ba;
+        pb = (pb << width) | bb;
+        rema -= xa;
+        remb -= xb;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        if (rho_a >= 1) *out_a = from_key(cand[npad - rho_a]);
-        if (rho_b >= 1) *out_b = from_key(cand[npad - rho_b]);
-        wsum[0] = __float_as_uint(*out_a);
-        wsum[1] = __float_as_uint(*out_b);
-    }
-    __syncthreads();
-    *out_a = __uint_as_float(wsum[0]);
-    *out_b = __uint_as_float(wsum[1]);
-    __syncthreads();
-    return true;
+    *key_a = pa;
+    *key_b = pb;
 }
 
 // ----------------------------------------------------------------------------
@@ -226,10 +283,10 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
         phase_mark(st, 14);
     }
     extern __shared__ uint32_t dyn[];
-    uint32_t* cand = dyn;                 // up to 4096 candidate keys
-    uint32_t* xch = cand + kBandSortMax;  // bitonic exchange area (4096 words)
+    uint32_t* skeys = dyn;               // the sample's keys (last CTA only), kSampleMax words
+    uint32_t* h2 = skeys + kSampleMax;   // select histograms, 2 x 2048 words
     __shared__ uint32_t hist[2048];
-    __shared__ uint32_t wsum[32];
+    __shared__ uint32_t wsum[64];
     __shared__ uint32_t bcast[4];
     __shared__ int flag;
     for (int i = threadIdx.x; i < 2048; i += kBlk) hist[i] = 0u;
@@ -273,28 +330,34 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
         hist[i] = __ldcg(ghist + i);
         ghist[i] = 0u;  // ready for the next call
     }
+    // the sample's keys into shared memory, eight loads in flight per thread
+    for (int s0 = 0; s0 < m; s0 += 8 * kBlk) {
+        float yv[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int s = s0 + q * kBlk + threadIdx.x;
+            yv[q] = s < m ? __ldcg(sample_out + s) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int s = s0 + q * kBlk + threadIdx.x;
+            if (s < m) skeys[s] = to_key(yv[q]);
+        }
+    }
     __syncthreads();
     float aR = INFINITY, aL = -INFINITY;
-    const int64_t rmax = lad.h[0] <= m ? lad.h[0] : lad.l[0];
-    if (rmax >= 1 && top_ranks(sample_out, m, rmax, lad.l[0], lad.h[0] <= m ? lad.h[0] : 0, hist,
-                               wsum, bcast, cand, xch, &aR, &aL)) {
-        // both order statistics read off the sorted top candidates
-    } else {
-        if (lad.l[0] >= 1) {
-            const uint32_t kk = block_select_desc(GlobalSampleKeyGet{sample_out}, m, lad.l[0],
-                                                  hist, wsum, bcast);
-            aR = from_key(kk);
-        }
-        if (lad.h[0] <= m) {
-            const uint32_t kk = block_select_desc(GlobalSampleKeyGet{sample_out}, m, lad.h[0],
-                                                  hist, wsum, bcast);
-            aL = from_key(kk);
-        }
+    {
+        const int64_t ra = lad.l[0] >= 1 ? lad.l[0] : 0;
+        const int64_t rb = lad.h[0] <= m ? lad.h[0] : 0;
+        uint32_t ka = 0u, kb = 0u;
+        select_two_ranks(skeys, m, hist, ra, rb, h2, wsum, bcast, &ka, &kb);
+        if (ra >= 1) aR = from_key(ka);
+        if (rb >= 1) aL = from_key(kb);
     }
     phase_mark(st, 1);
     if (force_miss) {
         uint32_t kmax = 0;
-        for (int s = threadIdx.x; s < m; s += kBlk) kmax = max(kmax, to_key(__ldcg(sample_out + s)));
+        for (int s = threadIdx.x; s < m; s += kBlk) kmax = max(kmax, skeys[s]);
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, d));
         if (threadIdx.x == 0) bcast[3] = 0u;
@@ -962,9 +1025,13 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
 // Returns #{edges 0..nbin with F >= k}; F at edge 0 and edge nbin go to
 // sm->binF.  With want >= 0 the tails of the sub-bracket [e_want, e_want+1)
 // go to sm->sub.  Every thread of the (1024-thread) block must call it.
+// With want == -2 the thread that sees the straddle locally (F >= k at edge j,
+// F < k at edge j + 1) leaves j in sm->bcast[7] and the sub-bracket tails in
+// sm->sub; sm->bcast[6] counts such claims (one when F is monotone).
 __device__ int bin_scan(const BinLayout& BL, const unsigned long long* __restrict__ bins,
                         const Tails& tl, double k, double t, SolveSmemAll* sm, int want) {
     const int b0 = 2 * threadIdx.x, b1 = b0 + 1;
+    if (want == -2 && threadIdx.x == 0) sm->bcast[6] = 0u;  // read after the scans' barriers
     const double e0 = (double)bin_edge(BL, b0), e1 = (double)bin_edge(BL, b1);
     const double e2 = (double)bin_edge(BL, b1 + 1);
     const double g0 = (e1 > e0) ? cold_exp((e0 - e1) / t) : 1.0;
@@ -995,6 +1062,18 @@ __device__ int bin_scan(const BinLayout& BL, const unsigned long long* __restric
     if (b0 == nb) sm->binF[1] = F0;
     if (b1 == nb) sm->binF[1] = F1;
     if (b1 + 1 == nb) sm->binF[1] = F2;
+    if (want == -2) {
+        auto claim = [&](int j, double SL, double SR, double cR) {
+            if (atomicAdd(&sm->bcast[6], 1u) == 0u) {
+                sm->bcast[7] = (uint32_t)j;
+                sm->sub.SL = SL;
+                sm->sub.SR = SR;
+                sm->sub.cntR = cR;
+            }
+        };
+        if (b0 < nb && F0 >= k && F1 < k) claim(b0, P0, Q1, A1);
+        if (b1 < nb && F1 >= k && F2 < k) claim(b1, P1, Q2, A2);
+    }
     if (want >= 0) {
         // lower end e_want: weights below it; upper end e_want+1: weights and count above it
         if (b0 == want) sm->sub.SL = P0;
@@ -1147,7 +1226,7 @@ __device__ int solve_exact(float* cur, float* nxt, long long nb, Tails tl, doubl
 __device__ int plan_with_bins(const unsigned long long* __restrict__ bins, const BinLayout& BL,
                               const Tails& tl, double k, double t, SolveSmemAll* sm,
                               RowState* st) {
-    const int cntF = bin_scan(BL, bins, tl, k, t, sm, -1);
+    const int cntF = bin_scan(BL, bins, tl, k, t, sm, -2);
     const double FL = tl.hasL ? sm->binF[0] : INFINITY;
     const double FR = tl.hasR ? sm->binF[1] : -INFINITY;
     if (!(FL >= k && FR <= k)) {
@@ -1163,7 +1242,19 @@ __device__ int plan_with_bins(const unsigned long long* __restrict__ bins, const
     if (jc < 0) jc = 0;
     if (jc > BL.nbin - 1) jc = BL.nbin - 1;
     __syncthreads();
-    bin_scan(BL, bins, tl, k, t, sm, jc);
+    if (sm->bcast[6] == 1u && (int)sm->bcast[7] == jc) {
+        // the first scan already left this bin's tails
+        if (threadIdx.x == 0) {
+            sm->sub.hasL = true;
+            sm->sub.aL = bin_edge(BL, jc);
+            const float hi = bin_edge(BL, jc + 1);
+            sm->sub.hasR = isfinite(hi);
+            sm->sub.aR = hi;
+        }
+        __syncthreads();
+    } else {
+        bin_scan(BL, bins, tl, k, t, sm, jc);
+    }
     if ((long long)bins[jc] > kBandSortMax) return -1;
     if (threadIdx.x == 0) {
         st->sub_bin = jc;
@@ -1210,14 +1301,16 @@ __device__ void refold_row(const float* __restrict__ r, int64_t n, float aL, flo
     *nb = (long long)sm->cnt;
 }
 
-__global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r, int64_t n,
+// One CTA of 1024 threads; 64 registers each (the whole register file) keeps
+// the fp64 scans' spills down.
+__global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_t n,
                                                      double k, double t, RowState* st,
                                                      float* __restrict__ band0,
                                                      float* __restrict__ band1,
                                                      const unsigned long long* __restrict__ bins,
                                                      const float* __restrict__ sample, int m,
                                                      Ladder lad, double* __restrict__ b_out,
-                                                     WsHeader* hdr) {
+                                                     WsHeader* hdr, int split) {
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
     phase_mark(st, 2);
@@ -1259,10 +1352,22 @@ __global__ void __launch_bounds__(kBlk) solve_kernel(const float* __restrict__ r
         int via_bins = -1;
         if (nb > kBandSortMax && attempt == 1) {
             // the fold built the band histogram for this first bracket; the
-            // chosen bin is extracted and solved by the next two kernels
+            // chosen bin is extracted and solved by the next two kernels when
+            // they were launched (split), else here
             const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
-            via_bins = plan_with_bins(bins, BL, tl, k, t, sm, st);
-            if (via_bins == 1) {
+            if (!split) {
+                via_bins = solve_with_bins(cur, nb, bins, BL, tl, k, t, sm, nullptr);
+                if (via_bins == 1) {
+                    b = sm->res.b;
+                    done = true;
+                    certified = true;
+                } else if (via_bins == 0) {
+                    certified = false;
+                }
+            } else {
+                via_bins = plan_with_bins(bins, BL, tl, k, t, sm, st);
+            }
+            if (split && via_bins == 1) {
                 phase_mark(st, 3);
                 if (threadIdx.x == 0) {
                     st->stage = 1;
@@ -1386,7 +1491,7 @@ __global__ void __launch_bounds__(256) extract_kernel(const float* __restrict__ 
 // Exact solve on the extracted bin with the rest of the row folded into its
 // tails.  If rounding in the fixed-point histogram chose the wrong bin (its own
 // end check fails), the single-CTA histogram solve walks to the right one.
-__global__ void __launch_bounds__(kBlk) solve2_kernel(double k, double t, RowState* st,
+__global__ void __maxnreg__(64) solve2_kernel(double k, double t, RowState* st,
                                                       float* __restrict__ band0,
                                                       float* __restrict__ sub,
                                                       const unsigned long long* __restrict__ bins,
@@ -1406,7 +1511,31 @@ __global__ void __launch_bounds__(kBlk) solve2_kernel(double k, double t, RowSta
     s.cntR = st->sub_cntR;
     double b = nan("");
     bool ok = false;
-    if (ns <= kBandSortMax) {
+    if (ns <= kWarpSortMax) {
+        // a small bin (the usual case): one warp sorts it in registers and
+        // solves it, with no block barrier on the way
+        if (threadIdx.x < 32) {
+            uint32_t key[kWarpSortMax / 32];
+#pragma unroll
+            for (int e = 0; e < kWarpSortMax / 32; ++e) {
+                const long long j = (long long)threadIdx.x * (kWarpSortMax / 32) + e;
+                key[e] = j < ns ? to_key(sub[j]) : 0xffffffffu;
+            }
+            bitonic_sort_row<kWarpSortMax / 32, 32, 32>(key, threadIdx.x, nullptr);
+#pragma unroll
+            for (int e = 0; e < kWarpSortMax / 32; ++e) {
+                const long long j = (long long)threadIdx.x * (kWarpSortMax / 32) + e;
+                if (j < ns) sm->u.sort.sorted[j] = from_key(key[e]);
+            }
+            __syncwarp();
+            phase_mark(st, 13);
+            solve_sorted_block<FloatGet, true>(FloatGet{sm->u.sort.sorted}, ns, s, k, t, &sm->ss,
+                                               &sm->res);
+        }
+        __syncthreads();
+        ok = sm->res.F_aL >= k && sm->res.F_aR <= k;
+        b = sm->res.b;
+    } else if (ns <= kBandSortMax) {
         if (ns <= kBlk) sort_band_into<1>(sub, ns, sm);
         else if (ns <= 2 * kBlk) sort_band_into<2>(sub, ns, sm);
         else sort_band_into<4>(sub, ns, sm);
@@ -1475,7 +1604,7 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     // device's copy of the module)
     static unsigned long long attr_devices = 0ull;
     const size_t solve_smem = sizeof(SolveSmemAll);
-    const size_t sample_smem = (size_t)2 * kBandSortMax * sizeof(uint32_t);
+    const size_t sample_smem = ((size_t)kSampleMax + 2 * 2048) * sizeof(uint32_t);
     int dev = 0;
     cudaGetDevice(&dev);
     const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
@@ -1513,20 +1642,34 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                                                         buf.bins, buf.fold_part, buf.ticket, hdr,
                                                         vec);
     }
+    // The band of the first bracket holds about n (h - l) / m scores.  When it
+    // should fit the on-chip sort with some room to spare, the solve kernel finishes
+    // by itself and the grid-wide extraction and second solve are not launched;
+    // a band that turns out larger is still solved exactly, inside the solve
+    // kernel.
+    const int64_t lo_rank = rank_l[0] > 0 ? rank_l[0] : 0;
+    const int64_t hi_rank = rank_h[0] < m ? rank_h[0] : m;
+    const double expect_band = (double)n * (double)(hi_rank - lo_rank) / (double)m;
+    const int split =
+        ((flags & LAPSUM_FLAG_ONE_CTA_SOLVE) == 0 && (force_miss || expect_band > 0.75 * kBandSortMax))
+            ? 1
+            : 0;
     {
         ProfScope ps_("bracket_solve", st);
         solve_kernel<<<1, kBlk, solve_smem, st>>>(r_row, n, k, t, st_row, buf.band[0], buf.band[1],
-                                              buf.bins, sample, m, lad, b_out, hdr);
+                                              buf.bins, sample, m, lad, b_out, hdr, split);
     }
-    {
-        ProfScope ps_("bracket_extract", st);
-        extract_kernel<<<bracket_fold_grid() / 2 > 0 ? bracket_fold_grid() / 2 : 1, 256, 0, st>>>(
-            buf.band[0], st_row, buf.band[1]);
-    }
-    {
-        ProfScope ps_("bracket_solve2", st);
-        solve2_kernel<<<1, kBlk, solve_smem, st>>>(k, t, st_row, buf.band[0], buf.band[1],
-                                                   buf.bins, b_out, hdr);
+    if (split) {
+        {
+            ProfScope ps_("bracket_extract", st);
+            extract_kernel<<<bracket_fold_grid() / 2 > 0 ? bracket_fold_grid() / 2 : 1, 256, 0,
+                             st>>>(buf.band[0], st_row, buf.band[1]);
+        }
+        {
+            ProfScope ps_("bracket_solve2", st);
+            solve2_kernel<<<1, kBlk, solve_smem, st>>>(k, t, st_row, buf.band[0], buf.band[1],
+                                                       buf.bins, b_out, hdr);
+        }
     }
     return cudaGetLastError();
 }

@@ -263,7 +263,7 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
     if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
     if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
     const int rp = resolve_path(n, path);
-    if (rp < 0 || (path & ~0x3ff) != 0) return LAPSUM_EINVAL;
+    if (rp < 0 || (path & ~0x7ff) != 0) return LAPSUM_EINVAL;
     if (n > INT32_MAX && rp != LAPSUM_PATH_BRACKET) return LAPSUM_EINVAL;
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
     const Layout L = make_layout(B, n, rp);

@@ -246,7 +246,7 @@ __device__ inline long long block_excl_suffix_ll(long long v, long long* wt) {
 // exponential:  Bh = 0: b = sR + t ln(2c/Ah);  Ah = 0: b = sL + t ln(Bh/(-2c)).
 // The result is clamped into [sL, sR].
 // ---------------------------------------------------------------------------
-__device__ inline double segment_root(bool hasL, double sL, double Bh, bool hasR, double sR,
+static __device__ __noinline__ double segment_root(bool hasL, double sL, double Bh, bool hasR, double sR,
                                       double Ah, double c, double t) {
     hasL = hasL && Bh > 0.0;
     hasR = hasR && Ah > 0.0;

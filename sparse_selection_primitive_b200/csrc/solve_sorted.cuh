@@ -120,12 +120,28 @@ __device__ void warp_find_crossing(const GapFn<Get>& gap, long long lo, long lon
     }
 }
 
-// Whole-block solve.  Every thread of the block must call it; the result is
-// valid in `out` for every thread after return.
-template <class Get>
+// Team barrier and count: the whole block, or (WARP) a single warp.
+template <bool WARP>
+__device__ __forceinline__ void team_sync() {
+    if (WARP) __syncwarp();
+    else __syncthreads();
+}
+template <bool WARP>
+__device__ __forceinline__ int team_count(bool pred) {
+    if (WARP) return __popc(__ballot_sync(0xffffffffu, pred));
+    return __syncthreads_count(pred);
+}
+
+// Whole-team solve: every thread of the block (or, with WARP, every lane of
+// the one calling warp) must call it; the result is valid in `out` for every
+// thread of the team after return.  The warp form serves small bands without
+// any block barrier.
+template <class Get, bool WARP = false>
 __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, double k, double t,
                                    SolveScratch* sm, SolveResult* out) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int tid = WARP ? (int)(threadIdx.x & 31) : (int)threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int nthreads = WARP ? 32 : (int)blockDim.x, nwarps = nthreads >> 5;
     GapFn<Get> gap{get, nb, tl, 1.0 / t};
     const double P_start = tl.hasL ? tl.SL : 0.0;
     const double Q_end = tl.hasR ? tl.SR : 0.0;
@@ -138,11 +154,11 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
             out->F_aL = tl.hasL ? tl.cntR - 0.5 * tl.SR * cold_exp(lnw) + 0.5 * tl.SL : INFINITY;
             out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * tl.SL * cold_exp(lnw) : -INFINITY;
         }
-        __syncthreads();
+        team_sync<WARP>();
         return;
     }
 
-    const long long chunk = (nb + blockDim.x - 1) / blockDim.x;
+    const long long chunk = (nb + nthreads - 1) / nthreads;
     const long long lo = min(nb, (long long)tid * chunk), hi = min(nb, lo + chunk);
     const bool valid = lo < hi;
     Aff af = aff_id(), ab = aff_id();
@@ -163,7 +179,7 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
     if (lane == 31) eb = aff_id();
     if (lane == 31) sm->wf[warp] = inc_f;
     if (lane == 0) sm->wb[warp] = inc_b;
-    __syncthreads();
+    team_sync<WARP>();
     {
         Aff pre = aff_id();
         for (int w = 0; w < warp; ++w) pre = aff_then(pre, sm->wf[w]);
@@ -178,7 +194,7 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
     const double Q_lo = fma(ab.a, Q_after, ab.c);
     const double G_lo = tl.cntR + (double)(nb - lo) - 0.5 * Q_lo + 0.5 * (P_lo - 1.0);
     const double P_end = fma(af.a, P_before, af.c);    // P_{hi-1}
-    const int count = __syncthreads_count(valid && G_lo >= k);
+    const int count = team_count<WARP>(valid && G_lo >= k);
     const int T = count - 1;
     if (tid == 0) sm->d[0] = Q_lo;                      // Q_0
     if (valid && hi == nb) sm->d[1] = P_end;            // P_{nb-1}
@@ -188,7 +204,7 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
         sm->d[2] = P_before;
         sm->d[3] = Q_after;
     }
-    __syncthreads();
+    team_sync<WARP>();
 
     if (count > 0 && warp == 0) {
         long long js;
@@ -200,7 +216,7 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
             sm->d[5] = Qr;
         }
     }
-    __syncthreads();
+    team_sync<WARP>();
     if (tid == 0) {
         double b;
         long long js;
@@ -223,7 +239,7 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
                             : INFINITY;
         out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * gap(nb) * Pl : -INFINITY;
     }
-    __syncthreads();
+    team_sync<WARP>();
 }
 
 }  // namespace lapsum

@@ -36,6 +36,26 @@ constexpr size_t kAlignSup = 256;
 
 size_t up256(size_t x) { return (x + kAlignSup - 1) / kAlignSup * kAlignSup; }
 
+// L2 eviction-priority hints: the list (entries and gathered v, a few percent
+// of the row) is read again by pass B, so pass A keeps it with evict_last
+// while the gathers of v stream through.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint2 ld_keep(const uint2* p, uint64_t pol) {
+    uint2 v;
+    asm volatile("ld.global.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ void st_keep(float* p, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol)
+                 : "memory");
+}
+
 __device__ __forceinline__ void sup_add(float ax, float vv, float& mu, double& s, double& sv) {
     if (ax < mu) {
         const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(ax - mu);
@@ -69,6 +89,7 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     int bad = match ? 0 : 1;
     float mu = INFINITY, amin = INFINITY;
     double s = 0.0, sv = 0.0;
+    const uint64_t keep = l2_evict_last_policy();
     // count of share i of group gi: (tile gi * group + i / 8, share i % 8), or 0
     auto share_count = [&](int64_t gi) -> uint32_t {
         const int64_t t0 = gi * group;
@@ -128,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
                         else hi = mid - 1;
                     }
                     slot[u] = lo * kSupCap + (int32_t)(j - pre[lo]);
-                    e[u] = __ldcs(ent + slot[u]);
+                    e[u] = ld_keep(ent + slot[u], keep);
                     gpos[u] = (lo / kShares) * kTile;
                 }
             }
@@ -150,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
                 const float ax = fabsf(__uint_as_float(e[u].y));
                 amin = fminf(amin, ax);
                 sup_add(ax, vv[u], mu, s, sv);
-                val[slot[u]] = vv[u];
+                st_keep(val + slot[u], vv[u], keep);
             }
         }
     }

@@ -116,6 +116,21 @@ def test_large_band_through_histogram(cuda_device):
     check_row(r[0], v[0], k, t, b, p, label="large band", sum_ref="fp32")
 
 
+def test_large_band_solved_in_one_cta(cuda_device):
+    # The same large first band solved without the grid-wide extraction: the
+    # single solve CTA walks the histogram and extracts the bin itself (the
+    # path a band takes when it turns out far larger than the ranks predict).
+    n = 1 << 20
+    r, v = random_rows(8, 1, n, "normal_q64")
+    k, t = n / 2.0, 0.05
+    ws, p, b = _forward(r[0], k, t, flags=L.FLAG_ONE_CTA_SOLVE)
+    info = L.row_info(ws, 0)
+    assert info["n_band"] > 4096 and info["attempts"] == 1
+    check_row(r[0], v[0], k, t, b, p, label="large band, one CTA", sum_ref="fp32")
+    _, _, b2 = _forward(r[0], k, t)
+    assert abs(b2 - b) <= 1e-12 * max(1.0, abs(b))
+
+
 def test_large_band_exact_narrowing_after_a_miss(cuda_device):
     # After a failed first bracket the widened band is re-folded by one CTA
     # without a histogram, so it is narrowed by exact histogram levels.
