@@ -542,6 +542,7 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     __syncthreads();
     FoldAcc acc{0u, 0.0, 0.0, false};
     uint32_t far_right = 0u;
+    float far_right_f = 0.f;  // full trips' count (exact: at most 2^24 per thread)
     float xsum = 0.f;
     bool bad = false;
     unsigned long long* counter = &st->n_band;
@@ -623,14 +624,23 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
 #pragma unroll
                 for (int qq = 0; qq < U; ++qq) nv[qq] = __ldcs(p + step + (int64_t)qq * nthreads);
             }
-            uint32_t m = 0u;
+            // full trips: the compares give 1.0 / 0.0, the near mask is built
+            // exactly in fp32 (16 bits) and the far-right count in a float
+            // (exact to 2^24 per thread), all on the floating-point pipes
+            float mf = 0.f;
 #pragma unroll
             for (int qq = 0; qq < U; ++qq) {
-                classify(cur[qq].x, true, m, 4 * qq);
-                classify(cur[qq].y, true, m, 4 * qq + 1);
-                classify(cur[qq].z, true, m, 4 * qq + 2);
-                classify(cur[qq].w, true, m, 4 * qq + 3);
+                const float xv[4] = {cur[qq].x, cur[qq].y, cur[qq].z, cur[qq].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float gl = xv[c] >= aLf ? 1.f : 0.f;
+                    const float gr = xv[c] >= aRf ? 1.f : 0.f;
+                    mf = fmaf(gl - gr, (float)(1u << (4 * qq + c)), mf);
+                    far_right_f += gr;
+                    xsum += xv[c];
+                }
             }
+            const uint32_t m = (uint32_t)mf;
             if (__any_sync(0xffffffffu, m != 0u)) {
 #pragma unroll
                 for (int qq = 0; qq < U; ++qq)
@@ -685,7 +695,7 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
         }
     }
     while (tail != head) drain((int)min(32u, tail - head));
-    acc.cntR += far_right;
+    acc.cntR += far_right + (uint32_t)far_right_f;
     acc.bad |= bad;
     __syncthreads();
     band_flush(sband, scount, band, counter, cap, BL, inv_t, bins, &gbase);
