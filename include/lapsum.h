@@ -57,10 +57,13 @@ enum lapsum_status {
 
 /* Solver selection (low byte of `path`). */
 enum lapsum_path {
-    LAPSUM_PATH_AUTO = 0,     /* n <= 4096: bitonic; n <= 2^20: radix full sort; else bracketing */
+    LAPSUM_PATH_AUTO = 0,     /* n <= 4096: bitonic; n <= 2^18: bracketing, one CTA per row;
+                                 else bracketing over the whole GPU */
     LAPSUM_PATH_FULLSORT = 1, /* full sort: bitonic for n <= 4096, radix above */
     LAPSUM_PATH_BRACKET = 2,  /* probabilistic bracketing (any n >= 2) */
-    LAPSUM_PATH_RADIX = 3     /* full sort with the radix sorter at any n */
+    LAPSUM_PATH_RADIX = 3,    /* full sort with the radix sorter at any n */
+    LAPSUM_PATH_ROWBRACKET = 4 /* probabilistic bracketing with one CTA per row: sample, order
+                                  statistics, fold and band solve in one kernel (n <= 2^20) */
 };
 
 /* Test and diagnostic flags, OR-ed into `path`. */

@@ -30,7 +30,7 @@ __all__ = [
     "support_bytes",
 ]
 
-PATHS = {"auto": 0, "fullsort": 1, "bracket": 2, "radix": 3}
+PATHS = {"auto": 0, "fullsort": 1, "bracket": 2, "radix": 3, "rowbracket": 4}
 FLAG_FORCE_MISS = 0x100
 FLAG_NO_RETRY = 0x200
 FLAG_ONE_CTA_SOLVE = 0x400

@@ -262,6 +262,20 @@ __device__ void select_two_ranks(const uint32_t* keys, int m, const uint32_t* hi
 // ----------------------------------------------------------------------------
 // 1. Localization sample.
 // ----------------------------------------------------------------------------
+// Sample s of a row: a uniform index I (high half of z1 * n) and Laplace(0, t)
+// noise by the inverse CDF, u = 24 bits of z2 centred in (-1/2, 1/2); z1, z2
+// are SplitMix64 outputs 2s and 2s + 1 of the stream (seed, counters from c0).
+__device__ __forceinline__ float draw_sample(const float* __restrict__ r, int64_t n, double t,
+                                             uint64_t seed, uint64_t c0, int s) {
+    const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
+    const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
+    const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
+    const float rv = __ldg(r + I);
+    const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
+    const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
+    const float eps = (u < 0.0 ? 1.f : -1.f) * (float)t * logf(a);
+    return rv + eps;
+}
 // Grid of m / 1024 CTAs: every thread draws one sample and every CTA adds its
 // samples to a global histogram of the keys' top 11 bits; the last CTA to
 // finish (atomic ticket) selects the two order statistics from it and clears
@@ -295,14 +309,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
         const int s = blockIdx.x * kBlk + threadIdx.x;
         uint32_t bn = 0xffffffffu;
         if (s < m) {
-            const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
-            const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
-            const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
-            const float rv = __ldg(r + I);
-            const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
-            const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
-            const float eps = (u < 0.0 ? 1.f : -1.f) * (float)t * logf(a);
-            const float y = rv + eps;
+            const float y = draw_sample(r, n, t, seed, c0, s);
             sample_out[s] = y;
             bn = to_key(y) >> 21;
         }
@@ -1279,72 +1286,101 @@ __device__ int plan_with_bins(const unsigned long long* __restrict__ bins, const
     return 1;
 }
 
-// Single-CTA fold of the whole row (used only after a failed bracket).
-__device__ void refold_row(const float* __restrict__ r, int64_t n, float aL, float aR, double t,
-                           float* band, SolveSmemAll* sm, Tails& tl, long long* nb) {
-    const float inv_t = (float)(1.0 / t);
+// Single-CTA fold of one row: the tail sums and right count of [aL, aR), the
+// band scores appended to `band` (capacity n; order depends on timing, the
+// solve sorts it).  Four 16-byte loads per thread in flight per trip; every
+// score takes one exponential (masked inside the band).  Sets *bad when a
+// score is NaN or infinite.
+__device__ void refold_row(const float* __restrict__ r, int64_t n, int vec, float aL, float aR,
+                           double t, float* band, SolveSmemAll* sm, Tails& tl, long long* nb,
+                           bool* bad) {
+    const float k2 = (float)(kLog2e / t);
     if (threadIdx.x == 0) sm->cnt = 0ull;
     __syncthreads();
-    FoldAcc acc{0u, 0.0, 0.0, false};
-    const int64_t iters = (n + blockDim.x - 1) / blockDim.x;
-    for (int64_t it = 0; it < iters; ++it) {
-        const int64_t i = it * blockDim.x + threadIdx.x;
-        bool bb = false;
-        float x = 0.f;
-        if (i < n) {
-            x = r[i];
-            fold_one(x, aL, aR, inv_t, acc, bb);
+    double SL = 0.0, SR = 0.0;
+    uint32_t cR = 0u;
+    float probe = 0.f;  // NaN once a score is NaN or infinite
+    auto one = [&](float x, float& sl, float& sr) {
+        const bool right = x >= aR, left = x < aL;
+        const bool inb = x >= aL && x < aR;
+        const float e = ex2_ftz((right ? aR - x : (left ? x - aL : 0.f)) * k2);
+        sr += right ? e : 0.f;
+        sl += left ? e : 0.f;
+        cR += right ? 1u : 0u;
+        probe = fmaf(x, 0.f, probe);
+        if (inb) {  // rare
+            const unsigned long long pos = atomicAdd(&sm->cnt, 1ull);
+            if (pos < (unsigned long long)n) band[pos] = x;
         }
-        band_append(bb, x, band, &sm->cnt, (unsigned long long)n);
+    };
+    if (vec) {
+        const int64_t n4 = n >> 2;
+        const float4* r4 = reinterpret_cast<const float4*>(r);
+        constexpr int U = 4;
+        const int64_t per_trip = (int64_t)U * blockDim.x;
+        for (int64_t i0 = 0; i0 < n4; i0 += per_trip) {
+            float4 v[U];
+#pragma unroll
+            for (int q = 0; q < U; ++q) {
+                const int64_t i = i0 + (int64_t)q * blockDim.x + threadIdx.x;
+                v[q] = i < n4 ? __ldcg(r4 + i) : make_float4(NAN, NAN, NAN, NAN);
+            }
+            float sl = 0.f, sr = 0.f;
+#pragma unroll
+            for (int q = 0; q < U; ++q) {
+                if (i0 + (int64_t)q * blockDim.x + threadIdx.x >= n4) continue;
+                one(v[q].x, sl, sr);
+                one(v[q].y, sl, sr);
+                one(v[q].z, sl, sr);
+                one(v[q].w, sl, sr);
+            }
+            SL += (double)sl;
+            SR += (double)sr;
+        }
+        for (int64_t i = (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) {
+            float sl = 0.f, sr = 0.f;
+            one(r[i], sl, sr);
+            SL += (double)sl;
+            SR += (double)sr;
+        }
+    } else {
+        for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+            float sl = 0.f, sr = 0.f;
+            one(r[i], sl, sr);
+            SL += (double)sl;
+            SR += (double)sr;
+        }
     }
-    const double sL = block_sum_d(acc.SL, sm->red);
-    const double sR = block_sum_d(acc.SR, sm->red);
-    const long long cR = block_sum_ll((long long)acc.cntR, sm->lred);
-    __syncthreads();
+    const double sL = block_sum_d(SL, sm->red);
+    const double sR = block_sum_d(SR, sm->red);
+    const long long cnt = block_sum_ll((long long)cR, sm->lred);
+    const int any_bad = __syncthreads_or(!(probe == 0.f));
     tl.hasL = isfinite(aL);
     tl.aL = aL;
     tl.SL = sL;
     tl.hasR = isfinite(aR);
     tl.aR = aR;
     tl.SR = sR;
-    tl.cntR = (double)cR;
+    tl.cntR = (double)cnt;
     *nb = (long long)sm->cnt;
+    if (bad) *bad = any_bad != 0;
 }
 
-// One CTA of 1024 threads; 64 registers each (the whole register file) keeps
-// the fp64 scans' spills down.
-__global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_t n,
-                                                     double k, double t, RowState* st,
-                                                     float* __restrict__ band0,
-                                                     float* __restrict__ band1,
-                                                     const unsigned long long* __restrict__ bins,
-                                                     const float* __restrict__ sample, int m,
-                                                     Ladder lad, double* __restrict__ b_out,
-                                                     WsHeader* hdr, int split) {
-    extern __shared__ __align__(16) unsigned char dsm[];
-    SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
-    phase_mark(st, 2);
-    if (threadIdx.x == 0) {
-        sm->bcast[2] = 0xffffffffu;
-        sm->bcast[3] = 0u;
-    }
-    __syncthreads();
-    if (st->status & kDevNonFinite) {
-        if (threadIdx.x == 0) {
-            st->b = nan("");
-            *b_out = nan("");
-        }
-        return;
-    }
-    Tails tl;
-    tl.hasL = isfinite(st->a_L);
-    tl.aL = st->a_L;
-    tl.SL = st->S_L;
-    tl.hasR = isfinite(st->a_R);
-    tl.aR = st->a_R;
-    tl.SR = st->S_R;
-    tl.cntR = (double)st->cnt_R;
-    long long nb = (long long)st->n_band;
+// The attempt loop of the band solve, shared by the grid pipeline's solve
+// kernel and the one-CTA-per-row kernel.  Solves the current band exactly
+// once its bracket certifies; otherwise widens the failing end by one rung of
+// the ladder (select_key(rank) gives the key of that sample order statistic)
+// and folds the row again.  On the first attempt a band too large for the
+// on-chip sort goes through the fold's histogram (`bins`, when given; with
+// `split` the chosen bin is left for the extract and second solve kernels and
+// the function returns true at once).  Otherwise writes b, the record and the
+// status, and returns false.
+template <class SelectKey>
+__device__ bool bracket_attempts(const float* __restrict__ r, int64_t n, int vec, double k,
+                                 double t, RowState* st, float* band0, float* band1,
+                                 const unsigned long long* __restrict__ bins, int split, int m,
+                                 const Ladder& lad, SelectKey select_key, Tails tl, long long nb,
+                                 SolveSmemAll* sm, double* b_out, WsHeader* hdr) {
     int rungL = st->rung_L, rungR = st->rung_R;
     const int max_attempts = st->max_attempts;
     int attempt = 1;
@@ -1360,7 +1396,7 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
         cert = tl;
         nb_cert = nb;
         int via_bins = -1;
-        if (nb > kBandSortMax && attempt == 1) {
+        if (bins != nullptr && nb > kBandSortMax && attempt == 1) {
             // the fold built the band histogram for this first bracket; the
             // chosen bin is extracted and solved by the next two kernels when
             // they were launched (split), else here
@@ -1385,7 +1421,7 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
                     st->refine_levels = 0;
                     st->certified = 1;
                 }
-                return;
+                return true;
             } else if (via_bins == 0) {
                 certified = false;
             }
@@ -1416,23 +1452,15 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
         if (!tl.hasR) aR = INFINITY;
         if (fail_left) {
             ++rungL;
-            if (rungL >= kLadder - 1 || lad.h[rungL] > m) {
-                aL = -INFINITY;
-            } else {
-                aL = from_key(block_select_desc(GlobalSampleKeyGet{sample}, m, lad.h[rungL],
-                                                sm->u.sel_hist, sm->wsum, sm->bcast + 4));
-            }
+            if (rungL >= kLadder - 1 || lad.h[rungL] > m) aL = -INFINITY;
+            else aL = from_key(select_key(lad.h[rungL]));
         } else {
             ++rungR;
-            if (rungR >= kLadder - 1 || lad.l[rungR] < 1) {
-                aR = INFINITY;
-            } else {
-                aR = from_key(block_select_desc(GlobalSampleKeyGet{sample}, m, lad.l[rungR],
-                                                sm->u.sel_hist, sm->wsum, sm->bcast + 4));
-            }
+            if (rungR >= kLadder - 1 || lad.l[rungR] < 1) aR = INFINITY;
+            else aR = from_key(select_key(lad.l[rungR]));
         }
         ++attempt;
-        refold_row(r, n, aL, aR, t, band0, sm, tl, &nb);
+        refold_row(r, n, vec, aL, aR, t, band0, sm, tl, &nb, nullptr);
     }
     phase_mark(st, 12);
     if (threadIdx.x == 0) {
@@ -1455,6 +1483,162 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
         st->b = b;
         *b_out = b;
     }
+    __syncthreads();
+    return false;
+}
+
+// One CTA of 1024 threads; 64 registers each (the whole register file) keeps
+// the fp64 scans' spills down.
+__global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_t n, int vec,
+                                             double k, double t, RowState* st,
+                                             float* __restrict__ band0,
+                                             float* __restrict__ band1,
+                                             const unsigned long long* __restrict__ bins,
+                                             const float* __restrict__ sample, int m,
+                                             Ladder lad, double* __restrict__ b_out,
+                                             WsHeader* hdr, int split) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    phase_mark(st, 2);
+    if (threadIdx.x == 0) {
+        sm->bcast[2] = 0xffffffffu;
+        sm->bcast[3] = 0u;
+    }
+    __syncthreads();
+    if (st->status & kDevNonFinite) {
+        if (threadIdx.x == 0) {
+            st->b = nan("");
+            *b_out = nan("");
+        }
+        return;
+    }
+    Tails tl;
+    tl.hasL = isfinite(st->a_L);
+    tl.aL = st->a_L;
+    tl.SL = st->S_L;
+    tl.hasR = isfinite(st->a_R);
+    tl.aR = st->a_R;
+    tl.SR = st->S_R;
+    tl.cntR = (double)st->cnt_R;
+    const long long nb = (long long)st->n_band;
+    auto select_key = [&](int64_t rank) {
+        return block_select_desc(GlobalSampleKeyGet{sample}, m, rank, sm->u.sel_hist, sm->wsum,
+                                 sm->bcast + 4);
+    };
+    bracket_attempts(r, n, vec, k, t, st, band0, band1, bins, split, m, lad, select_key, tl, nb,
+                     sm, b_out, hdr);
+}
+
+// ----------------------------------------------------------------------------
+// The whole bracketing pipeline for one row in one CTA (rows of moderate
+// length, many rows per call): the sample is drawn straight into shared
+// memory, its two order statistics are selected there, the CTA folds the row
+// (four 16-byte loads per thread in flight), and the attempt loop solves the
+// band with the same widening ladder as the grid pipeline.  Rows run in
+// parallel, one CTA each; no kernel boundary separates the steps.
+// ----------------------------------------------------------------------------
+struct RowBracketSmem {
+    uint32_t hist1[2048];  // sample keys by their top 11 bits
+    uint32_t h2[2 * 2048];
+    uint32_t wsum[64];
+    uint32_t bcast[4];
+};
+constexpr size_t kRowBracketFixedSmem = sizeof(SolveSmemAll) + sizeof(RowBracketSmem);
+
+__global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, int64_t ld,
+                                                  int64_t n, double k, double t, uint64_t seed,
+                                                  int m, Ladder lad, int force_miss,
+                                                  int max_attempts, int vec, RowState* rows,
+                                                  float* __restrict__ band0_all,
+                                                  float* __restrict__ band1_all,
+                                                  double* __restrict__ b_all, WsHeader* hdr) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    RowBracketSmem* rb = reinterpret_cast<RowBracketSmem*>(dsm + sizeof(SolveSmemAll));
+    uint32_t* keys = reinterpret_cast<uint32_t*>(dsm + kRowBracketFixedSmem);  // m words
+    const int64_t row = blockIdx.x;
+    const float* rr = r + row * ld;
+    RowState* st = rows + row;
+    float* band0 = band0_all + row * n;
+    float* band1 = band1_all + row * n;
+    double* b_out = b_all + row;
+    for (int i = threadIdx.x; i < (int)(sizeof(RowState) / 4); i += blockDim.x)
+        reinterpret_cast<uint32_t*>(st)[i] = 0u;
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) rb->hist1[i] = 0u;
+    __syncthreads();
+    // 1. the sample, as keys, with its level-1 histogram
+    const uint64_t c0 = (uint64_t)row << 32;
+    for (int s0 = 0; s0 < m; s0 += blockDim.x) {  // same trip count in every lane
+        const int s = s0 + threadIdx.x;
+        uint32_t bn = 0xffffffffu;
+        if (s < m) {
+            const uint32_t key = to_key(draw_sample(rr, n, t, seed, c0, s));
+            keys[s] = key;
+            bn = key >> 21;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bn);
+        if (bn != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
+            atomicAdd(&rb->hist1[bn], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    // 2. the bracket's order statistics
+    float aR = INFINITY, aL = -INFINITY;
+    {
+        const int64_t ra = lad.l[0] >= 1 ? lad.l[0] : 0;
+        const int64_t rbk = lad.h[0] <= m ? lad.h[0] : 0;
+        uint32_t ka = 0u, kb = 0u;
+        select_two_ranks(keys, m, rb->hist1, ra, rbk, rb->h2, rb->wsum, rb->bcast, &ka, &kb);
+        if (ra >= 1) aR = from_key(ka);
+        if (rbk >= 1) aL = from_key(kb);
+    }
+    if (force_miss) {
+        // a bracket above every sample value: F(a_L) < k, so it must fail
+        uint32_t kmax = 0u;
+        for (int s = threadIdx.x; s < m; s += blockDim.x) kmax = max(kmax, keys[s]);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, d));
+        if (threadIdx.x == 0) rb->bcast[3] = 0u;
+        __syncthreads();
+        if ((threadIdx.x & 31) == 0) atomicMax(&rb->bcast[3], kmax);
+        __syncthreads();
+        const float top = from_key(rb->bcast[3]);
+        aL = top + fabsf(top) + 1.f;
+        aR = INFINITY;
+    }
+    if (threadIdx.x == 0) {
+        st->ladder_R[0] = aR;
+        st->ladder_L[0] = aL;
+        st->rung_L = force_miss ? -1 : 0;
+        st->rung_R = 0;
+        st->sample_m = m;
+        st->rank_l = (int32_t)lad.l[0];
+        st->rank_h = (int32_t)lad.h[0];
+        st->max_attempts = max_attempts;
+        st->force_miss = force_miss;
+        st->path = LAPSUM_PATH_ROWBRACKET;
+    }
+    // 3. the fold
+    Tails tl;
+    long long nb = 0;
+    bool bad = false;
+    refold_row(rr, n, vec, aL, aR, t, band0, sm, tl, &nb, &bad);
+    if (bad) {
+        if (threadIdx.x == 0) {
+            st->status |= kDevNonFinite;
+            set_status(hdr, kDevNonFinite);
+            st->b = nan("");
+            *b_out = nan("");
+        }
+        return;
+    }
+    // 4. certification, exact solve and widening
+    auto select_key = [&](int64_t rank) {
+        uint32_t ka = 0u, kb = 0u;
+        select_two_ranks(keys, m, rb->hist1, rank, 0, rb->h2, rb->wsum, rb->bcast, &ka, &kb);
+        return ka;
+    };
+    bracket_attempts(rr, n, vec, k, t, st, band0, band1, nullptr, 0, m, lad, select_key, tl, nb,
+                     sm, b_out, hdr);
 }
 
 // Scores of the chosen histogram bin, gathered from the band by the whole
@@ -1591,6 +1775,34 @@ __global__ void __maxnreg__(64) solve2_kernel(double k, double t, RowState* st,
 
 }  // namespace
 
+size_t rowbracket_smem(int m) { return kRowBracketFixedSmem + (size_t)m * sizeof(uint32_t); }
+
+cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, double k, double t,
+                              uint64_t seed, int m, int64_t rank_l[kLadder],
+                              int64_t rank_h[kLadder], int flags, RowState* rows, float* band0,
+                              float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st) {
+    static unsigned long long attr_devices = 0ull;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if ((attr_devices & bit) == 0ull || bit == 0ull) {
+        cudaFuncSetAttribute(rowbracket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)rowbracket_smem(kSampleMax));
+        attr_devices |= bit;
+    }
+    Ladder lad;
+    for (int i = 0; i < kLadder; ++i) {
+        lad.l[i] = rank_l[i];
+        lad.h[i] = rank_h[i];
+    }
+    const int force_miss = (flags & LAPSUM_FLAG_FORCE_MISS) ? 1 : 0;
+    const int max_attempts = (flags & LAPSUM_FLAG_NO_RETRY) ? 1 : kMaxAttempts;
+    ProfScope ps_("rowbracket", st);
+    rowbracket_kernel<<<(unsigned)B, kBlk, rowbracket_smem(m), st>>>(
+        r, ld, n, k, t, seed, m, lad, force_miss, max_attempts, vec, rows, band0, band1, b, hdr);
+    return cudaGetLastError();
+}
+
 int bracket_fold_grid() {
     static int grid = 0;
     if (grid == 0) {
@@ -1666,8 +1878,9 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
             : 0;
     {
         ProfScope ps_("bracket_solve", st);
-        solve_kernel<<<1, kBlk, solve_smem, st>>>(r_row, n, k, t, st_row, buf.band[0], buf.band[1],
-                                              buf.bins, sample, m, lad, b_out, hdr, split);
+        solve_kernel<<<1, kBlk, solve_smem, st>>>(r_row, n, vec, k, t, st_row, buf.band[0],
+                                              buf.band[1], buf.bins, sample, m, lad, b_out, hdr,
+                                              split);
     }
     if (split) {
         {

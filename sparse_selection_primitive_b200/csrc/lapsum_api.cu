@@ -20,6 +20,8 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr int64_t kOnchipMax = 4096;
 constexpr int64_t kRadixMax = int64_t(1) << 20;
+constexpr int64_t kRowBracketAuto = int64_t(1) << 18;  // AUTO: one CTA per row up to here
+constexpr int64_t kRowBracketMax = int64_t(1) << 20;
 constexpr int kFoldGridMax = 4096;
 constexpr int64_t kGridYMax = 65535;
 constexpr double kBracketAlpha = 1e-6;  // miss probability allowed per bracket end
@@ -30,7 +32,9 @@ int resolve_path(int64_t n, int path) {
     switch (path & 0xff) {
         case LAPSUM_PATH_AUTO:
             return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT
-                                   : (n <= kRadixMax ? LAPSUM_PATH_RADIX : LAPSUM_PATH_BRACKET);
+                   : n <= kRowBracketAuto ? LAPSUM_PATH_ROWBRACKET
+                                          : LAPSUM_PATH_BRACKET;
+        case LAPSUM_PATH_ROWBRACKET: return n <= kRowBracketMax ? LAPSUM_PATH_ROWBRACKET : -1;
         case LAPSUM_PATH_FULLSORT:
             return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT : LAPSUM_PATH_RADIX;
         case LAPSUM_PATH_BRACKET: return LAPSUM_PATH_BRACKET;
@@ -60,7 +64,7 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
     // sample kernel's 2048-bin key histogram (all self-clearing)
     L.tickets = take((size_t)B * 2 * sizeof(uint32_t) + (2 + 2048) * sizeof(uint32_t));
     L.fold_ticket = L.tickets + (size_t)B * 2 * sizeof(uint32_t);
-    L.rows = take((size_t)B * 512);
+    L.rows = take((size_t)B * sizeof(RowState));
     L.partials = take((size_t)B * (size_t)tiles * 4 * sizeof(double));
     L.row_R = take((size_t)B * sizeof(double));
     if (n > kOnchipMax) {  // windowed backward of long rows
@@ -76,6 +80,10 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
         L.seg_hist = take((size_t)B * 1024 * sizeof(uint32_t));
         L.tile_hist = take((size_t)B * 256 * (size_t)rt * sizeof(uint32_t));
         L.plan = take((size_t)B * 8 * sizeof(int32_t));
+    }
+    if (rpath == LAPSUM_PATH_ROWBRACKET) {
+        L.band0 = take((size_t)B * (size_t)n * sizeof(float));
+        L.band1 = take((size_t)B * (size_t)n * sizeof(float));
     }
     if (rpath == LAPSUM_PATH_BRACKET) {
         L.sample = take((size_t)B * kSampleMax * sizeof(float));
@@ -139,6 +147,20 @@ void binomial_ranks(int64_t m, double q, double alpha, int64_t* l, int64_t* h) {
     *h = hi;
     std::lock_guard<std::mutex> g(mu);
     if (cache.size() < 64) cache.push_back(Entry{m, q, alpha, lo, hi});
+}
+
+// Ranks of the bracket ladder: the binomial ranks, then each end moved out by
+// a factor of 4 per rung, the last rung open.
+void bracket_ladder(int m, double q, int64_t rl[kLadder], int64_t rh[kLadder]) {
+    int64_t l0, h0;
+    binomial_ranks(m, q, kBracketAlpha, &l0, &h0);
+    for (int i = 0; i < kLadder - 1; ++i) {
+        rl[i] = l0 >> (2 * i);
+        rh[i] = h0 << (2 * i);
+        if (rh[i] > m) rh[i] = m + 1;
+    }
+    rl[kLadder - 1] = 0;
+    rh[kLadder - 1] = m + 1;
 }
 
 int sample_size(int64_t n, double k) {
@@ -286,7 +308,7 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
         return cuda_status(e);
     }
     if (rp == LAPSUM_PATH_RADIX) {
-        e = cudaMemsetAsync(rows, 0, (size_t)B * 512, st);
+        e = cudaMemsetAsync(rows, 0, (size_t)B * sizeof(RowState), st);
         if (e != cudaSuccess) return LAPSUM_ECUDA;
         RadixBuffers rb;
         rb.keys[0] = reinterpret_cast<uint32_t*>(w + L.keys0);
@@ -306,6 +328,14 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
             if (e == cudaSuccess)
                 e = launch_rowsolve_sorted_keys(sub, nb, n, k, t, b + r0, rows + r0, hdr, st);
         }
+    } else if (rp == LAPSUM_PATH_ROWBRACKET) {
+        const int m = sample_size(n, k);
+        int64_t rl[kLadder], rh[kLadder];
+        bracket_ladder(m, k / (double)n, rl, rh);
+        e = launch_rowbracket(r, ld, B, n, k, t, seed, m, rl, rh, path, rows,
+                              reinterpret_cast<float*>(w + L.band0),
+                              reinterpret_cast<float*>(w + L.band1), b, hdr,
+                              (aligned16(r) && (ld % 4) == 0) ? 1 : 0, st);
     } else {
         BracketBuffers bb;
         bb.sample = reinterpret_cast<float*>(w + L.sample);
@@ -317,16 +347,8 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
         bb.fold_grid = bracket_fold_grid();
         if (bb.fold_grid > kFoldGridMax) bb.fold_grid = kFoldGridMax;
         const int m = sample_size(n, k);
-        int64_t l0, h0;
-        binomial_ranks(m, k / (double)n, kBracketAlpha, &l0, &h0);
         int64_t rl[kLadder], rh[kLadder];
-        for (int i = 0; i < kLadder - 1; ++i) {
-            rl[i] = l0 >> (2 * i);
-            rh[i] = h0 << (2 * i);
-            if (rh[i] > m) rh[i] = m + 1;
-        }
-        rl[kLadder - 1] = 0;
-        rh[kLadder - 1] = m + 1;
+        bracket_ladder(m, k / (double)n, rl, rh);
         for (int64_t row = 0; row < B && e == cudaSuccess; ++row) {
             e = launch_bracket_row(r + row * ld, n, k, t, seed, row, m, rl, rh, path, bb,
                                    rows + row, b + row, hdr, st);
@@ -464,7 +486,7 @@ int lapsum_row_info_get(void* ws, int64_t row, lapsum_row_info* out, void* strea
     if (h.last_B <= 0 || row >= h.last_B || h.last_path == LAPSUM_PATH_FULLSORT)
         return LAPSUM_EINVAL;
     const Layout L = make_layout(h.last_B, h.last_n, (int)h.last_path);
-    const char* base = static_cast<const char*>(ws) + L.rows + (size_t)row * 512;
+    const char* base = static_cast<const char*>(ws) + L.rows + (size_t)row * sizeof(RowState);
     e = cudaMemcpyAsync(&rs, base, sizeof(rs), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return LAPSUM_ECUDA;

@@ -69,8 +69,9 @@ struct RowState {
     float sub_aL, sub_aR;      // sub-bracket [sub_aL, sub_aR) = that bin's edges
     int32_t sub_hasR, pad1;
     double sub_SL, sub_SR, sub_cntR;  // tails of the sub-bracket
-    double scratch[32];       // kernel-to-kernel scalars (phase timestamps)
+    double scratch[37];       // kernel-to-kernel scalars (phase timestamps)
 };
+static_assert(sizeof(RowState) == 512, "row records are 512-byte slots of the workspace");
 static_assert(sizeof(RowState) <= 512, "row record fits its slot");
 
 // ---------------------------------------------------------------------------

@@ -119,6 +119,12 @@ struct BracketBuffers {
     int fold_grid;
 };
 int bracket_fold_grid();
+// The whole bracketing pipeline with one CTA per row (rows up to 2^20 scores):
+// b[row] and rows[row] for every row; band0/band1: B * n floats each.
+cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, double k, double t,
+                              uint64_t seed, int m, int64_t rank_l[kLadder],
+                              int64_t rank_h[kLadder], int flags, RowState* rows, float* band0,
+                              float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st);
 cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t, uint64_t seed,
                                int64_t row, int m, int64_t rank_l[kLadder],
                                int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,

@@ -54,6 +54,17 @@ def test_radix_sizes(cuda_device, n):
                       label=f"radix n={n} k={k} row={i}")
 
 
+@pytest.mark.parametrize("n", [2, 100, 4097, 8191, 65536, 70001, 300000])
+def test_rowbracket_sizes(cuda_device, n):
+    B = 3
+    r, v = random_rows(40 + n, B, n)
+    for k in k_values(n):
+        out = run_gpu(r, k, 0.02, path="rowbracket", v=v)
+        for i in range(B):
+            check_row(r[i], v[i], k, 0.02, out["b"][i], out["p"][i], out["g"][i],
+                      label=f"rowbracket n={n} k={k} row={i}")
+
+
 @pytest.mark.parametrize("n", [64, 5000, 65536, 300000])
 def test_bracket_sizes(cuda_device, n):
     r, v = random_rows(30 + n, 1, n)
@@ -64,7 +75,7 @@ def test_bracket_sizes(cuda_device, n):
 
 
 @pytest.mark.parametrize("dist", ["normal", "normal_q64", "abs_t3", "mix_nu"])
-@pytest.mark.parametrize("path", ["fullsort", "radix", "bracket"])
+@pytest.mark.parametrize("path", ["fullsort", "radix", "bracket", "rowbracket"])
 def test_distributions_and_ties(cuda_device, dist, path):
     n = 3000 if path == "fullsort" else 20000
     r, v = random_rows(7, 2, n, dist)
@@ -75,7 +86,7 @@ def test_distributions_and_ties(cuda_device, dist, path):
                       label=f"{path} {dist} k={k} t={t}")
 
 
-@pytest.mark.parametrize("path", ["fullsort", "radix", "bracket"])
+@pytest.mark.parametrize("path", ["fullsort", "radix", "bracket", "rowbracket"])
 def test_degenerate_rows(cuda_device, path):
     n = 1000 if path == "fullsort" else 9000
     # all equal: p = k/n everywhere
@@ -104,7 +115,7 @@ def test_k_extremes(cuda_device):
     n = 777
     r, v = random_rows(9, 1, n)
     for k in (1e-6, 1e-3, n - 1e-3, n - 1e-6):
-        for path in ("fullsort", "radix", "bracket"):
+        for path in ("fullsort", "radix", "bracket", "rowbracket"):
             out = run_gpu(r, k, 0.2, path=path, v=v)
             check_row(r[0], v[0], k, 0.2, out["b"][0], out["p"][0], out["g"][0],
                       label=f"{path} k={k}")
@@ -116,7 +127,7 @@ def test_strided_rows_and_unaligned(cuda_device):
     r, v = random_rows(11, B, ld)
     full = torch.from_numpy(r).cuda()
     vv = torch.from_numpy(v).cuda()
-    for path in ("fullsort", "radix"):
+    for path in ("fullsort", "radix", "rowbracket"):
         sub = full[:, 1:1 + n]
         p, b = L.forward(sub, 12.0, 0.1, path=path)
         g = L.backward(sub, b, vv[:, 1:1 + n], 0.1)
@@ -127,7 +138,7 @@ def test_strided_rows_and_unaligned(cuda_device):
 
 
 def test_nonfinite_scores_reported(cuda_device):
-    for path, n in (("fullsort", 100), ("radix", 5000), ("bracket", 5000)):
+    for path, n in (("fullsort", 100), ("radix", 5000), ("bracket", 5000), ("rowbracket", 5000)):
         r, _ = random_rows(1, 2, n)
         r[1, n // 2] = np.nan
         ws = L.Workspace(2, n, 3.0, path)
@@ -135,13 +146,13 @@ def test_nonfinite_scores_reported(cuda_device):
         assert L.read_status(ws) == 3, path
         bb = b.cpu().numpy()
         assert math.isnan(bb[1]), path
-        if path != "bracket":
+        if path != "bracket":  # the grid pipeline solves one row at a time
             assert not math.isnan(bb[0])
         assert L.read_status(ws) == 0  # cleared by the read
 
 
 def test_sum_f_output(cuda_device):
-    for path, n in (("fullsort", 1000), ("radix", 6000), ("bracket", 6000)):
+    for path, n in (("fullsort", 1000), ("radix", 6000), ("bracket", 6000), ("rowbracket", 6000)):
         r, _ = random_rows(2, 2, n)
         out = run_gpu(r, 20.0, 0.05, path=path, want_sum_f=True)
         for i in range(2):
@@ -160,7 +171,8 @@ def test_autograd_matches_library_backward(cuda_device):
 
 
 def test_repeat_calls_are_deterministic(cuda_device):
-    for path, n in (("fullsort", 2000), ("radix", 20000), ("bracket", 20000)):
+    for path, n in (("fullsort", 2000), ("radix", 20000), ("bracket", 20000),
+                    ("rowbracket", 20000)):
         r, v = random_rows(6, 2, n)
         a = run_gpu(r, 50.0, 0.05, path=path, v=v)
         c = run_gpu(r, 50.0, 0.05, path=path, v=v)
@@ -282,3 +294,26 @@ def test_autograd_long_rows_use_support(cuda_device):
     scale = g.abs().max().item()
     assert (rt.grad - g).abs().max().item() <= 1e-5 * scale
 
+
+
+def test_rowbracket_forced_miss_widens(cuda_device):
+    # every row starts from a bracket above all its samples and is widened
+    B, n = 4, 30000
+    r, v = random_rows(93, B, n, "mix_nu")
+    ws = L.Workspace(B, n, 50.0, "rowbracket")
+    rt = torch.from_numpy(r).cuda()
+    p, b = L.forward(rt, 50.0, 0.01, path=L.PATHS["rowbracket"] | L.FLAG_FORCE_MISS, ws=ws)
+    for i in range(B):
+        info = L.row_info(ws, i)
+        assert info["attempts"] >= 2 and info["path"] == 4
+        check_row(r[i], v[i], 50.0, 0.01, b[i].item(), p[i].cpu().numpy().astype(np.float64),
+                  label=f"rowbracket forced miss row {i}")
+
+
+def test_rowbracket_matches_radix(cuda_device):
+    B, n = 8, 65536
+    r, _ = random_rows(94, B, n, "normal_q64")
+    a = run_gpu(r, 1024.0, 0.02, path="rowbracket")
+    c = run_gpu(r, 1024.0, 0.02, path="radix")
+    for i in range(B):
+        assert abs(a["b"][i] - c["b"][i]) <= 1e-6 * max(0.02, abs(c["b"][i]))
