@@ -60,6 +60,9 @@ def configure(lib):
     lib.lso_vjp.restype = None
     lib.lso_vjp.argtypes = [_dp, _dp, ctypes.c_int64, ctypes.c_double, ctypes.c_double, _dp,
                             _dp, _dp]
+    lib.lso_vjp_kt.restype = None
+    lib.lso_vjp_kt.argtypes = [_dp, _dp, ctypes.c_int64, ctypes.c_double, ctypes.c_double, _dp,
+                               _dp]
     lib.lso_fold.restype = None
     lib.lso_fold.argtypes = [_dp, ctypes.c_int64, ctypes.c_double, ctypes.c_double,
                              ctypes.c_double, _i64p, _i64p, _i64p, _dp, _dp]
@@ -161,6 +164,19 @@ def vjp(r, v, b: float, t: float):
     _lib().lso_vjp(_ptr(a), _ptr(w), a.size, float(b), float(t), _ptr(g), ctypes.byref(R),
                    ctypes.byref(sf))
     return g, R.value, sf.value
+
+
+def vjp_kt(r, v, b: float, t: float):
+    """Returns (dL/dk, dL/dt) of L = sum_i v_i p_i."""
+    a = _f64(r)
+    w = _f64(v)
+    if a.size != w.size:
+        raise OracleError("r and v differ in length")
+    gk = ctypes.c_double(0.0)
+    gt = ctypes.c_double(0.0)
+    _lib().lso_vjp_kt(_ptr(a), _ptr(w), a.size, float(b), float(t), ctypes.byref(gk),
+                      ctypes.byref(gt))
+    return gk.value, gt.value
 
 
 def fold(r, aL: float, aR: float, t: float) -> dict:

@@ -208,6 +208,36 @@ void lso_vjp(const double* r, const double* v, int64_t n, double b, double t, do
 }
 
 /* ---------------------------------------------------------------------------
+ * Gradients of L = sum_i v_i p_i with respect to the budget k and the
+ * temperature t (section 2.1's budget equation differentiated implicitly,
+ * the same way as the VJP above).  With x_i = (r_i - b)/t, f_i = 0.5 e^{-|x_i|}:
+ *   db/dk = -t / sum f            so  dL/dk = sum v f / sum f;
+ *   db/dt = -sum f x / sum f      so  dL/dt = -(1/t) sum_i v_i f_i (x_i - xbar),
+ *   xbar = sum f x / sum f.
+ * The weights are shifted by min |x| as in lso_vjp; dL/dt carries the shift
+ * back through 0.5 e^{-mu}.
+ * ------------------------------------------------------------------------- */
+void lso_vjp_kt(const double* r, const double* v, int64_t n, double b, double t, double* g_k,
+                double* g_t) {
+    double mu = INFINITY;
+    for (int64_t i = 0; i < n; ++i) {
+        double ax = fabs(r[i] - b) / t;
+        if (ax < mu) mu = ax;
+    }
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;  /* sums of w, w v, w x, w v x */
+    for (int64_t i = 0; i < n; ++i) {
+        double x = (r[i] - b) / t;
+        double wt = exp(-(fabs(x) - mu));
+        a0 += wt;
+        a1 += wt * v[i];
+        a2 += wt * x;
+        a3 += wt * v[i] * x;
+    }
+    *g_k = a1 / a0;
+    *g_t = -(1.0 / t) * 0.5 * exp(-mu) * (a3 - a1 * a2 / a0);
+}
+
+/* ---------------------------------------------------------------------------
  * Probabilistic bracketing, step 2 (fold): with a bracket [aL, aR),
  *   cnt_R = #{r >= aR},  S_R = sum_{r >= aR} exp(-(r - aR)/t),
  *   cnt_L = #{r <  aL},  S_L = sum_{r <  aL} exp( (r - aL)/t),

@@ -397,11 +397,14 @@ cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* 
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    int64_t per_row = ((int64_t)sms * 8 + B - 1) / B;
+    // As a fallback (need != nullptr) it usually has nothing to do: one CTA
+    // per SM keeps the cost of launching it small.
+    const int64_t cta_per_sm = need != nullptr ? 1 : 8;
+    int64_t per_row = ((int64_t)sms * cta_per_sm + B - 1) / B;
     if (per_row > stream_tiles(n)) per_row = stream_tiles(n);
     if (per_row < 1) per_row = 1;
     const dim3 rgrid((unsigned)per_row, (unsigned)B);
-    int64_t apply_row = ((int64_t)sms * 16 + B - 1) / B;
+    int64_t apply_row = ((int64_t)sms * (need != nullptr ? 1 : 16) + B - 1) / B;
     if (apply_row > stream_tiles(n)) apply_row = stream_tiles(n);
     if (apply_row < 1) apply_row = 1;
     const dim3 grid_apply((unsigned)apply_row, (unsigned)B);

@@ -30,6 +30,10 @@ MUTANTS = [
      [pins.test_single_score_closed_form]),
     ("vjp_missing_inv_t", "g[i] = (f / t) * (v[i] - R);", "g[i] = f * (v[i] - R);",
      [lambda: pins.test_vjp_central_finite_differences(0, 12, 3.0, 0.5)]),
+    ("vjp_t_sign", "*g_t = -(1.0 / t) * 0.5", "*g_t = (1.0 / t) * 0.5",
+     [lambda: pins.test_vjp_kt_central_finite_differences(0, 12, 3.0, 0.5)]),
+    ("vjp_t_drops_mean", "(a3 - a1 * a2 / a0)", "(a3)",
+     [lambda: pins.test_vjp_kt_central_finite_differences(0, 12, 3.0, 0.5)]),
     ("vjp_unweighted_mean", "swv += w * v[i];", "swv += v[i];",
      [lambda: pins.test_vjp_identities(0)]),
     ("vjp_abs_dropped", "double f = 0.5 * exp(-fabs(r[i] - b) / t);",

@@ -222,6 +222,43 @@ def test_vjp_central_finite_differences(seed, n, k, t):
     assert checked >= n - 1
 
 
+@pytest.mark.parametrize("seed,n,k,t", [(0, 12, 3.0, 0.5), (1, 40, 7.5, 0.05), (2, 64, 1.5, 2.0),
+                                        (3, 30, 20.0, 0.01)])
+def test_vjp_kt_central_finite_differences(seed, n, k, t):
+    # dL/dk and dL/dt of L = sum v p against central differences of the full
+    # solve (b to full fp64 resolution at each shifted k or t)
+    rng = np.random.default_rng(300 + seed)
+    r = rng.standard_normal(n)
+    v = rng.standard_normal(n)
+    b = oracle.solve_b(r, k, t)
+    gk, gt = oracle.vjp_kt(r, v, b, t)
+    hk, ht = 1e-6 * max(1.0, k), 1e-6 * t
+    fdk = (_loss(r, v, k + hk, t) - _loss(r, v, k - hk, t)) / (2 * hk)
+    fdt = (_loss(r, v, k, t + ht) - _loss(r, v, k, t - ht)) / (2 * ht)
+    assert abs(fdk - gk) <= 1e-6 * max(1.0, abs(gk)), (fdk, gk)
+    assert abs(fdt - gt) <= 1e-5 * max(1.0, abs(gt)), (fdt, gt)
+
+
+def test_vjp_kt_identities():
+    # sum p = k for every k and t: with v = 1, dL/dk = 1 and dL/dt = 0; both
+    # gradients are linear in v, and a constant shift of the scores moves neither
+    rng = np.random.default_rng(9)
+    n, k, t = 25, 4.0, 0.3
+    r = rng.standard_normal(n)
+    b = oracle.solve_b(r, k, t)
+    gk, gt = oracle.vjp_kt(r, np.ones(n), b, t)
+    assert abs(gk - 1.0) <= 1e-12 and abs(gt) <= 1e-12
+    v1, v2 = rng.standard_normal(n), rng.standard_normal(n)
+    a1, a2 = oracle.vjp_kt(r, v1, b, t), oracle.vjp_kt(r, v2, b, t)
+    a3 = oracle.vjp_kt(r, 2.0 * v1 - 3.0 * v2, b, t)
+    assert abs(a3[0] - (2 * a1[0] - 3 * a2[0])) <= 1e-12
+    assert abs(a3[1] - (2 * a1[1] - 3 * a2[1])) <= 1e-10
+    c = 5.5
+    bs = oracle.solve_b(r + c, k, t)
+    s1 = oracle.vjp_kt(r + c, v1, bs, t)
+    assert abs(s1[0] - a1[0]) <= 1e-10 and abs(s1[1] - a1[1]) <= 1e-8
+
+
 def test_jacobian_symmetric_and_matches_fd():
     rng = np.random.default_rng(5)
     n, k, t = 8, 3.0, 0.3
