@@ -158,6 +158,22 @@ int lapsum_backward_support(const float* r, int64_t ld, const double* b, const f
                             size_t support_bytes, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Gradients of L = sum_i v_i p_i with respect to each row's budget k and
+ * temperature t, for learning them.  The pages give only the analytic VJP in
+ * the scores (section 2.1); these follow from the same implicit
+ * differentiation of the budget equation: with x_i = (r_i - b)/t and
+ * f_i = 0.5 exp(-|x_i|),
+ *     g_k[row] = dL/dk = sum_i v_i f_i / sum_i f_i,
+ *     g_t[row] = dL/dt = -(1/t) sum_i v_i f_i (x_i - xbar),  xbar = sum f x / sum f.
+ * One pass over r and v (8 bytes per score); weights shifted by the row's
+ * smallest |x| as in lapsum_backward.  g_k and g_t are device arrays of B
+ * doubles (either may be NULL, not both); ws is a lapsum_backward workspace.
+ */
+int lapsum_backward_kt(const float* r, int64_t ld, const double* b, const float* v, int64_t B,
+                       int64_t n, double t, double* g_k, double* g_t, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
  * Synchronises `stream`, copies the sticky device status word to
  * *device_status (LAPSUM_OK, or a LAPSUM_E* code for the first condition
  * seen) and clears it.  Returns LAPSUM_OK or LAPSUM_ECUDA.

@@ -26,7 +26,7 @@ from . import _build
 __all__ = [
     "LapSumError", "Workspace", "forward", "backward", "read_status", "row_info", "sample_values",
     "workspace_bytes", "soft_topk", "LapSumTopK", "PATHS", "FLAG_FORCE_MISS", "FLAG_NO_RETRY",
-    "FLAG_ONE_CTA_SOLVE", "library_path", "profile_enable", "profile_read", "backward_noalloc", "Support",
+    "FLAG_ONE_CTA_SOLVE", "library_path", "profile_enable", "backward_kt", "profile_read", "backward_noalloc", "Support",
     "support_bytes",
 ]
 
@@ -111,6 +111,9 @@ def _lib():
         lib.lapsum_backward_support.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64,
                                                 ctypes.c_double, _vp, ctypes.c_size_t, _vp,
                                                 ctypes.c_size_t, _vp]
+        lib.lapsum_backward_kt.restype = ctypes.c_int
+        lib.lapsum_backward_kt.argtypes = [_vp, _c_i64, _vp, _vp, _c_i64, _c_i64, ctypes.c_double,
+                                           _vp, _vp, _vp, ctypes.c_size_t, _vp]
         lib.lapsum_sample_get.restype = ctypes.c_int
         lib.lapsum_sample_get.argtypes = [_vp, _c_i64, _vp, _c_i64, _vp]
         _LIB = lib
@@ -303,6 +306,29 @@ def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Wo
     return g[0] if squeeze else g
 
 
+def backward_kt(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float,
+                ws: Workspace = None):
+    """(dL/dk, dL/dt) per row of L = sum v p, as float64 tensors of B entries."""
+    r2 = _as_rows(r)
+    v2 = _as_rows(v)
+    B, n = r2.shape
+    if v2.shape != r2.shape:
+        raise ValueError("v must have the shape of r")
+    if _ld(v2) != _ld(r2):
+        v2 = v2.contiguous()
+        r2 = r2.contiguous()
+    if b.dtype != torch.float64 or not b.is_cuda or b.numel() != B:
+        raise TypeError("b must be a float64 CUDA tensor with one entry per row")
+    if ws is None or not ws.fits_backward(B, n):
+        ws = Workspace(B, n, 0.5, "fullsort", r2.device)
+    gk = torch.empty(B, dtype=torch.float64, device=r2.device)
+    gt = torch.empty(B, dtype=torch.float64, device=r2.device)
+    _check(_lib().lapsum_backward_kt(r2.data_ptr(), _ld(r2), b.data_ptr(), v2.data_ptr(), B, n,
+                                     float(t), gk.data_ptr(), gt.data_ptr(), ws.ptr, ws.nbytes,
+                                     _stream_ptr(r2.device)), "lapsum_backward_kt")
+    return gk, gt
+
+
 def backward_noalloc(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float,
                      g: torch.Tensor = None):
     """Backward without a workspace, for callers that cannot allocate device memory.
@@ -383,19 +409,34 @@ class LapSumTopK(torch.autograd.Function):
         rd = r.detach()
         B = 1 if rd.dim() == 1 else rd.shape[0]
         n = rd.shape[-1]
+        kf = float(k)
+        tf = float(t)
         sup = Support(B, n, rd.device) if support_bytes(B, n) > 0 else None
-        p, b = forward(rd, k, t, path=path, seed=seed, support=sup)
+        p, b = forward(rd, kf, tf, path=path, seed=seed, support=sup)
         ctx.save_for_backward(r, b)
-        ctx.t = t
+        ctx.t = tf
         ctx.sup = sup
+        ctx.kt_grad = (isinstance(k, torch.Tensor) and k.requires_grad,
+                       isinstance(t, torch.Tensor) and t.requires_grad)
+        ctx.kt_like = (k, t)
         return p
 
     @staticmethod
     def backward(ctx, gp):
         r, b = ctx.saved_tensors
-        g = backward(r.detach(), b, gp.contiguous(), ctx.t, support=ctx.sup)
+        v = gp.contiguous()
+        g = backward(r.detach(), b, v, ctx.t, support=ctx.sup)
         ctx.sup = None
-        return g, None, None, None, None
+        gk = gt = None
+        if any(ctx.kt_grad):
+            # k and t are shared by every row: their gradients sum over rows
+            gks, gts = backward_kt(r.detach(), b, v, ctx.t)
+            k, t = ctx.kt_like
+            if ctx.kt_grad[0]:
+                gk = gks.sum().to(k.dtype).reshape(k.shape)
+            if ctx.kt_grad[1]:
+                gt = gts.sum().to(t.dtype).reshape(t.shape)
+        return g, gk, gt, None, None
 
 
 def soft_topk(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0) -> torch.Tensor:

@@ -65,7 +65,7 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
     L.tickets = take((size_t)B * 2 * sizeof(uint32_t) + (2 + 2048) * sizeof(uint32_t));
     L.fold_ticket = L.tickets + (size_t)B * 2 * sizeof(uint32_t);
     L.rows = take((size_t)B * sizeof(RowState));
-    L.partials = take((size_t)B * (size_t)tiles * 4 * sizeof(double));
+    L.partials = take((size_t)B * (size_t)(tiles > 2 ? tiles : 2) * 4 * sizeof(double));
     L.row_R = take((size_t)B * sizeof(double));
     if (n > kOnchipMax) {  // windowed backward of long rows
         // the pass CTAs of a row split the capacity evenly (rounded up per CTA)
@@ -453,6 +453,32 @@ int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v,
                                        t, partials + r0 * stream_tiles(n) * 4, row_R + r0,
                                        tickets + B + r0, vec, st);
         }
+    }
+    return cuda_status(e);
+}
+
+int lapsum_backward_kt(const float* r, int64_t ld, const double* b, const float* v, int64_t B,
+                       int64_t n, double t, double* g_k, double* g_t, void* ws, size_t ws_bytes,
+                       void* stream) {
+    if (r == nullptr || b == nullptr || v == nullptr || (g_k == nullptr && g_t == nullptr))
+        return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const Layout L = make_layout(B, n, LAPSUM_PATH_FULLSORT);
+    if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+    char* w = static_cast<char*>(ws);
+    uint32_t* tickets = reinterpret_cast<uint32_t*>(w + L.tickets);
+    double* partials = reinterpret_cast<double*>(w + L.partials);
+    const int vec = (aligned16(r) && aligned16(v) && (ld % 4) == 0) ? 1 : 0;
+    const int64_t slots = stream_tiles(n) > 2 ? stream_tiles(n) : 2;
+    cudaError_t e = cudaSuccess;
+    for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
+        const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+        e = launch_backward_kt(r + r0 * ld, ld, b + r0, v + r0 * ld, nb, n, t,
+                               partials + r0 * slots * 4, tickets + B + r0,
+                               g_k ? g_k + r0 : nullptr, g_t ? g_t + r0 : nullptr, vec,
+                               static_cast<cudaStream_t>(stream));
     }
     return cuda_status(e);
 }

@@ -90,6 +90,13 @@ cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* 
                                       double* partials, double* row_R, uint32_t* tickets, int vec,
                                       const uint32_t* need, cudaStream_t st);
 
+// Gradients of sum v p with respect to k and t, per row; partials: the
+// backward partials region (max(tiles, 2) * 4 doubles per row).
+cudaError_t launch_backward_kt(const float* r, int64_t ld, const double* b, const float* v,
+                               int64_t B, int64_t n, double t, double* partials,
+                               uint32_t* tickets, double* g_k, double* g_t, int vec,
+                               cudaStream_t st);
+
 // --- windowed backward (scores with |x| <= 90 only) ----------------------------
 struct WinEntry {
     uint32_t idx;  // position in the row

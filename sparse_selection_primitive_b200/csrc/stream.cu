@@ -353,6 +353,107 @@ __global__ void __launch_bounds__(kThreads) bwd_apply_kernel(
     }
 }
 
+// Gradients of L = sum v p with respect to k and t, per row (implicit
+// derivatives of the budget equation, "Fast LapSum" pages section 2.1):
+//   dL/dk = sum v f / sum f,   dL/dt = -(1/t) sum_i v_i f_i (x_i - xbar),
+//   xbar = sum f x / sum f,  x = (r - b)/t,  f = 0.5 exp(-|x|).
+// One pass over (r, v): each thread keeps (mu, S, Sv, Sx, Svx) with weights
+// w = exp(-(|x| - mu)), mu its smallest |x| so far (a smaller one rescales the
+// sums once); CTA records of 8 doubles are combined in CTA order by the row's
+// last CTA.
+__device__ __forceinline__ void kt_add(float a, float x, float vv, float& mu, double& s0,
+                                       double& s1, double& s2, double& s3) {
+    if (a < mu) {
+        const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(a - mu);
+        s0 *= sc;
+        s1 *= sc;
+        s2 *= sc;
+        s3 *= sc;
+        mu = a;
+    }
+    const float w = __expf(mu - a);
+    s0 += (double)w;
+    s1 += (double)(w * vv);
+    s2 += (double)(w * x);
+    s3 += (double)(w * vv * x);
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads) bwd_kt_kernel(
+    const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
+    const float* __restrict__ v, int64_t n, double t, double* __restrict__ partials,
+    uint32_t* __restrict__ tickets, double* __restrict__ g_k, double* __restrict__ g_t) {
+    __shared__ double red[kThreads / 32];
+    __shared__ float fred[kThreads / 32];
+    __shared__ int flag;
+    const int64_t row = blockIdx.y;
+    const int64_t nblk = gridDim.x;
+    const Thr th = make_thr(b[row], t);
+    const float* rr = r + row * ld;
+    const float* vr = v + row * ld;
+    float mu = INFINITY;
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    const int64_t stride = nblk * kThreads;
+    const int64_t gt0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    auto one = [&](float rv, float vv) {
+        const float x = scaled_margin(rv, th);
+        kt_add(fabsf(x), x, vv, mu, s0, s1, s2, s3);
+    };
+    if constexpr (VEC) {
+        const int64_t n4 = n >> 2;
+        const float4* r4 = reinterpret_cast<const float4*>(rr);
+        const float4* v4 = reinterpret_cast<const float4*>(vr);
+        for (int64_t i = gt0; i < n4; i += stride) {
+            const float4 x = __ldcs(r4 + i), y = __ldcs(v4 + i);
+            one(x.x, y.x);
+            one(x.y, y.y);
+            one(x.z, y.z);
+            one(x.w, y.w);
+        }
+        for (int64_t j = (n4 << 2) + gt0; j < n; j += stride) one(rr[j], vr[j]);
+    } else {
+        for (int64_t j = gt0; j < n; j += stride) one(rr[j], vr[j]);
+    }
+    const float mb = block_min_f(mu, fred);
+    const double sc = (mu == INFINITY) ? 0.0 : exp((double)mb - (double)mu);
+    s0 = block_sum_d(s0 * sc, red);
+    s1 = block_sum_d(s1 * sc, red);
+    s2 = block_sum_d(s2 * sc, red);
+    s3 = block_sum_d(s3 * sc, red);
+    if (threadIdx.x == 0) {
+        double* pr = partials + (row * nblk + blockIdx.x) * 8;
+        pr[0] = (double)mb;
+        pr[1] = s0;
+        pr[2] = s1;
+        pr[3] = s2;
+        pr[4] = s3;
+    }
+    if (last_block_of_row(&tickets[row], (uint32_t)nblk, &flag)) {
+        float mloc = INFINITY;
+        for (int64_t i = threadIdx.x; i < nblk; i += kThreads)
+            mloc = fminf(mloc, (float)partials[(row * nblk + i) * 8]);
+        const double mrow = (double)block_min_f(mloc, fred);
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+        for (int64_t i = threadIdx.x; i < nblk; i += kThreads) {
+            const double* pr = partials + (row * nblk + i) * 8;
+            if (pr[0] == INFINITY) continue;
+            const double f = exp(mrow - pr[0]);
+            a0 += pr[1] * f;
+            a1 += pr[2] * f;
+            a2 += pr[3] * f;
+            a3 += pr[4] * f;
+        }
+        a0 = block_sum_d(a0, red);
+        a1 = block_sum_d(a1, red);
+        a2 = block_sum_d(a2, red);
+        a3 = block_sum_d(a3, red);
+        if (threadIdx.x == 0) {
+            if (g_k) g_k[row] = a1 / a0;
+            if (g_t) g_t[row] = -(1.0 / t) * 0.5 * exp(-mrow) * (a3 - a1 * a2 / a0);
+        }
+    }
+}
+
 }  // namespace
 
 int64_t stream_tiles(int64_t n) { return (n + kStreamTile - 1) / kStreamTile; }
@@ -439,6 +540,37 @@ cudaError_t launch_backward_stream(const float* r, int64_t ld, const double* b, 
                                    double* row_R, uint32_t* tickets, int vec, cudaStream_t st) {
     return launch_backward_stream_if(r, ld, b, v, g, B, n, t, partials, row_R, tickets, vec,
                                      nullptr, st);
+}
+
+}  // namespace lapsum
+
+namespace lapsum {
+
+cudaError_t launch_backward_kt(const float* r, int64_t ld, const double* b, const float* v,
+                               int64_t B, int64_t n, double t, double* partials,
+                               uint32_t* tickets, double* g_k, double* g_t, int vec,
+                               cudaStream_t st) {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    // records of 8 doubles: at most half as many CTAs per row as the partials
+    // region has 4-double slots per row (max(tiles, 2))
+    int64_t cap = stream_tiles(n) > 2 ? stream_tiles(n) / 2 : 1;
+    int64_t per_row = ((int64_t)sms * 8 + B - 1) / B;
+    if (per_row > cap) per_row = cap;
+    if (per_row < 1) per_row = 1;
+    const dim3 grid((unsigned)per_row, (unsigned)B);
+    ProfScope ps_("bwd_kt", st);
+    if (vec)
+        bwd_kt_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, tickets, g_k,
+                                                       g_t);
+    else
+        bwd_kt_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, tickets, g_k,
+                                                        g_t);
+    return cudaGetLastError();
 }
 
 }  // namespace lapsum

@@ -317,3 +317,46 @@ def test_rowbracket_matches_radix(cuda_device):
     c = run_gpu(r, 1024.0, 0.02, path="radix")
     for i in range(B):
         assert abs(a["b"][i] - c["b"][i]) <= 1e-6 * max(0.02, abs(c["b"][i]))
+
+
+# ---------------------------------------------------------------------------
+# Gradients with respect to k and t.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,n,k,t,dist", [
+    (3, 100, 7.0, 0.3, "normal"),
+    (2, 5000, 40.0, 0.02, "normal_q64"),
+    (1, 70001, 300.0, 0.005, "mix_nu"),
+    (2, 1 << 18, 2000.0, 1.0, "normal"),
+])
+def test_backward_kt_matches_oracle(cuda_device, B, n, k, t, dist):
+    r, v = random_rows(71 + n, B, n, dist)
+    rt = torch.from_numpy(r).cuda()
+    vt = torch.from_numpy(v).cuda()
+    _, b = L.forward(rt, k, t)
+    gk, gt = L.backward_kt(rt, b, vt, t)
+    gk, gt, bb = gk.cpu().numpy(), gt.cpu().numpy(), b.cpu().numpy()
+    for i in range(B):
+        b_ref = oracle.solve_b(r[i], k, t)
+        assert abs(bb[i] - b_ref) <= 1e-5 * max(t, abs(b_ref))
+        rk, rt_ = oracle.vjp_kt(r[i], v[i], b_ref, t)
+        assert abs(gk[i] - rk) <= 1e-4 * max(1.0, abs(rk)), (i, gk[i], rk)
+        assert abs(gt[i] - rt_) <= 1e-4 * max(abs(rt_), 1e-3 * abs(rk) / t), (i, gt[i], rt_)
+
+
+def test_autograd_learnable_k_and_t(cuda_device):
+    B, n = 4, 3000
+    r, v = random_rows(72, B, n)
+    rt = torch.from_numpy(r).cuda().requires_grad_(True)
+    k = torch.tensor(25.0, dtype=torch.float64, device="cuda", requires_grad=True)
+    t = torch.tensor(0.05, dtype=torch.float64, device="cuda", requires_grad=True)
+    p = L.soft_topk(rt, k, t)
+    p.backward(torch.from_numpy(v).cuda())
+    gk_ref = gt_ref = 0.0
+    for i in range(B):
+        b_ref = oracle.solve_b(r[i], 25.0, 0.05)
+        a, c = oracle.vjp_kt(r[i], v[i], b_ref, 0.05)
+        gk_ref += a
+        gt_ref += c
+    assert abs(k.grad.item() - gk_ref) <= 1e-4 * max(1.0, abs(gk_ref))
+    assert abs(t.grad.item() - gt_ref) <= 1e-4 * max(1.0, abs(gt_ref))
+    assert rt.grad is not None and torch.isfinite(rt.grad).all()
