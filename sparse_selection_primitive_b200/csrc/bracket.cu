@@ -288,6 +288,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
                                                       uint32_t* __restrict__ ghist,
                                                       uint32_t* __restrict__ ticket,
                                                       RowState* st) {
+    pdl_wait();
     if (blockIdx.x == 0) {
         // this kernel starts the row's forward: clear its record and histogram
         for (int i = threadIdx.x; i < (int)(sizeof(RowState) / 4); i += kBlk)
@@ -518,6 +519,7 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
                                                             double* __restrict__ part,
                                                             uint32_t* __restrict__ ticket,
                                                             WsHeader* hdr, int vec) {
+    pdl_wait();
     __shared__ double red[kFoldThreads / 32];
     __shared__ long long lred[kFoldThreads / 32];
     __shared__ float sband[kStage];
@@ -1497,6 +1499,7 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
                                              const float* __restrict__ sample, int m,
                                              Ladder lad, double* __restrict__ b_out,
                                              WsHeader* hdr, int split) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
     phase_mark(st, 2);
@@ -1552,6 +1555,7 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
                                                   float* __restrict__ band0_all,
                                                   float* __restrict__ band1_all,
                                                   double* __restrict__ b_all, WsHeader* hdr) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
     RowBracketSmem* rb = reinterpret_cast<RowBracketSmem*>(dsm + sizeof(SolveSmemAll));
@@ -1645,6 +1649,7 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
 // grid (the band is large; the bin holds at most 4096 scores).
 __global__ void __launch_bounds__(256) extract_kernel(const float* __restrict__ band,
                                                       RowState* st, float* __restrict__ sub) {
+    pdl_wait();
     if (st->stage != 1) return;
     if (blockIdx.x == 0) phase_mark(st, 18);
     const long long nb = (long long)st->n_band;
@@ -1690,6 +1695,7 @@ __global__ void __maxnreg__(64) solve2_kernel(double k, double t, RowState* st,
                                                       float* __restrict__ sub,
                                                       const unsigned long long* __restrict__ bins,
                                                       double* __restrict__ b_out, WsHeader* hdr) {
+    pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
     if (st->stage != 1) return;
@@ -1798,7 +1804,7 @@ cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, 
     const int force_miss = (flags & LAPSUM_FLAG_FORCE_MISS) ? 1 : 0;
     const int max_attempts = (flags & LAPSUM_FLAG_NO_RETRY) ? 1 : kMaxAttempts;
     ProfScope ps_("rowbracket", st);
-    rowbracket_kernel<<<(unsigned)B, kBlk, rowbracket_smem(m), st>>>(
+    launch_pdl(rowbracket_kernel, dim3((unsigned)B), dim3(kBlk), rowbracket_smem(m), st, 
         r, ld, n, k, t, seed, m, lad, force_miss, max_attempts, vec, rows, band0, band1, b, hdr);
     return cudaGetLastError();
 }
@@ -1852,14 +1858,14 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     const uint64_t c0 = (uint64_t)row << 32;
     {
         ProfScope ps_("bracket_sample", st);
-        sample_kernel<<<(m + kBlk - 1) / kBlk, kBlk, sample_smem, st>>>(
+        launch_pdl(sample_kernel, dim3((m + kBlk - 1) / kBlk), dim3(kBlk), sample_smem, st, 
             r_row, n, t, seed, c0, m, lad, force_miss, max_attempts, sample, buf.bins,
             buf.ticket + 2, buf.ticket + 1, st_row);
     }
     const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
     {
         ProfScope ps_("bracket_fold", st);
-        fold_kernel<<<buf.fold_grid, kFoldThreads, kFoldDynSmem, st>>>(r_row, n, t, st_row,
+        launch_pdl(fold_kernel, dim3(buf.fold_grid), dim3(kFoldThreads), kFoldDynSmem, st, r_row, n, t, st_row,
                                                                     buf.band[0],
                                                         buf.bins, buf.fold_part, buf.ticket, hdr,
                                                         vec);
@@ -1878,19 +1884,19 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
             : 0;
     {
         ProfScope ps_("bracket_solve", st);
-        solve_kernel<<<1, kBlk, solve_smem, st>>>(r_row, n, vec, k, t, st_row, buf.band[0],
+        launch_pdl(solve_kernel, dim3(1), dim3(kBlk), solve_smem, st, r_row, n, vec, k, t, st_row, buf.band[0],
                                               buf.band[1], buf.bins, sample, m, lad, b_out, hdr,
                                               split);
     }
     if (split) {
         {
             ProfScope ps_("bracket_extract", st);
-            extract_kernel<<<bracket_fold_grid() / 2 > 0 ? bracket_fold_grid() / 2 : 1, 256, 0,
-                             st>>>(buf.band[0], st_row, buf.band[1]);
+            const int xgrid = bracket_fold_grid() / 2 > 0 ? bracket_fold_grid() / 2 : 1;
+            launch_pdl(extract_kernel, dim3(xgrid), dim3(256), 0, st, buf.band[0], st_row, buf.band[1]);
         }
         {
             ProfScope ps_("bracket_solve2", st);
-            solve2_kernel<<<1, kBlk, solve_smem, st>>>(k, t, st_row, buf.band[0], buf.band[1],
+            launch_pdl(solve2_kernel, dim3(1), dim3(kBlk), solve_smem, st, k, t, st_row, buf.band[0], buf.band[1],
                                                        buf.bins, b_out, hdr);
         }
     }

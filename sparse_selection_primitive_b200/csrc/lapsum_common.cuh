@@ -418,6 +418,12 @@ __device__ __forceinline__ void phase_mark(RowState* st, int slot) {
     }
 }
 
+// Programmatic dependent launch: kernels of the long-row pipelines are
+// launched so that they may be scheduled while the previous kernel on the
+// stream drains; each calls pdl_wait() before it touches any memory, which
+// returns once the previous grid has finished and its writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void set_status(WsHeader* hdr, uint32_t bits) {
     atomicOr(&hdr->status, bits);
 }

@@ -18,6 +18,25 @@ struct ProfScope {
     ~ProfScope() { prof_end(st); }
 };
 
+// Launch with programmatic stream serialization (see pdl_wait): the kernel may
+// start while the previous kernel on the stream finishes.  Every kernel
+// launched this way calls pdl_wait() before its first memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // --- on-chip full sort (n <= 4096) -------------------------------------------
 int onchip_npad(int64_t n);
 cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,

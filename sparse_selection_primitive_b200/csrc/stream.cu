@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
                                                         WsHeader* hdr, int record_call,
                                                         int64_t B_total, int path_code,
                                                         SupportView sup) {
+    pdl_wait();
     __shared__ double red[kThreads / 32];
     __shared__ int flag;
     const int64_t row = blockIdx.y;
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     const float* __restrict__ v, int64_t n, double t, double* __restrict__ partials,
     double* __restrict__ row_R, uint32_t* __restrict__ tickets,
     const uint32_t* __restrict__ need) {
+    pdl_wait();
     __shared__ double red[kThreads / 32];
     __shared__ float fred[kThreads / 32];
     __shared__ int flag;
@@ -333,6 +335,7 @@ __global__ void __launch_bounds__(kThreads) bwd_apply_kernel(
     const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
     const float* __restrict__ v, float* __restrict__ g, int64_t n, double t,
     const double* __restrict__ row_R, const uint32_t* __restrict__ need) {
+    pdl_wait();
     const int64_t row = blockIdx.y;
     if (need != nullptr && need[row] == 0u) return;
     const Thr th = make_thr(b[row], t);
@@ -383,6 +386,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kt_kernel(
     const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
     const float* __restrict__ v, int64_t n, double t, double* __restrict__ partials,
     uint32_t* __restrict__ tickets, double* __restrict__ g_k, double* __restrict__ g_t) {
+    pdl_wait();
     __shared__ double red[kThreads / 32];
     __shared__ float fred[kThreads / 32];
     __shared__ int flag;
@@ -466,8 +470,8 @@ cudaError_t launch_emit(const float* r, int64_t ld, float* p, double* b, double*
     ProfScope ps_("emit", st);
     const SupportView sv = sup ? *sup : SupportView{};
 #define LAPSUM_EMIT(V, S, U)                                                                  \
-    emit_kernel<V, S, U><<<grid, kThreads, 0, st>>>(r, ld, p, b, sumf, n, t, partials, tickets, \
-                                                    hdr, record_call, B_total, path_code, sv)
+    launch_pdl(emit_kernel<V, S, U>, grid, dim3(kThreads), 0, st, r, ld, p, b, sumf, n, t,    \
+               partials, tickets, hdr, record_call, B_total, path_code, sv)
     if (sup) {
         if (vec) {
             if (sumf) LAPSUM_EMIT(true, true, true);
@@ -512,23 +516,23 @@ cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* 
     if (vec) {
         {
             ProfScope ps_("bwd_reduce", st);
-            bwd_reduce_kernel<true><<<rgrid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, row_R,
+            launch_pdl(bwd_reduce_kernel<true>, dim3(rgrid), dim3(kThreads), 0, st, r, ld, b, v, n, t, partials, row_R,
                                                                 tickets, need);
         }
         {
             ProfScope ps_("bwd_apply", st);
-            bwd_apply_kernel<true><<<grid_apply, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R,
+            launch_pdl(bwd_apply_kernel<true>, dim3(grid_apply), dim3(kThreads), 0, st, r, ld, b, v, g, n, t, row_R,
                                                                     need);
         }
     } else {
         {
             ProfScope ps_("bwd_reduce", st);
-            bwd_reduce_kernel<false><<<rgrid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials,
+            launch_pdl(bwd_reduce_kernel<false>, dim3(rgrid), dim3(kThreads), 0, st, r, ld, b, v, n, t, partials,
                                                                  row_R, tickets, need);
         }
         {
             ProfScope ps_("bwd_apply", st);
-            bwd_apply_kernel<false><<<grid_apply, kThreads, 0, st>>>(r, ld, b, v, g, n, t, row_R,
+            launch_pdl(bwd_apply_kernel<false>, dim3(grid_apply), dim3(kThreads), 0, st, r, ld, b, v, g, n, t, row_R,
                                                                      need);
         }
     }
@@ -565,10 +569,10 @@ cudaError_t launch_backward_kt(const float* r, int64_t ld, const double* b, cons
     const dim3 grid((unsigned)per_row, (unsigned)B);
     ProfScope ps_("bwd_kt", st);
     if (vec)
-        bwd_kt_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, tickets, g_k,
+        launch_pdl(bwd_kt_kernel<true>, dim3(grid), dim3(kThreads), 0, st, r, ld, b, v, n, t, partials, tickets, g_k,
                                                        g_t);
     else
-        bwd_kt_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, partials, tickets, g_k,
+        launch_pdl(bwd_kt_kernel<false>, dim3(grid), dim3(kThreads), 0, st, r, ld, b, v, n, t, partials, tickets, g_k,
                                                         g_t);
     return cudaGetLastError();
 }

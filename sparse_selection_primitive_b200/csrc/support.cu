@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     const double* __restrict__ b, const float* __restrict__ v, int64_t ld, int64_t n,
     int64_t B_total, int group, SupportView sup, double* __restrict__ partials,
     double* __restrict__ row_R, uint32_t* __restrict__ tickets, uint32_t* __restrict__ dense_flag) {
+    pdl_wait();
     __shared__ uint32_t pre[kThreads + 1];  // exclusive prefix of the group's share counts
     __shared__ uint32_t wtot[kThreads / 32];
     __shared__ double red[kThreads / 32];
@@ -239,6 +240,7 @@ template <bool VEC>
 __global__ void __launch_bounds__(kThreads) sup_write_kernel(
     SupportView sup, const uint32_t* __restrict__ dense_flag, const double* __restrict__ row_R,
     float* __restrict__ g, int64_t ld, int64_t n, double t) {
+    pdl_wait();
     __shared__ __align__(16) float stage[kShares][kTile / kShares];
     const int64_t row = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -366,16 +368,16 @@ cudaError_t launch_backward_support(const float* r, int64_t ld, const double* b,
     const int64_t per_row = ngroups < want ? ngroups : want;
     {
         ProfScope ps_("sup_reduce", st);
-        sup_reduce_kernel<<<dim3((unsigned)per_row, (unsigned)B), kThreads, 0, st>>>(
+        launch_pdl(sup_reduce_kernel, dim3(dim3((unsigned)per_row, (unsigned)B)), dim3(kThreads), 0, st, 
             b, v, ld, n, B_total, (int)group, sup, partials, row_R, tickets, dense_flag);
     }
     {
         ProfScope ps_("sup_write", st);
         const dim3 grid((unsigned)tiles, (unsigned)B);
         if (vec)
-            sup_write_kernel<true><<<grid, kThreads, 0, st>>>(sup, dense_flag, row_R, g, ld, n, t);
+            launch_pdl(sup_write_kernel<true>, dim3(grid), dim3(kThreads), 0, st, sup, dense_flag, row_R, g, ld, n, t);
         else
-            sup_write_kernel<false><<<grid, kThreads, 0, st>>>(sup, dense_flag, row_R, g, ld, n,
+            launch_pdl(sup_write_kernel<false>, dim3(grid), dim3(kThreads), 0, st, sup, dense_flag, row_R, g, ld, n,
                                                                 t);
     }
     // rows the list could not serve: dense recompute (exits at once otherwise)

@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kThreads) window_pass_kernel(
     const float* __restrict__ v, int64_t n, double t, WinEntry* __restrict__ list,
     uint32_t cap_cta, uint2* __restrict__ tab, uint32_t* __restrict__ wflag,
     double* __restrict__ partials, double* __restrict__ row_R, uint32_t* __restrict__ tickets) {
+    pdl_wait();
     __shared__ int scnt, ovf, tstart;
     __shared__ double red[kThreads / 32];
     __shared__ float fred[kThreads / 32];
@@ -223,6 +224,7 @@ __global__ void __launch_bounds__(kThreads) window_write_kernel(
     const WinEntry* __restrict__ list, uint32_t cap_cta, int64_t pass_blocks,
     const uint2* __restrict__ tab, const uint32_t* __restrict__ wflag,
     const double* __restrict__ row_R, float* __restrict__ g, int64_t ld, int64_t n, double t) {
+    pdl_wait();
     const int64_t row = blockIdx.y;
     if (wflag[row]) return;  // the dense kernels own this row
     const int64_t ntiles = (n + kTile - 1) / kTile;
@@ -289,21 +291,21 @@ cudaError_t launch_backward_window(const float* r, int64_t ld, const double* b, 
     {
         ProfScope ps_("window_pass", st);
         if (vec)
-            window_pass_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, wb.list, cap_cta,
+            launch_pdl(window_pass_kernel<true>, dim3(grid), dim3(kThreads), 0, st, r, ld, b, v, n, t, wb.list, cap_cta,
                                                                 wb.tab, wb.flag, partials, row_R,
                                                                 tickets);
         else
-            window_pass_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, b, v, n, t, wb.list,
+            launch_pdl(window_pass_kernel<false>, dim3(grid), dim3(kThreads), 0, st, r, ld, b, v, n, t, wb.list,
                                                                  cap_cta, wb.tab, wb.flag,
                                                                  partials, row_R, tickets);
     }
     {
         ProfScope ps_("window_write", st);
         if (vec)
-            window_write_kernel<true><<<wgrid, kThreads, 0, st>>>(wb.list, cap_cta, per_row, wb.tab,
+            launch_pdl(window_write_kernel<true>, dim3(wgrid), dim3(kThreads), 0, st, wb.list, cap_cta, per_row, wb.tab,
                                                                   wb.flag, row_R, g, ld, n, t);
         else
-            window_write_kernel<false><<<wgrid, kThreads, 0, st>>>(wb.list, cap_cta, per_row,
+            launch_pdl(window_write_kernel<false>, dim3(wgrid), dim3(kThreads), 0, st, wb.list, cap_cta, per_row,
                                                                    wb.tab, wb.flag, row_R, g, ld,
                                                                    n, t);
     }
