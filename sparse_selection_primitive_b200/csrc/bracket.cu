@@ -815,7 +815,7 @@ __device__ void sort_band_into(const float* band, long long nb, SolveSmemAll* sm
         const long long j = (long long)threadIdx.x * E + e;
         key[e] = j < nb ? to_key(band[j]) : 0xffffffffu;
     }
-    bitonic_sort_block_rolled<E, kBlk>(key, threadIdx.x, sm->u.sort.xch);
+    bitonic_sort_row<E, kBlk, kBlk>(key, threadIdx.x, sm->u.sort.xch);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const long long j = (long long)threadIdx.x * E + e;
@@ -1431,7 +1431,13 @@ __device__ bool bracket_attempts(const float* __restrict__ r, int64_t n, int vec
         if (via_bins >= 0) {
             // handled through the histogram
         } else if (nb <= kBandSortMax) {
-            solve_small_band(cur, nb, tl, k, t, sm);
+            phase_mark(st, 19);
+            if (nb <= kBlk) sort_band_into<1>(cur, nb, sm);
+            else if (nb <= 2 * kBlk) sort_band_into<2>(cur, nb, sm);
+            else sort_band_into<4>(cur, nb, sm);
+            phase_mark(st, 20);
+            solve_sorted_block(FloatGet{sm->u.sort.sorted}, nb, tl, k, t, &sm->ss, &sm->res);
+            phase_mark(st, 21);
             certified = sm->res.F_aL >= k && sm->res.F_aR <= k;
             if (certified) {
                 b = sm->res.b;
