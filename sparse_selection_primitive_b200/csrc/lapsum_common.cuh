@@ -188,18 +188,25 @@ __device__ __forceinline__ Aff warp_scan_bwd(Aff v, int lane) {
 // Block-wide exclusive scans of affine maps (every thread calls; `wt` holds
 // blockDim.x/32 maps of shared memory).  Forward: composition of the maps of
 // all lower threads (thread 0 applied first).  Backward: of all higher
-// threads (the last thread applied first).
+// threads (the last thread applied first).  Two levels of warp scans: the
+// warps' aggregates are scanned by warp 0, not walked one by one.
 __device__ inline Aff block_excl_scan_fwd(const Aff& v, Aff* wt) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const Aff inc = warp_scan_fwd(v, lane);
     Aff ex = shfl_up_aff(inc, 1);
     if (lane == 0) ex = aff_id();
     __syncthreads();
     if (lane == 31) wt[w] = inc;
     __syncthreads();
-    Aff pre = aff_id();
-    for (int u = 0; u < w; ++u) pre = aff_then(pre, wt[u]);
-    return aff_then(pre, ex);
+    if (w == 0) {
+        const Aff a = lane < nw ? wt[lane] : aff_id();
+        const Aff sc = warp_scan_fwd(a, lane);
+        Aff e = shfl_up_aff(sc, 1);
+        if (lane == 0) e = aff_id();
+        if (lane < nw) wt[lane] = e;
+    }
+    __syncthreads();
+    return aff_then(wt[w], ex);
 }
 __device__ inline Aff block_excl_scan_bwd(const Aff& v, Aff* wt) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -209,9 +216,17 @@ __device__ inline Aff block_excl_scan_bwd(const Aff& v, Aff* wt) {
     __syncthreads();
     if (lane == 0) wt[w] = inc;
     __syncthreads();
-    Aff suf = aff_id();
-    for (int u = nw - 1; u > w; --u) suf = aff_then(suf, wt[u]);
-    return aff_then(suf, ex);
+    if (w == 0) {
+        // aggregates of warps lane..nw-1, the last applied first; lanes past
+        // nw hold the identity
+        const Aff a = lane < nw ? wt[lane] : aff_id();
+        const Aff sc = warp_scan_bwd(a, lane);
+        Aff e = shfl_down_aff(sc, 1);
+        if (lane == 31) e = aff_id();
+        if (lane < nw) wt[lane] = e;
+    }
+    __syncthreads();
+    return aff_then(wt[w], ex);
 }
 // Block-wide exclusive suffix sum of a count (sum over higher threads).
 __device__ inline long long block_excl_suffix_ll(long long v, long long* wt) {
@@ -225,9 +240,19 @@ __device__ inline long long block_excl_suffix_ll(long long v, long long* wt) {
     __syncthreads();
     if (lane == 0) wt[w] = inc;
     __syncthreads();
-    long long s = inc - v;
-    for (int u = w + 1; u < nw; ++u) s += wt[u];
-    return s;
+    if (w == 0) {  // suffix sums of the warps' totals, exclusive
+        long long a = lane < nw ? wt[lane] : 0ll;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const long long o = __shfl_down_sync(0xffffffffu, a, d);
+            if (lane + d < 32) a += o;
+        }
+        const long long own = lane < nw ? wt[lane] : 0ll;
+        __syncwarp();
+        if (lane < nw) wt[lane] = a - own;
+    }
+    __syncthreads();
+    return inc - v + wt[w];
 }
 
 // ---------------------------------------------------------------------------

@@ -177,16 +177,28 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
     Aff eb = shfl_down_aff(inc_b, 1);
     if (lane == 0) ef = aff_id();
     if (lane == 31) eb = aff_id();
-    if (lane == 31) sm->wf[warp] = inc_f;
-    if (lane == 0) sm->wb[warp] = inc_b;
-    team_sync<WARP>();
-    {
-        Aff pre = aff_id();
-        for (int w = 0; w < warp; ++w) pre = aff_then(pre, sm->wf[w]);
-        ef = aff_then(pre, ef);
-        Aff suf = aff_id();
-        for (int w = nwarps - 1; w > warp; --w) suf = aff_then(suf, sm->wb[w]);
-        eb = aff_then(suf, eb);
+    if (!WARP && nwarps > 1) {
+        // the warps' aggregates, scanned by warp 0 (both directions)
+        if (lane == 31) sm->wf[warp] = inc_f;
+        if (lane == 0) sm->wb[warp] = inc_b;
+        team_sync<WARP>();
+        if (warp == 0) {
+            const Aff a = lane < nwarps ? sm->wf[lane] : aff_id();
+            const Aff c = lane < nwarps ? sm->wb[lane] : aff_id();
+            const Aff sa = warp_scan_fwd(a, lane);
+            const Aff sc = warp_scan_bwd(c, lane);
+            Aff ea = shfl_up_aff(sa, 1);
+            Aff ec = shfl_down_aff(sc, 1);
+            if (lane == 0) ea = aff_id();
+            if (lane == 31) ec = aff_id();
+            if (lane < nwarps) {
+                sm->wf[lane] = ea;
+                sm->wb[lane] = ec;
+            }
+        }
+        team_sync<WARP>();
+        ef = aff_then(sm->wf[warp], ef);
+        eb = aff_then(sm->wb[warp], eb);
     }
     const double P_before = fma(ef.a, P_start, ef.c);  // P_{lo-1}
     const double Q_after = fma(eb.a, Q_end, eb.c);     // Q_hi
