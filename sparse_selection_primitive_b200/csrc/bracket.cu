@@ -183,8 +183,14 @@ __device__ void select_two_ranks(const uint32_t* keys, int m, const uint32_t* hi
     // case for a small budget) one warp sorts them all and reads both ranks off.
     const uint32_t low = wb ? pb : pa;
     const uint32_t ncand = wb ? xb + hist1[pb] : xa + hist1[pa];
-    if (ncand <= (uint32_t)kWarpSortMax) {
-        uint32_t* cand = h2;
+    // A long sample whose candidates fit one block-wide sort (two keys per
+    // thread): the sort takes less time than two radix levels, each a pass
+    // over all m keys.
+    const bool warp_sort = ncand <= (uint32_t)kWarpSortMax;
+    const bool block_sort = !warp_sort && ncand <= 2u * kBlk && m >= 8 * kBlk;
+    if (warp_sort || block_sort) {
+        const uint32_t cap = warp_sort ? (uint32_t)kWarpSortMax : 2u * kBlk;
+        uint32_t* cand = h2;  // cap words; the block sort exchanges through h2 + 2 kBlk
         if (threadIdx.x == 0) bcast[0] = 0u;
         __syncthreads();
         for (int s0 = 0; s0 < m; s0 += blockDim.x) {  // same trip count in every lane
@@ -197,10 +203,25 @@ __device__ void select_two_ranks(const uint32_t* keys, int m, const uint32_t* hi
             uint32_t base = 0;
             if (lane == leader) base = atomicAdd(&bcast[0], (uint32_t)__popc(ball));
             base = __shfl_sync(0xffffffffu, base, leader);
-            if (take) cand[base + __popc(ball & ((1u << lane) - 1u))] = k;
+            const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+            if (take && pos < cap) cand[pos] = k;
         }
         __syncthreads();
-        if (threadIdx.x < 32) {
+        if (block_sort) {
+            uint32_t key[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const uint32_t j = threadIdx.x * 2 + e;
+                key[e] = j < ncand ? cand[j] : 0u;  // padding sorts first
+            }
+            bitonic_sort_row<2, kBlk, kBlk>(key, threadIdx.x, h2 + 2 * kBlk);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int j = threadIdx.x * 2 + e;
+                if (wa && j == 2 * kBlk - ra) bcast[2] = key[e];
+                if (wb && j == 2 * kBlk - rb) bcast[3] = key[e];
+            }
+        } else if (threadIdx.x < 32) {
             constexpr int E = kWarpSortMax / 32;
             uint32_t key[E];
 #pragma unroll
@@ -236,15 +257,10 @@ __device__ void select_two_ranks(const uint32_t* keys, int m, const uint32_t* hi
             const uint32_t k = s < m ? keys[s] : 0u;
             const bool ina = s < m && wa && (k >> psh) == pa;
             const bool inb = s < m && wb && (k >> psh) == pb;
-            if (!__any_sync(0xffffffffu, ina || inb)) continue;
-            // lanes with the same digit add once (ties crowd into one bin)
-            const uint32_t da = ina ? ((k >> sh) & dmask) : 0xffffffffu;
-            const unsigned peers_a = __match_any_sync(0xffffffffu, da);
-            if (ina && lane == __ffs(peers_a) - 1) atomicAdd(&h2[da], (uint32_t)__popc(peers_a));
-            const uint32_t db = inb ? ((k >> sh) & dmask) : 0xffffffffu;
-            const unsigned peers_b = __match_any_sync(0xffffffffu, db);
-            if (inb && lane == __ffs(peers_b) - 1)
-                atomicAdd(&h2[2048 + db], (uint32_t)__popc(peers_b));
+            // (the digits below the prefix spread over the bins, so plain
+            // shared-memory atomics rarely collide)
+            if (ina) atomicAdd(&h2[(k >> sh) & dmask], 1u);
+            if (inb) atomicAdd(&h2[2048 + ((k >> sh) & dmask)], 1u);
         }
         __syncthreads();
         uint32_t ba, bb;
@@ -657,17 +673,28 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
                 push_staged(m);
             }
         }
-        // Remainder: the last partial trip, with bounds checks.
+        // Remainder: the last partial trip (at most U vectors per thread, a
+        // grid-uniform count), its loads issued together, with bounds checks.
         const int64_t rem_iters = (n4 - full * step + nthreads - 1) / nthreads;
-        for (int64_t it = 0; it < rem_iters; ++it) {
-            const int64_t i = full * step + it * nthreads + gtid;
-            const bool ok = i < n4;
-            const float4 v = ok ? __ldcs(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float xs[4] = {v.x, v.y, v.z, v.w};
-            uint32_t m = 0u;
+        {
+            float4 rv[U];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) classify(xs[j], ok, m, j);
-            if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 4);
+            for (int qq = 0; qq < U; ++qq) {
+                const int64_t i = full * step + (int64_t)qq * nthreads + gtid;
+                rv[qq] = (qq < rem_iters && i < n4) ? __ldcs(r4 + i)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int qq = 0; qq < U; ++qq) {
+                if (qq >= rem_iters) break;
+                const int64_t i = full * step + (int64_t)qq * nthreads + gtid;
+                const bool ok = i < n4;
+                const float xs[4] = {rv[qq].x, rv[qq].y, rv[qq].z, rv[qq].w};
+                uint32_t m = 0u;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) classify(xs[j], ok, m, j);
+                if (__any_sync(0xffffffffu, m != 0u)) push(xs, m, 4);
+            }
         }
         // tail elements (n not a multiple of 4)
         const int64_t rem0 = n4 << 2;
@@ -1293,26 +1320,34 @@ __device__ int plan_with_bins(const unsigned long long* __restrict__ bins, const
 // solve sorts it).  Four 16-byte loads per thread in flight per trip; every
 // score takes one exponential (masked inside the band).  Sets *bad when a
 // score is NaN or infinite.
-__device__ void refold_row(const float* __restrict__ r, int64_t n, int vec, float aL, float aR,
+__device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, int vec, float aL, float aR,
                            double t, float* band, SolveSmemAll* sm, Tails& tl, long long* nb,
                            bool* bad) {
     const float k2 = (float)(kLog2e / t);
+    const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) sm->cnt = 0ull;
     __syncthreads();
     double SL = 0.0, SR = 0.0;
     uint32_t cR = 0u;
     float probe = 0.f;  // NaN once a score is NaN or infinite
-    auto one = [&](float x, float& sl, float& sr) {
-        const bool right = x >= aR, left = x < aL;
-        const bool inb = x >= aL && x < aR;
+    // One score (ok = in range).  Every lane of the warp calls it together:
+    // the band scores of the warp take their slots with one atomic.
+    auto one = [&](float x, bool ok, float& sl, float& sr) {
+        const bool right = ok && x >= aR, left = ok && x < aL;
+        const bool inb = ok && x >= aL && x < aR;
         const float e = ex2_ftz((right ? aR - x : (left ? x - aL : 0.f)) * k2);
         sr += right ? e : 0.f;
         sl += left ? e : 0.f;
         cR += right ? 1u : 0u;
-        probe = fmaf(x, 0.f, probe);
-        if (inb) {  // rare
-            const unsigned long long pos = atomicAdd(&sm->cnt, 1ull);
-            if (pos < (unsigned long long)n) band[pos] = x;
+        if (ok) probe = fmaf(x, 0.f, probe);
+        const unsigned ball = __ballot_sync(0xffffffffu, inb);
+        if (ball != 0u) {
+            const int leader = __ffs(ball) - 1;
+            unsigned long long base = 0ull;
+            if (lane == leader) base = atomicAdd(&sm->cnt, (unsigned long long)__popc(ball));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            const unsigned long long pos = base + __popc(ball & ((1u << lane) - 1u));
+            if (inb && pos < (unsigned long long)n) band[pos] = x;
         }
     };
     if (vec) {
@@ -1320,35 +1355,39 @@ __device__ void refold_row(const float* __restrict__ r, int64_t n, int vec, floa
         const float4* r4 = reinterpret_cast<const float4*>(r);
         constexpr int U = 4;
         const int64_t per_trip = (int64_t)U * blockDim.x;
-        for (int64_t i0 = 0; i0 < n4; i0 += per_trip) {
+        for (int64_t i0 = 0; i0 < n4; i0 += per_trip) {  // same trip count in every lane
             float4 v[U];
 #pragma unroll
             for (int q = 0; q < U; ++q) {
                 const int64_t i = i0 + (int64_t)q * blockDim.x + threadIdx.x;
-                v[q] = i < n4 ? __ldcg(r4 + i) : make_float4(NAN, NAN, NAN, NAN);
+                v[q] = i < n4 ? __ldcg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
             float sl = 0.f, sr = 0.f;
 #pragma unroll
             for (int q = 0; q < U; ++q) {
-                if (i0 + (int64_t)q * blockDim.x + threadIdx.x >= n4) continue;
-                one(v[q].x, sl, sr);
-                one(v[q].y, sl, sr);
-                one(v[q].z, sl, sr);
-                one(v[q].w, sl, sr);
+                const bool ok = i0 + (int64_t)q * blockDim.x + threadIdx.x < n4;
+                one(v[q].x, ok, sl, sr);
+                one(v[q].y, ok, sl, sr);
+                one(v[q].z, ok, sl, sr);
+                one(v[q].w, ok, sl, sr);
             }
             SL += (double)sl;
             SR += (double)sr;
         }
-        for (int64_t i = (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) {
+        if (threadIdx.x < 32) {  // the last n mod 4 scores, by warp 0
+            const int64_t i = (n4 << 2) + threadIdx.x;
+            const bool ok = i < n;
             float sl = 0.f, sr = 0.f;
-            one(r[i], sl, sr);
+            one(ok ? r[i] : 0.f, ok, sl, sr);
             SL += (double)sl;
             SR += (double)sr;
         }
     } else {
-        for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+        for (int64_t i0 = 0; i0 < n; i0 += blockDim.x) {  // same trip count in every lane
+            const int64_t i = i0 + threadIdx.x;
+            const bool ok = i < n;
             float sl = 0.f, sr = 0.f;
-            one(r[i], sl, sr);
+            one(ok ? r[i] : 0.f, ok, sl, sr);
             SL += (double)sl;
             SR += (double)sr;
         }
@@ -1576,21 +1615,33 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
         reinterpret_cast<uint32_t*>(st)[i] = 0u;
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) rb->hist1[i] = 0u;
     __syncthreads();
+    phase_mark(st, 14);
     // 1. the sample, as keys, with its level-1 histogram
     const uint64_t c0 = (uint64_t)row << 32;
-    for (int s0 = 0; s0 < m; s0 += blockDim.x) {  // same trip count in every lane
-        const int s = s0 + threadIdx.x;
-        uint32_t bn = 0xffffffffu;
-        if (s < m) {
-            const uint32_t key = to_key(draw_sample(rr, n, t, seed, c0, s));
-            keys[s] = key;
-            bn = key >> 21;
+    constexpr int kDraws = 4;  // samples per thread with their gathers in flight together
+    for (int s0 = 0; s0 < m; s0 += kDraws * blockDim.x) {  // same trip count in every lane
+        float y[kDraws];
+#pragma unroll
+        for (int u = 0; u < kDraws; ++u) {
+            const int s = s0 + u * blockDim.x + threadIdx.x;
+            y[u] = s < m ? draw_sample(rr, n, t, seed, c0, s) : 0.f;
         }
-        const unsigned peers = __match_any_sync(0xffffffffu, bn);
-        if (bn != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
-            atomicAdd(&rb->hist1[bn], (uint32_t)__popc(peers));
+#pragma unroll
+        for (int u = 0; u < kDraws; ++u) {
+            const int s = s0 + u * blockDim.x + threadIdx.x;
+            uint32_t bn = 0xffffffffu;
+            if (s < m) {
+                const uint32_t key = to_key(y[u]);
+                keys[s] = key;
+                bn = key >> 21;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, bn);
+            if (bn != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
+                atomicAdd(&rb->hist1[bn], (uint32_t)__popc(peers));
+        }
     }
     __syncthreads();
+    phase_mark(st, 15);
     // 2. the bracket's order statistics
     float aR = INFINITY, aL = -INFINITY;
     {
@@ -1601,6 +1652,7 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
         if (ra >= 1) aR = from_key(ka);
         if (rbk >= 1) aL = from_key(kb);
     }
+    phase_mark(st, 0);
     if (force_miss) {
         // a bracket above every sample value: F(a_L) < k, so it must fail
         uint32_t kmax = 0u;
@@ -1632,6 +1684,7 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
     long long nb = 0;
     bool bad = false;
     refold_row(rr, n, vec, aL, aR, t, band0, sm, tl, &nb, &bad);
+    phase_mark(st, 16);
     if (bad) {
         if (threadIdx.x == 0) {
             st->status |= kDevNonFinite;

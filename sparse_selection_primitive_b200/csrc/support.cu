@@ -92,10 +92,12 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     double s = 0.0, sv = 0.0;
     const uint64_t keep = l2_evict_last_policy();
     // count of share i of group gi: (tile gi * group + i / 8, share i % 8), or 0
+    // (the buffer holds a list for this (n, B) whatever it was written for,
+    // so the counts load without waiting for the match test)
     auto share_count = [&](int64_t gi) -> uint32_t {
         const int64_t t0 = gi * group;
         const int64_t t1 = t0 + group < tiles ? t0 + group : tiles;
-        if (!match || gi >= ngroups || t0 + (int64_t)threadIdx.x / kShares >= t1) return 0u;
+        if (gi >= ngroups || t0 + (int64_t)threadIdx.x / kShares >= t1) return 0u;
         return __ldcs(sup.cnt + (row * tiles + t0) * kShares + threadIdx.x);
     };
     // persistent over groups of tiles; the next group's counts load while
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     uint32_t c_next = share_count(blockIdx.x);
     for (int64_t gi = blockIdx.x; gi < ngroups; gi += nblk) {
         const int64_t t0 = gi * group;
-        uint32_t c = c_next;
+        uint32_t c = match ? c_next : 0u;
         if (c > (uint32_t)kSupCap) {
             bad = 1;
             c = 0;

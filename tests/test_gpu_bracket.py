@@ -33,10 +33,22 @@ def _forward(r, k, t, flags=0, seed=0):
     return ws, p.cpu().numpy()[0].astype(np.float64), b.item()
 
 
-@pytest.mark.parametrize("n,k,t,seed", [(200000, 150.0, 0.01, 0), (1 << 20, 1000.0, 0.005, 7),
-                                        (50000, 25000.0, 0.3, 3)])
-def test_sample_and_bracket_match_oracle(cuda_device, n, k, t, seed):
-    r, _ = random_rows(seed, 1, n, "mix_nu")
+# The order statistics come from one of three selections, by the number of
+# sample keys in the wanted top-11-bit bins and above: one warp sorts them
+# (a few, e.g. normal scores and a small budget), the whole block sorts them
+# (up to 2048 of a 32768-key sample, e.g. the uniform half of mix_nu near its
+# edge), or two radix levels narrow them (a dense top bin: uniform(3, 4)
+# puts half the sample in [3.5, 4); or a short sample).
+@pytest.mark.parametrize("n,k,t,seed,dist", [(200000, 150.0, 0.01, 0, "mix_nu"),
+                                             (1 << 20, 1000.0, 0.005, 7, "mix_nu"),
+                                             (50000, 25000.0, 0.3, 3, "mix_nu"),
+                                             (1 << 20, 100.0, 0.01, 5, "normal"),
+                                             (1 << 20, 2000.0, 0.002, 9, "uniform34")])
+def test_sample_and_bracket_match_oracle(cuda_device, n, k, t, seed, dist):
+    if dist == "uniform34":
+        r = np.random.default_rng(seed).uniform(3.0, 4.0, (1, n)).astype(np.float32)
+    else:
+        r, _ = random_rows(seed, 1, n, dist)
     ws, _, _ = _forward(r[0], k, t, seed=seed)
     info = L.row_info(ws, 0)
     m = info["sample_m"]
