@@ -138,7 +138,6 @@ __device__ __forceinline__ double gap_factor(float lo, float hi, double inv_t) {
 // routine is fetched once and then stays hot.
 static __device__ __noinline__ double cold_exp(double x) { return exp(x); }
 static __device__ __noinline__ double cold_log(double x) { return log(x); }
-static __device__ __noinline__ double cold_log1p(double x) { return log1p(x); }
 __device__ __forceinline__ double gap_factor_cold(float lo, float hi, double inv_t) {
     return cold_exp(((double)lo - (double)hi) * inv_t);
 }
@@ -271,36 +270,51 @@ __device__ inline long long block_excl_suffix_ll(long long v, long long* wt) {
 // A missing anchor (no scores on that side, weight 0) leaves a single
 // exponential:  Bh = 0: b = sR + t ln(2c/Ah);  Ah = 0: b = sL + t ln(Bh/(-2c)).
 // The result is clamped into [sL, sR].
+//
+// With rho = Ah Bh delta / c^2 the larger magnitude |c| + S is |c| (1 + sqrt(1
+// + rho)), or sqrt(Ah Bh delta) (sqrt(1/rho) + sqrt(1 + 1/rho)) when rho > 1,
+// so that ln(|c| + S) costs one exponential and one logarithm after ln Ah,
+// ln Bh and ln |c|, and ln(S - c) for c < 0 is ln(Ah Bh delta) - ln(|c| + S).
+// Every lane of one warp calls it with the same arguments: lanes 0, 1 and 2
+// take the three first logarithms at once, and all lanes return b.
 // ---------------------------------------------------------------------------
-static __device__ __noinline__ double segment_root(bool hasL, double sL, double Bh, bool hasR, double sR,
-                                      double Ah, double c, double t) {
+static __device__ __noinline__ double segment_root(bool hasL, double sL, double Bh, bool hasR,
+                                                   double sR, double Ah, double c, double t) {
+    const int lane = threadIdx.x & 31;
     hasL = hasL && Bh > 0.0;
     hasR = hasR && Ah > 0.0;
-    double b;
     if (!hasL && !hasR) return nan("");
-    if (!hasL) {
-        b = sR + t * cold_log(2.0 * c / Ah);
-    } else if (!hasR) {
-        b = sL + t * cold_log(Bh / (-2.0 * c));
+    double arg = 1.0;
+    if (!hasL) arg = 2.0 * c / Ah;
+    else if (!hasR) arg = Bh / (-2.0 * c);
+    else arg = lane == 0 ? Ah : (lane == 1 ? Bh : fabs(c));
+    if (lane > 2) arg = 1.0;
+    const double lg = cold_log(arg);
+    const double l0 = __shfl_sync(0xffffffffu, lg, 0);
+    if (!hasL) return sR + t * l0;
+    if (!hasR) return sL + t * l0;
+    const double l1 = __shfl_sync(0xffffffffu, lg, 1);
+    const double l2 = __shfl_sync(0xffffffffu, lg, 2);
+    const double lnd = (sL - sR) / t, lnA = l0, lnB = l1;
+    double ln_y;
+    if (c == 0.0) {
+        ln_y = 0.5 * (lnB + lnd - lnA);
     } else {
-        double lnd = (sL - sR) / t;
-        double lnA = cold_log(Ah), lnB = cold_log(Bh);
-        double ln_y;
-        if (c == 0.0) {
-            ln_y = 0.5 * (lnB + lnd - lnA);
+        const double lnc = l2;
+        const double lnrho = lnA + lnB + lnd - 2.0 * lnc;
+        double L;  // ln(|c| + S)
+        if (lnrho <= 0.0) {
+            const double rho = cold_exp(lnrho);
+            L = lnc + cold_log(1.0 + sqrt(1.0 + rho));
         } else {
-            double lnc = cold_log(fabs(c));
-            double lnrho = lnA + lnB + lnd - 2.0 * lnc;  // rho = Ah Bh delta / c^2
-            double lnS = lnrho > 0.0 ? 0.5 * (lnA + lnB + lnd) + 0.5 * cold_log1p(cold_exp(-lnrho))
-                                     : lnc + 0.5 * cold_log1p(cold_exp(lnrho));
-            double rc = cold_exp(lnc - lnS);                   // |c| / S <= 1
-            if (c > 0.0) ln_y = lnS + cold_log1p(rc) - lnA;     // ln(c + S) - ln Ah
-            else ln_y = lnB + lnd - (lnS + cold_log1p(rc));    // ln Bh + ln delta - ln(S - c)
+            const double sg = cold_exp(-lnrho);
+            L = 0.5 * (lnA + lnB + lnd) + cold_log(sqrt(sg) + sqrt(1.0 + sg));
         }
-        b = sR + t * ln_y;
-        if (b < sL) b = sL;
-        if (b > sR) b = sR;
+        ln_y = c > 0.0 ? L - lnA : lnB + lnd - L;
     }
+    double b = sR + t * ln_y;
+    if (b < sL) b = sL;
+    if (b > sR) b = sR;
     return b;
 }
 

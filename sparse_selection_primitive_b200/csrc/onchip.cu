@@ -133,6 +133,14 @@ __device__ __forceinline__ float row_min_f(float v, float* red) {
     }
 }
 
+// Barrier over the threads of one row: a row held by one warp needs only the
+// warp's own barrier, so the rows of a CTA run their steps independently.
+template <int E, int RT, int CTA>
+__device__ __forceinline__ void row_sync() {
+    if constexpr (Shape<E, RT, CTA>::WPR == 1) __syncwarp();
+    else __syncthreads();
+}
+
 template <int E, int RT, int CTA>
 __global__ void __launch_bounds__(CTA, 3 * 256 / CTA > 0 ? 3 * 256 / CTA : 1) onchip_forward_kernel(
     const float* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
@@ -157,7 +165,7 @@ __global__ void __launch_bounds__(CTA, 3 * 256 / CTA > 0 ? 3 * 256 / CTA : 1) on
     const float* rrow = r + (row_ok ? row : 0) * ld;
     const double inv_t = 1.0 / t;
 
-    if (threadIdx.x < S::ROWS) row_flag[threadIdx.x] = 0;
+    if (tid == 0) row_flag[rloc] = 0;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         hdr->last_B = B;
         hdr->last_n = n;
@@ -174,7 +182,7 @@ __global__ void __launch_bounds__(CTA, 3 * 256 / CTA > 0 ? 3 * 256 / CTA : 1) on
         key[e] = valid[e] ? to_key(orig[e]) : kPadKey;
         bad |= valid[e] && !finite_f(orig[e]);
     }
-    __syncthreads();
+    row_sync<E, RT, CTA>();
     if (bad) atomicOr(&row_flag[rloc], 1);
 
     bitonic_sort_row<E, RT, CTA>(key, tid, xch);
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(CTA, 3 * 256 / CTA > 0 ? 3 * 256 / CTA : 1) on
 #pragma unroll
     for (int e = 0; e < E; ++e) s[e] = from_key(key[e]);
     last_key[threadIdx.x] = key[E - 1];
-    __syncthreads();
+    row_sync<E, RT, CTA>();
     const float s_prev = (tid > 0) ? from_key(last_key[threadIdx.x - 1]) : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -194,7 +202,7 @@ __global__ void __launch_bounds__(CTA, 3 * 256 / CTA > 0 ? 3 * 256 / CTA : 1) on
         g[e] = (j >= 1 && j < n) ? gap_factor(sp, s[e], inv_t) : 0.0;
     }
     first_gap[threadIdx.x] = g[0];
-    __syncthreads();
+    row_sync<E, RT, CTA>();
     const double g_next = (tid + 1 < RT) ? first_gap[threadIdx.x + 1] : 0.0;
 
     // Thread aggregates of the forward (prefix) and backward (suffix) maps.
@@ -266,22 +274,24 @@ __global__ void __launch_bounds__(CTA, 3 * 256 / CTA > 0 ? 3 * 256 / CTA : 1) on
             anchor[rloc][3] = Q[e];
         }
     }
-    __syncthreads();
-    if (tid == 0) {
+    row_sync<E, RT, CTA>();
+    if (tid < 32) {  // the row's first warp takes the root together
         double bb;
         if (row_flag[rloc] || !row_ok) {
             bb = nan("");
-            if (row_ok) set_status(hdr, kDevNonFinite);
+            if (row_ok && tid == 0) set_status(hdr, kDevNonFinite);
         } else {
             const bool hasL = jstar >= 1, hasR = jstar < n;
             bb = segment_root(hasL, anchor[rloc][0], hasL ? anchor[rloc][1] : 0.0, hasR,
                               anchor[rloc][2], hasR ? anchor[rloc][3] : 0.0,
                               (double)(n - jstar) - k, t);
         }
-        row_b[rloc] = bb;
-        if (row_ok) b_out[row] = bb;
+        if (tid == 0) {
+            row_b[rloc] = bb;
+            if (row_ok) b_out[row] = bb;
+        }
     }
-    __syncthreads();
+    row_sync<E, RT, CTA>();
 
     // Emit p_i = sigma((r_i - b)/t) in the original order, and sum f.
     const Thr th = make_thr(row_b[rloc], t);

@@ -147,12 +147,19 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
     const double Q_end = tl.hasR ? tl.SR : 0.0;
 
     if (nb == 0) {
-        if (tid == 0) {
-            out->jstar = 0;
-            out->b = segment_root(tl.hasL, tl.aL, tl.SL, tl.hasR, tl.aR, tl.SR, tl.cntR - k, t);
-            const double lnw = (tl.hasL && tl.hasR) ? ((double)tl.aL - (double)tl.aR) / t : -INFINITY;
-            out->F_aL = tl.hasL ? tl.cntR - 0.5 * tl.SR * cold_exp(lnw) + 0.5 * tl.SL : INFINITY;
-            out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * tl.SL * cold_exp(lnw) : -INFINITY;
+        if (tid < 32) {  // one warp takes the root
+            const double b = segment_root(tl.hasL, tl.aL, tl.SL, tl.hasR, tl.aR, tl.SR,
+                                          tl.cntR - k, t);
+            if (tid == 0) {
+                out->jstar = 0;
+                out->b = b;
+                const double lnw =
+                    (tl.hasL && tl.hasR) ? ((double)tl.aL - (double)tl.aR) / t : -INFINITY;
+                out->F_aL = tl.hasL ? tl.cntR - 0.5 * tl.SR * cold_exp(lnw) + 0.5 * tl.SL
+                                    : INFINITY;
+                out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * tl.SL * cold_exp(lnw)
+                                    : -INFINITY;
+            }
         }
         team_sync<WARP>();
         return;
@@ -229,7 +236,7 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
         }
     }
     team_sync<WARP>();
-    if (tid == 0) {
+    if (tid < 32) {  // one warp takes the root; lane 0 writes the result
         double b;
         long long js;
         if (count == 0) {
@@ -244,12 +251,17 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
             b = segment_root(true, get(js - 1), sm->d[4], hasR, sR, Ah,
                              tl.cntR + (double)(nb - js) - k, t);
         }
-        out->b = b;
-        out->jstar = js;
-        const double Q0 = sm->d[0], Pl = sm->d[1];
-        out->F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * gap(0) * Q0 + 0.5 * tl.SL
-                            : INFINITY;
-        out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * gap(nb) * Pl : -INFINITY;
+        // the end gap factors, one lane each
+        const double g_end = lane == 1 ? gap(nb) : (lane == 0 ? gap(0) : 0.0);
+        const double g_nb = __shfl_sync(0xffffffffu, g_end, 1);
+        if (lane == 0) {
+            out->b = b;
+            out->jstar = js;
+            const double Q0 = sm->d[0], Pl = sm->d[1];
+            out->F_aL = tl.hasL ? tl.cntR + (double)nb - 0.5 * g_end * Q0 + 0.5 * tl.SL
+                                : INFINITY;
+            out->F_aR = tl.hasR ? tl.cntR - 0.5 * tl.SR + 0.5 * g_nb * Pl : -INFINITY;
+        }
     }
     team_sync<WARP>();
 }
