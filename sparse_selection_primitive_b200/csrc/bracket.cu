@@ -1315,7 +1315,7 @@ __device__ int plan_with_bins(const unsigned long long* __restrict__ bins, const
     return 1;
 }
 
-// Single-CTA fold of one row: the tail sums and right count of [aL, aR), the
+// Single-CTA fold (kBlk threads) of one row: the tail sums and right count of [aL, aR), the
 // band scores appended to `band` (capacity n; order depends on timing, the
 // solve sorts it).  Four 16-byte loads per thread in flight per trip; every
 // score takes one exponential (masked inside the band).  Sets *bad when a
@@ -1352,20 +1352,19 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
     };
     if (vec) {
         const int64_t n4 = n >> 2;
-        const float4* r4 = reinterpret_cast<const float4*>(r);
         constexpr int U = 4;
-        const int64_t per_trip = (int64_t)U * blockDim.x;
-        for (int64_t i0 = 0; i0 < n4; i0 += per_trip) {  // same trip count in every lane
+        constexpr int64_t per_trip = (int64_t)U * kBlk;
+        const float4* p4 = reinterpret_cast<const float4*>(r) + threadIdx.x;
+        for (int64_t i0 = 0; i0 < n4; i0 += per_trip, p4 += per_trip) {  // same trip count in every lane
+            const int64_t rem = n4 - i0 - (int64_t)threadIdx.x;  // this thread's vectors left
             float4 v[U];
 #pragma unroll
-            for (int q = 0; q < U; ++q) {
-                const int64_t i = i0 + (int64_t)q * blockDim.x + threadIdx.x;
-                v[q] = i < n4 ? __ldcg(r4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            for (int q = 0; q < U; ++q)
+                v[q] = (int64_t)q * kBlk < rem ? __ldcg(p4 + q * kBlk) : make_float4(0.f, 0.f, 0.f, 0.f);
             float sl = 0.f, sr = 0.f;
 #pragma unroll
             for (int q = 0; q < U; ++q) {
-                const bool ok = i0 + (int64_t)q * blockDim.x + threadIdx.x < n4;
+                const bool ok = (int64_t)q * kBlk < rem;
                 one(v[q].x, ok, sl, sr);
                 one(v[q].y, ok, sl, sr);
                 one(v[q].z, ok, sl, sr);
@@ -1383,7 +1382,7 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
             SR += (double)sr;
         }
     } else {
-        for (int64_t i0 = 0; i0 < n; i0 += blockDim.x) {  // same trip count in every lane
+        for (int64_t i0 = 0; i0 < n; i0 += kBlk) {  // same trip count in every lane
             const int64_t i = i0 + threadIdx.x;
             const bool ok = i < n;
             float sl = 0.f, sr = 0.f;

@@ -142,7 +142,7 @@ __device__ __forceinline__ void row_sync() {
 }
 
 template <int E, int RT, int CTA>
-__global__ void __launch_bounds__(CTA, 3 * 256 / CTA > 0 ? 3 * 256 / CTA : 1) onchip_forward_kernel(
+__global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel(
     const float* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
     double* __restrict__ sumf_out, int64_t B, int n, double k, double t, WsHeader* hdr, int vec) {
     using S = Shape<E, RT, CTA>;
