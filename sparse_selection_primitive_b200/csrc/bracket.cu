@@ -1330,24 +1330,39 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
     double SL = 0.0, SR = 0.0;
     uint32_t cR = 0u;
     float probe = 0.f;  // NaN once a score is NaN or infinite
-    // One score (ok = in range).  Every lane of the warp calls it together:
-    // the band scores of the warp take their slots with one atomic.
-    auto one = [&](float x, bool ok, float& sl, float& sr) {
+    // One score (ok = in range): the tail terms; returns whether it is in the band.
+    auto fold1 = [&](float x, bool ok, float& sl, float& sr) -> bool {
         const bool right = ok && x >= aR, left = ok && x < aL;
-        const bool inb = ok && x >= aL && x < aR;
         const float e = ex2_ftz((right ? aR - x : (left ? x - aL : 0.f)) * k2);
         sr += right ? e : 0.f;
         sl += left ? e : 0.f;
         cR += right ? 1u : 0u;
         if (ok) probe = fmaf(x, 0.f, probe);
-        const unsigned ball = __ballot_sync(0xffffffffu, inb);
+        return ok && !right && !left;
+    };
+    // Band scores are staged per warp (128 slots of the sort's exchange
+    // buffer, free during the fold) and moved to the band with one atomic per
+    // 96 or more, so the warps do not queue on one shared counter.
+    constexpr uint32_t kWarpStage = 128;
+    float* stg = reinterpret_cast<float*>(sm->u.sort.xch) + (threadIdx.x >> 5) * kWarpStage;
+    uint32_t wc = 0u;  // warp-uniform: scores staged
+    auto flush = [&]() {
+        unsigned long long base = 0ull;
+        if (lane == 0 && wc != 0u) base = atomicAdd(&sm->cnt, (unsigned long long)wc);
+        base = __shfl_sync(0xffffffffu, base, 0);
+        __syncwarp();
+        for (uint32_t i = lane; i < wc; i += 32)
+            if (base + i < (unsigned long long)n) band[base + i] = stg[i];
+        __syncwarp();
+        wc = 0u;
+    };
+    // Every lane of the warp calls it together.
+    auto append = [&](bool take, float x) {
+        const unsigned ball = __ballot_sync(0xffffffffu, take);
         if (ball != 0u) {
-            const int leader = __ffs(ball) - 1;
-            unsigned long long base = 0ull;
-            if (lane == leader) base = atomicAdd(&sm->cnt, (unsigned long long)__popc(ball));
-            base = __shfl_sync(0xffffffffu, base, leader);
-            const unsigned long long pos = base + __popc(ball & ((1u << lane) - 1u));
-            if (inb && pos < (unsigned long long)n) band[pos] = x;
+            if (take) stg[wc + __popc(ball & ((1u << lane) - 1u))] = x;
+            wc += (uint32_t)__popc(ball);
+            if (wc > kWarpStage - 32u) flush();
         }
     };
     if (vec) {
@@ -1361,23 +1376,36 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
 #pragma unroll
             for (int q = 0; q < U; ++q)
                 v[q] = (int64_t)q * kBlk < rem ? __ldcg(p4 + q * kBlk) : make_float4(0.f, 0.f, 0.f, 0.f);
+            // the tails first, with the trip's band scores marked in bm (bit 4q + c);
+            // the appends stay off this path, so it holds no more than the loads
             float sl = 0.f, sr = 0.f;
+            uint32_t bm = 0u;
 #pragma unroll
             for (int q = 0; q < U; ++q) {
                 const bool ok = (int64_t)q * kBlk < rem;
-                one(v[q].x, ok, sl, sr);
-                one(v[q].y, ok, sl, sr);
-                one(v[q].z, ok, sl, sr);
-                one(v[q].w, ok, sl, sr);
+                bm |= (uint32_t)fold1(v[q].x, ok, sl, sr) << (4 * q);
+                bm |= (uint32_t)fold1(v[q].y, ok, sl, sr) << (4 * q + 1);
+                bm |= (uint32_t)fold1(v[q].z, ok, sl, sr) << (4 * q + 2);
+                bm |= (uint32_t)fold1(v[q].w, ok, sl, sr) << (4 * q + 3);
             }
             SL += (double)sl;
             SR += (double)sr;
+            if (__any_sync(0xffffffffu, bm != 0u)) {
+#pragma unroll
+                for (int q = 0; q < U; ++q) {
+                    append((bm >> (4 * q)) & 1u, v[q].x);
+                    append((bm >> (4 * q + 1)) & 1u, v[q].y);
+                    append((bm >> (4 * q + 2)) & 1u, v[q].z);
+                    append((bm >> (4 * q + 3)) & 1u, v[q].w);
+                }
+            }
         }
         if (threadIdx.x < 32) {  // the last n mod 4 scores, by warp 0
             const int64_t i = (n4 << 2) + threadIdx.x;
             const bool ok = i < n;
+            const float x = ok ? r[i] : 0.f;
             float sl = 0.f, sr = 0.f;
-            one(ok ? r[i] : 0.f, ok, sl, sr);
+            append(fold1(x, ok, sl, sr), x);
             SL += (double)sl;
             SR += (double)sr;
         }
@@ -1385,12 +1413,14 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
         for (int64_t i0 = 0; i0 < n; i0 += kBlk) {  // same trip count in every lane
             const int64_t i = i0 + threadIdx.x;
             const bool ok = i < n;
+            const float x = ok ? r[i] : 0.f;
             float sl = 0.f, sr = 0.f;
-            one(ok ? r[i] : 0.f, ok, sl, sr);
+            append(fold1(x, ok, sl, sr), x);
             SL += (double)sl;
             SR += (double)sr;
         }
     }
+    flush();
     const double sL = block_sum_d(SL, sm->red);
     const double sR = block_sum_d(SR, sm->red);
     const long long cnt = block_sum_ll((long long)cR, sm->lred);
