@@ -1647,27 +1647,10 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
     phase_mark(st, 14);
     // 1. the sample, as keys, with its level-1 histogram
     const uint64_t c0 = (uint64_t)row << 32;
-    constexpr int kDraws = 4;  // samples per thread with their gathers in flight together
-    for (int s0 = 0; s0 < m; s0 += kDraws * blockDim.x) {  // same trip count in every lane
-        float y[kDraws];
-#pragma unroll
-        for (int u = 0; u < kDraws; ++u) {
-            const int s = s0 + u * blockDim.x + threadIdx.x;
-            y[u] = s < m ? draw_sample(rr, n, t, seed, c0, s) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < kDraws; ++u) {
-            const int s = s0 + u * blockDim.x + threadIdx.x;
-            uint32_t bn = 0xffffffffu;
-            if (s < m) {
-                const uint32_t key = to_key(y[u]);
-                keys[s] = key;
-                bn = key >> 21;
-            }
-            const unsigned peers = __match_any_sync(0xffffffffu, bn);
-            if (bn != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
-                atomicAdd(&rb->hist1[bn], (uint32_t)__popc(peers));
-        }
+    for (int s = threadIdx.x; s < m; s += blockDim.x) {
+        const uint32_t key = to_key(draw_sample(rr, n, t, seed, c0, s));
+        keys[s] = key;
+        atomicAdd(&rb->hist1[key >> 21], 1u);
     }
     __syncthreads();
     phase_mark(st, 15);
