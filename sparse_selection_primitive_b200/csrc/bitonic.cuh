@@ -57,58 +57,4 @@ __device__ __forceinline__ void bitonic_sort_row(uint32_t (&key)[E], int tid, ui
     }
 }
 
-// The same network over a whole CTA (RT = CTA) with the stage loops kept as
-// loops.  A kernel that sorts once per launch (one CTA solving a band) would
-// fetch every unrolled stage cold into the instruction cache; this form's few
-// hundred instructions are fetched once and then run from the cache.
-template <int E, int CTA>
-__device__ void bitonic_sort_block_rolled(uint32_t (&key)[E], int tid, uint32_t* xch) {
-    static_assert(E == 1 || E == 2 || E == 4, "1, 2 or 4 keys per thread");
-    constexpr int NPAD = E * CTA;
-#pragma unroll 1
-    for (int size = 2; size <= NPAD; size <<= 1) {
-#pragma unroll 1
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            if (stride < E) {
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-#pragma unroll
-                    for (int sbit = 1; sbit < E; sbit <<= 1) {
-                        const int pe = e ^ sbit;
-                        if (sbit == stride && pe > e) {
-                            const bool asc = (((tid * E + e) & size) == 0);
-                            const uint32_t lo = min(key[e], key[pe]), hi = max(key[e], key[pe]);
-                            key[e] = asc ? lo : hi;
-                            key[pe] = asc ? hi : lo;
-                        }
-                    }
-                }
-            } else if (stride < 32 * E) {
-                const int ls = stride / E;
-                const bool asc = (((tid * E) & size) == 0);
-                const bool keep_min = (((tid & ls) == 0) == asc);
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const uint32_t o = __shfl_xor_sync(0xffffffffu, key[e], ls);
-                    key[e] = keep_min ? min(key[e], o) : max(key[e], o);
-                }
-            } else {
-                const int ts = stride / E;
-                const bool asc = (((tid * E) & size) == 0);
-                const bool keep_min = (((tid & ts) == 0) == asc);
-                const int partner = tid ^ ts;
-#pragma unroll
-                for (int e = 0; e < E; ++e) xch[e * CTA + tid] = key[e];
-                __syncthreads();
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const uint32_t o = xch[e * CTA + partner];
-                    key[e] = keep_min ? min(key[e], o) : max(key[e], o);
-                }
-                __syncthreads();
-            }
-        }
-    }
-}
-
 }  // namespace lapsum

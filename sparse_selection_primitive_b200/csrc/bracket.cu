@@ -461,22 +461,6 @@ __device__ __forceinline__ void bin_add(float x, const BinLayout& BL, float inv_
 
 constexpr int kStage = 1024;  // band scores staged per CTA before one global append
 
-// One lane appends one band score to the CTA staging buffer (or, when it is
-// full, straight to the global band).
-__device__ __forceinline__ void band_stage_lane(float x, float* sband, int* scount, float* band,
-                                                unsigned long long* counter,
-                                                unsigned long long cap, const BinLayout& BL,
-                                                float inv_t, unsigned long long* bins) {
-    const int pos = atomicAdd(scount, 1);
-    if (pos < kStage) {
-        sband[pos] = x;
-    } else {
-        const unsigned long long g = atomicAdd(counter, 1ull);
-        if (g < cap) band[g] = x;
-        bin_add(x, BL, inv_t, bins);
-    }
-}
-
 // Warp-aggregated append of the lanes with `take` to the CTA's staging buffer;
 // lanes past its capacity go straight to the global band (rare).
 __device__ __forceinline__ void band_stage(bool take, float x, float* sband, int* scount,
@@ -778,25 +762,6 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     }
 }
 
-// Warp-aggregated append of the lanes with `take` into band[] (capacity cap).
-__device__ __forceinline__ void band_append(bool take, float x, float* band,
-                                            unsigned long long* counter, unsigned long long cap) {
-    const unsigned ball = __ballot_sync(0xffffffffu, take);
-    if (ball == 0) return;
-    const int lane = threadIdx.x & 31;
-    const int leader = __ffs(ball) - 1;
-    unsigned long long base = 0;
-    if (lane == leader) base = atomicAdd(counter, (unsigned long long)__popc(ball));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (take) {
-        const unsigned long long pos = base + __popc(ball & ((1u << lane) - 1u));
-        if (pos < cap) band[pos] = x;
-    }
-}
-
-// ----------------------------------------------------------------------------
-// 3-4. Exact band solve, certification, narrowing and widening (one CTA).
-// ----------------------------------------------------------------------------
 struct FloatGet {
     const float* s;
     __device__ __forceinline__ float operator()(long long j) const { return s[j]; }
