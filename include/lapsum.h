@@ -30,7 +30,8 @@
  *     lapsum_read_status and lapsum_row_info.
  *   - Argument errors are detected on the host, returned at once, and launch
  *     nothing.  Conditions found on the device (non-finite scores, exhausted
- *     bracket retries) are OR-ed into a sticky status word inside the
+ *     bracket retries, per-row budgets outside (0, n)) are OR-ed into a
+ *     sticky status word inside the
  *     workspace and reported by lapsum_read_status, which also clears it.
  *   - Calls that share a workspace must be ordered on one stream (or be
  *     otherwise serialised); concurrent calls on one workspace race.
@@ -118,6 +119,27 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
  */
 int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v, float* g,
                     int64_t B, int64_t n, double t, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Forward with a budget per row: as lapsum_forward, with k[row] (fp64, DEVICE
+ * memory, B entries, read in stream order) in place of the shared k.  The
+ * pages fix one budget per operator call; a budget per row is the next step
+ * the same equation allows (every row is solved on its own).  Rows are
+ * solved by the sort-based solvers: LAPSUM_PATH_AUTO and LAPSUM_PATH_FULLSORT
+ * give the on-chip sort for n <= 4096 and the radix full sort above, and
+ * LAPSUM_PATH_RADIX forces the latter; the bracketing paths return
+ * LAPSUM_EINVAL (their sample ranks come from a budget known on the host).
+ * The workspace is lapsum_workspace_bytes(B, n, k, LAPSUM_PATH_FULLSORT) for
+ * any valid k.  `support` (may be NULL; see the gradient support below, same
+ * rules when not NULL) receives the gradient support of rows with n > 4096.
+ * A row whose k[row] is not in (0, n) gets b = NaN and p = NaN, and the
+ * workspace status reads LAPSUM_EINVAL (lapsum_read_status); the other rows
+ * are unaffected.  Host-side errors as lapsum_forward, plus LAPSUM_EINVAL for
+ * k == NULL.
+ */
+int lapsum_forward_rowk(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
+                        int64_t n, const double* k, double t, int path, void* ws, size_t ws_bytes,
+                        void* support, size_t support_bytes, void* stream);
 
 /*
  * Gradient support: a forward-to-backward hand-over for rows with n > 4096.

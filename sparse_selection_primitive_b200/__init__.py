@@ -114,6 +114,10 @@ def _lib():
         lib.lapsum_backward_kt.restype = ctypes.c_int
         lib.lapsum_backward_kt.argtypes = [_vp, _c_i64, _vp, _vp, _c_i64, _c_i64, ctypes.c_double,
                                            _vp, _vp, _vp, ctypes.c_size_t, _vp]
+        lib.lapsum_forward_rowk.restype = ctypes.c_int
+        lib.lapsum_forward_rowk.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64, _vp,
+                                            ctypes.c_double, ctypes.c_int, _vp, ctypes.c_size_t,
+                                            _vp, ctypes.c_size_t, _vp]
         lib.lapsum_sample_get.restype = ctypes.c_int
         lib.lapsum_sample_get.argtypes = [_vp, _c_i64, _vp, _c_i64, _vp]
         _LIB = lib
@@ -225,18 +229,35 @@ def _check_out(out: torch.Tensor, ref: torch.Tensor, ld: int, what: str):
         raise ValueError(f"{what} must be float32 CUDA with the shape and row stride of r")
 
 
-def forward(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0, ws: Workspace = None,
+def _row_budgets(k, B: int, device):
+    """k as a per-row budget tensor (float64 on the scores' device), or None for
+    a shared scalar budget.  A 1-D tensor with one entry per row is per-row."""
+    if isinstance(k, torch.Tensor) and k.dim() == 1:
+        if k.numel() != B:
+            raise ValueError("a per-row k needs one entry per row")
+        return k.detach().to(device=device, dtype=torch.float64).contiguous()
+    return None
+
+
+def forward(r: torch.Tensor, k, t: float, path="auto", seed: int = 0, ws: Workspace = None,
             want_sum_f: bool = False, p: torch.Tensor = None, b: torch.Tensor = None,
             support: Support = None):
     """Returns (p, b[, sum_f]) for each row of r (float32 CUDA, rows x n or n).
 
-    With ``support`` (a Support for the same B, n) the forward also lists the
-    gradient support for backward(..., support=...)."""
+    k is a number shared by every row, or a 1-D tensor with one budget per row
+    (lapsum_forward_rowk: the sort-based solvers).  With ``support`` (a Support
+    for the same B, n) the forward also lists the gradient support for
+    backward(..., support=...)."""
     squeeze = r.dim() == 1
     r2 = _as_rows(r)
     B, n = r2.shape
     ld = _ld(r2)
     code = _path_code(path)
+    k_rows = _row_budgets(k, B, r2.device)
+    if k_rows is not None:
+        k = 0.5 * n  # any valid budget sizes the workspace of the sort-based solvers
+        if (code & 0xFF) == PATHS["auto"]:
+            code = (code & ~0xFF) | PATHS["fullsort"]
     if ws is None or not ws.fits(B, n, k, code):
         ws = Workspace(B, n, k, code, r2.device)
     if p is None:
@@ -249,7 +270,16 @@ def forward(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0, ws:
     elif b.dtype != torch.float64 or b.numel() != B or not b.is_contiguous():
         raise ValueError("b must be a contiguous float64 CUDA tensor with one entry per row")
     sf = torch.empty(B, dtype=torch.float64, device=r2.device) if want_sum_f else None
-    if support is not None:
+    if k_rows is not None:
+        if support is not None and not support.fits(B, n):
+            raise ValueError("support buffer too small for (B, n)")
+        _check(_lib().lapsum_forward_rowk(
+            r2.data_ptr(), ld, p.data_ptr(), b.data_ptr(),
+            sf.data_ptr() if sf is not None else None, B, n, k_rows.data_ptr(), float(t), code,
+            ws.ptr, ws.nbytes, support.ptr if support is not None else None,
+            support.nbytes if support is not None else 0, _stream_ptr(r2.device)),
+            "lapsum_forward_rowk")
+    elif support is not None:
         if not support.fits(B, n):
             raise ValueError("support buffer too small for (B, n)")
         _check(_lib().lapsum_forward_support(
@@ -409,7 +439,8 @@ class LapSumTopK(torch.autograd.Function):
         rd = r.detach()
         B = 1 if rd.dim() == 1 else rd.shape[0]
         n = rd.shape[-1]
-        kf = float(k)
+        per_row = isinstance(k, torch.Tensor) and k.dim() == 1
+        kf = k.detach() if per_row else float(k)
         tf = float(t)
         sup = Support(B, n, rd.device) if support_bytes(B, n) > 0 else None
         p, b = forward(rd, kf, tf, path=path, seed=seed, support=sup)
@@ -429,16 +460,21 @@ class LapSumTopK(torch.autograd.Function):
         ctx.sup = None
         gk = gt = None
         if any(ctx.kt_grad):
-            # k and t are shared by every row: their gradients sum over rows
+            # a shared k or t gets the sum over rows of the per-row gradients;
+            # a per-row k (one entry per row) gets them row by row
             gks, gts = backward_kt(r.detach(), b, v, ctx.t)
             k, t = ctx.kt_like
             if ctx.kt_grad[0]:
-                gk = gks.sum().to(k.dtype).reshape(k.shape)
+                if k.dim() == 1:
+                    gk = gks.reshape(-1).to(k.dtype)
+                else:
+                    gk = gks.sum().to(k.dtype).reshape(k.shape)
             if ctx.kt_grad[1]:
                 gt = gts.sum().to(t.dtype).reshape(t.shape)
         return g, gk, gt, None, None
 
 
-def soft_topk(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0) -> torch.Tensor:
-    """Differentiable soft top-k probabilities p with sum p = k per row."""
+def soft_topk(r: torch.Tensor, k, t: float, path="auto", seed: int = 0) -> torch.Tensor:
+    """Differentiable soft top-k probabilities p with sum p = k per row (k a number,
+    or a 1-D tensor with one budget per row)."""
     return LapSumTopK.apply(r, k, t, path, seed)

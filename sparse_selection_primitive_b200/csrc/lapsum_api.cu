@@ -278,14 +278,21 @@ namespace {
 // The forward of lapsum_forward and lapsum_forward_support; `support` is null
 // for the former.
 int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
-                 int64_t n, double k, double t, int path, uint64_t seed, void* ws, size_t ws_bytes,
-                 void* support, size_t support_size, void* stream) {
+                 int64_t n, double k, const double* k_rows, double t, int path, uint64_t seed,
+                 void* ws, size_t ws_bytes, void* support, size_t support_size, void* stream) {
     if (r == nullptr || p == nullptr || b == nullptr) return LAPSUM_EINVAL;
     if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
-    if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
+    if (k_rows == nullptr && (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)))
+        return LAPSUM_EINVAL;
     if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
-    const int rp = resolve_path(n, path);
+    int rp = resolve_path(n, path);
     if (rp < 0 || (path & ~0x7ff) != 0) return LAPSUM_EINVAL;
+    if (k_rows != nullptr) {
+        // per-row budgets: the sort-based solvers (the bracketing paths take
+        // their sample ranks from a budget known on the host)
+        if ((path & 0xff) == LAPSUM_PATH_AUTO) rp = resolve_path(n, LAPSUM_PATH_FULLSORT);
+        if (rp != LAPSUM_PATH_FULLSORT && rp != LAPSUM_PATH_RADIX) return LAPSUM_EINVAL;
+    }
     if (n > INT32_MAX && rp != LAPSUM_PATH_BRACKET) return LAPSUM_EINVAL;
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
     const Layout L = make_layout(B, n, rp);
@@ -304,7 +311,7 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
     cudaError_t e = cudaSuccess;
 
     if (rp == LAPSUM_PATH_FULLSORT) {
-        e = launch_onchip_forward(r, ld, p, b, sum_f, B, (int)n, k, t, hdr, vec, st);
+        e = launch_onchip_forward(r, ld, p, b, sum_f, B, (int)n, k, k_rows, t, hdr, vec, st);
         return cuda_status(e);
     }
     if (rp == LAPSUM_PATH_RADIX) {
@@ -326,7 +333,8 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
             sub.plan += r0 * 8;
             e = launch_radix_sort_rows(r + r0 * ld, ld, nb, n, sub, rows + r0, hdr, st);
             if (e == cudaSuccess)
-                e = launch_rowsolve_sorted_keys(sub, nb, n, k, t, b + r0, rows + r0, hdr, st);
+                e = launch_rowsolve_sorted_keys(sub, nb, n, k, k_rows ? k_rows + r0 : nullptr, t,
+                                                b + r0, rows + r0, hdr, st);
         }
     } else if (rp == LAPSUM_PATH_ROWBRACKET) {
         const int m = sample_size(n, k);
@@ -373,8 +381,16 @@ extern "C" {
 int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
                    int64_t n, double k, double t, int path, uint64_t seed, void* ws,
                    size_t ws_bytes, void* stream) {
-    return forward_impl(r, ld, p, b, sum_f, B, n, k, t, path, seed, ws, ws_bytes, nullptr, 0,
-                        stream);
+    return forward_impl(r, ld, p, b, sum_f, B, n, k, nullptr, t, path, seed, ws, ws_bytes,
+                        nullptr, 0, stream);
+}
+
+int lapsum_forward_rowk(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
+                        int64_t n, const double* k, double t, int path, void* ws, size_t ws_bytes,
+                        void* support, size_t support_size, void* stream) {
+    if (k == nullptr) return LAPSUM_EINVAL;
+    return forward_impl(r, ld, p, b, sum_f, B, n, 0.0, k, t, path, 0, ws, ws_bytes, support,
+                        support_size, stream);
 }
 
 int lapsum_forward_support(const float* r, int64_t ld, float* p, double* b, double* sum_f,
@@ -382,7 +398,7 @@ int lapsum_forward_support(const float* r, int64_t ld, float* p, double* b, doub
                            void* ws, size_t ws_bytes, void* support, size_t support_size,
                            void* stream) {
     if (support == nullptr && n > kOnchipMax) return LAPSUM_EWORKSPACE;
-    return forward_impl(r, ld, p, b, sum_f, B, n, k, t, path, seed, ws, ws_bytes, support,
+    return forward_impl(r, ld, p, b, sum_f, B, n, k, nullptr, t, path, seed, ws, ws_bytes, support,
                         support_size, stream);
 }
 
@@ -494,6 +510,7 @@ int lapsum_read_status(void* ws, void* stream, int* device_status) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return LAPSUM_ECUDA;
     *device_status = (bits & kDevNonFinite) ? LAPSUM_ENONFINITE
+                     : (bits & kDevBadBudget) ? LAPSUM_EINVAL
                      : (bits & kDevBracketExhausted) ? LAPSUM_EBRACKET
                                                      : LAPSUM_OK;
     return LAPSUM_OK;

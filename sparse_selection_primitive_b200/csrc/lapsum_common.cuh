@@ -20,6 +20,7 @@ namespace lapsum {
 enum : uint32_t {
     kDevNonFinite = 1u << 0,
     kDevBracketExhausted = 1u << 1,
+    kDevBadBudget = 1u << 2,  // a per-row budget outside (0, n)
 };
 
 constexpr int kMaxAttempts = 7;     // 1 + 3 widenings per side; the last rungs are open

@@ -39,9 +39,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // --- on-chip full sort (n <= 4096) -------------------------------------------
 int onchip_npad(int64_t n);
+// k_rows (device, B entries) when not null gives each row its own budget.
 cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,
-                                  int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
-                                  cudaStream_t st);
+                                  int64_t B, int n, double k, const double* k_rows, double t,
+                                  WsHeader* hdr, int vec, cudaStream_t st);
 cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
                                    float* g, int64_t B, int n, double t, int vec, cudaStream_t st);
 
@@ -59,8 +60,8 @@ cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_
                                    cudaStream_t st);
 // Solve every row from its sorted keys (one CTA per row); writes b and RowState.
 cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
-                                        double t, double* b, RowState* rows, WsHeader* hdr,
-                                        cudaStream_t st);
+                                        const double* k_rows, double t, double* b, RowState* rows,
+                                        WsHeader* hdr, cudaStream_t st);
 
 // --- streaming kernels over long rows ----------------------------------------
 constexpr int kStreamTile = 4096;  // elements per CTA tile of the streaming kernels

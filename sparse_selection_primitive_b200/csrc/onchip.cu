@@ -144,7 +144,8 @@ __device__ __forceinline__ void row_sync() {
 template <int E, int RT, int CTA>
 __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel(
     const float* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
-    double* __restrict__ sumf_out, int64_t B, int n, double k, double t, WsHeader* hdr, int vec) {
+    double* __restrict__ sumf_out, int64_t B, int n, double k, const double* __restrict__ k_rows,
+    double t, WsHeader* hdr, int vec) {
     using S = Shape<E, RT, CTA>;
     __shared__ uint32_t xch[(RT > 32) ? CTA * E : 1];
     __shared__ uint32_t last_key[CTA];
@@ -164,6 +165,10 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
     const bool row_ok = row < B;
     const float* rrow = r + (row_ok ? row : 0) * ld;
     const double inv_t = 1.0 / t;
+    // the row's budget: the shared k, or its own entry of k_rows (checked here: a
+    // budget outside (0, n) gives b = NaN and a status bit)
+    const double kr = (k_rows != nullptr && row_ok) ? k_rows[row] : k;
+    const bool k_ok = kr > 0.0 && kr < (double)n;
 
     if (tid == 0) row_flag[rloc] = 0;
     if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -184,6 +189,7 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
     }
     row_sync<E, RT, CTA>();
     if (bad) atomicOr(&row_flag[rloc], 1);
+    if (tid == 0 && !k_ok) atomicOr(&row_flag[rloc], 2);
 
     bitonic_sort_row<E, RT, CTA>(key, tid, xch);
 
@@ -257,7 +263,7 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
         y = (j < n) ? fma(gn, y, 1.0) : 0.0;
         Q[e] = y;
         const double G = (double)(n - j) - 0.5 * Q[e] + 0.5 * (P[e] - 1.0);
-        cnt += (j < n && G >= k) ? 1 : 0;
+        cnt += (j < n && G >= kr) ? 1 : 0;
     }
     const int jstar = row_sum_i<E, RT, CTA>(cnt, ired);
 
@@ -277,14 +283,16 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
     row_sync<E, RT, CTA>();
     if (tid < 32) {  // the row's first warp takes the root together
         double bb;
-        if (row_flag[rloc] || !row_ok) {
+        const int flag = row_flag[rloc];
+        if (flag || !row_ok) {
             bb = nan("");
-            if (row_ok && tid == 0) set_status(hdr, kDevNonFinite);
+            if (row_ok && tid == 0)
+                set_status(hdr, ((flag & 1) ? kDevNonFinite : 0u) | ((flag & 2) ? kDevBadBudget : 0u));
         } else {
             const bool hasL = jstar >= 1, hasR = jstar < n;
             bb = segment_root(hasL, anchor[rloc][0], hasL ? anchor[rloc][1] : 0.0, hasR,
                               anchor[rloc][2], hasR ? anchor[rloc][3] : 0.0,
-                              (double)(n - jstar) - k, t);
+                              (double)(n - jstar) - kr, t);
         }
         if (tid == 0) {
             row_b[rloc] = bb;
@@ -361,13 +369,14 @@ __global__ void __launch_bounds__(CTA) onchip_backward_kernel(
 
 template <int E, int RT, int CTA>
 cudaError_t launch_fwd(const float* r, int64_t ld, float* p, double* b, double* sumf, int64_t B,
-                       int n, double k, double t, WsHeader* hdr, int vec, cudaStream_t st) {
+                       int n, double k, const double* k_rows, double t, WsHeader* hdr, int vec,
+                       cudaStream_t st) {
     using S = Shape<E, RT, CTA>;
     const int64_t grid = (B + S::ROWS - 1) / S::ROWS;
     {
         ProfScope ps_("onchip_fwd", st);
         onchip_forward_kernel<E, RT, CTA>
-        <<<(unsigned)grid, CTA, 0, st>>>(r, ld, p, b, sumf, B, n, k, t, hdr, vec);
+        <<<(unsigned)grid, CTA, 0, st>>>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec);
     }
     return cudaGetLastError();
 }
@@ -393,17 +402,17 @@ int onchip_npad(int64_t n) {
 }
 
 cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,
-                                  int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
-                                  cudaStream_t st) {
+                                  int64_t B, int n, double k, const double* k_rows, double t,
+                                  WsHeader* hdr, int vec, cudaStream_t st) {
     switch (onchip_npad(n)) {
-        case 32: return launch_fwd<1, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
-        case 64: return launch_fwd<2, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
-        case 128: return launch_fwd<4, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
-        case 256: return launch_fwd<8, 32, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
-        case 512: return launch_fwd<8, 64, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
-        case 1024: return launch_fwd<8, 128, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
-        case 2048: return launch_fwd<8, 256, 256>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
-        case 4096: return launch_fwd<8, 512, 512>(r, ld, p, b, sumf, B, n, k, t, hdr, vec, st);
+        case 32: return launch_fwd<1, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
+        case 64: return launch_fwd<2, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
+        case 128: return launch_fwd<4, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
+        case 256: return launch_fwd<8, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
+        case 512: return launch_fwd<8, 64, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
+        case 1024: return launch_fwd<8, 128, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
+        case 2048: return launch_fwd<8, 256, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
+        case 4096: return launch_fwd<8, 512, 512>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
         default: return cudaErrorInvalidValue;
     }
 }

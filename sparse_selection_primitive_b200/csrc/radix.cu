@@ -265,18 +265,27 @@ struct KeyGet {
 
 __global__ void __launch_bounds__(1024) rowsolve_keys_kernel(const uint32_t* __restrict__ k0,
                                                               const uint32_t* __restrict__ k1,
-                                                              int64_t n, double k, double t,
+                                                              int64_t n, double k,
+                                                              const double* __restrict__ k_rows,
+                                                              double t,
                                                               const int32_t* __restrict__ plan,
                                                               double* __restrict__ b_out,
-                                                              RowState* rows) {
+                                                              RowState* rows, WsHeader* hdr) {
     __shared__ SolveScratch sm;
     __shared__ SolveResult res;
     const int64_t row = blockIdx.x;
     const uint32_t* keys = (plan[row * 8 + 4] ? k1 : k0) + row * n;
     Tails tl{false, 0.f, 0.0, false, 0.f, 0.0, 0.0};
-    solve_sorted_block(KeyGet{keys}, (long long)n, tl, k, t, &sm, &res);
+    // the row's budget: the shared k or its own entry of k_rows (outside (0, n): b = NaN)
+    const double kr = k_rows != nullptr ? k_rows[row] : k;
+    const bool k_ok = kr > 0.0 && kr < (double)n;
+    solve_sorted_block(KeyGet{keys}, (long long)n, tl, k_ok ? kr : 0.5 * (double)n, t, &sm, &res);
     if (threadIdx.x == 0) {
-        const double b = (rows[row].status & kDevNonFinite) ? nan("") : res.b;
+        if (!k_ok) {
+            rows[row].status |= kDevBadBudget;
+            set_status(hdr, kDevBadBudget);
+        }
+        const double b = ((rows[row].status & kDevNonFinite) || !k_ok) ? nan("") : res.b;
         rows[row].b = b;
         rows[row].path = LAPSUM_PATH_RADIX;
         rows[row].attempts = 1;
@@ -331,13 +340,12 @@ cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_
 }
 
 cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
-                                        double t, double* b, RowState* rows, WsHeader* hdr,
-                                        cudaStream_t st) {
-    (void)hdr;
+                                        const double* k_rows, double t, double* b, RowState* rows,
+                                        WsHeader* hdr, cudaStream_t st) {
     {
         ProfScope ps_("rowsolve", st);
-        rowsolve_keys_kernel<<<(unsigned)B, 1024, 0, st>>>(buf.keys[0], buf.keys[1], n, k, t,
-                                                       buf.plan, b, rows);
+        rowsolve_keys_kernel<<<(unsigned)B, 1024, 0, st>>>(buf.keys[0], buf.keys[1], n, k, k_rows,
+                                                       t, buf.plan, b, rows, hdr);
     }
     return cudaGetLastError();
 }
