@@ -263,13 +263,15 @@ def main():
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_buf = torch.empty(2 * l2_bytes // 4 + 1024, dtype=torch.float32, device=dev)
 
-    def run_workload(w, r_h, v_h, steps, warmup, table=False):
+    def run_workload(w, r_h, v_h, steps, warmup, table=False, k_rows=None):
         rd = torch.from_numpy(r_h).to(dev)
         vd = torch.from_numpy(v_h).to(dev)
         pd = torch.empty_like(rd)
         gd = torch.empty_like(rd)
         bd = torch.empty(w.B, dtype=torch.float64, device=dev)
-        ws = L.Workspace(w.B, w.n, w.k, "auto", dev)
+        # one budget per row (lapsum_forward_rowk) when k_rows is given
+        kk = w.k if k_rows is None else torch.from_numpy(k_rows).to(dev)
+        ws = L.Workspace(w.B, w.n, w.k, "auto" if k_rows is None else "fullsort", dev)
         # rows longer than 4096 hand the gradient support from forward to
         # backward, as the autograd wrapper does
         sup = L.Support(w.B, w.n, dev) if L.support_bytes(w.B, w.n) > 0 else None
@@ -277,7 +279,7 @@ def main():
         flush = working < 2 * l2_bytes
 
         def fwd():
-            L.forward(rd, w.k, w.t, ws=ws, p=pd, b=bd, support=sup)
+            L.forward(rd, kk, w.t, ws=ws, p=pd, b=bd, support=sup)
 
         def bwd():
             L.backward(rd, bd, vd, w.t, ws=ws, g=gd, support=sup)
@@ -449,6 +451,22 @@ def main():
                 table[name]["bracket"] = RW["bracket"]
             del RW
             torch.cuda.empty_cache()
+        # the router shape with one budget per row (integers 4..12, seeded)
+        wk = WORKLOADS["moe_router_16384x256"]
+        rr, vv = make_inputs(wk, seed=0)
+        kr = np.random.default_rng(1).integers(4, 13, wk.B).astype(np.float64)
+        RW = run_workload(wk, rr, vv, 10, 3, table=True, k_rows=kr)
+        T = RW["table"]
+        table["moe_router_16384x256_rowk"] = {
+            "k_rows": "integers 4..12 (numpy default_rng(1))",
+            "fwd_ms": round(T["fwd_ms"], 5), "bwd_ms": round(T["bwd_ms"], 5),
+            "fwdbwd_graph_ms": round(T["fwdbwd_graph_ms"], 5),
+            "fwdbwd_graph_elements_per_s": wk.elements / (T["fwdbwd_graph_ms"] / 1e3),
+            "path_frac_of_peak": (path_step_bytes(wk, 0) / (T["fwdbwd_graph_ms"] / 1e3) / 1e9
+                                  / peak_gbs),
+        }
+        del RW
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
