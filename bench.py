@@ -343,6 +343,58 @@ def main():
                 res["table"]["bwd_without_support_ms"] = statistics.median(tp)
         return res
 
+    def router_bf16_row(peak_gbs):
+        """The router shape through the router form: bf16 scores, p and the list of
+        p > 1e-3 (at most 16 per row) in the forward, g from bf16 scores."""
+        wk = WORKLOADS["moe_router_16384x256"]
+        rr, vv = make_inputs(wk, seed=0)
+        rd = torch.from_numpy(rr).to(dev).to(torch.bfloat16)
+        vd = torch.from_numpy(vv).to(dev)
+        ws = L.Workspace(wk.B, wk.n, wk.k, "fullsort", dev)
+        out = {}
+
+        def fwd():
+            out["fw"] = L.forward_router(rd, wk.k, wk.t, eps=1e-3, cap=16, ws=ws)
+
+        def bwd():
+            out["g"] = L.backward_router(rd, out["fw"][1], vd, wk.t)
+
+        for _ in range(3):
+            fwd()
+            bwd()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fwd()
+            bwd()
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(graph):
+            fwd()
+            bwd()
+        torch.cuda.synchronize(dev)
+        times = []
+        for _ in range(10):
+            flush_buf.zero_()
+            s_ev = torch.cuda.Event(enable_timing=True)
+            e_ev = torch.cuda.Event(enable_timing=True)
+            s_ev.record(stream)
+            graph.replay()
+            e_ev.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(s_ev.elapsed_time(e_ev))
+        ms = statistics.median(times)
+        # bytes: r (2 B) and p (4 B) in the forward, r (2 B), v and g (4 B each) in the
+        # backward, plus the list (16 x 8 B per row)
+        nbytes = wk.elements * (2 + 4 + 2 + 4 + 4) + wk.B * 16 * 8
+        del graph
+        return {"scores": "bf16", "select": "p > 1e-3, at most 16 per row",
+                "fwdbwd_graph_ms": round(ms, 5),
+                "fwdbwd_graph_elements_per_s": wk.elements / (ms / 1e3),
+                "path_frac_of_peak": nbytes / (ms / 1e3) / 1e9 / peak_gbs}
+
     peak_gbs, peak_kind = load_peaks()
     R = run_workload(w, r_h, v_h, args.steps, args.warmup)
     sampler = ClockSampler(local)
@@ -466,6 +518,8 @@ def main():
                                   / peak_gbs),
         }
         del RW
+        torch.cuda.empty_cache()
+        table["moe_router_16384x256_bf16_select"] = router_bf16_row(peak_gbs)
         torch.cuda.empty_cache()
 
     cpu = None

@@ -67,6 +67,12 @@ enum lapsum_path {
                                   statistics, fold and band solve in one kernel (n <= 2^20) */
 };
 
+/* Score element types of the router entry points. */
+enum lapsum_dtype {
+    LAPSUM_DTYPE_F32 = 0,  /* float */
+    LAPSUM_DTYPE_BF16 = 1  /* bfloat16, passed as its 16-bit patterns (uint16_t) */
+};
+
 /* Test and diagnostic flags, OR-ed into `path`. */
 enum lapsum_flags {
     LAPSUM_FLAG_FORCE_MISS = 0x100, /* bracketing: start from a bracket that excludes b */
@@ -119,6 +125,31 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
  */
 int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v, float* g,
                     int64_t B, int64_t n, double t, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Router form for short rows (n <= 4096, the on-chip sort), e.g. the scores of
+ * a mixture-of-experts router: scores r of type `dtype` (fp32, or bf16 bit
+ * patterns widened exactly to fp32), p (fp32) and b (fp64) as lapsum_forward,
+ * and, when sel_cnt is not NULL, the sparse support of each row next to p:
+ * sel_idx[row*cap + j] and sel_p[row*cap + j], j < min(cap, sel_cnt[row]),
+ * are the positions (ascending) and values of the scores with p > eps, and
+ * sel_cnt[row] is their number (it may exceed cap; the list then holds the
+ * first cap).  The decision p > eps is taken on the fp32 p that is written.
+ * sel_idx/sel_p/sel_cnt are device arrays of B*cap, B*cap and B entries, all
+ * NULL or all given; cap >= 1 and eps >= 0 when given.  ws as lapsum_forward
+ * with LAPSUM_PATH_FULLSORT.  The pages state the problem for real-valued
+ * scores; a narrower score type and the support list are this library's
+ * additions for that use.  lapsum_backward_router: g (fp32) from scores of
+ * `dtype` and fp32 v, as lapsum_backward (no workspace).  Errors: LAPSUM_EINVAL
+ * for n > 4096, an unknown dtype or inconsistent selection arguments, else as
+ * lapsum_forward / lapsum_backward.
+ */
+int lapsum_forward_router(const void* r, int dtype, int64_t ld, float* p, double* b, int64_t B,
+                          int64_t n, double k, double t, float eps, int32_t cap, int32_t* sel_idx,
+                          float* sel_p, int32_t* sel_cnt, void* ws, size_t ws_bytes,
+                          void* stream);
+int lapsum_backward_router(const void* r, int dtype, int64_t ld, const double* b, const float* v,
+                           float* g, int64_t B, int64_t n, double t, void* stream);
 
 /*
  * Forward with a budget per row: as lapsum_forward, with k[row] (fp64, DEVICE

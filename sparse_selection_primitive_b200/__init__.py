@@ -114,6 +114,14 @@ def _lib():
         lib.lapsum_backward_kt.restype = ctypes.c_int
         lib.lapsum_backward_kt.argtypes = [_vp, _c_i64, _vp, _vp, _c_i64, _c_i64, ctypes.c_double,
                                            _vp, _vp, _vp, ctypes.c_size_t, _vp]
+        lib.lapsum_forward_router.restype = ctypes.c_int
+        lib.lapsum_forward_router.argtypes = [_vp, ctypes.c_int, _c_i64, _vp, _vp, _c_i64, _c_i64,
+                                              ctypes.c_double, ctypes.c_double, ctypes.c_float,
+                                              ctypes.c_int32, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                              _vp]
+        lib.lapsum_backward_router.restype = ctypes.c_int
+        lib.lapsum_backward_router.argtypes = [_vp, ctypes.c_int, _c_i64, _vp, _vp, _vp, _c_i64,
+                                               _c_i64, ctypes.c_double, _vp]
         lib.lapsum_forward_rowk.restype = ctypes.c_int
         lib.lapsum_forward_rowk.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64, _vp,
                                             ctypes.c_double, ctypes.c_int, _vp, ctypes.c_size_t,
@@ -334,6 +342,61 @@ def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Wo
                                       g.data_ptr(), B, n, float(t), ws.ptr, ws.nbytes,
                                       _stream_ptr(r2.device)), "lapsum_backward")
     return g[0] if squeeze else g
+
+
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+def _router_rows(x: torch.Tensor) -> torch.Tensor:
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if x.dim() != 2 or x.dtype not in _DTYPES or not x.is_cuda:
+        raise TypeError("router scores must be a float32 or bfloat16 CUDA tensor, rows x n")
+    if x.stride(1) != 1 or (x.shape[0] > 1 and x.stride(0) < x.shape[1]):
+        x = x.contiguous()
+    return x
+
+
+def forward_router(r: torch.Tensor, k: float, t: float, eps: float = None, cap: int = None,
+                   ws: Workspace = None):
+    """Router form for rows of n <= 4096 (lapsum_forward_router): r is float32 or
+    bfloat16.  Returns (p, b), or with eps and cap also (idx, vals, cnt): per row
+    the positions and values of p > eps (at most cap, ascending) and their count."""
+    r2 = _router_rows(r)
+    B, n = r2.shape
+    ld = r2.stride(0) if B > 1 else n
+    if ws is None or not ws.fits(B, n, 0.5 * n, "fullsort"):
+        ws = Workspace(B, n, 0.5 * n, "fullsort", r2.device)
+    p = torch.empty((B, ld), dtype=torch.float32, device=r2.device)[:, :n]
+    b = torch.empty(B, dtype=torch.float64, device=r2.device)
+    want = eps is not None
+    if want:
+        idx = torch.full((B, cap), -1, dtype=torch.int32, device=r2.device)
+        vals = torch.zeros((B, cap), dtype=torch.float32, device=r2.device)
+        cnt = torch.empty(B, dtype=torch.int32, device=r2.device)
+    _check(_lib().lapsum_forward_router(
+        r2.data_ptr(), _DTYPES[r2.dtype], ld, p.data_ptr(), b.data_ptr(), B, n, float(k),
+        float(t), float(eps) if want else 0.0, int(cap) if want else 0,
+        idx.data_ptr() if want else None, vals.data_ptr() if want else None,
+        cnt.data_ptr() if want else None, ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
+        "lapsum_forward_router")
+    if r.dim() == 1:
+        p = p[0]
+    return (p, b, idx, vals, cnt) if want else (p, b)
+
+
+def backward_router(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float):
+    """g (float32) for router scores r (float32 or bfloat16), n <= 4096."""
+    r2 = _router_rows(r)
+    B, n = r2.shape
+    v2 = v.reshape(B, n).to(torch.float32).contiguous()
+    if r2.stride(0) != n and B > 1:
+        r2 = r2.contiguous()
+    g = torch.empty((B, n), dtype=torch.float32, device=r2.device)
+    _check(_lib().lapsum_backward_router(r2.data_ptr(), _DTYPES[r2.dtype], n, b.data_ptr(),
+                                         v2.data_ptr(), g.data_ptr(), B, n, float(t),
+                                         _stream_ptr(r2.device)), "lapsum_backward_router")
+    return g[0] if r.dim() == 1 else g
 
 
 def backward_kt(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float,

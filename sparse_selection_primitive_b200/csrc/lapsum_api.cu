@@ -385,6 +385,42 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
                         nullptr, 0, stream);
 }
 
+int lapsum_forward_router(const void* r, int dtype, int64_t ld, float* p, double* b, int64_t B,
+                          int64_t n, double k, double t, float eps, int32_t cap, int32_t* sel_idx,
+                          float* sel_p, int32_t* sel_cnt, void* ws, size_t ws_bytes,
+                          void* stream) {
+    if (r == nullptr || p == nullptr || b == nullptr) return LAPSUM_EINVAL;
+    if (dtype != LAPSUM_DTYPE_F32 && dtype != LAPSUM_DTYPE_BF16) return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || n > kOnchipMax || ld < n) return LAPSUM_EINVAL;
+    if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    const bool want_sel = sel_cnt != nullptr;
+    if (want_sel != (sel_idx != nullptr) || want_sel != (sel_p != nullptr)) return LAPSUM_EINVAL;
+    if (want_sel && (cap < 1 || !(eps >= 0.f) || !std::isfinite(eps))) return LAPSUM_EINVAL;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const Layout L = make_layout(B, n, LAPSUM_PATH_FULLSORT);
+    if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(static_cast<char*>(ws) + L.header);
+    const int bf16 = dtype == LAPSUM_DTYPE_BF16 ? 1 : 0;
+    const int vec = (aligned16(r) && aligned16(p) && (ld % (bf16 ? 8 : 4)) == 0) ? 1 : 0;
+    return cuda_status(launch_onchip_router(r, bf16, ld, p, b, B, (int)n, k, t, hdr, vec, sel_idx,
+                                            sel_p, sel_cnt, want_sel ? cap : 0, eps,
+                                            (cudaStream_t)stream));
+}
+
+int lapsum_backward_router(const void* r, int dtype, int64_t ld, const double* b, const float* v,
+                           float* g, int64_t B, int64_t n, double t, void* stream) {
+    if (r == nullptr || b == nullptr || v == nullptr || g == nullptr) return LAPSUM_EINVAL;
+    if (dtype != LAPSUM_DTYPE_F32 && dtype != LAPSUM_DTYPE_BF16) return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || n > kOnchipMax || ld < n) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    const int bf16 = dtype == LAPSUM_DTYPE_BF16 ? 1 : 0;
+    const int vec =
+        (aligned16(r) && aligned16(v) && aligned16(g) && (ld % (bf16 ? 8 : 4)) == 0) ? 1 : 0;
+    return cuda_status(launch_onchip_backward_router(r, bf16, ld, b, v, g, B, (int)n, t, vec,
+                                                     (cudaStream_t)stream));
+}
+
 int lapsum_forward_rowk(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
                         int64_t n, const double* k, double t, int path, void* ws, size_t ws_bytes,
                         void* support, size_t support_size, void* stream) {

@@ -45,6 +45,16 @@ cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* 
                                   WsHeader* hdr, int vec, cudaStream_t st);
 cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
                                    float* g, int64_t B, int n, double t, int vec, cudaStream_t st);
+// The router form: scores as fp32 (bf16 = 0) or bf16 bit patterns (bf16 = 1),
+// and optionally (sel_cnt != null) the per-row list of positions and values of
+// p > eps (at most cap per row) with its count.
+cudaError_t launch_onchip_router(const void* r, int bf16, int64_t ld, float* p, double* b,
+                                 int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
+                                 int32_t* sel_idx, float* sel_val, int32_t* sel_cnt, int cap,
+                                 float eps, cudaStream_t st);
+cudaError_t launch_onchip_backward_router(const void* r, int bf16, int64_t ld, const double* b,
+                                          const float* v, float* g, int64_t B, int n, double t,
+                                          int vec, cudaStream_t st);
 
 // --- radix full sort (segmented LSD, keys only) ------------------------------
 constexpr int kRadixTile = 4096;

@@ -58,6 +58,37 @@ __device__ __forceinline__ void load_row(const float* __restrict__ row, int n, i
     }
 }
 
+// The same for bf16 scores (bit patterns; bf16 is the upper half of fp32, so
+// the widening is exact): eight per 16-byte load.
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+template <int E>
+__device__ __forceinline__ void load_row(const uint16_t* __restrict__ row, int n, int tid, bool vec,
+                                         bool row_ok, float (&x)[E], bool (&valid)[E]) {
+    const int base = tid * E;
+    if constexpr (E % 8 == 0) {
+        if (vec && row_ok && base + E <= n) {
+#pragma unroll
+            for (int q = 0; q < E / 8; ++q) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + base) + q);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    x[8 * q + 2 * h] = __uint_as_float(w[h] << 16);
+                    x[8 * q + 2 * h + 1] = __uint_as_float(w[h] & 0xffff0000u);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) valid[e] = true;
+            return;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        valid[e] = row_ok && (base + e < n);
+        x[e] = valid[e] ? bf16_to_f32(__ldg(row + base + e)) : 0.f;
+    }
+}
+
 template <int E>
 __device__ __forceinline__ void store_row(float* __restrict__ row, int n, int tid, bool vec,
                                           bool row_ok, const float (&y)[E]) {
@@ -133,6 +164,38 @@ __device__ __forceinline__ float row_min_f(float v, float* red) {
     }
 }
 
+// Exclusive prefix of an int over the threads of one row (thread order);
+// *total gets the row's sum.
+template <int E, int RT, int CTA>
+__device__ __forceinline__ int row_excl_scan_i(int v, int* red, int* total) {
+    using S = Shape<E, RT, CTA>;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc += o;
+    }
+    if constexpr (S::WPR == 1) {
+        *total = __shfl_sync(0xffffffffu, inc, 31);
+        return inc - v;
+    } else {
+        if (lane == 31) red[w] = inc;
+        __syncthreads();
+        const int w0 = (w / S::WPR) * S::WPR;
+        int before = 0, all = 0;
+#pragma unroll
+        for (int i = 0; i < S::WPR; ++i) {
+            const int c = red[w0 + i];
+            before += (w0 + i < w) ? c : 0;
+            all += c;
+        }
+        __syncthreads();
+        *total = all;
+        return before + inc - v;
+    }
+}
+
 // Barrier over the threads of one row: a row held by one warp needs only the
 // warp's own barrier, so the rows of a CTA run their steps independently.
 template <int E, int RT, int CTA>
@@ -141,11 +204,21 @@ __device__ __forceinline__ void row_sync() {
     else __syncthreads();
 }
 
-template <int E, int RT, int CTA>
+// Selection list of the router form: per row, the positions (ascending) and
+// values of the scores with p > eps, at most cap of them, and their count.
+struct SelectOut {
+    int32_t* idx;
+    float* val;
+    int32_t* cnt;
+    int cap;
+    float eps;
+};
+
+template <int E, int RT, int CTA, class In>
 __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel(
-    const float* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
+    const In* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
     double* __restrict__ sumf_out, int64_t B, int n, double k, const double* __restrict__ k_rows,
-    double t, WsHeader* hdr, int vec) {
+    double t, WsHeader* hdr, int vec, SelectOut sel) {
     using S = Shape<E, RT, CTA>;
     __shared__ uint32_t xch[(RT > 32) ? CTA * E : 1];
     __shared__ uint32_t last_key[CTA];
@@ -163,7 +236,7 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
     const int warp = threadIdx.x >> 5;
     const int64_t row = (int64_t)blockIdx.x * S::ROWS + rloc;
     const bool row_ok = row < B;
-    const float* rrow = r + (row_ok ? row : 0) * ld;
+    const In* rrow = r + (row_ok ? row : 0) * ld;
     const double inv_t = 1.0 / t;
     // the row's budget: the shared k, or its own entry of k_rows (checked here: a
     // budget outside (0, n) gives b = NaN and a status bit)
@@ -317,11 +390,31 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
         const double tot = row_sum_d<E, RT, CTA>(sf, dred);
         if (tid == 0 && row_ok) sumf_out[row] = tot;
     }
+    if (sel.cnt != nullptr) {  // the same for every thread of the grid
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) c += (valid[e] && pv[e] > sel.eps) ? 1 : 0;
+        int total = 0;
+        int o = row_excl_scan_i<E, RT, CTA>(c, ired, &total);
+        if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                if (valid[e] && pv[e] > sel.eps) {
+                    if (o < sel.cap) {
+                        sel.idx[row * sel.cap + o] = tid * E + e;
+                        sel.val[row * sel.cap + o] = pv[e];
+                    }
+                    ++o;
+                }
+            }
+            if (tid == 0) sel.cnt[row] = total;
+        }
+    }
 }
 
-template <int E, int RT, int CTA>
+template <int E, int RT, int CTA, class In>
 __global__ void __launch_bounds__(CTA) onchip_backward_kernel(
-    const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
+    const In* __restrict__ r, int64_t ld, const double* __restrict__ b,
     const float* __restrict__ v, float* __restrict__ g, int64_t B, int n, double t, int vec) {
     using S = Shape<E, RT, CTA>;
     __shared__ float fred[S::NW];
@@ -335,7 +428,7 @@ __global__ void __launch_bounds__(CTA) onchip_backward_kernel(
     float rv[E], vv[E];
     bool valid[E];
     load_row<E>(r + off, n, tid, vec != 0, row_ok, rv, valid);
-    load_row<E>(v + off, n, tid, vec != 0, row_ok, vv, valid);
+    load_row<E>(v + off, n, tid, vec != 0, row_ok, vv, valid);  // (same validity)
     const Thr th = make_thr(row_ok ? b[row] : 0.0, t);
     float ax[E];
     float mloc = INFINITY;
@@ -367,30 +460,63 @@ __global__ void __launch_bounds__(CTA) onchip_backward_kernel(
     store_row<E>(g + off, n, tid, vec != 0, row_ok, gv);
 }
 
-template <int E, int RT, int CTA>
-cudaError_t launch_fwd(const float* r, int64_t ld, float* p, double* b, double* sumf, int64_t B,
+template <int E, int RT, int CTA, class In>
+cudaError_t launch_fwd(const In* r, int64_t ld, float* p, double* b, double* sumf, int64_t B,
                        int n, double k, const double* k_rows, double t, WsHeader* hdr, int vec,
-                       cudaStream_t st) {
+                       const SelectOut& sel, cudaStream_t st) {
     using S = Shape<E, RT, CTA>;
     const int64_t grid = (B + S::ROWS - 1) / S::ROWS;
     {
         ProfScope ps_("onchip_fwd", st);
-        onchip_forward_kernel<E, RT, CTA>
-        <<<(unsigned)grid, CTA, 0, st>>>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec);
+        onchip_forward_kernel<E, RT, CTA, In>
+        <<<(unsigned)grid, CTA, 0, st>>>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel);
     }
     return cudaGetLastError();
 }
 
-template <int E, int RT, int CTA>
-cudaError_t launch_bwd(const float* r, int64_t ld, const double* b, const float* v, float* g,
+template <int E, int RT, int CTA, class In>
+cudaError_t launch_bwd(const In* r, int64_t ld, const double* b, const float* v, float* g,
                        int64_t B, int n, double t, int vec, cudaStream_t st) {
     using S = Shape<E, RT, CTA>;
     const int64_t grid = (B + S::ROWS - 1) / S::ROWS;
     {
         ProfScope ps_("onchip_bwd", st);
-        onchip_backward_kernel<E, RT, CTA><<<(unsigned)grid, CTA, 0, st>>>(r, ld, b, v, g, B, n, t, vec);
+        onchip_backward_kernel<E, RT, CTA, In><<<(unsigned)grid, CTA, 0, st>>>(r, ld, b, v, g, B, n, t, vec);
     }
     return cudaGetLastError();
+}
+
+template <class In>
+cudaError_t onchip_forward_any(const In* r, int64_t ld, float* p, double* b, double* sumf,
+                               int64_t B, int n, double k, const double* k_rows, double t,
+                               WsHeader* hdr, int vec, const SelectOut& sel, cudaStream_t st) {
+    switch (onchip_npad(n)) {
+        case 32: return launch_fwd<1, 32, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        case 64: return launch_fwd<2, 32, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        case 128: return launch_fwd<4, 32, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        case 256: return launch_fwd<8, 32, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        case 512: return launch_fwd<8, 64, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        case 1024: return launch_fwd<8, 128, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        case 2048: return launch_fwd<8, 256, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        case 4096: return launch_fwd<8, 512, 512, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <class In>
+cudaError_t onchip_backward_any(const In* r, int64_t ld, const double* b, const float* v, float* g,
+                                int64_t B, int n, double t, int vec, cudaStream_t st) {
+    switch (onchip_npad(n)) {
+        case 32: return launch_bwd<1, 32, 256, In>(r, ld, b, v, g, B, n, t, vec, st);
+        case 64: return launch_bwd<2, 32, 256, In>(r, ld, b, v, g, B, n, t, vec, st);
+        case 128: return launch_bwd<4, 32, 256, In>(r, ld, b, v, g, B, n, t, vec, st);
+        case 256: return launch_bwd<8, 32, 256, In>(r, ld, b, v, g, B, n, t, vec, st);
+        case 512: return launch_bwd<8, 64, 256, In>(r, ld, b, v, g, B, n, t, vec, st);
+        case 1024: return launch_bwd<8, 128, 256, In>(r, ld, b, v, g, B, n, t, vec, st);
+        case 2048: return launch_bwd<8, 256, 256, In>(r, ld, b, v, g, B, n, t, vec, st);
+        case 4096: return launch_bwd<8, 512, 512, In>(r, ld, b, v, g, B, n, t, vec, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -404,32 +530,34 @@ int onchip_npad(int64_t n) {
 cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,
                                   int64_t B, int n, double k, const double* k_rows, double t,
                                   WsHeader* hdr, int vec, cudaStream_t st) {
-    switch (onchip_npad(n)) {
-        case 32: return launch_fwd<1, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        case 64: return launch_fwd<2, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        case 128: return launch_fwd<4, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        case 256: return launch_fwd<8, 32, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        case 512: return launch_fwd<8, 64, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        case 1024: return launch_fwd<8, 128, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        case 2048: return launch_fwd<8, 256, 256>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        case 4096: return launch_fwd<8, 512, 512>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, st);
-        default: return cudaErrorInvalidValue;
-    }
+    return onchip_forward_any<float>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec,
+                                     SelectOut{nullptr, nullptr, nullptr, 0, 0.f}, st);
 }
 
 cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
                                    float* g, int64_t B, int n, double t, int vec, cudaStream_t st) {
-    switch (onchip_npad(n)) {
-        case 32: return launch_bwd<1, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
-        case 64: return launch_bwd<2, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
-        case 128: return launch_bwd<4, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
-        case 256: return launch_bwd<8, 32, 256>(r, ld, b, v, g, B, n, t, vec, st);
-        case 512: return launch_bwd<8, 64, 256>(r, ld, b, v, g, B, n, t, vec, st);
-        case 1024: return launch_bwd<8, 128, 256>(r, ld, b, v, g, B, n, t, vec, st);
-        case 2048: return launch_bwd<8, 256, 256>(r, ld, b, v, g, B, n, t, vec, st);
-        case 4096: return launch_bwd<8, 512, 512>(r, ld, b, v, g, B, n, t, vec, st);
-        default: return cudaErrorInvalidValue;
-    }
+    return onchip_backward_any<float>(r, ld, b, v, g, B, n, t, vec, st);
+}
+
+cudaError_t launch_onchip_router(const void* r, int bf16, int64_t ld, float* p, double* b,
+                                 int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
+                                 int32_t* sel_idx, float* sel_val, int32_t* sel_cnt, int cap,
+                                 float eps, cudaStream_t st) {
+    const SelectOut sel{sel_idx, sel_val, sel_cnt, cap, eps};
+    if (bf16)
+        return onchip_forward_any<uint16_t>(static_cast<const uint16_t*>(r), ld, p, b, nullptr, B,
+                                            n, k, nullptr, t, hdr, vec, sel, st);
+    return onchip_forward_any<float>(static_cast<const float*>(r), ld, p, b, nullptr, B, n, k,
+                                     nullptr, t, hdr, vec, sel, st);
+}
+
+cudaError_t launch_onchip_backward_router(const void* r, int bf16, int64_t ld, const double* b,
+                                          const float* v, float* g, int64_t B, int n, double t,
+                                          int vec, cudaStream_t st) {
+    if (bf16)
+        return onchip_backward_any<uint16_t>(static_cast<const uint16_t*>(r), ld, b, v, g, B, n, t,
+                                             vec, st);
+    return onchip_backward_any<float>(static_cast<const float*>(r), ld, b, v, g, B, n, t, vec, st);
 }
 
 }  // namespace lapsum
