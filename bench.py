@@ -351,13 +351,17 @@ def main():
         rd = torch.from_numpy(rr).to(dev).to(torch.bfloat16)
         vd = torch.from_numpy(vv).to(dev)
         ws = L.Workspace(wk.B, wk.n, wk.k, "fullsort", dev)
-        out = {}
+        outs = (torch.empty((wk.B, wk.n), device=dev),
+                torch.empty(wk.B, dtype=torch.float64, device=dev),
+                torch.empty((wk.B, 16), dtype=torch.int32, device=dev),
+                torch.empty((wk.B, 16), device=dev), torch.empty(wk.B, dtype=torch.int32, device=dev))
+        gd = torch.empty((wk.B, wk.n), device=dev)
 
         def fwd():
-            out["fw"] = L.forward_router(rd, wk.k, wk.t, eps=1e-3, cap=16, ws=ws)
+            L.forward_router(rd, wk.k, wk.t, eps=1e-3, cap=16, ws=ws, out=outs)
 
         def bwd():
-            out["g"] = L.backward_router(rd, out["fw"][1], vd, wk.t)
+            L.backward_router(rd, outs[1], vd, wk.t, g=gd)
 
         for _ in range(3):
             fwd()

@@ -358,22 +358,33 @@ def _router_rows(x: torch.Tensor) -> torch.Tensor:
 
 
 def forward_router(r: torch.Tensor, k: float, t: float, eps: float = None, cap: int = None,
-                   ws: Workspace = None):
+                   ws: Workspace = None, out=None):
     """Router form for rows of n <= 4096 (lapsum_forward_router): r is float32 or
     bfloat16.  Returns (p, b), or with eps and cap also (idx, vals, cnt): per row
-    the positions and values of p > eps (at most cap, ascending) and their count."""
+    the positions and values of p > eps (at most cap, ascending) and their count;
+    list slots past the count are left as they were.  ``out`` may hold the
+    output tensors to fill: (p, b) or (p, b, idx, vals, cnt), p with r's row
+    stride."""
     r2 = _router_rows(r)
     B, n = r2.shape
     ld = r2.stride(0) if B > 1 else n
     if ws is None or not ws.fits(B, n, 0.5 * n, "fullsort"):
         ws = Workspace(B, n, 0.5 * n, "fullsort", r2.device)
-    p = torch.empty((B, ld), dtype=torch.float32, device=r2.device)[:, :n]
-    b = torch.empty(B, dtype=torch.float64, device=r2.device)
     want = eps is not None
-    if want:
-        idx = torch.full((B, cap), -1, dtype=torch.int32, device=r2.device)
-        vals = torch.zeros((B, cap), dtype=torch.float32, device=r2.device)
-        cnt = torch.empty(B, dtype=torch.int32, device=r2.device)
+    if out is not None:
+        p, b = out[0], out[1]
+        _check_out(p, r2, ld, "p")
+        if want:
+            idx, vals, cnt = out[2], out[3], out[4]
+            if idx.shape != (B, cap) or vals.shape != (B, cap) or cnt.numel() != B:
+                raise ValueError("selection outputs must be (B, cap), (B, cap) and (B,)")
+    else:
+        p = torch.empty((B, ld), dtype=torch.float32, device=r2.device)[:, :n]
+        b = torch.empty(B, dtype=torch.float64, device=r2.device)
+        if want:
+            idx = torch.empty((B, cap), dtype=torch.int32, device=r2.device)
+            vals = torch.empty((B, cap), dtype=torch.float32, device=r2.device)
+            cnt = torch.empty(B, dtype=torch.int32, device=r2.device)
     _check(_lib().lapsum_forward_router(
         r2.data_ptr(), _DTYPES[r2.dtype], ld, p.data_ptr(), b.data_ptr(), B, n, float(k),
         float(t), float(eps) if want else 0.0, int(cap) if want else 0,
@@ -385,14 +396,18 @@ def forward_router(r: torch.Tensor, k: float, t: float, eps: float = None, cap: 
     return (p, b, idx, vals, cnt) if want else (p, b)
 
 
-def backward_router(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float):
+def backward_router(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float,
+                    g: torch.Tensor = None):
     """g (float32) for router scores r (float32 or bfloat16), n <= 4096."""
     r2 = _router_rows(r)
     B, n = r2.shape
     v2 = v.reshape(B, n).to(torch.float32).contiguous()
     if r2.stride(0) != n and B > 1:
         r2 = r2.contiguous()
-    g = torch.empty((B, n), dtype=torch.float32, device=r2.device)
+    if g is None:
+        g = torch.empty((B, n), dtype=torch.float32, device=r2.device)
+    elif g.shape != (B, n) or g.dtype != torch.float32 or not g.is_contiguous():
+        raise ValueError("g must be a contiguous float32 (B, n) tensor")
     _check(_lib().lapsum_backward_router(r2.data_ptr(), _DTYPES[r2.dtype], n, b.data_ptr(),
                                          v2.data_ptr(), g.data_ptr(), B, n, float(t),
                                          _stream_ptr(r2.device)), "lapsum_backward_router")

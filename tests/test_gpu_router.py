@@ -66,7 +66,10 @@ def test_router_selection_list(cuda_device, dtype, n, eps, cap):
     B, k, t = 40, 8.0, 0.05
     r, _ = random_rows(403 + n, B, n)
     rt = torch.from_numpy(r).to(dtype).cuda()
-    p, b, idx, vals, cnt = L.forward_router(rt, k, t, eps=eps, cap=cap)
+    out = (torch.empty((B, n), device="cuda"), torch.empty(B, dtype=torch.float64, device="cuda"),
+           torch.full((B, cap), -1, dtype=torch.int32, device="cuda"),
+           torch.zeros((B, cap), device="cuda"), torch.empty(B, dtype=torch.int32, device="cuda"))
+    p, b, idx, vals, cnt = L.forward_router(rt, k, t, eps=eps, cap=cap, out=out)
     torch.cuda.synchronize()
     p, idx, vals, cnt = p.cpu().numpy(), idx.cpu().numpy(), vals.cpu().numpy(), cnt.cpu().numpy()
     for i in range(B):
