@@ -74,6 +74,8 @@ def configure(lib):
     lib.lso_binom_ranks.restype = None
     lib.lso_binom_ranks.argtypes = [ctypes.c_int64, ctypes.c_double, ctypes.c_double, _i64p,
                                     _i64p]
+    lib.lso_hard_topk.restype = ctypes.c_int
+    lib.lso_hard_topk.argtypes = [_dp, ctypes.c_int64, ctypes.c_double, _dp, _dp]
     lib.lso_bracket_from_sample.restype = None
     lib.lso_bracket_from_sample.argtypes = [_dp, ctypes.c_int64, ctypes.c_int64,
                                             ctypes.c_int64, _dp, _dp]
@@ -217,3 +219,15 @@ def bracket_from_sample(y, l: int, h: int):
     _lib().lso_bracket_from_sample(_ptr(a), a.size, int(l), int(h), ctypes.byref(aL),
                                    ctypes.byref(aR))
     return aL.value, aR.value
+
+
+def hard_topk(r, k: float):
+    """Zero-temperature limit: (b, p) with p the hard top-k mask, tied scores at the
+    boundary sharing the remaining budget (lso_hard_topk)."""
+    a = _f64(r)
+    b = ctypes.c_double(0.0)
+    p = np.empty_like(a)
+    st = _lib().lso_hard_topk(_ptr(a), a.size, float(k), ctypes.byref(b), _ptr(p))
+    if st != 0:
+        raise OracleError(f"lso_hard_topk failed with status {st}")
+    return b.value, p

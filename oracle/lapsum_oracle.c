@@ -333,3 +333,50 @@ void lso_bracket_from_sample(const double* y, int64_t m, int64_t l, int64_t h, d
     *aL = (h <= m) ? s[m - h] : -INFINITY;
     free(s);
 }
+
+/* ---------------------------------------------------------------------------
+ * Zero-temperature limit (hard top-k).  Section 2.3 of the pages ties the
+ * method to DFTopK, whose threshold is the midpoint of the k-th and (k+1)-th
+ * largest scores, as the t -> 0 limit.  The limit of the balance equation,
+ * written out here for any real k in (0, n):
+ *   c = the ceil(k)-th largest score, a = #{r > c}, m = #{r = c}
+ *   (so a < k <= a + m);
+ *   - k < a + m: b = c, and the scores equal to c share the remaining budget,
+ *     p = (k - a)/m each (sigma of the common limit of (c - b)/t);
+ *   - k = a + m (k an integer at a gap of the sorted order): b is the
+ *     midpoint of c and d = the largest score below c, and p is the 0/1 mask
+ *     of the scores above b.
+ * Either way sum p = k.  The sort is plain qsort on a copy.
+ * ------------------------------------------------------------------------- */
+int lso_hard_topk(const double* r, int64_t n, double k, double* b_out, double* p) {
+    if (r == NULL || n < 1 || !(k > 0.0) || !(k < (double)n)) return LSO_EINVAL;
+    for (int64_t i = 0; i < n; ++i)
+        if (!isfinite(r[i])) return LSO_ENONFINITE;
+    double* s = (double*)malloc((size_t)n * sizeof(double));
+    if (s == NULL) return LSO_EINVAL;
+    memcpy(s, r, (size_t)n * sizeof(double));
+    qsort(s, (size_t)n, sizeof(double), cmp_double);  /* ascending */
+    const int64_t rank = (int64_t)ceil(k);              /* 1-based, from the top */
+    const double c = s[n - rank];
+    int64_t a = 0, m = 0;
+    double d = -INFINITY;
+    for (int64_t i = 0; i < n; ++i) {
+        if (s[i] > c) ++a;
+        else if (s[i] == c) ++m;
+        else if (s[i] > d) d = s[i];
+    }
+    free(s);
+    double b, frac;
+    if (k < (double)(a + m)) {
+        b = c;
+        frac = (k - (double)a) / (double)m;
+    } else {
+        b = 0.5 * (c + d);
+        frac = 1.0;  /* every score equal to c lies above b */
+    }
+    *b_out = b;
+    if (p != NULL)
+        for (int64_t i = 0; i < n; ++i)
+            p[i] = r[i] > c ? 1.0 : (r[i] == c ? frac : 0.0);
+    return LSO_OK;
+}

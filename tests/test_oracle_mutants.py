@@ -47,6 +47,13 @@ MUTANTS = [
      [pins.test_fold_reconstructs_budget_inside_bracket]),
     ("splitmix_constant", "0xBF58476D1CE4E5B9ull", "0xBF58476D1CE4E5B8ull",
      [pins.test_splitmix64_published_vector]),
+    ("hard_rank_floor", "(int64_t)ceil(k);", "(int64_t)floor(k) + 1;",
+     [pins.test_hard_topk_worked_cases]),
+    ("hard_tie_share", "frac = (k - (double)a) / (double)m;",
+     "frac = (k - (double)a) / (double)(m + 1);",
+     [pins.test_hard_topk_worked_cases]),
+    ("hard_midpoint", "b = 0.5 * (c + d);", "b = c;",
+     [lambda: pins.test_hard_topk_is_the_soft_solution_at_tiny_temperature(0, 40, 7.0, 0.0)]),
     ("order_stat_index", "*aR = (l >= 1) ? s[m - l] : INFINITY;",
      "*aR = (l >= 1) ? s[m - l - 1] : INFINITY;",
      [pins.test_bracket_order_statistics]),

@@ -361,3 +361,66 @@ def test_bracket_order_statistics():
         aL, aR = oracle.bracket_from_sample(y, l, h)
         assert aR == (desc[l - 1] if l >= 1 else math.inf)
         assert aL == (desc[h - 1] if h <= y.size else -math.inf)
+
+
+# ---------------------------------------------------------------------------
+# Zero-temperature limit (hard top-k): "Fast LapSum: Exact Differentiable Top-k
+# at Million Scale" (gist.science explainer pages), section 2.3: DFTopK's
+# midpoint threshold is the t -> 0 limit of LapSum.  Pinned by hand-worked
+# cases, by the soft oracle itself at a temperature far below the gaps (a
+# different code path: bisection on the smooth budget), and by invariants.
+# ---------------------------------------------------------------------------
+
+def test_hard_topk_worked_cases():
+    # integer k at a gap: midpoint of the k-th and (k+1)-th largest, 0/1 mask
+    b, p = oracle.hard_topk([5.0, 4.0, 3.0, 1.0], 2.0)
+    assert b == 3.5 and list(p) == [1.0, 1.0, 0.0, 0.0]
+    # a tie group straddles the budget: b is the tied value, the group shares
+    # the remaining budget equally
+    b, p = oracle.hard_topk([3.0, 2.0, 2.0, 2.0, 1.0], 2.0)
+    assert b == 2.0 and np.allclose(p, [1.0, 1 / 3, 1 / 3, 1 / 3, 0.0], rtol=0, atol=1e-15)
+    # a fractional budget lands on one score
+    b, p = oracle.hard_topk([5.0, 4.0, 3.0], 1.5)
+    assert b == 4.0 and list(p) == [1.0, 0.5, 0.0]
+    # the whole tie group inside the budget: a gap below it
+    b, p = oracle.hard_topk([7.0, 6.0, 6.0, 2.0, 0.0], 3.0)
+    assert b == 4.0 and list(p) == [1.0, 1.0, 1.0, 0.0, 0.0]
+
+
+@pytest.mark.parametrize("seed,n,k,grid", [(0, 40, 7.0, 0.0), (1, 25, 12.0, 0.25),
+                                           (2, 60, 13.5, 0.0), (3, 33, 4.25, 0.5)])
+def test_hard_topk_is_the_soft_solution_at_tiny_temperature(seed, n, k, grid):
+    rng = np.random.default_rng(seed)
+    r = rng.standard_normal(n)
+    if grid > 0:
+        r = np.round(r / grid) * grid  # ties, at the boundary for some k
+    b_h, p_h = oracle.hard_topk(r, k)
+    gaps = np.diff(np.unique(r))
+    t = float(np.min(gaps)) / 80.0    # every neighbour weight below e^-80
+    b_s = oracle.solve_b(r, k, t)
+    p_s = oracle.emit_p(r, b_s, t)
+    assert abs(b_s - b_h) <= 3 * t   # the soft b sits within a few t of the limit
+    # p at a score equal to b moves by db/(2t): allow a few fp64 ulps of b over t
+    tol_p = max(1e-12, 8 * np.finfo(float).eps * max(1.0, abs(b_s)) / t)
+    assert np.max(np.abs(p_s - p_h)) <= tol_p
+    assert abs(np.sum(p_h) - k) <= 1e-12
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_hard_topk_invariants(seed):
+    rng = np.random.default_rng(seed)
+    n = 50
+    r = np.round(rng.standard_normal(n) * 4) / 4
+    for k in (1.0, 9.0, 17.5, 48.75):
+        b, p = oracle.hard_topk(r, k)
+        assert abs(np.sum(p) - k) <= 1e-12
+        assert np.all((p >= 0) & (p <= 1))
+        order = np.argsort(r)
+        assert np.all(np.diff(p[order]) >= 0)          # monotone in r
+        perm = rng.permutation(n)
+        b2, p2 = oracle.hard_topk(r[perm], k)          # permutation
+        assert b2 == b and np.array_equal(p2, p[perm])
+        b3, p3 = oracle.hard_topk(r + 2.5, k)          # shift
+        assert b3 == b + 2.5 and np.array_equal(p3, p)
+        b4, p4 = oracle.hard_topk(-r, n - k)           # mirror
+        assert b4 == -b and np.allclose(p4, 1.0 - p, rtol=0, atol=1e-15)
