@@ -127,6 +127,27 @@ int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v,
                     int64_t B, int64_t n, double t, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Zero-temperature limit (hard top-k).  "Fast LapSum: Exact Differentiable
+ * Top-k at Million Scale" (gist.science explainer pages), section 2.3, names
+ * DFTopK's threshold -- the midpoint of the k-th and (k+1)-th largest scores
+ * -- as LapSum's limit at t -> 0.  For each row, with c the ceil(k)-th largest
+ * score, a = #{r > c} and m = #{r = c} (-0 and +0 are one value):
+ *   k < a + m:  b = c, p = 1 above c, (k - a)/m at c, 0 below;
+ *   k = a + m:  b = (c + d)/2 with d the largest score below c, p the 0/1
+ *               mask of the scores above b.
+ * So sum p = k, as at every t > 0 (ties at the boundary share the remaining
+ * budget instead of a fixed 1/2).  k is real in (0, n); n >= 2.  Solvers: the
+ * on-chip sort for n <= 4096 and the radix full sort above (LAPSUM_PATH_AUTO
+ * or LAPSUM_PATH_FULLSORT), or LAPSUM_PATH_RADIX; the bracketing paths return
+ * LAPSUM_EINVAL.  ws: lapsum_workspace_bytes(B, n, k, LAPSUM_PATH_FULLSORT)
+ * (or LAPSUM_PATH_RADIX when that path is asked for).  Rows with a non-finite
+ * score get b = NaN and p = NaN (status LAPSUM_ENONFINITE).  The limit has no
+ * useful gradient (p is piecewise constant in r); there is no backward.
+ */
+int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t B, int64_t n,
+                        double k, int path, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Router form for short rows (n <= 4096, the on-chip sort), e.g. the scores of
  * a mixture-of-experts router: scores r of type `dtype` (fp32, or bf16 bit
  * patterns widened exactly to fp32), p (fp32) and b (fp64) as lapsum_forward,

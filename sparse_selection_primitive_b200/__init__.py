@@ -114,6 +114,9 @@ def _lib():
         lib.lapsum_backward_kt.restype = ctypes.c_int
         lib.lapsum_backward_kt.argtypes = [_vp, _c_i64, _vp, _vp, _c_i64, _c_i64, ctypes.c_double,
                                            _vp, _vp, _vp, ctypes.c_size_t, _vp]
+        lib.lapsum_forward_hard.restype = ctypes.c_int
+        lib.lapsum_forward_hard.argtypes = [_vp, _c_i64, _vp, _vp, _c_i64, _c_i64, ctypes.c_double,
+                                            ctypes.c_int, _vp, ctypes.c_size_t, _vp]
         lib.lapsum_forward_router.restype = ctypes.c_int
         lib.lapsum_forward_router.argtypes = [_vp, ctypes.c_int, _c_i64, _vp, _vp, _c_i64, _c_i64,
                                               ctypes.c_double, ctypes.c_double, ctypes.c_float,
@@ -342,6 +345,26 @@ def backward(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float, ws: Wo
                                       g.data_ptr(), B, n, float(t), ws.ptr, ws.nbytes,
                                       _stream_ptr(r2.device)), "lapsum_backward")
     return g[0] if squeeze else g
+
+
+def hard_topk(r: torch.Tensor, k: float, path="auto", ws: Workspace = None):
+    """Zero-temperature limit (lapsum_forward_hard): (p, b) per row of r (float32
+    CUDA): p = 1 above the boundary score c = the ceil(k)-th largest, 0 below,
+    and the scores equal to c share the remaining budget (sum p = k)."""
+    squeeze = r.dim() == 1
+    r2 = _as_rows(r)
+    B, n = r2.shape
+    ld = _ld(r2)
+    code = _path_code(path)
+    wpath = "fullsort" if (code & 0xFF) == PATHS["auto"] else code
+    if ws is None or not ws.fits(B, n, k, wpath):
+        ws = Workspace(B, n, k, wpath, r2.device)
+    p = _like_rows(r2, ld)
+    b = torch.empty(B, dtype=torch.float64, device=r2.device)
+    _check(_lib().lapsum_forward_hard(r2.data_ptr(), ld, p.data_ptr(), b.data_ptr(), B, n,
+                                      float(k), code, ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
+           "lapsum_forward_hard")
+    return (p[0] if squeeze else p), b
 
 
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}

@@ -385,6 +385,48 @@ int lapsum_forward(const float* r, int64_t ld, float* p, double* b, double* sum_
                         nullptr, 0, stream);
 }
 
+int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t B, int64_t n,
+                        double k, int path, void* ws, size_t ws_bytes, void* stream) {
+    if (r == nullptr || p == nullptr || b == nullptr) return LAPSUM_EINVAL;
+    if (B < 1 || n < 2 || ld < n || n > INT32_MAX) return LAPSUM_EINVAL;
+    if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
+    int rp = resolve_path(n, (path & 0xff) == LAPSUM_PATH_AUTO ? LAPSUM_PATH_FULLSORT : path);
+    if ((path & ~0xff) != 0 || (rp != LAPSUM_PATH_FULLSORT && rp != LAPSUM_PATH_RADIX))
+        return LAPSUM_EINVAL;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const Layout L = make_layout(B, n, rp);
+    if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* w = static_cast<char*>(ws);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(w + L.header);
+    RowState* rows = reinterpret_cast<RowState*>(w + L.rows);
+    const int vec = (aligned16(r) && aligned16(p) && (ld % 4) == 0) ? 1 : 0;
+    if (rp == LAPSUM_PATH_FULLSORT)
+        return cuda_status(launch_onchip_hard(r, ld, p, b, B, (int)n, k, hdr, vec, st));
+    cudaError_t e = cudaMemsetAsync(rows, 0, (size_t)B * sizeof(RowState), st);
+    if (e != cudaSuccess) return LAPSUM_ECUDA;
+    RadixBuffers rb;
+    rb.keys[0] = reinterpret_cast<uint32_t*>(w + L.keys0);
+    rb.keys[1] = reinterpret_cast<uint32_t*>(w + L.keys1);
+    rb.seg_hist = reinterpret_cast<uint32_t*>(w + L.seg_hist);
+    rb.tile_hist = reinterpret_cast<uint32_t*>(w + L.tile_hist);
+    rb.plan = reinterpret_cast<int32_t*>(w + L.plan);
+    for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
+        const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+        RadixBuffers sub = rb;
+        sub.keys[0] += r0 * n;
+        sub.keys[1] += r0 * n;
+        sub.seg_hist += r0 * 1024;
+        sub.tile_hist += r0 * 256 * radix_tiles(n);
+        sub.plan += r0 * 8;
+        e = launch_radix_sort_rows(r + r0 * ld, ld, nb, n, sub, rows + r0, hdr, st);
+        if (e == cudaSuccess)
+            e = launch_rowhard_sorted_keys(sub, nb, n, k, r + r0 * ld, ld, p + r0 * ld, b + r0,
+                                           rows + r0, vec, st);
+    }
+    return cuda_status(e);
+}
+
 int lapsum_forward_router(const void* r, int dtype, int64_t ld, float* p, double* b, int64_t B,
                           int64_t n, double k, double t, float eps, int32_t cap, int32_t* sel_idx,
                           float* sel_p, int32_t* sel_cnt, void* ws, size_t ws_bytes,

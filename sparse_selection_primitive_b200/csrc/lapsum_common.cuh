@@ -70,7 +70,10 @@ struct RowState {
     float sub_aL, sub_aR;      // sub-bracket [sub_aL, sub_aR) = that bin's edges
     int32_t sub_hasR, pad1;
     double sub_SL, sub_SR, sub_cntR;  // tails of the sub-bracket
-    double scratch[37];       // kernel-to-kernel scalars (phase timestamps)
+    float hard_c;             // zero-temperature mode: the boundary score c and
+    int32_t pad2;             //   the share p of the scores equal to c
+    double hard_frac;
+    double scratch[35];       // kernel-to-kernel scalars (phase timestamps)
 };
 static_assert(sizeof(RowState) == 512, "row records are 512-byte slots of the workspace");
 static_assert(sizeof(RowState) <= 512, "row record fits its slot");

@@ -45,6 +45,9 @@ cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* 
                                   WsHeader* hdr, int vec, cudaStream_t st);
 cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
                                    float* g, int64_t B, int n, double t, int vec, cudaStream_t st);
+// Zero-temperature limit (hard top-k) of rows of n <= 4096: sort, boundary group, p.
+cudaError_t launch_onchip_hard(const float* r, int64_t ld, float* p, double* b, int64_t B, int n,
+                               double k, WsHeader* hdr, int vec, cudaStream_t st);
 // The router form: scores as fp32 (bf16 = 0) or bf16 bit patterns (bf16 = 1),
 // and optionally (sel_cnt != null) the per-row list of positions and values of
 // p > eps (at most cap per row) with its count.
@@ -72,6 +75,12 @@ cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_
 cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
                                         const double* k_rows, double t, double* b, RowState* rows,
                                         WsHeader* hdr, cudaStream_t st);
+// Zero-temperature limit of every row from its sorted keys (one CTA per row),
+// then p from r (one CTA per tile); b, the boundary score and its share go to
+// the row records.
+cudaError_t launch_rowhard_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
+                                       const float* r, int64_t ld, float* p, double* b,
+                                       RowState* rows, int vec, cudaStream_t st);
 
 // --- streaming kernels over long rows ----------------------------------------
 constexpr int kStreamTile = 4096;  // elements per CTA tile of the streaming kernels

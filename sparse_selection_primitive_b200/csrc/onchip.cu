@@ -412,6 +412,90 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
     }
 }
 
+// Zero-temperature limit ("Fast LapSum: Exact Differentiable Top-k at Million
+// Scale", gist.science explainer pages, section 2.3: DFTopK's midpoint
+// threshold is LapSum at t -> 0).  After the sort, c is the rank-th largest
+// score (rank = ceil(k)), a = #{r > c}, m = #{r = c}: when k < a + m the
+// scores equal to c share the remaining budget, p = (k - a)/m, and b = c;
+// otherwise (k = a + m) b is the midpoint of c and the largest score below c,
+// and p is the 0/1 mask.  -0 is read as +0, so equal values are one group.
+template <int E, int RT, int CTA>
+__global__ void __launch_bounds__(CTA) onchip_hard_kernel(
+    const float* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
+    int64_t B, int n, double k, int rank, WsHeader* hdr, int vec) {
+    using S = Shape<E, RT, CTA>;
+    __shared__ uint32_t xch[(RT > 32) ? CTA * E : 1];
+    __shared__ int ired[S::NW];
+    __shared__ uint32_t row_key[S::ROWS][2];  // c, then the largest key below c
+    __shared__ int row_flag[S::ROWS];
+    __shared__ double row_val[S::ROWS][2];    // b, share of the scores equal to c
+    const int rloc = threadIdx.x / RT;
+    const int tid = threadIdx.x % RT;
+    const int64_t row = (int64_t)blockIdx.x * S::ROWS + rloc;
+    const bool row_ok = row < B;
+    if (tid == 0) row_flag[rloc] = 0;
+    float orig[E];
+    bool valid[E];
+    load_row<E>(r + (row_ok ? row : 0) * ld, n, tid, vec != 0, row_ok, orig, valid);
+    uint32_t key[E];
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        orig[e] += 0.f;  // -0 -> +0
+        key[e] = valid[e] ? to_key(orig[e]) : kPadKey;
+        bad |= valid[e] && !finite_f(orig[e]);
+    }
+    row_sync<E, RT, CTA>();
+    if (bad) atomicOr(&row_flag[rloc], 1);
+    bitonic_sort_row<E, RT, CTA>(key, tid, xch);
+    const int q = n - rank;  // ascending position of c
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (tid * E + e == q) row_key[rloc][0] = key[e];
+    row_sync<E, RT, CTA>();
+    const uint32_t ck = row_key[rloc][0];
+    int lt = 0, eq = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const bool in = tid * E + e < n;
+        lt += (in && key[e] < ck) ? 1 : 0;
+        eq += (in && key[e] == ck) ? 1 : 0;
+    }
+    lt = row_sum_i<E, RT, CTA>(lt, ired);
+    eq = row_sum_i<E, RT, CTA>(eq, ired);
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (tid * E + e == lt - 1) row_key[rloc][1] = key[e];
+    row_sync<E, RT, CTA>();
+    if (tid == 0) {
+        const float c = from_key(ck);
+        const double a = (double)(n - lt - eq), m = (double)eq;
+        double bb, frac;
+        if (k < a + m) {
+            bb = (double)c;
+            frac = (k - a) / m;
+        } else {
+            bb = 0.5 * ((double)c + (double)from_key(row_key[rloc][1]));
+            frac = 1.0;
+        }
+        if (row_flag[rloc] || !row_ok) {
+            bb = nan("");
+            if (row_ok) set_status(hdr, kDevNonFinite);
+        }
+        row_val[rloc][0] = bb;
+        row_val[rloc][1] = frac;
+        if (row_ok) b_out[row] = bb;
+    }
+    row_sync<E, RT, CTA>();
+    const double bb = row_val[rloc][0];
+    const float c = from_key(ck), share = (float)row_val[rloc][1];
+    float pv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        pv[e] = isnan(bb) ? bb : (orig[e] > c ? 1.f : (orig[e] == c ? share : 0.f));
+    store_row<E>(p + (row_ok ? row : 0) * ld, n, tid, vec != 0, row_ok, pv);
+}
+
 template <int E, int RT, int CTA, class In>
 __global__ void __launch_bounds__(CTA) onchip_backward_kernel(
     const In* __restrict__ r, int64_t ld, const double* __restrict__ b,
@@ -503,6 +587,19 @@ cudaError_t onchip_forward_any(const In* r, int64_t ld, float* p, double* b, dou
     }
 }
 
+template <int E, int RT, int CTA>
+cudaError_t launch_hard(const float* r, int64_t ld, float* p, double* b, int64_t B, int n,
+                        double k, int rank, WsHeader* hdr, int vec, cudaStream_t st) {
+    using S = Shape<E, RT, CTA>;
+    const int64_t grid = (B + S::ROWS - 1) / S::ROWS;
+    {
+        ProfScope ps_("onchip_hard", st);
+        onchip_hard_kernel<E, RT, CTA><<<(unsigned)grid, CTA, 0, st>>>(r, ld, p, b, B, n, k, rank,
+                                                                       hdr, vec);
+    }
+    return cudaGetLastError();
+}
+
 template <class In>
 cudaError_t onchip_backward_any(const In* r, int64_t ld, const double* b, const float* v, float* g,
                                 int64_t B, int n, double t, int vec, cudaStream_t st) {
@@ -537,6 +634,22 @@ cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* 
 cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
                                    float* g, int64_t B, int n, double t, int vec, cudaStream_t st) {
     return onchip_backward_any<float>(r, ld, b, v, g, B, n, t, vec, st);
+}
+
+cudaError_t launch_onchip_hard(const float* r, int64_t ld, float* p, double* b, int64_t B, int n,
+                               double k, WsHeader* hdr, int vec, cudaStream_t st) {
+    const int rank = (int)ceil(k);
+    switch (onchip_npad(n)) {
+        case 32: return launch_hard<1, 32, 256>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        case 64: return launch_hard<2, 32, 256>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        case 128: return launch_hard<4, 32, 256>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        case 256: return launch_hard<8, 32, 256>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        case 512: return launch_hard<8, 64, 256>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        case 1024: return launch_hard<8, 128, 256>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        case 2048: return launch_hard<8, 256, 256>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        case 4096: return launch_hard<8, 512, 512>(r, ld, p, b, B, n, k, rank, hdr, vec, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_onchip_router(const void* r, int bf16, int64_t ld, float* p, double* b,

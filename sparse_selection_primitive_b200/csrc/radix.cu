@@ -293,7 +293,118 @@ __global__ void __launch_bounds__(1024) rowsolve_keys_kernel(const uint32_t* __r
     }
 }
 
+// Zero-temperature limit of a sorted row (section 2.3 of the pages: DFTopK's
+// midpoint threshold is LapSum at t -> 0): c = the rank-th largest key, its
+// group of equal scores [lo, hi) found by two 1024-way searches of the sorted
+// keys (-0 and +0 read as one value), then b and the share of the group as in
+// the on-chip kernel.  One CTA per row.
+__device__ __forceinline__ uint32_t canon_key(uint32_t kk) {
+    return kk == 0x7fffffffu ? 0x80000000u : kk;  // the key of -0 as the key of +0
+}
+// First index in [lo, hi) whose canonical key is >= target (strict: > target),
+// or hi.  Every thread of the CTA calls it.
+__device__ int64_t block_lower_bound(const uint32_t* __restrict__ keys, int64_t lo, int64_t hi,
+                                     uint32_t target, bool strict) {
+    while (hi > lo) {
+        const int64_t step = (hi - lo + blockDim.x - 1) / blockDim.x;
+        const int64_t pos = lo + (int64_t)threadIdx.x * step;
+        bool below = false;
+        if (pos < hi) {
+            const uint32_t kk = canon_key(keys[pos]);
+            below = strict ? kk <= target : kk < target;
+        }
+        const int cnt = __syncthreads_count(below);  // probes before the answer
+        const int64_t nlo = cnt > 0 ? lo + (int64_t)(cnt - 1) * step + 1 : lo;
+        int64_t nhi = lo + (int64_t)cnt * step;
+        if (nhi > hi) nhi = hi;
+        lo = nlo;
+        hi = nhi;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(1024) rowhard_keys_kernel(const uint32_t* __restrict__ k0,
+                                                             const uint32_t* __restrict__ k1,
+                                                             int64_t n, double k, int64_t rank,
+                                                             const int32_t* __restrict__ plan,
+                                                             double* __restrict__ b_out,
+                                                             RowState* rows) {
+    const int64_t row = blockIdx.x;
+    const uint32_t* keys = (plan[row * 8 + 4] ? k1 : k0) + row * n;
+    const int64_t q = n - rank;
+    const uint32_t ck = canon_key(keys[q]);
+    const int64_t lo = block_lower_bound(keys, 0, q + 1, ck, false);
+    const int64_t hi = block_lower_bound(keys, q, n, ck, true);
+    if (threadIdx.x == 0) {
+        const float c = from_key(ck);
+        const double a = (double)(n - hi), m = (double)(hi - lo);
+        double b, frac;
+        if (k < a + m) {
+            b = (double)c;
+            frac = (k - a) / m;
+        } else {  // lo >= 1 here: k = a + m < n
+            b = 0.5 * ((double)c + (double)from_key(canon_key(keys[lo - 1])));
+            frac = 1.0;
+        }
+        if (rows[row].status & kDevNonFinite) b = nan("");
+        rows[row].b = b;
+        rows[row].hard_c = c;
+        rows[row].hard_frac = frac;
+        rows[row].path = LAPSUM_PATH_RADIX;
+        rows[row].attempts = 1;
+        b_out[row] = b;
+    }
+}
+
+// p of the zero-temperature limit: 1 above c, the share at c, 0 below; NaN rows
+// stay NaN.  One CTA per 4096-score tile.
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads) hard_emit_kernel(const float* __restrict__ r,
+                                                             int64_t ld, float* __restrict__ p,
+                                                             int64_t n, const RowState* rows) {
+    const int64_t row = blockIdx.y;
+    const RowState& rs = rows[row];
+    const float c = rs.hard_c, share = (float)rs.hard_frac;
+    const bool nan_row = isnan(rs.b);
+    const float* rr = r + row * ld;
+    float* pr = p + row * ld;
+    auto one = [&](float x) {
+        x += 0.f;
+        return nan_row ? __int_as_float(0x7fc00000) : (x > c ? 1.f : (x == c ? share : 0.f));
+    };
+    const int64_t base = (int64_t)blockIdx.x * 4096;
+    if (VEC && base + 4096 <= n) {
+        const float4* r4 = reinterpret_cast<const float4*>(rr + base);
+        float4* p4 = reinterpret_cast<float4*>(pr + base);
+        for (int i = threadIdx.x; i < 1024; i += kThreads) {
+            const float4 v = __ldcs(r4 + i);
+            __stcs(p4 + i, make_float4(one(v.x), one(v.y), one(v.z), one(v.w)));
+        }
+    } else {
+        for (int64_t i = base + threadIdx.x; i < base + 4096 && i < n; i += kThreads)
+            pr[i] = one(rr[i]);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_rowhard_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
+                                       const float* r, int64_t ld, float* p, double* b,
+                                       RowState* rows, int vec, cudaStream_t st) {
+    const int64_t rank = (int64_t)ceil(k);
+    {
+        ProfScope ps_("rowhard", st);
+        rowhard_keys_kernel<<<(unsigned)B, 1024, 0, st>>>(buf.keys[0], buf.keys[1], n, k, rank,
+                                                          buf.plan, b, rows);
+    }
+    const dim3 grid((unsigned)((n + 4095) / 4096), (unsigned)B);
+    {
+        ProfScope ps_("hard_emit", st);
+        if (vec) hard_emit_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, p, n, rows);
+        else hard_emit_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, p, n, rows);
+    }
+    return cudaGetLastError();
+}
 
 int64_t radix_tiles(int64_t n) { return (n + kRadixTile - 1) / kRadixTile; }
 
