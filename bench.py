@@ -343,6 +343,42 @@ def main():
                 res["table"]["bwd_without_support_ms"] = statistics.median(tp)
         return res
 
+    def hard_row(wk, peak_gbs):
+        """The zero-temperature limit (lapsum_forward_hard) on a workload's scores:
+        the on-chip sort for short rows, the radix sort for long ones."""
+        rr, _ = make_inputs(wk, seed=0)
+        rd = torch.from_numpy(rr).to(dev)
+        ws = L.Workspace(wk.B, wk.n, wk.k, "fullsort", dev)
+        for _ in range(3):
+            L.hard_topk(rd, wk.k, ws=ws)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            L.hard_topk(rd, wk.k, ws=ws)
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(graph):
+            L.hard_topk(rd, wk.k, ws=ws)
+        torch.cuda.synchronize(dev)
+        times = []
+        for _ in range(10):
+            flush_buf.zero_()
+            s_ev = torch.cuda.Event(enable_timing=True)
+            e_ev = torch.cuda.Event(enable_timing=True)
+            s_ev.record(stream)
+            graph.replay()
+            e_ev.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(s_ev.elapsed_time(e_ev))
+        ms = statistics.median(times)
+        del graph
+        return {"mode": "zero-temperature limit (forward only)",
+                "solver": "on-chip sort" if wk.n <= 4096 else "radix full sort",
+                "fwd_graph_ms": round(ms, 5), "fwd_elements_per_s": wk.elements / (ms / 1e3),
+                "path_frac_of_peak": 8 * wk.elements / (ms / 1e3) / 1e9 / peak_gbs}
+
     def router_bf16_row(peak_gbs):
         """The router shape through the router form: bf16 scores, p and the list of
         p > 1e-3 (at most 16 per row) in the forward, g from bf16 scores."""
@@ -525,6 +561,9 @@ def main():
         torch.cuda.empty_cache()
         table["moe_router_16384x256_bf16_select"] = router_bf16_row(peak_gbs)
         torch.cuda.empty_cache()
+        for name in ("moe_router_16384x256", "memory_select_256x65536"):
+            table[name + "_hard"] = hard_row(WORKLOADS[name], peak_gbs)
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
