@@ -88,3 +88,38 @@ def test_workspace_sizes(lib):
     # the radix path holds two key buffers; the bracket path holds two band buffers
     assert wb(256, 65536, 1024.0) >= 2 * 256 * 65536 * 4
     assert wb(1, 10**8, 1e5) >= 2 * 10**8 * 4
+
+
+def test_new_entry_points_reject_bad_arguments_on_host(lib):
+    """Per-row budgets, the router form and the zero-temperature limit validate
+    their arguments before any launch (no GPU needed)."""
+    ws = ctypes.c_void_p(256)
+    d = ctypes.c_void_p(4096)
+    vp = ctypes.c_void_p
+    rowk = lib.lapsum_forward_rowk
+    rowk.argtypes = [vp, ctypes.c_int64, vp, vp, vp, ctypes.c_int64, ctypes.c_int64, vp,
+                     ctypes.c_double, ctypes.c_int, vp, ctypes.c_size_t, vp, ctypes.c_size_t, vp]
+    assert rowk(d, 8, d, d, None, 1, 8, None, 0.1, 0, ws, 1 << 20, None, 0, None) == 1  # k NULL
+    assert rowk(d, 8, d, d, None, 1, 8, d, 0.0, 0, ws, 1 << 20, None, 0, None) == 1     # t <= 0
+    assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 2, ws, 1 << 20, None, 0, None) == 1     # bracket
+    assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 4, ws, 1 << 20, None, 0, None) == 1     # rowbracket
+    assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 0, None, 1 << 20, None, 0, None) == 2   # no ws
+    router = lib.lapsum_forward_router
+    router.argtypes = [vp, ctypes.c_int, ctypes.c_int64, vp, vp, ctypes.c_int64, ctypes.c_int64,
+                       ctypes.c_double, ctypes.c_double, ctypes.c_float, ctypes.c_int32, vp, vp,
+                       vp, vp, ctypes.c_size_t, vp]
+    ok = (d, 0, 8, d, d, 1, 8, 2.0, 0.1, 0.0, 0, None, None, None, ws, 1 << 20, None)
+    assert router(*ok[:1], 2, *ok[2:]) == 1                                   # unknown dtype
+    assert router(*ok[:6], 5000, *ok[7:]) == 1                                # n > 4096
+    assert router(*ok[:11], d, None, None, *ok[14:]) == 1                     # partial list args
+    assert router(*ok[:9], 1e-3, 0, d, d, d, *ok[14:]) == 1                   # cap < 1
+    assert router(*ok[:9], -1.0, 4, d, d, d, *ok[14:]) == 1                   # eps < 0
+    assert router(*ok[:14], None, 1 << 20, None) == 2                         # no ws
+    hard = lib.lapsum_forward_hard
+    hard.argtypes = [vp, ctypes.c_int64, vp, vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                     ctypes.c_int, vp, ctypes.c_size_t, vp]
+    assert hard(d, 8, d, d, 1, 8, 8.0, 0, ws, 1 << 20, None) == 1   # k = n
+    assert hard(d, 8, d, d, 1, 8, 0.0, 0, ws, 1 << 20, None) == 1   # k = 0
+    assert hard(d, 8, d, d, 1, 1, 0.5, 0, ws, 1 << 20, None) == 1   # n < 2
+    assert hard(d, 8, d, d, 1, 8, 2.0, 2, ws, 1 << 20, None) == 1   # bracket
+    assert hard(d, 8, d, d, 1, 8, 2.0, 0, None, 1 << 20, None) == 2  # no ws
