@@ -271,7 +271,9 @@ def main():
         bd = torch.empty(w.B, dtype=torch.float64, device=dev)
         # one budget per row (lapsum_forward_rowk) when k_rows is given
         kk = w.k if k_rows is None else torch.from_numpy(k_rows).to(dev)
-        ws = L.Workspace(w.B, w.n, w.k, "auto" if k_rows is None else "fullsort", dev)
+        ws = (L.Workspace(w.B, w.n, w.k, "auto", dev) if k_rows is None else
+              L.Workspace(w.B, w.n, 1.0, "auto", dev,
+                          nbytes=L._lib().lapsum_workspace_bytes_rowk(w.B, w.n, 0)))
         # rows longer than 4096 hand the gradient support from forward to
         # backward, as the autograd wrapper does
         sup = L.Support(w.B, w.n, dev) if L.support_bytes(w.B, w.n) > 0 else None
@@ -556,6 +558,23 @@ def main():
             "fwdbwd_graph_elements_per_s": wk.elements / (T["fwdbwd_graph_ms"] / 1e3),
             "path_frac_of_peak": (path_step_bytes(wk, 0) / (T["fwdbwd_graph_ms"] / 1e3) / 1e9
                                   / peak_gbs),
+        }
+        del RW
+        torch.cuda.empty_cache()
+        # the memory-selection shape with one budget per row (768..1280, seeded):
+        # the one-CTA-per-row bracketing with ranks computed per row on the device
+        wk = WORKLOADS["memory_select_256x65536"]
+        rr, vv = make_inputs(wk, seed=0)
+        kr = np.random.default_rng(1).integers(768, 1281, wk.B).astype(np.float64)
+        RW = run_workload(wk, rr, vv, 10, 3, table=True, k_rows=kr)
+        T = RW["table"]
+        table["memory_select_256x65536_rowk"] = {
+            "k_rows": "integers 768..1280 (numpy default_rng(1))",
+            "fwd_ms": round(T["fwd_ms"], 5), "bwd_ms": round(T["bwd_ms"], 5),
+            "fwdbwd_graph_ms": round(T["fwdbwd_graph_ms"], 5),
+            "fwdbwd_graph_elements_per_s": wk.elements / (T["fwdbwd_graph_ms"] / 1e3),
+            "path_frac_of_peak": (path_step_bytes(wk, RW["near"]) / (T["fwdbwd_graph_ms"] / 1e3)
+                                  / 1e9 / peak_gbs),
         }
         del RW
         torch.cuda.empty_cache()

@@ -176,19 +176,21 @@ int lapsum_backward_router(const void* r, int dtype, int64_t ld, const double* b
  * Forward with a budget per row: as lapsum_forward, with k[row] (fp64, DEVICE
  * memory, B entries, read in stream order) in place of the shared k.  The
  * pages fix one budget per operator call; a budget per row is the next step
- * the same equation allows (every row is solved on its own).  Rows are
- * solved by the sort-based solvers: LAPSUM_PATH_AUTO and LAPSUM_PATH_FULLSORT
- * give the on-chip sort for n <= 4096 and the radix full sort above, and
- * LAPSUM_PATH_RADIX forces the latter; the bracketing paths return
- * LAPSUM_EINVAL (their sample ranks come from a budget known on the host).
- * The workspace is lapsum_workspace_bytes(B, n, k, LAPSUM_PATH_FULLSORT) for
- * any valid k.  `support` (may be NULL; see the gradient support below, same
+ * the same equation allows (every row is solved on its own).  Solvers:
+ * LAPSUM_PATH_AUTO gives the on-chip sort for n <= 4096, the one-CTA-per-row
+ * bracketing for n <= 2^18 (each row's sample size and binomial ranks are
+ * computed on the device from its budget) and the radix full sort above;
+ * LAPSUM_PATH_FULLSORT, LAPSUM_PATH_RADIX and LAPSUM_PATH_ROWBRACKET (n <=
+ * 2^20) select one; LAPSUM_PATH_BRACKET returns LAPSUM_EINVAL.  The workspace
+ * is lapsum_workspace_bytes_rowk(B, n, path) bytes (0 for an invalid size or
+ * path).  `support` (may be NULL; see the gradient support below, same
  * rules when not NULL) receives the gradient support of rows with n > 4096.
  * A row whose k[row] is not in (0, n) gets b = NaN and p = NaN, and the
  * workspace status reads LAPSUM_EINVAL (lapsum_read_status); the other rows
  * are unaffected.  Host-side errors as lapsum_forward, plus LAPSUM_EINVAL for
  * k == NULL.
  */
+size_t lapsum_workspace_bytes_rowk(int64_t B, int64_t n, int path);
 int lapsum_forward_rowk(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,
                         int64_t n, const double* k, double t, int path, void* ws, size_t ws_bytes,
                         void* support, size_t support_bytes, void* stream);

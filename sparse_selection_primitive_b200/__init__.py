@@ -125,6 +125,8 @@ def _lib():
         lib.lapsum_backward_router.restype = ctypes.c_int
         lib.lapsum_backward_router.argtypes = [_vp, ctypes.c_int, _c_i64, _vp, _vp, _vp, _c_i64,
                                                _c_i64, ctypes.c_double, _vp]
+        lib.lapsum_workspace_bytes_rowk.restype = ctypes.c_size_t
+        lib.lapsum_workspace_bytes_rowk.argtypes = [_c_i64, _c_i64, ctypes.c_int]
         lib.lapsum_forward_rowk.restype = ctypes.c_int
         lib.lapsum_forward_rowk.argtypes = [_vp, _c_i64, _vp, _vp, _vp, _c_i64, _c_i64, _vp,
                                             ctypes.c_double, ctypes.c_int, _vp, ctypes.c_size_t,
@@ -162,9 +164,9 @@ class Workspace:
     ``lapsum_workspace_init``.
     """
 
-    def __init__(self, B: int, n: int, k: float, path="auto", device=None):
+    def __init__(self, B: int, n: int, k: float, path="auto", device=None, nbytes: int = None):
         device = torch.device(device or "cuda")
-        self.nbytes = workspace_bytes(B, n, k, path)
+        self.nbytes = workspace_bytes(B, n, k, path) if nbytes is None else int(nbytes)
         if self.nbytes == 0:
             raise LapSumError(1, "workspace_bytes")
         self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
@@ -266,10 +268,12 @@ def forward(r: torch.Tensor, k, t: float, path="auto", seed: int = 0, ws: Worksp
     code = _path_code(path)
     k_rows = _row_budgets(k, B, r2.device)
     if k_rows is not None:
-        k = 0.5 * n  # any valid budget sizes the workspace of the sort-based solvers
-        if (code & 0xFF) == PATHS["auto"]:
-            code = (code & ~0xFF) | PATHS["fullsort"]
-    if ws is None or not ws.fits(B, n, k, code):
+        need = int(_lib().lapsum_workspace_bytes_rowk(B, n, code))
+        if need == 0:
+            raise LapSumError(1, "lapsum_workspace_bytes_rowk")
+        if ws is None or ws.nbytes < need:
+            ws = Workspace(B, n, 1.0, code, r2.device, nbytes=need)
+    elif ws is None or not ws.fits(B, n, k, code):
         ws = Workspace(B, n, k, code, r2.device)
     if p is None:
         p = _like_rows(r2, ld)

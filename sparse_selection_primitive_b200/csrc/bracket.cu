@@ -1588,12 +1588,13 @@ struct RowBracketSmem {
 constexpr size_t kRowBracketFixedSmem = sizeof(SolveSmemAll) + sizeof(RowBracketSmem);
 
 __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, int64_t ld,
-                                                  int64_t n, double k, double t, uint64_t seed,
-                                                  int m, Ladder lad, int force_miss,
+                                                  int64_t n, double k0, double t, uint64_t seed,
+                                                  int m0, Ladder lad0, int force_miss,
                                                   int max_attempts, int vec, RowState* rows,
                                                   float* __restrict__ band0_all,
                                                   float* __restrict__ band1_all,
-                                                  double* __restrict__ b_all, WsHeader* hdr) {
+                                                  double* __restrict__ b_all, WsHeader* hdr,
+                                                  const RowBudget* __restrict__ budgets) {
     pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
@@ -1609,6 +1610,30 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
         reinterpret_cast<uint32_t*>(st)[i] = 0u;
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) rb->hist1[i] = 0u;
     __syncthreads();
+    // the row's budget, sample size and ladder: shared, or its own entry
+    double k = k0;
+    int m = m0;
+    Ladder lad = lad0;
+    if (budgets != nullptr) {
+        const RowBudget& bg = budgets[row];
+        if (!bg.ok) {  // a budget outside (0, n): b = NaN and a status bit
+            if (threadIdx.x == 0) {
+                st->status |= kDevBadBudget;
+                set_status(hdr, kDevBadBudget);
+                st->path = LAPSUM_PATH_ROWBRACKET;
+                st->b = nan("");
+                *b_out = nan("");
+            }
+            return;
+        }
+        k = bg.k;
+        m = bg.m;
+#pragma unroll
+        for (int i = 0; i < kLadder; ++i) {
+            lad.l[i] = bg.l[i];
+            lad.h[i] = bg.h[i];
+        }
+    }
     phase_mark(st, 14);
     // 1. the sample, as keys, with its level-1 histogram
     const uint64_t c0 = (uint64_t)row << 32;
@@ -1822,7 +1847,8 @@ size_t rowbracket_smem(int m) { return kRowBracketFixedSmem + (size_t)m * sizeof
 cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, double k, double t,
                               uint64_t seed, int m, int64_t rank_l[kLadder],
                               int64_t rank_h[kLadder], int flags, RowState* rows, float* band0,
-                              float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st) {
+                              float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st,
+                              const RowBudget* budgets) {
     static unsigned long long attr_devices = 0ull;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1841,7 +1867,100 @@ cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, 
     const int max_attempts = (flags & LAPSUM_FLAG_NO_RETRY) ? 1 : kMaxAttempts;
     ProfScope ps_("rowbracket", st);
     launch_pdl(rowbracket_kernel, dim3((unsigned)B), dim3(kBlk), rowbracket_smem(m), st, 
-        r, ld, n, k, t, seed, m, lad, force_miss, max_attempts, vec, rows, band0, band1, b, hdr);
+        r, ld, n, k, t, seed, m, lad, force_miss, max_attempts, vec, rows, band0, band1, b, hdr,
+        budgets);
+    return cudaGetLastError();
+}
+
+namespace {
+// One warp per row: the sample size (4096 doubled up to 32768 while below 64/q)
+// and the binomial order-statistic ranks of the bracket (the largest l with
+// P(C < l) <= alpha and the smallest h with P(C >= h) <= alpha, C ~ Bin(m, q),
+// q = k/n), then the ladder: each end moved out by 4x per rung, the last open.
+// The tails are summed 32 terms at a time with a warp prefix sum, in the same
+// order as a sequential sum up from 0 and down from mq + 40 sd + 64.
+__global__ void __launch_bounds__(256) row_budget_kernel(const double* __restrict__ k_rows,
+                                                         int64_t B, int64_t n, double alpha,
+                                                         RowBudget* __restrict__ out) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= B) return;  // the whole warp
+    const double k = k_rows[row];
+    RowBudget* o = out + row;
+    if (!(k > 0.0 && k < (double)n)) {
+        if (lane == 0) {
+            o->k = k;
+            o->m = 0;
+            o->ok = 0;
+        }
+        return;
+    }
+    const double q = k / (double)n;
+    int m = 4096;
+    while (m < kSampleMax && (double)m < 64.0 / q) m <<= 1;
+    const double lgm = lgamma((double)m + 1.0), lq = log(q), l1q = log1p(-q);
+    auto pmf = [&](int64_t c) {
+        return exp(lgm - lgamma((double)c + 1.0) - lgamma((double)(m - c) + 1.0) +
+                   (double)c * lq + (double)(m - c) * l1q);
+    };
+    auto inclusive = [&](double v) {
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const double u = __shfl_up_sync(0xffffffffu, v, d);
+            if (lane >= d) v += u;
+        }
+        return v;
+    };
+    // lower tail: lo = the first c whose cumulative probability exceeds alpha
+    int64_t lo = m + 1;
+    double carry = 0.0;
+    for (int64_t base = 0; base <= m; base += 32) {
+        const int64_t c = base + lane;
+        const double cdf = carry + inclusive(c <= m ? pmf(c) : 0.0);
+        const unsigned over = __ballot_sync(0xffffffffu, c <= m && cdf > alpha);
+        if (over != 0u) {
+            lo = base + (__ffs(over) - 1);
+            break;
+        }
+        carry = __shfl_sync(0xffffffffu, cdf, 31);
+    }
+    // upper tail, summed down from top: hi = one above the first c whose
+    // cumulative probability exceeds alpha (0 when none does)
+    const double mean = (double)m * q, sd = sqrt((double)m * q * (1.0 - q));
+    int64_t top = (int64_t)ceil(mean + 40.0 * sd + 64.0);
+    if (top > m) top = m;
+    int64_t hi = 0;
+    carry = 0.0;
+    for (int64_t base = 0; base <= top; base += 32) {
+        const int64_t c = top - base - lane;
+        const double sf = carry + inclusive(c >= 0 ? pmf(c) : 0.0);
+        const unsigned over = __ballot_sync(0xffffffffu, c >= 0 && sf > alpha);
+        if (over != 0u) {
+            hi = top - base - (__ffs(over) - 1) + 1;
+            break;
+        }
+        carry = __shfl_sync(0xffffffffu, sf, 31);
+    }
+    if (hi > m) hi = m + 1;
+    if (lane == 0) {
+        o->k = k;
+        o->m = m;
+        o->ok = 1;
+        for (int i = 0; i < kLadder - 1; ++i) {
+            o->l[i] = lo >> (2 * i);
+            const int64_t h = hi << (2 * i);
+            o->h[i] = h > m ? (int64_t)m + 1 : h;
+        }
+        o->l[kLadder - 1] = 0;
+        o->h[kLadder - 1] = (int64_t)m + 1;
+    }
+}
+}  // namespace
+
+cudaError_t launch_row_budgets(const double* k_rows, int64_t B, int64_t n, double alpha,
+                               RowBudget* out, cudaStream_t st) {
+    ProfScope ps_("row_budgets", st);
+    row_budget_kernel<<<(unsigned)((B + 7) / 8), 256, 0, st>>>(k_rows, B, n, alpha, out);
     return cudaGetLastError();
 }
 

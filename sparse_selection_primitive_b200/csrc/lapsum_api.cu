@@ -28,6 +28,23 @@ constexpr double kBracketAlpha = 1e-6;  // miss probability allowed per bracket 
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+// Solver for per-row budgets: the sort-based solvers and the one-CTA-per-row
+// bracketing (its sample ranks are computed per row on the device); not the
+// whole-GPU bracketing.
+int resolve_path_rowk(int64_t n, int path) {
+    switch (path & 0xff) {
+        case LAPSUM_PATH_AUTO:
+            return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT
+                   : n <= kRowBracketAuto ? LAPSUM_PATH_ROWBRACKET
+                                          : LAPSUM_PATH_RADIX;
+        case LAPSUM_PATH_FULLSORT:
+            return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT : LAPSUM_PATH_RADIX;
+        case LAPSUM_PATH_RADIX: return LAPSUM_PATH_RADIX;
+        case LAPSUM_PATH_ROWBRACKET: return n <= kRowBracketMax ? LAPSUM_PATH_ROWBRACKET : -1;
+        default: return -1;
+    }
+}
+
 int resolve_path(int64_t n, int path) {
     switch (path & 0xff) {
         case LAPSUM_PATH_AUTO:
@@ -46,7 +63,7 @@ int resolve_path(int64_t n, int path) {
 struct Layout {
     size_t header, rows, partials, row_R, tickets, wlist, wtab, wflag;
     size_t keys0, keys1, seg_hist, tile_hist, plan;
-    size_t sample, band0, band1, bins, fold_part, fold_ticket;
+    size_t sample, band0, band1, bins, fold_part, fold_ticket, budgets;
     size_t total;
 };
 
@@ -84,6 +101,7 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
     if (rpath == LAPSUM_PATH_ROWBRACKET) {
         L.band0 = take((size_t)B * (size_t)n * sizeof(float));
         L.band1 = take((size_t)B * (size_t)n * sizeof(float));
+        L.budgets = take((size_t)B * sizeof(RowBudget));  // per-row budgets' ladders
     }
     if (rpath == LAPSUM_PATH_BRACKET) {
         L.sample = take((size_t)B * kSampleMax * sizeof(float));
@@ -254,6 +272,13 @@ size_t lapsum_workspace_bytes(int64_t B, int64_t n, double k, int path) {
     return make_layout(B, n, rp).total;
 }
 
+size_t lapsum_workspace_bytes_rowk(int64_t B, int64_t n, int path) {
+    if (B < 1 || n < 1) return 0;
+    const int rp = resolve_path_rowk(n, path);
+    if (rp < 0) return 0;
+    return make_layout(B, n, rp).total;
+}
+
 size_t lapsum_backward_workspace_bytes(int64_t B, int64_t n) {
     if (B < 1 || n < 1) return 0;
     return make_layout(B, n, LAPSUM_PATH_FULLSORT).total;
@@ -285,14 +310,8 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
     if (k_rows == nullptr && (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)))
         return LAPSUM_EINVAL;
     if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
-    int rp = resolve_path(n, path);
+    const int rp = k_rows != nullptr ? resolve_path_rowk(n, path) : resolve_path(n, path);
     if (rp < 0 || (path & ~0x7ff) != 0) return LAPSUM_EINVAL;
-    if (k_rows != nullptr) {
-        // per-row budgets: the sort-based solvers (the bracketing paths take
-        // their sample ranks from a budget known on the host)
-        if ((path & 0xff) == LAPSUM_PATH_AUTO) rp = resolve_path(n, LAPSUM_PATH_FULLSORT);
-        if (rp != LAPSUM_PATH_FULLSORT && rp != LAPSUM_PATH_RADIX) return LAPSUM_EINVAL;
-    }
     if (n > INT32_MAX && rp != LAPSUM_PATH_BRACKET) return LAPSUM_EINVAL;
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
     const Layout L = make_layout(B, n, rp);
@@ -337,13 +356,22 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
                                                 b + r0, rows + r0, hdr, st);
         }
     } else if (rp == LAPSUM_PATH_ROWBRACKET) {
-        const int m = sample_size(n, k);
         int64_t rl[kLadder], rh[kLadder];
-        bracket_ladder(m, k / (double)n, rl, rh);
+        RowBudget* budgets = nullptr;
+        int m = kSampleMax;
+        if (k_rows != nullptr) {
+            budgets = reinterpret_cast<RowBudget*>(w + L.budgets);
+            for (int i = 0; i < kLadder; ++i) rl[i] = rh[i] = 0;
+            e = launch_row_budgets(k_rows, B, n, kBracketAlpha, budgets, st);
+            if (e != cudaSuccess) return LAPSUM_ECUDA;
+        } else {
+            m = sample_size(n, k);
+            bracket_ladder(m, k / (double)n, rl, rh);
+        }
         e = launch_rowbracket(r, ld, B, n, k, t, seed, m, rl, rh, path, rows,
                               reinterpret_cast<float*>(w + L.band0),
                               reinterpret_cast<float*>(w + L.band1), b, hdr,
-                              (aligned16(r) && (ld % 4) == 0) ? 1 : 0, st);
+                              (aligned16(r) && (ld % 4) == 0) ? 1 : 0, st, budgets);
     } else {
         BracketBuffers bb;
         bb.sample = reinterpret_cast<float*>(w + L.sample);

@@ -165,12 +165,24 @@ struct BracketBuffers {
     int fold_grid;
 };
 int bracket_fold_grid();
+// Sample size and bracket ladder of one row with its own budget (filled on the
+// device from k[row]); ok = 0 for a budget outside (0, n).
+struct RowBudget {
+    double k;
+    int32_t m, ok;
+    int64_t l[kLadder], h[kLadder];
+};
+cudaError_t launch_row_budgets(const double* k_rows, int64_t B, int64_t n, double alpha,
+                               RowBudget* out, cudaStream_t st);
 // The whole bracketing pipeline with one CTA per row (rows up to 2^20 scores):
-// b[row] and rows[row] for every row; band0/band1: B * n floats each.
+// b[row] and rows[row] for every row; band0/band1: B * n floats each.  With
+// `budgets` (not null) each row takes k, m and its ladder from its entry, and m
+// is the shared-memory capacity for the sample.
 cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, double k, double t,
                               uint64_t seed, int m, int64_t rank_l[kLadder],
                               int64_t rank_h[kLadder], int flags, RowState* rows, float* band0,
-                              float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st);
+                              float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st,
+                              const RowBudget* budgets = nullptr);
 cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t, uint64_t seed,
                                int64_t row, int m, int64_t rank_l[kLadder],
                                int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,

@@ -102,7 +102,6 @@ def test_new_entry_points_reject_bad_arguments_on_host(lib):
     assert rowk(d, 8, d, d, None, 1, 8, None, 0.1, 0, ws, 1 << 20, None, 0, None) == 1  # k NULL
     assert rowk(d, 8, d, d, None, 1, 8, d, 0.0, 0, ws, 1 << 20, None, 0, None) == 1     # t <= 0
     assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 2, ws, 1 << 20, None, 0, None) == 1     # bracket
-    assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 4, ws, 1 << 20, None, 0, None) == 1     # rowbracket
     assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 0, None, 1 << 20, None, 0, None) == 2   # no ws
     router = lib.lapsum_forward_router
     router.argtypes = [vp, ctypes.c_int, ctypes.c_int64, vp, vp, ctypes.c_int64, ctypes.c_int64,

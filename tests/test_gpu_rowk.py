@@ -77,7 +77,7 @@ def test_rowk_invalid_budget_on_the_radix_path(cuda_device):
     k = np.array([40.0, 6000.0, 2.5])
     rt = torch.from_numpy(r).cuda()
     ws = L.Workspace(B, n, 1.0, "fullsort")
-    p, b = L.forward(rt, torch.tensor(k, device="cuda"), t, ws=ws)
+    p, b = L.forward(rt, torch.tensor(k, device="cuda"), t, ws=ws, path="fullsort")
     torch.cuda.synchronize()
     bb, pp = b.cpu().numpy(), p.cpu().numpy()
     assert math.isnan(bb[1]) and np.isnan(pp[1]).all()
@@ -97,12 +97,58 @@ def test_rowk_equal_budgets_match_the_shared_budget(cuda_device, n, path):
     assert torch.equal(b1, b2) and torch.equal(p1, p2)
 
 
-@pytest.mark.parametrize("path", ["bracket", "rowbracket"])
-def test_rowk_refused_on_the_bracketing_paths(cuda_device, path):
+def test_rowk_refused_on_the_whole_gpu_bracketing(cuda_device):
     r, _ = random_rows(314, 2, 20000)
     rt = torch.from_numpy(r).cuda()
     with pytest.raises(L.LapSumError):
-        L.forward(rt, torch.tensor([5.0, 9.0], device="cuda"), 0.05, path=path)
+        L.forward(rt, torch.tensor([5.0, 9.0], device="cuda"), 0.05, path="bracket")
+
+
+@pytest.mark.parametrize("B,n,dist,path", [(5, 20000, "normal", "auto"),
+                                           (3, 65536, "normal_q64", "auto"),
+                                           (2, 300000, "mix_nu", "rowbracket")])
+def test_rowk_one_cta_per_row_bracketing(cuda_device, B, n, dist, path):
+    """Each row's sample size and binomial ranks come from its own budget, on the
+    device; they must equal the oracle's for that budget, and b, p, g must match."""
+    r, v = random_rows(317 + n, B, n, dist)
+    rng = np.random.default_rng(n + 1)
+    k = rng.uniform(1.0, n / 3.0, B)
+    k[0] = 3.0
+    kt = torch.tensor(k, dtype=torch.float64, device="cuda")
+    rt = torch.from_numpy(r).cuda()
+    ws = L.Workspace(B, n, 1.0, "auto", nbytes=L._lib().lapsum_workspace_bytes_rowk(B, n, 0))
+    p, b = L.forward(rt, kt, 0.02, path=path, ws=ws)
+    g = L.backward(rt, b, torch.from_numpy(v).cuda(), 0.02)
+    torch.cuda.synchronize()
+    p, bb, g = p.cpu().numpy().astype(np.float64), b.cpu().numpy(), g.cpu().numpy()
+    for i in range(B):
+        info = L.row_info(ws, i)
+        assert info["path"] == 4, info
+        m = info["sample_m"]
+        q = float(k[i]) / n
+        want_m = 4096
+        while want_m < 32768 and want_m < 64.0 / q:
+            want_m *= 2
+        assert m == want_m
+        l, h = oracle.binom_ranks(m, q, 1e-6)
+        assert (info["rank_l"], info["rank_h"]) == (l, h), (i, info, l, h)
+        check_row(r[i], v[i], float(k[i]), 0.02, bb[i], p[i], g[i].astype(np.float64),
+                  label=f"row {i}")
+
+
+def test_rowk_bad_budget_on_the_one_cta_bracketing(cuda_device):
+    B, n = 3, 10000
+    r, _ = random_rows(318, B, n)
+    k = np.array([25.0, -1.0, 100.0])
+    rt = torch.from_numpy(r).cuda()
+    ws = L.Workspace(B, n, 1.0, "auto", nbytes=L._lib().lapsum_workspace_bytes_rowk(B, n, 0))
+    p, b = L.forward(rt, torch.tensor(k, device="cuda"), 0.05, ws=ws)
+    torch.cuda.synchronize()
+    bb, pp = b.cpu().numpy(), p.cpu().numpy()
+    assert math.isnan(bb[1]) and np.isnan(pp[1]).all()
+    for i in (0, 2):
+        check_row(r[i], None, float(k[i]), 0.05, bb[i], pp[i].astype(np.float64))
+    assert L.read_status(ws) == 1
 
 
 def test_rowk_autograd_gradient_per_row(cuda_device):
