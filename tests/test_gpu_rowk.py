@@ -6,12 +6,13 @@ b)/t) = k for one row; every row is solved on its own, so a budget per row is
 the same equation with k_row in place of k.  Each row is compared with the
 oracle solved at its own budget, at the tolerances of the other parity tests:
 
-* on-chip rows (n <= 4096) and radix full-sort rows (n > 4096), with
+* on-chip rows (n <= 4096), one-CTA-per-row bracketing rows and radix rows, with
   fractional budgets, budgets near 0 and near n, and ragged lengths;
 * a row whose budget lies outside (0, n) gets b = NaN and p = NaN, the status
   word reads LAPSUM_EINVAL, and the other rows are unaffected;
 * equal budgets give the bits of the shared-budget call on the same solver;
-* the bracketing paths refuse a per-row budget on the host;
+* the whole-GPU bracketing refuses a per-row budget on the host; the one-CTA
+  bracketing takes its ranks per row on the device, equal to the oracle's;
 * autograd: the gradient of a per-row k tensor is the oracle's dL/dk per row;
 * the support hand-over of long rows with per-row budgets.
 """
