@@ -545,6 +545,21 @@ class LapSumTopK(torch.autograd.Function):
         B = 1 if rd.dim() == 1 else rd.shape[0]
         n = rd.shape[-1]
         per_row = isinstance(k, torch.Tensor) and k.dim() == 1
+        ctx.bf16 = rd.dtype == torch.bfloat16
+        if ctx.bf16:
+            # bf16 scores: the router form (rows of n <= 4096, one shared k); p is
+            # fp32, the gradient with respect to r comes back in bf16
+            if n > 4096 or per_row:
+                raise ValueError("bf16 scores need rows of n <= 4096 and one shared k")
+            tf = float(t)
+            p, b = forward_router(rd, float(k), tf)
+            ctx.save_for_backward(r, b)
+            ctx.t = tf
+            ctx.sup = None
+            ctx.kt_grad = (isinstance(k, torch.Tensor) and k.requires_grad,
+                           isinstance(t, torch.Tensor) and t.requires_grad)
+            ctx.kt_like = (k, t)
+            return p
         kf = k.detach() if per_row else float(k)
         tf = float(t)
         sup = Support(B, n, rd.device) if support_bytes(B, n) > 0 else None
@@ -561,13 +576,17 @@ class LapSumTopK(torch.autograd.Function):
     def backward(ctx, gp):
         r, b = ctx.saved_tensors
         v = gp.contiguous()
-        g = backward(r.detach(), b, v, ctx.t, support=ctx.sup)
+        if ctx.bf16:
+            g = backward_router(r.detach(), b, v, ctx.t).to(torch.bfloat16)
+        else:
+            g = backward(r.detach(), b, v, ctx.t, support=ctx.sup)
         ctx.sup = None
         gk = gt = None
         if any(ctx.kt_grad):
             # a shared k or t gets the sum over rows of the per-row gradients;
             # a per-row k (one entry per row) gets them row by row
-            gks, gts = backward_kt(r.detach(), b, v, ctx.t)
+            r32 = r.detach().float() if ctx.bf16 else r.detach()
+            gks, gts = backward_kt(r32, b, v, ctx.t)
             k, t = ctx.kt_like
             if ctx.kt_grad[0]:
                 if k.dim() == 1:

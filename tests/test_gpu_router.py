@@ -91,3 +91,27 @@ def test_router_refuses_long_rows_and_bad_selection(cuda_device):
         L.forward_router(r, 5.0, 0.1)
     with pytest.raises(L.LapSumError):
         L.forward_router(torch.zeros((2, 100), device="cuda"), 5.0, 0.1, eps=-1.0, cap=4)
+
+
+def test_router_bf16_autograd(cuda_device):
+    """soft_topk on bf16 scores: p from the router form, the gradient with respect to
+    r equal to lapsum_backward_router's rounded to bf16, and dL/dk and dL/dt from
+    the widened scores as the oracle gives them."""
+    B, n, t = 12, 256, 0.05
+    r, v = random_rows(404, B, n)
+    rb = torch.from_numpy(r).to(torch.bfloat16).cuda().requires_grad_(True)
+    k = torch.tensor(8.0, dtype=torch.float64, device="cuda", requires_grad=True)
+    p = L.soft_topk(rb, k, t)
+    vt = torch.from_numpy(v).cuda()
+    p.backward(vt)
+    assert p.dtype == torch.float32 and rb.grad.dtype == torch.bfloat16
+    p2, b2 = L.forward_router(rb.detach(), 8.0, t)
+    g2 = L.backward_router(rb.detach(), b2, vt, t).to(torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(p.detach(), p2) and torch.equal(rb.grad, g2)
+    r64 = rb.detach().to(torch.float64).cpu().numpy()
+    gk_ref = 0.0
+    for i in range(B):
+        b_ref = oracle.solve_b(r64[i], 8.0, t)
+        gk_ref += oracle.vjp_kt(r64[i], v[i], b_ref, t)[0]
+    assert abs(k.grad.item() - gk_ref) <= 1e-4 * max(1.0, abs(gk_ref))
