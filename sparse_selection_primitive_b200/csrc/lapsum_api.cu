@@ -19,7 +19,6 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int64_t kOnchipMax = 4096;
-constexpr int64_t kRadixMax = int64_t(1) << 20;
 constexpr int64_t kRowBracketAuto = int64_t(1) << 18;  // AUTO: one CTA per row up to here
 constexpr int64_t kRowBracketMax = int64_t(1) << 20;
 constexpr int kFoldGridMax = 4096;

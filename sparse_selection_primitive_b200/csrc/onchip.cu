@@ -29,6 +29,7 @@ struct Shape {
     static constexpr int WPR = RT / 32;  // warps per row
     static constexpr int NW = CTA / 32;
     static_assert(RT % 32 == 0 && CTA % RT == 0, "rows are whole warps");
+    static_assert(NPAD <= 4096, "on-chip rows hold at most 4096 keys");
 };
 
 // Load E consecutive elements of a row (idx = tid*E + e), padding past n.
