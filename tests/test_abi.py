@@ -122,3 +122,20 @@ def test_new_entry_points_reject_bad_arguments_on_host(lib):
     assert hard(d, 8, d, d, 1, 1, 0.5, 0, ws, 1 << 20, None) == 1   # n < 2
     assert hard(d, 8, d, d, 1, 8, 2.0, 2, ws, 1 << 20, None) == 1   # bracket
     assert hard(d, 8, d, d, 1, 8, 2.0, 0, None, 1 << 20, None) == 2  # no ws
+
+
+def test_per_row_budget_workspace_sizes(lib):
+    """lapsum_workspace_bytes_rowk follows the per-row solver choice: the on-chip
+    sort, the one-CTA bracketing (band buffers), the radix sort (key buffers); the
+    whole-GPU bracketing has no per-row form."""
+    f = lib.lapsum_workspace_bytes_rowk
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
+    assert f(0, 100, 0) == 0 and f(4, 0, 0) == 0
+    assert f(4, 100, 2) == 0                      # whole-GPU bracketing
+    assert f(4, 2_000_000, 4) == 0                # one-CTA bracketing is for n <= 2^20
+    small = f(16, 256, 0)
+    assert small > 0 and small % 256 == 0
+    assert f(256, 65536, 0) >= 2 * 256 * 65536 * 4        # band buffers
+    assert f(2, 1 << 19, 0) >= 2 * 2 * (1 << 19) * 4       # radix key buffers
+    assert f(256, 65536, 3) >= 2 * 256 * 65536 * 4         # radix forced
