@@ -24,15 +24,16 @@
  *     never allocates, frees or retains device memory.
  *   - Rows are row-major with leading dimension ld >= n (elements): element i
  *     of row j of r, p, v and g is at [j * ld + i].  Vectorised loads are used
- *     when the base pointers are 16-byte aligned and ld is a multiple of 4.
+ *     when the base pointers are 16-byte aligned and ld is a multiple of 4
+ *     (of 8 for bf16 scores).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  All work is ordered on it; no call synchronises the host except
  *     lapsum_read_status and lapsum_row_info.
  *   - Argument errors are detected on the host, returned at once, and launch
  *     nothing.  Conditions found on the device (non-finite scores, exhausted
  *     bracket retries, per-row budgets outside (0, n)) are OR-ed into a
- *     sticky status word inside the
- *     workspace and reported by lapsum_read_status, which also clears it.
+ *     sticky status word inside the workspace and reported by
+ *     lapsum_read_status, which also clears it.
  *   - Calls that share a workspace must be ordered on one stream (or be
  *     otherwise serialised); concurrent calls on one workspace race.
  */
@@ -49,7 +50,8 @@ extern "C" {
 /* Return codes and device status bits. */
 enum lapsum_status {
     LAPSUM_OK = 0,
-    LAPSUM_EINVAL = 1,     /* B < 1, n < 1, ld < n, !(0 < k < n), !(t > 0), NULL pointer, bad path */
+    LAPSUM_EINVAL = 1,     /* B < 1, n < 1, ld < n, !(0 < k < n), !(t > 0), NULL pointer, bad path;
+                              device: a per-row budget outside (0, n); b of that row is NaN */
     LAPSUM_EWORKSPACE = 2, /* ws NULL, not 256-byte aligned, or smaller than lapsum_workspace_bytes */
     LAPSUM_ENONFINITE = 3, /* device: a score was NaN or infinite; b of that row is NaN */
     LAPSUM_EBRACKET = 4,   /* device: every allowed bracket failed certification; b is NaN */
