@@ -17,7 +17,10 @@
  *     f_i = 0.5 exp(-|r_i - b|/t) = sigma'((r_i-b)/t);
  *   - section 2.2 "Probabilistic bracketing", steps 1-2: a sample of
  *     Laplace-noised scores, a bracket [a_L, a_R) from binomial order
- *     statistics, and the fold of out-of-bracket scores into tail sums.
+ *     statistics, and the fold of out-of-bracket scores into tail sums;
+ *   - section 2.3 "Relation to DFTopK": the zero-temperature limit of the
+ *     operator (the midpoint threshold, with tied boundary scores sharing the
+ *     remaining budget), written out in lso_hard_topk.
  *
  * The threshold solve is the plain definition, not the paper's fast solver:
  * a full sort (used only to bound the search), then bisection on b with the
@@ -29,7 +32,8 @@
  * two-point row), a high-precision segment-by-segment quadratic brute force on
  * tiny rows, invariants (shift, scale, permutation, mirror), the zero
  * temperature limit, central finite differences of the VJP, the published
- * SplitMix64 test vector and scipy's binomial distribution.
+ * SplitMix64 test vector and scipy's binomial distribution; the hard top-k by
+ * worked cases and by the soft solve far below the score gaps.
  */
 #include <math.h>
 #include <stdint.h>
