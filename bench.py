@@ -168,6 +168,48 @@ def oracle_sample_run(w, r_row, v_row, n_sample):
     return n_s, k_s, time.perf_counter() - t0
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_timings(w, r, v, budget=1 << 20):
+    """The fp64 oracle, single-threaded, on a bounded sample of a workload: whole
+    rows up to about `budget` scores for batched shapes, else a prefix of row 0
+    (k scaled to keep k/n).  Forward (solve b, emit p), backward (VJP) and both,
+    in elements per second, with the host's CPU model and core count."""
+    import oracle
+    if w.n <= budget:
+        rows = max(1, min(w.B, budget // w.n))
+        n_s, k_s = w.n, w.k
+    else:
+        rows, n_s = 1, budget
+        k_s = min(max(w.k * n_s / w.n, 1e-3), n_s - 1e-3)
+    tf = tb = 0.0
+    for i in range(rows):
+        rr, vv = r[i, :n_s], v[i, :n_s]
+        t0 = time.perf_counter()
+        b = oracle.solve_b(rr, k_s, w.t)
+        oracle.emit_p(rr, b, w.t)
+        t1 = time.perf_counter()
+        oracle.vjp(rr, vv, b, w.t)
+        t2 = time.perf_counter()
+        tf += t1 - t0
+        tb += t2 - t1
+    el = rows * n_s
+    return {"fwd_elements_per_s": el / tf, "bwd_elements_per_s": el / tb,
+            "fwdbwd_elements_per_s": el / (tf + tb), "cores": 1, "cpu": cpu_model(),
+            "host_cpu_count": os.cpu_count(),
+            "sample": (f"{rows} whole rows" if n_s == w.n else
+                       f"first {n_s} scores of row 0, k={k_s:g} (same k/n)")}
+
+
 def cpu_sample_size(w):
     # about 10 s of single-thread oracle work on this box's cores
     return min(w.elements, 1 << 23)
@@ -178,7 +220,7 @@ def cpu_baseline(w, r, v):
     return {"value": n_s / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"first {n_s} scores of row 0 of {w.name}, k={k_s:g} (same k/n), "
                       f"t={w.t}; fp64 full sort + bisection, p, VJP; {sec:.1f} s single thread",
-            "host_cpu_count": os.cpu_count()}
+            "cpu": cpu_model(), "host_cpu_count": os.cpu_count()}
 
 
 def run_reference(args, rank, world):
@@ -263,7 +305,7 @@ def main():
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_buf = torch.empty(2 * l2_bytes // 4 + 1024, dtype=torch.float32, device=dev)
 
-    def run_workload(w, r_h, v_h, steps, warmup, table=False, k_rows=None):
+    def run_workload(w, r_h, v_h, steps, warmup, table=False, k_rows=None, path="auto"):
         rd = torch.from_numpy(r_h).to(dev)
         vd = torch.from_numpy(v_h).to(dev)
         pd = torch.empty_like(rd)
@@ -271,8 +313,8 @@ def main():
         bd = torch.empty(w.B, dtype=torch.float64, device=dev)
         # one budget per row (lapsum_forward_rowk) when k_rows is given
         kk = w.k if k_rows is None else torch.from_numpy(k_rows).to(dev)
-        ws = (L.Workspace(w.B, w.n, w.k, "auto", dev) if k_rows is None else
-              L.Workspace(w.B, w.n, 1.0, "auto", dev,
+        ws = (L.Workspace(w.B, w.n, w.k, path, dev) if k_rows is None else
+              L.Workspace(w.B, w.n, 1.0, path, dev,
                           nbytes=L._lib().lapsum_workspace_bytes_rowk(w.B, w.n, 0)))
         # rows longer than 4096 hand the gradient support from forward to
         # backward, as the autograd wrapper does
@@ -281,7 +323,7 @@ def main():
         flush = working < 2 * l2_bytes
 
         def fwd():
-            L.forward(rd, kk, w.t, ws=ws, p=pd, b=bd, support=sup)
+            L.forward(rd, kk, w.t, path=path, ws=ws, p=pd, b=bd, support=sup)
 
         def bwd():
             L.backward(rd, bd, vd, w.t, ws=ws, g=gd, support=sup)
@@ -328,7 +370,7 @@ def main():
         res = {"flush": flush, "ws": ws, "rd": rd, "vd": vd, "pd": pd, "gd": gd, "bd": bd,
                "fwd": fwd, "bwd": bwd, "timed": timed, "graph": graph, "sup": sup}
         res["near"] = support_count(r_h, bd.cpu().numpy(), w.t) if sup is not None else 0
-        if w.path == "bracket":
+        if w.path == "bracket" and path == "auto":
             info = L.row_info(ws, 0)
             res["bracket"] = {key: info[key] for key in ("attempts", "n_band", "refine_levels",
                                                        "sample_m", "rank_l", "rank_h")}
@@ -533,16 +575,42 @@ def main():
                 "fwd_elements_per_s": wk.elements / (T["fwd_ms"] / 1e3),
                 "bwd_elements_per_s": wk.elements / (T["bwd_ms"] / 1e3),
                 "fwdbwd_elements_per_s": wk.elements / (T["fwdbwd_ms"] / 1e3),
-                "fwdbwd_algorithmic_gbs": STEP_BYTES_PER_ELEMENT[wk.path] * wk.elements
+                # the survey's fixed per-score byte count over the step time: a
+                # reference figure, not bytes this path moves (it can exceed the
+                # peak where the path skips passes the count assumes)
+                "fwdbwd_survey_bytes_gbs": STEP_BYTES_PER_ELEMENT[wk.path] * wk.elements
                 / (T["fwdbwd_ms"] / 1e3) / 1e9,
             }
-            table[name]["fwdbwd_frac_of_peak"] = table[name]["fwdbwd_algorithmic_gbs"] / peak_gbs
+            table[name]["oracle"] = oracle_timings(wk, rr, vv)
             if "bwd_without_support_ms" in T:
                 table[name]["bwd_without_support_ms"] = round(T["bwd_without_support_ms"], 5)
             table[name]["path_frac_of_peak"] = (path_step_bytes(wk, RW["near"])
                                                 / (T["fwdbwd_graph_ms"] / 1e3) / 1e9 / peak_gbs)
             if "bracket" in RW:
                 table[name]["bracket"] = RW["bracket"]
+            del RW
+            torch.cuda.empty_cache()
+        # the full-sort solver (radix sort of every row) on the memory-selection
+        # shape, as that configuration names it, and on the 10^8-score row, for
+        # the bracketed-versus-full-sort comparison
+        for name in ("memory_select_256x65536", "extreme_1e8"):
+            wk = WORKLOADS[name]
+            rr, vv = (r_h, v_h) if name == w.name else make_inputs(wk, seed=0)
+            RW = run_workload(wk, rr, vv, 10, 3, table=True, path="fullsort")
+            T = RW["table"]
+            table[name + "_fullsort"] = {
+                "solver": "radix full sort",
+                "fwd_ms": round(T["fwd_ms"], 5), "bwd_ms": round(T["bwd_ms"], 5),
+                "fwdbwd_ms": round(T["fwdbwd_ms"], 5),
+                "fwdbwd_graph_ms": round(T["fwdbwd_graph_ms"], 5),
+                "fwdbwd_graph_elements_per_s": wk.elements / (T["fwdbwd_graph_ms"] / 1e3),
+                "fwd_elements_per_s": wk.elements / (T["fwd_ms"] / 1e3),
+                "bwd_elements_per_s": wk.elements / (T["bwd_ms"] / 1e3),
+                # r, p, v, g and the support list only: the sort's key passes
+                # come on top of these bytes
+                "endpoint_bytes_frac_of_peak": (path_step_bytes(wk, RW["near"])
+                                                / (T["fwdbwd_graph_ms"] / 1e3) / 1e9 / peak_gbs),
+            }
             del RW
             torch.cuda.empty_cache()
         # the router shape with one budget per row (integers 4..12, seeded)
@@ -602,12 +670,14 @@ def main():
             "timing": "CUDA-graph replay of one fwd+bwd step; eager calls in eager_ms_per_step",
             "eager_ms_per_step": eager_ms_max,
             "eager_value": elements / (eager_ms_max / 1e3),
-            "step_algorithmic_gbs": step_gbs,
-            "step_frac_of_peak": step_gbs / peak_gbs,
-            "step_bytes_note": "step_* count the fixed per-element bytes of the method's two "
-                               "passes (fwd 12, bwd 20 B/score on long rows); path_* count what "
-                               "this path must move: r read by the fold, r read + p written by "
-                               "the emit, g written, plus 36 B per gradient-support entry",
+            "survey_bytes_gbs": step_gbs,
+            "survey_bytes_over_peak": step_gbs / peak_gbs,
+            "step_bytes_note": "survey_bytes_* divide the survey's fixed per-score count (fwd "
+                               "12, bwd 20 B/score on long rows) by the step time: a reference "
+                               "figure, not a fraction of bytes moved (this path skips re-reads "
+                               "the count assumes, so it can exceed 1); path_* count what this "
+                               "path must move: r read by the fold, r read + p written by the "
+                               "emit, g written, plus 36 B per gradient-support entry",
             "path_step_bytes": path_bytes,
             "path_support_entries": R["near"],
             "path_frac_of_peak": path_gbs / peak_gbs,

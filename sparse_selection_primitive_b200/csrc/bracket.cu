@@ -23,6 +23,9 @@
 //                   solve with the tails as virtual end anchors.  A failed
 //                   bracket moves the failing end to the next rung of its
 //                   ladder (4x the rank, then open) and the same CTA re-folds r.
+#include <atomic>
+#include <type_traits>
+
 #include "bitonic.cuh"
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
@@ -292,10 +295,16 @@ __device__ __forceinline__ float draw_sample(const float* __restrict__ r, int64_
     const float eps = (u < 0.0 ? 1.f : -1.f) * (float)t * logf(a);
     return rv + eps;
 }
-// Grid of m / 1024 CTAs: every thread draws one sample and every CTA adds its
-// samples to a global histogram of the keys' top 11 bits; the last CTA to
-// finish (atomic ticket) selects the two order statistics from it and clears
-// the histogram for the next call.
+// Grid of m / 1024 CTAs: every thread draws one sample.  The order statistics
+// of the bracket are found in one of two ways:
+//  - top_h > 0 (both ranks at most top_h, and (m / 1024) * top_h <= 4096): each
+//    CTA sorts its 1024 keys and keeps its top_h largest, which must hold every
+//    sample of global rank <= top_h; the last CTA to finish (atomic ticket)
+//    sorts those candidates and reads the two ranks off;
+//  - otherwise every CTA adds its samples to a global histogram of the keys'
+//    top 11 bits, and the last CTA stages the whole sample in shared memory and
+//    selects the two order statistics by radix levels, then clears the
+//    histogram for the next call.
 __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ r, int64_t n,
                                                       double t, uint64_t seed, uint64_t c0, int m,
                                                       Ladder lad, int force_miss, int max_attempts,
@@ -303,42 +312,51 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
                                                       unsigned long long* __restrict__ bins,
                                                       uint32_t* __restrict__ ghist,
                                                       uint32_t* __restrict__ ticket,
-                                                      RowState* st) {
+                                                      RowState* st, int top_h,
+                                                      uint32_t* __restrict__ cand, int clear_bins,
+                                                      uint32_t* __restrict__ sup_flag) {
     pdl_wait();
     if (blockIdx.x == 0) {
-        // this kernel starts the row's forward: clear its record and histogram
+        // this kernel starts the row's forward: clear its record, histogram
+        // and gradient-support flags
         for (int i = threadIdx.x; i < (int)(sizeof(RowState) / 4); i += kBlk)
             reinterpret_cast<uint32_t*>(st)[i] = 0u;
-        for (int i = threadIdx.x; i < 3 * kBins; i += kBlk) bins[i] = 0ull;
+        if (sup_flag != nullptr && threadIdx.x == 0) *sup_flag = 0u;
+        if (clear_bins)
+            for (int i = threadIdx.x; i < 3 * kBins; i += kBlk) bins[i] = 0ull;
         __syncthreads();
         phase_mark(st, 14);
     }
     extern __shared__ uint32_t dyn[];
-    uint32_t* skeys = dyn;               // the sample's keys (last CTA only), kSampleMax words
-    uint32_t* h2 = skeys + kSampleMax;   // select histograms, 2 x 2048 words
     __shared__ uint32_t hist[2048];
     __shared__ uint32_t wsum[64];
     __shared__ uint32_t bcast[4];
     __shared__ int flag;
-    for (int i = threadIdx.x; i < 2048; i += kBlk) hist[i] = 0u;
-    __syncthreads();
-    {
-        const int s = blockIdx.x * kBlk + threadIdx.x;
-        uint32_t bn = 0xffffffffu;
-        if (s < m) {
-            const float y = draw_sample(r, n, t, seed, c0, s);
-            sample_out[s] = y;
-            bn = to_key(y) >> 21;
-        }
+    const int s = blockIdx.x * kBlk + threadIdx.x;
+    uint32_t key = 0u;  // samples past m (none when m is a multiple of kBlk) sort first
+    if (s < m) {
+        const float y = draw_sample(r, n, t, seed, c0, s);
+        sample_out[s] = y;
+        key = to_key(y);
+    }
+    if (top_h > 0) {
+        uint32_t kk[1] = {key};
+        bitonic_sort_row<1, kBlk, kBlk>(kk, threadIdx.x, hist);
+        if (threadIdx.x >= kBlk - top_h)
+            cand[blockIdx.x * top_h + (threadIdx.x - (kBlk - top_h))] = kk[0];
+    } else {
+        for (int i = threadIdx.x; i < 2048; i += kBlk) hist[i] = 0u;
+        __syncthreads();
+        const uint32_t bn = s < m ? key >> 21 : 0xffffffffu;
         // lanes with the same bin add once (samples crowd into few top bins)
         const unsigned peers = __match_any_sync(0xffffffffu, bn);
         if (bn != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
             atomicAdd(&hist[bn], (uint32_t)__popc(peers));
+        __syncthreads();
+        for (int i = threadIdx.x; i < 2048; i += kBlk)
+            if (hist[i] != 0u) atomicAdd(&ghist[i], hist[i]);
     }
-    __syncthreads();
     if (blockIdx.x == 0) phase_mark(st, 15);
-    for (int i = threadIdx.x; i < 2048; i += kBlk)
-        if (hist[i] != 0u) atomicAdd(&ghist[i], hist[i]);
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -350,45 +368,73 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
     if (!flag) return;
     __threadfence();
     phase_mark(st, 0);
-    for (int i = threadIdx.x; i < 2048; i += kBlk) {
-        hist[i] = __ldcg(ghist + i);
-        ghist[i] = 0u;  // ready for the next call
-    }
-    // the sample's keys into shared memory, eight loads in flight per thread
-    for (int s0 = 0; s0 < m; s0 += 8 * kBlk) {
-        float yv[8];
+    const int64_t ra = lad.l[0] >= 1 ? lad.l[0] : 0;
+    const int64_t rb = lad.h[0] <= m ? lad.h[0] : 0;
+    uint32_t ka = 0u, kb = 0u, kmax = 0u;
+    if (top_h > 0) {
+        // the candidates, sorted ascending: the r-th largest sits at npad - r
+        const int c = (int)gridDim.x * top_h;
+        auto pick = [&](auto e_tag) {
+            constexpr int E = decltype(e_tag)::value;
+            uint32_t kk[E];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int s = s0 + q * kBlk + threadIdx.x;
-            yv[q] = s < m ? __ldcg(sample_out + s) : 0.f;
-        }
+            for (int e = 0; e < E; ++e) {
+                const int j = threadIdx.x * E + e;
+                kk[e] = j < c ? __ldcg(cand + j) : 0u;
+            }
+            bitonic_sort_row<E, kBlk, kBlk>(kk, threadIdx.x, dyn);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int s = s0 + q * kBlk + threadIdx.x;
-            if (s < m) skeys[s] = to_key(yv[q]);
+            for (int e = 0; e < E; ++e) {
+                const int j = threadIdx.x * E + e;
+                if (ra >= 1 && j == E * kBlk - ra) bcast[0] = kk[e];
+                if (rb >= 1 && j == E * kBlk - rb) bcast[1] = kk[e];
+                if (j == E * kBlk - 1) bcast[2] = kk[e];
+            }
+        };
+        if (c <= kBlk) pick(std::integral_constant<int, 1>{});
+        else if (c <= 2 * kBlk) pick(std::integral_constant<int, 2>{});
+        else pick(std::integral_constant<int, 4>{});
+        __syncthreads();
+        ka = bcast[0];
+        kb = bcast[1];
+        kmax = bcast[2];
+    } else {
+        uint32_t* skeys = dyn;               // the sample's keys, kSampleMax words
+        uint32_t* h2 = skeys + kSampleMax;   // select histograms, 2 x 2048 words
+        for (int i = threadIdx.x; i < 2048; i += kBlk) {
+            hist[i] = __ldcg(ghist + i);
+            ghist[i] = 0u;  // ready for the next call
         }
-    }
-    __syncthreads();
-    float aR = INFINITY, aL = -INFINITY;
-    {
-        const int64_t ra = lad.l[0] >= 1 ? lad.l[0] : 0;
-        const int64_t rb = lad.h[0] <= m ? lad.h[0] : 0;
-        uint32_t ka = 0u, kb = 0u;
+        // the sample's keys into shared memory, eight loads in flight per thread
+        for (int s0 = 0; s0 < m; s0 += 8 * kBlk) {
+            float yv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int sq = s0 + q * kBlk + threadIdx.x;
+                yv[q] = sq < m ? __ldcg(sample_out + sq) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int sq = s0 + q * kBlk + threadIdx.x;
+                if (sq < m) skeys[sq] = to_key(yv[q]);
+            }
+        }
+        __syncthreads();
         select_two_ranks(skeys, m, hist, ra, rb, h2, wsum, bcast, &ka, &kb);
-        if (ra >= 1) aR = from_key(ka);
-        if (rb >= 1) aL = from_key(kb);
-    }
-    phase_mark(st, 1);
-    if (force_miss) {
-        uint32_t kmax = 0;
-        for (int s = threadIdx.x; s < m; s += kBlk) kmax = max(kmax, skeys[s]);
+        if (force_miss) {
+            for (int sq = threadIdx.x; sq < m; sq += kBlk) kmax = max(kmax, skeys[sq]);
 #pragma unroll
-        for (int d = 16; d > 0; d >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, d));
-        if (threadIdx.x == 0) bcast[3] = 0u;
-        __syncthreads();
-        if ((threadIdx.x & 31) == 0) atomicMax(&bcast[3], kmax);
-        __syncthreads();
+            for (int d = 16; d > 0; d >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, d));
+            if (threadIdx.x == 0) bcast[3] = 0u;
+            __syncthreads();
+            if ((threadIdx.x & 31) == 0) atomicMax(&bcast[3], kmax);
+            __syncthreads();
+            kmax = bcast[3];
+        }
     }
+    const float aR = ra >= 1 ? from_key(ka) : INFINITY;
+    const float aL = rb >= 1 ? from_key(kb) : -INFINITY;
+    phase_mark(st, 1);
     if (threadIdx.x == 0) {
         st->ladder_R[0] = aR;
         st->ladder_L[0] = aL;
@@ -396,7 +442,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
         st->rung_R = 0;
         if (force_miss) {
             // A bracket above every sample value: F(a_L) < k, so it must fail.
-            const float top = from_key(bcast[3]);
+            const float top = from_key(kmax);
             st->a_L = top + fabsf(top) + 1.f;
             st->a_R = INFINITY;
             st->rung_L = -1;
@@ -481,7 +527,7 @@ __device__ __forceinline__ void band_stage(bool take, float x, float* sband, int
         } else {
             const unsigned long long g = atomicAdd(counter, 1ull);
             if (g < cap) band[g] = x;
-            bin_add(x, BL, inv_t, bins);
+            if (bins != nullptr) bin_add(x, BL, inv_t, bins);
         }
     }
 }
@@ -499,7 +545,7 @@ __device__ __forceinline__ void band_flush(const float* sband, int scount, float
     for (int i = threadIdx.x; i < ns; i += blockDim.x) {
         const float x = sband[i];
         if (gb + i < cap) band[gb + i] = x;
-        bin_add(x, BL, inv_t, bins);
+        if (bins != nullptr) bin_add(x, BL, inv_t, bins);
     }
 }
 
@@ -517,17 +563,14 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
                                                             float* __restrict__ band,
                                                             unsigned long long* __restrict__ bins,
                                                             double* __restrict__ part,
-                                                            uint32_t* __restrict__ ticket,
-                                                            WsHeader* hdr, int vec) {
+                                                            int vec, int hist) {
     pdl_wait();
-    __shared__ double red[kFoldThreads / 32];
-    __shared__ long long lred[kFoldThreads / 32];
+    __shared__ double red4[kFoldThreads / 32][4];
     __shared__ float sband[kStage];
     // dynamic: per-warp queues (kQ floats each), then per-warp staging rows
     extern __shared__ __align__(16) float fold_dyn[];
     __shared__ int scount;
     __shared__ unsigned long long gbase;
-    __shared__ int flag;
     const float aL = st->a_L, aR = st->a_R;
     // Scores more than 90 t below the bracket add exactly 0 to the left tail
     // sum in fp32, and scores more than 90 t above it add 1 to the right count
@@ -540,7 +583,10 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     // near scores however sparse they are.  Non-finite scores are caught by a
     // running sum (checked exactly if it overflows).
     const float aLf = aL - (float)(90.0 * t), aRf = aR + (float)(90.0 * t);
+    // the band histogram only when the solve will use it (a band expected too
+    // large for the on-chip sort)
     const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
+    if (!hist) bins = nullptr;
     const float inv_t = (float)(1.0 / t);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float* q = fold_dyn + warp * kQ;
@@ -620,10 +666,25 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
         const int64_t step = (int64_t)U * nthreads;
         const int64_t full = n4 / step;
         const float4* p = r4 + gtid;
+        // The last partial trip (at most U vectors per thread, a grid-uniform
+        // count) is loaded with bounds checks into the prefetch registers
+        // while the last full trip is processed, so that a short row has all
+        // its loads in flight at once.
+        const int64_t rem_iters = (n4 - full * step + nthreads - 1) / nthreads;
         float4 nv[U];
+        auto load_rem = [&]() {
+#pragma unroll
+            for (int qq = 0; qq < U; ++qq) {
+                const int64_t i = full * step + (int64_t)qq * nthreads + gtid;
+                nv[qq] = (qq < rem_iters && i < n4) ? __ldcs(r4 + i)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        };
         if (full > 0) {
 #pragma unroll
             for (int qq = 0; qq < U; ++qq) nv[qq] = __ldcs(p + (int64_t)qq * nthreads);
+        } else {
+            load_rem();
         }
         for (int64_t it = 0; it < full; ++it, p += step) {
             float4 cur[U];
@@ -632,6 +693,8 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
             if (it + 1 < full) {
 #pragma unroll
                 for (int qq = 0; qq < U; ++qq) nv[qq] = __ldcs(p + step + (int64_t)qq * nthreads);
+            } else {
+                load_rem();
             }
             // full trips: the compares give 1.0 / 0.0, the near mask is built
             // exactly in fp32 (16 bits) and the far-right count in a float
@@ -657,23 +720,14 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
                 push_staged(m);
             }
         }
-        // Remainder: the last partial trip (at most U vectors per thread, a
-        // grid-uniform count), its loads issued together, with bounds checks.
-        const int64_t rem_iters = (n4 - full * step + nthreads - 1) / nthreads;
+        // Remainder: the last partial trip, loaded above.
         {
-            float4 rv[U];
-#pragma unroll
-            for (int qq = 0; qq < U; ++qq) {
-                const int64_t i = full * step + (int64_t)qq * nthreads + gtid;
-                rv[qq] = (qq < rem_iters && i < n4) ? __ldcs(r4 + i)
-                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
 #pragma unroll
             for (int qq = 0; qq < U; ++qq) {
                 if (qq >= rem_iters) break;
                 const int64_t i = full * step + (int64_t)qq * nthreads + gtid;
                 const bool ok = i < n4;
-                const float xs[4] = {rv[qq].x, rv[qq].y, rv[qq].z, rv[qq].w};
+                const float xs[4] = {nv[qq].x, nv[qq].y, nv[qq].z, nv[qq].w};
                 uint32_t m = 0u;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) classify(xs[j], ok, m, j);
@@ -719,47 +773,18 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     acc.bad |= bad;
     __syncthreads();
     band_flush(sband, scount, band, counter, cap, BL, inv_t, bins, &gbase);
-    const long long cR = block_sum_ll((long long)acc.cntR, lred);
-    const double sL = block_sum_d(acc.SL, red);
-    const double sR = block_sum_d(acc.SR, red);
-    const int any_bad = __syncthreads_or(acc.bad);
+    // the CTA's record (count, left sum, right sum, non-finite flag), summed
+    // into thread 0 in a fixed order
+    // the CTA's record (count, left sum, right sum, non-finite flag), summed
+    // into thread 0 in a fixed order; the solve kernel combines the records
+    double rec[4] = {(double)acc.cntR, acc.SL, acc.SR, acc.bad ? 1.0 : 0.0};
+    block_sum4_to0(rec, red4);
     if (threadIdx.x == 0) {
-        part[blockIdx.x * 4 + 0] = (double)cR;
-        part[blockIdx.x * 4 + 1] = sL;
-        part[blockIdx.x * 4 + 2] = sR;
-        part[blockIdx.x * 4 + 3] = any_bad ? 1.0 : 0.0;
+        double2* pr = reinterpret_cast<double2*>(part) + 2 * blockIdx.x;
+        pr[0] = make_double2(rec[0], rec[1]);
+        pr[1] = make_double2(rec[2], rec[3]);
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t prev = atomicAdd(ticket, 1u);
-        flag = (prev == gridDim.x - 1);
-        if (flag) *ticket = 0u;
-    }
-    __syncthreads();
-    if (!flag) return;
-    __threadfence();
-    double c = 0.0, a = 0.0, bsum = 0.0, badsum = 0.0;
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x) {
-        c += part[i * 4 + 0];
-        a += part[i * 4 + 1];
-        bsum += part[i * 4 + 2];
-        badsum += part[i * 4 + 3];
-    }
-    c = block_sum_d(c, red);
-    a = block_sum_d(a, red);
-    bsum = block_sum_d(bsum, red);
-    badsum = block_sum_d(badsum, red);
-    phase_mark(st, 17);
-    if (threadIdx.x == 0) {
-        st->cnt_R = (unsigned long long)c;
-        st->S_L = a;
-        st->S_R = bsum;
-        if (badsum > 0.0) {
-            st->status |= kDevNonFinite;
-            set_status(hdr, kDevNonFinite);
-        }
-    }
+    if (blockIdx.x == 0) phase_mark(st, 17);
 }
 
 struct FloatGet {
@@ -782,6 +807,8 @@ struct SolveSmemAll {
     uint32_t wsum[32];
     uint32_t bcast[8];
     unsigned long long cnt;
+    double sred[32][8];  // per-warp partial sums of block_sums
+    double sres[8];      // and their totals
     int flag;
     union {
         struct {
@@ -1411,7 +1438,7 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
 // the function returns true at once).  Otherwise writes b, the record and the
 // status, and returns false.
 template <class SelectKey>
-__device__ bool bracket_attempts(const float* __restrict__ r, int64_t n, int vec, double k,
+__device__ __noinline__ bool bracket_attempts(const float* __restrict__ r, int64_t n, int vec, double k,
                                  double t, RowState* st, float* band0, float* band1,
                                  const unsigned long long* __restrict__ bins, int split, int m,
                                  const Ladder& lad, SelectKey select_key, Tails tl, long long nb,
@@ -1528,6 +1555,60 @@ __device__ bool bracket_attempts(const float* __restrict__ r, int64_t n, int vec
     return false;
 }
 
+// ----------------------------------------------------------------------------
+// Exact solve of a band of at most kBandSortMax scores without sorting it (the
+// usual first attempt).  Every thread holds up to four band scores.
+//  1. Certification: F(a_L) >= k >= F(a_R) from the tails and the band.
+//  2. Multisection on the band's own values: the segment (lo, hi) of the
+//     threshold curve that holds b starts as the bracket; each round takes
+//     three band scores strictly inside it as candidates, evaluates F at them
+//     (exact counts, fp32 exponentials, fp64 sums) and keeps the tightest
+//     candidates with F >= k and F < k, until no band score lies strictly
+//     inside.  lo and hi are then neighbouring values of the sorted order (or
+//     a bracket end).
+//  3. Confirmation in fp64: with P = sum over scores <= lo of e^{(s-lo)/t},
+//     Q = sum over scores >= hi of e^{-(s-hi)/t}, m scores >= hi and
+//     delta = e^{(lo-hi)/t},  F(lo) = m - delta Q/2 + P/2 and
+//     F(hi) = m - Q/2 + delta P/2; when rounding in step 2 picked a neighbour
+//     of the right segment, the segment moves by one value.  The root is then
+//     the closed form of the segment, as after the sorted scan.
+// Returns 1 (b in sm->res), 0 (the bracket failed: F at its ends in sm->res)
+// or -1 (not settled within the round limits: the caller sorts instead).
+// ----------------------------------------------------------------------------
+// Sums of up to eight doubles over the block, fixed order; the result is
+// valid in every thread.
+template <int N>
+__device__ __forceinline__ void block_sums(double (&v)[N], SolveSmemAll* sm) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = warp_sum_d(v[i]);
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) sm->sred[w][i] = v[i];
+    }
+    __syncthreads();
+    if (w == 0) {  // the 32 warp sums, one per lane, summed by warp 0
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const double a = warp_sum_d(sm->sred[lane][i]);
+            if (lane == 0) sm->sres[i] = a;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = sm->sres[i];
+}
+
+// The first attempt on a band small enough for the on-chip sort (the usual
+// case): sort, scan and root in a function of its own, so that this path keeps
+// its registers and its code compact, apart from the widening and narrowing
+// machinery.  Returns true when the bracket certifies (b in sm->res).
+__device__ __noinline__ bool first_small_band(const float* __restrict__ band, long long nb,
+                                              Tails tl, double k, double t, SolveSmemAll* sm) {
+    solve_small_band(band, nb, tl, k, t, sm);
+    return sm->res.F_aL >= k && sm->res.F_aR <= k;
+}
+
 // One CTA of 1024 threads; 64 registers each (the whole register file) keeps
 // the fp64 scans' spills down.
 __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_t n, int vec,
@@ -1537,7 +1618,8 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
                                              const unsigned long long* __restrict__ bins,
                                              const float* __restrict__ sample, int m,
                                              Ladder lad, double* __restrict__ b_out,
-                                             WsHeader* hdr, int split) {
+                                             WsHeader* hdr, int split,
+                                             const double* __restrict__ fold_part, int nfold) {
     pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
@@ -1546,7 +1628,30 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
         sm->bcast[2] = 0xffffffffu;
         sm->bcast[3] = 0u;
     }
-    __syncthreads();
+    {
+        // the fold CTAs' records, combined in CTA order: right count, tail
+        // sums and the non-finite flag of the row
+        double tot[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int i = threadIdx.x; i < nfold; i += kBlk) {
+            const double2 p0 = __ldcg(reinterpret_cast<const double2*>(fold_part) + 2 * i);
+            const double2 p1 = __ldcg(reinterpret_cast<const double2*>(fold_part) + 2 * i + 1);
+            tot[0] += p0.x;
+            tot[1] += p0.y;
+            tot[2] += p1.x;
+            tot[3] += p1.y;
+        }
+        block_sums<4>(tot, sm);
+        if (threadIdx.x == 0) {
+            st->cnt_R = (unsigned long long)tot[0];
+            st->S_L = tot[1];
+            st->S_R = tot[2];
+            if (tot[3] > 0.0) {
+                st->status |= kDevNonFinite;
+                set_status(hdr, kDevNonFinite);
+            }
+        }
+        __syncthreads();
+    }
     if (st->status & kDevNonFinite) {
         if (threadIdx.x == 0) {
             st->b = nan("");
@@ -1563,6 +1668,27 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
     tl.SR = st->S_R;
     tl.cntR = (double)st->cnt_R;
     const long long nb = (long long)st->n_band;
+    if (nb <= kBandSortMax && st->max_attempts >= 1) {
+        phase_mark(st, 19);
+        const bool ok = first_small_band(band0, nb, tl, k, t, sm);
+        phase_mark(st, 21);
+        if (ok) {
+            if (threadIdx.x == 0) {
+                const double b = sm->res.b;
+                st->attempts = 1;
+                st->refine_levels = 0;
+                st->a_L = tl.hasL ? tl.aL : -INFINITY;
+                st->a_R = tl.hasR ? tl.aR : INFINITY;
+                st->n_band = (unsigned long long)nb;
+                st->certified = 1;
+                st->b = b;
+                *b_out = b;
+            }
+            phase_mark(st, 12);
+            return;
+        }
+        __syncthreads();
+    }
     auto select_key = [&](int64_t rank) {
         return block_select_desc(GlobalSampleKeyGet{sample}, m, rank, sm->u.sel_hist, sm->wsum,
                                  sm->bcast + 4);
@@ -1594,7 +1720,8 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
                                                   float* __restrict__ band0_all,
                                                   float* __restrict__ band1_all,
                                                   double* __restrict__ b_all, WsHeader* hdr,
-                                                  const RowBudget* __restrict__ budgets) {
+                                                  const RowBudget* __restrict__ budgets,
+                                                  uint32_t* __restrict__ sup_flags) {
     pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
@@ -1608,6 +1735,7 @@ __global__ void __maxnreg__(64) rowbracket_kernel(const float* __restrict__ r, i
     double* b_out = b_all + row;
     for (int i = threadIdx.x; i < (int)(sizeof(RowState) / 4); i += blockDim.x)
         reinterpret_cast<uint32_t*>(st)[i] = 0u;
+    if (sup_flags != nullptr && threadIdx.x == 0) sup_flags[row] = 0u;
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) rb->hist1[i] = 0u;
     __syncthreads();
     // the row's budget, sample size and ladder: shared, or its own entry
@@ -1848,7 +1976,7 @@ cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, 
                               uint64_t seed, int m, int64_t rank_l[kLadder],
                               int64_t rank_h[kLadder], int flags, RowState* rows, float* band0,
                               float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st,
-                              const RowBudget* budgets) {
+                              const RowBudget* budgets, uint32_t* sup_flags) {
     static unsigned long long attr_devices = 0ull;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1868,7 +1996,7 @@ cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, 
     ProfScope ps_("rowbracket", st);
     launch_pdl(rowbracket_kernel, dim3((unsigned)B), dim3(kBlk), rowbracket_smem(m), st, 
         r, ld, n, k, t, seed, m, lad, force_miss, max_attempts, vec, rows, band0, band1, b, hdr,
-        budgets);
+        budgets, sup_flags);
     return cudaGetLastError();
 }
 
@@ -1965,24 +2093,29 @@ cudaError_t launch_row_budgets(const double* k_rows, int64_t B, int64_t n, doubl
 }
 
 int bracket_fold_grid() {
-    static int grid = 0;
-    if (grid == 0) {
-        int dev = 0, sms = 148, per = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // one resident wave of fold CTAs, per device
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> per_sm[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool cached = dev >= 0 && dev < kMaxDevices;
+    int per = cached ? per_sm[dev].load(std::memory_order_relaxed) : 0;
+    if (per == 0) {
         cudaFuncSetAttribute(fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kFoldDynSmem);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fold_kernel, kFoldThreads,
                                                       kFoldDynSmem);
-        grid = sms * (per > 0 ? per : 1);
+        if (per < 1) per = 1;
+        if (cached) per_sm[dev].store(per, std::memory_order_relaxed);
     }
-    return grid;
+    return device_sm_count() * per;
 }
 
 cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t, uint64_t seed,
                                int64_t row, int m, int64_t rank_l[kLadder],
                                int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,
-                               RowState* st_row, double* b_out, WsHeader* hdr, cudaStream_t st) {
+                               RowState* st_row, double* b_out, WsHeader* hdr,
+                               uint32_t* sup_flag, cudaStream_t st) {
     // dynamic shared memory limits, set once per device (they belong to the
     // device's copy of the module)
     static unsigned long long attr_devices = 0ull;
@@ -2011,25 +2144,12 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     const int max_attempts = (flags & LAPSUM_FLAG_NO_RETRY) ? 1 : kMaxAttempts;
     float* sample = buf.sample + row * (int64_t)kSampleMax;
     const uint64_t c0 = (uint64_t)row << 32;
-    {
-        ProfScope ps_("bracket_sample", st);
-        launch_pdl(sample_kernel, dim3((m + kBlk - 1) / kBlk), dim3(kBlk), sample_smem, st, 
-            r_row, n, t, seed, c0, m, lad, force_miss, max_attempts, sample, buf.bins,
-            buf.ticket + 2, buf.ticket + 1, st_row);
-    }
-    const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
-    {
-        ProfScope ps_("bracket_fold", st);
-        launch_pdl(fold_kernel, dim3(buf.fold_grid), dim3(kFoldThreads), kFoldDynSmem, st, r_row, n, t, st_row,
-                                                                    buf.band[0],
-                                                        buf.bins, buf.fold_part, buf.ticket, hdr,
-                                                        vec);
-    }
+    const int sgrid = (m + kBlk - 1) / kBlk;
     // The band of the first bracket holds about n (h - l) / m scores.  When it
-    // should fit the on-chip sort with some room to spare, the solve kernel finishes
-    // by itself and the grid-wide extraction and second solve are not launched;
-    // a band that turns out larger is still solved exactly, inside the solve
-    // kernel.
+    // should fit the on-chip sort with some room to spare, the solve kernel
+    // finishes by itself, the fold builds no band histogram, and the grid-wide
+    // extraction and second solve are not launched; a band that turns out
+    // larger is still solved exactly, inside the solve kernel.
     const int64_t lo_rank = rank_l[0] > 0 ? rank_l[0] : 0;
     const int64_t hi_rank = rank_h[0] < m ? rank_h[0] : m;
     const double expect_band = (double)n * (double)(hi_rank - lo_rank) / (double)m;
@@ -2037,11 +2157,30 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
         ((flags & LAPSUM_FLAG_ONE_CTA_SOLVE) == 0 && (force_miss || expect_band > 0.75 * kBandSortMax))
             ? 1
             : 0;
+    // the fold builds the band histogram for the split solve, and for the
+    // one-CTA histogram solve when that is asked for
+    const int hist = (split || (flags & LAPSUM_FLAG_ONE_CTA_SOLVE) != 0) ? 1 : 0;
+    // both bracket ranks among each sample CTA's top_h keys: candidate selection
+    const int64_t need = rank_h[0] <= m ? rank_h[0] : (rank_l[0] >= 1 ? rank_l[0] : 0);
+    const int top_h = (need >= 1 && need <= kBlk && (int64_t)sgrid * need <= 4 * kBlk) ? (int)need : 0;
+    const size_t smem = top_h > 0 ? (size_t)4 * kBlk * sizeof(uint32_t) : sample_smem;
+    {
+        ProfScope ps_("bracket_sample", st);
+        launch_pdl(sample_kernel, dim3(sgrid), dim3(kBlk), smem, st, r_row, n, t, seed, c0, m,
+                   lad, force_miss, max_attempts, sample, buf.bins, buf.ticket + 2,
+                   buf.ticket + 1, st_row, top_h, buf.cand, hist, sup_flag);
+    }
+    const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
+    {
+        ProfScope ps_("bracket_fold", st);
+        launch_pdl(fold_kernel, dim3(buf.fold_grid), dim3(kFoldThreads), kFoldDynSmem, st, r_row,
+                   n, t, st_row, buf.band[0], buf.bins, buf.fold_part, vec, hist);
+    }
     {
         ProfScope ps_("bracket_solve", st);
-        launch_pdl(solve_kernel, dim3(1), dim3(kBlk), solve_smem, st, r_row, n, vec, k, t, st_row, buf.band[0],
-                                              buf.band[1], buf.bins, sample, m, lad, b_out, hdr,
-                                              split);
+        launch_pdl(solve_kernel, dim3(1), dim3(kBlk), solve_smem, st, r_row, n, vec, k, t, st_row,
+                   buf.band[0], buf.band[1], hist ? buf.bins : nullptr, sample, m, lad, b_out,
+                   hdr, split, (const double*)buf.fold_part, buf.fold_grid);
     }
     if (split) {
         {

@@ -4,6 +4,7 @@
 // Solver choice follows "Fast LapSum: Exact Differentiable Top-k at Million
 // Scale" (gist.science explainer pages), section 2.2: the full-sort solver
 // where sorting is affordable, probabilistic bracketing for n > 10^6.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -62,7 +63,7 @@ int resolve_path(int64_t n, int path) {
 struct Layout {
     size_t header, rows, partials, row_R, tickets, wlist, wtab, wflag;
     size_t keys0, keys1, seg_hist, tile_hist, plan;
-    size_t sample, band0, band1, bins, fold_part, fold_ticket, budgets;
+    size_t sample, band0, band1, bins, fold_part, fold_ticket, budgets, cand;
     size_t total;
 };
 
@@ -108,6 +109,7 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
         L.band1 = take((size_t)n * sizeof(float));
         L.bins = take((size_t)3 * kBins * sizeof(unsigned long long));
         L.fold_part = take((size_t)kFoldGridMax * 4 * sizeof(double));
+        L.cand = take((size_t)4096 * sizeof(uint32_t));
     }
     L.total = off;
     return L;
@@ -225,6 +227,22 @@ Profiler& profiler() {
 
 }  // namespace
 
+int device_sm_count() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 1;
+    if (dev >= 0 && dev < kMaxDevices) cache[dev].store(sms, std::memory_order_relaxed);
+    return sms;
+}
+
 void prof_begin(const char* name, cudaStream_t st) {
     Profiler& p = profiler();
     if (!p.on) return;
@@ -327,6 +345,9 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
     double* partials = reinterpret_cast<double*>(w + L.partials);
     const int vec = (aligned16(r) && aligned16(p) && (ld % 4) == 0) ? 1 : 0;
     cudaError_t e = cudaSuccess;
+    // the gradient support's per-row flags are cleared by the first kernel of
+    // the bracketing paths, and here for the radix path
+    const SupportView sv_all = want_sup ? support_view(support, B, n) : SupportView{};
 
     if (rp == LAPSUM_PATH_FULLSORT) {
         e = launch_onchip_forward(r, ld, p, b, sum_f, B, (int)n, k, k_rows, t, hdr, vec, st);
@@ -334,6 +355,8 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
     }
     if (rp == LAPSUM_PATH_RADIX) {
         e = cudaMemsetAsync(rows, 0, (size_t)B * sizeof(RowState), st);
+        if (e == cudaSuccess && want_sup)
+            e = cudaMemsetAsync(sv_all.flags, 0, (size_t)B * sizeof(uint32_t), st);
         if (e != cudaSuccess) return LAPSUM_ECUDA;
         RadixBuffers rb;
         rb.keys[0] = reinterpret_cast<uint32_t*>(w + L.keys0);
@@ -370,7 +393,8 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
         e = launch_rowbracket(r, ld, B, n, k, t, seed, m, rl, rh, path, rows,
                               reinterpret_cast<float*>(w + L.band0),
                               reinterpret_cast<float*>(w + L.band1), b, hdr,
-                              (aligned16(r) && (ld % 4) == 0) ? 1 : 0, st, budgets);
+                              (aligned16(r) && (ld % 4) == 0) ? 1 : 0, st, budgets,
+                              want_sup ? sv_all.flags : nullptr);
     } else {
         BracketBuffers bb;
         bb.sample = reinterpret_cast<float*>(w + L.sample);
@@ -378,6 +402,7 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
         bb.band[1] = reinterpret_cast<float*>(w + L.band1);
         bb.bins = reinterpret_cast<unsigned long long*>(w + L.bins);
         bb.fold_part = reinterpret_cast<double*>(w + L.fold_part);
+        bb.cand = reinterpret_cast<uint32_t*>(w + L.cand);
         bb.ticket = reinterpret_cast<uint32_t*>(w + L.fold_ticket);
         bb.fold_grid = bracket_fold_grid();
         if (bb.fold_grid > kFoldGridMax) bb.fold_grid = kFoldGridMax;
@@ -386,11 +411,11 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
         bracket_ladder(m, k / (double)n, rl, rh);
         for (int64_t row = 0; row < B && e == cudaSuccess; ++row) {
             e = launch_bracket_row(r + row * ld, n, k, t, seed, row, m, rl, rh, path, bb,
-                                   rows + row, b + row, hdr, st);
+                                   rows + row, b + row, hdr,
+                                   want_sup ? sv_all.flags + row : nullptr, st);
         }
     }
     if (e != cudaSuccess) return LAPSUM_ECUDA;
-    const SupportView sv_all = want_sup ? support_view(support, B, n) : SupportView{};
     for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
         const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
         const SupportView sv = want_sup ? support_rows(sv_all, r0, n) : SupportView{};

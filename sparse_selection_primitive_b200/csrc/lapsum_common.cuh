@@ -428,6 +428,26 @@ __device__ inline float block_max_f(float v, float* red) {
     for (int i = 1; i < nw; ++i) s = fmaxf(s, red[i]);
     return s;
 }
+// Block-wide sums of four doubles at once, valid in thread 0 only (one
+// barrier); `red` needs blockDim.x/32 rows.  Fixed order, deterministic.
+__device__ inline void block_sum4_to0(double (&v)[4], double (*red)[4]) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = warp_sum_d(v[i]);
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) red[w][i] = v[i];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            double s = 0.0;
+            for (int u = 0; u < nw; ++u) s += red[u][i];
+            v[i] = s;
+        }
+    }
+}
 __device__ inline long long block_sum_ll(long long v, long long* red) {
     int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll

@@ -8,6 +8,9 @@
 
 namespace lapsum {
 
+// Number of SMs of the current device (looked up once per device).
+int device_sm_count();
+
 // Optional per-kernel CUDA-event timing (lapsum_profile_enable).  A ProfScope
 // records an event pair around the launches in its lifetime when enabled.
 void prof_begin(const char* name, cudaStream_t st);
@@ -92,9 +95,12 @@ int64_t stream_tiles(int64_t n);
 constexpr int kSupWarps = 8;
 constexpr int kSupCap = 256;
 constexpr float kSupWindow = 90.f;  // f == 0 in fp32 beyond this |x|
+constexpr uint32_t kSupOverflow = 1u;  // a share held more scores than its capacity
+constexpr uint32_t kSupNear = 2u;      // some score of the row has |x| <= 50
 struct SupportView {
     int64_t* hdr;    // [0] n and [1] B of the forward that wrote the list
     double* b;       // [B] threshold of each row at that forward
+    uint32_t* flags; // [B] kSupOverflow | kSupNear, cleared by the forward's first kernel
     uint32_t* cnt;   // [B][tiles][8] entries found per share (> kSupCap: overflow)
     uint2* ent;      // [B][tiles][8][kSupCap] (position in the tile, x bits)
     float* val;      // [B][tiles][8][kSupCap] v at each entry (written by the backward)
@@ -162,6 +168,7 @@ struct BracketBuffers {
     unsigned long long* bins;  // band histogram of the first bracket: [3][2048]
     double* fold_part;   // fold partials, one record per CTA
     uint32_t* ticket;    // last-block counters: [0] fold, [1] sample; [2..2050) sample histogram
+    uint32_t* cand;      // the sample CTAs' top keys (at most 4096)
     int fold_grid;
 };
 int bracket_fold_grid();
@@ -182,10 +189,11 @@ cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, 
                               uint64_t seed, int m, int64_t rank_l[kLadder],
                               int64_t rank_h[kLadder], int flags, RowState* rows, float* band0,
                               float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st,
-                              const RowBudget* budgets = nullptr);
+                              const RowBudget* budgets = nullptr, uint32_t* sup_flags = nullptr);
 cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t, uint64_t seed,
                                int64_t row, int m, int64_t rank_l[kLadder],
                                int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,
-                               RowState* st_row, double* b_out, WsHeader* hdr, cudaStream_t st);
+                               RowState* st_row, double* b_out, WsHeader* hdr,
+                               uint32_t* sup_flag, cudaStream_t st);
 
 }  // namespace lapsum

@@ -73,11 +73,8 @@ extern "C" int lapsum_backward_noalloc(const float* r, int64_t ld, const double*
                    : LAPSUM_ECUDA;
     // The long-row reduction runs about 8 CTAs per SM over all rows; each CTA
     // leaves one record, and every record must fit in the array.
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return LAPSUM_ECUDA;
-    if ((int64_t)sms * 8 + B > kNoAllocRecords) return LAPSUM_EINVAL;
+    // (the same per-device SM count sizes the launch's grid)
+    if ((int64_t)device_sm_count() * 8 + B > kNoAllocRecords) return LAPSUM_EINVAL;
     void* base = nullptr;
     if (scratch_address(&base) != cudaSuccess) return LAPSUM_ECUDA;
     char* s = static_cast<char*>(base);

@@ -12,89 +12,12 @@
 // row results are deterministic.  No CTA ever waits for another.
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
+#include "stream_common.cuh"
 
 namespace lapsum {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kPer = kStreamTile / kThreads;  // 16
-
-// Swizzled slot of value j (0..15) in a lane's 16-float staging row, so that a
-// warp's 16-byte stores of the four float4 groups hit distinct banks.
-__device__ __forceinline__ int stage_slot16(int lane, int j) {
-    return lane * 16 + ((((j >> 2) ^ (lane >> 1)) & 3) << 2) + (j & 3);
-}
-
-template <bool VEC>
-__device__ __forceinline__ void load_tile(const float* __restrict__ row, int64_t n, int64_t base,
-                                          float (&x)[kPer], bool (&ok)[kPer]) {
-    if constexpr (VEC) {
-#pragma unroll
-        for (int q = 0; q < kPer / 4; ++q) {
-            const int64_t i0 = base + ((int64_t)q * kThreads + threadIdx.x) * 4;
-            if (i0 + 4 <= n) {
-                const float4 v = __ldcs(reinterpret_cast<const float4*>(row + i0));
-                x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) ok[4 * q + c] = true;
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    ok[4 * q + c] = i0 + c < n;
-                    x[4 * q + c] = ok[4 * q + c] ? row[i0 + c] : 0.f;
-                }
-            }
-        }
-    } else {
-        // scalar accesses in the same element order as the float4 path
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int64_t i = base + ((int64_t)(q / 4) * kThreads + threadIdx.x) * 4 + q % 4;
-            ok[q] = i < n;
-            x[q] = ok[q] ? row[i] : 0.f;
-        }
-    }
-}
-
-template <bool VEC>
-__device__ __forceinline__ void store_tile(float* __restrict__ row, int64_t n, int64_t base,
-                                           const float (&y)[kPer]) {
-    if constexpr (VEC) {
-#pragma unroll
-        for (int q = 0; q < kPer / 4; ++q) {
-            const int64_t i0 = base + ((int64_t)q * kThreads + threadIdx.x) * 4;
-            if (i0 + 4 <= n) {
-                __stcs(reinterpret_cast<float4*>(row + i0),
-                       make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    if (i0 + c < n) row[i0 + c] = y[4 * q + c];
-            }
-        }
-    } else {
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int64_t i = base + ((int64_t)(q / 4) * kThreads + threadIdx.x) * 4 + q % 4;
-            if (i < n) row[i] = y[q];
-        }
-    }
-}
-
-// True for exactly one CTA per row: the last to finish.  Release/acquire
-// through a fence around the ticket; the winner resets the ticket.
-__device__ __forceinline__ bool last_block_of_row(uint32_t* ticket, uint32_t nblocks, int* flag) {
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t prev = atomicAdd(ticket, 1u);
-        *flag = (prev == nblocks - 1);
-        if (*flag) *ticket = 0u;
-    }
-    __syncthreads();
-    if (*flag) __threadfence();
-    return *flag != 0;
-}
+using namespace stream_detail;
 
 // p = sigma((r - b)/t) for one 4096-score tile per CTA; sum f per row when
 // asked for (per-tile partials, combined in tile order by the row's last CTA).
@@ -143,6 +66,7 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
     float* stg = mstage + (SUP ? warp * 32 * kPer : 0);
     const int64_t share = (row * tiles + blockIdx.x) * kSupWarps + warp;
     uint32_t nm = 0u;  // near mask of this thread's 16 scores
+    bool near50 = false;  // some score with |x| <= 50 (the support serves the row)
     if (SUP && blockIdx.x == 0 && threadIdx.x == 0) sup.b[row] = brow;
     if (VEC && base + kStreamTile <= n) {
         const float4* r4 = reinterpret_cast<const float4*>(rr + base);
@@ -161,6 +85,7 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
                                cdf_from(m3, e3)));
             if (SUMF) sf += 0.5 * (double)((e0 + e1) + (e2 + e3));
             if (SUP) {
+                near50 |= fminf(fminf(fabsf(m0), fabsf(m1)), fminf(fabsf(m2), fabsf(m3))) <= 50.f;
                 nm |= (fabsf(m0) <= kSupWindow ? 1u : 0u) << (4 * q);
                 nm |= (fabsf(m1) <= kSupWindow ? 1u : 0u) << (4 * q + 1);
                 nm |= (fabsf(m2) <= kSupWindow ? 1u : 0u) << (4 * q + 2);
@@ -180,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
             y[q] = cdf_from(xs, e);
             if (SUMF && ok[q]) sf += 0.5 * (double)e;
             if (SUP) {
+                near50 |= ok[q] && fabsf(xs) <= 50.f;
                 nm |= ((ok[q] && fabsf(xs) <= kSupWindow) ? 1u : 0u) << q;
                 stg[stage_slot16(lane, q)] = xs;
             }
@@ -210,7 +136,15 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
             ++at;
         }
     }
-    if (SUP && lane == 0) sup.cnt[share] = cnt;
+    if (SUP) {
+        // the row's flags for the backward (set once: a read before each OR)
+        const bool any50 = __any_sync(0xffffffffu, near50);
+        if (lane == 0) {
+            sup.cnt[share] = cnt;
+            const uint32_t want = (any50 ? kSupNear : 0u) | (cnt > (uint32_t)kSupCap ? kSupOverflow : 0u);
+            if (want != 0u && (__ldcg(sup.flags + row) & want) != want) atomicOr(sup.flags + row, want);
+        }
+    }
     if (!SUMF) return;
     sf = block_sum_d(sf, red);
     if (threadIdx.x == 0) partials[row * tiles + blockIdx.x] = sf;
@@ -223,31 +157,9 @@ __global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float
 }
 
 // Pass 1 of the VJP.  Each CTA walks a strided share of the row's float4
-// groups and keeps, per thread, (mu, S, Sv) with mu the smallest |x| seen and
-// S = sum exp(-(|x| - mu)), Sv = sum v exp(-(|x| - mu)); a smaller |x| rescales
-// the sums once.  The CTA then reduces to one record, and the last CTA of the
-// row combines the records in CTA order into R = Sv / S.
-// Four scores at a time: a new minimum rescales the fp64 sums once, then the
-// four weights are summed in fp32 (each at most 1) and added in fp64.
-__device__ __forceinline__ void online_add4(float a0, float a1, float a2, float a3, float v0,
-                                            float v1, float v2, float v3, float& mu, double& s,
-                                            double& sv) {
-    const float m4 = fminf(fminf(a0, a1), fminf(a2, a3));
-    if (m4 < mu) {
-        const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(m4 - mu);
-        s *= sc;
-        sv *= sc;
-        mu = m4;
-    }
-    const float w0 = __expf(mu - a0), w1 = __expf(mu - a1), w2 = __expf(mu - a2),
-                w3 = __expf(mu - a3);
-    s += (double)((w0 + w1) + (w2 + w3));
-    sv += (double)(fmaf(w0, v0, w1 * v1) + fmaf(w2, v2, w3 * v3));
-}
-__device__ __forceinline__ void online_add(float ax, float vv, float& mu, double& s, double& sv) {
-    online_add4(ax, INFINITY, INFINITY, INFINITY, vv, 0.f, 0.f, 0.f, mu, s, sv);
-}
-
+// groups with the online sums (mu, S, Sv); the CTA then reduces to one record,
+// and the last CTA of the row combines the records in CTA order into
+// R = Sv / S.
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
@@ -496,12 +408,7 @@ cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* 
                                       double* partials, double* row_R, uint32_t* tickets, int vec,
                                       const uint32_t* need, cudaStream_t st) {
     // pass 1 runs persistent CTAs: about 8 per SM over all rows, at most one per tile
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int sms = device_sm_count();
     // As a fallback (need != nullptr) it usually has nothing to do: one CTA
     // per SM keeps the cost of launching it small.
     const int64_t cta_per_sm = need != nullptr ? 1 : 8;
@@ -554,12 +461,7 @@ cudaError_t launch_backward_kt(const float* r, int64_t ld, const double* b, cons
                                int64_t B, int64_t n, double t, double* partials,
                                uint32_t* tickets, double* g_k, double* g_t, int vec,
                                cudaStream_t st) {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int sms = device_sm_count();
     // records of 8 doubles: at most half as many CTAs per row as the partials
     // region has 4-double slots per row (max(tiles, 2))
     int64_t cap = stream_tiles(n) > 2 ? stream_tiles(n) / 2 : 1;

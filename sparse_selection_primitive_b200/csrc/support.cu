@@ -18,20 +18,24 @@
 //   zeroed in shared memory, its entries are placed, and it is written out
 //   with coalesced 16-byte stores, so every g value is written exactly once.
 //
-// A row is handed to the dense two-pass kernels when its list overflowed, was
-// written for another (n, B) or another b, holds an index out of range, or
-// its smallest |x| is above 50 (then scores outside the list could weigh in R).
+// A row is computed densely (v and r read everywhere) by the same two kernels
+// when its list overflowed, was written for another (n, B) or another b, or
+// no score of the row has |x| <= 50 (then scores outside the list could weigh
+// in R); the forward's emit pass records the first and the last of these per
+// row, so every CTA knows the row's mode before it starts.
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
+#include "stream_common.cuh"
 
 namespace lapsum {
 namespace {
 
+using stream_detail::online_add;
+using stream_detail::online_add4;
 constexpr int kThreads = 256;
 constexpr int kTile = kStreamTile;
 constexpr int kShares = kSupWarps;
 constexpr int kGroupMax = kThreads / kShares;  // tiles per pass-A CTA (one share per thread)
-constexpr float kDenseAbove = 50.f;
 constexpr size_t kAlignSup = 256;
 
 size_t up256(size_t x) { return (x + kAlignSup - 1) / kAlignSup * kAlignSup; }
@@ -68,10 +72,22 @@ __device__ __forceinline__ void sup_add(float ax, float vv, float& mu, double& s
     sv += (double)(w * vv);
 }
 
+// The row's mode: the list serves it unless it was written for another call
+// shape or threshold, overflowed, or no score has |x| <= 50.
+__device__ __forceinline__ bool row_is_dense(const SupportView& sup, const double* b,
+                                             int64_t row, int64_t n, int64_t B_total) {
+    const bool match = sup.hdr[0] == n && sup.hdr[1] == B_total &&
+                       __double_as_longlong(sup.b[row]) == __double_as_longlong(b[row]);
+    const uint32_t fl = sup.flags[row];
+    return !match || (fl & kSupOverflow) != 0u || (fl & kSupNear) == 0u;
+}
+
+template <bool VEC>
 __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
-    const double* __restrict__ b, const float* __restrict__ v, int64_t ld, int64_t n,
-    int64_t B_total, int group, SupportView sup, double* __restrict__ partials,
-    double* __restrict__ row_R, uint32_t* __restrict__ tickets, uint32_t* __restrict__ dense_flag) {
+    const float* __restrict__ r, const double* __restrict__ b, const float* __restrict__ v,
+    int64_t ld, int64_t n, double t, int64_t B_total, int group, SupportView sup,
+    double* __restrict__ partials, double* __restrict__ row_R, uint32_t* __restrict__ tickets,
+    uint32_t* __restrict__ dense_flag) {
     pdl_wait();
     __shared__ uint32_t pre[kThreads + 1];  // exclusive prefix of the group's share counts
     __shared__ uint32_t wtot[kThreads / 32];
@@ -84,12 +100,32 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     const int64_t ngroups = (tiles + group - 1) / group;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* vr = v + row * ld;
-    // the list must come from a forward over the same (n, B) with this b
-    const bool match = sup.hdr[0] == n && sup.hdr[1] == B_total &&
-                       __double_as_longlong(sup.b[row]) == __double_as_longlong(b[row]);
-    int bad = match ? 0 : 1;
-    float mu = INFINITY, amin = INFINITY;
+    const bool dense = row_is_dense(sup, b, row, n, B_total);
+    float mu = INFINITY;
     double s = 0.0, sv = 0.0;
+    if (dense) {
+        // every score of the row: this CTA's strided share of it
+        const Thr th = make_thr(b[row], t);
+        const float* rr = r + row * ld;
+        const int64_t stride = nblk * kThreads;
+        const int64_t gt = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+        if (VEC) {
+            const int64_t n4 = n >> 2;
+            const float4* r4 = reinterpret_cast<const float4*>(rr);
+            const float4* v4 = reinterpret_cast<const float4*>(vr);
+            for (int64_t i = gt; i < n4; i += stride) {
+                const float4 x0 = __ldcs(r4 + i), y0 = __ldcs(v4 + i);
+                online_add4(fabsf(scaled_margin(x0.x, th)), fabsf(scaled_margin(x0.y, th)),
+                            fabsf(scaled_margin(x0.z, th)), fabsf(scaled_margin(x0.w, th)), y0.x,
+                            y0.y, y0.z, y0.w, mu, s, sv);
+            }
+            for (int64_t j = (n4 << 2) + gt; j < n; j += stride)
+                online_add(fabsf(scaled_margin(rr[j], th)), vr[j], mu, s, sv);
+        } else {
+            for (int64_t j = gt; j < n; j += stride)
+                online_add(fabsf(scaled_margin(rr[j], th)), vr[j], mu, s, sv);
+        }
+    }
     const uint64_t keep = l2_evict_last_policy();
     // count of share i of group gi: (tile gi * group + i / 8, share i % 8), or 0
     // (the buffer holds a list for this (n, B) whatever it was written for,
@@ -102,14 +138,11 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     };
     // persistent over groups of tiles; the next group's counts load while
     // the current group's entries are gathered
-    uint32_t c_next = share_count(blockIdx.x);
-    for (int64_t gi = blockIdx.x; gi < ngroups; gi += nblk) {
+    uint32_t c_next = dense ? 0u : share_count(blockIdx.x);
+    for (int64_t gi = dense ? ngroups : blockIdx.x; gi < ngroups; gi += nblk) {
         const int64_t t0 = gi * group;
-        uint32_t c = match ? c_next : 0u;
-        if (c > (uint32_t)kSupCap) {
-            bad = 1;
-            c = 0;
-        }
+        uint32_t c = c_next;
+        if (c > (uint32_t)kSupCap) c = 0;  // an overflowed row is dense (not reached)
         // block exclusive scan of the counts
         uint32_t inc = c;
 #pragma unroll
@@ -160,10 +193,7 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
             for (int u = 0; u < U; ++u) {
                 if (!ok[u]) continue;
                 gpos[u] += (int32_t)(e[u].x & (kTile - 1));
-                if (e[u].x >= (uint32_t)kTile || gpos[u] >= lim) {
-                    ok[u] = false;
-                    bad = 1;
-                }
+                if (gpos[u] >= lim) ok[u] = false;  // never past the row
             }
             float vv[U];
 #pragma unroll
@@ -172,25 +202,21 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
             for (int u = 0; u < U; ++u) {
                 if (!ok[u]) continue;
                 const float ax = fabsf(__uint_as_float(e[u].y));
-                amin = fminf(amin, ax);
                 sup_add(ax, vv[u], mu, s, sv);
                 st_keep(val + slot[u], vv[u], keep);
             }
         }
     }
-    // CTA record (mu, S, Sv, min |x| or -1 when the list cannot serve the row)
-    const int anybad_cta = __syncthreads_or(bad);
+    // CTA record (mu, S, Sv)
     const float mb = block_min_f(mu, fred);
     const double sc = (mu == INFINITY) ? 0.0 : exp((double)mb - (double)mu);
     s = block_sum_d(s * sc, red);
     sv = block_sum_d(sv * sc, red);
-    const float am = block_min_f(amin, fred);
     if (threadIdx.x == 0) {
         double* pr = partials + (row * nblk + blockIdx.x) * 4;
         pr[0] = (double)mb;
         pr[1] = s;
         pr[2] = sv;
-        pr[3] = anybad_cta ? -1.0 : (double)am;
     }
     __threadfence();
     __syncthreads();
@@ -202,17 +228,10 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     __syncthreads();
     if (!flag) return;
     __threadfence();
-    float mloc = INFINITY, aloc = INFINITY;
-    int rbad = 0;
-    for (int64_t k = threadIdx.x; k < nblk; k += kThreads) {
-        const double* pr = partials + (row * nblk + k) * 4;
-        mloc = fminf(mloc, (float)pr[0]);
-        if (pr[3] < 0.0) rbad = 1;
-        else aloc = fminf(aloc, (float)pr[3]);
-    }
+    float mloc = INFINITY;
+    for (int64_t k = threadIdx.x; k < nblk; k += kThreads)
+        mloc = fminf(mloc, (float)partials[(row * nblk + k) * 4]);
     const double mrow = (double)block_min_f(mloc, fred);
-    const float arow = block_min_f(aloc, fred);
-    const int anybad = __syncthreads_or(rbad);
     double a = 0.0, av = 0.0;
     for (int64_t k = threadIdx.x; k < nblk; k += kThreads) {
         const double* pr = partials + (row * nblk + k) * 4;
@@ -224,8 +243,8 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     a = block_sum_d(a, red);
     av = block_sum_d(av, red);
     if (threadIdx.x == 0) {
-        row_R[row] = a > 0.0 ? av / a : 0.0;
-        dense_flag[row] = (anybad || arow > kDenseAbove) ? 1u : 0u;
+        row_R[row] = dense ? av / a : (a > 0.0 ? av / a : 0.0);
+        dense_flag[row] = dense ? 1u : 0u;
     }
 }
 
@@ -238,9 +257,11 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
 // together (the entries speculatively), so a tile costs one memory round
 // trip; the share is zeroed in the warp's 2 KB of shared memory, its entries
 // are placed, and it is written with 16-byte streaming stores.
+// Rows computed densely take g = (f/t)(v - R) from r and v over the tile.
 template <bool VEC>
 __global__ void __launch_bounds__(kThreads) sup_write_kernel(
     SupportView sup, const uint32_t* __restrict__ dense_flag, const double* __restrict__ row_R,
+    const float* __restrict__ r, const double* __restrict__ b, const float* __restrict__ v,
     float* __restrict__ g, int64_t ld, int64_t n, double t) {
     pdl_wait();
     __shared__ __align__(16) float stage[kShares][kTile / kShares];
@@ -258,7 +279,31 @@ __global__ void __launch_bounds__(kThreads) sup_write_kernel(
     const uint32_t c = __ldcs(sup.cnt + share);  // <= kSupCap: checked by pass A
     const uint2 e0 = __ldcs(ent + lane);
     const float v0 = __ldcs(val + lane);
-    if (dflag) return;  // the dense kernels own this row
+    if (dflag) {
+        // four scores at a time, in the striped order of the other tile kernels
+        const Thr th = make_thr(b[row], t);
+        const float* rr = r + row * ld;
+        const float* vr = v + row * ld;
+        float* gr = g + row * ld;
+        auto g_of = [&](float x, float vv) {
+            const float f = 0.5f * neg_abs_exp(scaled_margin(x, th));
+            return f * th.inv_t * (float)((double)vv - R);
+        };
+#pragma unroll 1
+        for (int q = 0; q < kTile / (4 * kThreads); ++q) {
+            const int64_t i0 = base + ((int64_t)q * kThreads + threadIdx.x) * 4;
+            if (VEC && i0 + 4 <= n) {
+                const float4 x = __ldcs(reinterpret_cast<const float4*>(rr + i0));
+                const float4 y = __ldcs(reinterpret_cast<const float4*>(vr + i0));
+                __stcs(reinterpret_cast<float4*>(gr + i0),
+                       make_float4(g_of(x.x, y.x), g_of(x.y, y.y), g_of(x.z, y.z), g_of(x.w, y.w)));
+            } else {
+                for (int c = 0; c < 4; ++c)
+                    if (i0 + c < n) gr[i0 + c] = g_of(rr[i0 + c], vr[i0 + c]);
+            }
+        }
+        return;
+    }
     const float hinv = (float)(0.5 / t);
     float* st = stage[warp];
     float4* s4 = reinterpret_cast<float4*>(st);
@@ -287,18 +332,8 @@ __global__ void __launch_bounds__(kThreads) sup_write_kernel(
     }
 }
 
-int sm_count() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    return sms;
-}
-
 struct SupOffsets {
-    size_t hdr, b, cnt, ent, val, total;
+    size_t hdr, b, flags, cnt, ent, val, total;
 };
 
 SupOffsets sup_offsets(int64_t B, int64_t n) {
@@ -312,6 +347,7 @@ SupOffsets sup_offsets(int64_t B, int64_t n) {
     };
     o.hdr = take(2 * sizeof(int64_t));
     o.b = take((size_t)B * sizeof(double));
+    o.flags = take((size_t)B * sizeof(uint32_t));
     o.cnt = take((size_t)B * tiles * kShares * sizeof(uint32_t));
     o.ent = take((size_t)B * tiles * kShares * kSupCap * sizeof(uint2));
     o.val = take((size_t)B * tiles * kShares * kSupCap * sizeof(float));
@@ -329,6 +365,7 @@ SupportView support_view(void* base, int64_t B, int64_t n) {
     SupportView s;
     s.hdr = reinterpret_cast<int64_t*>(p + o.hdr);
     s.b = reinterpret_cast<double*>(p + o.b);
+    s.flags = reinterpret_cast<uint32_t*>(p + o.flags);
     s.cnt = reinterpret_cast<uint32_t*>(p + o.cnt);
     s.ent = reinterpret_cast<uint2*>(p + o.ent);
     s.val = reinterpret_cast<float*>(p + o.val);
@@ -339,6 +376,7 @@ SupportView support_rows(const SupportView& s, int64_t r0, int64_t n) {
     const int64_t per_row = stream_tiles(n) * kShares;
     SupportView o = s;
     o.b += r0;
+    o.flags += r0;
     o.cnt += r0 * per_row;
     o.ent += r0 * per_row * kSupCap;
     o.val += r0 * per_row * kSupCap;
@@ -353,12 +391,13 @@ cudaError_t launch_backward_support(const float* r, int64_t ld, const double* b,
     const int64_t tiles = stream_tiles(n);
     // pass A: one wave of resident CTAs walking groups of up to 32 tiles;
     // pass B: one CTA per tile
-    static int cap_a = 0;
-    if (cap_a == 0) {
+    static int per_sm_a = 0;
+    if (per_sm_a == 0) {
         int pa = 0;
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pa, sup_reduce_kernel, kThreads, 0);
-        cap_a = (pa > 0 ? pa : 1) * sm_count();
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pa, sup_reduce_kernel<true>, kThreads, 0);
+        per_sm_a = pa > 0 ? pa : 1;
     }
+    const int cap_a = per_sm_a * device_sm_count();
     int64_t want = cap_a / B;
     if (want < 1) want = 1;
     // groups of at most 32 tiles, as many per CTA as it takes, all CTAs alike
@@ -370,21 +409,25 @@ cudaError_t launch_backward_support(const float* r, int64_t ld, const double* b,
     const int64_t per_row = ngroups < want ? ngroups : want;
     {
         ProfScope ps_("sup_reduce", st);
-        launch_pdl(sup_reduce_kernel, dim3(dim3((unsigned)per_row, (unsigned)B)), dim3(kThreads), 0, st, 
-            b, v, ld, n, B_total, (int)group, sup, partials, row_R, tickets, dense_flag);
+        const dim3 grid((unsigned)per_row, (unsigned)B);
+        if (vec)
+            launch_pdl(sup_reduce_kernel<true>, grid, dim3(kThreads), 0, st, r, b, v, ld, n, t,
+                       B_total, (int)group, sup, partials, row_R, tickets, dense_flag);
+        else
+            launch_pdl(sup_reduce_kernel<false>, grid, dim3(kThreads), 0, st, r, b, v, ld, n, t,
+                       B_total, (int)group, sup, partials, row_R, tickets, dense_flag);
     }
     {
         ProfScope ps_("sup_write", st);
         const dim3 grid((unsigned)tiles, (unsigned)B);
         if (vec)
-            launch_pdl(sup_write_kernel<true>, dim3(grid), dim3(kThreads), 0, st, sup, dense_flag, row_R, g, ld, n, t);
+            launch_pdl(sup_write_kernel<true>, grid, dim3(kThreads), 0, st, sup, dense_flag, row_R,
+                       r, b, v, g, ld, n, t);
         else
-            launch_pdl(sup_write_kernel<false>, dim3(grid), dim3(kThreads), 0, st, sup, dense_flag, row_R, g, ld, n,
-                                                                t);
+            launch_pdl(sup_write_kernel<false>, grid, dim3(kThreads), 0, st, sup, dense_flag, row_R,
+                       r, b, v, g, ld, n, t);
     }
-    // rows the list could not serve: dense recompute (exits at once otherwise)
-    return launch_backward_stream_if(r, ld, b, v, g, B, n, t, partials, row_R, tickets, vec,
-                                     dense_flag, st);
+    return cudaGetLastError();
 }
 
 }  // namespace lapsum

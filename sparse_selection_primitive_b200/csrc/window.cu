@@ -253,15 +253,6 @@ __global__ void __launch_bounds__(kThreads) window_write_kernel(
     }
 }
 
-int sm_count() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    return sms;
-}
 
 }  // namespace
 
@@ -280,13 +271,13 @@ cudaError_t launch_backward_window(const float* r, int64_t ld, const double* b, 
                                    const WindowBuffers& wb, double* partials, double* row_R,
                                    uint32_t* tickets, int vec, cudaStream_t st) {
     const int64_t ntiles = window_tiles(n);
-    int64_t per_row = ((int64_t)sm_count() * 8 + B - 1) / B;
+    int64_t per_row = ((int64_t)device_sm_count() * 8 + B - 1) / B;
     if (per_row > ntiles) per_row = ntiles;
     if (per_row < 1) per_row = 1;
     // each pass CTA owns an equal share of the row's list capacity
     const uint32_t cap_cta = (uint32_t)(((int64_t)window_capacity(n) + per_row - 1) / per_row);
     const dim3 grid((unsigned)per_row, (unsigned)B);
-    int64_t wr = ntiles < (int64_t)sm_count() * 8 ? ntiles : (int64_t)sm_count() * 8;
+    int64_t wr = ntiles < (int64_t)device_sm_count() * 8 ? ntiles : (int64_t)device_sm_count() * 8;
     const dim3 wgrid((unsigned)wr, (unsigned)B);
     {
         ProfScope ps_("window_pass", st);

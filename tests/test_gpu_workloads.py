@@ -4,7 +4,8 @@ configuration the benchmark times (AUTO path, one call over all rows).
 * single row n=1024 and the MoE batch: oracle on every row (C1) or on a
   seeded sample of rows plus the first and last (16384 x 256);
 * memory-selection batch 256 x 65536: every row's b against the stored oracle
-  thresholds, p and g on a sample of rows;
+  thresholds, p and g on a sample of rows, with the AUTO solver and with the
+  full-sort (radix) solver the configuration names;
 * the two bracketing rows (n = 3,342,336 and 10^8): b against the stored
   oracle threshold and, independently, against the oracle's sign function at
   b +- tolerance; p and g on every element; the bracketing b also against
@@ -68,6 +69,25 @@ def test_memory_select_batch(cuda_device):
         check_row(r[i], v[i], w.k, w.t, out["b"][i], out["p"][i], out["g"][i], b_ref=b_ref[i],
                   label=f"{w.name} row {i}")
     assert np.max(np.abs(out["p"].sum(axis=1) - w.k)) <= 1e-3
+
+
+def test_memory_select_batch_full_sort(cuda_device):
+    # The configuration as it is written: the full-sort solver (radix sort of
+    # every row) on the whole 256 x 65536 batch, forward and gradient-support
+    # backward as the benchmark runs them; every row's b against the stored
+    # oracle thresholds, p and g element by element on a sample of rows.
+    w = WORKLOADS["memory_select_256x65536"]
+    ref = stored(w.name)
+    r, v = make_inputs(w)
+    out = run_gpu(r, w.k, w.t, path="fullsort", v=v, support=True)
+    b_ref = np.array(ref["b"])
+    err = np.abs(out["b"] - b_ref) / np.maximum(w.t, np.abs(b_ref))
+    assert err.max() <= TOL_B, err.max()
+    for i in [0, 1, 100, 200, 255]:
+        check_row(r[i], v[i], w.k, w.t, out["b"][i], out["p"][i], out["g"][i], b_ref=b_ref[i],
+                  label=f"{w.name} full sort row {i}")
+    assert np.max(np.abs(out["p"].sum(axis=1) - w.k)) <= 1e-3
+    assert out["p"].min() >= 0.0 and out["p"].max() <= 1.0
 
 
 def _bracket_row(name, cuda_device):
