@@ -1602,10 +1602,31 @@ __device__ __forceinline__ void block_sums(double (&v)[N], SolveSmemAll* sm) {
 // The first attempt on a band small enough for the on-chip sort (the usual
 // case): sort, scan and root in a function of its own, so that this path keeps
 // its registers and its code compact, apart from the widening and narrowing
-// machinery.  Returns true when the bracket certifies (b in sm->res).
-__device__ __noinline__ bool first_small_band(const float* __restrict__ band, long long nb,
-                                              Tails tl, double k, double t, SolveSmemAll* sm) {
-    solve_small_band(band, nb, tl, k, t, sm);
+// machinery.  pre[e] holds band score e * kBlk + threadIdx.x (loaded early by
+// the caller; the sort does not care where each key starts).  Returns true
+// when the bracket certifies (b in sm->res).
+template <int E>
+__device__ void sort_preloaded(const float (&pre)[4], long long nb, SolveSmemAll* sm) {
+    uint32_t key[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const long long j = (long long)e * kBlk + threadIdx.x;
+        key[e] = j < nb ? to_key(pre[e]) : 0xffffffffu;
+    }
+    bitonic_sort_row<E, kBlk, kBlk>(key, threadIdx.x, sm->u.sort.xch);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const long long j = (long long)threadIdx.x * E + e;
+        if (j < nb) sm->u.sort.sorted[j] = from_key(key[e]);
+    }
+    __syncthreads();
+}
+__device__ __noinline__ bool first_small_band(const float (&pre)[4], long long nb, Tails tl,
+                                              double k, double t, SolveSmemAll* sm) {
+    if (nb <= kBlk) sort_preloaded<1>(pre, nb, sm);
+    else if (nb <= 2 * kBlk) sort_preloaded<2>(pre, nb, sm);
+    else sort_preloaded<4>(pre, nb, sm);
+    solve_sorted_block(FloatGet{sm->u.sort.sorted}, nb, tl, k, t, &sm->ss, &sm->res);
     return sm->res.F_aL >= k && sm->res.F_aR <= k;
 }
 
@@ -1628,6 +1649,18 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
         sm->bcast[2] = 0xffffffffu;
         sm->bcast[3] = 0u;
     }
+    // every load this kernel needs first is issued at once: the row record,
+    // the fold CTAs' records and the first 4096 band scores (read as far as
+    // the row is long; only the first n_band are used)
+    const float aL0 = st->a_L, aR0 = st->a_R;
+    const long long nb = (long long)st->n_band;
+    float pre[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int64_t j = (int64_t)e * kBlk + threadIdx.x;
+        pre[e] = j < n ? __ldcg(band0 + j) : 0.f;
+    }
+    Tails tl;
     {
         // the fold CTAs' records, combined in CTA order: right count, tail
         // sums and the non-finite flag of the row
@@ -1650,27 +1683,24 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
                 set_status(hdr, kDevNonFinite);
             }
         }
-        __syncthreads();
-    }
-    if (st->status & kDevNonFinite) {
-        if (threadIdx.x == 0) {
-            st->b = nan("");
-            *b_out = nan("");
+        if (tot[3] > 0.0) {
+            if (threadIdx.x == 0) {
+                st->b = nan("");
+                *b_out = nan("");
+            }
+            return;
         }
-        return;
+        tl.hasL = isfinite(aL0);
+        tl.aL = aL0;
+        tl.SL = tot[1];
+        tl.hasR = isfinite(aR0);
+        tl.aR = aR0;
+        tl.SR = tot[2];
+        tl.cntR = tot[0];
     }
-    Tails tl;
-    tl.hasL = isfinite(st->a_L);
-    tl.aL = st->a_L;
-    tl.SL = st->S_L;
-    tl.hasR = isfinite(st->a_R);
-    tl.aR = st->a_R;
-    tl.SR = st->S_R;
-    tl.cntR = (double)st->cnt_R;
-    const long long nb = (long long)st->n_band;
-    if (nb <= kBandSortMax && st->max_attempts >= 1) {
+    if (nb <= kBandSortMax) {
         phase_mark(st, 19);
-        const bool ok = first_small_band(band0, nb, tl, k, t, sm);
+        const bool ok = first_small_band(pre, nb, tl, k, t, sm);
         phase_mark(st, 21);
         if (ok) {
             if (threadIdx.x == 0) {

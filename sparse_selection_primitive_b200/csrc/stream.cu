@@ -29,7 +29,7 @@ using namespace stream_detail;
 // order, and records how many it found (a count above the share's capacity
 // marks an overflow; the backward then recomputes the row densely).
 template <bool VEC, bool SUMF, bool SUP>
-__global__ void __launch_bounds__(kThreads, SUP ? 5 : 1) emit_kernel(const float* __restrict__ r, int64_t ld,
+__global__ void __launch_bounds__(kThreads, SUP ? 6 : 1) emit_kernel(const float* __restrict__ r, int64_t ld,
                                                         float* __restrict__ p,
                                                         const double* __restrict__ b,
                                                         double* __restrict__ sumf, int64_t n,

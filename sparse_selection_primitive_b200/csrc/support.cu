@@ -60,6 +60,46 @@ __device__ __forceinline__ void st_keep(float* p, float v, uint64_t pol) {
                  : "memory");
 }
 
+// Merges a record (m, s, sv) -- sums of weights relative to e^{-m} -- into
+// the running (mu, S, Sv); a smaller m rescales the running sums.
+__device__ __forceinline__ void online_merge(float m, double s, double sv, float& mu, double& S,
+                                             double& Sv) {
+    if (m == INFINITY) return;
+    if (m < mu) {
+        const double sc = (mu == INFINITY) ? 0.0 : exp((double)m - (double)mu);
+        S *= sc;
+        Sv *= sc;
+        mu = m;
+    }
+    const double f = exp((double)mu - (double)m);
+    S += s * f;
+    Sv += sv * f;
+}
+
+// The online sums of every thread of the CTA combined into thread 0 (one
+// barrier): warp shuffles, then thread 0 merges the warps in order.
+__device__ __forceinline__ void cta_online_combine(float& mu, double& s, double& sv, float* wmu,
+                                                   double* ws, double* wsv) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const float mw = warp_min_f(mu);
+    const double sc = (mu == INFINITY) ? 0.0 : exp((double)mw - (double)mu);
+    const double s_w = warp_sum_d(s * sc), sv_w = warp_sum_d(sv * sc);
+    if (lane == 0) {
+        wmu[w] = mw;
+        ws[w] = s_w;
+        wsv[w] = sv_w;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = INFINITY;
+        double a = 0.0, av = 0.0;
+        for (int u = 0; u < kThreads / 32; ++u) online_merge(wmu[u], ws[u], wsv[u], m, a, av);
+        mu = m;
+        s = a;
+        sv = av;
+    }
+}
+
 __device__ __forceinline__ void sup_add(float ax, float vv, float& mu, double& s, double& sv) {
     if (ax < mu) {
         const double sc = (mu == INFINITY) ? 0.0 : (double)__expf(ax - mu);
@@ -91,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     pdl_wait();
     __shared__ uint32_t pre[kThreads + 1];  // exclusive prefix of the group's share counts
     __shared__ uint32_t wtot[kThreads / 32];
-    __shared__ double red[kThreads / 32];
-    __shared__ float fred[kThreads / 32];
+    __shared__ float wmu[kThreads / 32];
+    __shared__ double ws[kThreads / 32], wsv[kThreads / 32];
     __shared__ int flag;
     const int64_t row = blockIdx.y;
     const int64_t nblk = gridDim.x;
@@ -207,20 +247,14 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
             }
         }
     }
-    // CTA record (mu, S, Sv)
-    const float mb = block_min_f(mu, fred);
-    const double sc = (mu == INFINITY) ? 0.0 : exp((double)mb - (double)mu);
-    s = block_sum_d(s * sc, red);
-    sv = block_sum_d(sv * sc, red);
+    // CTA record (mu, S, Sv): one barrier
+    cta_online_combine(mu, s, sv, wmu, ws, wsv);
     if (threadIdx.x == 0) {
         double* pr = partials + (row * nblk + blockIdx.x) * 4;
-        pr[0] = (double)mb;
+        pr[0] = (double)mu;
         pr[1] = s;
         pr[2] = sv;
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
+        __threadfence();
         const uint32_t prev = atomicAdd(&tickets[row], 1u);
         flag = (prev == (uint32_t)nblk - 1u);
         if (flag) tickets[row] = 0u;
@@ -228,20 +262,14 @@ __global__ void __launch_bounds__(kThreads, 5) sup_reduce_kernel(
     __syncthreads();
     if (!flag) return;
     __threadfence();
+    // the row's records in CTA order, each thread's share combined online
     float mloc = INFINITY;
-    for (int64_t k = threadIdx.x; k < nblk; k += kThreads)
-        mloc = fminf(mloc, (float)partials[(row * nblk + k) * 4]);
-    const double mrow = (double)block_min_f(mloc, fred);
     double a = 0.0, av = 0.0;
     for (int64_t k = threadIdx.x; k < nblk; k += kThreads) {
         const double* pr = partials + (row * nblk + k) * 4;
-        if (pr[0] == INFINITY) continue;
-        const double f = exp(mrow - pr[0]);
-        a += pr[1] * f;
-        av += pr[2] * f;
+        online_merge((float)__ldcg(pr), __ldcg(pr + 1), __ldcg(pr + 2), mloc, a, av);
     }
-    a = block_sum_d(a, red);
-    av = block_sum_d(av, red);
+    cta_online_combine(mloc, a, av, wmu, ws, wsv);
     if (threadIdx.x == 0) {
         row_R[row] = dense ? av / a : (a > 0.0 ? av / a : 0.0);
         dense_flag[row] = dense ? 1u : 0u;
