@@ -72,7 +72,8 @@ enum lapsum_path {
 /* Score element types of the router entry points. */
 enum lapsum_dtype {
     LAPSUM_DTYPE_F32 = 0,  /* float */
-    LAPSUM_DTYPE_BF16 = 1  /* bfloat16, passed as its 16-bit patterns (uint16_t) */
+    LAPSUM_DTYPE_BF16 = 1, /* bfloat16, passed as its 16-bit patterns (uint16_t) */
+    LAPSUM_DTYPE_F16 = 2   /* IEEE half, passed as its 16-bit patterns (uint16_t) */
 };
 
 /* Test and diagnostic flags, OR-ed into `path`. */
@@ -151,8 +152,8 @@ int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t
 
 /*
  * Router form for short rows (n <= 4096, the on-chip sort), e.g. the scores of
- * a mixture-of-experts router: scores r of type `dtype` (fp32, or bf16 bit
- * patterns widened exactly to fp32), p (fp32) and b (fp64) as lapsum_forward,
+ * a mixture-of-experts router: scores r of type `dtype` (fp32, or bf16 or fp16
+ * bit patterns widened exactly to fp32), p (fp32) and b (fp64) as lapsum_forward,
  * and, when sel_cnt is not NULL, the sparse support of each row next to p:
  * sel_idx[row*cap + j] and sel_p[row*cap + j], j < min(cap, sel_cnt[row]),
  * are the positions (ascending) and values of the scores with p > eps, and
@@ -175,15 +176,43 @@ int lapsum_backward_router(const void* r, int dtype, int64_t ld, const double* b
                            float* g, int64_t B, int64_t n, double t, void* stream);
 
 /*
+ * Scores of a 16-bit type at any row length: lapsum_forward_lowp and
+ * lapsum_backward_lowp take r as `dtype` (LAPSUM_DTYPE_BF16 or _F16 bit
+ * patterns, or LAPSUM_DTYPE_F32) with row stride ld, and otherwise behave as
+ * lapsum_forward_support / lapsum_backward_support (support may be NULL: then
+ * as lapsum_forward / lapsum_backward).  The values solved for are the exact
+ * fp32 widenings of the scores (section 2.1 of the pages states the problem
+ * for real scores; a narrower storage type is this library's addition).
+ * Rows of n <= 4096 with LAPSUM_PATH_AUTO or LAPSUM_PATH_FULLSORT read the
+ * 16-bit scores directly in the on-chip kernels; longer rows (or another
+ * path) first widen the rows into the tail of ws (one streaming pass, 2 bytes
+ * read and 4 written per score) and then run the fp32 solvers on the copy.
+ * p, b, sum_f, v and g are as in the fp32 calls (g is fp32).  Workspace:
+ * lapsum_workspace_bytes_lowp(B, n, ld, k, path) and
+ * lapsum_backward_workspace_bytes_lowp(B, n, ld) bytes (0: invalid sizes or
+ * path; the backward of rows with n <= 4096 needs none, ws may then be NULL).
+ * Errors: LAPSUM_EINVAL for an unknown dtype, else as the fp32 calls.
+ */
+size_t lapsum_workspace_bytes_lowp(int64_t B, int64_t n, int64_t ld, double k, int path);
+size_t lapsum_backward_workspace_bytes_lowp(int64_t B, int64_t n, int64_t ld);
+int lapsum_forward_lowp(const void* r, int dtype, int64_t ld, float* p, double* b, double* sum_f,
+                        int64_t B, int64_t n, double k, double t, int path, uint64_t seed,
+                        void* ws, size_t ws_bytes, void* support, size_t support_bytes,
+                        void* stream);
+int lapsum_backward_lowp(const void* r, int dtype, int64_t ld, const double* b, const float* v,
+                         float* g, int64_t B, int64_t n, double t, const void* support,
+                         size_t support_bytes, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Forward with a budget per row: as lapsum_forward, with k[row] (fp64, DEVICE
  * memory, B entries, read in stream order) in place of the shared k.  The
  * pages fix one budget per operator call; a budget per row is the next step
  * the same equation allows (every row is solved on its own).  Solvers:
  * LAPSUM_PATH_AUTO gives the on-chip sort for n <= 4096, the one-CTA-per-row
- * bracketing for n <= 2^18 (each row's sample size and binomial ranks are
- * computed on the device from its budget) and the radix full sort above;
- * LAPSUM_PATH_FULLSORT, LAPSUM_PATH_RADIX and LAPSUM_PATH_ROWBRACKET (n <=
- * 2^20) select one; LAPSUM_PATH_BRACKET returns LAPSUM_EINVAL.  The workspace
+ * bracketing for n <= 2^18 and the whole-GPU bracketing above (both compute
+ * each row's sample size and binomial ranks on the device from its budget);
+ * LAPSUM_PATH_FULLSORT, LAPSUM_PATH_RADIX, LAPSUM_PATH_ROWBRACKET (n <= 2^20)
+ * and LAPSUM_PATH_BRACKET select one.  The workspace
  * is lapsum_workspace_bytes_rowk(B, n, path) bytes (0 for an invalid size or
  * path).  `support` (may be NULL; see the gradient support below, same
  * rules when not NULL) receives the gradient support of rows with n > 4096.
@@ -318,6 +347,9 @@ int lapsum_profile_read(lapsum_kernel_time* out, int max_entries, int* n_entries
  * nothing.
  * The first call on each device looks up the array's device address (one
  * cudaGetSymbolAddress); make that first call before any stream capture.
+ * Calls made outside a capture look the address up again (a device reset
+ * reloads the library's device code and may move the array); calls made
+ * while a capture records the stream use the address of the last lookup.
  * Every call on a device shares the one array and clears the part that must
  * start at zero itself, so calls that overlap on the GPU (different streams
  * without ordering between them) race and give wrong results; order them.

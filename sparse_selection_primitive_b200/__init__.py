@@ -27,7 +27,7 @@ __all__ = [
     "LapSumError", "Workspace", "forward", "backward", "read_status", "row_info", "sample_values",
     "workspace_bytes", "soft_topk", "LapSumTopK", "PATHS", "FLAG_FORCE_MISS", "FLAG_NO_RETRY",
     "FLAG_ONE_CTA_SOLVE", "library_path", "profile_enable", "backward_kt", "profile_read", "backward_noalloc", "Support",
-    "support_bytes",
+    "support_bytes", "forward_lowp", "backward_lowp",
 ]
 
 PATHS = {"auto": 0, "fullsort": 1, "bracket": 2, "radix": 3, "rowbracket": 4}
@@ -133,6 +133,20 @@ def _lib():
                                             _vp, ctypes.c_size_t, _vp]
         lib.lapsum_sample_get.restype = ctypes.c_int
         lib.lapsum_sample_get.argtypes = [_vp, _c_i64, _vp, _c_i64, _vp]
+        lib.lapsum_workspace_bytes_lowp.restype = ctypes.c_size_t
+        lib.lapsum_workspace_bytes_lowp.argtypes = [_c_i64, _c_i64, _c_i64, ctypes.c_double,
+                                                    ctypes.c_int]
+        lib.lapsum_backward_workspace_bytes_lowp.restype = ctypes.c_size_t
+        lib.lapsum_backward_workspace_bytes_lowp.argtypes = [_c_i64, _c_i64, _c_i64]
+        lib.lapsum_forward_lowp.restype = ctypes.c_int
+        lib.lapsum_forward_lowp.argtypes = [_vp, ctypes.c_int, _c_i64, _vp, _vp, _vp, _c_i64,
+                                            _c_i64, ctypes.c_double, ctypes.c_double, ctypes.c_int,
+                                            ctypes.c_uint64, _vp, ctypes.c_size_t, _vp,
+                                            ctypes.c_size_t, _vp]
+        lib.lapsum_backward_lowp.restype = ctypes.c_int
+        lib.lapsum_backward_lowp.argtypes = [_vp, ctypes.c_int, _c_i64, _vp, _vp, _vp, _c_i64,
+                                             _c_i64, ctypes.c_double, _vp, ctypes.c_size_t, _vp,
+                                             ctypes.c_size_t, _vp]
         _LIB = lib
     return _LIB
 
@@ -258,7 +272,7 @@ def forward(r: torch.Tensor, k, t: float, path="auto", seed: int = 0, ws: Worksp
     """Returns (p, b[, sum_f]) for each row of r (float32 CUDA, rows x n or n).
 
     k is a number shared by every row, or a 1-D tensor with one budget per row
-    (lapsum_forward_rowk: the sort-based solvers).  With ``support`` (a Support
+    (lapsum_forward_rowk: every solver).  With ``support`` (a Support
     for the same B, n) the forward also lists the gradient support for
     backward(..., support=...)."""
     squeeze = r.dim() == 1
@@ -371,14 +385,15 @@ def hard_topk(r: torch.Tensor, k: float, path="auto", ws: Workspace = None):
     return (p[0] if squeeze else p), b
 
 
-_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 
 
 def _router_rows(x: torch.Tensor) -> torch.Tensor:
     if x.dim() == 1:
         x = x.unsqueeze(0)
     if x.dim() != 2 or x.dtype not in _DTYPES or not x.is_cuda:
-        raise TypeError("router scores must be a float32 or bfloat16 CUDA tensor, rows x n")
+        raise TypeError("router scores must be a float32, bfloat16 or float16 CUDA tensor, "
+                        "rows x n")
     if x.stride(1) != 1 or (x.shape[0] > 1 and x.stride(0) < x.shape[1]):
         x = x.contiguous()
     return x
@@ -438,6 +453,63 @@ def backward_router(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float,
     _check(_lib().lapsum_backward_router(r2.data_ptr(), _DTYPES[r2.dtype], n, b.data_ptr(),
                                          v2.data_ptr(), g.data_ptr(), B, n, float(t),
                                          _stream_ptr(r2.device)), "lapsum_backward_router")
+    return g[0] if r.dim() == 1 else g
+
+
+def _lowp_rows(x: torch.Tensor) -> torch.Tensor:
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if x.dim() != 2 or x.dtype not in _DTYPES or not x.is_cuda:
+        raise TypeError("scores must be a float32, bfloat16 or float16 CUDA tensor, rows x n")
+    if x.stride(1) != 1 or (x.shape[0] > 1 and x.stride(0) < x.shape[1]):
+        x = x.contiguous()
+    return x
+
+
+def forward_lowp(r: torch.Tensor, k: float, t: float, path="auto", seed: int = 0,
+                 want_sum_f: bool = False, support: Support = None, ws_bytes: int = None):
+    """Forward on scores of any of float32, bfloat16, float16 and any row length
+    (lapsum_forward_lowp: the on-chip kernels read 16-bit scores directly; longer
+    rows are widened exactly into the workspace first).  Returns (p, b[, sum_f])
+    with p float32 in r's row stride; ``support`` as in forward()."""
+    r2 = _lowp_rows(r)
+    B, n = r2.shape
+    ld = r2.stride(0) if B > 1 else n
+    code = _path_code(path)
+    nbytes = int(_lib().lapsum_workspace_bytes_lowp(B, n, ld, float(k), code))
+    if nbytes == 0:
+        raise LapSumError(1, "lapsum_workspace_bytes_lowp")
+    ws = Workspace(B, n, k, path, r2.device, nbytes=nbytes)
+    p = torch.empty((B, ld), dtype=torch.float32, device=r2.device)[:, :n]
+    b = torch.empty(B, dtype=torch.float64, device=r2.device)
+    sf = torch.empty(B, dtype=torch.float64, device=r2.device) if want_sum_f else None
+    sup_ptr, sup_n = (support.ptr, support.nbytes) if support is not None else (None, 0)
+    _check(_lib().lapsum_forward_lowp(
+        r2.data_ptr(), _DTYPES[r2.dtype], ld, p.data_ptr(), b.data_ptr(),
+        sf.data_ptr() if want_sum_f else None, B, n, float(k), float(t), code, int(seed),
+        ws.ptr, ws.nbytes, sup_ptr, sup_n, _stream_ptr(r2.device)), "lapsum_forward_lowp")
+    if r.dim() == 1:
+        p = p[0]
+    return (p, b, sf) if want_sum_f else (p, b)
+
+
+def backward_lowp(r: torch.Tensor, b: torch.Tensor, v: torch.Tensor, t: float,
+                  support: Support = None):
+    """g (float32) for scores r of float32, bfloat16 or float16 (lapsum_backward_lowp)."""
+    r2 = _lowp_rows(r)
+    B, n = r2.shape
+    ld = r2.stride(0) if B > 1 else n
+    v2 = v.reshape(B, n).to(torch.float32)
+    v2 = torch.empty((B, ld), dtype=torch.float32, device=r2.device)[:, :n].copy_(v2) \
+        if ld != n else v2.contiguous()
+    g = torch.empty((B, ld), dtype=torch.float32, device=r2.device)[:, :n]
+    nbytes = int(_lib().lapsum_backward_workspace_bytes_lowp(B, n, ld))
+    ws = Workspace(B, n, 0.5 * n, "auto", r2.device, nbytes=nbytes)
+    sup_ptr, sup_n = (support.ptr, support.nbytes) if support is not None else (None, 0)
+    _check(_lib().lapsum_backward_lowp(r2.data_ptr(), _DTYPES[r2.dtype], ld, b.data_ptr(),
+                                       v2.data_ptr(), g.data_ptr(), B, n, float(t), sup_ptr,
+                                       sup_n, ws.ptr, ws.nbytes, _stream_ptr(r2.device)),
+           "lapsum_backward_lowp")
     return g[0] if r.dim() == 1 else g
 
 
@@ -545,17 +617,18 @@ class LapSumTopK(torch.autograd.Function):
         B = 1 if rd.dim() == 1 else rd.shape[0]
         n = rd.shape[-1]
         per_row = isinstance(k, torch.Tensor) and k.dim() == 1
-        ctx.bf16 = rd.dtype == torch.bfloat16
-        if ctx.bf16:
-            # bf16 scores: the router form (rows of n <= 4096, one shared k); p is
-            # fp32, the gradient with respect to r comes back in bf16
-            if n > 4096 or per_row:
-                raise ValueError("bf16 scores need rows of n <= 4096 and one shared k")
+        ctx.lowp = rd.dtype in (torch.bfloat16, torch.float16)
+        if ctx.lowp:
+            # 16-bit scores (one shared k): lapsum_forward_lowp; p is fp32, the
+            # gradient with respect to r comes back in r's dtype
+            if per_row:
+                raise ValueError("16-bit scores take one shared k")
             tf = float(t)
-            p, b = forward_router(rd, float(k), tf)
+            sup = Support(B, n, rd.device) if support_bytes(B, n) > 0 else None
+            p, b = forward_lowp(rd, float(k), tf, path=path, seed=seed, support=sup)
             ctx.save_for_backward(r, b)
             ctx.t = tf
-            ctx.sup = None
+            ctx.sup = sup
             ctx.kt_grad = (isinstance(k, torch.Tensor) and k.requires_grad,
                            isinstance(t, torch.Tensor) and t.requires_grad)
             ctx.kt_like = (k, t)
@@ -576,8 +649,8 @@ class LapSumTopK(torch.autograd.Function):
     def backward(ctx, gp):
         r, b = ctx.saved_tensors
         v = gp.contiguous()
-        if ctx.bf16:
-            g = backward_router(r.detach(), b, v, ctx.t).to(torch.bfloat16)
+        if ctx.lowp:
+            g = backward_lowp(r.detach(), b, v, ctx.t, support=ctx.sup).to(r.dtype)
         else:
             g = backward(r.detach(), b, v, ctx.t, support=ctx.sup)
         ctx.sup = None
@@ -585,7 +658,7 @@ class LapSumTopK(torch.autograd.Function):
         if any(ctx.kt_grad):
             # a shared k or t gets the sum over rows of the per-row gradients;
             # a per-row k (one entry per row) gets them row by row
-            r32 = r.detach().float() if ctx.bf16 else r.detach()
+            r32 = r.detach().float() if ctx.lowp else r.detach()
             gks, gts = backward_kt(r32, b, v, ctx.t)
             k, t = ctx.kt_like
             if ctx.kt_grad[0]:

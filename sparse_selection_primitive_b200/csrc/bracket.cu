@@ -314,8 +314,23 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
                                                       uint32_t* __restrict__ ticket,
                                                       RowState* st, int top_h,
                                                       uint32_t* __restrict__ cand, int clear_bins,
-                                                      uint32_t* __restrict__ sup_flag) {
+                                                      uint32_t* __restrict__ sup_flag,
+                                                      const RowBudget* __restrict__ bud,
+                                                      WsHeader* hdr) {
     pdl_wait();
+    if (bud != nullptr) {
+        // the row's own budget: sample size, ranks and the candidate mode
+        // (every CTA of the grid of kSampleMax / kBlk takes part in the ticket)
+        m = bud->m;
+        for (int i = 0; i < kLadder; ++i) {
+            lad.l[i] = bud->l[i];
+            lad.h[i] = bud->h[i];
+        }
+        const int64_t need = lad.h[0] <= m ? lad.h[0] : (lad.l[0] >= 1 ? lad.l[0] : 0);
+        top_h = (need >= 1 && need <= kBlk && (int64_t)gridDim.x * need <= 4 * kBlk) ? (int)need
+                                                                                      : 0;
+    }
+    const bool bad_budget = bud != nullptr && !bud->ok;
     if (blockIdx.x == 0) {
         // this kernel starts the row's forward: clear its record, histogram
         // and gradient-support flags
@@ -333,8 +348,8 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
     __shared__ uint32_t bcast[4];
     __shared__ int flag;
     const int s = blockIdx.x * kBlk + threadIdx.x;
-    uint32_t key = 0u;  // samples past m (none when m is a multiple of kBlk) sort first
-    if (s < m) {
+    uint32_t key = 0u;  // samples past m sort first
+    if (s < m && !bad_budget) {
         const float y = draw_sample(r, n, t, seed, c0, s);
         sample_out[s] = y;
         key = to_key(y);
@@ -347,7 +362,7 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
     } else {
         for (int i = threadIdx.x; i < 2048; i += kBlk) hist[i] = 0u;
         __syncthreads();
-        const uint32_t bn = s < m ? key >> 21 : 0xffffffffu;
+        const uint32_t bn = (s < m && !bad_budget) ? key >> 21 : 0xffffffffu;
         // lanes with the same bin add once (samples crowd into few top bins)
         const unsigned peers = __match_any_sync(0xffffffffu, bn);
         if (bn != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1)
@@ -368,6 +383,18 @@ __global__ void __launch_bounds__(kBlk) sample_kernel(const float* __restrict__ 
     if (!flag) return;
     __threadfence();
     phase_mark(st, 0);
+    if (bad_budget) {
+        // a budget outside (0, n): b = NaN and a status bit; the later kernels
+        // of the row see the bit and return
+        for (int i = threadIdx.x; i < 2048; i += kBlk) ghist[i] = 0u;
+        if (threadIdx.x == 0) {
+            st->status |= kDevBadBudget;
+            set_status(hdr, kDevBadBudget);
+            st->path = LAPSUM_PATH_BRACKET;
+            st->b = nan("");
+        }
+        return;
+    }
     const int64_t ra = lad.l[0] >= 1 ? lad.l[0] : 0;
     const int64_t rb = lad.h[0] <= m ? lad.h[0] : 0;
     uint32_t ka = 0u, kb = 0u, kmax = 0u;
@@ -571,6 +598,7 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     extern __shared__ __align__(16) float fold_dyn[];
     __shared__ int scount;
     __shared__ unsigned long long gbase;
+    if (st->status & kDevBadBudget) return;
     const float aL = st->a_L, aR = st->a_R;
     // Scores more than 90 t below the bracket add exactly 0 to the left tail
     // sum in fp32, and scores more than 90 t above it add 1 to the right count
@@ -1640,10 +1668,23 @@ __global__ void __maxnreg__(64) solve_kernel(const float* __restrict__ r, int64_
                                              const float* __restrict__ sample, int m,
                                              Ladder lad, double* __restrict__ b_out,
                                              WsHeader* hdr, int split,
-                                             const double* __restrict__ fold_part, int nfold) {
+                                             const double* __restrict__ fold_part, int nfold,
+                                             const RowBudget* __restrict__ bud) {
     pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    if (bud != nullptr) {
+        if (!bud->ok) {
+            if (threadIdx.x == 0) *b_out = nan("");
+            return;
+        }
+        k = bud->k;
+        m = bud->m;
+        for (int i = 0; i < kLadder; ++i) {
+            lad.l[i] = bud->l[i];
+            lad.h[i] = bud->h[i];
+        }
+    }
     phase_mark(st, 2);
     if (threadIdx.x == 0) {
         sm->bcast[2] = 0xffffffffu;
@@ -1913,11 +1954,13 @@ __global__ void __maxnreg__(64) solve2_kernel(double k, double t, RowState* st,
                                                       float* __restrict__ band0,
                                                       float* __restrict__ sub,
                                                       const unsigned long long* __restrict__ bins,
-                                                      double* __restrict__ b_out, WsHeader* hdr) {
+                                                      double* __restrict__ b_out, WsHeader* hdr,
+                                                      const RowBudget* __restrict__ bud) {
     pdl_wait();
     extern __shared__ __align__(16) unsigned char dsm[];
     SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
     if (st->stage != 1) return;
+    if (bud != nullptr) k = bud->k;
     phase_mark(st, 4);
     const long long ns = (long long)st->n_sub;
     Tails s;
@@ -2145,7 +2188,7 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                                int64_t row, int m, int64_t rank_l[kLadder],
                                int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,
                                RowState* st_row, double* b_out, WsHeader* hdr,
-                               uint32_t* sup_flag, cudaStream_t st) {
+                               uint32_t* sup_flag, const RowBudget* bud, cudaStream_t st) {
     // dynamic shared memory limits, set once per device (they belong to the
     // device's copy of the module)
     static unsigned long long attr_devices = 0ull;
@@ -2174,7 +2217,10 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     const int max_attempts = (flags & LAPSUM_FLAG_NO_RETRY) ? 1 : kMaxAttempts;
     float* sample = buf.sample + row * (int64_t)kSampleMax;
     const uint64_t c0 = (uint64_t)row << 32;
-    const int sgrid = (m + kBlk - 1) / kBlk;
+    // With a per-row budget (bud) the sample size and ranks are on the device:
+    // the sample grid covers the largest sample, and the split solve kernels
+    // are always launched (they return at once when the band was small).
+    const int sgrid = bud != nullptr ? kSampleMax / kBlk : (m + kBlk - 1) / kBlk;
     // The band of the first bracket holds about n (h - l) / m scores.  When it
     // should fit the on-chip sort with some room to spare, the solve kernel
     // finishes by itself, the fold builds no band histogram, and the grid-wide
@@ -2184,7 +2230,8 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     const int64_t hi_rank = rank_h[0] < m ? rank_h[0] : m;
     const double expect_band = (double)n * (double)(hi_rank - lo_rank) / (double)m;
     const int split =
-        ((flags & LAPSUM_FLAG_ONE_CTA_SOLVE) == 0 && (force_miss || expect_band > 0.75 * kBandSortMax))
+        ((flags & LAPSUM_FLAG_ONE_CTA_SOLVE) == 0 &&
+         (bud != nullptr || force_miss || expect_band > 0.75 * kBandSortMax))
             ? 1
             : 0;
     // the fold builds the band histogram for the split solve, and for the
@@ -2192,13 +2239,17 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
     const int hist = (split || (flags & LAPSUM_FLAG_ONE_CTA_SOLVE) != 0) ? 1 : 0;
     // both bracket ranks among each sample CTA's top_h keys: candidate selection
     const int64_t need = rank_h[0] <= m ? rank_h[0] : (rank_l[0] >= 1 ? rank_l[0] : 0);
-    const int top_h = (need >= 1 && need <= kBlk && (int64_t)sgrid * need <= 4 * kBlk) ? (int)need : 0;
-    const size_t smem = top_h > 0 ? (size_t)4 * kBlk * sizeof(uint32_t) : sample_smem;
+    const int top_h = (bud == nullptr && need >= 1 && need <= kBlk &&
+                       (int64_t)sgrid * need <= 4 * kBlk)
+                          ? (int)need
+                          : 0;
+    const size_t smem = (bud == nullptr && top_h > 0) ? (size_t)4 * kBlk * sizeof(uint32_t)
+                                                      : sample_smem;
     {
         ProfScope ps_("bracket_sample", st);
         launch_pdl(sample_kernel, dim3(sgrid), dim3(kBlk), smem, st, r_row, n, t, seed, c0, m,
                    lad, force_miss, max_attempts, sample, buf.bins, buf.ticket + 2,
-                   buf.ticket + 1, st_row, top_h, buf.cand, hist, sup_flag);
+                   buf.ticket + 1, st_row, top_h, buf.cand, hist, sup_flag, bud, hdr);
     }
     const int vec = ((reinterpret_cast<uintptr_t>(r_row) & 15u) == 0) ? 1 : 0;
     {
@@ -2210,7 +2261,7 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
         ProfScope ps_("bracket_solve", st);
         launch_pdl(solve_kernel, dim3(1), dim3(kBlk), solve_smem, st, r_row, n, vec, k, t, st_row,
                    buf.band[0], buf.band[1], hist ? buf.bins : nullptr, sample, m, lad, b_out,
-                   hdr, split, (const double*)buf.fold_part, buf.fold_grid);
+                   hdr, split, (const double*)buf.fold_part, buf.fold_grid, bud);
     }
     if (split) {
         {
@@ -2220,8 +2271,8 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
         }
         {
             ProfScope ps_("bracket_solve2", st);
-            launch_pdl(solve2_kernel, dim3(1), dim3(kBlk), solve_smem, st, k, t, st_row, buf.band[0], buf.band[1],
-                                                       buf.bins, b_out, hdr);
+            launch_pdl(solve2_kernel, dim3(1), dim3(kBlk), solve_smem, st, k, t, st_row,
+                       buf.band[0], buf.band[1], buf.bins, b_out, hdr, bud);
         }
     }
     return cudaGetLastError();

@@ -28,19 +28,19 @@ constexpr double kBracketAlpha = 1e-6;  // miss probability allowed per bracket 
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Solver for per-row budgets: the sort-based solvers and the one-CTA-per-row
-// bracketing (its sample ranks are computed per row on the device); not the
-// whole-GPU bracketing.
+// Solver for per-row budgets: as for a shared budget; the bracketing solvers
+// compute each row's sample size and binomial ranks on the device.
 int resolve_path_rowk(int64_t n, int path) {
     switch (path & 0xff) {
         case LAPSUM_PATH_AUTO:
             return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT
                    : n <= kRowBracketAuto ? LAPSUM_PATH_ROWBRACKET
-                                          : LAPSUM_PATH_RADIX;
+                                          : LAPSUM_PATH_BRACKET;
         case LAPSUM_PATH_FULLSORT:
             return n <= kOnchipMax ? LAPSUM_PATH_FULLSORT : LAPSUM_PATH_RADIX;
         case LAPSUM_PATH_RADIX: return LAPSUM_PATH_RADIX;
         case LAPSUM_PATH_ROWBRACKET: return n <= kRowBracketMax ? LAPSUM_PATH_ROWBRACKET : -1;
+        case LAPSUM_PATH_BRACKET: return LAPSUM_PATH_BRACKET;
         default: return -1;
     }
 }
@@ -110,12 +110,17 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
         L.bins = take((size_t)3 * kBins * sizeof(unsigned long long));
         L.fold_part = take((size_t)kFoldGridMax * 4 * sizeof(double));
         L.cand = take((size_t)4096 * sizeof(uint32_t));
+        L.budgets = take((size_t)B * sizeof(RowBudget));  // per-row budgets' ladders
     }
     L.total = off;
     return L;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(int dtype) {
+    return dtype == LAPSUM_DTYPE_F32 || dtype == LAPSUM_DTYPE_BF16 || dtype == LAPSUM_DTYPE_F16;
+}
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA; }
 
@@ -406,13 +411,23 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
         bb.ticket = reinterpret_cast<uint32_t*>(w + L.fold_ticket);
         bb.fold_grid = bracket_fold_grid();
         if (bb.fold_grid > kFoldGridMax) bb.fold_grid = kFoldGridMax;
-        const int m = sample_size(n, k);
+        int m = kSampleMax;
         int64_t rl[kLadder], rh[kLadder];
-        bracket_ladder(m, k / (double)n, rl, rh);
+        RowBudget* budgets = nullptr;
+        if (k_rows != nullptr) {
+            // each row's sample size and ladder, on the device
+            budgets = reinterpret_cast<RowBudget*>(w + L.budgets);
+            for (int i = 0; i < kLadder; ++i) rl[i] = rh[i] = 0;
+            e = launch_row_budgets(k_rows, B, n, kBracketAlpha, budgets, st);
+        } else {
+            m = sample_size(n, k);
+            bracket_ladder(m, k / (double)n, rl, rh);
+        }
         for (int64_t row = 0; row < B && e == cudaSuccess; ++row) {
             e = launch_bracket_row(r + row * ld, n, k, t, seed, row, m, rl, rh, path, bb,
                                    rows + row, b + row, hdr,
-                                   want_sup ? sv_all.flags + row : nullptr, st);
+                                   want_sup ? sv_all.flags + row : nullptr,
+                                   budgets != nullptr ? budgets + row : nullptr, st);
         }
     }
     if (e != cudaSuccess) return LAPSUM_ECUDA;
@@ -484,7 +499,7 @@ int lapsum_forward_router(const void* r, int dtype, int64_t ld, float* p, double
                           float* sel_p, int32_t* sel_cnt, void* ws, size_t ws_bytes,
                           void* stream) {
     if (r == nullptr || p == nullptr || b == nullptr) return LAPSUM_EINVAL;
-    if (dtype != LAPSUM_DTYPE_F32 && dtype != LAPSUM_DTYPE_BF16) return LAPSUM_EINVAL;
+    if (!valid_dtype(dtype)) return LAPSUM_EINVAL;
     if (B < 1 || n < 1 || n > kOnchipMax || ld < n) return LAPSUM_EINVAL;
     if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
     if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
@@ -495,24 +510,98 @@ int lapsum_forward_router(const void* r, int dtype, int64_t ld, float* p, double
     const Layout L = make_layout(B, n, LAPSUM_PATH_FULLSORT);
     if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
     WsHeader* hdr = reinterpret_cast<WsHeader*>(static_cast<char*>(ws) + L.header);
-    const int bf16 = dtype == LAPSUM_DTYPE_BF16 ? 1 : 0;
-    const int vec = (aligned16(r) && aligned16(p) && (ld % (bf16 ? 8 : 4)) == 0) ? 1 : 0;
-    return cuda_status(launch_onchip_router(r, bf16, ld, p, b, B, (int)n, k, t, hdr, vec, sel_idx,
-                                            sel_p, sel_cnt, want_sel ? cap : 0, eps,
+    const int vec =
+        (aligned16(r) && aligned16(p) && (ld % (dtype == LAPSUM_DTYPE_F32 ? 4 : 8)) == 0) ? 1 : 0;
+    return cuda_status(launch_onchip_router(r, dtype, ld, p, b, nullptr, B, (int)n, k, t, hdr, vec,
+                                            sel_idx, sel_p, sel_cnt, want_sel ? cap : 0, eps,
                                             (cudaStream_t)stream));
 }
 
 int lapsum_backward_router(const void* r, int dtype, int64_t ld, const double* b, const float* v,
                            float* g, int64_t B, int64_t n, double t, void* stream) {
     if (r == nullptr || b == nullptr || v == nullptr || g == nullptr) return LAPSUM_EINVAL;
-    if (dtype != LAPSUM_DTYPE_F32 && dtype != LAPSUM_DTYPE_BF16) return LAPSUM_EINVAL;
+    if (!valid_dtype(dtype)) return LAPSUM_EINVAL;
     if (B < 1 || n < 1 || n > kOnchipMax || ld < n) return LAPSUM_EINVAL;
     if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
-    const int bf16 = dtype == LAPSUM_DTYPE_BF16 ? 1 : 0;
-    const int vec =
-        (aligned16(r) && aligned16(v) && aligned16(g) && (ld % (bf16 ? 8 : 4)) == 0) ? 1 : 0;
-    return cuda_status(launch_onchip_backward_router(r, bf16, ld, b, v, g, B, (int)n, t, vec,
+    const int vec = (aligned16(r) && aligned16(v) && aligned16(g) &&
+                     (ld % (dtype == LAPSUM_DTYPE_F32 ? 4 : 8)) == 0)
+                        ? 1
+                        : 0;
+    return cuda_status(launch_onchip_backward_router(r, dtype, ld, b, v, g, B, (int)n, t, vec,
                                                      (cudaStream_t)stream));
+}
+
+size_t lapsum_workspace_bytes_lowp(int64_t B, int64_t n, int64_t ld, double k, int path) {
+    if (B < 1 || n < 1 || ld < n) return 0;
+    const size_t base = lapsum_workspace_bytes(B, n, k, path);
+    if (base == 0) return 0;
+    return up(base) + up((size_t)B * (size_t)ld * sizeof(float));
+}
+
+size_t lapsum_backward_workspace_bytes_lowp(int64_t B, int64_t n, int64_t ld) {
+    if (B < 1 || n < 1 || ld < n) return 0;
+    return up(lapsum_backward_workspace_bytes(B, n)) + up((size_t)B * (size_t)ld * sizeof(float));
+}
+
+int lapsum_forward_lowp(const void* r, int dtype, int64_t ld, float* p, double* b, double* sum_f,
+                        int64_t B, int64_t n, double k, double t, int path, uint64_t seed,
+                        void* ws, size_t ws_bytes, void* support, size_t support_size,
+                        void* stream) {
+    if (r == nullptr || p == nullptr || b == nullptr || !valid_dtype(dtype)) return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
+    if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    if (dtype == LAPSUM_DTYPE_F32)
+        return forward_impl(static_cast<const float*>(r), ld, p, b, sum_f, B, n, k, nullptr, t,
+                            path, seed, ws, ws_bytes, support, support_size, stream);
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const int pc = path & 0xff;
+    if (n <= kOnchipMax && (pc == LAPSUM_PATH_AUTO || pc == LAPSUM_PATH_FULLSORT)) {
+        // the on-chip kernels read the 16-bit scores themselves
+        const Layout L = make_layout(B, n, LAPSUM_PATH_FULLSORT);
+        if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
+        WsHeader* hdr = reinterpret_cast<WsHeader*>(static_cast<char*>(ws) + L.header);
+        const int vec = (aligned16(r) && aligned16(p) && (ld % 8) == 0) ? 1 : 0;
+        return cuda_status(launch_onchip_router(r, dtype, ld, p, b, sum_f, B, (int)n, k, t, hdr,
+                                                vec, nullptr, nullptr, nullptr, 0, 0.f,
+                                                (cudaStream_t)stream));
+    }
+    const size_t base = lapsum_workspace_bytes(B, n, k, path);
+    if (base == 0) return LAPSUM_EINVAL;
+    if (ws_bytes < up(base) + up((size_t)B * (size_t)ld * sizeof(float))) return LAPSUM_EWORKSPACE;
+    float* wide = reinterpret_cast<float*>(static_cast<char*>(ws) + up(base));
+    if (launch_widen(r, dtype, ld, B, n, wide, (cudaStream_t)stream) != cudaSuccess)
+        return LAPSUM_ECUDA;
+    return forward_impl(wide, ld, p, b, sum_f, B, n, k, nullptr, t, path, seed, ws, up(base),
+                        support, support_size, stream);
+}
+
+int lapsum_backward_lowp(const void* r, int dtype, int64_t ld, const double* b, const float* v,
+                         float* g, int64_t B, int64_t n, double t, const void* support,
+                         size_t support_size, void* ws, size_t ws_bytes, void* stream) {
+    if (r == nullptr || b == nullptr || v == nullptr || g == nullptr || !valid_dtype(dtype))
+        return LAPSUM_EINVAL;
+    if (B < 1 || n < 1 || ld < n) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    if (dtype == LAPSUM_DTYPE_F32 || n <= kOnchipMax) {
+        if (n <= kOnchipMax)
+            return lapsum_backward_router(r, dtype, ld, b, v, g, B, n, t, stream);
+        const float* rf = static_cast<const float*>(r);
+        return support != nullptr
+                   ? lapsum_backward_support(rf, ld, b, v, g, B, n, t, support, support_size, ws,
+                                             ws_bytes, stream)
+                   : lapsum_backward(rf, ld, b, v, g, B, n, t, ws, ws_bytes, stream);
+    }
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
+    const size_t base = up(lapsum_backward_workspace_bytes(B, n));
+    if (ws_bytes < base + up((size_t)B * (size_t)ld * sizeof(float))) return LAPSUM_EWORKSPACE;
+    float* wide = reinterpret_cast<float*>(static_cast<char*>(ws) + base);
+    if (launch_widen(r, dtype, ld, B, n, wide, (cudaStream_t)stream) != cudaSuccess)
+        return LAPSUM_ECUDA;
+    return support != nullptr
+               ? lapsum_backward_support(wide, ld, b, v, g, B, n, t, support, support_size, ws,
+                                         base, stream)
+               : lapsum_backward(wide, ld, b, v, g, B, n, t, ws, base, stream);
 }
 
 int lapsum_forward_rowk(const float* r, int64_t ld, float* p, double* b, double* sum_f, int64_t B,

@@ -51,16 +51,21 @@ cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, 
 // Zero-temperature limit (hard top-k) of rows of n <= 4096: sort, boundary group, p.
 cudaError_t launch_onchip_hard(const float* r, int64_t ld, float* p, double* b, int64_t B, int n,
                                double k, WsHeader* hdr, int vec, cudaStream_t st);
-// The router form: scores as fp32 (bf16 = 0) or bf16 bit patterns (bf16 = 1),
-// and optionally (sel_cnt != null) the per-row list of positions and values of
-// p > eps (at most cap per row) with its count.
-cudaError_t launch_onchip_router(const void* r, int bf16, int64_t ld, float* p, double* b,
-                                 int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
-                                 int32_t* sel_idx, float* sel_val, int32_t* sel_cnt, int cap,
-                                 float eps, cudaStream_t st);
-cudaError_t launch_onchip_backward_router(const void* r, int bf16, int64_t ld, const double* b,
+// The router form: scores of any lapsum_dtype (16-bit types as bit patterns,
+// widened exactly), optional sum f per row, and optionally (sel_cnt != null)
+// the per-row list of positions and values of p > eps (at most cap per row)
+// with its count.
+cudaError_t launch_onchip_router(const void* r, int dtype, int64_t ld, float* p, double* b,
+                                 double* sumf, int64_t B, int n, double k, double t, WsHeader* hdr,
+                                 int vec, int32_t* sel_idx, float* sel_val, int32_t* sel_cnt,
+                                 int cap, float eps, cudaStream_t st);
+cudaError_t launch_onchip_backward_router(const void* r, int dtype, int64_t ld, const double* b,
                                           const float* v, float* g, int64_t B, int n, double t,
                                           int vec, cudaStream_t st);
+// Rows of 16-bit scores (bf16 or fp16 bit patterns) widened exactly to fp32:
+// dst[row * ld + i] for i < n (the same row stride as the source).
+cudaError_t launch_widen(const void* src, int dtype, int64_t ld, int64_t B, int64_t n, float* dst,
+                         cudaStream_t st);
 
 // --- radix full sort (segmented LSD, keys only) ------------------------------
 constexpr int kRadixTile = 4096;
@@ -194,6 +199,6 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                                int64_t row, int m, int64_t rank_l[kLadder],
                                int64_t rank_h[kLadder], int flags, const BracketBuffers& buf,
                                RowState* st_row, double* b_out, WsHeader* hdr,
-                               uint32_t* sup_flag, cudaStream_t st);
+                               uint32_t* sup_flag, const RowBudget* bud, cudaStream_t st);
 
 }  // namespace lapsum

@@ -35,15 +35,21 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 std::mutex g_mu;
 void* g_scratch_ptr[kNoAllocMaxDevices] = {nullptr};
 
-// Device address of the scratch array on the current device (looked up once
-// per device; host code cannot use the symbol itself as a device pointer).
-cudaError_t scratch_address(void** out) {
+// Device address of the scratch array on the current device.  Host code
+// cannot use the symbol itself as a device pointer.  The address is looked up
+// on every call made outside a stream capture (so that a device reset, which
+// reloads the module and may move the array, leaves no stale address behind)
+// and kept per device for calls made while a capture records the stream.
+cudaError_t scratch_address(cudaStream_t st, void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(st, &cap);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> g(g_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone || g_scratch_ptr[dev] == nullptr) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
@@ -76,7 +82,7 @@ extern "C" int lapsum_backward_noalloc(const float* r, int64_t ld, const double*
     // (the same per-device SM count sizes the launch's grid)
     if ((int64_t)device_sm_count() * 8 + B > kNoAllocRecords) return LAPSUM_EINVAL;
     void* base = nullptr;
-    if (scratch_address(&base) != cudaSuccess) return LAPSUM_ECUDA;
+    if (scratch_address(st, &base) != cudaSuccess) return LAPSUM_ECUDA;
     char* s = static_cast<char*>(base);
     double* partials = reinterpret_cast<double*>(s);
     double* row_R = reinterpret_cast<double*>(s + kPartialBytes);

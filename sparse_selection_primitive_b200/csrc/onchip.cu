@@ -13,6 +13,8 @@
 // exchange through shuffles, and only partners in another warp go through
 // shared memory.  The scan carries fp64 affine maps (gap factor, 1) whose
 // composition is a warp shuffle scan plus one shared-memory step across warps.
+#include <cuda_fp16.h>
+
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
 #include "bitonic.cuh"
@@ -87,6 +89,40 @@ __device__ __forceinline__ void load_row(const uint16_t* __restrict__ row, int n
     for (int e = 0; e < E; ++e) {
         valid[e] = row_ok && (base + e < n);
         x[e] = valid[e] ? bf16_to_f32(__ldg(row + base + e)) : 0.f;
+    }
+}
+
+// The same for fp16 scores (IEEE half bit patterns, widened exactly to fp32).
+struct F16Bits {
+    uint16_t bits;
+};
+__device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+template <int E>
+__device__ __forceinline__ void load_row(const F16Bits* __restrict__ row_in, int n, int tid,
+                                         bool vec, bool row_ok, float (&x)[E], bool (&valid)[E]) {
+    const uint16_t* row = reinterpret_cast<const uint16_t*>(row_in);
+    const int base = tid * E;
+    if constexpr (E % 8 == 0) {
+        if (vec && row_ok && base + E <= n) {
+#pragma unroll
+            for (int q = 0; q < E / 8; ++q) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + base) + q);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    x[8 * q + 2 * h] = f16_to_f32((uint16_t)(w[h] & 0xffffu));
+                    x[8 * q + 2 * h + 1] = f16_to_f32((uint16_t)(w[h] >> 16));
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) valid[e] = true;
+            return;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        valid[e] = row_ok && (base + e < n);
+        x[e] = valid[e] ? f16_to_f32(__ldg(row + base + e)) : 0.f;
     }
 }
 
@@ -653,24 +689,30 @@ cudaError_t launch_onchip_hard(const float* r, int64_t ld, float* p, double* b, 
     }
 }
 
-cudaError_t launch_onchip_router(const void* r, int bf16, int64_t ld, float* p, double* b,
-                                 int64_t B, int n, double k, double t, WsHeader* hdr, int vec,
-                                 int32_t* sel_idx, float* sel_val, int32_t* sel_cnt, int cap,
-                                 float eps, cudaStream_t st) {
+cudaError_t launch_onchip_router(const void* r, int dtype, int64_t ld, float* p, double* b,
+                                 double* sumf, int64_t B, int n, double k, double t, WsHeader* hdr,
+                                 int vec, int32_t* sel_idx, float* sel_val, int32_t* sel_cnt,
+                                 int cap, float eps, cudaStream_t st) {
     const SelectOut sel{sel_idx, sel_val, sel_cnt, cap, eps};
-    if (bf16)
-        return onchip_forward_any<uint16_t>(static_cast<const uint16_t*>(r), ld, p, b, nullptr, B,
+    if (dtype == LAPSUM_DTYPE_BF16)
+        return onchip_forward_any<uint16_t>(static_cast<const uint16_t*>(r), ld, p, b, sumf, B,
                                             n, k, nullptr, t, hdr, vec, sel, st);
-    return onchip_forward_any<float>(static_cast<const float*>(r), ld, p, b, nullptr, B, n, k,
+    if (dtype == LAPSUM_DTYPE_F16)
+        return onchip_forward_any<F16Bits>(static_cast<const F16Bits*>(r), ld, p, b, sumf, B, n,
+                                           k, nullptr, t, hdr, vec, sel, st);
+    return onchip_forward_any<float>(static_cast<const float*>(r), ld, p, b, sumf, B, n, k,
                                      nullptr, t, hdr, vec, sel, st);
 }
 
-cudaError_t launch_onchip_backward_router(const void* r, int bf16, int64_t ld, const double* b,
+cudaError_t launch_onchip_backward_router(const void* r, int dtype, int64_t ld, const double* b,
                                           const float* v, float* g, int64_t B, int n, double t,
                                           int vec, cudaStream_t st) {
-    if (bf16)
+    if (dtype == LAPSUM_DTYPE_BF16)
         return onchip_backward_any<uint16_t>(static_cast<const uint16_t*>(r), ld, b, v, g, B, n, t,
                                              vec, st);
+    if (dtype == LAPSUM_DTYPE_F16)
+        return onchip_backward_any<F16Bits>(static_cast<const F16Bits*>(r), ld, b, v, g, B, n, t,
+                                            vec, st);
     return onchip_backward_any<float>(static_cast<const float*>(r), ld, b, v, g, B, n, t, vec, st);
 }
 

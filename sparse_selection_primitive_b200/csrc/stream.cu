@@ -10,6 +10,8 @@
 // bytes).  Per-row reductions go through per-tile partials in the workspace;
 // the last CTA of a row (atomic ticket) combines them in tile order, so the
 // row results are deterministic.  No CTA ever waits for another.
+#include <cuda_fp16.h>
+
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
 #include "stream_common.cuh"
@@ -370,9 +372,67 @@ __global__ void __launch_bounds__(kThreads) bwd_kt_kernel(
     }
 }
 
+// Exact widening of 16-bit scores to fp32: 8 scores per thread per trip
+// (16-byte loads, two 16-byte stores) where the row allows, else one by one.
+template <int DT>
+__device__ __forceinline__ float widen1(uint16_t h) {
+    if constexpr (DT == LAPSUM_DTYPE_BF16) return __uint_as_float((uint32_t)h << 16);
+    else return __half2float(__ushort_as_half(h));
+}
+template <int DT>
+__global__ void __launch_bounds__(kThreads) widen_kernel(const uint16_t* __restrict__ src,
+                                                         int64_t ld, int64_t n, int vec,
+                                                         float* __restrict__ dst) {
+    const int64_t row = blockIdx.y;
+    const uint16_t* s = src + row * ld;
+    float* d = dst + row * ld;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    const int64_t gt = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (vec) {
+        const int64_t n8 = n >> 3;
+        for (int64_t i = gt; i < n8; i += stride) {
+            const uint4 u = __ldcs(reinterpret_cast<const uint4*>(s) + i);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            float y[8];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                y[2 * h] = widen1<DT>((uint16_t)(w[h] & 0xffffu));
+                y[2 * h + 1] = widen1<DT>((uint16_t)(w[h] >> 16));
+            }
+            float4* d4 = reinterpret_cast<float4*>(d) + 2 * i;
+            __stcs(d4, make_float4(y[0], y[1], y[2], y[3]));
+            __stcs(d4 + 1, make_float4(y[4], y[5], y[6], y[7]));
+        }
+        for (int64_t j = (n8 << 3) + gt; j < n; j += stride) d[j] = widen1<DT>(s[j]);
+    } else {
+        for (int64_t j = gt; j < n; j += stride) d[j] = widen1<DT>(s[j]);
+    }
+}
+
 }  // namespace
 
 int64_t stream_tiles(int64_t n) { return (n + kStreamTile - 1) / kStreamTile; }
+
+cudaError_t launch_widen(const void* src, int dtype, int64_t ld, int64_t B, int64_t n, float* dst,
+                         cudaStream_t st) {
+    // 16-byte accesses when both rows start on 16-byte boundaries throughout
+    const int vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(dst) & 15u) == 0 && (ld % 8) == 0)
+                        ? 1
+                        : 0;
+    int64_t per_row = ((int64_t)device_sm_count() * 8 + B - 1) / B;
+    const int64_t need = (n / 8 + kThreads - 1) / kThreads;
+    if (per_row > need) per_row = need;
+    if (per_row < 1) per_row = 1;
+    const dim3 grid((unsigned)per_row, (unsigned)B);
+    ProfScope ps_("widen", st);
+    const uint16_t* s = static_cast<const uint16_t*>(src);
+    if (dtype == LAPSUM_DTYPE_BF16)
+        widen_kernel<LAPSUM_DTYPE_BF16><<<grid, kThreads, 0, st>>>(s, ld, n, vec, dst);
+    else
+        widen_kernel<LAPSUM_DTYPE_F16><<<grid, kThreads, 0, st>>>(s, ld, n, vec, dst);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_emit(const float* r, int64_t ld, float* p, double* b, double* sumf,
                         int64_t B, int64_t n, double t, double* partials, uint32_t* tickets,

@@ -101,14 +101,14 @@ def test_new_entry_points_reject_bad_arguments_on_host(lib):
                      ctypes.c_double, ctypes.c_int, vp, ctypes.c_size_t, vp, ctypes.c_size_t, vp]
     assert rowk(d, 8, d, d, None, 1, 8, None, 0.1, 0, ws, 1 << 20, None, 0, None) == 1  # k NULL
     assert rowk(d, 8, d, d, None, 1, 8, d, 0.0, 0, ws, 1 << 20, None, 0, None) == 1     # t <= 0
-    assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 2, ws, 1 << 20, None, 0, None) == 1     # bracket
+    assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 9, ws, 1 << 20, None, 0, None) == 1     # bad path
     assert rowk(d, 8, d, d, None, 1, 8, d, 0.1, 0, None, 1 << 20, None, 0, None) == 2   # no ws
     router = lib.lapsum_forward_router
     router.argtypes = [vp, ctypes.c_int, ctypes.c_int64, vp, vp, ctypes.c_int64, ctypes.c_int64,
                        ctypes.c_double, ctypes.c_double, ctypes.c_float, ctypes.c_int32, vp, vp,
                        vp, vp, ctypes.c_size_t, vp]
     ok = (d, 0, 8, d, d, 1, 8, 2.0, 0.1, 0.0, 0, None, None, None, ws, 1 << 20, None)
-    assert router(*ok[:1], 2, *ok[2:]) == 1                                   # unknown dtype
+    assert router(*ok[:1], 3, *ok[2:]) == 1                                   # unknown dtype
     assert router(*ok[:6], 5000, *ok[7:]) == 1                                # n > 4096
     assert router(*ok[:11], d, None, None, *ok[14:]) == 1                     # partial list args
     assert router(*ok[:9], 1e-3, 0, d, d, d, *ok[14:]) == 1                   # cap < 1
@@ -126,16 +126,62 @@ def test_new_entry_points_reject_bad_arguments_on_host(lib):
 
 def test_per_row_budget_workspace_sizes(lib):
     """lapsum_workspace_bytes_rowk follows the per-row solver choice: the on-chip
-    sort, the one-CTA bracketing (band buffers), the radix sort (key buffers); the
-    whole-GPU bracketing has no per-row form."""
+    sort, the one-CTA bracketing (band buffers), the radix sort (key buffers) and
+    the whole-GPU bracketing (per-row ladders next to its buffers)."""
     f = lib.lapsum_workspace_bytes_rowk
     f.restype = ctypes.c_size_t
     f.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
     assert f(0, 100, 0) == 0 and f(4, 0, 0) == 0
-    assert f(4, 100, 2) == 0                      # whole-GPU bracketing
+    assert f(4, 5_000_000, 2) >= f(1, 5_000_000, 2) > 0   # whole-GPU bracketing
+    assert f(4, 100, 9) == 0                      # unknown path
     assert f(4, 2_000_000, 4) == 0                # one-CTA bracketing is for n <= 2^20
     small = f(16, 256, 0)
     assert small > 0 and small % 256 == 0
     assert f(256, 65536, 0) >= 2 * 256 * 65536 * 4        # band buffers
-    assert f(2, 1 << 19, 0) >= 2 * 2 * (1 << 19) * 4       # radix key buffers
+    assert f(2, 1 << 19, 3) >= 2 * 2 * (1 << 19) * 4       # radix key buffers
+    assert f(2, 1 << 19, 0) >= 2 * (1 << 19) * 4           # AUTO: whole-GPU bracketing bands
     assert f(256, 65536, 3) >= 2 * 256 * 65536 * 4         # radix forced
+
+
+def test_low_precision_entry_points_on_host(lib):
+    """lapsum_forward_lowp / lapsum_backward_lowp: argument checks before any
+    launch, and workspace sizes that add the widened rows (B x ld fp32) to the
+    fp32 solver's workspace."""
+    vp = ctypes.c_void_p
+    d = ctypes.c_void_p(4096)
+    ws = ctypes.c_void_p(256)
+    fw = lib.lapsum_forward_lowp
+    fw.restype = ctypes.c_int
+    fw.argtypes = [vp, ctypes.c_int, ctypes.c_int64, vp, vp, vp, ctypes.c_int64, ctypes.c_int64,
+                   ctypes.c_double, ctypes.c_double, ctypes.c_int, ctypes.c_uint64, vp,
+                   ctypes.c_size_t, vp, ctypes.c_size_t, vp]
+    ok = [d, 1, 5000, d, d, None, 1, 5000, 10.0, 0.1, 0, 0, ws, 1 << 30, None, 0, None]
+    bad = list(ok); bad[1] = 3
+    assert fw(*bad) == 1                          # unknown dtype
+    bad = list(ok); bad[8] = 5000.0
+    assert fw(*bad) == 1                          # k = n
+    bad = list(ok); bad[2] = 4000
+    assert fw(*bad) == 1                          # ld < n
+    bad = list(ok); bad[12] = None
+    assert fw(*bad) == 2                          # no workspace
+    bad = list(ok); bad[13] = 1024
+    assert fw(*bad) == 2                          # workspace too small
+    bw = lib.lapsum_backward_lowp
+    bw.restype = ctypes.c_int
+    bw.argtypes = [vp, ctypes.c_int, ctypes.c_int64, vp, vp, vp, ctypes.c_int64, ctypes.c_int64,
+                   ctypes.c_double, vp, ctypes.c_size_t, vp, ctypes.c_size_t, vp]
+    assert bw(d, 7, 5000, d, d, d, 1, 5000, 0.1, None, 0, ws, 1 << 30, None) == 1
+    assert bw(d, 2, 5000, d, d, d, 1, 5000, -0.1, None, 0, ws, 1 << 30, None) == 1
+    assert bw(d, 2, 5000, d, d, d, 1, 5000, 0.1, None, 0, ws, 64, None) == 2
+    sz = lib.lapsum_workspace_bytes_lowp
+    sz.restype = ctypes.c_size_t
+    sz.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int]
+    base = lib.lapsum_workspace_bytes
+    base.restype = ctypes.c_size_t
+    base.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_double, ctypes.c_int]
+    assert sz(2, 70001, 70008, 300.0, 3) >= base(2, 70001, 300.0, 3) + 2 * 70008 * 4
+    assert sz(2, 70001, 70000, 300.0, 3) == 0     # ld < n
+    bsz = lib.lapsum_backward_workspace_bytes_lowp
+    bsz.restype = ctypes.c_size_t
+    bsz.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+    assert bsz(3, 9000, 9005) >= 3 * 9005 * 4 and bsz(0, 9000, 9000) == 0

@@ -11,8 +11,9 @@ oracle solved at its own budget, at the tolerances of the other parity tests:
 * a row whose budget lies outside (0, n) gets b = NaN and p = NaN, the status
   word reads LAPSUM_EINVAL, and the other rows are unaffected;
 * equal budgets give the bits of the shared-budget call on the same solver;
-* the whole-GPU bracketing refuses a per-row budget on the host; the one-CTA
-  bracketing takes its ranks per row on the device, equal to the oracle's;
+* both bracketing arrangements (one CTA per row, and the whole GPU on each row)
+  take their sample size and ranks per row on the device, equal to the
+  oracle's; an out-of-range budget gives that row NaN there too;
 * autograd: the gradient of a per-row k tensor is the oracle's dL/dk per row;
 * the support hand-over of long rows with per-row budgets.
 """
@@ -98,11 +99,52 @@ def test_rowk_equal_budgets_match_the_shared_budget(cuda_device, n, path):
     assert torch.equal(b1, b2) and torch.equal(p1, p2)
 
 
-def test_rowk_refused_on_the_whole_gpu_bracketing(cuda_device):
-    r, _ = random_rows(314, 2, 20000)
+@pytest.mark.parametrize("B,n,dist", [(2, 400000, "mix_nu"), (3, 300001, "abs_t3")])
+def test_rowk_whole_gpu_bracketing(cuda_device, B, n, dist):
+    """The whole-GPU bracketing with one budget per row: each row's sample size
+    and ranks come from its own budget on the device (equal to the oracle's);
+    b, p and g must match the oracle solved at that budget."""
+    r, v = random_rows(319 + n, B, n, dist)
+    rng = np.random.default_rng(n + 7)
+    k = rng.uniform(2.0, n / 50.0, B)
+    k[0] = 40.0
+    kt = torch.tensor(k, dtype=torch.float64, device="cuda")
     rt = torch.from_numpy(r).cuda()
-    with pytest.raises(L.LapSumError):
-        L.forward(rt, torch.tensor([5.0, 9.0], device="cuda"), 0.05, path="bracket")
+    ws = L.Workspace(B, n, 1.0, "auto", nbytes=L._lib().lapsum_workspace_bytes_rowk(B, n, 2))
+    sup = L.Support(B, n)
+    p, b = L.forward(rt, kt, 0.02, path="bracket", ws=ws, support=sup)
+    g = L.backward(rt, b, torch.from_numpy(v).cuda(), 0.02, support=sup)
+    torch.cuda.synchronize()
+    assert L.read_status(ws) == 0
+    p, bb, g = p.cpu().numpy().astype(np.float64), b.cpu().numpy(), g.cpu().numpy()
+    for i in range(B):
+        info = L.row_info(ws, i)
+        assert info["path"] == 2, info
+        m = info["sample_m"]
+        q = float(k[i]) / n
+        want_m = 4096
+        while want_m < 32768 and want_m < 64.0 / q:
+            want_m *= 2
+        assert m == want_m
+        l, h = oracle.binom_ranks(m, q, 1e-6)
+        assert (info["rank_l"], info["rank_h"]) == (l, h), (i, info, l, h)
+        check_row(r[i], v[i], float(k[i]), 0.02, bb[i], p[i], g[i].astype(np.float64),
+                  label=f"row {i}")
+
+
+def test_rowk_bad_budget_on_the_whole_gpu_bracketing(cuda_device):
+    B, n = 3, 300000
+    r, _ = random_rows(321, B, n, "mix_nu")
+    k = np.array([150.0, float(n), 400.0])  # the middle budget is out of range
+    rt = torch.from_numpy(r).cuda()
+    ws = L.Workspace(B, n, 1.0, "auto", nbytes=L._lib().lapsum_workspace_bytes_rowk(B, n, 2))
+    p, b = L.forward(rt, torch.tensor(k, device="cuda"), 0.05, path="bracket", ws=ws)
+    torch.cuda.synchronize()
+    bb, pp = b.cpu().numpy(), p.cpu().numpy()
+    assert math.isnan(bb[1]) and np.isnan(pp[1]).all()
+    for i in (0, 2):
+        check_row(r[i], None, float(k[i]), 0.05, bb[i], pp[i].astype(np.float64))
+    assert L.read_status(ws) == 1
 
 
 @pytest.mark.parametrize("B,n,dist,path", [(5, 20000, "normal", "auto"),
@@ -117,7 +159,8 @@ def test_rowk_one_cta_per_row_bracketing(cuda_device, B, n, dist, path):
     k[0] = 3.0
     kt = torch.tensor(k, dtype=torch.float64, device="cuda")
     rt = torch.from_numpy(r).cuda()
-    ws = L.Workspace(B, n, 1.0, "auto", nbytes=L._lib().lapsum_workspace_bytes_rowk(B, n, 0))
+    ws = L.Workspace(B, n, 1.0, "auto",
+                     nbytes=L._lib().lapsum_workspace_bytes_rowk(B, n, L.PATHS[path]))
     p, b = L.forward(rt, kt, 0.02, path=path, ws=ws)
     g = L.backward(rt, b, torch.from_numpy(v).cuda(), 0.02)
     torch.cuda.synchronize()

@@ -4,7 +4,8 @@ lapsum_backward_noalloc serves callers that cannot allocate device memory
 when they need the gradient (capture under a no-allocation rule, hosts that
 reserve all device memory up front, plugin hosts that own every allocation).
 It must give the same g as lapsum_backward, within the tests' VJP tolerance,
-on two calls in a row (its scratch array keeps the previous call's contents).
+on two calls in a row (its scratch array keeps the previous call's contents),
+and match the oracle's VJP on a row.
 This file is collected last on purpose.
 """
 import ctypes
@@ -13,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import sparse_selection_primitive_b200 as L
 from workloads import random_rows
 
@@ -51,6 +53,11 @@ def test_noalloc_backward_matches_regular(cuda_device, B, n, k, t, path):
     # the Python wrapper reaches the same entry point
     g2 = L.backward_noalloc(r, b, v, t)
     assert float((g2 - g_ref).abs().max()) <= TOL_G * scale
+    # and one row of it against the oracle (its own threshold and VJP)
+    i = B - 1
+    g_or, _, _ = oracle.vjp(r_h[i], v_h[i], oracle.solve_b(r_h[i], k, t), t)
+    dg = float(np.max(np.abs(g2[i].cpu().numpy().astype(np.float64) - g_or)))
+    assert dg <= TOL_G * float(np.max(np.abs(g_or))), dg
 
 
 def test_noalloc_backward_rejects_too_many_rows(cuda_device):
