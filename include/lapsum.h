@@ -140,12 +140,21 @@ int lapsum_backward(const float* r, int64_t ld, const double* b, const float* v,
  *               mask of the scores above b.
  * So sum p = k, as at every t > 0 (ties at the boundary share the remaining
  * budget instead of a fixed 1/2).  k is real in (0, n); n >= 2.  Solvers: the
- * on-chip sort for n <= 4096 and the radix full sort above (LAPSUM_PATH_AUTO
- * or LAPSUM_PATH_FULLSORT), or LAPSUM_PATH_RADIX; the bracketing paths return
- * LAPSUM_EINVAL.  ws: lapsum_workspace_bytes(B, n, k, LAPSUM_PATH_FULLSORT)
- * (or LAPSUM_PATH_RADIX when that path is asked for).  Rows with a non-finite
- * score get b = NaN and p = NaN (status LAPSUM_ENONFINITE).  The limit has no
- * useful gradient (p is piecewise constant in r); there is no backward.
+ * on-chip sort for n <= 4096 (LAPSUM_PATH_AUTO or LAPSUM_PATH_FULLSORT); for
+ * longer rows LAPSUM_PATH_AUTO and LAPSUM_PATH_BRACKET use bracketing without
+ * a full sort (section 2.2's steps with plain samples: their binomial order
+ * statistics bracket the ceil(k)-th largest score, one pass counts the scores
+ * above the bracket, keeps the band inside it and the largest score below it,
+ * and the boundary group is read off the sorted band; an exact selection over
+ * the row takes over when the bracket misses; LAPSUM_FLAG_FORCE_MISS forces
+ * that case for tests), falling back to the radix sort when the bracket ranks
+ * are too large for the sample's candidate lists (budgets near n/2);
+ * LAPSUM_PATH_FULLSORT and LAPSUM_PATH_RADIX take the radix full sort;
+ * LAPSUM_PATH_ROWBRACKET returns LAPSUM_EINVAL.  ws: lapsum_workspace_bytes(B,
+ * n, k, LAPSUM_PATH_FULLSORT) for AUTO and FULLSORT, or with LAPSUM_PATH_RADIX
+ * for the other paths.  Rows with a non-finite score get b = NaN and p = NaN
+ * (status LAPSUM_ENONFINITE).  The limit has no useful gradient (p is
+ * piecewise constant in r); there is no backward.
  */
 int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t B, int64_t n,
                         double k, int path, void* ws, size_t ws_bytes, void* stream);

@@ -374,7 +374,8 @@ def hard_topk(r: torch.Tensor, k: float, path="auto", ws: Workspace = None):
     B, n = r2.shape
     ld = _ld(r2)
     code = _path_code(path)
-    wpath = "fullsort" if (code & 0xFF) == PATHS["auto"] else code
+    # the full-sort workspace for AUTO and FULLSORT, the radix one otherwise
+    wpath = "fullsort" if (code & 0xFF) in (PATHS["auto"], PATHS["fullsort"]) else "radix"
     if ws is None or not ws.fits(B, n, k, wpath):
         ws = Workspace(B, n, k, wpath, r2.device)
     p = _like_rows(r2, ld)

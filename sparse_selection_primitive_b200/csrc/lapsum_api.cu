@@ -457,9 +457,15 @@ int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t
     if (r == nullptr || p == nullptr || b == nullptr) return LAPSUM_EINVAL;
     if (B < 1 || n < 2 || ld < n || n > INT32_MAX) return LAPSUM_EINVAL;
     if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
-    int rp = resolve_path(n, (path & 0xff) == LAPSUM_PATH_AUTO ? LAPSUM_PATH_FULLSORT : path);
-    if ((path & ~0xff) != 0 || (rp != LAPSUM_PATH_FULLSORT && rp != LAPSUM_PATH_RADIX))
+    const int pc = path & 0xff;
+    if ((path & ~0x1ff) != 0 || pc == LAPSUM_PATH_ROWBRACKET || pc > LAPSUM_PATH_ROWBRACKET)
         return LAPSUM_EINVAL;
+    // long rows: bracketing for AUTO and BRACKET (when both bracket ranks fit
+    // the sample CTAs' candidate lists), the radix full sort otherwise; the
+    // workspace is the full-sort one either way
+    int rp = n <= kOnchipMax && (pc == LAPSUM_PATH_AUTO || pc == LAPSUM_PATH_FULLSORT)
+                 ? LAPSUM_PATH_FULLSORT
+                 : LAPSUM_PATH_RADIX;
     if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return LAPSUM_EWORKSPACE;
     const Layout L = make_layout(B, n, rp);
     if (ws_bytes < L.total) return LAPSUM_EWORKSPACE;
@@ -470,6 +476,28 @@ int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t
     const int vec = (aligned16(r) && aligned16(p) && (ld % 4) == 0) ? 1 : 0;
     if (rp == LAPSUM_PATH_FULLSORT)
         return cuda_status(launch_onchip_hard(r, ld, p, b, B, (int)n, k, hdr, vec, st));
+    if (n > kOnchipMax && (pc == LAPSUM_PATH_AUTO || pc == LAPSUM_PATH_BRACKET)) {
+        const int m = sample_size(n, k);
+        int64_t rl[kLadder], rh[kLadder];
+        bracket_ladder(m, k / (double)n, rl, rh);
+        const int64_t need = rh[0] <= m ? rh[0] : (rl[0] >= 1 ? rl[0] : 0);
+        const int sgrid = m / 1024;
+        if (need >= 1 && need <= 1024 && (int64_t)sgrid * need <= 4096) {
+            const int64_t lo = rl[0] >= 1 ? rl[0] : 0;
+            const int64_t hi = rh[0] <= m ? rh[0] : 0;
+            cudaError_t e = cudaSuccess;
+            for (int64_t r0 = 0; r0 < B && e == cudaSuccess; r0 += kGridYMax) {
+                const int64_t nb = (B - r0 < kGridYMax) ? B - r0 : kGridYMax;
+                e = launch_hard_bracket(
+                    r + r0 * ld, ld, p + r0 * ld, b + r0, nb, n, k, 0, m, lo, hi, (int)need,
+                    (path & LAPSUM_FLAG_FORCE_MISS) ? 1 : 0, rows + r0,
+                    reinterpret_cast<float*>(w + L.keys0) + r0 * n,
+                    reinterpret_cast<uint32_t*>(w + L.keys1) + r0 * 4096,
+                    reinterpret_cast<uint32_t*>(w + L.tickets) + r0, hdr, B, vec, st);
+            }
+            return cuda_status(e);
+        }
+    }
     cudaError_t e = cudaMemsetAsync(rows, 0, (size_t)B * sizeof(RowState), st);
     if (e != cudaSuccess) return LAPSUM_ECUDA;
     RadixBuffers rb;

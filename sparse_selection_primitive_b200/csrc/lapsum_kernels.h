@@ -83,6 +83,21 @@ cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_
 cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
                                         const double* k_rows, double t, double* b, RowState* rows,
                                         WsHeader* hdr, cudaStream_t st);
+// p of the zero-temperature limit from each row's record (boundary score c
+// and its share): one CTA per 4096-score tile.
+cudaError_t launch_hard_emit(const float* r, int64_t ld, float* p, int64_t B, int64_t n,
+                             const RowState* rows, int vec, cudaStream_t st);
+// The zero-temperature limit through bracketing (rows of n > 4096, in
+// parallel): plain samples, their binomial order statistics as the bracket,
+// one pass for the count above it, the band and the largest score below it,
+// and one CTA per row for the boundary group (an exact selection over the row
+// when the bracket misses); then p.  band: B * n floats; cand: B * 4096 keys;
+// tickets: B self-resetting counters; top_h as in the soft sample kernel.
+cudaError_t launch_hard_bracket(const float* r, int64_t ld, float* p, double* b, int64_t B,
+                                int64_t n, double k, uint64_t seed, int m, int64_t rank_l,
+                                int64_t rank_h, int top_h, int force_miss, RowState* rows,
+                                float* band, uint32_t* cand, uint32_t* tickets, WsHeader* hdr,
+                                int64_t B_total, int vec, cudaStream_t st);
 // Zero-temperature limit of every row from its sorted keys (one CTA per row),
 // then p from r (one CTA per tile); b, the boundary score and its share go to
 // the row records.

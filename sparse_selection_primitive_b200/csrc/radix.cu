@@ -397,12 +397,15 @@ cudaError_t launch_rowhard_sorted_keys(const RadixBuffers& buf, int64_t B, int64
         rowhard_keys_kernel<<<(unsigned)B, 1024, 0, st>>>(buf.keys[0], buf.keys[1], n, k, rank,
                                                           buf.plan, b, rows);
     }
+    return launch_hard_emit(r, ld, p, B, n, rows, vec, st);
+}
+
+cudaError_t launch_hard_emit(const float* r, int64_t ld, float* p, int64_t B, int64_t n,
+                             const RowState* rows, int vec, cudaStream_t st) {
     const dim3 grid((unsigned)((n + 4095) / 4096), (unsigned)B);
-    {
-        ProfScope ps_("hard_emit", st);
-        if (vec) hard_emit_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, p, n, rows);
-        else hard_emit_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, p, n, rows);
-    }
+    ProfScope ps_("hard_emit", st);
+    if (vec) hard_emit_kernel<true><<<grid, kThreads, 0, st>>>(r, ld, p, n, rows);
+    else hard_emit_kernel<false><<<grid, kThreads, 0, st>>>(r, ld, p, n, rows);
     return cudaGetLastError();
 }
 

@@ -120,7 +120,8 @@ def test_new_entry_points_reject_bad_arguments_on_host(lib):
     assert hard(d, 8, d, d, 1, 8, 8.0, 0, ws, 1 << 20, None) == 1   # k = n
     assert hard(d, 8, d, d, 1, 8, 0.0, 0, ws, 1 << 20, None) == 1   # k = 0
     assert hard(d, 8, d, d, 1, 1, 0.5, 0, ws, 1 << 20, None) == 1   # n < 2
-    assert hard(d, 8, d, d, 1, 8, 2.0, 2, ws, 1 << 20, None) == 1   # bracket
+    assert hard(d, 8, d, d, 1, 8, 2.0, 4, ws, 1 << 20, None) == 1   # one CTA per row: no
+    assert hard(d, 8, d, d, 1, 8, 2.0, 0x202, ws, 1 << 20, None) == 1  # unknown flag
     assert hard(d, 8, d, d, 1, 8, 2.0, 0, None, 1 << 20, None) == 2  # no ws
 
 
