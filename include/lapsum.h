@@ -342,6 +342,62 @@ int lapsum_profile_enable(int on);
 int lapsum_profile_read(lapsum_kernel_time* out, int max_entries, int* n_entries);
 
 /*
+ * One row split over several devices (section 2.2's bracketing, with the row's
+ * scores in contiguous shards, one per device and process).  Each device holds
+ * the shard [offset, offset + n_shard) of a row of n scores; the caller moves
+ * the small results between the steps (e.g. NCCL all-reduce / all-gather) and
+ * every device then takes the same decisions:
+ *   1. lapsum_bracket_plan (host): the sample size m and the rank ladders
+ *      rank_l[4], rank_h[4] of the row (as the single-device bracketing);
+ *   2. lapsum_shard_sample: y[s] (m floats, device) = draw s of the row's
+ *      sample (the single-device sample, seed as lapsum_forward) when its
+ *      index lies in this shard, else 0; summing y over the devices gives the
+ *      whole sample exactly;
+ *   3. lapsum_sample_bracket: ends = (a_L, a_R) (2 floats, device) from the
+ *      whole sample: the rank_h-th and rank_l-th largest (0 = open end);
+ *   4. lapsum_shard_fold: this shard folded with the bracket: rec (5 doubles,
+ *      device) = (scores >= a_R, sum e^{(r - a_L)/t} below a_L, sum
+ *      e^{-(r - a_R)/t} at or above a_R, non-finite flag, band size) and the
+ *      band scores into band (capacity n_shard floats);
+ *   5. lapsum_shard_band_solve: with every device's rec (recs[w * 5 + i]) and
+ *      band (bands[w * stride + j], j < its band size): out (4 doubles,
+ *      device) = (b, F(a_L), F(a_R), certified 1/0); when not certified the
+ *      caller widens the failing end to its next rung (F(a_L) < k: rank_h,
+ *      else rank_l) and repeats from step 3; b is NaN for a non-finite row;
+ *   6. lapsum_shard_emit: p of this shard from b (device);
+ *   backward: lapsum_shard_vjp_partial gives rec (3 doubles, device: the
+ *   shard's smallest |x| and shifted sums of f and v f) and
+ *   lapsum_shard_vjp_apply g of this shard from every device's rec (recs[w *
+ *   3 + i], merged in device order).
+ * The records are combined in device order, so every device computes the same
+ * b bit for bit.  Workspace: lapsum_shard_workspace_bytes(n_shard) bytes
+ * (cleared once with lapsum_workspace_init; steps 4 and the backward), and for
+ * step 5 a scratch of lapsum_shard_band_bytes(world * stride) bytes, 256-byte
+ * aligned.  Errors: LAPSUM_EINVAL for bad sizes, ranks or parameters,
+ * LAPSUM_EWORKSPACE, LAPSUM_ECUDA.  All pointers are device pointers except
+ * the outputs of lapsum_bracket_plan.
+ */
+int lapsum_bracket_plan(int64_t n, double k, int32_t* m, int64_t* rank_l, int64_t* rank_h);
+size_t lapsum_shard_workspace_bytes(int64_t n_shard);
+size_t lapsum_shard_band_bytes(int64_t n_band_total);
+int lapsum_shard_sample(const float* r, int64_t n_shard, int64_t offset, int64_t n, double t,
+                        uint64_t seed, int32_t m, float* y, void* stream);
+int lapsum_sample_bracket(const float* y, int32_t m, int64_t rank_l, int64_t rank_h, float* ends,
+                          void* stream);
+int lapsum_shard_fold(const float* r, int64_t n_shard, const float* ends, double t, double* rec,
+                      float* band, void* ws, size_t ws_bytes, void* stream);
+int lapsum_shard_band_solve(const float* bands, int64_t stride, const double* recs, int32_t world,
+                            const float* ends, double k, double t, double* out, void* scratch,
+                            size_t scratch_bytes, void* stream);
+int lapsum_shard_emit(const float* r, int64_t n_shard, const double* b, double t, float* p,
+                      void* stream);
+int lapsum_shard_vjp_partial(const float* r, const float* v, int64_t n_shard, const double* b,
+                             double t, double* rec, void* ws, size_t ws_bytes, void* stream);
+int lapsum_shard_vjp_apply(const float* r, const float* v, int64_t n_shard, const double* b,
+                           double t, const double* recs, int32_t world, float* g, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
  * lapsum_backward_noalloc: the same result as lapsum_backward, for callers
  * that cannot allocate device memory (no workspace argument).  The pages have
  * no counterpart of this call; it exists for code that must not allocate at

@@ -37,6 +37,7 @@ namespace {
 constexpr int kBlk = 1024;
 constexpr int kWarpSortMax = 256;  // bands up to this size are sorted and solved by one warp
 constexpr int kFoldThreads = 256;
+constexpr int kFoldGridMaxShard = 4096;  // fold records of the split-row pieces
 
 struct Ladder {
     int64_t l[kLadder];  // descending ranks for a_R (0 = open)
@@ -281,19 +282,12 @@ __device__ void select_two_ranks(const uint32_t* keys, int m, const uint32_t* hi
 // ----------------------------------------------------------------------------
 // 1. Localization sample.
 // ----------------------------------------------------------------------------
-// Sample s of a row: a uniform index I (high half of z1 * n) and Laplace(0, t)
-// noise by the inverse CDF, u = 24 bits of z2 centred in (-1/2, 1/2); z1, z2
-// are SplitMix64 outputs 2s and 2s + 1 of the stream (seed, counters from c0).
+// Sample s of a row: r[I] plus Laplace(0, t) noise (sample_index, sample_noise).
 __device__ __forceinline__ float draw_sample(const float* __restrict__ r, int64_t n, double t,
                                              uint64_t seed, uint64_t c0, int s) {
-    const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
-    const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
-    const int64_t I = (int64_t)__umul64hi(z1, (uint64_t)n);
+    const int64_t I = sample_index(seed, c0, s, n);
     const float rv = __ldg(r + I);
-    const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
-    const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
-    const float eps = (u < 0.0 ? 1.f : -1.f) * (float)t * logf(a);
-    return rv + eps;
+    return rv + sample_noise(seed, c0, s, t);
 }
 // Grid of m / 1024 CTAs: every thread draws one sample.  The order statistics
 // of the bracket are found in one of two ways:
@@ -2041,7 +2035,191 @@ __global__ void __maxnreg__(64) solve2_kernel(double k, double t, RowState* st,
     }
 }
 
+// ----------------------------------------------------------------------------
+// Pieces of the bracketing pipeline for one row split over several devices
+// (each holds a contiguous shard; the host exchanges the small results
+// between them).  The sample is the single-device row's sample: draw s is
+// taken by the shard that holds its index.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) shard_sample_kernel(const float* __restrict__ r,
+                                                           int64_t n_shard, int64_t offset,
+                                                           int64_t n, double t, uint64_t seed,
+                                                           int m, float* __restrict__ y) {
+    const int s = blockIdx.x * 256 + threadIdx.x;
+    if (s >= m) return;
+    const int64_t I = sample_index(seed, 0ull, s, n);
+    const int64_t j = I - offset;
+    y[s] = (j >= 0 && j < n_shard) ? __ldg(r + j) + sample_noise(seed, 0ull, s, t) : 0.f;
+}
+
+// The two order statistics of a complete sample (ranks counted from the top;
+// 0 = open end): ends[0] = a_L (rank_h), ends[1] = a_R (rank_l).
+__global__ void __launch_bounds__(kBlk) sample_bracket_kernel(const float* __restrict__ y, int m,
+                                                              int64_t rank_l, int64_t rank_h,
+                                                              float* __restrict__ ends) {
+    __shared__ uint32_t hist[2048];
+    __shared__ uint32_t wsum[32];
+    __shared__ uint32_t bcast[4];
+    float aL = -INFINITY, aR = INFINITY;
+    if (rank_h >= 1 && rank_h <= m)
+        aL = from_key(block_select_desc(GlobalSampleKeyGet{y}, m, rank_h, hist, wsum, bcast));
+    if (rank_l >= 1 && rank_l <= m)
+        aR = from_key(block_select_desc(GlobalSampleKeyGet{y}, m, rank_l, hist, wsum, bcast));
+    if (threadIdx.x == 0) {
+        ends[0] = aL;
+        ends[1] = aR;
+    }
+}
+
+__global__ void shard_fold_setup_kernel(const float* __restrict__ ends, RowState* st) {
+    for (int i = 0; i < (int)(sizeof(RowState) / 4); ++i) reinterpret_cast<uint32_t*>(st)[i] = 0u;
+    st->a_L = ends[0];
+    st->a_R = ends[1];
+}
+
+// The fold CTAs' records combined in CTA order into rec = (right count, left
+// sum, right sum, non-finite flag, band size).
+__global__ void __launch_bounds__(kBlk) shard_fold_records_kernel(
+    const double* __restrict__ part, int nfold, const RowState* st, double* __restrict__ rec) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    double tot[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int i = threadIdx.x; i < nfold; i += kBlk) {
+        tot[0] += part[4 * i];
+        tot[1] += part[4 * i + 1];
+        tot[2] += part[4 * i + 2];
+        tot[3] += part[4 * i + 3];
+    }
+    block_sums<4>(tot, sm);
+    if (threadIdx.x == 0) {
+        rec[0] = tot[0];
+        rec[1] = tot[1];
+        rec[2] = tot[2];
+        rec[3] = tot[3];
+        rec[4] = (double)st->n_band;
+    }
+}
+
+// The exact solve on the gathered band: the shards' records are combined in
+// shard order into the tails, the shards' band segments are copied into one
+// array, and the band is solved with the tails as virtual anchors (sorted on
+// chip, or narrowed by exact histogram levels when large).  out = (b, F(a_L),
+// F(a_R), certified).
+__global__ void __maxnreg__(64) shard_band_solve_kernel(
+    const float* __restrict__ bands, int64_t stride, const double* __restrict__ recs, int world,
+    const float* __restrict__ ends, double k, double t, float* __restrict__ cur,
+    float* __restrict__ nxt, double* __restrict__ out) {
+    extern __shared__ __align__(16) unsigned char dsm[];
+    SolveSmemAll* sm = reinterpret_cast<SolveSmemAll*>(dsm);
+    Tails tl;
+    tl.aL = ends[0];
+    tl.aR = ends[1];
+    tl.hasL = isfinite(tl.aL);
+    tl.hasR = isfinite(tl.aR);
+    double cr = 0.0, sl = 0.0, sr = 0.0, bad = 0.0;
+    long long nb = 0;
+    for (int w = 0; w < world; ++w) {
+        cr += recs[5 * w];
+        sl += recs[5 * w + 1];
+        sr += recs[5 * w + 2];
+        bad += recs[5 * w + 3];
+        const long long nw = (long long)recs[5 * w + 4];
+        for (long long j = threadIdx.x; j < nw; j += kBlk) cur[nb + j] = bands[w * stride + j];
+        nb += nw;
+    }
+    tl.cntR = cr;
+    tl.SL = sl;
+    tl.SR = sr;
+    __syncthreads();
+    if (bad > 0.0) {
+        if (threadIdx.x == 0) {
+            out[0] = nan("");
+            out[1] = INFINITY;
+            out[2] = -INFINITY;
+            out[3] = 1.0;  // settled: the row has a non-finite score
+        }
+        return;
+    }
+    int certified = 1;
+    if (nb <= kBandSortMax) {
+        solve_small_band(cur, nb, tl, k, t, sm);
+        certified = sm->res.F_aL >= k && sm->res.F_aR <= k;
+    } else {
+        int levels = 0;
+        certified = solve_exact(cur, nxt, nb, tl, k, t, sm, &levels) == 1;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        out[0] = certified ? sm->res.b : nan("");
+        out[1] = sm->res.F_aL;
+        out[2] = sm->res.F_aR;
+        out[3] = certified ? 1.0 : 0.0;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_shard_sample(const float* r, int64_t n_shard, int64_t offset, int64_t n,
+                                double t, uint64_t seed, int m, float* y, cudaStream_t st) {
+    shard_sample_kernel<<<(unsigned)((m + 255) / 256), 256, 0, st>>>(r, n_shard, offset, n, t, seed,
+                                                                   m, y);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sample_bracket(const float* y, int m, int64_t rank_l, int64_t rank_h,
+                                  float* ends, cudaStream_t st) {
+    sample_bracket_kernel<<<1, kBlk, 0, st>>>(y, m, rank_l, rank_h, ends);
+    return cudaGetLastError();
+}
+
+size_t shard_fold_workspace_bytes() {
+    return 512 + (size_t)kFoldGridMaxShard * 4 * sizeof(double);
+}
+
+cudaError_t launch_shard_fold(const float* r, int64_t n_shard, const float* ends, double t,
+                              double* rec, float* band, void* ws, cudaStream_t st) {
+    RowState* rs = static_cast<RowState*>(ws);
+    double* part = reinterpret_cast<double*>(static_cast<char*>(ws) + 512);
+    int grid = bracket_fold_grid();
+    if (grid > kFoldGridMaxShard) grid = kFoldGridMaxShard;
+    static unsigned long long attr_devices = 0ull;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if ((attr_devices & bit) == 0ull || bit == 0ull) {
+        cudaFuncSetAttribute(fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kFoldDynSmem);
+        cudaFuncSetAttribute(shard_fold_records_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(SolveSmemAll));
+        cudaFuncSetAttribute(shard_band_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(SolveSmemAll));
+        attr_devices |= bit;
+    }
+    shard_fold_setup_kernel<<<1, 1, 0, st>>>(ends, rs);
+    const int vec = ((reinterpret_cast<uintptr_t>(r) & 15u) == 0) ? 1 : 0;
+    fold_kernel<<<grid, kFoldThreads, kFoldDynSmem, st>>>(r, n_shard, t, rs, band, nullptr, part,
+                                                          vec, 0);
+    shard_fold_records_kernel<<<1, kBlk, sizeof(SolveSmemAll), st>>>(part, grid, rs, rec);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_shard_band_solve(const float* bands, int64_t stride, const double* recs,
+                                    int world, const float* ends, double k, double t, float* cur,
+                                    float* nxt, double* out, cudaStream_t st) {
+    static unsigned long long attr_devices = 0ull;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if ((attr_devices & bit) == 0ull || bit == 0ull) {
+        cudaFuncSetAttribute(shard_band_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(SolveSmemAll));
+        attr_devices |= bit;
+    }
+    shard_band_solve_kernel<<<1, kBlk, sizeof(SolveSmemAll), st>>>(bands, stride, recs, world,
+                                                                  ends, k, t, cur, nxt, out);
+    return cudaGetLastError();
+}
 
 size_t rowbracket_smem(int m) { return kRowBracketFixedSmem + (size_t)m * sizeof(uint32_t); }
 

@@ -60,8 +60,7 @@ __global__ void __launch_bounds__(kBlk) hard_sample_kernel(const float* __restri
     const int s = blockIdx.x * kBlk + threadIdx.x;
     uint32_t key[1] = {0u};
     if (s < m) {
-        const uint64_t z = splitmix64_at(seed, ((uint64_t)row << 32) + 2ull * (uint64_t)s);
-        const int64_t I = (int64_t)__umul64hi(z, (uint64_t)n);
+        const int64_t I = sample_index(seed, (uint64_t)row << 32, s, n);
         key[0] = hkey(__ldg(rr + I));
     }
     bitonic_sort_row<1, kBlk, kBlk>(key, threadIdx.x, xch);

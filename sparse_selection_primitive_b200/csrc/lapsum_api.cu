@@ -522,6 +522,103 @@ int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t
     return cuda_status(e);
 }
 
+int lapsum_bracket_plan(int64_t n, double k, int32_t* m, int64_t* rank_l, int64_t* rank_h) {
+    if (m == nullptr || rank_l == nullptr || rank_h == nullptr || n < 1) return LAPSUM_EINVAL;
+    if (!(k > 0.0) || !(k < (double)n) || !std::isfinite(k)) return LAPSUM_EINVAL;
+    *m = sample_size(n, k);
+    bracket_ladder(*m, k / (double)n, rank_l, rank_h);
+    return LAPSUM_OK;
+}
+
+size_t lapsum_shard_workspace_bytes(int64_t n_shard) {
+    if (n_shard < 1) return 0;
+    return up(shard_fold_workspace_bytes()) + up(vjp_shard_workspace_bytes());
+}
+
+size_t lapsum_shard_band_bytes(int64_t n_band_total) {
+    if (n_band_total < 0) return 0;
+    return 2 * up((size_t)(n_band_total > 0 ? n_band_total : 1) * sizeof(float));
+}
+
+int lapsum_shard_sample(const float* r, int64_t n_shard, int64_t offset, int64_t n, double t,
+                        uint64_t seed, int32_t m, float* y, void* stream) {
+    if (r == nullptr || y == nullptr || n_shard < 1 || offset < 0 || offset + n_shard > n)
+        return LAPSUM_EINVAL;
+    if (m < 1 || m > kSampleMax || !(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    return cuda_status(launch_shard_sample(r, n_shard, offset, n, t, seed, m, y,
+                                           (cudaStream_t)stream));
+}
+
+int lapsum_sample_bracket(const float* y, int32_t m, int64_t rank_l, int64_t rank_h, float* ends,
+                          void* stream) {
+    if (y == nullptr || ends == nullptr || m < 1 || m > kSampleMax) return LAPSUM_EINVAL;
+    if (rank_l < 0 || rank_h < 0 || (rank_l >= 1 && rank_h >= 1 && rank_l > rank_h))
+        return LAPSUM_EINVAL;
+    return cuda_status(launch_sample_bracket(y, m, rank_l, rank_h, ends, (cudaStream_t)stream));
+}
+
+int lapsum_shard_fold(const float* r, int64_t n_shard, const float* ends, double t, double* rec,
+                      float* band, void* ws, size_t ws_bytes, void* stream) {
+    if (r == nullptr || ends == nullptr || rec == nullptr || band == nullptr || n_shard < 1)
+        return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 ||
+        ws_bytes < lapsum_shard_workspace_bytes(n_shard))
+        return LAPSUM_EWORKSPACE;
+    return cuda_status(launch_shard_fold(r, n_shard, ends, t, rec, band, ws, (cudaStream_t)stream));
+}
+
+int lapsum_shard_band_solve(const float* bands, int64_t stride, const double* recs, int32_t world,
+                            const float* ends, double k, double t, double* out, void* scratch,
+                            size_t scratch_bytes, void* stream) {
+    if (bands == nullptr || recs == nullptr || ends == nullptr || out == nullptr || world < 1 ||
+        stride < 0)
+        return LAPSUM_EINVAL;
+    if (!(k > 0.0) || !std::isfinite(k) || !(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    const size_t half = scratch_bytes / 2 / kAlign * kAlign;
+    if (scratch == nullptr || (reinterpret_cast<uintptr_t>(scratch) % kAlign) != 0 ||
+        scratch_bytes < lapsum_shard_band_bytes((int64_t)world * stride))
+        return LAPSUM_EWORKSPACE;
+    float* cur = static_cast<float*>(scratch);
+    float* nxt = reinterpret_cast<float*>(static_cast<char*>(scratch) + half);
+    return cuda_status(launch_shard_band_solve(bands, stride, recs, world, ends, k, t, cur, nxt, out,
+                                               (cudaStream_t)stream));
+}
+
+int lapsum_shard_emit(const float* r, int64_t n_shard, const double* b, double t, float* p,
+                      void* stream) {
+    if (r == nullptr || b == nullptr || p == nullptr || n_shard < 1) return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    return cuda_status(launch_emit_p(r, p, b, n_shard, t, (cudaStream_t)stream));
+}
+
+int lapsum_shard_vjp_partial(const float* r, const float* v, int64_t n_shard, const double* b,
+                             double t, double* rec, void* ws, size_t ws_bytes, void* stream) {
+    if (r == nullptr || v == nullptr || b == nullptr || rec == nullptr || n_shard < 1)
+        return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 ||
+        ws_bytes < lapsum_shard_workspace_bytes(n_shard))
+        return LAPSUM_EWORKSPACE;
+    void* vws = static_cast<char*>(ws) + up(shard_fold_workspace_bytes());
+    return cuda_status(launch_vjp_partial(r, b, v, n_shard, t, rec, vws, (cudaStream_t)stream));
+}
+
+int lapsum_shard_vjp_apply(const float* r, const float* v, int64_t n_shard, const double* b,
+                           double t, const double* recs, int32_t world, float* g, void* ws,
+                           size_t ws_bytes, void* stream) {
+    if (r == nullptr || v == nullptr || b == nullptr || recs == nullptr || g == nullptr ||
+        n_shard < 1 || world < 1)
+        return LAPSUM_EINVAL;
+    if (!(t > 0.0) || !std::isfinite(t)) return LAPSUM_EINVAL;
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0 ||
+        ws_bytes < lapsum_shard_workspace_bytes(n_shard))
+        return LAPSUM_EWORKSPACE;
+    void* vws = static_cast<char*>(ws) + up(shard_fold_workspace_bytes());
+    return cuda_status(launch_vjp_apply(r, b, v, g, n_shard, t, recs, world, vws,
+                                        (cudaStream_t)stream));
+}
+
 int lapsum_forward_router(const void* r, int dtype, int64_t ld, float* p, double* b, int64_t B,
                           int64_t n, double k, double t, float eps, int32_t cap, int32_t* sel_idx,
                           float* sel_p, int32_t* sel_cnt, void* ws, size_t ws_bytes,

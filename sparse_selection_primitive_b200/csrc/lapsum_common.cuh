@@ -471,6 +471,21 @@ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t c) {
     return z ^ (z >> 31);
 }
 
+// Draw s of a row's localization sample (section 2.2 of the pages): the index
+// I = high half of z1 * n and Laplace(0, t) noise by the inverse CDF from 24
+// bits of z2, u centred in (-1/2, 1/2); z1, z2 are SplitMix64 outputs 2s and
+// 2s + 1 of the stream (seed, counters from c0).
+__device__ __forceinline__ int64_t sample_index(uint64_t seed, uint64_t c0, int64_t s, int64_t n) {
+    const uint64_t z1 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s);
+    return (int64_t)__umul64hi(z1, (uint64_t)n);
+}
+__device__ __forceinline__ float sample_noise(uint64_t seed, uint64_t c0, int64_t s, double t) {
+    const uint64_t z2 = splitmix64_at(seed, c0 + 2ull * (uint64_t)s + 1ull);
+    const double u = ((double)(z2 >> 40) + 0.5) * (1.0 / 16777216.0) - 0.5;
+    const float a = (float)(1.0 - 2.0 * fabs(u));  // exact: a multiple of 2^-24 in (0, 1]
+    return (u < 0.0 ? 1.f : -1.f) * (float)t * logf(a);
+}
+
 // Phase timestamps (ns, global timer) of the single-CTA bracketing steps, kept
 // in the row record's scratch words for diagnostics.
 __device__ __forceinline__ void phase_mark(RowState* st, int slot) {

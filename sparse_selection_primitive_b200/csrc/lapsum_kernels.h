@@ -155,6 +155,18 @@ cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* 
                                       double* partials, double* row_R, uint32_t* tickets, int vec,
                                       const uint32_t* need, cudaStream_t st);
 
+// The VJP of one shard of a row split over devices: its record (min |x|, S,
+// Sv) of the online sums, then g from the shards' records merged in shard
+// order (ws: vjp_shard_workspace_bytes(), the ticket at its start cleared
+// once); and p of a shard from b.
+size_t vjp_shard_workspace_bytes();
+cudaError_t launch_vjp_partial(const float* r, const double* b, const float* v, int64_t n,
+                               double t, double* rec, void* ws, cudaStream_t st);
+cudaError_t launch_vjp_apply(const float* r, const double* b, const float* v, float* g, int64_t n,
+                             double t, const double* recs, int world, void* ws, cudaStream_t st);
+cudaError_t launch_emit_p(const float* r, float* p, const double* b, int64_t n, double t,
+                          cudaStream_t st);
+
 // Gradients of sum v p with respect to k and t, per row; partials: the
 // backward partials region (max(tiles, 2) * 4 doubles per row).
 cudaError_t launch_backward_kt(const float* r, int64_t ld, const double* b, const float* v,
@@ -192,6 +204,26 @@ struct BracketBuffers {
     int fold_grid;
 };
 int bracket_fold_grid();
+// Pieces of the bracketing for one row split over several devices (contiguous
+// shards; the host exchanges the results between the steps).
+// y[s] = draw s of the row's sample when its index lies in this shard, else 0.
+cudaError_t launch_shard_sample(const float* r, int64_t n_shard, int64_t offset, int64_t n,
+                                double t, uint64_t seed, int m, float* y, cudaStream_t st);
+// ends = (a_L, a_R): the rank_h-th and rank_l-th largest of the complete sample.
+cudaError_t launch_sample_bracket(const float* y, int m, int64_t rank_l, int64_t rank_h,
+                                  float* ends, cudaStream_t st);
+// One shard folded with the bracket: rec = (count above a_R, left tail sum,
+// right tail sum, non-finite flag, band size), the band into `band` (capacity
+// n_shard); ws: shard_fold_workspace_bytes().
+size_t shard_fold_workspace_bytes();
+cudaError_t launch_shard_fold(const float* r, int64_t n_shard, const float* ends, double t,
+                              double* rec, float* band, void* ws, cudaStream_t st);
+// The exact solve on the shards' bands (bands[w * stride + j], j < rec_w band
+// size) with their tails: out = (b, F(a_L), F(a_R), certified); cur and nxt
+// hold the total band twice.
+cudaError_t launch_shard_band_solve(const float* bands, int64_t stride, const double* recs,
+                                    int world, const float* ends, double k, double t, float* cur,
+                                    float* nxt, double* out, cudaStream_t st);
 // Sample size and bracket ladder of one row with its own budget (filled on the
 // device from k[row]); ok = 0 for a budget outside (0, n).
 struct RowBudget {

@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
     const float* __restrict__ r, int64_t ld, const double* __restrict__ b,
     const float* __restrict__ v, int64_t n, double t, double* __restrict__ partials,
     double* __restrict__ row_R, uint32_t* __restrict__ tickets,
-    const uint32_t* __restrict__ need) {
+    const uint32_t* __restrict__ need, double* __restrict__ rec_out) {
     pdl_wait();
     __shared__ double red[kThreads / 32];
     __shared__ float fred[kThreads / 32];
@@ -239,7 +239,14 @@ __global__ void __launch_bounds__(kThreads) bwd_reduce_kernel(
         }
         a = block_sum_d(a, red);
         av = block_sum_d(av, red);
-        if (threadIdx.x == 0) row_R[row] = av / a;
+        if (threadIdx.x == 0) {
+            row_R[row] = av / a;
+            if (rec_out != nullptr) {  // the row's record (min |x|, S, Sv), unreduced
+                rec_out[0] = mrow;
+                rec_out[1] = a;
+                rec_out[2] = av;
+            }
+        }
     }
 }
 
@@ -409,9 +416,78 @@ __global__ void __launch_bounds__(kThreads) widen_kernel(const uint16_t* __restr
     }
 }
 
+// R of a row split over devices: the shards' records (min |x|, S, Sv)
+// merged in shard order.
+__global__ void vjp_combine_kernel(const double* __restrict__ recs, int world,
+                                   double* __restrict__ R) {
+    double mrow = INFINITY;
+    for (int w = 0; w < world; ++w) mrow = fmin(mrow, recs[3 * w]);
+    double a = 0.0, av = 0.0;
+    for (int w = 0; w < world; ++w) {
+        if (recs[3 * w] == INFINITY) continue;
+        const double f = exp(mrow - recs[3 * w]);
+        a += recs[3 * w + 1] * f;
+        av += recs[3 * w + 2] * f;
+    }
+    *R = av / a;
+}
+
 }  // namespace
 
 int64_t stream_tiles(int64_t n) { return (n + kStreamTile - 1) / kStreamTile; }
+
+size_t vjp_shard_workspace_bytes() {
+    return 256 + (size_t)device_sm_count() * 8 * 4 * sizeof(double) + 256;
+}
+
+cudaError_t launch_vjp_partial(const float* r, const double* b, const float* v, int64_t n,
+                               double t, double* rec, void* ws, cudaStream_t st) {
+    char* w = static_cast<char*>(ws);
+    uint32_t* ticket = reinterpret_cast<uint32_t*>(w);
+    double* row_R = reinterpret_cast<double*>(w + 64);
+    double* partials = reinterpret_cast<double*>(w + 256);
+    int64_t per_row = (int64_t)device_sm_count() * 8;
+    if (per_row > stream_tiles(n)) per_row = stream_tiles(n);
+    if (per_row < 1) per_row = 1;
+    const int vec = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(v)) & 15u) == 0;
+    if (vec)
+        bwd_reduce_kernel<true><<<(unsigned)per_row, kThreads, 0, st>>>(
+            r, n, b, v, n, t, partials, row_R, ticket, nullptr, rec);
+    else
+        bwd_reduce_kernel<false><<<(unsigned)per_row, kThreads, 0, st>>>(
+            r, n, b, v, n, t, partials, row_R, ticket, nullptr, rec);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_vjp_apply(const float* r, const double* b, const float* v, float* g, int64_t n,
+                             double t, const double* recs, int world, void* ws, cudaStream_t st) {
+    double* R = reinterpret_cast<double*>(static_cast<char*>(ws) + 128);
+    vjp_combine_kernel<<<1, 1, 0, st>>>(recs, world, R);
+    int64_t grid = (int64_t)device_sm_count() * 16;
+    if (grid > stream_tiles(n)) grid = stream_tiles(n);
+    if (grid < 1) grid = 1;
+    const int vec = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(v) |
+                      reinterpret_cast<uintptr_t>(g)) & 15u) == 0;
+    if (vec)
+        bwd_apply_kernel<true><<<(unsigned)grid, kThreads, 0, st>>>(r, n, b, v, g, n, t, R, nullptr);
+    else
+        bwd_apply_kernel<false><<<(unsigned)grid, kThreads, 0, st>>>(r, n, b, v, g, n, t, R,
+                                                                    nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_emit_p(const float* r, float* p, const double* b, int64_t n, double t,
+                          cudaStream_t st) {
+    const int vec = ((reinterpret_cast<uintptr_t>(r) | reinterpret_cast<uintptr_t>(p)) & 15u) == 0;
+    const dim3 grid((unsigned)stream_tiles(n), 1u);
+    if (vec)
+        emit_kernel<true, false, false><<<grid, kThreads, 0, st>>>(
+            r, n, p, b, nullptr, n, t, nullptr, nullptr, nullptr, 0, 1, 0, SupportView{});
+    else
+        emit_kernel<false, false, false><<<grid, kThreads, 0, st>>>(
+            r, n, p, b, nullptr, n, t, nullptr, nullptr, nullptr, 0, 1, 0, SupportView{});
+    return cudaGetLastError();
+}
 
 cudaError_t launch_widen(const void* src, int dtype, int64_t ld, int64_t B, int64_t n, float* dst,
                          cudaStream_t st) {
@@ -483,8 +559,8 @@ cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* 
     if (vec) {
         {
             ProfScope ps_("bwd_reduce", st);
-            launch_pdl(bwd_reduce_kernel<true>, dim3(rgrid), dim3(kThreads), 0, st, r, ld, b, v, n, t, partials, row_R,
-                                                                tickets, need);
+            launch_pdl(bwd_reduce_kernel<true>, dim3(rgrid), dim3(kThreads), 0, st, r, ld, b, v, n,
+                       t, partials, row_R, tickets, need, (double*)nullptr);
         }
         {
             ProfScope ps_("bwd_apply", st);
@@ -494,8 +570,8 @@ cudaError_t launch_backward_stream_if(const float* r, int64_t ld, const double* 
     } else {
         {
             ProfScope ps_("bwd_reduce", st);
-            launch_pdl(bwd_reduce_kernel<false>, dim3(rgrid), dim3(kThreads), 0, st, r, ld, b, v, n, t, partials,
-                                                                 row_R, tickets, need);
+            launch_pdl(bwd_reduce_kernel<false>, dim3(rgrid), dim3(kThreads), 0, st, r, ld, b, v,
+                       n, t, partials, row_R, tickets, need, (double*)nullptr);
         }
         {
             ProfScope ps_("bwd_apply", st);
