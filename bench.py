@@ -46,6 +46,7 @@ UNIT = "elements/s"
 # reads of its inputs and writes of its outputs, once).
 KERNEL_BYTES_PER_ELEMENT = {
     "onchip_fwd": 8,      # read r, write p
+    "onchip_search": 8,   # read r, write p
     "onchip_bwd": 12,     # read r, v, write g
     "emit": 8,            # read r, write p
     "bwd_reduce": 8,      # read r, v
@@ -62,7 +63,7 @@ KERNEL_BYTES_PER_ELEMENT = {
 # Algorithmic bytes per element of one fwd+bwd step, per solver: on-chip rows
 # move r, p, r, v, g once (20 B); the long-row paths read r twice in the
 # forward and r, v twice in the backward (32 B).
-STEP_BYTES_PER_ELEMENT = {"bitonic": 20, "radix": 20, "bracket": 32}
+STEP_BYTES_PER_ELEMENT = {"onchip": 20, "radix": 20, "bracket": 32}
 
 
 def load_peaks():
@@ -718,7 +719,7 @@ def path_step_bytes(w, near):
     measured, not here), r read and p written by the emit, g written by the
     backward, and per gradient-support entry 8 B listed + 8 B read back + 4 B
     v + 4 B kept + 8 + 4 B read by the write pass = 36 B."""
-    if w.path == "bitonic":
+    if w.path == "onchip":
         return 20 * w.elements
     return 16 * w.elements + 36 * near
 

@@ -60,7 +60,9 @@ enum lapsum_status {
 
 /* Solver selection (low byte of `path`). */
 enum lapsum_path {
-    LAPSUM_PATH_AUTO = 0,     /* n <= 4096: bitonic; n <= 2^18: bracketing, one CTA per row;
+    LAPSUM_PATH_AUTO = 0,     /* n <= 256: segment search without a sort (one warp per row;
+                                 a row it does not settle is sorted in the same kernel);
+                                 n <= 4096: bitonic; n <= 2^18: bracketing, one CTA per row;
                                  else bracketing over the whole GPU */
     LAPSUM_PATH_FULLSORT = 1, /* full sort: bitonic for n <= 4096, radix above */
     LAPSUM_PATH_BRACKET = 2,  /* probabilistic bracketing (any n >= 2) */
@@ -78,7 +80,9 @@ enum lapsum_dtype {
 
 /* Test and diagnostic flags, OR-ed into `path`. */
 enum lapsum_flags {
-    LAPSUM_FLAG_FORCE_MISS = 0x100, /* bracketing: start from a bracket that excludes b */
+    LAPSUM_FLAG_FORCE_MISS = 0x100, /* bracketing: start from a bracket that excludes b;
+                                       AUTO with n <= 256: skip the segment search, so
+                                       every row takes the in-kernel sort */
     LAPSUM_FLAG_NO_RETRY = 0x200,   /* bracketing: allow no widening (a miss => LAPSUM_EBRACKET) */
     LAPSUM_FLAG_ONE_CTA_SOLVE = 0x400 /* bracketing: solve every band inside the single-CTA
                                          solve kernel, without the grid-wide extraction that

@@ -355,7 +355,13 @@ int forward_impl(const float* r, int64_t ld, float* p, double* b, double* sum_f,
     const SupportView sv_all = want_sup ? support_view(support, B, n) : SupportView{};
 
     if (rp == LAPSUM_PATH_FULLSORT) {
-        e = launch_onchip_forward(r, ld, p, b, sum_f, B, (int)n, k, k_rows, t, hdr, vec, st);
+        // AUTO: the segment search on rows of n <= 256 (FORCE_MISS sends every
+        // row on to the sort inside the same kernel)
+        const int search = (path & 0xff) != LAPSUM_PATH_AUTO ? 0
+                           : (path & LAPSUM_FLAG_FORCE_MISS) ? 2
+                                                             : 1;
+        e = launch_onchip_forward(r, ld, p, b, sum_f, B, (int)n, k, k_rows, t, hdr, vec, search,
+                                  st);
         return cuda_status(e);
     }
     if (rp == LAPSUM_PATH_RADIX) {
@@ -638,7 +644,7 @@ int lapsum_forward_router(const void* r, int dtype, int64_t ld, float* p, double
     const int vec =
         (aligned16(r) && aligned16(p) && (ld % (dtype == LAPSUM_DTYPE_F32 ? 4 : 8)) == 0) ? 1 : 0;
     return cuda_status(launch_onchip_router(r, dtype, ld, p, b, nullptr, B, (int)n, k, t, hdr, vec,
-                                            sel_idx, sel_p, sel_cnt, want_sel ? cap : 0, eps,
+                                            sel_idx, sel_p, sel_cnt, want_sel ? cap : 0, eps, 1,
                                             (cudaStream_t)stream));
 }
 
@@ -689,6 +695,7 @@ int lapsum_forward_lowp(const void* r, int dtype, int64_t ld, float* p, double* 
         const int vec = (aligned16(r) && aligned16(p) && (ld % 8) == 0) ? 1 : 0;
         return cuda_status(launch_onchip_router(r, dtype, ld, p, b, sum_f, B, (int)n, k, t, hdr,
                                                 vec, nullptr, nullptr, nullptr, 0, 0.f,
+                                                pc == LAPSUM_PATH_AUTO ? 1 : 0,
                                                 (cudaStream_t)stream));
     }
     const size_t base = lapsum_workspace_bytes(B, n, k, path);

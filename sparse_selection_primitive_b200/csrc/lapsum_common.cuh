@@ -273,7 +273,9 @@ __device__ inline long long block_excl_suffix_ll(long long v, long long* wt) {
 //     c < 0:  ln y = ln Bh + ln delta - ln(S - c),      S = sqrt(c^2 + Ah Bh delta).
 // A missing anchor (no scores on that side, weight 0) leaves a single
 // exponential:  Bh = 0: b = sR + t ln(2c/Ah);  Ah = 0: b = sL + t ln(Bh/(-2c)).
-// The result is clamped into [sL, sR].
+// segment_root clamps the result into [sL, sR]; segment_root_raw returns the
+// root of this segment's formula wherever it lies (outside the segment when
+// the balancing segment is another one).
 //
 // With rho = Ah Bh delta / c^2 the larger magnitude |c| + S is |c| (1 + sqrt(1
 // + rho)), or sqrt(Ah Bh delta) (sqrt(1/rho) + sqrt(1 + 1/rho)) when rho > 1,
@@ -282,8 +284,13 @@ __device__ inline long long block_excl_suffix_ll(long long v, long long* wt) {
 // Every lane of one warp calls it with the same arguments: lanes 0, 1 and 2
 // take the three first logarithms at once, and all lanes return b.
 // ---------------------------------------------------------------------------
-static __device__ __noinline__ double segment_root(bool hasL, double sL, double Bh, bool hasR,
-                                                   double sR, double Ah, double c, double t) {
+// The body, inlined where it runs many times per warp (the on-chip search); the
+// single-CTA solvers call the out-of-line copy below.
+template <bool kInline>
+__device__ __forceinline__ double segment_root_body(bool hasL, double sL, double Bh, bool hasR,
+                                                    double sR, double Ah, double c, double t) {
+    auto lg = [](double v) { return kInline ? log(v) : cold_log(v); };
+    auto ex = [](double v) { return kInline ? exp(v) : cold_exp(v); };
     const int lane = threadIdx.x & 31;
     hasL = hasL && Bh > 0.0;
     hasR = hasR && Ah > 0.0;
@@ -293,12 +300,12 @@ static __device__ __noinline__ double segment_root(bool hasL, double sL, double 
     else if (!hasR) arg = Bh / (-2.0 * c);
     else arg = lane == 0 ? Ah : (lane == 1 ? Bh : fabs(c));
     if (lane > 2) arg = 1.0;
-    const double lg = cold_log(arg);
-    const double l0 = __shfl_sync(0xffffffffu, lg, 0);
+    const double lgv = lg(arg);
+    const double l0 = __shfl_sync(0xffffffffu, lgv, 0);
     if (!hasL) return sR + t * l0;
     if (!hasR) return sL + t * l0;
-    const double l1 = __shfl_sync(0xffffffffu, lg, 1);
-    const double l2 = __shfl_sync(0xffffffffu, lg, 2);
+    const double l1 = __shfl_sync(0xffffffffu, lgv, 1);
+    const double l2 = __shfl_sync(0xffffffffu, lgv, 2);
     const double lnd = (sL - sR) / t, lnA = l0, lnB = l1;
     double ln_y;
     if (c == 0.0) {
@@ -308,17 +315,28 @@ static __device__ __noinline__ double segment_root(bool hasL, double sL, double 
         const double lnrho = lnA + lnB + lnd - 2.0 * lnc;
         double L;  // ln(|c| + S)
         if (lnrho <= 0.0) {
-            const double rho = cold_exp(lnrho);
-            L = lnc + cold_log(1.0 + sqrt(1.0 + rho));
+            const double rho = ex(lnrho);
+            L = lnc + lg(1.0 + sqrt(1.0 + rho));
         } else {
-            const double sg = cold_exp(-lnrho);
-            L = 0.5 * (lnA + lnB + lnd) + cold_log(sqrt(sg) + sqrt(1.0 + sg));
+            const double sg = ex(-lnrho);
+            L = 0.5 * (lnA + lnB + lnd) + lg(sqrt(sg) + sqrt(1.0 + sg));
         }
         ln_y = c > 0.0 ? L - lnA : lnB + lnd - L;
     }
-    double b = sR + t * ln_y;
-    if (b < sL) b = sL;
-    if (b > sR) b = sR;
+    return sR + t * ln_y;
+}
+static __device__ __noinline__ double segment_root_raw(bool hasL, double sL, double Bh,
+                                                       bool hasR, double sR, double Ah, double c,
+                                                       double t) {
+    return segment_root_body<false>(hasL, sL, Bh, hasR, sR, Ah, c, t);
+}
+__device__ __forceinline__ double segment_root(bool hasL, double sL, double Bh, bool hasR,
+                                               double sR, double Ah, double c, double t) {
+    double b = segment_root_raw(hasL, sL, Bh, hasR, sR, Ah, c, t);
+    if (hasL && Bh > 0.0 && hasR && Ah > 0.0) {
+        if (b < sL) b = sL;
+        if (b > sR) b = sR;
+    }
     return b;
 }
 
@@ -383,6 +401,11 @@ __device__ __forceinline__ float warp_min_f(float v) {
 __device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, d));
+    return v;
+}
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
     return v;
 }
 __device__ __forceinline__ int warp_sum_i(int v) {

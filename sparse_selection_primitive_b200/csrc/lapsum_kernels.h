@@ -43,9 +43,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // --- on-chip full sort (n <= 4096) -------------------------------------------
 int onchip_npad(int64_t n);
 // k_rows (device, B entries) when not null gives each row its own budget.
+// search != 0 solves rows of n <= 256 by the segment search (no sort; rows it
+// leaves are sorted in the same kernel; 2 leaves every row to the sort);
+// otherwise, and for longer rows, the bitonic sort and scans.
 cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,
                                   int64_t B, int n, double k, const double* k_rows, double t,
-                                  WsHeader* hdr, int vec, cudaStream_t st);
+                                  WsHeader* hdr, int vec, int search, cudaStream_t st);
 cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
                                    float* g, int64_t B, int n, double t, int vec, cudaStream_t st);
 // Zero-temperature limit (hard top-k) of rows of n <= 4096: sort, boundary group, p.
@@ -58,7 +61,7 @@ cudaError_t launch_onchip_hard(const float* r, int64_t ld, float* p, double* b, 
 cudaError_t launch_onchip_router(const void* r, int dtype, int64_t ld, float* p, double* b,
                                  double* sumf, int64_t B, int n, double k, double t, WsHeader* hdr,
                                  int vec, int32_t* sel_idx, float* sel_val, int32_t* sel_cnt,
-                                 int cap, float eps, cudaStream_t st);
+                                 int cap, float eps, int search, cudaStream_t st);
 cudaError_t launch_onchip_backward_router(const void* r, int dtype, int64_t ld, const double* b,
                                           const float* v, float* g, int64_t B, int n, double t,
                                           int vec, cudaStream_t st);

@@ -251,30 +251,199 @@ struct SelectOut {
     float eps;
 };
 
+// Shared memory of the sort-and-scan solve of one CTA's rows.
+template <int E, int RT, int CTA>
+struct SortSmem {
+    uint32_t xch[(RT > 32) ? CTA * E : 1];
+    uint32_t last_key[CTA];
+    double first_gap[CTA];
+    Aff wf[CTA / 32], wb[CTA / 32];
+    int ired[CTA / 32];
+    double anchor[CTA / RT][4];
+};
+
+// Sort-and-scan solve of one row (section 2.2, full-sort solver): bitonic sort
+// of the keys (E per thread, pads last), gap factors, the prefix and suffix
+// scans of the threshold curve, the count of F(s_j) >= k and the closed-form
+// root in that segment.  Every thread of the CTA calls it when a row spans
+// several warps (the CTA synchronises); a row of one warp may call it alone.
+// The row's first warp returns b (NaN when `ok` is false); other threads
+// return 0.
+template <int E, int RT, int CTA>
+__device__ __forceinline__ double sort_solve_row(uint32_t (&key)[E], int n, double kr, double t,
+                                                 bool ok, SortSmem<E, RT, CTA>& sm) {
+    using S = Shape<E, RT, CTA>;
+    const int rloc = threadIdx.x / RT;
+    const int tid = threadIdx.x % RT;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const double inv_t = 1.0 / t;
+
+    bitonic_sort_row<E, RT, CTA>(key, tid, sm.xch);
+
+    // Sorted values and gap factors g_j = exp((s_{j-1} - s_j)/t), 0 at j = 0 and past n.
+    float s[E];
+    double g[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[e] = from_key(key[e]);
+    sm.last_key[threadIdx.x] = key[E - 1];
+    row_sync<E, RT, CTA>();
+    const float s_prev = (tid > 0) ? from_key(sm.last_key[threadIdx.x - 1]) : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = tid * E + e;
+        const float sp = (e == 0) ? s_prev : s[e - 1];
+        g[e] = (j >= 1 && j < n) ? gap_factor(sp, s[e], inv_t) : 0.0;
+    }
+    sm.first_gap[threadIdx.x] = g[0];
+    row_sync<E, RT, CTA>();
+    const double g_next = (tid + 1 < RT) ? sm.first_gap[threadIdx.x + 1] : 0.0;
+
+    // Thread aggregates of the forward (prefix) and backward (suffix) maps.
+    Aff af = aff_id(), ab = aff_id();
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = tid * E + e;
+        const Aff m = (j < n) ? Aff{g[e], 1.0} : aff_id();
+        af = aff_then(af, m);
+    }
+#pragma unroll
+    for (int e = E - 1; e >= 0; --e) {
+        const int j = tid * E + e;
+        const double gn = (e + 1 < E) ? g[e + 1] : g_next;
+        const Aff m = (j < n) ? Aff{gn, 1.0} : Aff{0.0, 0.0};
+        ab = aff_then(ab, m);
+    }
+    // Exclusive prefix (maps of earlier threads) and suffix (later threads).
+    Aff inc_f = warp_scan_fwd(af, lane);
+    Aff inc_b = warp_scan_bwd(ab, lane);
+    Aff ex_f = shfl_up_aff(inc_f, 1);
+    Aff ex_b = shfl_down_aff(inc_b, 1);
+    if (lane == 0) ex_f = aff_id();
+    if (lane == 31) ex_b = aff_id();
+    if constexpr (S::WPR > 1) {
+        if (lane == 31) sm.wf[warp] = inc_f;
+        if (lane == 0) sm.wb[warp] = inc_b;
+        __syncthreads();
+        const int w0 = (warp / S::WPR) * S::WPR;
+        Aff pre = aff_id();
+        for (int w = w0; w < warp; ++w) pre = aff_then(pre, sm.wf[w]);
+        ex_f = aff_then(pre, ex_f);
+        Aff suf = aff_id();
+        for (int w = w0 + S::WPR - 1; w > warp; --w) suf = aff_then(suf, sm.wb[w]);
+        ex_b = aff_then(suf, ex_b);
+    }
+
+    // Threshold curve G_j = F(s_j) = (n - j) - Q_j/2 + (P_j - 1)/2 and its count.
+    double P[E], Q[E];
+    double x = ex_f.c;  // P just before this thread's first element
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        x = fma(g[e], x, 1.0);
+        P[e] = x;
+    }
+    double y = ex_b.c;  // Q just after this thread's last element
+    int cnt = 0;
+#pragma unroll
+    for (int e = E - 1; e >= 0; --e) {
+        const int j = tid * E + e;
+        const double gn = (e + 1 < E) ? g[e + 1] : g_next;
+        y = (j < n) ? fma(gn, y, 1.0) : 0.0;
+        Q[e] = y;
+        const double G = (double)(n - j) - 0.5 * Q[e] + 0.5 * (P[e] - 1.0);
+        cnt += (j < n && G >= kr) ? 1 : 0;
+    }
+    const int jstar = row_sum_i<E, RT, CTA>(cnt, sm.ired);
+
+    // Anchors of the balancing segment: left = sorted position j*-1, right = j*.
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int j = tid * E + e;
+        if (j == jstar - 1) {
+            sm.anchor[rloc][0] = s[e];
+            sm.anchor[rloc][1] = P[e];
+        }
+        if (j == jstar && j < n) {
+            sm.anchor[rloc][2] = s[e];
+            sm.anchor[rloc][3] = Q[e];
+        }
+    }
+    row_sync<E, RT, CTA>();
+    double bb = 0.0;
+    if (tid < 32) {  // the row's first warp takes the root together
+        if (!ok) {
+            bb = nan("");
+        } else {
+            const bool hasL = jstar >= 1, hasR = jstar < n;
+            bb = segment_root(hasL, sm.anchor[rloc][0], hasL ? sm.anchor[rloc][1] : 0.0, hasR,
+                              sm.anchor[rloc][2], hasR ? sm.anchor[rloc][3] : 0.0,
+                              (double)(n - jstar) - kr, t);
+        }
+    }
+    return bb;
+}
+
+// Emit p_i = sigma((r_i - b)/t) in the original order; optionally the row's
+// sum of f and the router list of p > eps.  Every thread of the row calls it.
+template <int E, int RT, int CTA>
+__device__ __forceinline__ void emit_row(const float (&orig)[E], const bool (&valid)[E],
+                                         double bb, double t, float* __restrict__ prow, int n,
+                                         int tid, bool vec, bool row_ok, int64_t row,
+                                         double* __restrict__ sumf_out, const SelectOut& sel,
+                                         int* ired, double* dred) {
+    const Thr th = make_thr(bb, t);
+    float pv[E];
+    double sf = 0.0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const float xs = scaled_margin(orig[e], th);
+        const float ex = neg_abs_exp(xs);
+        pv[e] = cdf_from(xs, ex);
+        if (valid[e]) sf += 0.5 * (double)ex;
+    }
+    store_row<E>(prow, n, tid, vec, row_ok, pv);
+    if (sumf_out != nullptr) {
+        const double tot = row_sum_d<E, RT, CTA>(sf, dred);
+        if (tid == 0 && row_ok) sumf_out[row] = tot;
+    }
+    if (sel.cnt != nullptr) {  // the same for every thread of the grid
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) c += (valid[e] && pv[e] > sel.eps) ? 1 : 0;
+        int total = 0;
+        int o = row_excl_scan_i<E, RT, CTA>(c, ired, &total);
+        if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                if (valid[e] && pv[e] > sel.eps) {
+                    if (o < sel.cap) {
+                        sel.idx[row * sel.cap + o] = tid * E + e;
+                        sel.val[row * sel.cap + o] = pv[e];
+                    }
+                    ++o;
+                }
+            }
+            if (tid == 0) sel.cnt[row] = total;
+        }
+    }
+}
+
 template <int E, int RT, int CTA, class In>
 __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel(
     const In* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
     double* __restrict__ sumf_out, int64_t B, int n, double k, const double* __restrict__ k_rows,
     double t, WsHeader* hdr, int vec, SelectOut sel) {
     using S = Shape<E, RT, CTA>;
-    __shared__ uint32_t xch[(RT > 32) ? CTA * E : 1];
-    __shared__ uint32_t last_key[CTA];
-    __shared__ double first_gap[CTA];
-    __shared__ Aff wf[S::NW], wb[S::NW];
-    __shared__ int ired[S::NW];
+    __shared__ SortSmem<E, RT, CTA> sm;
     __shared__ double dred[S::NW];
-    __shared__ double anchor[S::ROWS][4];
     __shared__ int row_flag[S::ROWS];
     __shared__ double row_b[S::ROWS];
 
     const int rloc = threadIdx.x / RT;
     const int tid = threadIdx.x % RT;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
     const int64_t row = (int64_t)blockIdx.x * S::ROWS + rloc;
     const bool row_ok = row < B;
     const In* rrow = r + (row_ok ? row : 0) * ld;
-    const double inv_t = 1.0 / t;
     // the row's budget: the shared k, or its own entry of k_rows (checked here: a
     // budget outside (0, n) gives b = NaN and a status bit)
     const double kr = (k_rows != nullptr && row_ok) ? k_rows[row] : k;
@@ -300,153 +469,242 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
     row_sync<E, RT, CTA>();
     if (bad) atomicOr(&row_flag[rloc], 1);
     if (tid == 0 && !k_ok) atomicOr(&row_flag[rloc], 2);
-
-    bitonic_sort_row<E, RT, CTA>(key, tid, xch);
-
-    // Sorted values and gap factors g_j = exp((s_{j-1} - s_j)/t), 0 at j = 0 and past n.
-    float s[E];
-    double g[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) s[e] = from_key(key[e]);
-    last_key[threadIdx.x] = key[E - 1];
     row_sync<E, RT, CTA>();
-    const float s_prev = (tid > 0) ? from_key(last_key[threadIdx.x - 1]) : 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int j = tid * E + e;
-        const float sp = (e == 0) ? s_prev : s[e - 1];
-        g[e] = (j >= 1 && j < n) ? gap_factor(sp, s[e], inv_t) : 0.0;
-    }
-    first_gap[threadIdx.x] = g[0];
-    row_sync<E, RT, CTA>();
-    const double g_next = (tid + 1 < RT) ? first_gap[threadIdx.x + 1] : 0.0;
+    const int flag = row_flag[rloc];
 
-    // Thread aggregates of the forward (prefix) and backward (suffix) maps.
-    Aff af = aff_id(), ab = aff_id();
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int j = tid * E + e;
-        const Aff m = (j < n) ? Aff{g[e], 1.0} : aff_id();
-        af = aff_then(af, m);
-    }
-#pragma unroll
-    for (int e = E - 1; e >= 0; --e) {
-        const int j = tid * E + e;
-        const double gn = (e + 1 < E) ? g[e + 1] : g_next;
-        const Aff m = (j < n) ? Aff{gn, 1.0} : Aff{0.0, 0.0};
-        ab = aff_then(ab, m);
-    }
-    // Exclusive prefix (maps of earlier threads) and suffix (later threads).
-    Aff inc_f = warp_scan_fwd(af, lane);
-    Aff inc_b = warp_scan_bwd(ab, lane);
-    Aff ex_f = shfl_up_aff(inc_f, 1);
-    Aff ex_b = shfl_down_aff(inc_b, 1);
-    if (lane == 0) ex_f = aff_id();
-    if (lane == 31) ex_b = aff_id();
-    if constexpr (S::WPR > 1) {
-        if (lane == 31) wf[warp] = inc_f;
-        if (lane == 0) wb[warp] = inc_b;
-        __syncthreads();
-        const int w0 = (warp / S::WPR) * S::WPR;
-        Aff pre = aff_id();
-        for (int w = w0; w < warp; ++w) pre = aff_then(pre, wf[w]);
-        ex_f = aff_then(pre, ex_f);
-        Aff suf = aff_id();
-        for (int w = w0 + S::WPR - 1; w > warp; --w) suf = aff_then(suf, wb[w]);
-        ex_b = aff_then(suf, ex_b);
-    }
-
-    // Threshold curve G_j = F(s_j) = (n - j) - Q_j/2 + (P_j - 1)/2 and its count.
-    double P[E], Q[E];
-    double x = ex_f.c;  // P just before this thread's first element
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        x = fma(g[e], x, 1.0);
-        P[e] = x;
-    }
-    double y = ex_b.c;  // Q just after this thread's last element
-    int cnt = 0;
-#pragma unroll
-    for (int e = E - 1; e >= 0; --e) {
-        const int j = tid * E + e;
-        const double gn = (e + 1 < E) ? g[e + 1] : g_next;
-        y = (j < n) ? fma(gn, y, 1.0) : 0.0;
-        Q[e] = y;
-        const double G = (double)(n - j) - 0.5 * Q[e] + 0.5 * (P[e] - 1.0);
-        cnt += (j < n && G >= kr) ? 1 : 0;
-    }
-    const int jstar = row_sum_i<E, RT, CTA>(cnt, ired);
-
-    // Anchors of the balancing segment: left = sorted position j*-1, right = j*.
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int j = tid * E + e;
-        if (j == jstar - 1) {
-            anchor[rloc][0] = s[e];
-            anchor[rloc][1] = P[e];
-        }
-        if (j == jstar && j < n) {
-            anchor[rloc][2] = s[e];
-            anchor[rloc][3] = Q[e];
-        }
+    const double bb = sort_solve_row<E, RT, CTA>(key, n, kr, t, flag == 0 && row_ok, sm);
+    if (tid == 0) {
+        if (flag && row_ok)
+            set_status(hdr, ((flag & 1) ? kDevNonFinite : 0u) | ((flag & 2) ? kDevBadBudget : 0u));
+        row_b[rloc] = bb;
+        if (row_ok) b_out[row] = bb;
     }
     row_sync<E, RT, CTA>();
-    if (tid < 32) {  // the row's first warp takes the root together
-        double bb;
-        const int flag = row_flag[rloc];
-        if (flag || !row_ok) {
-            bb = nan("");
-            if (row_ok && tid == 0)
-                set_status(hdr, ((flag & 1) ? kDevNonFinite : 0u) | ((flag & 2) ? kDevBadBudget : 0u));
+    emit_row<E, RT, CTA>(orig, valid, row_b[rloc], t, p + (row_ok ? row : 0) * ld, n, tid,
+                         vec != 0, row_ok, row, sumf_out, sel, sm.ired, dred);
+}
+
+// ---------------------------------------------------------------------------
+// Rows of at most 256 scores, one warp each, solved without a sort (AUTO).
+//
+// F(c) = sum_i sigma((r_i - c)/t) is continuous and decreasing.  Between two
+// neighbouring scores sA <= c < sB it has the closed form of section 2.2's
+// root step: with m scores at or above sB, Bh = sum_{r <= sA} e^{(r - sA)/t}
+// and Ah = sum_{r >= sB} e^{-(r - sB)/t},
+//     F(c) = m - (Ah/2) e^{(c - sB)/t} + (Bh/2) e^{(sA - c)/t},
+// so the neighbours of one point c, a count and two sums of exponentials (each
+// term at most 1) give that segment's root.  When the root lies in the
+// segment it is b.  When it lies beyond sB, then F(sB) > k and b > sB; read
+// past sB, the formula keeps the crossed scores at 1 - e^{|x|}/2 where F has
+// e^{-|x|}/2, never more, so the formula's root lies in (sB, b]: moving c
+// there never overshoots, and each step leaves at least one score behind;
+// symmetrically on the left.  A move back across the
+// score just crossed can only come from rounding at a boundary where F = k,
+// and that score is then b.  The start is a point whose count of larger
+// scores is close to k, found by interpolating the count between the row's
+// extremes.  Rows that do not settle in kSearchSteps steps are sorted and
+// solved by the full-sort solver in the same warp.
+//
+// Accuracy: every exponential is fp32 and every term is at most 1, so Ah and
+// Bh carry a relative error of about 1e-6 and b one of about 1e-6 t.
+// ---------------------------------------------------------------------------
+constexpr int kSearchRounds = 6;  // count-interpolation rounds for the start
+constexpr int kSearchSteps = 8;   // segment steps before the row is sorted instead
+
+// The closed-form root of one segment (the log-domain form of section 2.2's
+// root step, as in segment_root), unclamped, in mixed precision: the
+// logarithms, exponentials and square roots of quantities of moderate size
+// (Ah, Bh, |c| in [1e-38, 256], rho or 1/rho in (0, 1]) use the hardware
+// approximations (about 2^-22 relative, or 2^-21 absolute for a logarithm near
+// 0), which move b by a few 1e-7 t; the scaled gap ln delta = (sL - sR)/t,
+// which can be large, and every sum that contains it stay in fp64, so b keeps
+// fp64 accuracy relative to the anchors.  Every lane of the warp calls it with
+// the same arguments; lanes 0, 1 and 2 take the three logarithms.
+// sqrt of x >= 0 from the hardware reciprocal square root (about 2^-22 relative)
+__device__ __forceinline__ float fast_sqrt(float x) { return x > 0.f ? x * rsqrtf(x) : 0.f; }
+
+__device__ __forceinline__ double search_root(bool hasL, float sL, float Bh, bool hasR, float sR,
+                                              float Ah, float c, double t, double inv_t) {
+    const int lane = threadIdx.x & 31;
+    if (!hasL && !hasR) return nan("");
+    float arg = 1.f;
+    if (!hasL) arg = 2.f * c / Ah;
+    else if (!hasR) arg = Bh / (-2.f * c);
+    else arg = lane == 0 ? Ah : (lane == 1 ? Bh : fabsf(c));
+    if (lane > 2) arg = 1.f;
+    const float lg = __logf(arg);
+    const double l0 = (double)__shfl_sync(0xffffffffu, lg, 0);
+    if (!hasL) return (double)sR + t * l0;
+    if (!hasR) return (double)sL + t * l0;
+    const double lnA = l0, lnB = (double)__shfl_sync(0xffffffffu, lg, 1);
+    const double lnd = ((double)sL - (double)sR) * inv_t;
+    double ln_y;
+    if (c == 0.f) {
+        ln_y = 0.5 * (lnB + lnd - lnA);
+    } else {
+        const double lnc = (double)__shfl_sync(0xffffffffu, lg, 2);
+        const double lnrho = lnA + lnB + lnd - 2.0 * lnc;
+        double L;  // ln(|c| + S)
+        if (lnrho <= 0.0) {
+            const float rho = __expf((float)lnrho);
+            L = lnc + (double)__logf(1.f + fast_sqrt(1.f + rho));
         } else {
-            const bool hasL = jstar >= 1, hasR = jstar < n;
-            bb = segment_root(hasL, anchor[rloc][0], hasL ? anchor[rloc][1] : 0.0, hasR,
-                              anchor[rloc][2], hasR ? anchor[rloc][3] : 0.0,
-                              (double)(n - jstar) - kr, t);
+            const float sg = __expf((float)-lnrho);
+            L = 0.5 * (lnA + lnB + lnd) + (double)__logf(fast_sqrt(sg) + fast_sqrt(1.f + sg));
         }
-        if (tid == 0) {
-            row_b[rloc] = bb;
-            if (row_ok) b_out[row] = bb;
-        }
+        ln_y = c > 0.f ? L - lnA : lnB + lnd - L;
     }
-    row_sync<E, RT, CTA>();
+    return (double)sR + t * ln_y;
+}
 
-    // Emit p_i = sigma((r_i - b)/t) in the original order, and sum f.
-    const Thr th = make_thr(row_b[rloc], t);
-    float pv[E];
-    double sf = 0.0;
+template <int E, bool FULL>
+__device__ __forceinline__ bool search_row(const float (&x)[E], const bool (&valid)[E], int n,
+                                           double k, double t, int max_steps, double* b_out) {
+    constexpr unsigned kFull = 0xffffffffu;
+    // FULL: every element of the warp is a score of the row (n = 32 E)
+    auto ok = [&](int e) { return FULL || valid[e]; };
+    float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-        const float xs = scaled_margin(orig[e], th);
-        const float ex = neg_abs_exp(xs);
-        pv[e] = cdf_from(xs, ex);
-        if (valid[e]) sf += 0.5 * (double)ex;
+        if (ok(e)) {
+            vmin = fminf(vmin, x[e]);
+            vmax = fmaxf(vmax, x[e]);
+        }
     }
-    store_row<E>(p + (row_ok ? row : 0) * ld, n, tid, vec != 0, row_ok, pv);
-    if (sumf_out != nullptr) {
-        const double tot = row_sum_d<E, RT, CTA>(sf, dred);
-        if (tid == 0 && row_ok) sumf_out[row] = tot;
+    // order-preserving keys carry the float extremes through the integer reductions
+    float lo = from_key(__reduce_min_sync(kFull, to_key(vmin)));
+    float hi = from_key(__reduce_max_sync(kFull, to_key(vmax)));
+
+    // Start: interpolate the count of larger scores between the extremes.
+    int nlo = n, nhi = 0;
+    const float kf = (float)k;
+    for (int round = 0; round < kSearchRounds && nlo - nhi > 2; ++round) {
+        float f = __fdividef((float)nlo - kf, (float)(nlo - nhi));
+        f = fminf(fmaxf(f, 0.0625f), 0.9375f);
+        const float c = fmaf(hi - lo, f, lo);
+        if (!(c > lo && c < hi)) break;
+        unsigned m = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) m += (ok(e) && x[e] > c) ? 1u : 0u;
+        m = __reduce_add_sync(kFull, m);
+        if ((double)m >= k) {
+            lo = c;
+            nlo = (int)m;
+        } else {
+            hi = c;
+            nhi = (int)m;
+        }
     }
-    if (sel.cnt != nullptr) {  // the same for every thread of the grid
-        int c = 0;
+    float c = ((double)nlo - k <= k - (double)nhi) ? lo : hi;
+
+    const float sc = (float)(1.0 / t) * kLog2e;
+    const double inv_t = 1.0 / t;
+    int dir = 0;  // last move: +1 right, -1 left
+    for (int step = 0; step < max_steps; ++step) {
+        // neighbours of c: sA = the largest score <= c, sB = the smallest above
+        float a = -INFINITY, bb = INFINITY;
+        unsigned m = 0;
 #pragma unroll
-        for (int e = 0; e < E; ++e) c += (valid[e] && pv[e] > sel.eps) ? 1 : 0;
-        int total = 0;
-        int o = row_excl_scan_i<E, RT, CTA>(c, ired, &total);
-        if (row_ok) {
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                if (valid[e] && pv[e] > sel.eps) {
-                    if (o < sel.cap) {
-                        sel.idx[row * sel.cap + o] = tid * E + e;
-                        sel.val[row * sel.cap + o] = pv[e];
-                    }
-                    ++o;
+        for (int e = 0; e < E; ++e) {
+            if (ok(e)) {
+                if (x[e] <= c) {
+                    a = fmaxf(a, x[e]);
+                } else {
+                    bb = fminf(bb, x[e]);
+                    ++m;
                 }
             }
-            if (tid == 0) sel.cnt[row] = total;
         }
+        const uint32_t ka = __reduce_max_sync(kFull, to_key(a));
+        const uint32_t kb = __reduce_min_sync(kFull, to_key(bb));
+        m = __reduce_add_sync(kFull, m);
+        const bool hasL = ka != to_key(-INFINITY), hasR = kb != to_key(INFINITY);
+        const float sA = from_key(ka), sB = from_key(kb);
+        float Bh = 0.f, Ah = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if (ok(e)) {
+                if (x[e] <= c) Bh += ex2_ftz((x[e] - sA) * sc);
+                else Ah += ex2_ftz((sB - x[e]) * sc);
+            }
+        }
+        Bh = warp_sum_f(Bh);
+        Ah = warp_sum_f(Ah);
+        const double rt =
+            search_root(hasL, sA, Bh, hasR, sB, Ah, (float)((double)m - k), t, inv_t);
+        if (!(rt == rt)) return false;
+        const bool right = hasR && rt > (double)sB;
+        const bool left = hasL && rt < (double)sA;
+        if (!right && !left) {
+            *b_out = rt;
+            return true;
+        }
+        const int d = right ? 1 : -1;
+        if (dir == -d) {  // back across the score just crossed: F = k there within rounding
+            *b_out = right ? (double)sB : (double)sA;
+            return true;
+        }
+        dir = d;
+        c = right ? fmaxf((float)rt, sB) : fminf((float)rt, nextafterf(sA, -INFINITY));
     }
+    return false;
+}
+
+// The sort-and-scan solve for a row the search left, out of line so that the
+// search keeps its registers; it reloads the row.
+template <int E, class In>
+__device__ __noinline__ double search_fallback_row(const In* rrow, int n, int vec, double k,
+                                                   double t, SortSmem<E, 32, 256>* sm) {
+    float x[E];
+    bool valid[E];
+    load_row<E>(rrow, n, threadIdx.x & 31, vec != 0, true, x, valid);
+    uint32_t key[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) key[e] = valid[e] ? to_key(x[e]) : kPadKey;
+    return sort_solve_row<E, 32, 256>(key, n, k, t, true, *sm);
+}
+
+template <int E, class In>
+__global__ void __launch_bounds__(256, 6) onchip_search_kernel(
+    const In* __restrict__ r, int64_t ld, float* __restrict__ p, double* __restrict__ b_out,
+    double* __restrict__ sumf_out, int64_t B, int n, double k, const double* __restrict__ k_rows,
+    double t, WsHeader* hdr, int vec, SelectOut sel, int max_steps) {
+    constexpr int RT = 32, CTA = 256;
+    __shared__ SortSmem<E, RT, CTA> sm;  // for rows the search leaves to the sort
+    __shared__ double dred[CTA / 32];
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (CTA / RT) + (threadIdx.x >> 5);
+    const bool row_ok = row < B;
+    const In* rrow = r + (row_ok ? row : 0) * ld;
+    const double kr = (k_rows != nullptr && row_ok) ? k_rows[row] : k;
+    const bool k_ok = kr > 0.0 && kr < (double)n;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        hdr->last_B = B;
+        hdr->last_n = n;
+        hdr->last_path = LAPSUM_PATH_FULLSORT;
+    }
+
+    float orig[E];
+    bool valid[E];
+    load_row<E>(rrow, n, lane, vec != 0, row_ok, orig, valid);
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < E; ++e) bad |= valid[e] && !finite_f(orig[e]);
+    bad = __any_sync(0xffffffffu, bad);
+
+    double bb = nan("");
+    if (row_ok) {  // uniform over the warp
+        if (bad || !k_ok) {
+            if (lane == 0)
+                set_status(hdr, (bad ? kDevNonFinite : 0u) | (!k_ok ? kDevBadBudget : 0u));
+        } else if (!(n == 32 * E ? search_row<E, true>(orig, valid, n, kr, t, max_steps, &bb)
+                                  : search_row<E, false>(orig, valid, n, kr, t, max_steps, &bb))) {
+            bb = search_fallback_row<E, In>(rrow, n, vec, kr, t, &sm);
+        }
+        if (lane == 0) b_out[row] = bb;
+    }
+    emit_row<E, RT, CTA>(orig, valid, bb, t, p + (row_ok ? row : 0) * ld, n, lane, vec != 0,
+                         row_ok, row, sumf_out, sel, sm.ired, dred);
 }
 
 // Zero-temperature limit ("Fast LapSum: Exact Differentiable Top-k at Million
@@ -607,10 +865,34 @@ cudaError_t launch_bwd(const In* r, int64_t ld, const double* b, const float* v,
     return cudaGetLastError();
 }
 
+template <int E, class In>
+cudaError_t launch_search(const In* r, int64_t ld, float* p, double* b, double* sumf, int64_t B,
+                          int n, double k, const double* k_rows, double t, WsHeader* hdr, int vec,
+                          const SelectOut& sel, int search, cudaStream_t st) {
+    const int64_t grid = (B + 7) / 8;
+    {
+        ProfScope ps_("onchip_search", st);
+        // search == 2: no segment steps, every row goes to the sort (a test switch)
+        onchip_search_kernel<E, In><<<(unsigned)grid, 256, 0, st>>>(
+            r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, search == 2 ? 0 : kSearchSteps);
+    }
+    return cudaGetLastError();
+}
+
 template <class In>
 cudaError_t onchip_forward_any(const In* r, int64_t ld, float* p, double* b, double* sumf,
                                int64_t B, int n, double k, const double* k_rows, double t,
-                               WsHeader* hdr, int vec, const SelectOut& sel, cudaStream_t st) {
+                               WsHeader* hdr, int vec, const SelectOut& sel, int search,
+                               cudaStream_t st) {
+    if (search) {
+        switch (onchip_npad(n)) {
+            case 32: return launch_search<1, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, search, st);
+            case 64: return launch_search<2, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, search, st);
+            case 128: return launch_search<4, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, search, st);
+            case 256: return launch_search<8, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, search, st);
+            default: break;  // longer rows: the sort
+        }
+    }
     switch (onchip_npad(n)) {
         case 32: return launch_fwd<1, 32, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
         case 64: return launch_fwd<2, 32, 256, In>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec, sel, st);
@@ -663,9 +945,9 @@ int onchip_npad(int64_t n) {
 
 cudaError_t launch_onchip_forward(const float* r, int64_t ld, float* p, double* b, double* sumf,
                                   int64_t B, int n, double k, const double* k_rows, double t,
-                                  WsHeader* hdr, int vec, cudaStream_t st) {
+                                  WsHeader* hdr, int vec, int search, cudaStream_t st) {
     return onchip_forward_any<float>(r, ld, p, b, sumf, B, n, k, k_rows, t, hdr, vec,
-                                     SelectOut{nullptr, nullptr, nullptr, 0, 0.f}, st);
+                                     SelectOut{nullptr, nullptr, nullptr, 0, 0.f}, search, st);
 }
 
 cudaError_t launch_onchip_backward(const float* r, int64_t ld, const double* b, const float* v,
@@ -692,16 +974,16 @@ cudaError_t launch_onchip_hard(const float* r, int64_t ld, float* p, double* b, 
 cudaError_t launch_onchip_router(const void* r, int dtype, int64_t ld, float* p, double* b,
                                  double* sumf, int64_t B, int n, double k, double t, WsHeader* hdr,
                                  int vec, int32_t* sel_idx, float* sel_val, int32_t* sel_cnt,
-                                 int cap, float eps, cudaStream_t st) {
+                                 int cap, float eps, int search, cudaStream_t st) {
     const SelectOut sel{sel_idx, sel_val, sel_cnt, cap, eps};
     if (dtype == LAPSUM_DTYPE_BF16)
         return onchip_forward_any<uint16_t>(static_cast<const uint16_t*>(r), ld, p, b, sumf, B,
-                                            n, k, nullptr, t, hdr, vec, sel, st);
+                                            n, k, nullptr, t, hdr, vec, sel, search, st);
     if (dtype == LAPSUM_DTYPE_F16)
         return onchip_forward_any<F16Bits>(static_cast<const F16Bits*>(r), ld, p, b, sumf, B, n,
-                                           k, nullptr, t, hdr, vec, sel, st);
+                                           k, nullptr, t, hdr, vec, sel, search, st);
     return onchip_forward_any<float>(static_cast<const float*>(r), ld, p, b, sumf, B, n, k,
-                                     nullptr, t, hdr, vec, sel, st);
+                                     nullptr, t, hdr, vec, sel, search, st);
 }
 
 cudaError_t launch_onchip_backward_router(const void* r, int dtype, int64_t ld, const double* b,

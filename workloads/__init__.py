@@ -39,7 +39,7 @@ class Workload:
     k: float
     t: float
     dist: str
-    path: str  # solver the workload is meant to exercise: "bitonic", "radix", "bracket"
+    path: str  # solver family the workload exercises: "onchip" (n <= 4096), "radix", "bracket"
     desc: str
 
     @property
@@ -49,10 +49,10 @@ class Workload:
 
 WORKLOADS = {
     "single_row_n1024": Workload(
-        "single_row_n1024", 1, 1024, 10.0, 0.1, "normal", "bitonic",
+        "single_row_n1024", 1, 1024, 10.0, 0.1, "normal", "onchip",
         "single row n=1024, k=10, t=0.1, r ~ N(0,1)"),
     "moe_router_16384x256": Workload(
-        "moe_router_16384x256", 16384, 256, 8.0, 0.05, "normal", "bitonic",
+        "moe_router_16384x256", 16384, 256, 8.0, 0.05, "normal", "onchip",
         "MoE-routing batch 16384 rows x 256, k=8, t=0.05, r ~ N(0,1)"),
     "memory_select_256x65536": Workload(
         "memory_select_256x65536", 256, 65536, 1024.0, 0.02, "normal_q64", "radix",
