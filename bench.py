@@ -268,6 +268,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--n-override", type=int, default=0,
                     help="profiling runs: shrink the workload's row length (k scaled to keep k/n)")
+    ap.add_argument("--path", default="auto", choices=["auto", "fullsort", "radix", "bracket", "rowbracket"],
+                    help="solver of the timed workload (default: the library's choice)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -484,7 +486,7 @@ def main():
                 "path_frac_of_peak": nbytes / (ms / 1e3) / 1e9 / peak_gbs}
 
     peak_gbs, peak_kind = load_peaks()
-    R = run_workload(w, r_h, v_h, args.steps, args.warmup)
+    R = run_workload(w, r_h, v_h, args.steps, args.warmup, path=args.path)
     sampler = ClockSampler(local)
     sampler.start()
     barrier()
@@ -666,7 +668,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "n": w.n, "k": w.k, "t": w.t,
-                       "distribution": w.dist, "solver": w.path,
+                       "distribution": w.dist,
+                       "solver": w.path if args.path == "auto" else args.path,
                        "l2": "flushed before each step" if R["flush"] else
                              "inputs larger than L2 (no flush)",
                        "parallelism": f"{world} independent instances (one per GPU)"},

@@ -95,7 +95,9 @@ Layout make_layout(int64_t B, int64_t n, int rpath) {
         L.keys0 = take((size_t)B * (size_t)n * sizeof(uint32_t));
         L.keys1 = take((size_t)B * (size_t)n * sizeof(uint32_t));
         L.seg_hist = take((size_t)B * 1024 * sizeof(uint32_t));
-        L.tile_hist = take((size_t)B * 256 * (size_t)rt * sizeof(uint32_t));
+        // per-tile digit histograms (legacy passes) or look-back words, plus
+        // the pass's tile counter (8 bytes) right after them
+        L.tile_hist = take((size_t)B * 256 * (size_t)rt * sizeof(uint32_t) + 256);
         L.plan = take((size_t)B * 8 * sizeof(int32_t));
     }
     if (rpath == LAPSUM_PATH_ROWBRACKET) {
@@ -860,7 +862,8 @@ int lapsum_read_status(void* ws, void* stream, int* device_status) {
     if (e == cudaSuccess) e = cudaMemsetAsync(&hdr->status, 0, sizeof(uint32_t), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return LAPSUM_ECUDA;
-    *device_status = (bits & kDevNonFinite) ? LAPSUM_ENONFINITE
+    *device_status = (bits & kDevWaitTimeout) ? LAPSUM_ECUDA
+                     : (bits & kDevNonFinite) ? LAPSUM_ENONFINITE
                      : (bits & kDevBadBudget) ? LAPSUM_EINVAL
                      : (bits & kDevBracketExhausted) ? LAPSUM_EBRACKET
                                                      : LAPSUM_OK;

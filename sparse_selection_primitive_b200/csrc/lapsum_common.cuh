@@ -21,6 +21,7 @@ enum : uint32_t {
     kDevNonFinite = 1u << 0,
     kDevBracketExhausted = 1u << 1,
     kDevBadBudget = 1u << 2,  // a per-row budget outside (0, n)
+    kDevWaitTimeout = 1u << 3,  // a bounded wait on another CTA ran out (results invalid)
 };
 
 constexpr int kMaxAttempts = 7;     // 1 + 3 widenings per side; the last rungs are open

@@ -71,21 +71,25 @@ __global__ void __launch_bounds__(kThreads) radix_prep_kernel(const float* __res
 
 // Per row: which digits are trivial, and which buffer holds the data before
 // each pass (plan[row][d], d = 0..4), plus the trivial mask in plan[row][5].
-__global__ void radix_plan_kernel(const uint32_t* __restrict__ seg_hist, int64_t B, int64_t n,
-                                  int32_t* __restrict__ plan) {
-    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (row >= B) return;
-    int par = 0, mask = 0;
-    for (int d = 0; d < 4; ++d) {
-        plan[row * 8 + d] = par;
-        uint32_t mx = 0;
-        for (int v = 0; v < 256; ++v) mx = max(mx, seg_hist[row * 1024 + d * 256 + v]);
-        const bool trivial = (int64_t)mx == n;
-        if (trivial) mask |= 1 << d;
-        else par ^= 1;
+// One CTA per row, one thread per digit value.
+__global__ void __launch_bounds__(256) radix_plan_kernel(const uint32_t* __restrict__ seg_hist,
+                                                         int64_t B, int64_t n,
+                                                         int32_t* __restrict__ plan) {
+    const int64_t row = blockIdx.x;
+    const uint32_t* h = seg_hist + row * 1024;
+    int mask = 0;
+#pragma unroll
+    for (int d = 0; d < 4; ++d)
+        if (__syncthreads_or((int64_t)h[d * 256 + threadIdx.x] == n)) mask |= 1 << d;
+    if (threadIdx.x == 0) {
+        int par = 0;
+        for (int d = 0; d < 4; ++d) {
+            plan[row * 8 + d] = par;
+            if (!(mask & (1 << d))) par ^= 1;
+        }
+        plan[row * 8 + 4] = par;
+        plan[row * 8 + 5] = mask;
     }
-    plan[row * 8 + 4] = par;
-    plan[row * 8 + 5] = mask;
 }
 
 __global__ void __launch_bounds__(kThreads) radix_upsweep_kernel(
@@ -173,7 +177,7 @@ __global__ void __launch_bounds__(256) radix_scan_wide_kernel(const uint32_t* __
     }
 }
 
-__global__ void __launch_bounds__(kThreads) radix_downsweep_kernel(
+__global__ void __launch_bounds__(kThreads, 4) radix_downsweep_kernel(
     uint32_t* __restrict__ k0, uint32_t* __restrict__ k1, int64_t n, int64_t tiles, int d,
     const int32_t* __restrict__ plan, const uint32_t* __restrict__ tile_hist) {
     __shared__ uint32_t wcnt[kWarps][256];
@@ -197,11 +201,17 @@ __global__ void __launch_bounds__(kThreads) radix_downsweep_kernel(
     // [w*512, (w+1)*512) of the tile, visited 32 at a time in index order.
     uint32_t key[kPerThread], lrank[kPerThread];
     const uint32_t lt = lanemask_lt();
+    // all loads first: the warp barriers of the ranking loop below would
+    // otherwise hold each load back until the previous key is ranked
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
+        key[e] = idx < n ? src[idx] : 0u;
+    }
 #pragma unroll
     for (int e = 0; e < kPerThread; ++e) {
         const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
         const bool ok = idx < n;
-        key[e] = ok ? src[idx] : 0u;
         const uint32_t dig = (key[e] >> shift) & 255u;
         const uint32_t peers = __match_any_sync(0xffffffffu, ok ? dig : 256u + lane);
         const int leader = __ffs(peers) - 1;
@@ -258,6 +268,141 @@ __global__ void __launch_bounds__(kThreads) radix_downsweep_kernel(
     }
 }
 
+// One digit pass in one kernel (for rows of fewer than 2^30 keys): each CTA
+// takes the next tile id from a counter, so every tile before it is already
+// running; it ranks its tile as the downsweep does, publishes its digit counts
+// (word = flag << 30 | count: 1 = the tile's own count, 2 = inclusive prefix
+// over the row's tiles so far) and walks back over its predecessors' words
+// until an inclusive one, which gives its scatter bases without an upsweep or
+// a scan.  Tile 0 publishes its inclusive counts at once, so every walk ends;
+// each wait is bounded and sets kDevWaitTimeout if it runs out.
+constexpr uint32_t kLbAgg = 1u << 30, kLbInc = 2u << 30, kLbMask = (1u << 30) - 1u;
+constexpr int kLbSpinMax = 1 << 22;
+
+__global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
+    uint32_t* __restrict__ k0, uint32_t* __restrict__ k1, int64_t n, int64_t tiles, int d,
+    const int32_t* __restrict__ plan, const uint32_t* __restrict__ seg_hist,
+    uint32_t* __restrict__ lb, unsigned long long* __restrict__ counter, WsHeader* hdr) {
+    __shared__ uint32_t wcnt[kWarps][256];
+    __shared__ uint32_t tstart[256];
+    __shared__ uint32_t gbase[256];
+    __shared__ uint32_t sorted[kRadixTile];
+    __shared__ unsigned long long s_id;
+    if (threadIdx.x == 0) s_id = atomicAdd(counter, 1ull);
+    __syncthreads();
+    const int64_t id = (int64_t)s_id;
+    const int64_t row = id / tiles, tile = id % tiles;
+    if (plan[row * 8 + 5] & (1 << d)) return;  // the whole row skips this digit
+    const int par = plan[row * 8 + d];
+    const uint32_t* src = (par ? k1 : k0) + row * n;
+    uint32_t* dst = (par ? k0 : k1) + row * n;
+    const int64_t base = tile * kRadixTile;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int shift = 8 * d;
+    const int v = threadIdx.x;
+
+    for (int i = threadIdx.x; i < kWarps * 256; i += kThreads) (&wcnt[0][0])[i] = 0;
+    // the row's digit bases: exclusive scan of its digit histogram
+    const uint32_t hc = seg_hist[row * 1024 + d * 256 + v];
+    tstart[v] = hc;
+    __syncthreads();
+    for (int off = 1; off < 256; off <<= 1) {
+        const uint32_t add = v >= off ? tstart[v - off] : 0u;
+        __syncthreads();
+        tstart[v] += add;
+        __syncthreads();
+    }
+    const uint32_t dbase = tstart[v] - hc;
+    __syncthreads();
+
+    uint32_t key[kPerThread], lrank[kPerThread];
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
+        key[e] = idx < n ? src[idx] : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
+        const bool ok = idx < n;
+        const uint32_t dig = (key[e] >> shift) & 255u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, ok ? dig : 256u + lane);
+        const int leader = __ffs(peers) - 1;
+        uint32_t bse = 0;
+        if (ok && lane == leader) {
+            bse = wcnt[warp][dig];
+            wcnt[warp][dig] = bse + __popc(peers);
+        }
+        bse = __shfl_sync(0xffffffffu, bse, leader);
+        lrank[e] = bse + __popc(peers & lt);
+        __syncwarp();
+    }
+    __syncthreads();
+    uint32_t cnt = 0;  // this tile's count of digit v
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t c = wcnt[w][v];
+        wcnt[w][v] = cnt;
+        cnt += c;
+    }
+    // publish, then walk back to the first inclusive word
+    volatile uint32_t* words = lb + row * tiles * 256;
+    words[tile * 256 + v] = (tile == 0 ? kLbInc : kLbAgg) | cnt;
+    uint32_t excl = 0;
+    bool timed_out = false;
+    if (tile > 0) {
+        int64_t j = tile - 1;
+        int spins = 0;
+        for (;;) {
+            const uint32_t w = words[j * 256 + v];
+            if ((w & ~kLbMask) == 0u) {
+                if (++spins > kLbSpinMax) {
+                    timed_out = true;
+                    break;
+                }
+                continue;
+            }
+            excl += w & kLbMask;
+            if ((w & ~kLbMask) == kLbInc || j == 0) break;
+            --j;
+        }
+        if (!timed_out) words[tile * 256 + v] = kLbInc | (excl + cnt);
+    }
+    if (__syncthreads_or(timed_out)) {  // the bases are unknown: write nothing
+        if (threadIdx.x == 0) set_status(hdr, kDevWaitTimeout);
+        return;
+    }
+    gbase[v] = dbase + excl;
+    tstart[v] = cnt;
+    __syncthreads();
+    // exclusive scan of the tile's digit counts -> local start of each digit
+    for (int off = 1; off < 256; off <<= 1) {
+        const uint32_t add = v >= off ? tstart[v - off] : 0u;
+        __syncthreads();
+        tstart[v] += add;
+        __syncthreads();
+    }
+    tstart[v] -= cnt;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
+        if (idx < n) {
+            const uint32_t dig = (key[e] >> shift) & 255u;
+            sorted[tstart[dig] + wcnt[warp][dig] + lrank[e]] = key[e];
+        }
+    }
+    __syncthreads();
+    const int valid = (int)min((int64_t)kRadixTile, n - base);
+    for (int i = threadIdx.x; i < valid; i += kThreads) {
+        const uint32_t kv = sorted[i];
+        const uint32_t dig = (kv >> shift) & 255u;
+        const uint32_t pos = gbase[dig] + (uint32_t)i - tstart[dig];
+        if ((int64_t)pos < n) dst[pos] = kv;
+    }
+}
+
 struct KeyGet {
     const uint32_t* k;
     __device__ __forceinline__ float operator()(long long j) const { return from_key(k[j]); }
@@ -279,7 +424,8 @@ __global__ void __launch_bounds__(1024) rowsolve_keys_kernel(const uint32_t* __r
     // the row's budget: the shared k or its own entry of k_rows (outside (0, n): b = NaN)
     const double kr = k_rows != nullptr ? k_rows[row] : k;
     const bool k_ok = kr > 0.0 && kr < (double)n;
-    solve_sorted_block(KeyGet{keys}, (long long)n, tl, k_ok ? kr : 0.5 * (double)n, t, &sm, &res);
+    solve_sorted_block<KeyGet, false, true>(KeyGet{keys}, (long long)n, tl,
+                                             k_ok ? kr : 0.5 * (double)n, t, &sm, &res);
     if (threadIdx.x == 0) {
         if (!k_ok) {
             rows[row].status |= kDevBadBudget;
@@ -424,7 +570,22 @@ cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_
     }
     {
         ProfScope ps_("radix_plan", st);
-        radix_plan_kernel<<<(unsigned)((B + 127) / 128), 128, 0, st>>>(buf.seg_hist, B, n, buf.plan);
+        radix_plan_kernel<<<(unsigned)B, 256, 0, st>>>(buf.seg_hist, B, n, buf.plan);
+    }
+    if (n < (int64_t)kLbMask) {
+        // one kernel per digit pass: look-back words instead of upsweep + scan
+        const size_t words = (size_t)B * 256 * (size_t)tiles * sizeof(uint32_t);
+        unsigned long long* counter =
+            reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(buf.tile_hist) + words);
+        for (int d = 0; d < 4; ++d) {
+            e = cudaMemsetAsync(buf.tile_hist, 0, words + sizeof(unsigned long long), st);
+            if (e != cudaSuccess) return e;
+            ProfScope ps_("radix_onesweep", st);
+            radix_onesweep_kernel<<<(unsigned)(tiles * B), kThreads, 0, st>>>(
+                buf.keys[0], buf.keys[1], n, tiles, d, buf.plan, buf.seg_hist, buf.tile_hist, counter,
+                hdr);
+        }
+        return cudaGetLastError();
     }
     for (int d = 0; d < 4; ++d) {
         {

@@ -44,25 +44,32 @@ struct SolveScratch {
     long long ll[4];
 };
 
-template <class Get>
+// HOT: a long array (a whole sorted row): factors are taken with the inlined
+// exponential, and each thread's chunk is summarised in closed form (see
+// solve_sorted_block); otherwise one out-of-line copy of the exponential
+// serves the single-CTA band solves.
+template <class Get, bool HOT = false>
 struct GapFn {
     Get get;
     long long nb;
     Tails tl;
     double inv_t;
+    __device__ __forceinline__ double factor(float lo, float hi) const {
+        return HOT ? gap_factor(lo, hi, inv_t) : gap_factor_cold(lo, hi, inv_t);
+    }
     // factor between positions j-1 and j (anchors at -1 and nb)
     __device__ __forceinline__ double operator()(long long j) const {
-        if (j <= 0) return (j == 0 && tl.hasL && nb > 0) ? gap_factor_cold(tl.aL, get(0), inv_t) : 0.0;
-        if (j >= nb) return (j == nb && tl.hasR) ? gap_factor_cold(get(nb - 1), tl.aR, inv_t) : 0.0;
-        return gap_factor_cold(get(j - 1), get(j), inv_t);
+        if (j <= 0) return (j == 0 && tl.hasL && nb > 0) ? factor(tl.aL, get(0)) : 0.0;
+        if (j >= nb) return (j == nb && tl.hasR) ? factor(get(nb - 1), tl.aR) : 0.0;
+        return factor(get(j - 1), get(j));
     }
 };
 
 // One warp narrows [lo, hi) -- whose first element satisfies F >= k -- to the
 // last element with F >= k.  P_before = P_{lo-1}, Q_after = Q_hi.  Lane 0
 // returns j* and the anchor weights through the out-parameters.
-template <class Get>
-__device__ void warp_find_crossing(const GapFn<Get>& gap, long long lo, long long hi,
+template <class Get, bool HOT>
+__device__ void warp_find_crossing(const GapFn<Get, HOT>& gap, long long lo, long long hi,
                                    double P_before, double Q_after, double k, long long* jstar,
                                    double* P_left, double* Q_right) {
     const int lane = threadIdx.x & 31;
@@ -136,13 +143,13 @@ __device__ __forceinline__ int team_count(bool pred) {
 // the one calling warp) must call it; the result is valid in `out` for every
 // thread of the team after return.  The warp form serves small bands without
 // any block barrier.
-template <class Get, bool WARP = false>
+template <class Get, bool WARP = false, bool HOT = false>
 __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, double k, double t,
                                    SolveScratch* sm, SolveResult* out) {
     const int tid = WARP ? (int)(threadIdx.x & 31) : (int)threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int nthreads = WARP ? 32 : (int)blockDim.x, nwarps = nthreads >> 5;
-    GapFn<Get> gap{get, nb, tl, 1.0 / t};
+    GapFn<Get, HOT> gap{get, nb, tl, 1.0 / t};
     const double P_start = tl.hasL ? tl.SL : 0.0;
     const double Q_end = tl.hasR ? tl.SR : 0.0;
 
@@ -170,13 +177,45 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
     const bool valid = lo < hi;
     Aff af = aff_id(), ab = aff_id();
     double g_first = 0.0;
-    for (long long j = lo; j < hi; ++j) {
-        const double gj = gap(j);
-        if (j == lo) g_first = gj;
-        af = aff_then(af, Aff{gj, 1.0});
-        if (j > lo) ab = aff_then(Aff{gj, 1.0}, ab);
+    if constexpr (HOT) {
+        // A long chunk's maps in closed form: the product of its gap factors
+        // telescopes, P_{hi-1} = gap(lo) e^{(s_lo - s_{hi-1})/t} P_{lo-1}
+        // + sum_{i in chunk} e^{(s_i - s_{hi-1})/t}, and likewise Q_lo from
+        // Q_hi; the sums take fp32 exponentials (every term at most 1) added
+        // in fp64, so three fp64 exponentials serve the whole chunk and no
+        // rounding compounds along it.
+        if (valid) {
+            const float s_first = get(lo), s_last = get(hi - 1);
+            const float sc = (float)(1.0 / t) * kLog2e;
+            double cf = 0.0, cb = 0.0;
+            for (long long j0 = lo; j0 < hi; j0 += 8) {
+                float cf8 = 0.f, cb8 = 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const long long j = j0 + u;
+                    if (j < hi) {
+                        const float x = get(j);
+                        cf8 += ex2_ftz((x - s_last) * sc);
+                        cb8 += ex2_ftz((s_first - x) * sc);
+                    }
+                }
+                cf += (double)cf8;
+                cb += (double)cb8;
+            }
+            const double span = exp(((double)s_first - (double)s_last) / t);
+            g_first = gap(lo);
+            af = Aff{g_first * span, cf};
+            ab = Aff{gap(hi) * span, cb};
+        }
+    } else {
+        for (long long j = lo; j < hi; ++j) {
+            const double gj = gap(j);
+            if (j == lo) g_first = gj;
+            af = aff_then(af, Aff{gj, 1.0});
+            if (j > lo) ab = aff_then(Aff{gj, 1.0}, ab);
+        }
+        if (valid) ab = aff_then(Aff{gap(hi), 1.0}, ab);
     }
-    if (valid) ab = aff_then(Aff{gap(hi), 1.0}, ab);
 
     const Aff inc_f = warp_scan_fwd(af, lane);
     const Aff inc_b = warp_scan_bwd(ab, lane);
