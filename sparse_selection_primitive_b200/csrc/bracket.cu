@@ -882,8 +882,8 @@ __device__ void certify_big_band(const float* band, long long nb, const Tails& t
     const double inv_t = 1.0 / t;
     for (long long j = threadIdx.x; j < nb; j += blockDim.x) {
         const float s = band[j];
-        if (tl.hasL) wl += (double)__expf((float)((tl.aL - s) * inv_t));
-        if (tl.hasR) vr += (double)__expf((float)((s - tl.aR) * inv_t));
+        if (tl.hasL) wl += (double)exp_neg((float)((s - tl.aL) * inv_t));
+        if (tl.hasR) vr += (double)exp_neg((float)((tl.aR - s) * inv_t));
         const uint32_t kk = to_key(s);
         lo = min(lo, kk);
         hi = max(hi, kk);
@@ -929,6 +929,7 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
                                   uint32_t kmin, uint32_t kmax, double k, double t,
                                   SolveSmemAll* sm, uint32_t* nkmin, uint32_t* nkmax) {
     const float inv_t = (float)(1.0 / t);
+    const double inv_td = 1.0 / t;  // the exact checks' arguments, in fp64
     const uint32_t range = kmax - kmin;
     int sh = 0;
     while ((range >> sh) >= (uint32_t)kRefineBins) ++sh;
@@ -1009,13 +1010,13 @@ __device__ long long refine_level(const float* in, long long nb, float* out, Tai
             bool take = false;
             if (hasHi && s >= Ehi) {
                 cr += 1;
-                sr += (double)__expf((Ehi - s) * inv_t);
+                sr += (double)exp_neg((float)(((double)s - (double)Ehi) * inv_td));
             } else if (hasLo && s < Elo) {
-                sl += (double)__expf((s - Elo) * inv_t);
+                sl += (double)exp_neg((float)(((double)Elo - (double)s) * inv_td));
             } else {
                 take = true;
-                if (hasLo) w += (double)__expf((Elo - s) * inv_t);
-                if (hasHi) v += (double)__expf((s - Ehi) * inv_t);
+                if (hasLo) w += (double)exp_neg((float)(((double)s - (double)Elo) * inv_td));
+                if (hasHi) v += (double)exp_neg((float)(((double)Ehi - (double)s) * inv_td));
                 const uint32_t kk = to_key(s);
                 lo = min(lo, kk);
                 hi = max(hi, kk);

@@ -101,17 +101,43 @@ __device__ __forceinline__ bool finite_f(float x) { return fabsf(x) <= 3.4028234
 // ---------------------------------------------------------------------------
 struct Thr {
     float hi, lo, inv_t;
+    float inv_lo;  // 1/t - inv_t
 };
 __device__ __forceinline__ Thr make_thr(double b, double t) {
     Thr h;
     h.hi = (float)b;
     h.lo = (float)(b - (double)h.hi);
     h.inv_t = (float)(1.0 / t);
+    h.inv_lo = (float)(1.0 / t - (double)h.inv_t);
     return h;
 }
 __device__ __forceinline__ float scaled_margin(float r, const Thr& h) {
     return __fmul_rn(__fsub_rn(__fsub_rn(r, h.hi), h.lo), h.inv_t);
 }
+// The same margin without a rounding error common to many scores: the
+// rounding of r - hi discards the bits of hi below the ulp of r - hi, the same
+// for every score of a binade, and 1/t's rounding is shared by all, so summed
+// over many p both bias the budget.  r - hi is taken exactly by Knuth's
+// two-sum and 1/t as a two-float pair.  Scores within a factor of two of hi
+// (every score that carries weight when t is small against |b|) give the same
+// result through scaled_margin, since r - hi is then exact (Sterbenz).
+__device__ __forceinline__ float scaled_margin_exact(float r, const Thr& h) {
+    const float s = __fsub_rn(r, h.hi);
+    const float rv = __fadd_rn(s, h.hi);  // r as recovered from s
+    const float hv = __fsub_rn(s, rv);    // -hi as recovered from s
+    const float err = __fadd_rn(__fsub_rn(r, rv), __fsub_rn(-h.hi, hv));
+    const float d = __fadd_rn(s, __fsub_rn(err, h.lo));
+    return fmaf(d, h.inv_t, __fmul_rn(d, h.inv_lo));
+}
+// The fast margin with 1/t as a two-float pair (its rounding is common to all
+// scores of a row).
+__device__ __forceinline__ float scaled_margin_it(float r, const Thr& h) {
+    const float d = __fsub_rn(__fsub_rn(r, h.hi), h.lo);
+    return fmaf(d, h.inv_t, __fmul_rn(d, h.inv_lo));
+}
+// Rows where some weighted score can lie outside [b/2, 2b]: t not small
+// against |b| (40 t covers |x| <= 20, below which e^{-|x|} < 2.1e-9).
+__device__ __forceinline__ bool soft_row(double b, double t) { return 40.0 * t >= fabs(b); }
 
 // 2^y with flush-to-zero for results below the smallest normal float (the
 // hardware ex2 approximation; about 2 ulp).  Flushing is harmless here: every
@@ -123,6 +149,32 @@ __device__ __forceinline__ float ex2_ftz(float y) {
     return r;
 }
 constexpr float kLog2e = 1.4426950408889634f;
+
+// e^{-a} for a >= 0 without the hardware approximation's bias: Cody and
+// Waite's reduction a = j ln2 + r, |r| <= ln2/2 (ln2 split into a head whose
+// product with any j < 512 is exact and a small tail), the Taylor polynomial
+// of e^{-r} to degree 7 (truncation below 6e-9 relative) by Horner's rule
+// with fused multiply-adds, and 2^{-j} from the exponent field.  About one ulp
+// with rounding errors of both signs, so that sums of many p stay on budget;
+// results below the smallest normal float are flushed to 0.
+__device__ __forceinline__ float exp_neg(float a) {
+    const float j = rintf(a * 1.44269504f);
+    if (j > 126.f) return 0.f;
+    float r = fmaf(-j, 0.693145751953125f, a);
+    r = fmaf(-j, 1.428606765330187e-6f, r);
+    const float s = -r;
+    float q = 1.0f / 5040.0f;
+    q = fmaf(q, s, 1.0f / 720.0f);
+    q = fmaf(q, s, 1.0f / 120.0f);
+    q = fmaf(q, s, 1.0f / 24.0f);
+    q = fmaf(q, s, 1.0f / 6.0f);
+    q = fmaf(q, s, 0.5f);
+    q = fmaf(q, s, 1.0f);
+    q = fmaf(q, s, 1.0f);
+    const float scale = __int_as_float((127 - (int)j) << 23);
+    const float e = q * scale;
+    return e >= 1.17549435e-38f ? e : 0.f;
+}
 
 // e = exp(-|x|); p = sigma(x) = x < 0 ? e/2 : 1 - e/2; f = e/2.  One exp.
 __device__ __forceinline__ float neg_abs_exp(float x) { return ex2_ftz(-fabsf(x) * kLog2e); }

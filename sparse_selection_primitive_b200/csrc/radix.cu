@@ -47,13 +47,22 @@ __global__ void __launch_bounds__(kThreads) radix_prep_kernel(const float* __res
     bool bad = false;
     const float* rr = r + row * ld;
     uint32_t* kk = keys + row * n;
-    for (int i = threadIdx.x; i < kRadixTile; i += kThreads) {
-        const int64_t idx = base + i;
-        if (idx < n) {
-            const float x = __ldg(rr + idx);
-            bad |= !finite_f(x);
-            const uint32_t key = to_key(x);
+    float xs[kPerThread];
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + e * kThreads + threadIdx.x;
+        xs[e] = idx < n ? __ldg(rr + idx) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e) {
+        const int64_t idx = base + e * kThreads + threadIdx.x;
+        const bool ok = idx < n;
+        const uint32_t key = to_key(xs[e]);
+        if (ok) {
+            bad |= !finite_f(xs[e]);
             kk[idx] = key;
+        }
+        if (ok) {
 #pragma unroll
             for (int d = 0; d < 4; ++d) atomicAdd(&h[d][(key >> (8 * d)) & 255u], 1u);
         }
@@ -279,6 +288,25 @@ __global__ void __launch_bounds__(kThreads, 4) radix_downsweep_kernel(
 constexpr uint32_t kLbAgg = 1u << 30, kLbInc = 2u << 30, kLbMask = (1u << 30) - 1u;
 constexpr int kLbSpinMax = 1 << 22;
 
+// Exclusive scan of one count per thread of a 256-thread block, in thread
+// order: warp shuffles, then the warps' totals through `wsum` (8 words).
+// Every thread calls it; `wsum` must not be reused before a block barrier.
+__device__ __forceinline__ uint32_t block256_excl_scan(uint32_t x, uint32_t* wsum) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t inc = x;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc += o;
+    }
+    if (lane == 31) wsum[w] = inc;
+    __syncthreads();
+    uint32_t pre = 0;
+#pragma unroll
+    for (int i = 0; i < kWarps; ++i) pre += i < w ? wsum[i] : 0u;
+    return pre + inc - x;
+}
+
 __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
     uint32_t* __restrict__ k0, uint32_t* __restrict__ k1, int64_t n, int64_t tiles, int d,
     const int32_t* __restrict__ plan, const uint32_t* __restrict__ seg_hist,
@@ -287,11 +315,15 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
     __shared__ uint32_t tstart[256];
     __shared__ uint32_t gbase[256];
     __shared__ uint32_t sorted[kRadixTile];
+    __shared__ uint32_t wsum[2][kWarps];
     __shared__ unsigned long long s_id;
     if (threadIdx.x == 0) s_id = atomicAdd(counter, 1ull);
     __syncthreads();
+    // ids run tile-major over the rows, so a tile's predecessor in its row
+    // started B ids earlier and has usually published its inclusive counts
     const int64_t id = (int64_t)s_id;
-    const int64_t row = id / tiles, tile = id % tiles;
+    const int64_t B = (int64_t)gridDim.x / tiles;
+    const int64_t tile = id / B, row = id % B;
     if (plan[row * 8 + 5] & (1 << d)) return;  // the whole row skips this digit
     const int par = plan[row * 8 + d];
     const uint32_t* src = (par ? k1 : k0) + row * n;
@@ -303,17 +335,7 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
 
     for (int i = threadIdx.x; i < kWarps * 256; i += kThreads) (&wcnt[0][0])[i] = 0;
     // the row's digit bases: exclusive scan of its digit histogram
-    const uint32_t hc = seg_hist[row * 1024 + d * 256 + v];
-    tstart[v] = hc;
-    __syncthreads();
-    for (int off = 1; off < 256; off <<= 1) {
-        const uint32_t add = v >= off ? tstart[v - off] : 0u;
-        __syncthreads();
-        tstart[v] += add;
-        __syncthreads();
-    }
-    const uint32_t dbase = tstart[v] - hc;
-    __syncthreads();
+    const uint32_t dbase = block256_excl_scan(seg_hist[row * 1024 + d * 256 + v], wsum[0]);
 
     uint32_t key[kPerThread], lrank[kPerThread];
     const uint32_t lt = lanemask_lt();
@@ -352,20 +374,30 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
     uint32_t excl = 0;
     bool timed_out = false;
     if (tile > 0) {
+        // read four predecessors per round trip, nearest first; stop at the
+        // first inclusive word, re-read from the first one not yet published
         int64_t j = tile - 1;
         int spins = 0;
-        for (;;) {
-            const uint32_t w = words[j * 256 + v];
-            if ((w & ~kLbMask) == 0u) {
-                if (++spins > kLbSpinMax) {
-                    timed_out = true;
-                    break;
-                }
-                continue;
+        bool done = false;
+        while (!done) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) w[q] = j - q >= 0 ? (uint32_t)words[(j - q) * 256 + v] : (uint32_t)kLbInc;
+            int adv = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (done || adv < q) continue;
+                const uint32_t f = w[q] & ~kLbMask;
+                if (f == 0u) continue;  // not published yet
+                excl += w[q] & kLbMask;
+                ++adv;
+                if (f == kLbInc) done = true;
             }
-            excl += w & kLbMask;
-            if ((w & ~kLbMask) == kLbInc || j == 0) break;
-            --j;
+            j -= adv;
+            if (!done && adv == 0 && ++spins > kLbSpinMax) {
+                timed_out = true;
+                break;
+            }
         }
         if (!timed_out) words[tile * 256 + v] = kLbInc | (excl + cnt);
     }
@@ -374,16 +406,8 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
         return;
     }
     gbase[v] = dbase + excl;
-    tstart[v] = cnt;
-    __syncthreads();
     // exclusive scan of the tile's digit counts -> local start of each digit
-    for (int off = 1; off < 256; off <<= 1) {
-        const uint32_t add = v >= off ? tstart[v - off] : 0u;
-        __syncthreads();
-        tstart[v] += add;
-        __syncthreads();
-    }
-    tstart[v] -= cnt;
+    tstart[v] = block256_excl_scan(cnt, wsum[1]);
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < kPerThread; ++e) {
@@ -408,7 +432,7 @@ struct KeyGet {
     __device__ __forceinline__ float operator()(long long j) const { return from_key(k[j]); }
 };
 
-__global__ void __launch_bounds__(1024) rowsolve_keys_kernel(const uint32_t* __restrict__ k0,
+__global__ void __launch_bounds__(512, 2) rowsolve_keys_kernel(const uint32_t* __restrict__ k0,
                                                               const uint32_t* __restrict__ k1,
                                                               int64_t n, double k,
                                                               const double* __restrict__ k_rows,
@@ -426,6 +450,158 @@ __global__ void __launch_bounds__(1024) rowsolve_keys_kernel(const uint32_t* __r
     const bool k_ok = kr > 0.0 && kr < (double)n;
     solve_sorted_block<KeyGet, false, true>(KeyGet{keys}, (long long)n, tl,
                                              k_ok ? kr : 0.5 * (double)n, t, &sm, &res);
+    if (threadIdx.x == 0) {
+        if (!k_ok) {
+            rows[row].status |= kDevBadBudget;
+            set_status(hdr, kDevBadBudget);
+        }
+        const double b = ((rows[row].status & kDevNonFinite) || !k_ok) ? nan("") : res.b;
+        rows[row].b = b;
+        rows[row].path = LAPSUM_PATH_RADIX;
+        rows[row].attempts = 1;
+        b_out[row] = b;
+    }
+}
+
+// Long sorted rows: the same solve over the whole GPU.  The row is cut into G
+// chunks; one CTA per chunk writes the chunk's prefix and suffix maps in
+// closed form (the product of its gap factors telescopes to gap(lo)
+// e^{(s_lo - s_{hi-1})/t}, and the sums take fp32 exponentials of terms at
+// most 1, added in fp64), and one CTA per row composes the G maps in chunk
+// order, takes the chunk where F crosses k, and solves that chunk with
+// everything before and after it folded into two anchors.
+constexpr int64_t kSolveChunkMin = 65536;
+constexpr int kSolveRecMax = 8192;  // chunks per row
+
+struct ChunkRec {
+    double fa, fc;  // P_{hi-1} = fa P_{lo-1} + fc
+    double ba, bc;  // Q_lo = ba Q_hi + bc
+    double g_lo;    // gap factor between positions lo-1 and lo (0 at the row's start)
+    double pad[3];
+};
+
+__global__ void __launch_bounds__(256) rowsolve_chunk_kernel(const uint32_t* __restrict__ k0,
+                                                              const uint32_t* __restrict__ k1,
+                                                              int64_t n, int64_t chunk, double t,
+                                                              const int32_t* __restrict__ plan,
+                                                              ChunkRec* __restrict__ rec) {
+    __shared__ double red[2][8];
+    const int64_t row = blockIdx.y, c = blockIdx.x;
+    const uint32_t* keys = (plan[row * 8 + 4] ? k1 : k0) + row * n;
+    const int64_t lo = c * chunk, hi = min(n, lo + chunk);
+    const float s_first = from_key(keys[lo]), s_last = from_key(keys[hi - 1]);
+    const float it = (float)(1.0 / t);  // 1/t as a two-float pair
+    const float it_lo = (float)(1.0 / t - (double)it);
+    float cf = 0.f, cb = 0.f;
+    double df = 0.0, db = 0.0;
+    int cnt = 0;
+    for (int64_t j = lo + threadIdx.x; j < hi; j += 256) {
+        const float x = from_key(__ldcs(keys + j));
+        cf += exp_neg(fmaf(s_last - x, it, (s_last - x) * it_lo));
+        cb += exp_neg(fmaf(x - s_first, it, (x - s_first) * it_lo));
+        if (++cnt == 16) {  // fp32 partial sums of 16 terms (each at most 1), then fp64
+            df += (double)cf;
+            db += (double)cb;
+            cf = cb = 0.f;
+            cnt = 0;
+        }
+    }
+    df += (double)cf;
+    db += (double)cb;
+    df = warp_sum_d(df);
+    db = warp_sum_d(db);
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    if (lane == 0) {
+        red[0][w] = df;
+        red[1][w] = db;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double sf = 0.0, sb = 0.0;
+        for (int i = 0; i < 8; ++i) {
+            sf += red[0][i];
+            sb += red[1][i];
+        }
+        const double inv_t = 1.0 / t;
+        const double span = exp(((double)s_first - (double)s_last) * inv_t);
+        const double g_lo = lo > 0 ? gap_factor(from_key(keys[lo - 1]), s_first, inv_t) : 0.0;
+        const double g_hi = hi < n ? gap_factor(s_last, from_key(keys[hi]), inv_t) : 0.0;
+        ChunkRec r;
+        r.fa = g_lo * span;
+        r.fc = sf;
+        r.ba = g_hi * span;
+        r.bc = sb;
+        r.g_lo = g_lo;
+        r.pad[0] = r.pad[1] = r.pad[2] = 0.0;
+        rec[row * gridDim.x + c] = r;
+    }
+}
+
+__global__ void __launch_bounds__(1024) rowsolve_combine_kernel(
+    const uint32_t* __restrict__ k0, const uint32_t* __restrict__ k1, int64_t n, int64_t chunk,
+    int G, double k, const double* __restrict__ k_rows, double t, const int32_t* __restrict__ plan,
+    const ChunkRec* __restrict__ recs, double* __restrict__ b_out, RowState* rows, WsHeader* hdr) {
+    __shared__ SolveScratch sm;
+    __shared__ SolveResult res;
+    __shared__ Aff wt[32];
+    __shared__ double sP, sQ;
+    __shared__ int wc[32];
+    const int64_t row = blockIdx.x;
+    const uint32_t* keys = (plan[row * 8 + 4] ? k1 : k0) + row * n;
+    const ChunkRec* rec = recs + row * G;
+    const double kr = k_rows != nullptr ? k_rows[row] : k;
+    const bool k_ok = kr > 0.0 && kr < (double)n;
+    const double kk = k_ok ? kr : 0.5 * (double)n;
+    // each thread composes a run of consecutive chunks
+    const int per = (G + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int c0 = min(G, (int)threadIdx.x * per), c1 = min(G, c0 + per);
+    Aff af = aff_id(), ab = aff_id();
+    for (int c = c0; c < c1; ++c) af = aff_then(af, Aff{rec[c].fa, rec[c].fc});
+    for (int c = c1 - 1; c >= c0; --c) ab = aff_then(Aff{rec[c].ba, rec[c].bc}, ab);
+    const Aff ef = block_excl_scan_fwd(af, wt);  // chunks before this run
+    const Aff eb = block_excl_scan_bwd(ab, wt);  // chunks after this run
+    // F at each chunk's first score: P_lo = 1 + g_lo P_{lo-1}, Q_lo = ba Q_hi + bc
+    double P = ef.c;   // P_{lo-1} of chunk c0 (P before the row is 0)
+    double Qs[kSolveRecMax / 1024];
+    double Q = eb.c;   // Q_hi of chunk c1 - 1 (Q after the row is 0)
+    for (int c = c1 - 1; c >= c0; --c) {
+        Q = fma(rec[c].ba, Q, rec[c].bc);
+        Qs[c - c0] = Q;  // Q_lo of chunk c
+    }
+    int cnt = 0;
+    for (int c = c0; c < c1; ++c) {
+        const double P_lo = fma(rec[c].g_lo, P, 1.0);
+        const double G_lo = (double)(n - (int64_t)c * chunk) - 0.5 * Qs[c - c0] + 0.5 * (P_lo - 1.0);
+        cnt += G_lo >= kk ? 1 : 0;
+        P = fma(rec[c].fa, P, rec[c].fc);  // P_{hi-1}
+    }
+    // the number of chunks with F(first score) >= k (F decreases along the row)
+    int total = warp_sum_i(cnt);
+    if ((threadIdx.x & 31) == 0) wc[threadIdx.x >> 5] = total;
+    __syncthreads();
+    total = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) total += wc[i];
+    const int T = total > 0 ? total - 1 : 0;
+    // anchors of chunk T: P_{lo_T - 1} and Q_{hi_T}, from the thread that owns T
+    if (T >= c0 && T < c1) {
+        double Pb = ef.c;
+        for (int c = c0; c < T; ++c) Pb = fma(rec[c].fa, Pb, rec[c].fc);
+        double Qa = eb.c;
+        for (int c = c1 - 1; c > T; --c) Qa = fma(rec[c].ba, Qa, rec[c].bc);
+        sP = Pb;
+        sQ = Qa;
+    }
+    __syncthreads();
+    const int64_t lo = (int64_t)T * chunk, hi = min(n, lo + chunk);
+    Tails tl;
+    tl.hasL = lo > 0;
+    tl.aL = lo > 0 ? from_key(keys[lo - 1]) : 0.f;
+    tl.SL = lo > 0 ? sP : 0.0;
+    tl.hasR = hi < n;
+    tl.aR = hi < n ? from_key(keys[hi]) : 0.f;
+    tl.SR = hi < n ? sQ : 0.0;
+    tl.cntR = (double)(n - hi);
+    solve_sorted_block<KeyGet, false, true>(KeyGet{keys + lo}, hi - lo, tl, kk, t, &sm, &res);
     if (threadIdx.x == 0) {
         if (!k_ok) {
             rows[row].status |= kDevBadBudget;
@@ -617,9 +793,30 @@ cudaError_t launch_radix_sort_rows(const float* r, int64_t ld, int64_t B, int64_
 cudaError_t launch_rowsolve_sorted_keys(const RadixBuffers& buf, int64_t B, int64_t n, double k,
                                         const double* k_rows, double t, double* b, RowState* rows,
                                         WsHeader* hdr, cudaStream_t st) {
+    if (n > 4 * kSolveChunkMin) {
+        // chunks of at least 65536 keys (a multiple of 4096), at most 8192 per row;
+        // the records take the look-back words' space, free once the sort is done
+        int64_t chunk = (n + kSolveRecMax - 1) / kSolveRecMax;
+        chunk = ((chunk + 4095) / 4096) * 4096;
+        if (chunk < kSolveChunkMin) chunk = kSolveChunkMin;
+        const int G = (int)((n + chunk - 1) / chunk);
+        ChunkRec* rec = reinterpret_cast<ChunkRec*>(buf.tile_hist);
+        {
+            ProfScope ps_("rowsolve_chunks", st);
+            rowsolve_chunk_kernel<<<dim3((unsigned)G, (unsigned)B), 256, 0, st>>>(
+                buf.keys[0], buf.keys[1], n, chunk, t, buf.plan, rec);
+        }
+        {
+            ProfScope ps_("rowsolve", st);
+            rowsolve_combine_kernel<<<(unsigned)B, 1024, 0, st>>>(buf.keys[0], buf.keys[1], n, chunk,
+                                                               G, k, k_rows, t, buf.plan, rec, b,
+                                                               rows, hdr);
+        }
+        return cudaGetLastError();
+    }
     {
         ProfScope ps_("rowsolve", st);
-        rowsolve_keys_kernel<<<(unsigned)B, 1024, 0, st>>>(buf.keys[0], buf.keys[1], n, k, k_rows,
+        rowsolve_keys_kernel<<<(unsigned)B, 512, 0, st>>>(buf.keys[0], buf.keys[1], n, k, k_rows,
                                                        t, buf.plan, b, rows, hdr);
     }
     return cudaGetLastError();

@@ -181,12 +181,13 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
         // A long chunk's maps in closed form: the product of its gap factors
         // telescopes, P_{hi-1} = gap(lo) e^{(s_lo - s_{hi-1})/t} P_{lo-1}
         // + sum_{i in chunk} e^{(s_i - s_{hi-1})/t}, and likewise Q_lo from
-        // Q_hi; the sums take fp32 exponentials (every term at most 1) added
-        // in fp64, so three fp64 exponentials serve the whole chunk and no
-        // rounding compounds along it.
+        // Q_hi; the sums take unbiased fp32 exponentials (every term at most
+        // 1) added in fp64, so three fp64 exponentials serve the whole chunk
+        // and no rounding compounds along it.
         if (valid) {
             const float s_first = get(lo), s_last = get(hi - 1);
-            const float sc = (float)(1.0 / t) * kLog2e;
+            const float it = (float)(1.0 / t);  // 1/t as a two-float pair
+            const float it_lo = (float)(1.0 / t - (double)it);
             double cf = 0.0, cb = 0.0;
             for (long long j0 = lo; j0 < hi; j0 += 8) {
                 float cf8 = 0.f, cb8 = 0.f;
@@ -195,8 +196,8 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
                     const long long j = j0 + u;
                     if (j < hi) {
                         const float x = get(j);
-                        cf8 += ex2_ftz((x - s_last) * sc);
-                        cb8 += ex2_ftz((s_first - x) * sc);
+                        cf8 += exp_neg(fmaf(s_last - x, it, (s_last - x) * it_lo));
+                        cb8 += exp_neg(fmaf(x - s_first, it, (x - s_first) * it_lo));
                     }
                 }
                 cf += (double)cf8;

@@ -12,6 +12,8 @@
 // row results are deterministic.  No CTA ever waits for another.
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
 #include "stream_common.cuh"
@@ -70,50 +72,63 @@ __global__ void __launch_bounds__(kThreads, SUP ? 6 : 1) emit_kernel(const float
     uint32_t nm = 0u;  // near mask of this thread's 16 scores
     bool near50 = false;  // some score with |x| <= 50 (the support serves the row)
     if (SUP && blockIdx.x == 0 && threadIdx.x == 0) sup.b[row] = brow;
-    if (VEC && base + kStreamTile <= n) {
-        const float4* r4 = reinterpret_cast<const float4*>(rr + base);
-        float4* p4 = reinterpret_cast<float4*>(pr + base);
-        float4 x[kPer / 4];
+    // Soft rows take margins without a common rounding error and unbiased
+    // exponentials, so that sums of very many p stay on budget; sharp rows
+    // (every weighted score within a factor of two of b) keep the fast forms,
+    // whose errors are then per score.  Two copies of the tile loop, chosen
+    // once per row.
+    auto tile = [&](auto soft_tag) {
+        constexpr bool SOFT = decltype(soft_tag)::value;
+        auto margin = [&](float x) {
+            return SOFT ? scaled_margin_exact(x, th) : scaled_margin_it(x, th);
+        };
+        auto expn = [&](float m) { return SOFT ? exp_neg(fabsf(m)) : neg_abs_exp(m); };
+        if (VEC && base + kStreamTile <= n) {
+            const float4* r4 = reinterpret_cast<const float4*>(rr + base);
+            float4* p4 = reinterpret_cast<float4*>(pr + base);
+            float4 x[kPer / 4];
 #pragma unroll
-        for (int q = 0; q < kPer / 4; ++q) x[q] = __ldcs(r4 + q * kThreads + threadIdx.x);
+            for (int q = 0; q < kPer / 4; ++q) x[q] = __ldcs(r4 + q * kThreads + threadIdx.x);
 #pragma unroll
-        for (int q = 0; q < kPer / 4; ++q) {
-            const float m0 = scaled_margin(x[q].x, th), m1 = scaled_margin(x[q].y, th);
-            const float m2 = scaled_margin(x[q].z, th), m3 = scaled_margin(x[q].w, th);
-            const float e0 = neg_abs_exp(m0), e1 = neg_abs_exp(m1), e2 = neg_abs_exp(m2),
-                        e3 = neg_abs_exp(m3);
-            __stcs(p4 + q * kThreads + threadIdx.x,
-                   make_float4(cdf_from(m0, e0), cdf_from(m1, e1), cdf_from(m2, e2),
-                               cdf_from(m3, e3)));
-            if (SUMF) sf += 0.5 * (double)((e0 + e1) + (e2 + e3));
-            if (SUP) {
-                near50 |= fminf(fminf(fabsf(m0), fabsf(m1)), fminf(fabsf(m2), fabsf(m3))) <= 50.f;
-                nm |= (fabsf(m0) <= kSupWindow ? 1u : 0u) << (4 * q);
-                nm |= (fabsf(m1) <= kSupWindow ? 1u : 0u) << (4 * q + 1);
-                nm |= (fabsf(m2) <= kSupWindow ? 1u : 0u) << (4 * q + 2);
-                nm |= (fabsf(m3) <= kSupWindow ? 1u : 0u) << (4 * q + 3);
-                *reinterpret_cast<float4*>(stg + stage_slot16(lane, 4 * q)) =
-                    make_float4(m0, m1, m2, m3);
+            for (int q = 0; q < kPer / 4; ++q) {
+                const float m0 = margin(x[q].x), m1 = margin(x[q].y);
+                const float m2 = margin(x[q].z), m3 = margin(x[q].w);
+                const float e0 = expn(m0), e1 = expn(m1), e2 = expn(m2), e3 = expn(m3);
+                __stcs(p4 + q * kThreads + threadIdx.x,
+                       make_float4(cdf_from(m0, e0), cdf_from(m1, e1), cdf_from(m2, e2),
+                                   cdf_from(m3, e3)));
+                if (SUMF) sf += 0.5 * (double)((e0 + e1) + (e2 + e3));
+                if (SUP) {
+                    near50 |= fminf(fminf(fabsf(m0), fabsf(m1)), fminf(fabsf(m2), fabsf(m3))) <= 50.f;
+                    nm |= (fabsf(m0) <= kSupWindow ? 1u : 0u) << (4 * q);
+                    nm |= (fabsf(m1) <= kSupWindow ? 1u : 0u) << (4 * q + 1);
+                    nm |= (fabsf(m2) <= kSupWindow ? 1u : 0u) << (4 * q + 2);
+                    nm |= (fabsf(m3) <= kSupWindow ? 1u : 0u) << (4 * q + 3);
+                    *reinterpret_cast<float4*>(stg + stage_slot16(lane, 4 * q)) =
+                        make_float4(m0, m1, m2, m3);
+                }
             }
-        }
-    } else {
-        float x[kPer], y[kPer];
-        bool ok[kPer];
-        load_tile<VEC>(rr, n, base, x, ok);
+        } else {
+            float x[kPer], y[kPer];
+            bool ok[kPer];
+            load_tile<VEC>(rr, n, base, x, ok);
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const float xs = scaled_margin(x[q], th);
-            const float e = neg_abs_exp(xs);
-            y[q] = cdf_from(xs, e);
-            if (SUMF && ok[q]) sf += 0.5 * (double)e;
-            if (SUP) {
-                near50 |= ok[q] && fabsf(xs) <= 50.f;
-                nm |= ((ok[q] && fabsf(xs) <= kSupWindow) ? 1u : 0u) << q;
-                stg[stage_slot16(lane, q)] = xs;
+            for (int q = 0; q < kPer; ++q) {
+                const float xs = margin(x[q]);
+                const float e = expn(xs);
+                y[q] = cdf_from(xs, e);
+                if (SUMF && ok[q]) sf += 0.5 * (double)e;
+                if (SUP) {
+                    near50 |= ok[q] && fabsf(xs) <= 50.f;
+                    nm |= ((ok[q] && fabsf(xs) <= kSupWindow) ? 1u : 0u) << q;
+                    stg[stage_slot16(lane, q)] = xs;
+                }
             }
+            store_tile<VEC>(pr, n, base, y);
         }
-        store_tile<VEC>(pr, n, base, y);
-    }
+    };
+    if (soft_row(brow, t)) tile(std::true_type{});
+    else tile(std::false_type{});
     uint32_t cnt = 0;  // warp-uniform: entries found in this warp's share
     if (SUP && __any_sync(0xffffffffu, nm != 0u)) {
         const int c = __popc(nm);

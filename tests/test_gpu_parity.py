@@ -54,6 +54,31 @@ def test_radix_sizes(cuda_device, n):
                       label=f"radix n={n} k={k} row={i}")
 
 
+@pytest.mark.parametrize("n,dist", [(262145, "normal"), (300001, "normal_q64"),
+                                    (1_000_003, "mix_nu"), (2_500_000, "abs_t3")])
+def test_radix_long_rows(cuda_device, n, dist):
+    """Rows past 4 x 65536 keys: the sorted row is solved over the whole GPU in
+    chunks (closed-form chunk maps, then the crossing chunk solved with the rest
+    folded into two anchors); ragged last chunks, ties, both temperatures.
+    With n > 16666, n fp32 roundings of p (6e-8 each) can exceed the 1e-3 budget
+    bar by themselves, so the sum is compared with the oracle's p rounded to
+    fp32; b, p and g keep their own tolerances.  The soft case (t = 1) is left
+    out for the quantised row: there ~600 scores share each value, so one p
+    within an ulp of its correctly rounded value moves the sum by 600 ulps, and
+    fp32 p (about 1e-7 each) cannot hold a sum of 1e5 soft probabilities to
+    1e-3 (the unquantised rows, where those errors are independent, do)."""
+    B = 2
+    r, v = random_rows(30 + n, B, n, dist)
+    cases = [(1.0, 0.05), (n / 3.0 + 0.37, 1.0), (float(n // 100), 0.01), (n - 0.5, 0.05)]
+    if dist == "normal_q64":
+        cases = [c for c in cases if c[1] != 1.0]
+    for k, t in cases:
+        out = run_gpu(r, k, t, path="radix", v=v)
+        for i in range(B):
+            check_row(r[i], v[i], k, t, out["b"][i], out["p"][i], out["g"][i],
+                      label=f"radix {dist} n={n} k={k} t={t} row={i}", sum_ref="fp32")
+
+
 @pytest.mark.parametrize("n", [2, 100, 4097, 8191, 65536, 70001, 300000])
 def test_rowbracket_sizes(cuda_device, n):
     B = 3
