@@ -114,29 +114,16 @@ __device__ __forceinline__ Thr make_thr(double b, double t) {
 __device__ __forceinline__ float scaled_margin(float r, const Thr& h) {
     return __fmul_rn(__fsub_rn(__fsub_rn(r, h.hi), h.lo), h.inv_t);
 }
-// The same margin without a rounding error common to many scores: the
-// rounding of r - hi discards the bits of hi below the ulp of r - hi, the same
-// for every score of a binade, and 1/t's rounding is shared by all, so summed
-// over many p both bias the budget.  r - hi is taken exactly by Knuth's
-// two-sum and 1/t as a two-float pair.  Scores within a factor of two of hi
-// (every score that carries weight when t is small against |b|) give the same
-// result through scaled_margin, since r - hi is then exact (Sterbenz).
-__device__ __forceinline__ float scaled_margin_exact(float r, const Thr& h) {
-    const float s = __fsub_rn(r, h.hi);
-    const float rv = __fadd_rn(s, h.hi);  // r as recovered from s
-    const float hv = __fsub_rn(s, rv);    // -hi as recovered from s
-    const float err = __fadd_rn(__fsub_rn(r, rv), __fsub_rn(-h.hi, hv));
-    const float d = __fadd_rn(s, __fsub_rn(err, h.lo));
-    return fmaf(d, h.inv_t, __fmul_rn(d, h.inv_lo));
-}
 // The fast margin with 1/t as a two-float pair (its rounding is common to all
 // scores of a row).
 __device__ __forceinline__ float scaled_margin_it(float r, const Thr& h) {
     const float d = __fsub_rn(__fsub_rn(r, h.hi), h.lo);
     return fmaf(d, h.inv_t, __fmul_rn(d, h.inv_lo));
 }
-// Rows where some weighted score can lie outside [b/2, 2b]: t not small
-// against |b| (40 t covers |x| <= 20, below which e^{-|x|} < 2.1e-9).
+// Soft rows: t not small against |b|.  On sharp rows (40 t < |b|) every score
+// that carries weight (|x| <= 20, beyond which e^{-|x|} < 2.1e-9) lies within
+// a factor of two of b, where r - hi is exact, and the fast margin's one
+// rounding stays below 2^-24 |x|.
 __device__ __forceinline__ bool soft_row(double b, double t) { return 40.0 * t >= fabs(b); }
 
 // 2^y with flush-to-zero for results below the smallest normal float (the

@@ -16,6 +16,8 @@
 // row at once (those histograms do not depend on the key order), so a digit
 // that is the same for every key of a row is known up front and its pass is
 // skipped for that row.  Each row tracks which ping-pong buffer holds it.
+#include <type_traits>
+
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
 #include "solve_sorted.cuh"
@@ -313,7 +315,6 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
     uint32_t* __restrict__ lb, unsigned long long* __restrict__ counter, WsHeader* hdr) {
     __shared__ uint32_t wcnt[kWarps][256];
     __shared__ uint32_t tstart[256];
-    __shared__ uint32_t gbase[256];
     __shared__ uint32_t sorted[kRadixTile];
     __shared__ uint32_t wsum[2][kWarps];
     __shared__ unsigned long long s_id;
@@ -339,27 +340,34 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
 
     uint32_t key[kPerThread], lrank[kPerThread];
     const uint32_t lt = lanemask_lt();
+    // tile-local 32-bit positions: warp w owns [w*512, (w+1)*512), visited 32
+    // at a time in index order, which keeps the rank stable
+    const int valid = (int)min((int64_t)kRadixTile, n - base);
+    const uint32_t* tsrc = src + base;
+    const int off0 = warp * (32 * kPerThread) + lane;
+    auto rank = [&](auto full_tag) {
+        constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
-        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
-        key[e] = idx < n ? src[idx] : 0u;
-    }
-#pragma unroll
-    for (int e = 0; e < kPerThread; ++e) {
-        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
-        const bool ok = idx < n;
-        const uint32_t dig = (key[e] >> shift) & 255u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, ok ? dig : 256u + lane);
-        const int leader = __ffs(peers) - 1;
-        uint32_t bse = 0;
-        if (ok && lane == leader) {
-            bse = wcnt[warp][dig];
-            wcnt[warp][dig] = bse + __popc(peers);
+        for (int e = 0; e < kPerThread; ++e) {
+            const int li = off0 + e * 32;
+            key[e] = (FULL || li < valid) ? tsrc[li] : 0u;
         }
-        bse = __shfl_sync(0xffffffffu, bse, leader);
-        lrank[e] = bse + __popc(peers & lt);
-        __syncwarp();
-    }
+#pragma unroll
+        for (int e = 0; e < kPerThread; ++e) {
+            const bool ok = FULL || off0 + e * 32 < valid;
+            const uint32_t dig = (key[e] >> shift) & 255u;
+            const uint32_t peers =
+                __match_any_sync(0xffffffffu, ok ? dig : 256u + (uint32_t)lane);
+            // every peer reads the digit's count before the lowest peer adds
+            // the group (one warp's shared accesses stay in program order)
+            const uint32_t old = ok ? wcnt[warp][dig] : 0u;
+            if (ok && (peers & lt) == 0u) wcnt[warp][dig] = old + __popc(peers);
+            lrank[e] = old + __popc(peers & lt);
+            __syncwarp();
+        }
+    };
+    if (valid == kRadixTile) rank(std::true_type{});
+    else rank(std::false_type{});
     __syncthreads();
     uint32_t cnt = 0;  // this tile's count of digit v
 #pragma unroll
@@ -405,24 +413,25 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
         if (threadIdx.x == 0) set_status(hdr, kDevWaitTimeout);
         return;
     }
-    gbase[v] = dbase + excl;
-    // exclusive scan of the tile's digit counts -> local start of each digit
-    tstart[v] = block256_excl_scan(cnt, wsum[1]);
+    // exclusive scan of the tile's digit counts -> local start of each digit;
+    // then per (warp, digit) the local slot base, and per digit the shift
+    // from a local slot to the global position
+    const uint32_t ts = block256_excl_scan(cnt, wsum[1]);
+    tstart[v] = dbase + excl - ts;  // global position of local slot 0 of digit v
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) wcnt[w][v] += ts;
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < kPerThread; ++e) {
-        const int64_t idx = base + warp * (32 * kPerThread) + e * 32 + lane;
-        if (idx < n) {
+        if (off0 + e * 32 < valid) {
             const uint32_t dig = (key[e] >> shift) & 255u;
-            sorted[tstart[dig] + wcnt[warp][dig] + lrank[e]] = key[e];
+            sorted[wcnt[warp][dig] + lrank[e]] = key[e];
         }
     }
     __syncthreads();
-    const int valid = (int)min((int64_t)kRadixTile, n - base);
     for (int i = threadIdx.x; i < valid; i += kThreads) {
         const uint32_t kv = sorted[i];
-        const uint32_t dig = (kv >> shift) & 255u;
-        const uint32_t pos = gbase[dig] + (uint32_t)i - tstart[dig];
+        const uint32_t pos = tstart[(kv >> shift) & 255u] + (uint32_t)i;
         if ((int64_t)pos < n) dst[pos] = kv;
     }
 }

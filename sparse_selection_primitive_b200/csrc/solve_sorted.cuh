@@ -186,18 +186,21 @@ __device__ void solve_sorted_block(Get get, long long nb, const Tails& tl, doubl
         // and no rounding compounds along it.
         if (valid) {
             const float s_first = get(lo), s_last = get(hi - 1);
-            const float it = (float)(1.0 / t);  // 1/t as a two-float pair
-            const float it_lo = (float)(1.0 / t - (double)it);
+            const double it = 1.0 / t;
             double cf = 0.0, cb = 0.0;
-            for (long long j0 = lo; j0 < hi; j0 += 8) {
+            for (long long j0 = lo; j0 < hi; j0 += 16) {
+                // the loads of 16 positions first, so that they overlap
+                float xs[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) xs[u] = j0 + u < hi ? get(j0 + u) : s_last;
                 float cf8 = 0.f, cb8 = 0.f;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const long long j = j0 + u;
-                    if (j < hi) {
-                        const float x = get(j);
-                        cf8 += exp_neg(fmaf(s_last - x, it, (s_last - x) * it_lo));
-                        cb8 += exp_neg(fmaf(x - s_first, it, (x - s_first) * it_lo));
+                for (int u = 0; u < 16; ++u) {
+                    if (j0 + u < hi) {
+                        // arguments in fp64: an fp32 difference of scores in
+                        // different binades rounds the same way for all of them
+                        cf8 += exp_neg((float)(((double)s_last - (double)xs[u]) * it));
+                        cb8 += exp_neg((float)(((double)xs[u] - (double)s_first) * it));
                     }
                 }
                 cf += (double)cf8;

@@ -72,17 +72,28 @@ __global__ void __launch_bounds__(kThreads, SUP ? 6 : 1) emit_kernel(const float
     uint32_t nm = 0u;  // near mask of this thread's 16 scores
     bool near50 = false;  // some score with |x| <= 50 (the support serves the row)
     if (SUP && blockIdx.x == 0 && threadIdx.x == 0) sup.b[row] = brow;
-    // Soft rows take margins without a common rounding error and unbiased
-    // exponentials, so that sums of very many p stay on budget; sharp rows
-    // (every weighted score within a factor of two of b) keep the fast forms,
-    // whose errors are then per score.  Two copies of the tile loop, chosen
-    // once per row.
+    // Soft rows (t not small against |b|) form p in fp64 and round it once,
+    // so that sums of very many soft p stay on budget (fp32 margins and
+    // exponentials leave errors of a fraction of an ulp that do not average
+    // out over 10^6 scores); sharp rows keep the fp32 forms.  Two copies of
+    // the tile loop, chosen once per row.
+    const double inv_td = 1.0 / t;
     auto tile = [&](auto soft_tag) {
         constexpr bool SOFT = decltype(soft_tag)::value;
-        auto margin = [&](float x) {
-            return SOFT ? scaled_margin_exact(x, th) : scaled_margin_it(x, th);
+        // margin, e^{-|margin|} and p of one score
+        auto mep = [&](float x, float& e, float& pv) {
+            if (SOFT) {
+                const double xd = ((double)x - brow) * inv_td;
+                const double ed = exp(-fabs(xd));
+                e = (float)ed;
+                pv = (float)(xd < 0.0 ? 0.5 * ed : 1.0 - 0.5 * ed);
+                return (float)xd;
+            }
+            const float m = scaled_margin_it(x, th);
+            e = neg_abs_exp(m);
+            pv = cdf_from(m, e);
+            return m;
         };
-        auto expn = [&](float m) { return SOFT ? exp_neg(fabsf(m)) : neg_abs_exp(m); };
         if (VEC && base + kStreamTile <= n) {
             const float4* r4 = reinterpret_cast<const float4*>(rr + base);
             float4* p4 = reinterpret_cast<float4*>(pr + base);
@@ -91,12 +102,11 @@ __global__ void __launch_bounds__(kThreads, SUP ? 6 : 1) emit_kernel(const float
             for (int q = 0; q < kPer / 4; ++q) x[q] = __ldcs(r4 + q * kThreads + threadIdx.x);
 #pragma unroll
             for (int q = 0; q < kPer / 4; ++q) {
-                const float m0 = margin(x[q].x), m1 = margin(x[q].y);
-                const float m2 = margin(x[q].z), m3 = margin(x[q].w);
-                const float e0 = expn(m0), e1 = expn(m1), e2 = expn(m2), e3 = expn(m3);
-                __stcs(p4 + q * kThreads + threadIdx.x,
-                       make_float4(cdf_from(m0, e0), cdf_from(m1, e1), cdf_from(m2, e2),
-                                   cdf_from(m3, e3)));
+                float e0, e1, e2, e3;
+                float4 pq;
+                const float m0 = mep(x[q].x, e0, pq.x), m1 = mep(x[q].y, e1, pq.y);
+                const float m2 = mep(x[q].z, e2, pq.z), m3 = mep(x[q].w, e3, pq.w);
+                __stcs(p4 + q * kThreads + threadIdx.x, pq);
                 if (SUMF) sf += 0.5 * (double)((e0 + e1) + (e2 + e3));
                 if (SUP) {
                     near50 |= fminf(fminf(fabsf(m0), fabsf(m1)), fminf(fabsf(m2), fabsf(m3))) <= 50.f;
@@ -114,9 +124,8 @@ __global__ void __launch_bounds__(kThreads, SUP ? 6 : 1) emit_kernel(const float
             load_tile<VEC>(rr, n, base, x, ok);
 #pragma unroll
             for (int q = 0; q < kPer; ++q) {
-                const float xs = margin(x[q]);
-                const float e = expn(xs);
-                y[q] = cdf_from(xs, e);
+                float e;
+                const float xs = mep(x[q], e, y[q]);
                 if (SUMF && ok[q]) sf += 0.5 * (double)e;
                 if (SUP) {
                     near50 |= ok[q] && fabsf(xs) <= 50.f;
