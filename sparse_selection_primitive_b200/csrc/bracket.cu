@@ -516,6 +516,23 @@ __device__ __forceinline__ void fold_one(float x, float aL, float aR, float inv_
     acc.SR += (double)sr;
 }
 
+// The same on a soft row (40 t >= |b|, where every score can carry weight):
+// the tail term in fp64, from an fp64 margin, so that the tail sums of 10^6
+// soft scores keep the budget (fp32 margins and exponentials leave errors of
+// a fraction of an ulp that do not average out).
+__device__ __forceinline__ void fold_one_soft(float x, float aL, float aR, double inv_td,
+                                              FoldAcc& acc, bool& in_band) {
+    acc.bad |= !finite_f(x);
+    const bool right = x >= aR, left = x < aL;
+    const double a = right ? ((double)x - (double)aR) * inv_td
+                           : (left ? ((double)aL - (double)x) * inv_td : 0.0);
+    const double e = exp(-a);
+    acc.cntR += right ? 1u : 0u;
+    acc.SR += right ? e : 0.0;
+    acc.SL += left ? e : 0.0;
+    in_band = !(right | left);
+}
+
 // Adds one band score to the fixed-point band histogram (global atomics).
 __device__ __forceinline__ void bin_add(float x, const BinLayout& BL, float inv_t,
                                         unsigned long long* bins) {
@@ -610,6 +627,11 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
     const BinLayout BL = make_bins(st->bin_kmin, st->bin_kmax);
     if (!hist) bins = nullptr;
     const float inv_t = (float)(1.0 / t);
+    const double inv_td = 1.0 / t;
+    // soft row: 40 t >= |b|, b judged by the bracket's finite ends (uniform)
+    const double bc = isfinite(aL) ? (isfinite(aR) ? 0.5 * ((double)aL + (double)aR) : (double)aL)
+                                   : (isfinite(aR) ? (double)aR : 0.0);
+    const bool soft = 40.0 * t >= fabs(bc);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float* q = fold_dyn + warp * kQ;
     float* stg = fold_dyn + (kFoldThreads / 32) * kQ + warp * (32 * 16);
@@ -630,7 +652,10 @@ __global__ void __launch_bounds__(kFoldThreads, 4) fold_kernel(const float* __re
         const bool ok = lane < cnt;
         const float x = ok ? q[(head + lane) & (kQ - 1)] : 0.f;
         bool inb = false;
-        if (ok) fold_one(x, aL, aR, inv_t, acc, inb);
+        if (ok) {
+            if (soft) fold_one_soft(x, aL, aR, inv_td, acc, inb);
+            else fold_one(x, aL, aR, inv_t, acc, inb);
+        }
         band_stage(inb, x, sband, &scount, band, counter, cap, BL, inv_t, bins);
         head += cnt;
     };
@@ -1339,6 +1364,12 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
                            double t, float* band, SolveSmemAll* sm, Tails& tl, long long* nb,
                            bool* bad) {
     const float k2 = (float)(kLog2e / t);
+    const double inv_td = 1.0 / t;
+    // soft row (40 t >= |b|, b judged by the bracket's finite ends): the tail
+    // terms in fp64, so that sums of very many soft scores keep the budget
+    const double bc = isfinite(aL) ? (isfinite(aR) ? 0.5 * ((double)aL + (double)aR) : (double)aL)
+                                   : (isfinite(aR) ? (double)aR : 0.0);
+    const bool soft = 40.0 * t >= fabs(bc);
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) sm->cnt = 0ull;
     __syncthreads();
@@ -1348,9 +1379,17 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
     // One score (ok = in range): the tail terms; returns whether it is in the band.
     auto fold1 = [&](float x, bool ok, float& sl, float& sr) -> bool {
         const bool right = ok && x >= aR, left = ok && x < aL;
-        const float e = ex2_ftz((right ? aR - x : (left ? x - aL : 0.f)) * k2);
-        sr += right ? e : 0.f;
-        sl += left ? e : 0.f;
+        if (soft) {
+            const double a = right ? ((double)x - (double)aR) * inv_td
+                                   : (left ? ((double)aL - (double)x) * inv_td : 0.0);
+            const double e = exp(-a);
+            SR += right ? e : 0.0;
+            SL += left ? e : 0.0;
+        } else {
+            const float e = ex2_ftz((right ? aR - x : (left ? x - aL : 0.f)) * k2);
+            sr += right ? e : 0.f;
+            sl += left ? e : 0.f;
+        }
         cR += right ? 1u : 0u;
         if (ok) probe = fmaf(x, 0.f, probe);
         return ok && !right && !left;

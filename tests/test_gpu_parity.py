@@ -74,6 +74,21 @@ def test_radix_long_rows(cuda_device, n, dist):
                       label=f"radix {dist} n={n} k={k} t={t} row={i}", sum_ref="auto")
 
 
+@pytest.mark.parametrize("n,dist,path", [(262145, "normal", "rowbracket"),
+                                         (1_000_003, "abs_t3", "bracket"),
+                                         (600_001, "normal_q64", "bracket")])
+def test_bracketing_soft_long_rows(cuda_device, n, dist, path):
+    """Soft rows (t = 1, far above the gaps: every score carries weight) of
+    2.6e5 to 1e6 scores through both bracketing arrangements: the fold's tail
+    terms and p are formed in fp64 on such rows, so that the budget bar holds
+    over 10^5 to 10^6 probabilities away from 0 and 1."""
+    r, v = random_rows(50 + n, 1, n, dist)
+    for k in (n / 3.0 + 0.37, float(n // 10)):
+        out = run_gpu(r, k, 1.0, path=path, v=v)
+        check_row(r[0], v[0], k, 1.0, out["b"][0], out["p"][0], out["g"][0],
+                  label=f"{path} {dist} n={n} k={k} t=1", sum_ref="auto")
+
+
 @pytest.mark.parametrize("n", [2, 100, 4097, 8191, 65536, 70001, 300000])
 def test_rowbracket_sizes(cuda_device, n):
     B = 3
