@@ -183,24 +183,6 @@ __device__ __forceinline__ double row_sum_d(double v, double* red) {
     }
 }
 template <int E, int RT, int CTA>
-__device__ __forceinline__ float row_sum_f(float v, float* red) {
-    using S = Shape<E, RT, CTA>;
-    v = warp_sum_f(v);
-    if constexpr (S::WPR == 1) {
-        return v;
-    } else {
-        const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        if (lane == 0) red[w] = v;
-        __syncthreads();
-        const int w0 = (w / S::WPR) * S::WPR;
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < S::WPR; ++i) s += red[w0 + i];
-        __syncthreads();
-        return s;
-    }
-}
-template <int E, int RT, int CTA>
 __device__ __forceinline__ float row_min_f(float v, float* red) {
     using S = Shape<E, RT, CTA>;
     v = warp_min_f(v);
@@ -815,6 +797,7 @@ __global__ void __launch_bounds__(CTA) onchip_backward_kernel(
     const float* __restrict__ v, float* __restrict__ g, int64_t B, int n, double t, int vec) {
     using S = Shape<E, RT, CTA>;
     __shared__ float fred[S::NW];
+    __shared__ double dred[S::NW];
     const int rloc = threadIdx.x / RT;
     const int tid = threadIdx.x % RT;
     const int64_t row = (int64_t)blockIdx.x * S::ROWS + rloc;
@@ -834,25 +817,24 @@ __global__ void __launch_bounds__(CTA) onchip_backward_kernel(
         mloc = fminf(mloc, ax[e]);
     }
     const float mu = row_min_f<E, RT, CTA>(mloc, fred);
-    // R = sum v f / sum f with weights w = exp(-(|x| - mu)) <= 1, summed in
-    // fp32 (at most 4096 terms of at most 1: a relative error near 1e-6, far
-    // inside the gradient's tolerance); f = e^{-mu} w / 2 takes the same
-    // exponential.
+    // R = sum v f / sum f with weights w = exp(-(|x| - mu)) <= 1, in fp64 (v - R
+    // cancels when one weight dominates, and every g is then that small);
+    // f = e^{-mu} w / 2 takes the same exponential.
     float wv[E];
-    float sw = 0.f, swv = 0.f;
+    double sw = 0.0, swv = 0.0;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         wv[e] = valid[e] ? __expf(mu - ax[e]) : 0.f;
-        sw += wv[e];
-        swv = fmaf(wv[e], vv[e], swv);
+        sw += (double)wv[e];
+        swv += (double)wv[e] * (double)vv[e];
     }
-    sw = row_sum_f<E, RT, CTA>(sw, fred);
-    swv = row_sum_f<E, RT, CTA>(swv, fred);
-    const float R = swv / sw;
+    sw = row_sum_d<E, RT, CTA>(sw, dred);
+    swv = row_sum_d<E, RT, CTA>(swv, dred);
+    const double R = swv / sw;
     const float scale = 0.5f * __expf(-mu) * th.inv_t;
     float gv[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) gv[e] = scale * wv[e] * (vv[e] - R);
+    for (int e = 0; e < E; ++e) gv[e] = scale * wv[e] * (float)((double)vv[e] - R);
     store_row<E>(g + off, n, tid, vec != 0, row_ok, gv);
 }
 
