@@ -402,9 +402,14 @@ __global__ void __launch_bounds__(kThreads, 4) radix_onesweep_kernel(
                 if (f == kLbInc) done = true;
             }
             j -= adv;
-            if (!done && adv == 0 && ++spins > kLbSpinMax) {
-                timed_out = true;
-                break;
+            if (!done && adv == 0) {
+                if (++spins > kLbSpinMax) {
+                    timed_out = true;
+                    break;
+                }
+                // a predecessor still ranking: yield the issue slots to the
+                // warps that are doing work
+                __nanosleep(100);
             }
         }
         if (!timed_out) words[tile * 256 + v] = kLbInc | (excl + cnt);
