@@ -164,7 +164,8 @@ int lapsum_forward_hard(const float* r, int64_t ld, float* p, double* b, int64_t
                         double k, int path, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Router form for short rows (n <= 4096, the on-chip sort), e.g. the scores of
+ * Router form for short rows (n <= 4096, on chip: the segment search for
+ * n <= 256, the sort above), e.g. the scores of
  * a mixture-of-experts router: scores r of type `dtype` (fp32, or bf16 or fp16
  * bit patterns widened exactly to fp32), p (fp32) and b (fp64) as lapsum_forward,
  * and, when sel_cnt is not NULL, the sparse support of each row next to p:
@@ -221,7 +222,8 @@ int lapsum_backward_lowp(const void* r, int dtype, int64_t ld, const double* b, 
  * memory, B entries, read in stream order) in place of the shared k.  The
  * pages fix one budget per operator call; a budget per row is the next step
  * the same equation allows (every row is solved on its own).  Solvers:
- * LAPSUM_PATH_AUTO gives the on-chip sort for n <= 4096, the one-CTA-per-row
+ * LAPSUM_PATH_AUTO gives the on-chip segment search for n <= 256 and the
+ * on-chip sort for n <= 4096, the one-CTA-per-row
  * bracketing for n <= 2^18 and the whole-GPU bracketing above (both compute
  * each row's sample size and binomial ranks on the device from its budget);
  * LAPSUM_PATH_FULLSORT, LAPSUM_PATH_RADIX, LAPSUM_PATH_ROWBRACKET (n <= 2^20)
