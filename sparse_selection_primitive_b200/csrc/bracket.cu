@@ -2222,11 +2222,8 @@ cudaError_t launch_shard_fold(const float* r, int64_t n_shard, const float* ends
     double* part = reinterpret_cast<double*>(static_cast<char*>(ws) + 512);
     int grid = bracket_fold_grid();
     if (grid > kFoldGridMaxShard) grid = kFoldGridMaxShard;
-    static unsigned long long attr_devices = 0ull;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-    if ((attr_devices & bit) == 0ull || bit == 0ull) {
+    static std::atomic<unsigned long long> attr_devices{0ull};
+    once_per_device(attr_devices, [&]() {
         cudaFuncSetAttribute(fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kFoldDynSmem);
         cudaFuncSetAttribute(shard_fold_records_kernel,
@@ -2234,8 +2231,7 @@ cudaError_t launch_shard_fold(const float* r, int64_t n_shard, const float* ends
                              (int)sizeof(SolveSmemAll));
         cudaFuncSetAttribute(shard_band_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sizeof(SolveSmemAll));
-        attr_devices |= bit;
-    }
+    });
     shard_fold_setup_kernel<<<1, 1, 0, st>>>(ends, rs);
     const int vec = ((reinterpret_cast<uintptr_t>(r) & 15u) == 0) ? 1 : 0;
     fold_kernel<<<grid, kFoldThreads, kFoldDynSmem, st>>>(r, n_shard, t, rs, band, nullptr, part,
@@ -2247,15 +2243,11 @@ cudaError_t launch_shard_fold(const float* r, int64_t n_shard, const float* ends
 cudaError_t launch_shard_band_solve(const float* bands, int64_t stride, const double* recs,
                                     int world, const float* ends, double k, double t, float* cur,
                                     float* nxt, double* out, cudaStream_t st) {
-    static unsigned long long attr_devices = 0ull;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-    if ((attr_devices & bit) == 0ull || bit == 0ull) {
+    static std::atomic<unsigned long long> attr_devices{0ull};
+    once_per_device(attr_devices, [&]() {
         cudaFuncSetAttribute(shard_band_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sizeof(SolveSmemAll));
-        attr_devices |= bit;
-    }
+    });
     shard_band_solve_kernel<<<1, kBlk, sizeof(SolveSmemAll), st>>>(bands, stride, recs, world,
                                                                   ends, k, t, cur, nxt, out);
     return cudaGetLastError();
@@ -2268,15 +2260,11 @@ cudaError_t launch_rowbracket(const float* r, int64_t ld, int64_t B, int64_t n, 
                               int64_t rank_h[kLadder], int flags, RowState* rows, float* band0,
                               float* band1, double* b, WsHeader* hdr, int vec, cudaStream_t st,
                               const RowBudget* budgets, uint32_t* sup_flags) {
-    static unsigned long long attr_devices = 0ull;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-    if ((attr_devices & bit) == 0ull || bit == 0ull) {
+    static std::atomic<unsigned long long> attr_devices{0ull};
+    once_per_device(attr_devices, [&]() {
         cudaFuncSetAttribute(rowbracket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)rowbracket_smem(kSampleMax));
-        attr_devices |= bit;
-    }
+    });
     Ladder lad;
     for (int i = 0; i < kLadder; ++i) {
         lad.l[i] = rank_l[i];
@@ -2409,13 +2397,10 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                                uint32_t* sup_flag, const RowBudget* bud, cudaStream_t st) {
     // dynamic shared memory limits, set once per device (they belong to the
     // device's copy of the module)
-    static unsigned long long attr_devices = 0ull;
+    static std::atomic<unsigned long long> attr_devices{0ull};
     const size_t solve_smem = sizeof(SolveSmemAll);
     const size_t sample_smem = ((size_t)kSampleMax + 2 * 2048) * sizeof(uint32_t);
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-    if ((attr_devices & bit) == 0ull || bit == 0ull) {
+    once_per_device(attr_devices, [&]() {
         cudaFuncSetAttribute(solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)solve_smem);
         cudaFuncSetAttribute(solve2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -2424,8 +2409,7 @@ cudaError_t launch_bracket_row(const float* r_row, int64_t n, double k, double t
                              (int)sample_smem);
         cudaFuncSetAttribute(fold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kFoldDynSmem);
-        attr_devices |= bit;
-    }
+    });
     Ladder lad;
     for (int i = 0; i < kLadder; ++i) {
         lad.l[i] = rank_l[i];

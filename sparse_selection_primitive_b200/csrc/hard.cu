@@ -405,15 +405,11 @@ cudaError_t launch_hard_bracket(const float* r, int64_t ld, float* p, double* b,
                            st>>>(r, ld, n, band, rows, hdr);
     }
     {
-        static unsigned long long attr_devices = 0ull;
-        int dev = 0;
-        cudaGetDevice(&dev);
-        const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-        if ((attr_devices & bit) == 0ull || bit == 0ull) {
+        static std::atomic<unsigned long long> attr_devices{0ull};
+        once_per_device(attr_devices, [&]() {
             cudaFuncSetAttribute(hard_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(HardSmem));
-            attr_devices |= bit;
-        }
+        });
         ProfScope ps_("hard_solve", st);
         hard_solve_kernel<<<(unsigned)B, kBlk, sizeof(HardSmem), st>>>(r, ld, n, k, rank, band, b,
                                                                        rows, hdr, B_total);

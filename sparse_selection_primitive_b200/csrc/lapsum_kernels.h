@@ -1,6 +1,7 @@
 // Host-side launchers of the Fast LapSum kernels (internal to the library).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -38,6 +39,21 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Runs `set` (kernel attributes, which are per device) the first time a
+// process reaches this point on the current device; `done` holds one bit per
+// device (devices past 63 set it every time).  Thread-safe: a race only sets
+// the same attribute twice.
+template <class F>
+inline void once_per_device(std::atomic<unsigned long long>& done, F set) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit == 0ull || (done.load(std::memory_order_acquire) & bit) == 0ull) {
+        set();
+        done.fetch_or(bit, std::memory_order_acq_rel);
+    }
 }
 
 // --- on-chip full sort (n <= 4096) -------------------------------------------

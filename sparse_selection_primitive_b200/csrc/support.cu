@@ -23,6 +23,8 @@
 // no score of the row has |x| <= 50 (then scores outside the list could weigh
 // in R); the forward's emit pass records the first and the last of these per
 // row, so every CTA knows the row's mode before it starts.
+#include <atomic>
+
 #include "lapsum_common.cuh"
 #include "lapsum_kernels.h"
 #include "stream_common.cuh"
@@ -419,11 +421,17 @@ cudaError_t launch_backward_support(const float* r, int64_t ld, const double* b,
     const int64_t tiles = stream_tiles(n);
     // pass A: one wave of resident CTAs walking groups of up to 32 tiles;
     // pass B: one CTA per tile
-    static int per_sm_a = 0;
+    // resident CTAs per SM of pass A, per device
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> per_sm[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int per_sm_a = (dev >= 0 && dev < kMaxDevices) ? per_sm[dev].load(std::memory_order_relaxed) : 0;
     if (per_sm_a == 0) {
         int pa = 0;
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pa, sup_reduce_kernel<true>, kThreads, 0);
         per_sm_a = pa > 0 ? pa : 1;
+        if (dev >= 0 && dev < kMaxDevices) per_sm[dev].store(per_sm_a, std::memory_order_relaxed);
     }
     const int cap_a = per_sm_a * device_sm_count();
     int64_t want = cap_a / B;
