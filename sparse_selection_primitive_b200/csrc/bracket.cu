@@ -1360,16 +1360,16 @@ __device__ int plan_with_bins(const unsigned long long* __restrict__ bins, const
 // solve sorts it).  Four 16-byte loads per thread in flight per trip; every
 // score takes one exponential (masked inside the band).  Sets *bad when a
 // score is NaN or infinite.
-__device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, int vec, float aL, float aR,
-                           double t, float* band, SolveSmemAll* sm, Tails& tl, long long* nb,
-                           bool* bad) {
+// SOFT: a soft row (40 t >= |b|, b judged by the bracket's finite ends), whose
+// tail terms are taken in fp64 so that sums of very many soft scores keep the
+// budget; refold_row picks the instance once per call.
+template <bool SOFT>
+__device__ __noinline__ void refold_row_t(const float* __restrict__ r, int64_t n, int vec, float aL,
+                                          float aR, double t, float* band, SolveSmemAll* sm,
+                                          Tails& tl, long long* nb, bool* bad) {
     const float k2 = (float)(kLog2e / t);
     const double inv_td = 1.0 / t;
-    // soft row (40 t >= |b|, b judged by the bracket's finite ends): the tail
-    // terms in fp64, so that sums of very many soft scores keep the budget
-    const double bc = isfinite(aL) ? (isfinite(aR) ? 0.5 * ((double)aL + (double)aR) : (double)aL)
-                                   : (isfinite(aR) ? (double)aR : 0.0);
-    const bool soft = 40.0 * t >= fabs(bc);
+    constexpr bool soft = SOFT;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) sm->cnt = 0ull;
     __syncthreads();
@@ -1379,7 +1379,7 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
     // One score (ok = in range): the tail terms; returns whether it is in the band.
     auto fold1 = [&](float x, bool ok, float& sl, float& sr) -> bool {
         const bool right = ok && x >= aR, left = ok && x < aL;
-        if (soft) {
+        if constexpr (soft) {
             const double a = right ? ((double)x - (double)aR) * inv_td
                                    : (left ? ((double)aL - (double)x) * inv_td : 0.0);
             const double e = exp(-a);
@@ -1488,6 +1488,15 @@ __device__ __noinline__ void refold_row(const float* __restrict__ r, int64_t n, 
     tl.cntR = (double)cnt;
     *nb = (long long)sm->cnt;
     if (bad) *bad = any_bad != 0;
+}
+
+__device__ void refold_row(const float* __restrict__ r, int64_t n, int vec, float aL, float aR,
+                           double t, float* band, SolveSmemAll* sm, Tails& tl, long long* nb,
+                           bool* bad) {
+    const double bc = isfinite(aL) ? (isfinite(aR) ? 0.5 * ((double)aL + (double)aR) : (double)aL)
+                                   : (isfinite(aR) ? (double)aR : 0.0);
+    if (40.0 * t >= fabs(bc)) refold_row_t<true>(r, n, vec, aL, aR, t, band, sm, tl, nb, bad);
+    else refold_row_t<false>(r, n, vec, aL, aR, t, band, sm, tl, nb, bad);
 }
 
 // The attempt loop of the band solve, shared by the grid pipeline's solve
