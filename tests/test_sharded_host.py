@@ -1,4 +1,4 @@
-"""Host logic of one row split over several devices, on CPU with two gloo ranks.
+"""Host logic of one row split over several devices, on CPU with two and three gloo ranks.
 
 The split-row path ("Fast LapSum: Exact Differentiable Top-k at Million
 Scale", gist.science explainer pages, section 2.2, with the row in shards)
@@ -131,27 +131,28 @@ def _rank_main(rank, world, port, cuts, force, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("force", [False, True])
-def test_two_gloo_ranks_split_one_row(force):
+@pytest.mark.parametrize("world,force", [(2, False), (2, True), (3, False)])
+def test_gloo_ranks_split_one_row(world, force):
     import oracle
     from workloads import random_rows
-    world, n = 2, 30000
-    cuts = [0, 11111, n]          # unequal shards
+    n = 30000
+    cuts = {2: [0, 11111, n], 3: [0, 7001, 19999, n]}[world]  # unequal shards
     port = _free_port()
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_rank_main, args=(world, port, cuts, force, out), nprocs=world, join=True,
                        start_method="spawn")
-    b0, att0, p0, g0 = out[0]
-    b1, att1, p1, g1 = out[1]
-    assert b0 == b1 and att0 == att1       # every rank takes the same decisions
+    res = [out[i] for i in range(world)]
+    # every rank takes the same decisions and finds the same b
+    assert all(x[0] == res[0][0] and x[1] == res[0][1] for x in res)
+    b0, att0 = res[0][0], res[0][1]
     assert att0 >= (2 if force else 1)
     r, v = random_rows(77, 1, n, "mix_nu")
     row = r[0].astype(np.float64)
     b_ref = oracle.solve_b(row, 40.0, 0.02)
     assert abs(b0 - b_ref) <= 1e-10 * max(0.02, abs(b_ref))
-    p = np.concatenate([p0, p1])
+    p = np.concatenate([x[2] for x in res])
     assert np.max(np.abs(p - oracle.emit_p(row, b_ref, 0.02))) <= 1e-8
-    g = np.concatenate([g0, g1])
+    g = np.concatenate([x[3] for x in res])
     g_ref, _, _ = oracle.vjp(row, v[0], b_ref, 0.02)
     assert np.max(np.abs(g - g_ref)) <= 1e-7 * np.max(np.abs(g_ref))
