@@ -581,10 +581,10 @@ def main():
                 "fwd_elements_per_s": wk.elements / (T["fwd_ms"] / 1e3),
                 "bwd_elements_per_s": wk.elements / (T["bwd_ms"] / 1e3),
                 "fwdbwd_elements_per_s": wk.elements / (T["fwdbwd_ms"] / 1e3),
-                # the survey's fixed per-score byte count over the step time: a
-                # reference figure, not bytes this path moves (it can exceed the
-                # peak where the path skips passes the count assumes)
-                "fwdbwd_survey_bytes_gbs": STEP_BYTES_PER_ELEMENT[wk.path] * wk.elements
+                # the fixed per-score byte count (STEP_BYTES_PER_ELEMENT) over the
+                # step time: a reference figure, not bytes this path moves (it can
+                # exceed the peak where the path skips passes the count assumes)
+                "fwdbwd_fixed_bytes_gbs": STEP_BYTES_PER_ELEMENT[wk.path] * wk.elements
                 / (T["fwdbwd_ms"] / 1e3) / 1e9,
             }
             table[name]["oracle"] = oracle_timings(wk, rr, vv)
@@ -677,10 +677,11 @@ def main():
             "timing": "CUDA-graph replay of one fwd+bwd step; eager calls in eager_ms_per_step",
             "eager_ms_per_step": eager_ms_max,
             "eager_value": elements / (eager_ms_max / 1e3),
-            "survey_bytes_gbs": step_gbs,
-            "survey_bytes_over_peak": step_gbs / peak_gbs,
-            "step_bytes_note": "survey_bytes_* divide the survey's fixed per-score count (fwd "
-                               "12, bwd 20 B/score on long rows) by the step time: a reference "
+            "fixed_bytes_gbs": step_gbs,
+            "fixed_bytes_over_peak": step_gbs / peak_gbs,
+            "step_bytes_note": "fixed_bytes_* divide a fixed per-score count (fwd 12, bwd 20 "
+                               "B/score on long rows: r read twice in the forward, r and v "
+                               "read twice and g written in the backward) by the step time: a reference "
                                "figure, not a fraction of bytes moved (this path skips re-reads "
                                "the count assumes, so it can exceed 1); path_* count what this "
                                "path must move: r read by the fold, r read + p written by the "
