@@ -498,12 +498,12 @@ __global__ void __launch_bounds__(CTA, CTA == 256 ? 4 : 1) onchip_forward_kernel
 // past sB, the formula keeps the crossed scores at 1 - e^{|x|}/2 where F has
 // e^{-|x|}/2, never more, so the formula's root lies in (sB, b]: moving c
 // there never overshoots, and each step leaves at least one score behind;
-// symmetrically on the left.  A move back across the
-// score just crossed can only come from rounding at a boundary where F = k,
-// and that score is then b.  The start is a point whose count of larger
-// scores is close to k, found by interpolating the count between the row's
-// extremes.  Rows that do not settle in kSearchSteps steps are sorted and
-// solved by the full-sort solver in the same warp.
+// symmetrically on the left.  A move back across the score just crossed can
+// only come from rounding at a boundary where F = k, and that score is then
+// b.  The start is a point whose count of larger scores is close to k, found
+// by interpolating the count between the row's extremes.  Rows that do not
+// settle in kSearchSteps steps are sorted and solved by the full-sort solver
+// in the same warp.
 //
 // Accuracy: every exponential is fp32 and every term is at most 1, so Ah and
 // Bh carry a relative error of about 1e-6 and b one of about 1e-6 t.
